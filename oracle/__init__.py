@@ -1,0 +1,234 @@
+"""fp64 CPU oracle for windowed low-bit GDN / KDA decode -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline / reference legs
+may import this package. It never touches the CUDA library and the CUDA library never touches
+it: both sides only share the seeded inputs made by ``workloads``.
+
+This module is argument marshalling around ``gdn_oracle.c`` (numpy <-> C pointers). Every
+function of the method lives in the C file, which states what it restates from the pages
+("LeapQuant: Efficient Linear Attention with Accurate Recurrent State Quantization", Abstract;
+"Low-Bit GDN Recurrent-State Quantization: ... Pure-Write Sliding Windows", Abstract).
+
+Parity unpinned: the compensator column-selection rule (top-r columns by max-abs). The pages
+name compensator tokens but give no selection rule and no numbers; the tests pin only that the
+taken-out columns plus the residual reproduce the state exactly.
+
+Conventions: a state S is [D][D] with row i = value channel, column j = key channel. Per-step
+arrays are time-major, ``[T][nh][D]``; the gate ``g = log a`` is ``[T][nh]`` (scalar, GDN) or
+``[T][nh][D]`` (per key channel, KDA).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+from . import build as _build
+
+FMT_NONE, FMT_INT8, FMT_INT4 = 0, 1, 2
+ROUND_NONE, ROUND_F32, ROUND_BF16 = 0, 1, 2
+_FMT = {"none": FMT_NONE, "int8": FMT_INT8, "int4_g32": FMT_INT4, "int4": FMT_INT4}
+_ROUND = {"none": ROUND_NONE, "f32": ROUND_F32, "bf16": ROUND_BF16}
+
+_lib = None
+_lib_path = None
+
+_d = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
+_i8 = np.ctypeslib.ndpointer(dtype=np.int8, flags="C_CONTIGUOUS")
+_u8 = np.ctypeslib.ndpointer(dtype=np.uint8, flags="C_CONTIGUOUS")
+_i32 = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
+_vp = ctypes.c_void_p
+_int = ctypes.c_int
+
+
+def load(path: Optional[str] = None):
+    """Load (building if needed) the oracle library. ``path`` selects another build of the
+    same source, e.g. a deliberately broken copy in a mutation test."""
+    global _lib, _lib_path
+    if path is None:
+        if _lib is not None and _lib_path == _build.OUT:
+            return _lib
+        path = _build.build()
+    lib = ctypes.CDLL(path)
+    lib.orc_num_threads.restype = _int
+    lib.orc_round_bf16.restype = ctypes.c_double
+    lib.orc_round_bf16.argtypes = [ctypes.c_double]
+    lib.orc_round_f32.restype = ctypes.c_double
+    lib.orc_round_f32.argtypes = [ctypes.c_double]
+    lib.orc_num_groups.restype = _int
+    lib.orc_num_groups.argtypes = [_int, _int]
+    lib.orc_quantize.restype = _int
+    lib.orc_quantize.argtypes = [_int, _int, _int, _d, _i8, _d]
+    lib.orc_dequantize.restype = None
+    lib.orc_dequantize.argtypes = [_int, _int, _i8, _d, _d]
+    lib.orc_pack_int4.restype = None
+    lib.orc_pack_int4.argtypes = [_int, _i8, _u8]
+    lib.orc_unpack_int4.restype = None
+    lib.orc_unpack_int4.argtypes = [_int, _u8, _i8]
+    lib.orc_select_columns.restype = _int
+    lib.orc_select_columns.argtypes = [_int, _int, _d, _i32]
+    lib.orc_plain_run.restype = None
+    lib.orc_plain_run.argtypes = [_int] * 5 + [_vp] * 8
+    lib.orc_o1_run.restype = _int
+    lib.orc_o1_run.argtypes = [_int] * 7 + [_vp] * 8
+    lib.orc_o2_run.restype = _int
+    lib.orc_o2_run.argtypes = [_int] * 9 + [_vp] * 17
+    if path == _build.OUT:
+        _lib, _lib_path = lib, path
+    return lib
+
+
+def num_threads(lib=None) -> int:
+    return (lib or load()).orc_num_threads()
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(_vp)
+
+
+def _f64(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------------------------
+# Roundings and the quantizer
+# ---------------------------------------------------------------------------------------------
+def round_bf16(x: float, lib=None) -> float:
+    return (lib or load()).orc_round_bf16(float(x))
+
+
+def round_bf16_array(a: np.ndarray, lib=None) -> np.ndarray:
+    lib = lib or load()
+    flat = np.asarray(a, dtype=np.float64).ravel()
+    return np.array([lib.orc_round_bf16(float(x)) for x in flat]).reshape(np.shape(a))
+
+
+def quantize(S: np.ndarray, fmt: str = "int8", prec32: bool = False, lib=None):
+    """S [D][D] -> (codes int8 [D][D], scales f64 [D][groups])."""
+    lib = lib or load()
+    S = _f64(S)
+    D = S.shape[0]
+    f = _FMT[fmt]
+    ng = lib.orc_num_groups(f, D)
+    codes = np.zeros((D, D), np.int8)
+    scales = np.zeros((D, ng), np.float64)
+    if lib.orc_quantize(D, f, int(prec32), S, codes, scales) != 0:
+        raise ValueError(f"bad format {fmt}")
+    return codes, scales
+
+
+def dequantize(codes: np.ndarray, scales: np.ndarray, fmt: str = "int8", lib=None) -> np.ndarray:
+    lib = lib or load()
+    D = codes.shape[0]
+    out = np.zeros((D, D), np.float64)
+    lib.orc_dequantize(D, _FMT[fmt], np.ascontiguousarray(codes, np.int8), _f64(scales), out)
+    return out
+
+
+def pack_int4(codes: np.ndarray, lib=None) -> np.ndarray:
+    lib = lib or load()
+    D = codes.shape[0]
+    out = np.zeros((D, D // 2), np.uint8)
+    lib.orc_pack_int4(D, np.ascontiguousarray(codes, np.int8), out)
+    return out
+
+
+def unpack_int4(packed: np.ndarray, lib=None) -> np.ndarray:
+    lib = lib or load()
+    D = packed.shape[0]
+    out = np.zeros((D, D), np.int8)
+    lib.orc_unpack_int4(D, np.ascontiguousarray(packed, np.uint8), out)
+    return out
+
+
+def select_columns(S: np.ndarray, r: int, lib=None):
+    """Compensator choice: (column indices in pick order, near-tie flag)."""
+    lib = lib or load()
+    S = _f64(S)
+    idx = np.zeros(max(r, 1), np.int32)
+    near = lib.orc_select_columns(S.shape[0], r, S, idx)
+    return idx[:r].copy(), bool(near)
+
+
+# ---------------------------------------------------------------------------------------------
+# The three formulations
+# ---------------------------------------------------------------------------------------------
+def _gate(g, T, nh, D):
+    g = _f64(g)
+    if g.ndim == 2:
+        return g.reshape(T, nh, 1), 1
+    return g.reshape(T, nh, D), D
+
+
+def plain_run(q, k, v, g, beta, S0=None, state_round: str = "none", want_o: bool = True, lib=None):
+    """fp64 recurrence. Returns (o [T][nh][D] or None, S_T [nh][D][D])."""
+    lib = lib or load()
+    q, k, v, beta = _f64(q), _f64(k), _f64(v), _f64(beta)
+    T, nh, D = k.shape
+    g, Dg = _gate(g, T, nh, D)
+    S0 = _f64(S0)
+    o = np.zeros((T, nh, D)) if want_o else None
+    S = np.zeros((nh, D, D))
+    lib.orc_plain_run(D, T, nh, Dg, _ROUND[state_round], _p(S0), _p(q), _p(k), _p(v), _p(g),
+                      _p(beta), _p(o), _p(S))
+    return o, S
+
+
+def o1_run(q, k, v, g, beta, W: int, r: int = 0, fmt: str = "int8", S0=None, lib=None):
+    """Literal matrix-form recurrence with window-end requantisation (fp64 decisions).
+    Returns (o, S_T, near_ties)."""
+    lib = lib or load()
+    q, k, v, beta = _f64(q), _f64(k), _f64(v), _f64(beta)
+    T, nh, D = k.shape
+    g, Dg = _gate(g, T, nh, D)
+    S0 = _f64(S0)
+    o = np.zeros((T, nh, D))
+    S = np.zeros((nh, D, D))
+    ties = lib.orc_o1_run(D, T, W, r, _FMT[fmt], nh, Dg, _p(S0), _p(q), _p(k), _p(v), _p(g),
+                          _p(beta), _p(o), _p(S))
+    return o, S, ties
+
+
+@dataclass
+class O2Result:
+    o: np.ndarray          # [T][nh][D] fp64, unrounded
+    codes: np.ndarray      # [nh][D][D] int8 (int4 codes unpacked, in [-7, 7])
+    scales: np.ndarray     # [nh][D][groups]
+    cidx: np.ndarray       # [nh][r]
+    cu: np.ndarray         # [nh][r][D]
+    pos: np.ndarray        # [nh]
+    bk: np.ndarray         # [nh][W][D]
+    bu: np.ndarray         # [nh][W][D]
+    bL: np.ndarray         # [nh][W][D]
+    S: np.ndarray          # [nh][D][D] logical state at the end
+    near_ties: int
+
+
+def o2_run(q, k, v, g, beta, W: int, r: int = 0, fmt: str = "int8", S0=None,
+           round_storage: bool = False, buf_round: str = "bf16", flush_mask=None,
+           lib=None) -> O2Result:
+    """Buffered-window form. ``round_storage`` mirrors GPU storage (fp32 state / L / scales,
+    ``buf_round`` write vectors, fp32 quantizer decisions)."""
+    lib = lib or load()
+    q, k, v, beta = _f64(q), _f64(k), _f64(v), _f64(beta)
+    T, nh, D = k.shape
+    g, Dg = _gate(g, T, nh, D)
+    S0 = _f64(S0)
+    f = _FMT[fmt]
+    ng = lib.orc_num_groups(FMT_INT8 if f == FMT_NONE else f, D)
+    res = O2Result(
+        o=np.zeros((T, nh, D)), codes=np.zeros((nh, D, D), np.int8),
+        scales=np.zeros((nh, D, ng)), cidx=np.zeros((nh, max(r, 0)), np.int32),
+        cu=np.zeros((nh, max(r, 0), D)), pos=np.zeros(nh, np.int32),
+        bk=np.zeros((nh, W, D)), bu=np.zeros((nh, W, D)), bL=np.zeros((nh, W, D)),
+        S=np.zeros((nh, D, D)), near_ties=0)
+    fm = None if flush_mask is None else np.ascontiguousarray(flush_mask, np.uint8).reshape(T, nh)
+    res.near_ties = lib.orc_o2_run(
+        D, T, W, r, f, nh, Dg, int(round_storage), _ROUND[buf_round], _p(S0), _p(q), _p(k),
+        _p(v), _p(g), _p(beta), _p(fm), _p(res.o), _p(res.codes), _p(res.scales),
+        _p(res.cidx) if r > 0 else None, _p(res.cu) if r > 0 else None, _p(res.pos),
+        _p(res.bk), _p(res.bu), _p(res.bL), _p(res.S))
+    return res

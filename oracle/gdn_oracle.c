@@ -1,0 +1,517 @@
+/*
+ * gdn_oracle.c -- plain, slow fp64 CPU oracle for gated delta-rule (GDN / KDA) decode over a
+ * windowed low-bit recurrent state.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the test suite, the smoke check and the benchmark's CPU
+ * baseline leg may load this library. It shares no code, header, table or helper with the CUDA
+ * library; both sides only see the same seeded inputs.
+ *
+ * What it restates (page title, part of the page):
+ *   [LQ] "LeapQuant: Efficient Linear Attention with Accurate Recurrent State Quantization"
+ *        (weekinpapers summary page), Abstract:
+ *          - GDN and KDA keep a fixed-size recurrent state that every decode step reads and
+ *            updates;
+ *          - per-window quantization: the state stays frozen in low bits for a window of
+ *            tokens and is quantized once, at the window's end;
+ *          - inside a window, outputs come from the frozen low-bit state plus buffered
+ *            high-precision updates;
+ *          - a few high-precision "compensator tokens" keep the state's largest outliers and
+ *            take the same update path as real tokens;
+ *          - the residual is smoothed before quantization (NOT restated here: the page gives
+ *            no mechanism).
+ *   [PW] "Low-Bit GDN Recurrent-State Quantization: Global Gradient-aware Allocation and
+ *        Pure-Write Sliding Windows", Abstract: quantized write-back errors feed into later
+ *        steps (why quantize-every-step, the window length 1 case, degrades).
+ *
+ * The recurrence, for one (sequence, head), state S in R^{d_v x d_k} (row i = value channel,
+ * column j = key channel), gate a_t in R^{d_k} (GDN: all entries equal; KDA: per key channel):
+ *
+ *     S_t = S_{t-1} Diag(a_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,      o_t = S_t q_t.
+ *
+ * The gate enters as its logarithm g_t = log a_t, so products of gates over a window are sums.
+ *
+ * Three formulations live here; none calls another's step code:
+ *   plain  -- the recurrence in fp64, optionally rounding the stored state to fp32 / bf16 after
+ *             each step (the high-precision-state baselines and the fp32 warm-up);
+ *   O1     -- the recurrence applied literally as matrix products (D x D transition matrix),
+ *             with the state replaced by dequant(quant(S - C)) + C after every W-th step;
+ *   O2     -- the buffered form: frozen low-bit state + buffered pairs (k_i, u_i, L_i) +
+ *             compensator pairs, flushed (materialised, requantised) when the window fills.
+ *             Optional storage roundings mirror what a GPU stores between steps.
+ *
+ * Readings of the pages where they are silent (each one is listed in the design notes):
+ *   - quantizer: symmetric absmax, s = absmax / 127 (int8, one scale per row) or absmax / 7
+ *     (int4, one scale per group of 32 key channels); c = clamp(round-half-even(x / s)); a zero
+ *     group has s = 0 and codes 0.
+ *   - windows are [0, W), [W, 2W), ... from the start of decode; the output of a window's last
+ *     step comes from the buffered form, before requantisation.
+ *   - compensators: at every quantization, the r key columns with the largest max-abs (ties to
+ *     the lower index) are taken out exactly as pairs (key e_j, value S[:, j]) and re-enter the
+ *     next window at cumulative gate 0. PARITY UNPINNED against the pages: they give no rule.
+ *     Only the exact decomposition S = residual + sum of pairs is pinned.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORC_FMT_NONE = 0, ORC_FMT_INT8 = 1, ORC_FMT_INT4 = 2 };
+enum { ORC_ROUND_NONE = 0, ORC_ROUND_F32 = 1, ORC_ROUND_BF16 = 2 };
+
+int orc_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------------------------------
+ * Storage roundings.
+ * bfloat16: 8 significant bits, the exponent range of IEEE single; round to nearest, ties to
+ * even. Written from that definition: find the quantum of x's binade (2^(e-8) where
+ * 2^(e-1) <= |x| < 2^e), clamp it at the subnormal quantum 2^-133, and round x / quantum
+ * to an integer with rint (ties to even in the default rounding mode).
+ * ---------------------------------------------------------------------------------------- */
+double orc_round_bf16(double x) {
+    if (x == 0.0 || !isfinite(x)) return x;
+    int e;
+    frexp(x, &e);                      /* x = m * 2^e, 0.5 <= |m| < 1 */
+    int qexp = e - 8;
+    if (qexp < -133) qexp = -133;
+    double quantum = ldexp(1.0, qexp);
+    double r = rint(x / quantum) * quantum;
+    if (fabs(r) > 3.3895313892515355e38) r = copysign(INFINITY, x); /* beyond the largest bf16 */
+    return r;
+}
+
+double orc_round_f32(double x) { return (double)(float)x; }
+
+static double round_to(int mode, double x) {
+    if (mode == ORC_ROUND_F32) return orc_round_f32(x);
+    if (mode == ORC_ROUND_BF16) return orc_round_bf16(x);
+    return x;
+}
+
+/* ------------------------------------------------------------------------------------------
+ * Quantizer. codes are one int8 per entry (int4 codes lie in [-7, 7]); scales are [D][groups].
+ * prec32 = 1 takes every decision in single precision, as a GPU does: the caller passes
+ * fp32-representable values, s = fp32(absmax / qmax) and x / s is rounded to fp32 before rint.
+ * (Rounding an fp64 quotient of two fp32 values to fp32 gives the correctly rounded fp32
+ * quotient, so this is IEEE single division.)
+ * ---------------------------------------------------------------------------------------- */
+static int fmt_qmax(int fmt) { return fmt == ORC_FMT_INT4 ? 7 : 127; }
+static int fmt_group(int fmt, int D) { return fmt == ORC_FMT_INT4 ? 32 : D; }
+
+int orc_num_groups(int fmt, int D) { return D / fmt_group(fmt, D); }
+
+static void quantize_group(const double* x, int n, int qmax, int prec32, int8_t* c, double* s_out) {
+    double m = 0.0;
+    for (int j = 0; j < n; ++j) m = fmax(m, fabs(x[j]));
+    double s = m / (double)qmax;
+    if (prec32) s = orc_round_f32(s);
+    *s_out = s;
+    for (int j = 0; j < n; ++j) {
+        if (s == 0.0) { c[j] = 0; continue; }
+        double t = x[j] / s;
+        if (prec32) t = orc_round_f32(t);
+        double r = rint(t);
+        if (r > qmax) r = qmax;
+        if (r < -qmax) r = -qmax;
+        c[j] = (int8_t)r;
+    }
+}
+
+/* S [D][D] -> codes [D][D], scales [D][groups]. Returns 0, or -1 for a bad format. */
+int orc_quantize(int D, int fmt, int prec32, const double* S, int8_t* codes, double* scales) {
+    if (fmt != ORC_FMT_INT8 && fmt != ORC_FMT_INT4) return -1;
+    int gs = fmt_group(fmt, D), ng = D / gs, qmax = fmt_qmax(fmt);
+    for (int i = 0; i < D; ++i)
+        for (int g = 0; g < ng; ++g)
+            quantize_group(S + (size_t)i * D + g * gs, gs, qmax, prec32,
+                           codes + (size_t)i * D + g * gs, scales + (size_t)i * ng + g);
+    return 0;
+}
+
+/* codes, scales -> S[i][j] = s_{i, group(j)} * c_ij */
+void orc_dequantize(int D, int fmt, const int8_t* codes, const double* scales, double* S) {
+    int gs = fmt_group(fmt, D), ng = D / gs;
+    for (int i = 0; i < D; ++i)
+        for (int j = 0; j < D; ++j)
+            S[(size_t)i * D + j] = scales[(size_t)i * ng + j / gs] * (double)codes[(size_t)i * D + j];
+}
+
+/* int4 packing: byte m of a row holds column 2m in its low nibble and 2m+1 in its high nibble,
+ * each a 4-bit two's complement number. */
+void orc_pack_int4(int D, const int8_t* codes, uint8_t* packed) {
+    for (int i = 0; i < D; ++i)
+        for (int m = 0; m < D / 2; ++m) {
+            unsigned lo = (unsigned)codes[(size_t)i * D + 2 * m] & 0xFu;
+            unsigned hi = (unsigned)codes[(size_t)i * D + 2 * m + 1] & 0xFu;
+            packed[(size_t)i * (D / 2) + m] = (uint8_t)(lo | (hi << 4));
+        }
+}
+
+void orc_unpack_int4(int D, const uint8_t* packed, int8_t* codes) {
+    for (int i = 0; i < D; ++i)
+        for (int m = 0; m < D / 2; ++m) {
+            unsigned b = packed[(size_t)i * (D / 2) + m];
+            int lo = (int)(b & 0xFu), hi = (int)(b >> 4);
+            codes[(size_t)i * D + 2 * m] = (int8_t)(lo >= 8 ? lo - 16 : lo);
+            codes[(size_t)i * D + 2 * m + 1] = (int8_t)(hi >= 8 ? hi - 16 : hi);
+        }
+}
+
+/* ------------------------------------------------------------------------------------------
+ * Compensator selection: the r columns with the largest max-abs over the rows, ties to the
+ * lower column index. Returns 1 when the r-th pick and the best column left out are within
+ * 1e-6 relative (a near tie: another correct implementation may pick differently).
+ * ---------------------------------------------------------------------------------------- */
+int orc_select_columns(int D, int r, const double* S, int* idx) {
+    double* colmax = (double*)calloc((size_t)D, sizeof(double));
+    char* taken = (char*)calloc((size_t)D, 1);
+    for (int j = 0; j < D; ++j)
+        for (int i = 0; i < D; ++i) colmax[j] = fmax(colmax[j], fabs(S[(size_t)i * D + j]));
+    double last = 0.0;
+    for (int c = 0; c < r; ++c) {
+        int best = -1;
+        for (int j = 0; j < D; ++j)
+            if (!taken[j] && (best < 0 || colmax[j] > colmax[best])) best = j;
+        taken[best] = 1;
+        idx[c] = best;
+        last = colmax[best];
+    }
+    int near = 0;
+    if (r > 0 && r < D) {
+        double rest = -1.0;
+        for (int j = 0; j < D; ++j)
+            if (!taken[j] && colmax[j] > rest) rest = colmax[j];
+        if (last - rest <= 1e-6 * fmax(last, rest)) near = 1;
+    }
+    free(colmax);
+    free(taken);
+    return near;
+}
+
+/* Window-end operation on a full state S (overwritten by the residual): take out r compensator
+ * columns exactly, then quantize the residual. fmt == NONE keeps the residual unquantized in S.
+ * Returns the near-tie flag of the column choice. */
+static int window_end(int D, int fmt, int r, int prec32, double* S, int8_t* codes, double* scales,
+                      int* cidx, double* cu) {
+    int near = orc_select_columns(D, r, S, cidx);
+    for (int c = 0; c < r; ++c)
+        for (int i = 0; i < D; ++i) {
+            cu[(size_t)c * D + i] = S[(size_t)i * D + cidx[c]];
+            S[(size_t)i * D + cidx[c]] = 0.0;
+        }
+    if (fmt != ORC_FMT_NONE) orc_quantize(D, fmt, prec32, S, codes, scales);
+    return near;
+}
+
+static double gate_log(const double* g, int Dg, int j) { return Dg == 1 ? g[0] : g[j]; }
+
+/* ------------------------------------------------------------------------------------------
+ * plain: the recurrence in fp64. The product S Diag(a)(I - beta k k^T) is expanded by
+ * distributivity, S' - beta (S' k) k^T with S' = S Diag(a). state_round rounds the stored
+ * state after each step (fp32 / bf16 state baselines); o_t is taken from the new state before
+ * that rounding. S0 may be NULL (zero state). o and S_out may be NULL.
+ * Layouts: S [nh][D][D]; q, k, v [T][nh][D]; g [T][nh][Dg] (Dg = 1 or D); beta [T][nh].
+ * ---------------------------------------------------------------------------------------- */
+void orc_plain_run(int D, int T, int nh, int Dg, int state_round, const double* S0,
+                   const double* q, const double* k, const double* v, const double* g,
+                   const double* beta, double* o, double* S_out) {
+#pragma omp parallel for schedule(dynamic)
+    for (int h = 0; h < nh; ++h) {
+        double* S = (double*)malloc(sizeof(double) * (size_t)D * D);
+        double* w = (double*)malloc(sizeof(double) * (size_t)D);
+        if (S0) memcpy(S, S0 + (size_t)h * D * D, sizeof(double) * (size_t)D * D);
+        else memset(S, 0, sizeof(double) * (size_t)D * D);
+        for (int t = 0; t < T; ++t) {
+            const double* kt = k + ((size_t)t * nh + h) * D;
+            const double* qt = q + ((size_t)t * nh + h) * D;
+            const double* vt = v + ((size_t)t * nh + h) * D;
+            const double* gt = g + ((size_t)t * nh + h) * Dg;
+            double bt = beta[(size_t)t * nh + h];
+            for (int i = 0; i < D; ++i)          /* S' = S Diag(a) */
+                for (int j = 0; j < D; ++j) S[(size_t)i * D + j] *= exp(gate_log(gt, Dg, j));
+            for (int i = 0; i < D; ++i) {        /* w = S' k */
+                double acc = 0.0;
+                for (int j = 0; j < D; ++j) acc += S[(size_t)i * D + j] * kt[j];
+                w[i] = acc;
+            }
+            for (int i = 0; i < D; ++i)          /* S' - beta w k^T + beta v k^T */
+                for (int j = 0; j < D; ++j)
+                    S[(size_t)i * D + j] += -bt * w[i] * kt[j] + bt * vt[i] * kt[j];
+            if (o) {
+                double* ot = o + ((size_t)t * nh + h) * D;
+                for (int i = 0; i < D; ++i) {
+                    double acc = 0.0;
+                    for (int j = 0; j < D; ++j) acc += S[(size_t)i * D + j] * qt[j];
+                    ot[i] = acc;
+                }
+            }
+            if (state_round != ORC_ROUND_NONE)
+                for (size_t e = 0; e < (size_t)D * D; ++e) S[e] = round_to(state_round, S[e]);
+        }
+        if (S_out) memcpy(S_out + (size_t)h * D * D, S, sizeof(double) * (size_t)D * D);
+        free(S);
+        free(w);
+    }
+}
+
+/* ------------------------------------------------------------------------------------------
+ * O1: the recurrence applied literally. Each step forms the D x D transition
+ *     M = Diag(a_t) (I - beta_t k_t k_t^T),   M[j][l] = a_t[j] (delta_jl - beta_t k_t[j] k_t[l])
+ * and sets S <- S M + beta_t v_t k_t^T, o_t = S q_t. Before the first step and after every
+ * W-th step, S <- dequant(quant(S - C)) + C, where C holds the r compensator columns of S
+ * (fmt NONE: S is left as it is). All decisions in fp64. Returns the number of near ties.
+ * ---------------------------------------------------------------------------------------- */
+static int dense_window_end(int D, int fmt, int r, double* S) {
+    if (fmt == ORC_FMT_NONE && r == 0) return 0;
+    int ng = orc_num_groups(fmt == ORC_FMT_NONE ? ORC_FMT_INT8 : fmt, D);
+    int8_t* codes = (int8_t*)malloc((size_t)D * D);
+    double* scales = (double*)malloc(sizeof(double) * (size_t)D * ng);
+    int* cidx = (int*)malloc(sizeof(int) * (size_t)(r > 0 ? r : 1));
+    double* cu = (double*)malloc(sizeof(double) * (size_t)(r > 0 ? r : 1) * D);
+    int near = window_end(D, fmt, r, 0, S, codes, scales, cidx, cu);
+    if (fmt != ORC_FMT_NONE) orc_dequantize(D, fmt, codes, scales, S);
+    for (int c = 0; c < r; ++c)
+        for (int i = 0; i < D; ++i) S[(size_t)i * D + cidx[c]] += cu[(size_t)c * D + i];
+    free(codes);
+    free(scales);
+    free(cidx);
+    free(cu);
+    return near;
+}
+
+int orc_o1_run(int D, int T, int W, int r, int fmt, int nh, int Dg, const double* S0,
+               const double* q, const double* k, const double* v, const double* g,
+               const double* beta, double* o, double* S_out) {
+    int ties = 0;
+#pragma omp parallel for schedule(dynamic) reduction(+ : ties)
+    for (int h = 0; h < nh; ++h) {
+        size_t DD = (size_t)D * D;
+        double* S = (double*)malloc(sizeof(double) * DD);
+        double* M = (double*)malloc(sizeof(double) * DD);
+        double* N = (double*)malloc(sizeof(double) * DD);
+        if (S0) memcpy(S, S0 + (size_t)h * DD, sizeof(double) * DD);
+        else memset(S, 0, sizeof(double) * DD);
+        ties += dense_window_end(D, fmt, r, S);
+        for (int t = 0; t < T; ++t) {
+            const double* kt = k + ((size_t)t * nh + h) * D;
+            const double* qt = q + ((size_t)t * nh + h) * D;
+            const double* vt = v + ((size_t)t * nh + h) * D;
+            const double* gt = g + ((size_t)t * nh + h) * Dg;
+            double bt = beta[(size_t)t * nh + h];
+            for (int j = 0; j < D; ++j)
+                for (int l = 0; l < D; ++l)
+                    M[(size_t)j * D + l] =
+                        exp(gate_log(gt, Dg, j)) * ((j == l ? 1.0 : 0.0) - bt * kt[j] * kt[l]);
+            for (int i = 0; i < D; ++i)
+                for (int l = 0; l < D; ++l) {
+                    double acc = 0.0;
+                    for (int j = 0; j < D; ++j) acc += S[(size_t)i * D + j] * M[(size_t)j * D + l];
+                    N[(size_t)i * D + l] = acc + bt * vt[i] * kt[l];
+                }
+            memcpy(S, N, sizeof(double) * DD);
+            if (o) {
+                double* ot = o + ((size_t)t * nh + h) * D;
+                for (int i = 0; i < D; ++i) {
+                    double acc = 0.0;
+                    for (int j = 0; j < D; ++j) acc += S[(size_t)i * D + j] * qt[j];
+                    ot[i] = acc;
+                }
+            }
+            if ((t + 1) % W == 0) ties += dense_window_end(D, fmt, r, S);
+        }
+        if (S_out) memcpy(S_out + (size_t)h * DD, S, sizeof(double) * DD);
+        free(S);
+        free(M);
+        free(N);
+    }
+    return ties;
+}
+
+/* ------------------------------------------------------------------------------------------
+ * O2: the buffered form. Per head the state is
+ *   F          the frozen state: dequant(codes, scales) (fmt NONE: an unquantized matrix);
+ *   (cidx, cu) r compensator pairs, key e_{cidx[c]}, value cu[c], entered at cumulative gate 0;
+ *   (bk, bu, bL)[0..P) buffered write pairs: key, write vector, cumulative log-gate vector;
+ *   P          pairs in the window so far.
+ * The logical state after the window's P steps, with L = bL[P-1] (0 if P == 0), is
+ *   S = F Diag(e^L) + sum_c cu_c (e_{cidx_c} * e^{L})^T + sum_i bu_i (bk_i * e^{L - bL_i})^T.
+ * A step at position P:
+ *   L_t = L + g_t;  x = e^{L_t} * k_t;  y = e^{L_t} * q_t
+ *   w  = F x + sum_c cu_c x[cidx_c] + sum_i bu_i <bk_i * e^{L_t - bL_i}, k_t>   (= S Diag(a_t) k_t)
+ *   r  = F y + sum_c cu_c y[cidx_c] + sum_i bu_i <bk_i * e^{L_t - bL_i}, q_t>   (= S Diag(a_t) q_t)
+ *   u_t = beta_t (v_t - w);  o_t = r + u_t <k_t, q_t>;  append (k_t, u_t, L_t)
+ * which is the recurrence through S Diag(a)(I - beta k k^T) + beta v k^T
+ *   = S Diag(a) + beta (v - S Diag(a) k) k^T.
+ * When P reaches W (or a flush is forced after the step) the logical state is materialised and
+ * the window-end operation (compensators out, residual quantized) makes the next F.
+ *
+ * round_storage = 1 mirrors what a GPU keeps between steps: the initial state and the
+ * materialised state are fp32, L is fp32, u_t is rounded to buf_round (bf16 / fp32), and the
+ * quantizer decides in fp32. round_storage = 0 keeps everything in fp64.
+ *
+ * Outputs (any may be NULL): o [T][nh][D]; codes [nh][D][D]; scales [nh][D][groups];
+ * cidx [nh][r]; cu [nh][r][D]; pos [nh]; bk, bu, bL [nh][W][D]; S_out [nh][D][D] (the logical
+ * state at the end); flush_mask [T][nh] forces a flush after step t of head h when nonzero.
+ * Returns the number of near ties met in compensator choices.
+ * ---------------------------------------------------------------------------------------- */
+typedef struct {
+    int D, W, r, fmt, Dg, round_storage, buf_round;
+} o2_cfg;
+
+typedef struct {
+    double *F, *scales, *cu, *bk, *bu, *bL;
+    int8_t* codes;
+    int* cidx;
+    int P;
+} o2_head;
+
+static void o2_current_L(const o2_cfg* c, const o2_head* s, double* L) {
+    for (int j = 0; j < c->D; ++j) L[j] = s->P > 0 ? s->bL[(size_t)(s->P - 1) * c->D + j] : 0.0;
+}
+
+/* Logical state at cumulative gate L (the window's current end), written into S. */
+static void o2_materialize(const o2_cfg* c, const o2_head* s, const double* L, double* S) {
+    int D = c->D;
+    for (int i = 0; i < D; ++i)
+        for (int j = 0; j < D; ++j) S[(size_t)i * D + j] = s->F[(size_t)i * D + j] * exp(L[j]);
+    for (int cc = 0; cc < c->r; ++cc) {
+        int j = s->cidx[cc];
+        for (int i = 0; i < D; ++i) S[(size_t)i * D + j] += s->cu[(size_t)cc * D + i] * exp(L[j]);
+    }
+    for (int p = 0; p < s->P; ++p)
+        for (int i = 0; i < D; ++i)
+            for (int j = 0; j < D; ++j)
+                S[(size_t)i * D + j] += s->bu[(size_t)p * D + i] * s->bk[(size_t)p * D + j] *
+                                        exp(L[j] - s->bL[(size_t)p * D + j]);
+}
+
+/* Quantize a full state S (destroyed) into the head's frozen part and compensators. */
+static int o2_set_frozen(const o2_cfg* c, o2_head* s, double* S) {
+    int D = c->D;
+    if (c->round_storage)
+        for (size_t e = 0; e < (size_t)D * D; ++e) S[e] = orc_round_f32(S[e]);
+    int near = window_end(D, c->fmt, c->r, c->round_storage, S, s->codes, s->scales, s->cidx, s->cu);
+    if (c->fmt != ORC_FMT_NONE) orc_dequantize(D, c->fmt, s->codes, s->scales, s->F);
+    else memcpy(s->F, S, sizeof(double) * (size_t)D * D);
+    s->P = 0;
+    return near;
+}
+
+static int o2_flush(const o2_cfg* c, o2_head* s, double* scratch_S, double* scratch_L) {
+    o2_current_L(c, s, scratch_L);
+    o2_materialize(c, s, scratch_L, scratch_S);
+    return o2_set_frozen(c, s, scratch_S);
+}
+
+static void o2_step(const o2_cfg* c, o2_head* s, const double* qt, const double* kt, const double* vt,
+                    const double* gt, double bt, double* ot, double* Lt, double* x, double* y,
+                    double* w, double* rr) {
+    int D = c->D;
+    o2_current_L(c, s, Lt);
+    for (int j = 0; j < D; ++j) {
+        Lt[j] = Lt[j] + gate_log(gt, c->Dg, j);
+        if (c->round_storage) Lt[j] = orc_round_f32(Lt[j]);
+        x[j] = exp(Lt[j]) * kt[j];
+        y[j] = exp(Lt[j]) * qt[j];
+    }
+    for (int i = 0; i < D; ++i) {
+        double a = 0.0, b = 0.0;
+        for (int j = 0; j < D; ++j) {
+            a += s->F[(size_t)i * D + j] * x[j];
+            b += s->F[(size_t)i * D + j] * y[j];
+        }
+        w[i] = a;
+        rr[i] = b;
+    }
+    for (int cc = 0; cc < c->r; ++cc) {
+        int j = s->cidx[cc];
+        for (int i = 0; i < D; ++i) {
+            w[i] += s->cu[(size_t)cc * D + i] * x[j];
+            rr[i] += s->cu[(size_t)cc * D + i] * y[j];
+        }
+    }
+    for (int p = 0; p < s->P; ++p) {
+        double a = 0.0, b = 0.0;
+        for (int j = 0; j < D; ++j) {
+            double f = exp(Lt[j] - s->bL[(size_t)p * D + j]);
+            a += s->bk[(size_t)p * D + j] * f * kt[j];
+            b += s->bk[(size_t)p * D + j] * f * qt[j];
+        }
+        for (int i = 0; i < D; ++i) {
+            w[i] += s->bu[(size_t)p * D + i] * a;
+            rr[i] += s->bu[(size_t)p * D + i] * b;
+        }
+    }
+    double kq = 0.0;
+    for (int j = 0; j < D; ++j) kq += kt[j] * qt[j];
+    double* un = s->bu + (size_t)s->P * D;
+    for (int i = 0; i < D; ++i) {
+        double u = bt * (vt[i] - w[i]);
+        if (c->round_storage) u = round_to(c->buf_round, u);
+        un[i] = u;
+        if (ot) ot[i] = rr[i] + u * kq;
+    }
+    memcpy(s->bk + (size_t)s->P * D, kt, sizeof(double) * (size_t)D);
+    memcpy(s->bL + (size_t)s->P * D, Lt, sizeof(double) * (size_t)D);
+    s->P += 1;
+}
+
+int orc_o2_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int round_storage,
+               int buf_round, const double* S0, const double* q, const double* k, const double* v,
+               const double* g, const double* beta, const uint8_t* flush_mask, double* o,
+               int8_t* codes_out, double* scales_out, int* cidx_out, double* cu_out, int* pos_out,
+               double* bk_out, double* bu_out, double* bL_out, double* S_out) {
+    o2_cfg c = {D, W, r, fmt, Dg, round_storage, buf_round};
+    int ng = orc_num_groups(fmt == ORC_FMT_NONE ? ORC_FMT_INT8 : fmt, D);
+    int ties = 0;
+#pragma omp parallel for schedule(dynamic) reduction(+ : ties)
+    for (int h = 0; h < nh; ++h) {
+        size_t DD = (size_t)D * D;
+        o2_head s;
+        s.F = (double*)calloc(DD, sizeof(double));
+        s.scales = (double*)calloc((size_t)D * ng, sizeof(double));
+        s.codes = (int8_t*)calloc(DD, 1);
+        s.cidx = (int*)calloc((size_t)(r > 0 ? r : 1), sizeof(int));
+        s.cu = (double*)calloc((size_t)(r > 0 ? r : 1) * D, sizeof(double));
+        s.bk = (double*)calloc((size_t)W * D, sizeof(double));
+        s.bu = (double*)calloc((size_t)W * D, sizeof(double));
+        s.bL = (double*)calloc((size_t)W * D, sizeof(double));
+        double* Sx = (double*)malloc(sizeof(double) * DD);
+        double* vec = (double*)malloc(sizeof(double) * (size_t)D * 5);
+        double *Lt = vec, *x = vec + D, *y = vec + 2 * D, *w = vec + 3 * D, *rr = vec + 4 * D;
+
+        if (S0) memcpy(Sx, S0 + (size_t)h * DD, sizeof(double) * DD);
+        else memset(Sx, 0, sizeof(double) * DD);
+        ties += o2_set_frozen(&c, &s, Sx);
+        for (int t = 0; t < T; ++t) {
+            size_t th = (size_t)t * nh + h;
+            o2_step(&c, &s, q + th * D, k + th * D, v + th * D, g + th * Dg, beta[th],
+                    o ? o + th * D : NULL, Lt, x, y, w, rr);
+            int forced = flush_mask && flush_mask[th];
+            if (s.P == W || forced) ties += o2_flush(&c, &s, Sx, Lt);
+        }
+        if (codes_out) memcpy(codes_out + h * DD, s.codes, DD);
+        if (scales_out) memcpy(scales_out + (size_t)h * D * ng, s.scales, sizeof(double) * (size_t)D * ng);
+        if (cidx_out && r > 0) memcpy(cidx_out + (size_t)h * r, s.cidx, sizeof(int) * (size_t)r);
+        if (cu_out && r > 0) memcpy(cu_out + (size_t)h * r * D, s.cu, sizeof(double) * (size_t)r * D);
+        if (pos_out) pos_out[h] = s.P;
+        if (bk_out) memcpy(bk_out + (size_t)h * W * D, s.bk, sizeof(double) * (size_t)W * D);
+        if (bu_out) memcpy(bu_out + (size_t)h * W * D, s.bu, sizeof(double) * (size_t)W * D);
+        if (bL_out) memcpy(bL_out + (size_t)h * W * D, s.bL, sizeof(double) * (size_t)W * D);
+        if (S_out) {
+            o2_current_L(&c, &s, Lt);
+            o2_materialize(&c, &s, Lt, S_out + h * DD);
+        }
+        free(s.F); free(s.scales); free(s.codes); free(s.cidx); free(s.cu);
+        free(s.bk); free(s.bu); free(s.bL); free(Sx); free(vec);
+    }
+    return ties;
+}

@@ -1,0 +1,419 @@
+"""Pins for the CPU oracle: checks against what the pages and the mathematics fix, never against
+the oracle's own formulas retyped.
+
+Each ``pin_*`` takes a loaded oracle library and raises AssertionError when the oracle is wrong.
+``test_oracle_pins.py`` runs them on the real oracle; ``test_oracle_mutants.py`` runs them on
+deliberately broken copies and requires every break to be caught.
+
+Kinds of pin used here:
+  - hand-worked fixtures under tests/golden (values fixed by arithmetic done by hand);
+  - closed forms: one write from a zero state, pure decay, exact retrieval with orthonormal keys,
+    the delta-rule write identity at the written key;
+  - agreement of independent formulations (literal matrix form, distributive plain form,
+    buffered windows) where the mathematics says they are equal;
+  - library routines for special cases: numpy rint / argsort, torch's bf16 conversion.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from golden_io import read
+
+
+def _softplus(x):
+    return np.log1p(np.exp(-np.abs(x))) + np.maximum(x, 0)
+
+
+def rand_inputs(seed, T, nh, D, gate="scalar", unit=True, outlier=False):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((T, nh, D))
+    k = rng.standard_normal((T, nh, D))
+    v = rng.standard_normal((T, nh, D))
+    if outlier:
+        k[..., 1] *= 20.0
+        v[..., 2] *= 20.0
+    if unit:
+        q /= np.linalg.norm(q, axis=-1, keepdims=True)
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((T, nh))))
+    gshape = (T, nh) if gate == "scalar" else (T, nh, D)
+    g = -_softplus(rng.standard_normal(gshape))
+    return q, k, v, g, beta
+
+
+def rel(a, b):
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def close(a, b, tol, what):
+    e = rel(a, b)
+    assert e <= tol, f"{what}: rel err {e:.3e} > {tol:.1e}"
+
+
+# ---------------------------------------------------------------------------------------------
+# Hand-worked fixtures
+# ---------------------------------------------------------------------------------------------
+def pin_golden_delta_rule_kda(lib):
+    gd = read("delta_rule_kda_2x2.txt")
+    D, T = 2, 2
+    S0 = gd["S0"].reshape(1, D, D)
+    q, k, v = (gd[n].reshape(T, 1, D) for n in ("q", "k", "v"))
+    g = np.log(gd["a"]).reshape(T, 1, D)
+    beta = gd["beta"].reshape(T, 1)
+    for t, Sname in ((1, "S1"), (2, "S2")):
+        o, S = oracle.plain_run(q[:t], k[:t], v[:t], g[:t], beta[:t], S0=S0, lib=lib)
+        assert np.allclose(S[0].ravel(), gd[Sname], atol=1e-12), ("plain", Sname, S[0])
+        assert np.allclose(o.ravel(), gd["o"][: t * D], atol=1e-12), ("plain o", o)
+        o1, S1, _ = oracle.o1_run(q[:t], k[:t], v[:t], g[:t], beta[:t], W=1, fmt="none",
+                                  S0=S0, lib=lib)
+        assert np.allclose(S1[0].ravel(), gd[Sname], atol=1e-12), ("O1", Sname, S1[0])
+        assert np.allclose(o1.ravel(), gd["o"][: t * D], atol=1e-12), ("O1 o", o1)
+        res = oracle.o2_run(q[:t], k[:t], v[:t], g[:t], beta[:t], W=4, fmt="none", S0=S0, lib=lib)
+        assert np.allclose(res.S[0].ravel(), gd[Sname], atol=1e-12), ("O2", Sname, res.S[0])
+        assert np.allclose(res.o.ravel(), gd["o"][: t * D], atol=1e-12), ("O2 o", res.o)
+
+
+def pin_golden_window_int8(lib):
+    gd = read("window_int8_2x2.txt")
+    D, T, W = 2, 3, 2
+    S0 = gd["S0"].reshape(1, D, D)
+    q, k, v = (gd[n].reshape(T, 1, D) for n in ("q", "k", "v"))
+    g = np.log(gd["a"]).reshape(T, 1)
+    beta = gd["beta"].reshape(T, 1)
+    res = oracle.o2_run(q, k, v, g, beta, W=W, fmt="int8", S0=S0, lib=lib)
+    assert np.allclose(res.o.ravel(), gd["o"], atol=1e-12), ("O2 o", res.o.ravel())
+    assert np.allclose(res.S[0].ravel(), gd["S3"], atol=1e-12), ("O2 S3", res.S[0])
+    r2 = oracle.o2_run(q[:2], k[:2], v[:2], g[:2], beta[:2], W=W, fmt="int8", S0=S0, lib=lib)
+    assert np.array_equal(r2.codes[0].ravel(), gd["codes_after_window1"].astype(np.int8)), r2.codes
+    assert np.allclose(r2.scales[0].ravel(), gd["scales_after_window1"], rtol=1e-15, atol=0)
+    assert r2.pos[0] == 0
+    o1, S1, _ = oracle.o1_run(q, k, v, g, beta, W=W, fmt="int8", S0=S0, lib=lib)
+    assert np.allclose(o1.ravel(), gd["o"], atol=1e-12), ("O1 o", o1.ravel())
+    assert np.allclose(S1[0].ravel(), gd["S3"], atol=1e-12), ("O1 S3", S1[0])
+
+
+def pin_golden_compensator(lib):
+    gd = read("compensator_2x2.txt")
+    D = 2
+    S0 = gd["S0"].reshape(1, D, D)
+    q, k, v = (gd[n].reshape(1, 1, D) for n in ("q", "k", "v"))
+    g = np.log(gd["a"]).reshape(1, 1, D)
+    beta = gd["beta"].reshape(1, 1)
+    r0 = oracle.o2_run(q[:0], k[:0], v[:0], g[:0], beta[:0], W=4, r=1, fmt="int8", S0=S0, lib=lib)
+    assert list(r0.cidx[0]) == [int(gd["comp_idx"][0])], r0.cidx
+    assert np.allclose(r0.cu[0].ravel(), gd["comp_u"], atol=0), r0.cu
+    assert np.array_equal(r0.codes[0].ravel(), gd["codes0"].astype(np.int8)), r0.codes
+    assert np.allclose(r0.scales[0].ravel(), gd["scales0"], rtol=1e-15, atol=0), r0.scales
+    assert np.allclose(r0.S[0], S0[0], atol=1e-12), r0.S
+    r1 = oracle.o2_run(q, k, v, g, beta, W=4, r=1, fmt="int8", S0=S0, lib=lib)
+    assert np.allclose(r1.o.ravel(), gd["o"], atol=1e-12), r1.o
+    o1, _, _ = oracle.o1_run(q, k, v, g, beta, W=4, r=1, fmt="int8", S0=S0, lib=lib)
+    assert np.allclose(o1.ravel(), gd["o"], atol=1e-12), o1
+
+
+def pin_golden_quantizer_int8(lib):
+    gd = read("quantizer_int8_rows.txt")
+    c, s = oracle.quantize(gd["S"].reshape(4, 4), "int8", lib=lib)
+    assert np.array_equal(c.ravel(), gd["codes"].astype(np.int8)), c
+    assert np.allclose(s.ravel(), gd["scales"], rtol=1e-15, atol=0), s
+    c32, s32 = oracle.quantize(gd["S"].reshape(4, 4), "int8", prec32=True, lib=lib)
+    assert np.array_equal(c32.ravel(), gd["codes"].astype(np.int8)), c32
+
+
+def pin_golden_int4(lib):
+    gd = read("int4_g32_row.txt")
+    D = 32
+    S = np.zeros((D, D))
+    S[0, : len(gd["row0"])] = gd["row0"]
+    c, s = oracle.quantize(S, "int4_g32", lib=lib)
+    want = np.zeros(D, np.int8)
+    want[: len(gd["codes0"])] = gd["codes0"]
+    assert np.array_equal(c[0], want), c[0]
+    assert s[0, 0] == gd["scale0"][0] and s[1, 0] == 0.0 and not c[1:].any()
+    packed = oracle.pack_int4(c, lib=lib)
+    wb = np.zeros(D // 2, np.uint8)
+    wb[: len(gd["bytes0"])] = gd["bytes0"]
+    assert np.array_equal(packed[0], wb), packed[0]
+    assert np.array_equal(oracle.unpack_int4(packed, lib=lib), c)
+
+
+# ---------------------------------------------------------------------------------------------
+# Quantizer, rounding and compensator choice against library routines and bounds
+# ---------------------------------------------------------------------------------------------
+def pin_quantizer_properties(lib):
+    rng = np.random.default_rng(7)
+    D = 64   # two int4 groups per row, so a wrong group index shows
+    for fmt, qmax in (("int8", 127), ("int4_g32", 7)):
+        S = rng.standard_normal((D, D)) * rng.uniform(0.01, 50, size=(D, 1))
+        S[:, 40:] *= 7.0
+        S[5] = 0.0
+        S[9, :32] = 0.0
+        S = S.astype(np.float32).astype(np.float64)
+        for prec32 in (False, True):
+            c, s = oracle.quantize(S, fmt, prec32=prec32, lib=lib)
+            ng = s.shape[1]
+            gsz = D // ng
+            assert gsz == (32 if fmt == "int4_g32" else D)
+            deq = oracle.dequantize(c, s, fmt, lib=lib)
+            srep = np.repeat(s, gsz, axis=1)
+            assert np.all(np.abs(S - deq) <= srep / 2 * (1 + 1e-6) + 1e-300), (fmt, prec32)
+            assert np.all(np.abs(c.astype(int)) <= qmax)
+            cg = np.abs(c.astype(int)).reshape(D, ng, gsz).max(axis=-1)
+            nz = np.abs(S).reshape(D, ng, gsz).max(axis=-1) > 0
+            assert np.all(cg[nz] == qmax), (fmt, "some nonzero group lacks a full-range code")
+            assert np.all(s[~nz] == 0) and np.all(cg[~nz] == 0)
+            # the same decisions through numpy (fp64) / numpy float32 arithmetic (prec32)
+            Sg = S.reshape(D, ng, gsz)
+            if prec32:
+                m = np.abs(Sg).max(axis=-1).astype(np.float32)
+                sref = (m / np.float32(qmax)).astype(np.float32)
+                with np.errstate(divide="ignore", invalid="ignore"):
+                    t = (Sg.astype(np.float32) / sref[..., None]).astype(np.float32)
+            else:
+                sref = np.abs(Sg).max(axis=-1) / qmax
+                with np.errstate(divide="ignore", invalid="ignore"):
+                    t = Sg / sref[..., None]
+            cref = np.where(sref[..., None] == 0, 0, np.clip(np.rint(t), -qmax, qmax))
+            assert np.array_equal(c.reshape(D, ng, gsz), cref.astype(np.int8)), (fmt, prec32)
+            assert np.array_equal(s, sref.astype(np.float64)), (fmt, prec32)
+    packed = oracle.pack_int4(rng.integers(-7, 8, size=(D, D)).astype(np.int8), lib=lib)
+    assert np.array_equal(oracle.pack_int4(oracle.unpack_int4(packed, lib=lib), lib=lib), packed)
+
+
+def pin_bf16_rounding(lib):
+    rng = np.random.default_rng(11)
+    x = np.concatenate([
+        rng.standard_normal(2000) * 10.0 ** rng.uniform(-30, 30, 2000),
+        rng.standard_normal(200) * 1e-39,                     # bf16 subnormals
+        np.array([1 + 2.0**-8, 1 + 3 * 2.0**-8, -(1 + 2.0**-8), 2.0**-133, 1.5 * 2.0**-133]),
+    ]).astype(np.float32)
+    want = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    got = np.array([lib.orc_round_bf16(float(v)) for v in x])
+    assert np.array_equal(got, want), np.flatnonzero(got != want)[:10]
+    assert lib.orc_round_bf16(1 + 2.0**-8) == 1.0
+    assert lib.orc_round_bf16(1 + 3 * 2.0**-8) == 1 + 2.0**-6
+
+
+def pin_select_columns_vs_sort(lib):
+    rng = np.random.default_rng(5)
+    for trial in range(20):
+        D, r = 16, int(rng.integers(1, 6))
+        S = rng.standard_normal((D, D)) * (1 + 10 * (rng.random(D) < 0.2))
+        if trial % 4 == 0:   # exact ties of column max-abs: lower index first
+            S[:, 3] = S[:, 9] = 0.0
+            S[0, 3] = 50.0
+            S[1, 9] = -50.0
+        idx, _ = oracle.select_columns(S, r, lib=lib)
+        ref = np.argsort(-np.abs(S).max(axis=0), kind="stable")[:r]
+        assert list(idx) == list(ref), (idx, ref)
+
+
+# ---------------------------------------------------------------------------------------------
+# Closed forms of the recurrence
+# ---------------------------------------------------------------------------------------------
+def _all_forms(q, k, v, g, beta, S0=None, W=3):
+    """State and outputs from the plain, literal and buffered (unquantized) forms."""
+    out = {}
+    o, S = oracle.plain_run(q, k, v, g, beta, S0=S0, lib=_all_forms.lib)
+    out["plain"] = (o, S)
+    o1, S1, _ = oracle.o1_run(q, k, v, g, beta, W=W, fmt="none", S0=S0, lib=_all_forms.lib)
+    out["O1"] = (o1, S1)
+    for w in (W, 10 ** 6):
+        r = oracle.o2_run(q, k, v, g, beta, W=w, fmt="none", S0=S0, lib=_all_forms.lib)
+        out[f"O2 W={w}"] = (r.o, r.S)
+    return out
+
+
+def pin_single_step_from_zero(lib):
+    _all_forms.lib = lib
+    for gate in ("scalar", "diag"):
+        q, k, v, g, beta = rand_inputs(3, 1, 3, 8, gate)
+        want_S = beta[0][:, None, None] * v[0][:, :, None] * k[0][:, None, :]
+        want_o = beta[0][:, None] * v[0] * np.sum(k[0] * q[0], axis=-1)[:, None]
+        for name, (o, S) in _all_forms(q, k, v, g, beta).items():
+            close(S, want_S, 1e-13, f"{name} S1 = beta v k^T ({gate})")
+            close(o[0], want_o, 1e-13, f"{name} o1 = beta v (k.q) ({gate})")
+        for fmt in ("int8",):
+            r = oracle.o2_run(q, k, v, g, beta, W=4, fmt=fmt, lib=lib)
+            close(r.S, want_S, 1e-13, f"O2 {fmt} from zero")
+            close(r.o[0], want_o, 1e-13, f"O2 {fmt} o1 from zero")
+
+
+def pin_delta_write_at_key(lib):
+    """With |k_t| = 1: S_t k_t = (1 - beta_t) S_{t-1} Diag(a_t) k_t + beta_t v_t, any state."""
+    _all_forms.lib = lib
+    T, nh, D = 5, 2, 6
+    q, k, v, g, beta = rand_inputs(4, T, nh, D, "diag")
+    S0 = np.random.default_rng(9).standard_normal((nh, D, D))
+    prev = {name: S0 for name in ("plain", "O1", "O2 W=3", f"O2 W={10**6}")}
+    for t in range(1, T + 1):
+        forms = _all_forms(q[:t], k[:t], v[:t], g[:t], beta[:t], S0=S0)
+        for name, (_, S) in forms.items():
+            Sp = prev[name] * np.exp(g[t - 1])[:, None, :]
+            lhs = np.einsum("hij,hj->hi", S, k[t - 1])
+            rhs = (1 - beta[t - 1])[:, None] * np.einsum("hij,hj->hi", Sp, k[t - 1]) \
+                + beta[t - 1][:, None] * v[t - 1]
+            close(lhs, rhs, 1e-12, f"{name}: write identity at step {t}")
+            prev[name] = S
+
+
+def pin_exact_retrieval(lib):
+    """a = 1, beta = 1, orthonormal keys: after writing (k_i, v_i), S k_i = v_i for all i."""
+    _all_forms.lib = lib
+    D, nh = 8, 2
+    rng = np.random.default_rng(12)
+    K = np.stack([np.linalg.qr(rng.standard_normal((D, D)))[0].T for _ in range(nh)], axis=1)
+    v = rng.standard_normal((D, nh, D))
+    q = rng.standard_normal((D, nh, D))
+    g = np.zeros((D, nh))
+    beta = np.ones((D, nh))
+    S0 = rng.standard_normal((nh, D, D))
+    for name, (_, S) in _all_forms(q, K, v, g, beta, S0=S0).items():
+        got = np.einsum("hij,thj->thi", S, K)
+        close(got, v, 1e-12, f"{name}: exact retrieval")
+
+
+def pin_pure_decay(lib):
+    """beta = 0: S_t = S_0 Diag(e^{L_t}), so o_t = S_0 (e^{L_t} * q_t); the gate scales key
+    columns, not value rows."""
+    _all_forms.lib = lib
+    T, nh, D = 6, 2, 5
+    q, k, v, g, beta = rand_inputs(6, T, nh, D, "diag")
+    beta[:] = 0.0
+    S0 = np.random.default_rng(2).standard_normal((nh, D, D))
+    L = np.cumsum(g, axis=0)
+    want = np.einsum("hij,thj->thi", S0, np.exp(L) * q)
+    for name, (o, _) in _all_forms(q, k, v, g, beta, S0=S0).items():
+        close(o, want, 1e-12, f"{name}: pure decay")
+    # scalar gate, int8 state: codes survive every flush; scales pick up e^{L_W} per window
+    q, k, v, g, beta = rand_inputs(8, 12, nh, 16, "scalar")
+    beta[:] = 0.0
+    S0 = np.random.default_rng(3).standard_normal((nh, 16, 16))
+    for r in (0, 2):
+        r0 = oracle.o2_run(q[:0], k[:0], v[:0], g[:0], beta[:0], W=4, r=r, S0=S0, lib=lib)
+        r12 = oracle.o2_run(q, k, v, g, beta, W=4, r=r, S0=S0, lib=lib)
+        assert r12.pos.tolist() == [0] * nh
+        assert np.array_equal(r12.codes, r0.codes), f"codes changed under pure decay (r={r})"
+        decay = np.exp(g.sum(axis=0))[:, None, None]
+        close(r12.scales, r0.scales * decay, 1e-12, f"scales under pure decay (r={r})")
+        if r:
+            assert np.array_equal(r12.cidx, r0.cidx)
+            close(r12.cu, r0.cu * decay, 1e-12, "compensators under pure decay")
+
+
+def pin_kda_uniform_gate_is_gdn(lib):
+    T, nh, D = 20, 3, 16
+    q, k, v, g, beta = rand_inputs(21, T, nh, D, "scalar")
+    gd = np.repeat(g[..., None], D, axis=-1)
+    a = oracle.o2_run(q, k, v, g, beta, W=6, r=2, S0=None, lib=lib)
+    b = oracle.o2_run(q, k, v, gd, beta, W=6, r=2, S0=None, lib=lib)
+    assert np.array_equal(a.o, b.o) and np.array_equal(a.codes, b.codes)
+    pa, _ = oracle.plain_run(q, k, v, g, beta, lib=lib)
+    pb, _ = oracle.plain_run(q, k, v, gd, beta, lib=lib)
+    assert np.array_equal(pa, pb)
+
+
+# ---------------------------------------------------------------------------------------------
+# Agreement of the formulations
+# ---------------------------------------------------------------------------------------------
+def pin_windowed_unquantized_is_plain(lib):
+    """Buffered windows with the identity quantizer are the plain recurrence, wherever the
+    windows end (natural or forced flushes), with or without compensator pairs."""
+    T, nh, D = 19, 2, 8
+    for gate in ("scalar", "diag"):
+        q, k, v, g, beta = rand_inputs(31, T, nh, D, gate)
+        S0 = np.random.default_rng(4).standard_normal((nh, D, D))
+        po, pS = oracle.plain_run(q, k, v, g, beta, S0=S0, lib=lib)
+        mask = np.random.default_rng(8).random((T, nh)) < 0.2
+        for W in (1, 2, 3, 8):
+            for r in (0, 2):
+                for fm in (None, mask):
+                    res = oracle.o2_run(q, k, v, g, beta, W=W, r=r, fmt="none", S0=S0,
+                                        flush_mask=fm, lib=lib)
+                    close(res.o, po, 1e-12, f"O2 none W={W} r={r} {gate}")
+                    close(res.S, pS, 1e-12, f"O2 none state W={W} r={r} {gate}")
+        o1, S1, _ = oracle.o1_run(q, k, v, g, beta, W=3, fmt="none", S0=S0, lib=lib)
+        close(o1, po, 1e-12, f"O1 none {gate}")
+        close(S1, pS, 1e-12, f"O1 none state {gate}")
+
+
+def pin_literal_equals_buffered_quantized(lib):
+    """O1 (dense, requantised every W steps) equals O2 (frozen low-bit state + buffer) for
+    int8 and int4, with and without compensators; W = 1 is quantize-every-step."""
+    for fmt, D in (("int8", 8), ("int4_g32", 32)):
+        T, nh = 11, 2
+        for gate in ("scalar", "diag"):
+            q, k, v, g, beta = rand_inputs(41 + D, T, nh, D, gate)
+            S0 = np.random.default_rng(D).standard_normal((nh, D, D))
+            for W in (1, 2, 3, 8):
+                for r in (0, 2):
+                    o1, S1, _ = oracle.o1_run(q, k, v, g, beta, W=W, r=r, fmt=fmt, S0=S0, lib=lib)
+                    res = oracle.o2_run(q, k, v, g, beta, W=W, r=r, fmt=fmt, S0=S0, lib=lib)
+                    close(res.o, o1, 1e-10, f"O1 vs O2 {fmt} {gate} W={W} r={r}")
+                    close(res.S, S1, 1e-10, f"O1 vs O2 state {fmt} {gate} W={W} r={r}")
+
+
+def pin_compensator_decomposition(lib):
+    """Right after quantization: state = dequant(codes) + compensator columns, exactly; the
+    taken columns are zero in the codes; the rest is within half a step of the input."""
+    D, nh, r = 16, 3, 3
+    rng = np.random.default_rng(13)
+    S0 = rng.standard_normal((nh, D, D))
+    S0[:, :, 4] *= 30.0
+    S0[:, :, 11] *= 12.0
+    res = oracle.o2_run(np.zeros((0, nh, D)), np.zeros((0, nh, D)), np.zeros((0, nh, D)),
+                        np.zeros((0, nh)), np.zeros((0, nh)), W=4, r=r, S0=S0, lib=lib)
+    for h in range(nh):
+        ref = np.argsort(-np.abs(S0[h]).max(axis=0), kind="stable")[:r]
+        assert list(res.cidx[h]) == list(ref)
+        deq = oracle.dequantize(res.codes[h], res.scales[h], "int8", lib=lib)
+        assert not res.codes[h][:, res.cidx[h]].any()
+        rebuilt = deq.copy()
+        rebuilt[:, res.cidx[h]] += res.cu[h].T
+        assert np.array_equal(rebuilt, res.S[h])
+        assert np.array_equal(res.cu[h].T, S0[h][:, res.cidx[h]])
+        keep = np.setdiff1d(np.arange(D), res.cidx[h])
+        assert np.all(np.abs(S0[h][:, keep] - deq[:, keep]) <= res.scales[h] / 2 * (1 + 1e-12))
+
+
+def pin_storage_roundings(lib):
+    """round_storage keeps exactly what a GPU stores: bf16 write vectors, fp32 log-gates,
+    fp32 scales and compensators."""
+    T, nh, D = 10, 2, 16
+    q, k, v, g, beta = rand_inputs(51, T, nh, D, "diag")
+    S0 = np.random.default_rng(1).standard_normal((nh, D, D)).astype(np.float32)
+    res = oracle.o2_run(q, k, v, g, beta, W=16, r=2, S0=S0, round_storage=True,
+                        buf_round="bf16", lib=lib)
+    P = int(res.pos[0])
+    bu = res.bu[:, :P]
+    assert np.array_equal(bu, torch.from_numpy(bu).to(torch.bfloat16).double().numpy())
+    bL = res.bL[:, :P]
+    assert np.array_equal(bL, bL.astype(np.float32).astype(np.float64))
+    assert np.array_equal(res.scales, res.scales.astype(np.float32).astype(np.float64))
+    assert np.array_equal(res.cu, res.cu.astype(np.float32).astype(np.float64))
+    exact = oracle.o2_run(q, k, v, g, beta, W=16, r=2, S0=S0, lib=lib)
+    close(res.o, exact.o, 2e-2, "storage roundings stay small")
+
+
+PINS = [
+    pin_golden_delta_rule_kda,
+    pin_golden_window_int8,
+    pin_golden_compensator,
+    pin_golden_quantizer_int8,
+    pin_golden_int4,
+    pin_quantizer_properties,
+    pin_bf16_rounding,
+    pin_select_columns_vs_sort,
+    pin_single_step_from_zero,
+    pin_delta_write_at_key,
+    pin_exact_retrieval,
+    pin_pure_decay,
+    pin_kda_uniform_gate_is_gdn,
+    pin_windowed_unquantized_is_plain,
+    pin_literal_equals_buffered_quantized,
+    pin_compensator_decomposition,
+    pin_storage_roundings,
+]

@@ -1,0 +1,106 @@
+"""Mutation check of the oracle's pins: each case plants one plausible mistake (a dropped term, a
+wrong sign, index or operand) in a temporary copy of the oracle's C source, builds it, and
+requires at least one pin to fail on it. The real oracle is never modified."""
+import os
+
+import pytest
+
+import oracle
+from oracle import build as orc_build
+from oracle_pins import PINS
+
+MUTANTS = [
+    ("plain: delta term sign",
+     "S[(size_t)i * D + j] += -bt * w[i] * kt[j] + bt * vt[i] * kt[j];",
+     "S[(size_t)i * D + j] += bt * w[i] * kt[j] + bt * vt[i] * kt[j];"),
+    ("plain: write outer product transposed",
+     "S[(size_t)i * D + j] += -bt * w[i] * kt[j] + bt * vt[i] * kt[j];",
+     "S[(size_t)i * D + j] += -bt * w[i] * kt[j] + bt * vt[j] * kt[i];"),
+    ("plain: gate applied to value rows",
+     "for (int j = 0; j < D; ++j) S[(size_t)i * D + j] *= exp(gate_log(gt, Dg, j));",
+     "for (int j = 0; j < D; ++j) S[(size_t)i * D + j] *= exp(gate_log(gt, Dg, i));"),
+    ("plain: output from the key instead of the query",
+     "for (int j = 0; j < D; ++j) acc += S[(size_t)i * D + j] * qt[j];\n                    ot[i] = acc;\n                }\n            }\n            if (state_round",
+     "for (int j = 0; j < D; ++j) acc += S[(size_t)i * D + j] * kt[j];\n                    ot[i] = acc;\n                }\n            }\n            if (state_round"),
+    ("O1: beta dropped from the transition",
+     "((j == l ? 1.0 : 0.0) - bt * kt[j] * kt[l])",
+     "((j == l ? 1.0 : 0.0) - kt[j] * kt[l])"),
+    ("O1: gate on the wrong side of the projection",
+     "exp(gate_log(gt, Dg, j)) * ((j == l",
+     "exp(gate_log(gt, Dg, l)) * ((j == l"),
+    ("O1: window end one step early",
+     "if ((t + 1) % W == 0) ties += dense_window_end(D, fmt, r, S);",
+     "if (t % W == 0) ties += dense_window_end(D, fmt, r, S);"),
+    ("O2: beta dropped from the write vector",
+     "double u = bt * (vt[i] - w[i]);",
+     "double u = (vt[i] - w[i]);"),
+    ("O2: buffer decay factor with the wrong sign",
+     "double f = exp(Lt[j] - s->bL[(size_t)p * D + j]);",
+     "double f = exp(s->bL[(size_t)p * D + j] - Lt[j]);"),
+    ("O2: output from w instead of r",
+     "if (ot) ot[i] = rr[i] + u * kq;",
+     "if (ot) ot[i] = w[i] + u * kq;"),
+    ("O2: current write dropped from the output",
+     "if (ot) ot[i] = rr[i] + u * kq;",
+     "if (ot) ot[i] = rr[i];"),
+    ("O2: compensators dropped from the step",
+     "w[i] += s->cu[(size_t)cc * D + i] * x[j];",
+     "w[i] += 0.0 * x[j];"),
+    ("O2: key used for the query projection",
+     "y[j] = exp(Lt[j]) * qt[j];",
+     "y[j] = exp(Lt[j]) * kt[j];"),
+    ("O2: log-gate not accumulated",
+     "Lt[j] = Lt[j] + gate_log(gt, c->Dg, j);",
+     "Lt[j] = gate_log(gt, c->Dg, j);"),
+    ("O2: compensator not decayed at materialisation",
+     "S[(size_t)i * D + j] += s->cu[(size_t)cc * D + i] * exp(L[j]);",
+     "S[(size_t)i * D + j] += s->cu[(size_t)cc * D + i];"),
+    ("O2: frozen state not decayed at materialisation",
+     "S[(size_t)i * D + j] = s->F[(size_t)i * D + j] * exp(L[j]);",
+     "S[(size_t)i * D + j] = s->F[(size_t)i * D + j];"),
+    ("quantizer: int8 range 128",
+     "return fmt == ORC_FMT_INT4 ? 7 : 127;",
+     "return fmt == ORC_FMT_INT4 ? 7 : 128;"),
+    ("quantizer: ties away from zero",
+     "double r = rint(t);",
+     "double r = round(t);"),
+    ("quantizer: truncation",
+     "double r = rint(t);",
+     "double r = trunc(t);"),
+    ("quantizer: group of the wrong column",
+     "S[(size_t)i * D + j] = scales[(size_t)i * ng + j / gs] * (double)codes[(size_t)i * D + j];",
+     "S[(size_t)i * D + j] = scales[(size_t)i * ng + (D - 1 - j) / gs] * (double)codes[(size_t)i * D + j];"),
+    ("int4: nibbles swapped",
+     "packed[(size_t)i * (D / 2) + m] = (uint8_t)(lo | (hi << 4));",
+     "packed[(size_t)i * (D / 2) + m] = (uint8_t)(hi | (lo << 4));"),
+    ("compensators: ties to the higher index",
+     "if (!taken[j] && (best < 0 || colmax[j] > colmax[best])) best = j;",
+     "if (!taken[j] && (best < 0 || colmax[j] >= colmax[best])) best = j;"),
+    ("compensators: chosen by column sum instead of max-abs",
+     "for (int i = 0; i < D; ++i) colmax[j] = fmax(colmax[j], fabs(S[(size_t)i * D + j]));",
+     "for (int i = 0; i < D; ++i) colmax[j] += S[(size_t)i * D + j];"),
+    ("bf16: one mantissa bit too many",
+     "int qexp = e - 8;",
+     "int qexp = e - 9;"),
+]
+
+
+def _build_mutant(tmp_path, original, replacement):
+    src = open(orc_build.SRC).read()
+    assert src.count(original) == 1, f"mutation anchor not unique: {original!r}"
+    path = os.path.join(tmp_path, "mutant.c")
+    with open(path, "w") as f:
+        f.write(src.replace(original, replacement))
+    return orc_build.compile_oracle(path, os.path.join(tmp_path, "libmutant.so"))
+
+
+@pytest.mark.parametrize("name,original,replacement", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(name, original, replacement, tmp_path):
+    lib = oracle.load(_build_mutant(str(tmp_path), original, replacement))
+    caught = []
+    for pin in PINS:
+        try:
+            pin(lib)
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"no pin catches: {name}"

@@ -1,0 +1,472 @@
+#!/usr/bin/env python
+"""Throughput of windowed int8-state GDN decode on B200.
+
+One step = initial quantization of the fp32 states + T decode steps (one kernel launch each, the
+window flush fused into every W-th) over the whole batch of the serving-scale workload
+(B=1024 sequences x H=32 heads, d=128, T=256, W=64, bf16 q/k/v/o, int8 state with per-row
+scales). The metric is head-steps per second; one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...     (one rank per GPU, weak scaling)
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, decode_inputs, outlier_scales, step_inputs, torch_dtype  # noqa: E402
+
+METRIC = "GDN decode head-steps/s (int8 windowed state); achieved HBM GB/s vs B200 peak"
+UNIT = "head-steps/s"
+PROFILE = os.path.join(ROOT, "profiles", "window_step_gdn-serving.md")
+KERNEL_SOURCES = ["bit_recurrent_state_gdn_b200/csrc/window_kernels.cuh",
+                  "bit_recurrent_state_gdn_b200/csrc/device_util.cuh"]
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="gdnq", choices=["gdnq", "reference"])
+    p.add_argument("--workload", default="gdn-serving")
+    p.add_argument("--batch", type=int, default=None, help="override B (profiling captures)")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-baselines", action="store_true")
+    p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--cpu-heads", type=int, default=1024)
+    p.add_argument("--ref-heads", type=int, default=256)
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------------------------
+# Algorithmic bytes (what the method must move; no re-reads)
+# ---------------------------------------------------------------------------------------------
+def step_bytes(wl, P: int) -> int:
+    """HBM bytes one decode step of one head must move at window position P."""
+    D, W, r = wl.D, wl.W, wl.r
+    act = 4 if wl.act == "f32" else 2
+    buf = 4 if wl.buf == "f32" else 2
+    lbytes = 4 * D if wl.gate == "diag" else 4
+    codes = D * D // 2 if wl.fmt == "int4_g32" else D * D
+    scales = 4 * D * (D // 32 if wl.fmt == "int4_g32" else 1)
+    comps = r * (4 + 4 * D)
+    pair = D * act + D * buf + lbytes
+    io_ = 4 * D * act + (4 * D if wl.gate == "diag" else 4) + 4 + 8  # q k v o, g, beta, pos r/w
+    read = codes + scales + comps + P * pair
+    write = pair if P + 1 < W else codes + scales + comps
+    return read + write + io_
+
+
+def avg_step_bytes(wl) -> float:
+    return sum(step_bytes(wl, P) for P in range(wl.W)) / wl.W
+
+
+def baseline_bytes(wl, state_bytes: int) -> int:
+    act = 4 if wl.act == "f32" else 2
+    return 2 * wl.D * wl.D * state_bytes + 4 * wl.D * act + 8
+
+
+def peak_hbm():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic():
+    """Per-launch DRAM bytes of the window-step kernel from the committed ncu summary, if the
+    kernel source still matches the one profiled; else None."""
+    try:
+        text = open(PROFILE).read()
+    except OSError:
+        return None, None
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    s = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+    if not m or not s or s.group(1) != kernel_sha():
+        return None, None
+    return float(m.group(1)), os.path.relpath(PROFILE, ROOT)
+
+
+def kernel_sha() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+# ---------------------------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ---------------------------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        import torch
+
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", sel, f"--query-gpu={self.Q}", "--format=csv,noheader",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return []
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        return [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+
+    @staticmethod
+    def summarise(rows, t0: float, t1: float):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        mhz, maxmhz, reasons = [], None, set()
+        for r in rows:
+            try:
+                ts = time.mktime(time.strptime(r[0].strip().split(".")[0], "%Y/%m/%d %H:%M:%S"))
+            except ValueError:
+                continue
+            if ts < int(t0) or ts > t1 + 1:
+                continue
+            try:
+                mhz.append(float(r[1].split()[0]))
+                maxmhz = float(r[2].split()[0])
+            except (ValueError, IndexError):
+                continue
+            for name, val in zip(names, r[5:9]):
+                if "Active" in val and "Not" not in val:
+                    reasons.add(name)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": maxmhz,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU oracle timing (the reported CPU baseline and the reference arm)
+# ---------------------------------------------------------------------------------------------
+def time_oracle(wl, q, k, v, g, beta, S0):
+    """Head-steps/s of the oracle's buffered-window decode (storage roundings on) over the
+    given inputs ([T][n][D] numpy) from fp32 states S0 [n][D][D]."""
+    import oracle
+
+    T, n = q.shape[0], q.shape[1]
+    t0 = time.perf_counter()
+    oracle.o2_run(q, k, v, g, beta, W=wl.W, r=wl.r, fmt=wl.fmt, S0=S0, round_storage=True,
+                  buf_round=wl.buf)
+    dt = time.perf_counter() - t0
+    return n * T / dt, dt, oracle.num_threads()
+
+
+def oracle_warm_state(wl, warm):
+    import oracle
+
+    if wl.warmup == 0:
+        n = warm["q"].shape[1] if warm["q"].ndim == 3 else 0
+        return __import__("numpy").zeros((n, wl.D, wl.D))
+    _, S = oracle.plain_run(warm["q"], warm["k"], warm["v"], warm["g"], warm["beta"],
+                            state_round="f32", want_o=False)
+    return S
+
+
+def cpu_inputs(wl, device="cpu"):
+    """Warm-up and decode inputs of a (small) workload as float64 numpy [T][heads][D]."""
+    import numpy as np
+
+    def flat(t, x):
+        return x.reshape(t, wl.heads, *x.shape[3:]).double().cpu().numpy()
+
+    warm = decode_inputs(wl, device, T=wl.warmup, phase="warmup")
+    dec = decode_inputs(wl, device)
+    w = {n: flat(wl.warmup, x) for n, x in warm.items()}
+    d = {n: flat(wl.T, x) for n, x in dec.items()}
+    return w, d
+
+
+def reference_arm(args, rank, world):
+    """The oracle as the reference implementation, timed on this machine's host cores."""
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    sample = wl.with_(B=max(1, args.ref_heads // wl.H))
+    w, d = cpu_inputs(sample)
+    S0 = oracle_warm_state(sample, w)
+    times, cores = [], 1
+    for i in range(args.warmup + args.steps):
+        hs, dt, cores = time_oracle(sample, d["q"], d["k"], d["v"], d["g"], d["beta"], S0)
+        if i >= args.warmup:
+            times.append(dt)
+    per_step = statistics.mean(times)
+    value = sample.heads * sample.T / per_step
+    desc = (f"oracle buffered-window decode, {sample.heads} heads ({sample.B} sequences x "
+            f"{sample.H}) x {sample.T} steps of the {wl.name} workload per step, inputs drawn on "
+            f"the CPU with the workload's recipe")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": bench_config(wl, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def bench_config(wl, n):
+    return {"workload": wl.name, "B": wl.B, "H": wl.H, "d_k": wl.D, "d_v": wl.D, "T": wl.T,
+            "W": wl.W, "r": wl.r, "gate": wl.gate, "state": wl.fmt, "act": wl.act,
+            "buf": wl.buf, "step": f"initial quantize + {wl.T} decode steps",
+            "l2": "no flush: the per-step working set is larger than the 126 MB L2",
+            "parallelism": f"dp{n} (disjoint sequences per GPU, no collective)"}
+
+
+# ---------------------------------------------------------------------------------------------
+# The GPU arm
+# ---------------------------------------------------------------------------------------------
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        reference_arm(args, rank, world)
+        return
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import bit_recurrent_state_gdn_b200 as gdn
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    wl0 = WORKLOADS[args.workload]
+    if args.batch:
+        wl0 = wl0.with_(B=args.batch)
+    wl = wl0.with_(seed=wl0.seed + 7919 * rank)   # disjoint sequences per rank
+    cfg = gdn.make_config(wl.B, wl.H, wl.D, wl.W, wl.r, wl.gate, wl.fmt, wl.act, wl.buf)
+
+    # ---- inputs resident in HBM: decode tokens and the fp32 warm-up states ------------------
+    inp = decode_inputs(wl, dev)
+    S0 = torch.zeros((wl.B, wl.H, wl.D, wl.D), dtype=torch.float32, device=dev)
+    bcfg32 = gdn.make_config(wl.B, wl.H, wl.D, gate=wl.gate, fmt="fp32", act=wl.act)
+    scales = outlier_scales(wl, dev)
+    o_w = torch.empty((wl.B, wl.H, wl.D), dtype=torch_dtype(wl.act), device=dev)
+    for t in range(wl.warmup):
+        s = step_inputs(wl, "warmup", t, dev, scales)
+        gdn.gdn_baseline_step(bcfg32, S0, s.q, s.k, s.v, s.g, s.beta, o_w)
+    state = gdn.GdnState.allocate(cfg, dev)
+    o = torch.empty_like(inp["q"])
+    torch.cuda.synchronize()
+
+    def one_step(ev=None):
+        if ev is not None:
+            ev[0].record()
+        gdn.gdn_state_quantize(cfg, S0, state)
+        if ev is not None:
+            ev[1].record()
+        gdn.gdn_decode_window_steps(cfg, state, inp["q"], inp["k"], inp["v"], inp["g"],
+                                    inp["beta"], o)
+        if ev is not None:
+            ev[2].record()
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        one_step(evs[i])
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    clocks = ClockSampler.summarise(sampler.stop(), t_wall0, t_wall1)
+    total_ms = evs[0][0].elapsed_time(evs[-1][2])
+    decode_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    quant_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    status = int(state.status[0].item())
+    if status != 0:
+        raise RuntimeError(f"device status word {status:#x} after the timed region")
+
+    head_steps = wl.heads * wl.T * args.steps * world
+    value = head_steps / (total_ms / 1e3)
+    launches = args.steps * wl.T
+    avg_launch_s = decode_ms / 1e3 / launches
+    alg_bytes = avg_step_bytes(wl) * wl.heads
+    peak, peak_kind = peak_hbm()
+    achieved = alg_bytes / avg_launch_s / 1e9
+    traffic, traffic_src = profiled_traffic()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "state_dtype": wl.fmt,
+        "data": "synthetic (seeded; fp32 warm-up recurrence over 512 tokens makes the states)",
+        "config": bench_config(wl0, world),
+        "roofline": {
+            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "traffic": traffic,
+            "kernel": "window_step_kernel (decode step + fused window flush)",
+            "algorithmic_bytes_per_launch": alg_bytes,
+            "avg_launch_us": avg_launch_s * 1e6, "peak_source": f"{peak_kind} hbm_gbs",
+            "traffic_source": traffic_src,
+        },
+        "quantize_ms_per_step": quant_ms / args.steps,
+        "gpu_launches": args.steps * (1 + wl.T),
+        "clocks": clocks,
+    }
+
+    # ---- high-precision-state baselines on the same inputs ---------------------------------
+    if not args.no_baselines:
+        line["baselines"] = {}
+        for fmt, sdt, sbytes in (("fp32", torch.float32, 4), ("bf16", torch.bfloat16, 2)):
+            bcfg = gdn.make_config(wl.B, wl.H, wl.D, gate=wl.gate, fmt=fmt, act=wl.act)
+            S = S0.to(sdt)
+            for t in range(4):
+                gdn.gdn_baseline_step(bcfg, S, inp["q"][t], inp["k"][t], inp["v"][t],
+                                      inp["g"][t], inp["beta"][t], o[t])
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record()
+            for t in range(wl.T):
+                gdn.gdn_baseline_step(bcfg, S, inp["q"][t], inp["k"][t], inp["v"][t],
+                                      inp["g"][t], inp["beta"][t], o[t])
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            hs = wl.heads * wl.T / (ms / 1e3)
+            gbs = baseline_bytes(wl, sbytes) * wl.heads * wl.T / (ms / 1e3) / 1e9
+            line["baselines"][f"{fmt}_state"] = {
+                "value": hs * world, "unit": UNIT, "achieved_gbs": gbs, "frac": gbs / peak,
+                "ms_per_run": ms, "int8_window_speedup": value / (hs * world)}
+            del S
+
+    # ---- end to end through the host-buffer entry point ------------------------------------
+    if not args.no_e2e:
+        line["e2e"] = e2e(args, wl, cfg, inp, S0, state, world, dev)
+
+    # ---- the oracle on the host cores (rank 0, one GPU) ------------------------------------
+    if not args.no_cpu and world == 1 and rank == 0:
+        line["cpu_baseline"] = cpu_baseline(args, wl, inp, dev)
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def e2e(args, wl, cfg, inp, S0, state, world, dev):
+    import torch
+    import torch.distributed as dist
+
+    import bit_recurrent_state_gdn_b200 as gdn
+
+    host = {n: t.cpu().pin_memory() for n, t in inp.items()}
+    hS0 = S0.cpu().pin_memory()
+    ho = torch.empty(inp["q"].shape, dtype=inp["q"].dtype).pin_memory()
+    dS = torch.empty_like(S0)
+    staging = torch.empty(gdn.gdn_host_staging_bytes(cfg), dtype=torch.uint8, device=dev)
+
+    def step():
+        dS.copy_(hS0, non_blocking=True)
+        gdn.gdn_state_quantize(cfg, dS, state)
+        gdn.gdn_decode_window_steps_host(cfg, state, host["q"], host["k"], host["v"], host["g"],
+                                         host["beta"], ho, staging)
+
+    step()
+    torch.cuda.synchronize()
+    n = max(1, min(args.steps, 3))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(n):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    h2d = hS0.numel() * 4 + sum(t.numel() * t.element_size() for t in host.values())
+    d2h = ho.numel() * ho.element_size()
+    return {"value": wl.heads * wl.T * n * world / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
+            "api": "gdn_decode_window_steps_host (pinned host buffers, copies pipelined)"}
+
+
+def cpu_baseline(args, wl, inp, dev):
+    import numpy as np
+    import torch
+
+    n_seq = max(1, min(wl.B, args.cpu_heads // wl.H))
+    heads = np.arange(n_seq * wl.H)
+    idx = torch.as_tensor(heads, device=dev)
+
+    def pick(x, T):
+        flat = x.reshape(T, wl.heads, *x.shape[3:])
+        return flat.index_select(1, idx).double().cpu().numpy()
+
+    d = {n: pick(x, wl.T) for n, x in inp.items()}
+    scales = outlier_scales(wl, dev)
+    warm = {n: [] for n in ("q", "k", "v", "g", "beta")}
+    for t in range(wl.warmup):
+        s = step_inputs(wl, "warmup", t, dev, scales)
+        for n in warm:
+            x = getattr(s, n)
+            warm[n].append(x.reshape(wl.heads, *x.shape[2:]).index_select(0, idx).double()
+                           .cpu().numpy())
+    warm = {n: np.stack(v) for n, v in warm.items()}
+    S0 = oracle_warm_state(wl, warm)
+    hs, dt, cores = time_oracle(wl, d["q"], d["k"], d["v"], d["g"], d["beta"], S0)
+    return {"value": hs, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{len(heads)} heads (sequences 0..{n_seq - 1}, all {wl.H} heads) x "
+                      f"{wl.T} steps of the same inputs, {dt:.1f} s"}
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,20 @@
+"""Windowed low-bit recurrent-state GDN / KDA decode for B200 (sm_100a).
+
+Python face of libgdnq (include/gdnq.h): the functions here carry the C ABI's names and only
+marshal arguments -- torch tensors to device pointers, the current CUDA stream, status codes to
+exceptions. Every step of the computation runs in the library's CUDA kernels.
+"""
+from .api import (  # noqa: F401
+    GdnError,
+    GdnState,
+    gdn_baseline_step,
+    gdn_decode_window_step,
+    gdn_decode_window_steps,
+    gdn_decode_window_steps_host,
+    gdn_host_staging_bytes,
+    gdn_state_materialize,
+    gdn_state_quantize,
+    gdn_state_sizes,
+    gdn_window_flush,
+    make_config,
+)

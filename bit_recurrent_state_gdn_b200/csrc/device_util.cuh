@@ -1,0 +1,145 @@
+// Device helpers for the sm_100a kernels: bulk async copies (TMA, 1-D form) completing on an
+// mbarrier, a bounded mbarrier wait, and exact code / bf16 conversions.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace gdnq {
+
+// Upper bound on mbarrier polls before a kernel gives up on a staging copy and reports
+// GDN_DEVICE_WAIT_TIMEOUT instead of spinning forever.
+constexpr uint32_t kWaitPollLimit = 1u << 24;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+// Makes the initialised barrier visible to the async (TMA) proxy.
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// Global -> shared bulk copy. dst, src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n"
+      " .reg .pred p;\n"
+      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Waits for the phase with the given parity to complete; false after kWaitPollLimit polls.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kWaitPollLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// e^x through the hardware base-2 exponential (flushes results below 2^-126 to zero).
+__device__ __forceinline__ float fast_exp(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x * 1.4426950408889634f));
+  return y;
+}
+
+// ---- exact conversions -------------------------------------------------------------------
+// Four int8 codes (two's complement, byte e = code e) to fp32: bias each byte to b + 128,
+// place it in the mantissa of 2^23 (0x4B0000xx = 2^23 + xx) and subtract 2^23 + 128.
+__device__ __forceinline__ void i8x4_to_f32(uint32_t w, float* f) {
+  const uint32_t x = w ^ 0x80808080u;
+  f[0] = __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7650)) - 8388736.f;
+  f[1] = __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7651)) - 8388736.f;
+  f[2] = __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7652)) - 8388736.f;
+  f[3] = __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7653)) - 8388736.f;
+}
+
+// Eight int4 codes (one 32-bit word: byte m holds column 2m low, 2m+1 high; 4-bit two's
+// complement) to fp32 in column order: bias each nibble to c + 8 and use the same 2^23 trick.
+__device__ __forceinline__ void i4x8_to_f32(uint32_t w, float* f) {
+  const uint32_t x = w ^ 0x88888888u;
+  const uint32_t lo = x & 0x0F0F0F0Fu, hi = (x >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    f[2 * m] = __uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650 + m)) - 8388616.f;
+    f[2 * m + 1] = __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650 + m)) - 8388616.f;
+  }
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+template <typename T>
+struct Num;
+
+template <>
+struct Num<float> {
+  __device__ __forceinline__ static float to_f(float x) { return x; }
+  __device__ __forceinline__ static float from_f(float x) { return x; }
+  // n consecutive elements (n a multiple of 4, p 16-byte aligned) to fp32
+  template <int N>
+  __device__ __forceinline__ static void load(const float* p, float* out) {
+#pragma unroll
+    for (int e = 0; e < N; e += 4) {
+      const float4 t = *reinterpret_cast<const float4*>(p + e);
+      out[e] = t.x;
+      out[e + 1] = t.y;
+      out[e + 2] = t.z;
+      out[e + 3] = t.w;
+    }
+  }
+};
+
+template <>
+struct Num<__nv_bfloat16> {
+  __device__ __forceinline__ static float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+  __device__ __forceinline__ static __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+  template <int N>
+  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float* out) {
+    if constexpr (N % 8 == 0) {
+#pragma unroll
+      for (int e = 0; e < N; e += 8) {
+        const uint4 t = *reinterpret_cast<const uint4*>(p + e);
+        out[e] = bf16_lo(t.x);
+        out[e + 1] = bf16_hi(t.x);
+        out[e + 2] = bf16_lo(t.y);
+        out[e + 3] = bf16_hi(t.y);
+        out[e + 4] = bf16_lo(t.z);
+        out[e + 5] = bf16_hi(t.z);
+        out[e + 6] = bf16_lo(t.w);
+        out[e + 7] = bf16_hi(t.w);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < N; ++e) out[e] = __bfloat162float(p[e]);
+    }
+  }
+};
+
+}  // namespace gdnq

@@ -1,0 +1,30 @@
+// Internal launch interface between the C ABI (api.cu) and the kernel translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "gdnq.h"
+
+namespace gdnq {
+
+struct WinArgs;
+struct BaseArgs;
+
+enum class WinOp { Step, Flush, Materialize, Quantize };
+
+// Largest dynamic shared memory per CTA on sm_100 (bytes).
+constexpr int kMaxSmemPerCta = 227 * 1024;
+
+// Dynamic shared memory a window kernel needs for this configuration.
+size_t window_smem_bytes(const gdn_config& cfg);
+
+// Launch one window kernel over `heads` CTAs. Returns cudaErrorNotSupported for a configuration
+// that is not instantiated (the C ABI rejects those earlier).
+cudaError_t launch_window_int8(WinOp op, const gdn_config& cfg, const WinArgs& a, int heads,
+                               cudaStream_t stream);
+cudaError_t launch_window_int4(WinOp op, const gdn_config& cfg, const WinArgs& a, int heads,
+                               cudaStream_t stream);
+cudaError_t launch_baseline(const gdn_config& cfg, const BaseArgs& a, int heads,
+                            cudaStream_t stream);
+
+}  // namespace gdnq

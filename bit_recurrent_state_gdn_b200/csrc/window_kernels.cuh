@@ -1,0 +1,753 @@
+// Windowed low-bit state kernels: decode step with the fused window flush, forced flush,
+// materialisation and initial quantization. One CTA of 256 threads per (sequence, head).
+//
+// Method: "LeapQuant: Efficient Linear Attention with Accurate Recurrent State Quantization",
+// Abstract -- the state is frozen in low bits for a window of tokens; each step reads the frozen
+// state plus buffered high-precision write pairs; the state is materialised and requantised once,
+// at the window's end, with its largest-outlier key columns kept aside as compensator pairs.
+//
+// Per step, with P pairs in the window and L_t = L_{t-1} + g_t the cumulative log-gate:
+//   x = e^{L_t} k_t, y = e^{L_t} q_t
+//   w = F x + sum_c cu_c x[j_c] + sum_{i<P} bu_i <bk_i e^{L_t - bL_i}, k_t>   (= S_{t-1} Diag(a_t) k_t)
+//   r = F y + sum_c cu_c y[j_c] + sum_{i<P} bu_i <bk_i e^{L_t - bL_i}, q_t>
+//   u_t = beta_t (v_t - w), o_t = r + u_t <k_t, q_t>
+// because S_{t-1} Diag(a)(I - beta k k^T) + beta v k^T = S_{t-1} Diag(a) + beta (v - S_{t-1} Diag(a) k) k^T.
+//
+// Data path of a CTA: one thread issues bulk async copies (TMA, 1-D) of the head's codes,
+// scales, the P buffered pairs and the compensators into shared memory, all completing on one
+// mbarrier; meanwhile the CTA loads the step's q, k and gate. Then
+//   phase 1  dual mat-vec over the codes (dequantised in registers, fp32 accumulate, shuffles);
+//   phase 2  per-pair coefficients <bk_i e^{..}, k_t>, <.., q_t>;
+//   phase 3  w, r corrections from the buffered write vectors and compensators;
+//   phase 4  u_t, o_t, append the pair (to HBM, or to shared memory when the window ends);
+//   phase 5  (window end only) materialise the state tile by tile in registers, pick
+//            compensator columns, absmax, requantise, store codes / scales / compensators.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "device_util.cuh"
+#include "gdnq.h"
+
+namespace gdnq {
+
+constexpr int kThreads = 256;
+
+template <int D_, bool DIAG_, bool INT4_, typename Act_, typename Buf_>
+struct WinCfg {
+  static constexpr int D = D_;
+  static constexpr bool DIAG = DIAG_;
+  static constexpr bool INT4 = INT4_;
+  using Act = Act_;
+  using Buf = Buf_;
+  static constexpr int NT = kThreads;
+  static constexpr int QMAX = INT4 ? 7 : 127;
+  static constexpr int GS = INT4 ? 32 : D;  // columns per scale
+  static constexpr int NG = D / GS;         // scales per row
+  static constexpr int ROW_BYTES = INT4 ? D / 2 : D;
+  static constexpr int CODE_BYTES = D * ROW_BYTES;
+  static constexpr int NSCALES = D * NG;
+  // mat-vec mapping: 16 columns per thread chunk, CPR chunks per row, RPP rows per pass
+  static constexpr int CPR = D / 16;
+  static constexpr int RPP = NT / CPR;
+  // tile mapping (flush / materialise / quantize): CG column groups of TC columns, RG row
+  // groups, TR rows per thread per pass
+  static constexpr int CG = 16;
+  static constexpr int RG = NT / CG;
+  static constexpr int TC = D / CG;
+  static constexpr int TR = (D / RG) >= 2 ? 2 : 1;
+  static constexpr int RPASS = RG * TR;
+  static constexpr int NPASS = D / RPASS;
+  // phase-3 mapping: one value channel per thread, G groups over the pairs
+  static constexpr int G = NT / D;
+  static_assert(D % 16 == 0 && D <= 128, "head size");
+  static_assert(!INT4 || D % 32 == 0, "int4 needs whole groups of 32");
+  static_assert(NPASS * RPASS == D, "tile passes");
+  static_assert(TC <= GS, "a thread's columns share one scale");
+};
+
+__host__ __device__ constexpr uint32_t align128(uint32_t x) { return (x + 127u) & ~127u; }
+
+// Shared-memory layout of a window kernel (byte offsets).
+struct SmemLayout {
+  uint32_t bar, codes, scales, bk, bu, bL, cidx, cu, vec, coef, red, total;
+};
+
+__host__ __device__ inline SmemLayout window_smem_layout(int D, int code_bytes, int nscales,
+                                                         int act_size, int buf_size, bool diag,
+                                                         int W, int r) {
+  const int Wp = (W + 3) & ~3, rp = (r + 3) & ~3;
+  SmemLayout L;
+  L.bar = 0;
+  L.codes = 128;
+  L.scales = align128(L.codes + code_bytes);
+  L.bk = align128(L.scales + 4u * nscales);
+  L.bu = align128(L.bk + (uint32_t)W * D * act_size);
+  L.bL = align128(L.bu + (uint32_t)W * D * buf_size);
+  L.cidx = align128(L.bL + 4u * (diag ? (uint32_t)W * D : (uint32_t)Wp));
+  L.cu = align128(L.cidx + 4u * rp);
+  L.vec = align128(L.cu + 4u * r * D);
+  L.coef = align128(L.vec + 4u * (7 * D + 64));
+  L.red = align128(L.coef + 4u * (3 * (W + r) + 4));
+  L.total = align128(L.red + 4u * 2 * kThreads);
+  return L;
+}
+
+template <class C>
+__host__ __device__ inline SmemLayout window_smem_layout(int W, int r) {
+  return window_smem_layout(C::D, C::CODE_BYTES, C::NSCALES, (int)sizeof(typename C::Act),
+                            (int)sizeof(typename C::Buf), C::DIAG, W, r);
+}
+
+// Kernel arguments: the state's device pointers and the step's inputs (unused ones null).
+struct WinArgs {
+  uint8_t* codes;
+  float* scales;
+  void* buf_k;
+  void* buf_u;
+  float* buf_L;
+  int32_t* comp_idx;
+  float* comp_u;
+  int32_t* pos;
+  int32_t* status;
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;
+  const float* beta;
+  void* o;
+  const float* S_in;       // quantize: fp32 states
+  float* S_out;            // materialise: fp32 states
+  const int32_t* seq_mask; // forced flush: [B] or null
+  int H, W, r;
+};
+
+__device__ __forceinline__ void report(int32_t* status, int bit) {
+  if (status) atomicOr(status, bit);
+}
+
+// ------------------------------------------------------------------------------------------
+// Staging: the head's frozen state, its first P buffered pairs and its compensators, copied
+// into shared memory with bulk async copies on one mbarrier. Returns false (after reporting)
+// when the bounded wait runs out; the caller then returns. Called by all threads.
+// ------------------------------------------------------------------------------------------
+template <class C>
+__device__ __forceinline__ void stage_issue(const WinArgs& a, const SmemLayout& L, uint8_t* sm,
+                                            int head, int P) {
+  using Act = typename C::Act;
+  using Buf = typename C::Buf;
+  constexpr int D = C::D;
+  const int W = a.W, r = a.r, Wp = (W + 3) & ~3, rp = (r + 3) & ~3;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.bar);
+  const uint32_t lbytes = C::DIAG ? 4u * P * D : 4u * ((P + 3) & ~3);
+  uint32_t bytes = C::CODE_BYTES + 4u * C::NSCALES;
+  if (P > 0) bytes += (uint32_t)P * D * (sizeof(Act) + sizeof(Buf)) + lbytes;
+  if (r > 0) bytes += 4u * rp + 4u * r * D;
+  mbar_init(bar, 1);
+  fence_barrier_init();
+  mbar_arrive_expect_tx(bar, bytes);
+  bulk_g2s(sm + L.codes, a.codes + (size_t)head * C::CODE_BYTES, C::CODE_BYTES, bar);
+  bulk_g2s(sm + L.scales, a.scales + (size_t)head * C::NSCALES, 4u * C::NSCALES, bar);
+  if (P > 0) {
+    bulk_g2s(sm + L.bk, static_cast<const Act*>(a.buf_k) + (size_t)head * W * D,
+             (uint32_t)P * D * sizeof(Act), bar);
+    bulk_g2s(sm + L.bu, static_cast<const Buf*>(a.buf_u) + (size_t)head * W * D,
+             (uint32_t)P * D * sizeof(Buf), bar);
+    bulk_g2s(sm + L.bL, a.buf_L + (size_t)head * (C::DIAG ? (size_t)W * D : (size_t)Wp), lbytes,
+             bar);
+  }
+  if (r > 0) {
+    bulk_g2s(sm + L.cidx, a.comp_idx + (size_t)head * rp, 4u * rp, bar);
+    bulk_g2s(sm + L.cu, a.comp_u + (size_t)head * r * D, 4u * r * D, bar);
+  }
+}
+
+__device__ __forceinline__ bool stage_wait(const WinArgs& a, const SmemLayout& L, uint8_t* sm) {
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.bar);
+  const int timed_out = mbar_wait_bounded(bar, 0) ? 0 : 1;
+  if (__syncthreads_or(timed_out)) {
+    if (threadIdx.x == 0) report(a.status, GDN_DEVICE_WAIT_TIMEOUT);
+    return false;
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------------------------------
+// Tile makers: fill acc[TR][TC] with the fp32 logical state at rows of pass `ps` and the
+// thread's columns. Thread (rg, cg) = (tid / CG, tid % CG) owns rows ps*RPASS + rg*TR + a and
+// columns cg*TC + b.
+// ------------------------------------------------------------------------------------------
+
+// Logical state from the staged window: frozen codes scaled by e^{L_end} (per column), plus
+// compensators, plus `npairs` buffered pairs. Before use, `colexp` holds e^{L_end[j]} for all
+// columns; for the scalar gate `fac[i]` holds e^{L_end - bL_i}; for the diagonal gate the bL
+// region holds kt_i[j] = bk_i[j] e^{L_end[j] - bL_i[j]} in fp32.
+template <class C>
+struct WindowTile {
+  const uint8_t* codes;
+  const float* scales;
+  const typename C::Act* bk;
+  const typename C::Buf* bu;
+  const float* ktil;
+  const float* fac;
+  const int32_t* cidx;
+  const float* cu;
+  const float* colexp;
+  int npairs, r;
+
+  __device__ __forceinline__ void operator()(int ps, float (&acc)[C::TR][C::TC]) const {
+    constexpr int D = C::D, TC = C::TC, TR = C::TR;
+    const int tid = threadIdx.x, cg = tid % C::CG, rg = tid / C::CG;
+    const int c0 = cg * TC;
+    float ce[TC];
+#pragma unroll
+    for (int b = 0; b < TC; ++b) ce[b] = colexp[c0 + b];
+#pragma unroll
+    for (int a = 0; a < TR; ++a) {
+      const int row = ps * C::RPASS + rg * TR + a;
+      float cv[TC];
+      if constexpr (C::INT4) {
+        static_assert(TC == 8, "int4 tile is 8 columns per thread");
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(codes + row * C::ROW_BYTES + c0 / 2);
+        i4x8_to_f32(w, cv);
+      } else if constexpr (TC == 8) {
+        const uint2 w = *reinterpret_cast<const uint2*>(codes + row * C::ROW_BYTES + c0);
+        i8x4_to_f32(w.x, cv);
+        i8x4_to_f32(w.y, cv + 4);
+      } else {
+#pragma unroll
+        for (int b = 0; b < TC; ++b)
+          cv[b] = (float)(int)reinterpret_cast<const int8_t*>(codes)[row * C::ROW_BYTES + c0 + b];
+      }
+      const float s = scales[row * C::NG + c0 / C::GS];
+#pragma unroll
+      for (int b = 0; b < TC; ++b) acc[a][b] = s * cv[b] * ce[b];
+    }
+    for (int c = 0; c < r; ++c) {
+      const int j = cidx[c];
+      if (j / TC == cg) {
+#pragma unroll
+        for (int b = 0; b < TC; ++b)
+          if (c0 + b == j) {
+#pragma unroll
+            for (int a = 0; a < TR; ++a)
+              acc[a][b] += cu[c * D + ps * C::RPASS + rg * TR + a] * ce[b];
+          }
+      }
+    }
+    for (int i = 0; i < npairs; ++i) {
+      float uu[TR], kk[TC];
+#pragma unroll
+      for (int a = 0; a < TR; ++a)
+        uu[a] = Num<typename C::Buf>::to_f(bu[i * D + ps * C::RPASS + rg * TR + a]);
+      if constexpr (C::DIAG) {
+#pragma unroll
+        for (int b = 0; b < TC; ++b) kk[b] = ktil[i * D + c0 + b];
+      } else {
+        if constexpr (TC % 8 == 0 || (TC % 4 == 0 && sizeof(typename C::Act) == 4)) {
+          Num<typename C::Act>::template load<TC>(bk + i * D + c0, kk);
+        } else {
+#pragma unroll
+          for (int b = 0; b < TC; ++b) kk[b] = Num<typename C::Act>::to_f(bk[i * D + c0 + b]);
+        }
+        const float f = fac[i];
+#pragma unroll
+        for (int a = 0; a < TR; ++a) uu[a] *= f;
+      }
+#pragma unroll
+      for (int a = 0; a < TR; ++a)
+#pragma unroll
+        for (int b = 0; b < TC; ++b) acc[a][b] = fmaf(uu[a], kk[b], acc[a][b]);
+    }
+  }
+};
+
+// fp32 states straight from HBM (initial quantization).
+template <class C>
+struct DenseTile {
+  const float* S;  // this head's [D][D]
+  __device__ __forceinline__ void operator()(int ps, float (&acc)[C::TR][C::TC]) const {
+    const int tid = threadIdx.x, cg = tid % C::CG, rg = tid / C::CG;
+#pragma unroll
+    for (int a = 0; a < C::TR; ++a) {
+      const int row = ps * C::RPASS + rg * C::TR + a;
+      if constexpr (C::TC % 4 == 0) {
+        Num<float>::load<C::TC>(S + (size_t)row * C::D + cg * C::TC, acc[a]);
+      } else {
+#pragma unroll
+        for (int b = 0; b < C::TC; ++b) acc[a][b] = S[(size_t)row * C::D + cg * C::TC + b];
+      }
+    }
+  }
+};
+
+// ------------------------------------------------------------------------------------------
+// Requantisation of the state that `make` produces: compensator columns (top r by max-abs,
+// ties to the lower index) go to comp_u / comp_idx in fp32 and are zeroed; each row (int4: each
+// 32-column group) gets s = absmax / QMAX and codes rint(x / s) clamped to [-QMAX, QMAX], both
+// with IEEE single division. Codes, scales and compensators are written straight to HBM; the
+// tile maker may still read the staged old state because rows of later passes are untouched
+// and the old compensators live in shared memory. `colmax` (D floats) and `sel` (r ints) are
+// shared scratch. Called by all threads.
+// ------------------------------------------------------------------------------------------
+template <class C, class Maker>
+__device__ void requantize_store(const Maker& make, int r, uint8_t* g_codes, float* g_scales,
+                                 int32_t* g_cidx, float* g_cu, float* colmax, int32_t* sel) {
+  constexpr int D = C::D, TR = C::TR, TC = C::TC, QMAX = C::QMAX;
+  const int tid = threadIdx.x, cg = tid % C::CG, rg = tid / C::CG;
+  const int lane = tid & 31, warp = tid >> 5;
+  float acc[TR][TC];
+
+  if (r > 0) {
+    for (int j = tid; j < D; j += C::NT) colmax[j] = 0.f;
+    __syncthreads();
+    for (int ps = 0; ps < C::NPASS; ++ps) {
+      make(ps, acc);
+#pragma unroll
+      for (int b = 0; b < TC; ++b) {
+        float m = 0.f;
+#pragma unroll
+        for (int a = 0; a < TR; ++a) m = fmaxf(m, fabsf(acc[a][b]));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+        if (lane < 16)
+          atomicMax(reinterpret_cast<unsigned int*>(colmax) + cg * TC + b, __float_as_uint(m));
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      for (int c = 0; c < r; ++c) {
+        float bv = -1.f;
+        int bj = D;
+        for (int j = lane; j < D; j += 32) {
+          const float v = colmax[j];
+          if (v > bv) { bv = v; bj = j; }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+          const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
+          if (ov > bv || (ov == bv && oj < bj)) { bv = ov; bj = oj; }
+        }
+        if (lane == 0) {
+          sel[c] = bj;
+          colmax[bj] = -2.f;  // taken
+        }
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+  }
+
+  for (int ps = 0; ps < C::NPASS; ++ps) {
+    make(ps, acc);
+    for (int c = 0; c < r; ++c) {
+      const int j = sel[c];
+      if (j / TC == cg) {
+#pragma unroll
+        for (int b = 0; b < TC; ++b)
+          if (cg * TC + b == j) {
+#pragma unroll
+            for (int a = 0; a < TR; ++a) {
+              g_cu[c * D + ps * C::RPASS + rg * TR + a] = acc[a][b];
+              acc[a][b] = 0.f;
+            }
+          }
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < TR; ++a) {
+      const int row = ps * C::RPASS + rg * TR + a;
+      float m = 0.f;
+#pragma unroll
+      for (int b = 0; b < TC; ++b) m = fmaxf(m, fabsf(acc[a][b]));
+      // lanes sharing a scale: 16 column groups per row (int8), 4 per 32-column group (int4)
+      constexpr int span = C::GS / TC;
+#pragma unroll
+      for (int off = span / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      const float s = __fdiv_rn(m, (float)QMAX);
+      int q[TC];
+#pragma unroll
+      for (int b = 0; b < TC; ++b) {
+        float t = s > 0.f ? rintf(__fdiv_rn(acc[a][b], s)) : 0.f;
+        t = fminf(fmaxf(t, (float)-QMAX), (float)QMAX);
+        q[b] = (int)t;
+      }
+      if constexpr (C::INT4) {
+        uint32_t wv = 0;
+#pragma unroll
+        for (int m2 = 0; m2 < TC / 2; ++m2)
+          wv |= (((uint32_t)q[2 * m2] & 0xFu) | (((uint32_t)q[2 * m2 + 1] & 0xFu) << 4)) << (8 * m2);
+        *reinterpret_cast<uint32_t*>(g_codes + row * C::ROW_BYTES + cg * TC / 2) = wv;
+        if (cg % span == 0) g_scales[row * C::NG + (cg * TC) / C::GS] = s;
+      } else {
+        if constexpr (TC == 8) {
+          uint2 wv;
+          wv.x = ((uint32_t)q[0] & 0xFFu) | (((uint32_t)q[1] & 0xFFu) << 8) |
+                 (((uint32_t)q[2] & 0xFFu) << 16) | (((uint32_t)q[3] & 0xFFu) << 24);
+          wv.y = ((uint32_t)q[4] & 0xFFu) | (((uint32_t)q[5] & 0xFFu) << 8) |
+                 (((uint32_t)q[6] & 0xFFu) << 16) | (((uint32_t)q[7] & 0xFFu) << 24);
+          *reinterpret_cast<uint2*>(g_codes + row * C::ROW_BYTES + cg * TC) = wv;
+        } else {
+#pragma unroll
+          for (int b = 0; b < TC; ++b)
+            reinterpret_cast<int8_t*>(g_codes)[row * C::ROW_BYTES + cg * TC + b] = (int8_t)q[b];
+        }
+        if (cg == 0) g_scales[row] = s;
+      }
+    }
+  }
+  if (tid < r) g_cidx[tid] = sel[tid];
+}
+
+// Window-end preparation in shared memory for the logical state at cumulative gate `Lend`
+// (per column in `Lvec` for the diagonal gate, scalar `Ls` otherwise) over `npairs` staged
+// pairs: colexp[j] = e^{Lend[j]}; scalar gate: fac[i] = e^{Lend - bL_i}; diagonal gate: the bL
+// region becomes bk_i[j] e^{Lend[j] - bL_i[j]} (fp32, in place).
+template <class C>
+__device__ __forceinline__ void prepare_window_end(uint8_t* sm, const SmemLayout& L, int npairs,
+                                                   const float* Lvec, float Ls, float* colexp,
+                                                   float* fac) {
+  constexpr int D = C::D;
+  float* bL = reinterpret_cast<float*>(sm + L.bL);
+  const typename C::Act* bk = reinterpret_cast<const typename C::Act*>(sm + L.bk);
+  for (int j = threadIdx.x; j < D; j += C::NT) colexp[j] = fast_exp(C::DIAG ? Lvec[j] : Ls);
+  if constexpr (C::DIAG) {
+    for (int e = threadIdx.x; e < npairs * D; e += C::NT) {
+      const int j = e % D;
+      bL[e] = Num<typename C::Act>::to_f(bk[e]) * fast_exp(Lvec[j] - bL[e]);
+    }
+  } else {
+    for (int i = threadIdx.x; i < npairs; i += C::NT) fac[i] = fast_exp(Ls - bL[i]);
+  }
+}
+
+template <class C>
+__device__ __forceinline__ WindowTile<C> window_tile(uint8_t* sm, const SmemLayout& L, int npairs,
+                                                     int r, const float* colexp,
+                                                     const float* fac) {
+  WindowTile<C> t;
+  t.codes = sm + L.codes;
+  t.scales = reinterpret_cast<const float*>(sm + L.scales);
+  t.bk = reinterpret_cast<const typename C::Act*>(sm + L.bk);
+  t.bu = reinterpret_cast<const typename C::Buf*>(sm + L.bu);
+  t.ktil = reinterpret_cast<const float*>(sm + L.bL);
+  t.fac = fac;
+  t.cidx = reinterpret_cast<const int32_t*>(sm + L.cidx);
+  t.cu = reinterpret_cast<const float*>(sm + L.cu);
+  t.colexp = colexp;
+  t.npairs = npairs;
+  t.r = r;
+  return t;
+}
+
+// ------------------------------------------------------------------------------------------
+// Decode step (+ fused window flush).
+// ------------------------------------------------------------------------------------------
+template <class C>
+__global__ void __launch_bounds__(kThreads) window_step_kernel(const WinArgs a) {
+  using Act = typename C::Act;
+  using Buf = typename C::Buf;
+  constexpr int D = C::D, CPR = C::CPR, RPP = C::RPP;
+  extern __shared__ __align__(128) uint8_t sm[];
+  const SmemLayout L = window_smem_layout<C>(a.W, a.r);
+  const int head = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+  const int W = a.W, r = a.r, Wp = (W + 3) & ~3;
+
+  const int P = a.pos[head];
+  if (P < 0 || P >= W) {
+    if (tid == 0) report(a.status, GDN_DEVICE_BAD_POS);
+    return;
+  }
+  const bool flush = (P + 1 == W);
+  if (tid == 0) stage_issue<C>(a, L, sm, head, P);
+
+  float* vec = reinterpret_cast<float*>(sm + L.vec);
+  float *kt = vec, *qt = vec + D, *xs = vec + 2 * D, *ys = vec + 3 * D, *Lt = vec + 4 * D;
+  float *pv = vec + 5 * D, *rv = vec + 6 * D, *misc = vec + 7 * D;  // misc: kq, sel (as int)
+  float* coef = reinterpret_cast<float*>(sm + L.coef);
+  float *ca = coef, *cb = coef + (W + r), *fac = coef + 2 * (W + r);
+  float* red = reinterpret_cast<float*>(sm + L.red);
+
+  const Act* kin = static_cast<const Act*>(a.k) + (size_t)head * D;
+  const Act* qin = static_cast<const Act*>(a.q) + (size_t)head * D;
+  const float* gL = a.buf_L + (size_t)head * (C::DIAG ? (size_t)W * D : (size_t)Wp);
+  float Ls = 0.f;  // scalar-gate L_t
+  if constexpr (!C::DIAG) Ls = (P > 0 ? gL[P - 1] : 0.f) + a.g[head];
+  if (tid < D) {
+    const float kj = Num<Act>::to_f(kin[tid]), qj = Num<Act>::to_f(qin[tid]);
+    kt[tid] = kj;
+    qt[tid] = qj;
+    float l;
+    if constexpr (C::DIAG) l = (P > 0 ? gL[(size_t)(P - 1) * D + tid] : 0.f) + a.g[(size_t)head * D + tid];
+    else l = Ls;
+    Lt[tid] = l;
+    const float e = fast_exp(l);
+    xs[tid] = e * kj;
+    ys[tid] = e * qj;
+  }
+  __syncthreads();
+  if (!stage_wait(a, L, sm)) return;
+
+  const uint8_t* s_codes = sm + L.codes;
+  const float* s_scales = reinterpret_cast<const float*>(sm + L.scales);
+  Act* s_bk = reinterpret_cast<Act*>(sm + L.bk);
+  Buf* s_bu = reinterpret_cast<Buf*>(sm + L.bu);
+  float* s_bL = reinterpret_cast<float*>(sm + L.bL);
+  const int32_t* s_cidx = reinterpret_cast<const int32_t*>(sm + L.cidx);
+  const float* s_cu = reinterpret_cast<const float*>(sm + L.cu);
+
+  // ---- phase 1: p = F x, r = F y ---------------------------------------------------------
+  {
+    const int c = tid % CPR;
+    float xr[16], yr[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      xr[e] = xs[c * 16 + e];
+      yr[e] = ys[c * 16 + e];
+    }
+    for (int row = tid / CPR; row < D; row += RPP) {
+      float cv[16];
+      if constexpr (C::INT4) {
+        const uint2 w = *reinterpret_cast<const uint2*>(s_codes + row * C::ROW_BYTES + c * 8);
+        i4x8_to_f32(w.x, cv);
+        i4x8_to_f32(w.y, cv + 8);
+      } else {
+        const uint4 w = *reinterpret_cast<const uint4*>(s_codes + row * C::ROW_BYTES + c * 16);
+        i8x4_to_f32(w.x, cv);
+        i8x4_to_f32(w.y, cv + 4);
+        i8x4_to_f32(w.z, cv + 8);
+        i8x4_to_f32(w.w, cv + 12);
+      }
+      float pa = 0.f, pb = 0.f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        pa = fmaf(cv[e], xr[e], pa);
+        pb = fmaf(cv[e], yr[e], pb);
+      }
+      if constexpr (C::INT4) {
+        const float s = s_scales[row * C::NG + (c * 16) / C::GS];
+        pa *= s;
+        pb *= s;
+      }
+#pragma unroll
+      for (int off = CPR / 2; off > 0; off >>= 1) {
+        pa += __shfl_xor_sync(0xffffffffu, pa, off);
+        pb += __shfl_xor_sync(0xffffffffu, pb, off);
+      }
+      if (c == 0) {
+        if constexpr (C::INT4) {
+          pv[row] = pa;
+          rv[row] = pb;
+        } else {
+          const float s = s_scales[row];
+          pv[row] = pa * s;
+          rv[row] = pb * s;
+        }
+      }
+    }
+  }
+
+  // ---- phase 2: pair coefficients -------------------------------------------------------
+  {
+    const int c = tid % CPR;
+    float kr[16], qr[16], lr[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      kr[e] = kt[c * 16 + e];
+      qr[e] = qt[c * 16 + e];
+      if constexpr (C::DIAG) lr[e] = Lt[c * 16 + e];
+    }
+    const int npass = (P + RPP - 1) / RPP;
+    for (int ps = 0; ps < npass; ++ps) {
+      const int i = ps * RPP + tid / CPR;
+      float pa = 0.f, pb = 0.f;
+      if (i < P) {
+        float kk[16];
+        if constexpr (sizeof(Act) == 2) Num<Act>::template load<16>(s_bk + i * D + c * 16, kk);
+        else Num<Act>::template load<16>(s_bk + i * D + c * 16, kk);
+        if constexpr (C::DIAG) {
+          float ll[16];
+          Num<float>::load<16>(s_bL + i * D + c * 16, ll);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) kk[e] *= fast_exp(lr[e] - ll[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          pa = fmaf(kk[e], kr[e], pa);
+          pb = fmaf(kk[e], qr[e], pb);
+        }
+      }
+#pragma unroll
+      for (int off = CPR / 2; off > 0; off >>= 1) {
+        pa += __shfl_xor_sync(0xffffffffu, pa, off);
+        pb += __shfl_xor_sync(0xffffffffu, pb, off);
+      }
+      if (c == 0 && i < P) {
+        if constexpr (!C::DIAG) {
+          const float f = fast_exp(Ls - s_bL[i]);
+          pa *= f;
+          pb *= f;
+        }
+        ca[i] = pa;
+        cb[i] = pb;
+      }
+    }
+    if (tid < r) {  // compensator pairs: key e_j entered at L = 0
+      const int j = s_cidx[tid] & (D - 1);  // in range even for a never-quantized state
+      ca[W + tid] = xs[j];
+      cb[W + tid] = ys[j];
+    }
+    if (tid < 32) {
+      float s = 0.f;
+      for (int j = lane; j < D; j += 32) s = fmaf(kt[j], qt[j], s);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+      if (lane == 0) misc[0] = s;
+    }
+  }
+  __syncthreads();
+
+  // ---- phase 3: corrections from the buffered write vectors and compensators -------------
+  {
+    const int v = tid % D, grp = tid / D;
+    float aw = 0.f, ar = 0.f;
+    for (int i = grp; i < P; i += C::G) {
+      const float u = Num<Buf>::to_f(s_bu[i * D + v]);
+      aw = fmaf(ca[i], u, aw);
+      ar = fmaf(cb[i], u, ar);
+    }
+    for (int cc = grp; cc < r; cc += C::G) {
+      const float u = s_cu[cc * D + v];
+      aw = fmaf(ca[W + cc], u, aw);
+      ar = fmaf(cb[W + cc], u, ar);
+    }
+    red[grp * 2 * D + v] = aw;
+    red[grp * 2 * D + D + v] = ar;
+  }
+  __syncthreads();
+
+  // ---- phase 4: write vector, output, append -------------------------------------------
+  if (tid < D) {
+    const int v = tid;
+    float w = pv[v], rr = rv[v];
+#pragma unroll
+    for (int gi = 0; gi < C::G; ++gi) {
+      w += red[gi * 2 * D + v];
+      rr += red[gi * 2 * D + D + v];
+    }
+    const float vin = Num<Act>::to_f(static_cast<const Act*>(a.v)[(size_t)head * D + v]);
+    const float u = a.beta[head] * (vin - w);
+    const Buf ub = Num<Buf>::from_f(u);
+    const float ur = Num<Buf>::to_f(ub);
+    static_cast<Act*>(a.o)[(size_t)head * D + v] = Num<Act>::from_f(rr + ur * misc[0]);
+    if (!flush) {
+      static_cast<Buf*>(a.buf_u)[((size_t)head * W + P) * D + v] = ub;
+      static_cast<Act*>(a.buf_k)[((size_t)head * W + P) * D + v] = kin[v];
+      if constexpr (C::DIAG) a.buf_L[((size_t)head * W + P) * D + v] = Lt[v];
+    } else {
+      s_bu[P * D + v] = ub;
+      s_bk[P * D + v] = kin[v];
+      if constexpr (C::DIAG) s_bL[P * D + v] = Lt[v];
+    }
+  }
+  if (tid == 0) {
+    if constexpr (!C::DIAG) {
+      if (!flush) a.buf_L[(size_t)head * Wp + P] = Ls;
+      else s_bL[P] = Ls;
+    }
+    a.pos[head] = flush ? 0 : P + 1;
+  }
+  if (!flush) return;
+
+  // ---- phase 5: window end -------------------------------------------------------------
+  __syncthreads();
+  float* colexp = xs;  // x, y are dead
+  prepare_window_end<C>(sm, L, P + 1, Lt, Ls, colexp, fac);
+  __syncthreads();
+  const WindowTile<C> tile = window_tile<C>(sm, L, P + 1, r, colexp, fac);
+  requantize_store<C>(tile, r, a.codes + (size_t)head * C::CODE_BYTES,
+                      a.scales + (size_t)head * C::NSCALES,
+                      a.comp_idx + (size_t)head * ((r + 3) & ~3), a.comp_u + (size_t)head * r * D,
+                      ys, reinterpret_cast<int32_t*>(misc + 4));
+}
+
+// ------------------------------------------------------------------------------------------
+// Forced flush (mode 0) and materialisation (mode 1) of the logical state at the current pos.
+// ------------------------------------------------------------------------------------------
+template <class C, int MODE>
+__global__ void __launch_bounds__(kThreads) window_state_kernel(const WinArgs a) {
+  constexpr int D = C::D;
+  extern __shared__ __align__(128) uint8_t sm[];
+  const SmemLayout L = window_smem_layout<C>(a.W, a.r);
+  const int head = blockIdx.x, tid = threadIdx.x;
+  const int W = a.W, r = a.r;
+  const int P = a.pos[head];
+  if (P < 0 || P >= W) {
+    if (tid == 0) report(a.status, GDN_DEVICE_BAD_POS);
+    return;
+  }
+  if (MODE == 0) {
+    if (P == 0) return;
+    if (a.seq_mask && a.seq_mask[head / a.H] == 0) return;
+  }
+  if (tid == 0) stage_issue<C>(a, L, sm, head, P);
+  __syncthreads();
+  if (!stage_wait(a, L, sm)) return;
+
+  float* vec = reinterpret_cast<float*>(sm + L.vec);
+  float *Lend = vec, *colexp = vec + D, *colmax = vec + 2 * D;
+  int32_t* sel = reinterpret_cast<int32_t*>(vec + 7 * D);
+  float* fac = reinterpret_cast<float*>(sm + L.coef);
+  const float* s_bL = reinterpret_cast<const float*>(sm + L.bL);
+  float Ls = 0.f;
+  if constexpr (C::DIAG) {
+    for (int j = tid; j < D; j += C::NT) Lend[j] = P > 0 ? s_bL[(P - 1) * D + j] : 0.f;
+  } else {
+    Ls = P > 0 ? s_bL[P - 1] : 0.f;
+  }
+  __syncthreads();
+  prepare_window_end<C>(sm, L, P, Lend, Ls, colexp, fac);
+  __syncthreads();
+  const WindowTile<C> tile = window_tile<C>(sm, L, P, r, colexp, fac);
+  if constexpr (MODE == 0) {
+    requantize_store<C>(tile, r, a.codes + (size_t)head * C::CODE_BYTES,
+                        a.scales + (size_t)head * C::NSCALES,
+                        a.comp_idx + (size_t)head * ((r + 3) & ~3),
+                        a.comp_u + (size_t)head * r * D, colmax, sel);
+    if (tid == 0) a.pos[head] = 0;
+  } else {
+    const int cg = tid % C::CG, rg = tid / C::CG;
+    float acc[C::TR][C::TC];
+    float* out = a.S_out + (size_t)head * D * D;
+    for (int ps = 0; ps < C::NPASS; ++ps) {
+      tile(ps, acc);
+#pragma unroll
+      for (int aa = 0; aa < C::TR; ++aa) {
+        const int row = ps * C::RPASS + rg * C::TR + aa;
+#pragma unroll
+        for (int b = 0; b < C::TC; ++b) out[(size_t)row * D + cg * C::TC + b] = acc[aa][b];
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Initial quantization of fp32 states.
+// ------------------------------------------------------------------------------------------
+template <class C>
+__global__ void __launch_bounds__(kThreads) quantize_kernel(const WinArgs a) {
+  constexpr int D = C::D;
+  __shared__ float colmax[D];
+  __shared__ int32_t sel[GDN_MAX_COMPENSATORS];
+  const int head = blockIdx.x;
+  DenseTile<C> tile;
+  tile.S = a.S_in + (size_t)head * D * D;
+  requantize_store<C>(tile, a.r, a.codes + (size_t)head * C::CODE_BYTES,
+                      a.scales + (size_t)head * C::NSCALES,
+                      a.comp_idx + (size_t)head * ((a.r + 3) & ~3),
+                      a.comp_u + (size_t)head * a.r * D, colmax, sel);
+  if (threadIdx.x == 0) a.pos[head] = 0;
+}
+
+}  // namespace gdnq

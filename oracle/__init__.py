@@ -75,7 +75,7 @@ def load(path: Optional[str] = None):
     lib.orc_o1_run.restype = _int
     lib.orc_o1_run.argtypes = [_int] * 7 + [_vp] * 8
     lib.orc_o2_run.restype = _int
-    lib.orc_o2_run.argtypes = [_int] * 9 + [_vp] * 17
+    lib.orc_o2_run.argtypes = [_int] * 9 + [_vp] * 18
     if path == _build.OUT:
         _lib, _lib_path = lib, path
     return lib
@@ -205,6 +205,7 @@ class O2Result:
     bL: np.ndarray         # [nh][W][D]
     S: np.ndarray          # [nh][D][D] logical state at the end
     near_ties: int
+    ties: np.ndarray       # [nh] near ties per head
 
 
 def o2_run(q, k, v, g, beta, W: int, r: int = 0, fmt: str = "int8", S0=None,
@@ -224,11 +225,11 @@ def o2_run(q, k, v, g, beta, W: int, r: int = 0, fmt: str = "int8", S0=None,
         scales=np.zeros((nh, D, ng)), cidx=np.zeros((nh, max(r, 0)), np.int32),
         cu=np.zeros((nh, max(r, 0), D)), pos=np.zeros(nh, np.int32),
         bk=np.zeros((nh, W, D)), bu=np.zeros((nh, W, D)), bL=np.zeros((nh, W, D)),
-        S=np.zeros((nh, D, D)), near_ties=0)
+        S=np.zeros((nh, D, D)), near_ties=0, ties=np.zeros(nh, np.int32))
     fm = None if flush_mask is None else np.ascontiguousarray(flush_mask, np.uint8).reshape(T, nh)
     res.near_ties = lib.orc_o2_run(
         D, T, W, r, f, nh, Dg, int(round_storage), _ROUND[buf_round], _p(S0), _p(q), _p(k),
         _p(v), _p(g), _p(beta), _p(fm), _p(res.o), _p(res.codes), _p(res.scales),
         _p(res.cidx) if r > 0 else None, _p(res.cu) if r > 0 else None, _p(res.pos),
-        _p(res.bk), _p(res.bu), _p(res.bL), _p(res.S))
+        _p(res.bk), _p(res.bu), _p(res.bL), _p(res.S), _p(res.ties))
     return res

@@ -227,6 +227,7 @@ void orc_plain_run(int D, int T, int nh, int Dg, int state_round, const double* 
     for (int h = 0; h < nh; ++h) {
         double* S = (double*)malloc(sizeof(double) * (size_t)D * D);
         double* w = (double*)malloc(sizeof(double) * (size_t)D);
+        double* a = (double*)malloc(sizeof(double) * (size_t)D);
         if (S0) memcpy(S, S0 + (size_t)h * D * D, sizeof(double) * (size_t)D * D);
         else memset(S, 0, sizeof(double) * (size_t)D * D);
         for (int t = 0; t < T; ++t) {
@@ -235,8 +236,9 @@ void orc_plain_run(int D, int T, int nh, int Dg, int state_round, const double* 
             const double* vt = v + ((size_t)t * nh + h) * D;
             const double* gt = g + ((size_t)t * nh + h) * Dg;
             double bt = beta[(size_t)t * nh + h];
+            for (int j = 0; j < D; ++j) a[j] = exp(gate_log(gt, Dg, j));
             for (int i = 0; i < D; ++i)          /* S' = S Diag(a) */
-                for (int j = 0; j < D; ++j) S[(size_t)i * D + j] *= exp(gate_log(gt, Dg, j));
+                for (int j = 0; j < D; ++j) S[(size_t)i * D + j] *= a[j];
             for (int i = 0; i < D; ++i) {        /* w = S' k */
                 double acc = 0.0;
                 for (int j = 0; j < D; ++j) acc += S[(size_t)i * D + j] * kt[j];
@@ -259,6 +261,7 @@ void orc_plain_run(int D, int T, int nh, int Dg, int state_round, const double* 
         if (S_out) memcpy(S_out + (size_t)h * D * D, S, sizeof(double) * (size_t)D * D);
         free(S);
         free(w);
+        free(a);
     }
 }
 
@@ -359,8 +362,9 @@ int orc_o1_run(int D, int T, int W, int r, int fmt, int nh, int Dg, const double
  *
  * Outputs (any may be NULL): o [T][nh][D]; codes [nh][D][D]; scales [nh][D][groups];
  * cidx [nh][r]; cu [nh][r][D]; pos [nh]; bk, bu, bL [nh][W][D]; S_out [nh][D][D] (the logical
- * state at the end); flush_mask [T][nh] forces a flush after step t of head h when nonzero.
- * Returns the number of near ties met in compensator choices.
+ * state at the end); ties_out [nh] (near ties met per head); flush_mask [T][nh] forces a flush
+ * after step t of head h when nonzero. Returns the number of near ties met in compensator
+ * choices.
  * ---------------------------------------------------------------------------------------- */
 typedef struct {
     int D, W, r, fmt, Dg, round_storage, buf_round;
@@ -468,7 +472,7 @@ int orc_o2_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int round_st
                int buf_round, const double* S0, const double* q, const double* k, const double* v,
                const double* g, const double* beta, const uint8_t* flush_mask, double* o,
                int8_t* codes_out, double* scales_out, int* cidx_out, double* cu_out, int* pos_out,
-               double* bk_out, double* bu_out, double* bL_out, double* S_out) {
+               double* bk_out, double* bu_out, double* bL_out, double* S_out, int* ties_out) {
     o2_cfg c = {D, W, r, fmt, Dg, round_storage, buf_round};
     int ng = orc_num_groups(fmt == ORC_FMT_NONE ? ORC_FMT_INT8 : fmt, D);
     int ties = 0;
@@ -490,14 +494,16 @@ int orc_o2_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int round_st
 
         if (S0) memcpy(Sx, S0 + (size_t)h * DD, sizeof(double) * DD);
         else memset(Sx, 0, sizeof(double) * DD);
-        ties += o2_set_frozen(&c, &s, Sx);
+        int hties = o2_set_frozen(&c, &s, Sx);
         for (int t = 0; t < T; ++t) {
             size_t th = (size_t)t * nh + h;
             o2_step(&c, &s, q + th * D, k + th * D, v + th * D, g + th * Dg, beta[th],
                     o ? o + th * D : NULL, Lt, x, y, w, rr);
             int forced = flush_mask && flush_mask[th];
-            if (s.P == W || forced) ties += o2_flush(&c, &s, Sx, Lt);
+            if (s.P == W || forced) hties += o2_flush(&c, &s, Sx, Lt);
         }
+        ties += hties;
+        if (ties_out) ties_out[h] = hties;
         if (codes_out) memcpy(codes_out + h * DD, s.codes, DD);
         if (scales_out) memcpy(scales_out + (size_t)h * D * ng, s.scales, sizeof(double) * (size_t)D * ng);
         if (cidx_out && r > 0) memcpy(cidx_out + (size_t)h * r, s.cidx, sizeof(int) * (size_t)r);

@@ -1,0 +1,206 @@
+"""Test harness: runs a workload through the CUDA library and through the CPU oracle on the
+same seeded inputs, and compares the two.
+
+GPU side: the initial state is the fp32 recurrence over the workload's warm-up tokens, run by the
+library's fp32-state baseline kernel; then initial quantization and T windowed decode steps.
+Oracle side: the same warm-up tokens through the oracle's plain recurrence (fp32 state storage),
+then the buffered-window form with GPU storage roundings (fp32 state / gates / scales, write
+vectors in the buffer dtype, single-precision quantizer decisions). Both sides make their own
+initial state; nothing the GPU computed is handed to the oracle.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+import bit_recurrent_state_gdn_b200 as gdn
+import oracle
+from workloads import Workload, decode_inputs, outlier_scales, step_inputs, torch_dtype
+
+
+def cfg_of(wl: Workload):
+    return gdn.make_config(wl.B, wl.H, wl.D, wl.W, wl.r, wl.gate, wl.fmt, wl.act, wl.buf)
+
+
+def gpu_warmup(wl: Workload, device="cuda") -> torch.Tensor:
+    """fp32 [B][H][D][D] initial states from the library's fp32-state baseline kernel."""
+    S = torch.zeros((wl.B, wl.H, wl.D, wl.D), dtype=torch.float32, device=device)
+    if wl.warmup == 0:
+        return S
+    cfg = gdn.make_config(wl.B, wl.H, wl.D, gate=wl.gate, fmt="fp32", act=wl.act)
+    scales = outlier_scales(wl, device)
+    o = torch.empty((wl.B, wl.H, wl.D), dtype=torch_dtype(wl.act), device=device)
+    for t in range(wl.warmup):
+        s = step_inputs(wl, "warmup", t, device, scales)
+        gdn.gdn_baseline_step(cfg, S, s.q, s.k, s.v, s.g, s.beta, o)
+    return S
+
+
+def _heads_np(x: torch.Tensor, heads: np.ndarray) -> np.ndarray:
+    """[T][B][H](...) device tensor -> [T][n](...) float64 numpy for the flat head indices."""
+    T = x.shape[0]
+    flat = x.reshape(T, -1, *x.shape[3:]) if x.dim() > 3 else x.reshape(T, -1)
+    idx = torch.as_tensor(heads, device=x.device, dtype=torch.long)
+    return flat.index_select(1, idx).double().cpu().numpy()
+
+
+def warmup_inputs_np(wl: Workload, heads: np.ndarray, device="cuda") -> dict:
+    scales = outlier_scales(wl, device)
+    idx = torch.as_tensor(heads, device=device, dtype=torch.long)
+    acc = {n: [] for n in ("q", "k", "v", "g", "beta")}
+    for t in range(wl.warmup):
+        s = step_inputs(wl, "warmup", t, device, scales)
+        for n in acc:
+            x = getattr(s, n)
+            flat = x.reshape(-1, *x.shape[2:]) if x.dim() > 2 else x.reshape(-1)
+            acc[n].append(flat.index_select(0, idx).double().cpu().numpy())
+    return {n: np.stack(v) if v else np.zeros((0,)) for n, v in acc.items()}
+
+
+def oracle_initial_state(wl: Workload, heads: np.ndarray, device="cuda") -> np.ndarray:
+    n = len(heads)
+    if wl.warmup == 0:
+        return np.zeros((n, wl.D, wl.D))
+    w = warmup_inputs_np(wl, heads, device)
+    _, S = oracle.plain_run(w["q"], w["k"], w["v"], w["g"], w["beta"], state_round="f32",
+                            want_o=False)
+    return S
+
+
+@dataclass
+class GpuRun:
+    o: torch.Tensor            # [T][B][H][D] act dtype
+    state: gdn.GdnState
+    S0: torch.Tensor           # fp32 initial states
+    inputs: dict
+
+
+def gpu_run(wl: Workload, device="cuda", T: int | None = None, inputs=None, S0=None) -> GpuRun:
+    cfg = cfg_of(wl)
+    T = wl.T if T is None else T
+    if inputs is None:
+        inputs = decode_inputs(wl, device, T)
+    if S0 is None:
+        S0 = gpu_warmup(wl, device)
+    state = gdn.GdnState.allocate(cfg, device)
+    gdn.gdn_state_quantize(cfg, S0, state)
+    o = torch.empty_like(inputs["q"])
+    if T > 0:
+        gdn.gdn_decode_window_steps(cfg, state, inputs["q"], inputs["k"], inputs["v"],
+                                    inputs["g"], inputs["beta"], o)
+    torch.cuda.synchronize()
+    return GpuRun(o, state, S0, inputs)
+
+
+def oracle_run(wl: Workload, heads: np.ndarray, inputs: dict, S0: np.ndarray, flush_mask=None):
+    q, k, v, g, beta = (_heads_np(inputs[n], heads) for n in ("q", "k", "v", "g", "beta"))
+    return oracle.o2_run(q, k, v, g, beta, W=wl.W, r=wl.r, fmt=wl.fmt, S0=S0,
+                         round_storage=True, buf_round=wl.buf, flush_mask=flush_mask)
+
+
+# ---------------------------------------------------------------------------------------------
+# Reading the GPU state back per head
+# ---------------------------------------------------------------------------------------------
+def gpu_codes(wl: Workload, st: gdn.GdnState, heads: np.ndarray) -> np.ndarray:
+    """Unpacked int8 codes [n][D][D] of the chosen heads."""
+    D = wl.D
+    if wl.fmt == "int4_g32":
+        packed = st.codes.view(-1, D, D // 2)[torch.as_tensor(heads, device=st.codes.device)]
+        return np.stack([oracle.unpack_int4(p) for p in packed.cpu().numpy()])
+    return st.codes.view(torch.int8).view(-1, D, D)[
+        torch.as_tensor(heads, device=st.codes.device)].cpu().numpy()
+
+
+def gpu_scales(wl: Workload, st: gdn.GdnState, heads: np.ndarray) -> np.ndarray:
+    ng = wl.D // 32 if wl.fmt == "int4_g32" else 1
+    return st.scales.view(-1, wl.D, ng)[torch.as_tensor(heads, device=st.scales.device)] \
+        .double().cpu().numpy()
+
+
+def gpu_comps(wl: Workload, st: gdn.GdnState, heads: np.ndarray):
+    rp = (wl.r + 3) // 4 * 4
+    h = torch.as_tensor(heads, device=st.pos.device)
+    cidx = st.comp_idx.view(-1, rp)[h][:, : wl.r].cpu().numpy()
+    cu = st.comp_u.view(-1, wl.r, wl.D)[h].double().cpu().numpy()
+    return cidx, cu
+
+
+def round_act(x: np.ndarray, act: str) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch_dtype(act)).double().numpy()
+
+
+def rel_l2(a, b) -> float:
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+# ---------------------------------------------------------------------------------------------
+# Acceptance bars (output rel-L2 2e-3; codes equal but for 1-LSB flips on <= 0.1% of entries;
+# scales and compensators to fp32 rounding; near-tie compensator heads reported apart)
+# ---------------------------------------------------------------------------------------------
+O_TOL = 2e-3
+FLIP_FRAC = 1e-3
+SCALE_TOL = 1e-4
+COMP_TOL = 1e-4
+
+
+@dataclass
+class Parity:
+    o_rel: float
+    o_rel_unrounded: float
+    flip_frac: float
+    max_code_diff: int
+    scale_rel: float
+    comp_rel: float
+    tie_heads: int
+    n_heads: int
+    pos_equal: bool
+
+    def check(self):
+        assert self.o_rel <= O_TOL, self
+        assert self.max_code_diff <= 1, self
+        assert self.flip_frac <= FLIP_FRAC, self
+        assert self.scale_rel <= SCALE_TOL, self
+        assert self.comp_rel <= COMP_TOL, self
+        assert self.tie_heads <= max(1, int(FLIP_FRAC * self.n_heads)), self
+        assert self.pos_equal, self
+
+
+def compare(wl: Workload, run: GpuRun, heads: np.ndarray, res) -> Parity:
+    T = run.o.shape[0]
+    o_gpu = _heads_np(run.o, heads) if T else np.zeros((0, len(heads), wl.D))
+    o_ref = round_act(res.o, wl.act)
+    ok = res.ties == 0
+    codes = gpu_codes(wl, run.state, heads)
+    diff = np.abs(codes[ok].astype(int) - res.codes[ok].astype(int))
+    sc = gpu_scales(wl, run.state, heads)
+    srel = np.abs(sc[ok] - res.scales[ok]) / np.maximum(np.abs(res.scales[ok]), 1e-30)
+    crel = 0.0
+    if wl.r > 0:
+        cidx, cu = gpu_comps(wl, run.state, heads)
+        assert np.array_equal(cidx[ok], res.cidx[ok]), "compensator columns differ"
+        crel = rel_l2(cu[ok], res.cu[ok]) if ok.any() else 0.0
+    pos = run.state.pos[torch.as_tensor(heads, device=run.state.pos.device)].cpu().numpy()
+    # a flipped code changes that row's scale only when the flip is the absmax entry; scales are
+    # compared where every code of the row agrees
+    rows_same = (diff.reshape(diff.shape[0], wl.D, -1).max(axis=-1) == 0) if diff.size else diff
+    srel_cmp = srel.reshape(srel.shape[0], wl.D, -1)
+    return Parity(
+        o_rel=rel_l2(o_gpu, o_ref), o_rel_unrounded=rel_l2(o_gpu, res.o),
+        flip_frac=float((diff > 0).mean()) if diff.size else 0.0,
+        max_code_diff=int(diff.max()) if diff.size else 0,
+        scale_rel=float(srel_cmp[rows_same].max()) if np.any(rows_same) else 0.0,
+        comp_rel=crel, tie_heads=int((~ok).sum()), n_heads=len(heads),
+        pos_equal=bool(np.array_equal(pos, res.pos)))
+
+
+def sample_heads(wl: Workload, n: int, seed: int = 0) -> np.ndarray:
+    """Every head of the first and the last sequence, plus random others (sorted, unique)."""
+    H, Bh = wl.H, wl.heads
+    first = np.arange(min(H, Bh))
+    last = np.arange(max(Bh - H, 0), Bh)
+    rng = np.random.default_rng(seed)
+    extra = rng.choice(Bh, size=min(max(n - len(first) - len(last), 0), Bh), replace=False)
+    return np.unique(np.concatenate([first, last, extra])).astype(np.int64)

@@ -1,0 +1,192 @@
+"""The C ABI on the host: the library loads, exports every symbol include/gdnq.h declares, sizes
+its buffers, and rejects bad arguments before touching a device. Every call here fails argument
+checks (or is an empty batch), so no kernel is launched and no pointer is dereferenced."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bit_recurrent_state_gdn_b200 as gdn
+from bit_recurrent_state_gdn_b200 import _abi, build
+from workloads import WORKLOADS
+
+HEADER = os.path.join(os.path.dirname(build.PKG), "include", "gdnq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _abi.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported_and_bound(lib):
+    names = declared_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), f"{n} not exported"
+        assert n in _abi.SIGNATURES, f"{n} not bound in the Python layer"
+    assert set(_abi.SIGNATURES) == set(names)
+
+
+def test_status_strings(lib):
+    assert lib.gdn_status_string(0) == b"GDN_OK"
+    assert lib.gdn_status_string(1) == b"GDN_ERR_INVALID_ARG"
+    assert lib.gdn_status_string(2) == b"GDN_ERR_UNSUPPORTED"
+    assert lib.gdn_status_string(3) == b"GDN_ERR_CUDA"
+    assert lib.gdn_status_string(4) == b"GDN_ERR_TIMEOUT"
+    assert lib.gdn_status_string(99) == b"GDN_UNKNOWN_STATUS"
+
+
+def _cfg(**kw):
+    base = dict(B=2, H=3, D=128, W=64, r=0, gate="scalar", fmt="int8", act="bf16", buf="bf16")
+    base.update(kw)
+    return gdn.make_config(**base)
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_state_sizes_of_the_workloads(name, lib):
+    wl = WORKLOADS[name]
+    cfg = gdn.make_config(wl.B, wl.H, wl.D, wl.W, wl.r, wl.gate, wl.fmt, wl.act, wl.buf)
+    s = gdn.gdn_state_sizes(cfg)
+    n, D, W = wl.heads, wl.D, wl.W
+    act = 4 if wl.act == "f32" else 2
+    buf = 4 if wl.buf == "f32" else 2
+    if wl.fmt == "int8":
+        assert s.codes == n * D * D and s.scales == n * D * 4
+    else:
+        assert s.codes == n * D * D // 2 and s.scales == n * D * (D // 32) * 4
+    assert s.buf_k == n * W * D * act and s.buf_u == n * W * D * buf
+    assert s.buf_L == n * 4 * (W * D if wl.gate == "diag" else (W + 3) // 4 * 4)
+    assert s.comp_idx == (n * 4 * ((wl.r + 3) // 4 * 4) if wl.r else 0)
+    assert s.comp_u == n * wl.r * D * 4
+    assert s.pos == n * 4
+    assert 0 < s.smem_step <= 227 * 1024
+
+
+BAD_CONFIGS = [
+    ("W=0", dict(W=0), _abi.GDN_ERR_INVALID_ARG),
+    ("r<0", dict(r=-1), _abi.GDN_ERR_INVALID_ARG),
+    ("r>d", dict(D=16, r=17), _abi.GDN_ERR_INVALID_ARG),
+    ("r>max", dict(r=17), _abi.GDN_ERR_UNSUPPORTED),
+    ("D=64", dict(D=64), _abi.GDN_ERR_UNSUPPORTED),
+    ("int4 D=16", dict(D=16, fmt="int4_g32"), _abi.GDN_ERR_UNSUPPORTED),
+    ("baseline fmt", dict(fmt="bf16"), _abi.GDN_ERR_INVALID_ARG),
+    ("window too big", dict(W=5000), _abi.GDN_ERR_UNSUPPORTED),
+    ("B<0", dict(B=-1), _abi.GDN_ERR_INVALID_ARG),
+]
+
+
+@pytest.mark.parametrize("name,kw,want", BAD_CONFIGS, ids=[c[0] for c in BAD_CONFIGS])
+def test_bad_config_rejected(name, kw, want, lib):
+    cfg = _cfg(**kw)
+    out = _abi.gdn_sizes()
+    assert lib.gdn_state_sizes(ctypes.byref(cfg), ctypes.byref(out)) == want
+    assert lib.gdn_last_error() != b""
+    st = _abi.gdn_state()
+    assert lib.gdn_decode_window_step(ctypes.byref(cfg), ctypes.byref(st), *[None] * 7) == want
+
+
+def test_raw_field_errors(lib):
+    out = _abi.gdn_sizes()
+    assert lib.gdn_state_sizes(None, ctypes.byref(out)) == _abi.GDN_ERR_INVALID_ARG
+    cfg = _cfg()
+    assert lib.gdn_state_sizes(ctypes.byref(cfg), None) == _abi.GDN_ERR_INVALID_ARG
+    for field, val in (("gate", 7), ("fmt", 9), ("act_dtype", 3), ("buf_dtype", -1)):
+        c = _cfg()
+        setattr(c, field, val)
+        assert lib.gdn_state_sizes(ctypes.byref(c), ctypes.byref(out)) == _abi.GDN_ERR_INVALID_ARG
+    c = _cfg()
+    c.d_v = 64
+    assert lib.gdn_state_sizes(ctypes.byref(c), ctypes.byref(out)) == _abi.GDN_ERR_UNSUPPORTED
+
+
+def _fake_state(misalign=None, null=None):
+    vals = {n: 0x10000 * (i + 1) for i, n in enumerate(_abi.STATE_FIELDS)}
+    vals["status"] = 0
+    if misalign:
+        vals[misalign] += 8
+    if null:
+        vals[null] = 0
+    return _abi.gdn_state(**vals)
+
+
+@pytest.mark.parametrize("field", ["codes", "scales", "buf_k", "buf_u", "buf_L", "pos"])
+def test_state_pointer_checks(field, lib):
+    cfg = _cfg()
+    q = ctypes.c_void_p(0x900000)
+    for st in (_fake_state(null=field), _fake_state(misalign=field)):
+        rc = lib.gdn_decode_window_step(ctypes.byref(cfg), ctypes.byref(st), q, q, q, q, q, q, None)
+        assert rc == _abi.GDN_ERR_INVALID_ARG
+        assert field.encode() in lib.gdn_last_error()
+
+
+def test_compensator_pointers_needed_only_with_r(lib):
+    st = _fake_state(null="comp_u")
+    cfg = _cfg(r=4)
+    rc = lib.gdn_window_flush(ctypes.byref(cfg), ctypes.byref(st), None, None)
+    assert rc == _abi.GDN_ERR_INVALID_ARG and b"comp_u" in lib.gdn_last_error()
+
+
+def test_input_pointer_checks(lib):
+    cfg = _cfg()
+    st = _fake_state()
+    good = ctypes.c_void_p(0x900000)
+    odd = ctypes.c_void_p(0x900001)       # not 2-byte aligned for bf16
+    args = [good] * 6
+    for i in range(6):
+        a = list(args)
+        a[i] = None
+        assert lib.gdn_decode_window_step(ctypes.byref(cfg), ctypes.byref(st), *a, None) \
+            == _abi.GDN_ERR_INVALID_ARG
+    a = list(args)
+    a[0] = odd
+    assert lib.gdn_decode_window_step(ctypes.byref(cfg), ctypes.byref(st), *a, None) \
+        == _abi.GDN_ERR_INVALID_ARG
+    assert lib.gdn_decode_window_steps(ctypes.byref(cfg), ctypes.byref(st), -1, *args, None) \
+        == _abi.GDN_ERR_INVALID_ARG
+
+
+def test_host_pipeline_checks(lib):
+    cfg = _cfg()
+    st = _fake_state()
+    need = lib.gdn_host_staging_bytes(ctypes.byref(cfg))
+    assert need > 0
+    h = ctypes.c_void_p(0x900000)
+    rc = lib.gdn_decode_window_steps_host(ctypes.byref(cfg), ctypes.byref(st), 3, h, h, h, h, h, h,
+                                          ctypes.c_void_p(0x800000), need - 1, None)
+    assert rc == _abi.GDN_ERR_INVALID_ARG and b"staging" in lib.gdn_last_error()
+    bad = _cfg(W=0)
+    assert lib.gdn_host_staging_bytes(ctypes.byref(bad)) == 0
+
+
+def test_empty_batch_needs_no_buffers(lib):
+    cfg = _cfg(B=0)
+    st = _abi.gdn_state()
+    assert lib.gdn_decode_window_step(ctypes.byref(cfg), ctypes.byref(st), *[None] * 7) == 0
+    assert lib.gdn_state_quantize(ctypes.byref(cfg), None, ctypes.byref(st), None) == 0
+    assert lib.gdn_window_flush(ctypes.byref(cfg), ctypes.byref(st), None, None) == 0
+    assert lib.gdn_state_materialize(ctypes.byref(cfg), ctypes.byref(st), None, None) == 0
+    base = _cfg(B=0, fmt="fp32")
+    assert lib.gdn_baseline_step(ctypes.byref(base), *[None] * 8) == 0
+
+
+def test_baseline_format_checks(lib):
+    cfg = _cfg(fmt="int8")
+    assert lib.gdn_baseline_step(ctypes.byref(cfg), *[None] * 8) == _abi.GDN_ERR_INVALID_ARG
+    cfg = _cfg(fmt="fp32")
+    s = ctypes.c_void_p(0x900008)         # state array must be 16-byte aligned
+    g = ctypes.c_void_p(0x900000)
+    assert lib.gdn_baseline_step(ctypes.byref(cfg), s, g, g, g, g, g, g, None) \
+        == _abi.GDN_ERR_INVALID_ARG
+
+
+def test_python_layer_raises_with_detail(lib):
+    with pytest.raises(gdn.GdnError, match="GDN_ERR_UNSUPPORTED.*head size"):
+        gdn.gdn_state_sizes(_cfg(D=64))

@@ -17,8 +17,8 @@ MUTANTS = [
      "S[(size_t)i * D + j] += -bt * w[i] * kt[j] + bt * vt[i] * kt[j];",
      "S[(size_t)i * D + j] += -bt * w[i] * kt[j] + bt * vt[j] * kt[i];"),
     ("plain: gate applied to value rows",
-     "for (int j = 0; j < D; ++j) S[(size_t)i * D + j] *= exp(gate_log(gt, Dg, j));",
-     "for (int j = 0; j < D; ++j) S[(size_t)i * D + j] *= exp(gate_log(gt, Dg, i));"),
+     "for (int j = 0; j < D; ++j) S[(size_t)i * D + j] *= a[j];",
+     "for (int j = 0; j < D; ++j) S[(size_t)i * D + j] *= a[i];"),
     ("plain: output from the key instead of the query",
      "for (int j = 0; j < D; ++j) acc += S[(size_t)i * D + j] * qt[j];\n                    ot[i] = acc;\n                }\n            }\n            if (state_round",
      "for (int j = 0; j < D; ++j) acc += S[(size_t)i * D + j] * kt[j];\n                    ot[i] = acc;\n                }\n            }\n            if (state_round"),

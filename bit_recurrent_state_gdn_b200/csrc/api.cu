@@ -118,15 +118,19 @@ gdn_status check_state(const gdn_config* c, const gdn_state* s) {
   return GDN_OK;
 }
 
-// Per-step inputs are read element by element: element alignment is enough.
+// Per-step inputs. The baseline step reads them element by element (element alignment is
+// enough); the window step copies q, k, v and a per-channel g with bulk async copies, which
+// need 16-byte aligned sources.
 gdn_status check_inputs(const gdn_config* c, const void* q, const void* k, const void* v,
-                        const float* g, const float* beta, const void* o) {
+                        const float* g, const float* beta, const void* o, bool bulk) {
   const unsigned ea = (unsigned)act_size(c);
+  const unsigned qa = bulk ? 16u : ea;
+  const unsigned ga = bulk && c->gate == GDN_GATE_DIAG ? 16u : 4u;
   gdn_status st;
-  if ((st = need_ptr(q, "q", ea)) != GDN_OK) return st;
-  if ((st = need_ptr(k, "k", ea)) != GDN_OK) return st;
-  if ((st = need_ptr(v, "v", ea)) != GDN_OK) return st;
-  if ((st = need_ptr(g, "g", 4)) != GDN_OK) return st;
+  if ((st = need_ptr(q, "q", qa)) != GDN_OK) return st;
+  if ((st = need_ptr(k, "k", qa)) != GDN_OK) return st;
+  if ((st = need_ptr(v, "v", qa)) != GDN_OK) return st;
+  if ((st = need_ptr(g, "g", ga)) != GDN_OK) return st;
   if ((st = need_ptr(beta, "beta", 4)) != GDN_OK) return st;
   if ((st = need_ptr(o, "o", ea)) != GDN_OK) return st;
   return GDN_OK;
@@ -191,8 +195,8 @@ size_t window_smem_bytes(const gdn_config& c) {
   const bool int4 = c.fmt == GDN_FMT_INT4_G32;
   const int code_bytes = int4 ? D * D / 2 : D * D;
   const int nscales = int4 ? D * (D / 32) : D;
-  return window_smem_layout(D, code_bytes, nscales, (int)act_size(&c), (int)buf_size(&c),
-                            c.gate == GDN_GATE_DIAG, c.W, c.r)
+  return win_layout(D, code_bytes, nscales, (int)act_size(&c), (int)buf_size(&c),
+                    c.gate == GDN_GATE_DIAG, c.W, c.r, 1, kMaxHeadsPerCta)
       .total;
 }
 
@@ -260,7 +264,7 @@ gdn_status gdn_decode_window_steps(const gdn_config* cfg, const gdn_state* state
   if (T < 0) return fail(GDN_ERR_INVALID_ARG, "T=%d must be >= 0", T);
   if (heads_of(cfg) == 0 || T == 0) return GDN_OK;
   if ((st = check_state(cfg, state)) != GDN_OK) return st;
-  if ((st = check_inputs(cfg, q, k, v, g, beta, o)) != GDN_OK) return st;
+  if ((st = check_inputs(cfg, q, k, v, g, beta, o, true)) != GDN_OK) return st;
   const size_t H = (size_t)heads_of(cfg), D = (size_t)cfg->d_k;
   const size_t act_step = H * D * act_size(cfg);
   const size_t g_step = H * (cfg->gate == GDN_GATE_DIAG ? D : 1);
@@ -396,7 +400,7 @@ gdn_status gdn_baseline_step(const gdn_config* cfg, void* S, const void* q, cons
   if (st != GDN_OK) return st;
   if (heads_of(cfg) == 0) return GDN_OK;
   if ((st = need_ptr(S, "S")) != GDN_OK) return st;
-  if ((st = check_inputs(cfg, q, k, v, g, beta, o)) != GDN_OK) return st;
+  if ((st = check_inputs(cfg, q, k, v, g, beta, o, false)) != GDN_OK) return st;
   gdnq::BaseArgs a{S, q, k, v, g, beta, o};
   cudaError_t e = gdnq::launch_baseline(*cfg, a, (int)heads_of(cfg), (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "gdn_baseline_step");

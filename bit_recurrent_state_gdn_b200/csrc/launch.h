@@ -15,7 +15,11 @@ enum class WinOp { Step, Flush, Materialize, Quantize };
 // Largest dynamic shared memory per CTA on sm_100 (bytes).
 constexpr int kMaxSmemPerCta = 227 * 1024;
 
-// Dynamic shared memory a window kernel needs for this configuration.
+// Most heads one persistent step CTA walks (its per-head pos / gate / beta live in shared memory).
+constexpr int kMaxHeadsPerCta = 1024;
+
+// Dynamic shared memory a window kernel needs for this configuration at the least (one stage,
+// the largest per-CTA head range).
 size_t window_smem_bytes(const gdn_config& cfg);
 
 // Launch one window kernel over `heads` CTAs. Returns cudaErrorNotSupported for a configuration

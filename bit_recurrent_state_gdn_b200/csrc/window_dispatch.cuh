@@ -1,6 +1,7 @@
 // Template dispatch from a runtime gdn_config to an instantiated window kernel configuration.
 #pragma once
 
+#include <algorithm>
 #include <atomic>
 
 #include "launch.h"
@@ -8,9 +9,10 @@
 
 namespace gdnq {
 
-// Raises a kernel's dynamic shared-memory limit once per device as needed.
-template <class Kernel>
-cudaError_t ensure_smem(Kernel k, size_t bytes) {
+// Raises a kernel's dynamic shared-memory limit as needed, once per (kernel, device): the cache
+// is a static of this instantiation, so every kernel has its own.
+template <auto Kernel>
+cudaError_t ensure_smem(size_t bytes) {
   static std::atomic<size_t> granted[64];
   if (bytes <= 48 * 1024) return cudaSuccess;
   int dev = 0;
@@ -18,27 +20,72 @@ cudaError_t ensure_smem(Kernel k, size_t bytes) {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) dev = 63;
   if (granted[dev].load() >= bytes) return cudaSuccess;
-  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e == cudaSuccess) granted[dev].store(bytes);
   return e;
 }
 
+// Streaming multiprocessors of the current device (cached per device).
+inline int num_sms() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  int n = cached[dev].load();
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev].store(n);
+  }
+  return n;
+}
+
+// Shape of a persistent step launch: two CTAs per SM with two stages each when they fit in
+// shared memory, else one CTA per SM with as many stages (up to 4) as fit.
+struct StepPlan {
+  int grid, per_cta, nstages;
+  size_t smem;
+};
+
+template <class C>
+StepPlan plan_step(int W, int r, int heads) {
+  constexpr int kSmemPerSm = 228 * 1024, kSmemPerCta = kMaxSmemPerCta, kReserved = 1024;
+  const int sms = num_sms();
+  auto smem_of = [&](int ns, int pc) { return (size_t)win_layout<C>(W, r, ns, pc).total; };
+  auto per = [&](int ctas) { return std::min(kMaxHeadsPerCta, std::max(1, (heads + ctas - 1) / ctas)); };
+  StepPlan p;
+  int bps = 2, ns = 2;
+  if (2 * (smem_of(2, per(2 * sms)) + kReserved) > (size_t)kSmemPerSm) {
+    bps = 1;
+    ns = 1;
+    for (int k = 4; k >= 2; --k)
+      if (smem_of(k, per(sms)) <= (size_t)kSmemPerCta) { ns = k; break; }
+  }
+  p.per_cta = per(bps * sms);
+  p.grid = (heads + p.per_cta - 1) / p.per_cta;
+  p.nstages = ns;
+  p.smem = smem_of(ns, p.per_cta);
+  return p;
+}
+
 template <class C>
 cudaError_t launch_window_cfg(WinOp op, const WinArgs& a, int heads, cudaStream_t st) {
-  const size_t smem = window_smem_layout<C>(a.W, a.r).total;
+  const size_t smem1 = win_layout<C>(a.W, a.r, 1, 0).total;
   cudaError_t e = cudaSuccess;
   switch (op) {
-    case WinOp::Step:
-      e = ensure_smem(window_step_kernel<C>, smem);
-      if (e == cudaSuccess) window_step_kernel<C><<<heads, kThreads, smem, st>>>(a);
+    case WinOp::Step: {
+      const StepPlan p = plan_step<C>(a.W, a.r, heads);
+      e = ensure_smem<window_step_kernel<C>>(p.smem);
+      if (e == cudaSuccess)
+        window_step_kernel<C><<<p.grid, kThreads, p.smem, st>>>(a, heads, p.per_cta, p.nstages);
       break;
+    }
     case WinOp::Flush:
-      e = ensure_smem(window_state_kernel<C, 0>, smem);
-      if (e == cudaSuccess) window_state_kernel<C, 0><<<heads, kThreads, smem, st>>>(a);
+      e = ensure_smem<window_state_kernel<C, 0>>(smem1);
+      if (e == cudaSuccess) window_state_kernel<C, 0><<<heads, kThreads, smem1, st>>>(a);
       break;
     case WinOp::Materialize:
-      e = ensure_smem(window_state_kernel<C, 1>, smem);
-      if (e == cudaSuccess) window_state_kernel<C, 1><<<heads, kThreads, smem, st>>>(a);
+      e = ensure_smem<window_state_kernel<C, 1>>(smem1);
+      if (e == cudaSuccess) window_state_kernel<C, 1><<<heads, kThreads, smem1, st>>>(a);
       break;
     case WinOp::Quantize:
       quantize_kernel<C><<<heads, kThreads, 0, st>>>(a);

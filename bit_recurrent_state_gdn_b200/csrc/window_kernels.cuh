@@ -69,35 +69,47 @@ struct WinCfg {
 
 __host__ __device__ constexpr uint32_t align128(uint32_t x) { return (x + 127u) & ~127u; }
 
-// Shared-memory layout of a window kernel (byte offsets).
-struct SmemLayout {
-  uint32_t bar, codes, scales, bk, bu, bL, cidx, cu, vec, coef, red, total;
+// Shared-memory layout of a window kernel (byte offsets). A stage holds one head's staged data
+// (frozen codes and scales, buffered pairs, compensators, and the step's q, k, v and, for the
+// diagonal gate, g); the CTA keeps `nstages` stages plus per-head scratch (vectors,
+// coefficients, reduction space) and, for the persistent step kernel, the pos / gate / beta of
+// its whole head range.
+struct WinLayout {
+  uint32_t codes, scales, bk, bu, bL, cidx, cu, q, k, v, g, stage_bytes;  // within a stage
+  uint32_t bars, stage0, vec, coef, red, harr, total;                     // within the CTA
 };
 
-__host__ __device__ inline SmemLayout window_smem_layout(int D, int code_bytes, int nscales,
-                                                         int act_size, int buf_size, bool diag,
-                                                         int W, int r) {
+__host__ __device__ inline WinLayout win_layout(int D, int code_bytes, int nscales, int act_size,
+                                                int buf_size, bool diag, int W, int r,
+                                                int nstages, int per_cta) {
   const int Wp = (W + 3) & ~3, rp = (r + 3) & ~3;
-  SmemLayout L;
-  L.bar = 0;
-  L.codes = 128;
+  WinLayout L;
+  L.codes = 0;
   L.scales = align128(L.codes + code_bytes);
   L.bk = align128(L.scales + 4u * nscales);
   L.bu = align128(L.bk + (uint32_t)W * D * act_size);
   L.bL = align128(L.bu + (uint32_t)W * D * buf_size);
   L.cidx = align128(L.bL + 4u * (diag ? (uint32_t)W * D : (uint32_t)Wp));
   L.cu = align128(L.cidx + 4u * rp);
-  L.vec = align128(L.cu + 4u * r * D);
+  L.q = align128(L.cu + 4u * r * D);
+  L.k = align128(L.q + (uint32_t)D * act_size);
+  L.v = align128(L.k + (uint32_t)D * act_size);
+  L.g = align128(L.v + (uint32_t)D * act_size);
+  L.stage_bytes = align128(L.g + (diag ? 4u * D : 0u));
+  L.bars = 0;
+  L.stage0 = 128;
+  L.vec = L.stage0 + (uint32_t)nstages * L.stage_bytes;
   L.coef = align128(L.vec + 4u * (7 * D + 64));
   L.red = align128(L.coef + 4u * (3 * (W + r) + 4));
-  L.total = align128(L.red + 4u * 2 * kThreads);
+  L.harr = align128(L.red + 4u * 2 * kThreads);
+  L.total = align128(L.harr + 12u * per_cta);
   return L;
 }
 
 template <class C>
-__host__ __device__ inline SmemLayout window_smem_layout(int W, int r) {
-  return window_smem_layout(C::D, C::CODE_BYTES, C::NSCALES, (int)sizeof(typename C::Act),
-                            (int)sizeof(typename C::Buf), C::DIAG, W, r);
+__host__ __device__ inline WinLayout win_layout(int W, int r, int nstages, int per_cta) {
+  return win_layout(C::D, C::CODE_BYTES, C::NSCALES, (int)sizeof(typename C::Act),
+                    (int)sizeof(typename C::Buf), C::DIAG, W, r, nstages, per_cta);
 }
 
 // Kernel arguments: the state's device pointers and the step's inputs (unused ones null).
@@ -128,44 +140,53 @@ __device__ __forceinline__ void report(int32_t* status, int bit) {
 }
 
 // ------------------------------------------------------------------------------------------
-// Staging: the head's frozen state, its first P buffered pairs and its compensators, copied
-// into shared memory with bulk async copies on one mbarrier. Returns false (after reporting)
-// when the bounded wait runs out; the caller then returns. Called by all threads.
+// Staging: one head's frozen state, its first P buffered pairs, its compensators and (with_io)
+// the step's q, k, v (and diagonal g), copied into a stage with bulk async copies completing on
+// the stage's mbarrier. Issued by one thread. An out-of-range P arms the barrier with no copies.
 // ------------------------------------------------------------------------------------------
 template <class C>
-__device__ __forceinline__ void stage_issue(const WinArgs& a, const SmemLayout& L, uint8_t* sm,
-                                            int head, int P) {
+__device__ __forceinline__ void stage_issue(const WinArgs& a, const WinLayout& L, uint8_t* st,
+                                            uint64_t* bar, int head, int P, bool with_io) {
   using Act = typename C::Act;
   using Buf = typename C::Buf;
   constexpr int D = C::D;
   const int W = a.W, r = a.r, Wp = (W + 3) & ~3, rp = (r + 3) & ~3;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.bar);
+  if (P < 0 || P >= W) {
+    mbar_arrive_expect_tx(bar, 0);
+    return;
+  }
   const uint32_t lbytes = C::DIAG ? 4u * P * D : 4u * ((P + 3) & ~3);
   uint32_t bytes = C::CODE_BYTES + 4u * C::NSCALES;
   if (P > 0) bytes += (uint32_t)P * D * (sizeof(Act) + sizeof(Buf)) + lbytes;
   if (r > 0) bytes += 4u * rp + 4u * r * D;
-  mbar_init(bar, 1);
-  fence_barrier_init();
+  if (with_io) bytes += 3u * D * sizeof(Act) + (C::DIAG ? 4u * D : 0u);
   mbar_arrive_expect_tx(bar, bytes);
-  bulk_g2s(sm + L.codes, a.codes + (size_t)head * C::CODE_BYTES, C::CODE_BYTES, bar);
-  bulk_g2s(sm + L.scales, a.scales + (size_t)head * C::NSCALES, 4u * C::NSCALES, bar);
+  bulk_g2s(st + L.codes, a.codes + (size_t)head * C::CODE_BYTES, C::CODE_BYTES, bar);
+  bulk_g2s(st + L.scales, a.scales + (size_t)head * C::NSCALES, 4u * C::NSCALES, bar);
   if (P > 0) {
-    bulk_g2s(sm + L.bk, static_cast<const Act*>(a.buf_k) + (size_t)head * W * D,
+    bulk_g2s(st + L.bk, static_cast<const Act*>(a.buf_k) + (size_t)head * W * D,
              (uint32_t)P * D * sizeof(Act), bar);
-    bulk_g2s(sm + L.bu, static_cast<const Buf*>(a.buf_u) + (size_t)head * W * D,
+    bulk_g2s(st + L.bu, static_cast<const Buf*>(a.buf_u) + (size_t)head * W * D,
              (uint32_t)P * D * sizeof(Buf), bar);
-    bulk_g2s(sm + L.bL, a.buf_L + (size_t)head * (C::DIAG ? (size_t)W * D : (size_t)Wp), lbytes,
+    bulk_g2s(st + L.bL, a.buf_L + (size_t)head * (C::DIAG ? (size_t)W * D : (size_t)Wp), lbytes,
              bar);
   }
   if (r > 0) {
-    bulk_g2s(sm + L.cidx, a.comp_idx + (size_t)head * rp, 4u * rp, bar);
-    bulk_g2s(sm + L.cu, a.comp_u + (size_t)head * r * D, 4u * r * D, bar);
+    bulk_g2s(st + L.cidx, a.comp_idx + (size_t)head * rp, 4u * rp, bar);
+    bulk_g2s(st + L.cu, a.comp_u + (size_t)head * r * D, 4u * r * D, bar);
+  }
+  if (with_io) {
+    bulk_g2s(st + L.q, static_cast<const Act*>(a.q) + (size_t)head * D, D * sizeof(Act), bar);
+    bulk_g2s(st + L.k, static_cast<const Act*>(a.k) + (size_t)head * D, D * sizeof(Act), bar);
+    bulk_g2s(st + L.v, static_cast<const Act*>(a.v) + (size_t)head * D, D * sizeof(Act), bar);
+    if constexpr (C::DIAG) bulk_g2s(st + L.g, a.g + (size_t)head * D, 4u * D, bar);
   }
 }
 
-__device__ __forceinline__ bool stage_wait(const WinArgs& a, const SmemLayout& L, uint8_t* sm) {
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.bar);
-  const int timed_out = mbar_wait_bounded(bar, 0) ? 0 : 1;
+// Bounded wait on a stage barrier by all threads; false (after reporting) when it ran out, in
+// which case every thread returns.
+__device__ __forceinline__ bool stage_wait(const WinArgs& a, uint64_t* bar, uint32_t parity) {
+  const int timed_out = mbar_wait_bounded(bar, parity) ? 0 : 1;
   if (__syncthreads_or(timed_out)) {
     if (threadIdx.x == 0) report(a.status, GDN_DEVICE_WAIT_TIMEOUT);
     return false;
@@ -402,15 +423,15 @@ __device__ void requantize_store(const Maker& make, int r, uint8_t* g_codes, flo
 
 // Window-end preparation in shared memory for the logical state at cumulative gate `Lend`
 // (per column in `Lvec` for the diagonal gate, scalar `Ls` otherwise) over `npairs` staged
-// pairs: colexp[j] = e^{Lend[j]}; scalar gate: fac[i] = e^{Lend - bL_i}; diagonal gate: the bL
-// region becomes bk_i[j] e^{Lend[j] - bL_i[j]} (fp32, in place).
+// pairs of stage `st`: colexp[j] = e^{Lend[j]}; scalar gate: fac[i] = e^{Lend - bL_i}; diagonal
+// gate: the stage's bL region becomes bk_i[j] e^{Lend[j] - bL_i[j]} (fp32, in place).
 template <class C>
-__device__ __forceinline__ void prepare_window_end(uint8_t* sm, const SmemLayout& L, int npairs,
+__device__ __forceinline__ void prepare_window_end(uint8_t* st, const WinLayout& L, int npairs,
                                                    const float* Lvec, float Ls, float* colexp,
                                                    float* fac) {
   constexpr int D = C::D;
-  float* bL = reinterpret_cast<float*>(sm + L.bL);
-  const typename C::Act* bk = reinterpret_cast<const typename C::Act*>(sm + L.bk);
+  float* bL = reinterpret_cast<float*>(st + L.bL);
+  const typename C::Act* bk = reinterpret_cast<const typename C::Act*>(st + L.bk);
   for (int j = threadIdx.x; j < D; j += C::NT) colexp[j] = fast_exp(C::DIAG ? Lvec[j] : Ls);
   if constexpr (C::DIAG) {
     for (int e = threadIdx.x; e < npairs * D; e += C::NT) {
@@ -423,18 +444,18 @@ __device__ __forceinline__ void prepare_window_end(uint8_t* sm, const SmemLayout
 }
 
 template <class C>
-__device__ __forceinline__ WindowTile<C> window_tile(uint8_t* sm, const SmemLayout& L, int npairs,
-                                                     int r, const float* colexp,
+__device__ __forceinline__ WindowTile<C> window_tile(const uint8_t* st, const WinLayout& L,
+                                                     int npairs, int r, const float* colexp,
                                                      const float* fac) {
   WindowTile<C> t;
-  t.codes = sm + L.codes;
-  t.scales = reinterpret_cast<const float*>(sm + L.scales);
-  t.bk = reinterpret_cast<const typename C::Act*>(sm + L.bk);
-  t.bu = reinterpret_cast<const typename C::Buf*>(sm + L.bu);
-  t.ktil = reinterpret_cast<const float*>(sm + L.bL);
+  t.codes = st + L.codes;
+  t.scales = reinterpret_cast<const float*>(st + L.scales);
+  t.bk = reinterpret_cast<const typename C::Act*>(st + L.bk);
+  t.bu = reinterpret_cast<const typename C::Buf*>(st + L.bu);
+  t.ktil = reinterpret_cast<const float*>(st + L.bL);
   t.fac = fac;
-  t.cidx = reinterpret_cast<const int32_t*>(sm + L.cidx);
-  t.cu = reinterpret_cast<const float*>(sm + L.cu);
+  t.cidx = reinterpret_cast<const int32_t*>(st + L.cidx);
+  t.cu = reinterpret_cast<const float*>(st + L.cu);
   t.colexp = colexp;
   t.npairs = npairs;
   t.r = r;
@@ -442,25 +463,19 @@ __device__ __forceinline__ WindowTile<C> window_tile(uint8_t* sm, const SmemLayo
 }
 
 // ------------------------------------------------------------------------------------------
-// Decode step (+ fused window flush).
+// One decode step (+ fused window flush) of one head whose data sit in stage `st`.
+// Called by all threads; ends with every thread done reading the stage's inputs.
 // ------------------------------------------------------------------------------------------
 template <class C>
-__global__ void __launch_bounds__(kThreads) window_step_kernel(const WinArgs a) {
+__device__ __forceinline__ void step_head(const WinArgs& a, const WinLayout& L, uint8_t* sm,
+                                          uint8_t* st, int head, int P, float g_scalar,
+                                          float beta) {
   using Act = typename C::Act;
   using Buf = typename C::Buf;
   constexpr int D = C::D, CPR = C::CPR, RPP = C::RPP;
-  extern __shared__ __align__(128) uint8_t sm[];
-  const SmemLayout L = window_smem_layout<C>(a.W, a.r);
-  const int head = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x, lane = tid & 31;
   const int W = a.W, r = a.r, Wp = (W + 3) & ~3;
-
-  const int P = a.pos[head];
-  if (P < 0 || P >= W) {
-    if (tid == 0) report(a.status, GDN_DEVICE_BAD_POS);
-    return;
-  }
   const bool flush = (P + 1 == W);
-  if (tid == 0) stage_issue<C>(a, L, sm, head, P);
 
   float* vec = reinterpret_cast<float*>(sm + L.vec);
   float *kt = vec, *qt = vec + D, *xs = vec + 2 * D, *ys = vec + 3 * D, *Lt = vec + 4 * D;
@@ -469,17 +484,27 @@ __global__ void __launch_bounds__(kThreads) window_step_kernel(const WinArgs a) 
   float *ca = coef, *cb = coef + (W + r), *fac = coef + 2 * (W + r);
   float* red = reinterpret_cast<float*>(sm + L.red);
 
-  const Act* kin = static_cast<const Act*>(a.k) + (size_t)head * D;
-  const Act* qin = static_cast<const Act*>(a.q) + (size_t)head * D;
-  const float* gL = a.buf_L + (size_t)head * (C::DIAG ? (size_t)W * D : (size_t)Wp);
+  const uint8_t* s_codes = st + L.codes;
+  const float* s_scales = reinterpret_cast<const float*>(st + L.scales);
+  Act* s_bk = reinterpret_cast<Act*>(st + L.bk);
+  Buf* s_bu = reinterpret_cast<Buf*>(st + L.bu);
+  float* s_bL = reinterpret_cast<float*>(st + L.bL);
+  const int32_t* s_cidx = reinterpret_cast<const int32_t*>(st + L.cidx);
+  const float* s_cu = reinterpret_cast<const float*>(st + L.cu);
+  const Act* s_q = reinterpret_cast<const Act*>(st + L.q);
+  const Act* s_k = reinterpret_cast<const Act*>(st + L.k);
+  const Act* s_v = reinterpret_cast<const Act*>(st + L.v);
+  const float* s_g = reinterpret_cast<const float*>(st + L.g);
+
+  // ---- gates and the scaled key / query -------------------------------------------------
   float Ls = 0.f;  // scalar-gate L_t
-  if constexpr (!C::DIAG) Ls = (P > 0 ? gL[P - 1] : 0.f) + a.g[head];
+  if constexpr (!C::DIAG) Ls = (P > 0 ? s_bL[P - 1] : 0.f) + g_scalar;
   if (tid < D) {
-    const float kj = Num<Act>::to_f(kin[tid]), qj = Num<Act>::to_f(qin[tid]);
+    const float kj = Num<Act>::to_f(s_k[tid]), qj = Num<Act>::to_f(s_q[tid]);
     kt[tid] = kj;
     qt[tid] = qj;
     float l;
-    if constexpr (C::DIAG) l = (P > 0 ? gL[(size_t)(P - 1) * D + tid] : 0.f) + a.g[(size_t)head * D + tid];
+    if constexpr (C::DIAG) l = (P > 0 ? s_bL[(P - 1) * D + tid] : 0.f) + s_g[tid];
     else l = Ls;
     Lt[tid] = l;
     const float e = fast_exp(l);
@@ -487,15 +512,6 @@ __global__ void __launch_bounds__(kThreads) window_step_kernel(const WinArgs a) 
     ys[tid] = e * qj;
   }
   __syncthreads();
-  if (!stage_wait(a, L, sm)) return;
-
-  const uint8_t* s_codes = sm + L.codes;
-  const float* s_scales = reinterpret_cast<const float*>(sm + L.scales);
-  Act* s_bk = reinterpret_cast<Act*>(sm + L.bk);
-  Buf* s_bu = reinterpret_cast<Buf*>(sm + L.bu);
-  float* s_bL = reinterpret_cast<float*>(sm + L.bL);
-  const int32_t* s_cidx = reinterpret_cast<const int32_t*>(sm + L.cidx);
-  const float* s_cu = reinterpret_cast<const float*>(sm + L.cu);
 
   // ---- phase 1: p = F x, r = F y ---------------------------------------------------------
   {
@@ -564,8 +580,7 @@ __global__ void __launch_bounds__(kThreads) window_step_kernel(const WinArgs a) 
       float pa = 0.f, pb = 0.f;
       if (i < P) {
         float kk[16];
-        if constexpr (sizeof(Act) == 2) Num<Act>::template load<16>(s_bk + i * D + c * 16, kk);
-        else Num<Act>::template load<16>(s_bk + i * D + c * 16, kk);
+        Num<Act>::template load<16>(s_bk + i * D + c * 16, kk);
         if constexpr (C::DIAG) {
           float ll[16];
           Num<float>::load<16>(s_bL + i * D + c * 16, ll);
@@ -636,18 +651,17 @@ __global__ void __launch_bounds__(kThreads) window_step_kernel(const WinArgs a) 
       w += red[gi * 2 * D + v];
       rr += red[gi * 2 * D + D + v];
     }
-    const float vin = Num<Act>::to_f(static_cast<const Act*>(a.v)[(size_t)head * D + v]);
-    const float u = a.beta[head] * (vin - w);
+    const float u = beta * (Num<Act>::to_f(s_v[v]) - w);
     const Buf ub = Num<Buf>::from_f(u);
     const float ur = Num<Buf>::to_f(ub);
     static_cast<Act*>(a.o)[(size_t)head * D + v] = Num<Act>::from_f(rr + ur * misc[0]);
     if (!flush) {
       static_cast<Buf*>(a.buf_u)[((size_t)head * W + P) * D + v] = ub;
-      static_cast<Act*>(a.buf_k)[((size_t)head * W + P) * D + v] = kin[v];
+      static_cast<Act*>(a.buf_k)[((size_t)head * W + P) * D + v] = s_k[v];
       if constexpr (C::DIAG) a.buf_L[((size_t)head * W + P) * D + v] = Lt[v];
     } else {
       s_bu[P * D + v] = ub;
-      s_bk[P * D + v] = kin[v];
+      s_bk[P * D + v] = s_k[v];
       if constexpr (C::DIAG) s_bL[P * D + v] = Lt[v];
     }
   }
@@ -663,9 +677,9 @@ __global__ void __launch_bounds__(kThreads) window_step_kernel(const WinArgs a) 
   // ---- phase 5: window end -------------------------------------------------------------
   __syncthreads();
   float* colexp = xs;  // x, y are dead
-  prepare_window_end<C>(sm, L, P + 1, Lt, Ls, colexp, fac);
+  prepare_window_end<C>(st, L, P + 1, Lt, Ls, colexp, fac);
   __syncthreads();
-  const WindowTile<C> tile = window_tile<C>(sm, L, P + 1, r, colexp, fac);
+  const WindowTile<C> tile = window_tile<C>(st, L, P + 1, r, colexp, fac);
   requantize_store<C>(tile, r, a.codes + (size_t)head * C::CODE_BYTES,
                       a.scales + (size_t)head * C::NSCALES,
                       a.comp_idx + (size_t)head * ((r + 3) & ~3), a.comp_u + (size_t)head * r * D,
@@ -673,13 +687,62 @@ __global__ void __launch_bounds__(kThreads) window_step_kernel(const WinArgs a) 
 }
 
 // ------------------------------------------------------------------------------------------
+// Decode step, persistent: CTA b owns heads [b * per_cta, (b + 1) * per_cta) and walks them in
+// order while up to nstages - 1 later heads are already being copied into their stages.
+// ------------------------------------------------------------------------------------------
+template <class C>
+__global__ void __launch_bounds__(kThreads, 2)
+    window_step_kernel(const WinArgs a, const int heads, const int per_cta, const int nstages) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  const WinLayout L = win_layout<C>(a.W, a.r, nstages, per_cta);
+  const int tid = threadIdx.x;
+  const int h0 = blockIdx.x * per_cta;
+  const int nh = min(per_cta, heads - h0);
+  if (nh <= 0) return;
+  int32_t* hpos = reinterpret_cast<int32_t*>(sm + L.harr);
+  float* hg = reinterpret_cast<float*>(hpos + per_cta);
+  float* hb = hg + per_cta;
+  for (int i = tid; i < nh; i += C::NT) {
+    hpos[i] = a.pos[h0 + i];
+    if constexpr (!C::DIAG) hg[i] = a.g[h0 + i];
+    hb[i] = a.beta[h0 + i];
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L.bars);
+  if (tid == 0) {
+    for (int s = 0; s < nstages; ++s) mbar_init(&bars[s], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (tid == 0)
+    for (int s = 0; s < nstages && s < nh; ++s)
+      stage_issue<C>(a, L, sm + L.stage0 + s * L.stage_bytes, &bars[s], h0 + s, hpos[s], true);
+  for (int n = 0; n < nh; ++n) {
+    const int s = n % nstages;
+    uint8_t* st = sm + L.stage0 + s * L.stage_bytes;
+    if (!stage_wait(a, &bars[s], (uint32_t)(n / nstages) & 1u)) return;
+    const int P = hpos[n];
+    if (P >= 0 && P < a.W) {
+      step_head<C>(a, L, sm, st, h0 + n, P, C::DIAG ? 0.f : hg[n], hb[n]);
+    } else if (tid == 0) {
+      report(a.status, GDN_DEVICE_BAD_POS);
+    }
+    __syncthreads();  // the stage and the per-head scratch are free again
+    if (tid == 0 && n + nstages < nh) {
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      stage_issue<C>(a, L, st, &bars[s], h0 + n + nstages, hpos[n + nstages], true);
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
 // Forced flush (mode 0) and materialisation (mode 1) of the logical state at the current pos.
+// One CTA per head, one stage.
 // ------------------------------------------------------------------------------------------
 template <class C, int MODE>
 __global__ void __launch_bounds__(kThreads) window_state_kernel(const WinArgs a) {
   constexpr int D = C::D;
   extern __shared__ __align__(128) uint8_t sm[];
-  const SmemLayout L = window_smem_layout<C>(a.W, a.r);
+  const WinLayout L = win_layout<C>(a.W, a.r, 1, 0);
   const int head = blockIdx.x, tid = threadIdx.x;
   const int W = a.W, r = a.r;
   const int P = a.pos[head];
@@ -691,15 +754,21 @@ __global__ void __launch_bounds__(kThreads) window_state_kernel(const WinArgs a)
     if (P == 0) return;
     if (a.seq_mask && a.seq_mask[head / a.H] == 0) return;
   }
-  if (tid == 0) stage_issue<C>(a, L, sm, head, P);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.bars);
+  uint8_t* st = sm + L.stage0;
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+    stage_issue<C>(a, L, st, bar, head, P, false);
+  }
   __syncthreads();
-  if (!stage_wait(a, L, sm)) return;
+  if (!stage_wait(a, bar, 0)) return;
 
   float* vec = reinterpret_cast<float*>(sm + L.vec);
   float *Lend = vec, *colexp = vec + D, *colmax = vec + 2 * D;
   int32_t* sel = reinterpret_cast<int32_t*>(vec + 7 * D);
   float* fac = reinterpret_cast<float*>(sm + L.coef);
-  const float* s_bL = reinterpret_cast<const float*>(sm + L.bL);
+  const float* s_bL = reinterpret_cast<const float*>(st + L.bL);
   float Ls = 0.f;
   if constexpr (C::DIAG) {
     for (int j = tid; j < D; j += C::NT) Lend[j] = P > 0 ? s_bL[(P - 1) * D + j] : 0.f;
@@ -707,9 +776,9 @@ __global__ void __launch_bounds__(kThreads) window_state_kernel(const WinArgs a)
     Ls = P > 0 ? s_bL[P - 1] : 0.f;
   }
   __syncthreads();
-  prepare_window_end<C>(sm, L, P, Lend, Ls, colexp, fac);
+  prepare_window_end<C>(st, L, P, Lend, Ls, colexp, fac);
   __syncthreads();
-  const WindowTile<C> tile = window_tile<C>(sm, L, P, r, colexp, fac);
+  const WindowTile<C> tile = window_tile<C>(st, L, P, r, colexp, fac);
   if constexpr (MODE == 0) {
     requantize_store<C>(tile, r, a.codes + (size_t)head * C::CODE_BYTES,
                         a.scales + (size_t)head * C::NSCALES,

@@ -19,9 +19,10 @@
  *   - All array arguments are DEVICE pointers unless the name says host; the caller owns and
  *     allocates every buffer (sizes from gdn_state_sizes). The library allocates no device
  *     memory and keeps no state between calls except a thread-local last-error message.
- *   - State buffers, fp32 state arrays (S) and the staging buffer must be 16-byte aligned; the
- *     per-step arrays q, k, v, o, g, beta, the status word and seq_mask need only their element
- *     alignment (GDN_ERR_INVALID_ARG otherwise).
+ *   - State buffers, fp32 state arrays (S), the staging buffer and, for the window step, q, k, v
+ *     and a per-channel g must be 16-byte aligned (they are moved with bulk async copies); o,
+ *     beta, a scalar g, the status word, seq_mask and the baseline step's inputs need only their
+ *     element alignment (GDN_ERR_INVALID_ARG otherwise).
  *   - Work is enqueued on `stream` and runs asynchronously; a GDN_OK return means the launch
  *     was accepted. Arguments are checked before anything is enqueued; on any error nothing is
  *     enqueued, except GDN_ERR_CUDA from a launch, after which outputs are undefined.

@@ -138,7 +138,7 @@ def test_input_pointer_checks(lib):
     cfg = _cfg()
     st = _fake_state()
     good = ctypes.c_void_p(0x900000)
-    odd = ctypes.c_void_p(0x900001)       # not 2-byte aligned for bf16
+    odd = ctypes.c_void_p(0x900008)       # bulk-copied q must be 16-byte aligned
     args = [good] * 6
     for i in range(6):
         a = list(args)

@@ -54,6 +54,16 @@ def build(force: bool = False, ptxas_info: bool = False, verbose: bool = False) 
     if not force and not ptxas_info and not _stale():
         return LIB
     os.makedirs(OBJ_DIR, exist_ok=True)
+    import fcntl
+
+    with open(os.path.join(OBJ_DIR, ".lock"), "w") as lock:  # one builder at a time
+        fcntl.flock(lock, fcntl.LOCK_EX)
+        if not force and not ptxas_info and not _stale():
+            return LIB
+        return _build_locked(ptxas_info, verbose)
+
+
+def _build_locked(ptxas_info: bool, verbose: bool) -> str:
     cc = nvcc()
     flags = _flags(ptxas_info)
 

@@ -62,6 +62,27 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return false;
 }
 
+// Tile swizzle of the stored state. A tile with RB-byte rows keeps its 16-byte chunks permuted
+// within each row: chunk c of row `row` lives at chunk c ^ x(row), x(row) = row & 7 for rows of
+// 128 bytes or more, (row * RB / 128) & (RB / 16 - 1) for shorter rows. Eight consecutive rows
+// read at one column then fall in distinct shared-memory banks, and a plain 1-D bulk copy of
+// the tile keeps the property. Returns the byte offset of logical byte b of the row.
+template <int RB>
+__host__ __device__ constexpr uint32_t swz(int row, int b) {
+  static_assert(RB >= 16 && (RB & (RB - 1)) == 0, "row bytes: a power of two >= 16");
+  if constexpr (RB >= 128) {
+    return (uint32_t)row * RB + ((((b >> 4) ^ (row & 7)) << 4) | (b & 15));
+  } else {
+    return (uint32_t)row * RB + ((((b >> 4) ^ ((row * RB / 128) & (RB / 16 - 1))) << 4) | (b & 15));
+  }
+}
+
+// Element offset of element `col` of row `row` in a swizzled tile of T with D columns.
+template <typename T, int D>
+__host__ __device__ constexpr uint32_t swz_el(int row, int col) {
+  return swz<D * (int)sizeof(T)>(row, col * (int)sizeof(T)) / (uint32_t)sizeof(T);
+}
+
 // e^x through the hardware base-2 exponential (flushes results below 2^-126 to zero).
 __device__ __forceinline__ float fast_exp(float x) {
   float y;

@@ -65,6 +65,8 @@ struct WinCfg {
   static_assert(!INT4 || D % 32 == 0, "int4 needs whole groups of 32");
   static_assert(NPASS * RPASS == D, "tile passes");
   static_assert(TC <= GS, "a thread's columns share one scale");
+  // Tensor-core (mma.sync) path: d = 128 with bf16 activations and bf16 buffers.
+  static constexpr bool MMA = D == 128 && sizeof(Act) == 2 && sizeof(Buf) == 2;
 };
 
 __host__ __device__ constexpr uint32_t align128(uint32_t x) { return (x + 127u) & ~127u; }
@@ -76,20 +78,28 @@ __host__ __device__ constexpr uint32_t align128(uint32_t x) { return (x + 127u) 
 // its whole head range.
 struct WinLayout {
   uint32_t codes, scales, bk, bu, bL, cidx, cu, q, k, v, g, stage_bytes;  // within a stage
-  uint32_t bars, stage0, vec, coef, red, harr, total;                     // within the CTA
+  uint32_t bars, stage0, vec, coef, red, tc, harr, total;                 // within the CTA
 };
+
+// Tensor-core scratch: int8 digit matrix of the phase-1 right-hand side [8][144 B], the bf16
+// [8][136] right-hand side of the pair-coefficient products, and the bf16 [8][Wr + 8] split
+// coefficients of the correction products (row strides padded against bank conflicts).
+__host__ __device__ constexpr uint32_t tc_scratch_bytes(int Wr) {
+  return 8u * 144 + 8u * 136 * 2 + 8u * (Wr + 8) * 2 + 64;
+}
 
 __host__ __device__ inline WinLayout win_layout(int D, int code_bytes, int nscales, int act_size,
                                                 int buf_size, bool diag, int W, int r,
                                                 int nstages, int per_cta) {
-  const int Wp = (W + 3) & ~3, rp = (r + 3) & ~3;
+  // buffer rows rounded up to 16: the mma k-steps read (zero-filled) rows past the window
+  const int Wp = (W + 3) & ~3, rp = (r + 3) & ~3, Wr = (W + 15) & ~15;
   WinLayout L;
   L.codes = 0;
   L.scales = align128(L.codes + code_bytes);
   L.bk = align128(L.scales + 4u * nscales);
-  L.bu = align128(L.bk + (uint32_t)W * D * act_size);
-  L.bL = align128(L.bu + (uint32_t)W * D * buf_size);
-  L.cidx = align128(L.bL + 4u * (diag ? (uint32_t)W * D : (uint32_t)Wp));
+  L.bu = align128(L.bk + (uint32_t)Wr * D * act_size);
+  L.bL = align128(L.bu + (uint32_t)Wr * D * buf_size);
+  L.cidx = align128(L.bL + 4u * (diag ? (uint32_t)Wr * D : (uint32_t)Wp));
   L.cu = align128(L.cidx + 4u * rp);
   L.q = align128(L.cu + 4u * r * D);
   L.k = align128(L.q + (uint32_t)D * act_size);
@@ -100,8 +110,9 @@ __host__ __device__ inline WinLayout win_layout(int D, int code_bytes, int nscal
   L.stage0 = 128;
   L.vec = L.stage0 + (uint32_t)nstages * L.stage_bytes;
   L.coef = align128(L.vec + 4u * (7 * D + 64));
-  L.red = align128(L.coef + 4u * (3 * (W + r) + 4));
-  L.harr = align128(L.red + 4u * 2 * kThreads);
+  L.red = align128(L.coef + 4u * (2 * (W + r) + Wr + 4));  // a[W+r], b[W+r], fac[Wr]
+  L.tc = align128(L.red + 4u * 2 * kThreads);
+  L.harr = align128(L.tc + tc_scratch_bytes(Wr));
   L.total = align128(L.harr + 12u * per_cta);
   return L;
 }
@@ -134,6 +145,21 @@ struct WinArgs {
   const int32_t* seq_mask; // forced flush: [B] or null
   int H, W, r;
 };
+
+// N consecutive logical elements (from column col0) of row `row` of a swizzled [rows][D] tile
+// of T, as fp32.
+template <typename T, int D, int N>
+__device__ __forceinline__ void load_sw(const T* base, int row, int col0, float* out) {
+  constexpr int EPC = 16 / (int)sizeof(T);  // elements per 16-byte chunk
+  if constexpr (N % EPC == 0) {
+#pragma unroll
+    for (int q = 0; q < N / EPC; ++q)
+      Num<T>::template load<EPC>(base + swz_el<T, D>(row, col0 + q * EPC), out + q * EPC);
+  } else {
+#pragma unroll
+    for (int e = 0; e < N; ++e) out[e] = Num<T>::to_f(base[swz_el<T, D>(row, col0 + e)]);
+  }
+}
 
 __device__ __forceinline__ void report(int32_t* status, int bit) {
   if (status) atomicOr(status, bit);
@@ -230,16 +256,16 @@ struct WindowTile {
       float cv[TC];
       if constexpr (C::INT4) {
         static_assert(TC == 8, "int4 tile is 8 columns per thread");
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(codes + row * C::ROW_BYTES + c0 / 2);
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(codes + swz<C::ROW_BYTES>(row, c0 / 2));
         i4x8_to_f32(w, cv);
       } else if constexpr (TC == 8) {
-        const uint2 w = *reinterpret_cast<const uint2*>(codes + row * C::ROW_BYTES + c0);
+        const uint2 w = *reinterpret_cast<const uint2*>(codes + swz<C::ROW_BYTES>(row, c0));
         i8x4_to_f32(w.x, cv);
         i8x4_to_f32(w.y, cv + 4);
       } else {
 #pragma unroll
         for (int b = 0; b < TC; ++b)
-          cv[b] = (float)(int)reinterpret_cast<const int8_t*>(codes)[row * C::ROW_BYTES + c0 + b];
+          cv[b] = (float)(int)reinterpret_cast<const int8_t*>(codes)[swz<C::ROW_BYTES>(row, c0 + b)];
       }
       const float s = scales[row * C::NG + c0 / C::GS];
 #pragma unroll
@@ -261,17 +287,13 @@ struct WindowTile {
       float uu[TR], kk[TC];
 #pragma unroll
       for (int a = 0; a < TR; ++a)
-        uu[a] = Num<typename C::Buf>::to_f(bu[i * D + ps * C::RPASS + rg * TR + a]);
+        uu[a] = Num<typename C::Buf>::to_f(
+            bu[swz_el<typename C::Buf, D>(i, ps * C::RPASS + rg * TR + a)]);
       if constexpr (C::DIAG) {
 #pragma unroll
         for (int b = 0; b < TC; ++b) kk[b] = ktil[i * D + c0 + b];
       } else {
-        if constexpr (TC % 8 == 0 || (TC % 4 == 0 && sizeof(typename C::Act) == 4)) {
-          Num<typename C::Act>::template load<TC>(bk + i * D + c0, kk);
-        } else {
-#pragma unroll
-          for (int b = 0; b < TC; ++b) kk[b] = Num<typename C::Act>::to_f(bk[i * D + c0 + b]);
-        }
+        load_sw<typename C::Act, D, TC>(bk, i, c0, kk);
         const float f = fac[i];
 #pragma unroll
         for (int a = 0; a < TR; ++a) uu[a] *= f;
@@ -399,7 +421,7 @@ __device__ void requantize_store(const Maker& make, int r, uint8_t* g_codes, flo
 #pragma unroll
         for (int m2 = 0; m2 < TC / 2; ++m2)
           wv |= (((uint32_t)q[2 * m2] & 0xFu) | (((uint32_t)q[2 * m2 + 1] & 0xFu) << 4)) << (8 * m2);
-        *reinterpret_cast<uint32_t*>(g_codes + row * C::ROW_BYTES + cg * TC / 2) = wv;
+        *reinterpret_cast<uint32_t*>(g_codes + swz<C::ROW_BYTES>(row, cg * TC / 2)) = wv;
         if (cg % span == 0) g_scales[row * C::NG + (cg * TC) / C::GS] = s;
       } else {
         if constexpr (TC == 8) {
@@ -408,11 +430,11 @@ __device__ void requantize_store(const Maker& make, int r, uint8_t* g_codes, flo
                  (((uint32_t)q[2] & 0xFFu) << 16) | (((uint32_t)q[3] & 0xFFu) << 24);
           wv.y = ((uint32_t)q[4] & 0xFFu) | (((uint32_t)q[5] & 0xFFu) << 8) |
                  (((uint32_t)q[6] & 0xFFu) << 16) | (((uint32_t)q[7] & 0xFFu) << 24);
-          *reinterpret_cast<uint2*>(g_codes + row * C::ROW_BYTES + cg * TC) = wv;
+          *reinterpret_cast<uint2*>(g_codes + swz<C::ROW_BYTES>(row, cg * TC)) = wv;
         } else {
 #pragma unroll
           for (int b = 0; b < TC; ++b)
-            reinterpret_cast<int8_t*>(g_codes)[row * C::ROW_BYTES + cg * TC + b] = (int8_t)q[b];
+            reinterpret_cast<int8_t*>(g_codes)[swz<C::ROW_BYTES>(row, cg * TC + b)] = (int8_t)q[b];
         }
         if (cg == 0) g_scales[row] = s;
       }
@@ -436,7 +458,8 @@ __device__ __forceinline__ void prepare_window_end(uint8_t* st, const WinLayout&
   if constexpr (C::DIAG) {
     for (int e = threadIdx.x; e < npairs * D; e += C::NT) {
       const int j = e % D;
-      bL[e] = Num<typename C::Act>::to_f(bk[e]) * fast_exp(Lvec[j] - bL[e]);
+      bL[e] = Num<typename C::Act>::to_f(bk[swz_el<typename C::Act, D>(e / D, j)]) *
+              fast_exp(Lvec[j] - bL[e]);
     }
   } else {
     for (int i = threadIdx.x; i < npairs; i += C::NT) fac[i] = fast_exp(Ls - bL[i]);
@@ -462,6 +485,10 @@ __device__ __forceinline__ WindowTile<C> window_tile(const uint8_t* st, const Wi
   return t;
 }
 
+}  // namespace gdnq
+#include "window_mma.cuh"
+namespace gdnq {
+
 // ------------------------------------------------------------------------------------------
 // One decode step (+ fused window flush) of one head whose data sit in stage `st`.
 // Called by all threads; ends with every thread done reading the stage's inputs.
@@ -473,6 +500,12 @@ __device__ __forceinline__ void step_head(const WinArgs& a, const WinLayout& L, 
   using Act = typename C::Act;
   using Buf = typename C::Buf;
   constexpr int D = C::D, CPR = C::CPR, RPP = C::RPP;
+  if constexpr (C::MMA) {
+    if (!C::DIAG || a.W <= kMmaDiagMaxW) {
+      step_head_mma<C>(a, L, sm, st, head, P, g_scalar, beta);
+      return;
+    }
+  }
   const int tid = threadIdx.x, lane = tid & 31;
   const int W = a.W, r = a.r, Wp = (W + 3) & ~3;
   const bool flush = (P + 1 == W);
@@ -525,11 +558,11 @@ __device__ __forceinline__ void step_head(const WinArgs& a, const WinLayout& L, 
     for (int row = tid / CPR; row < D; row += RPP) {
       float cv[16];
       if constexpr (C::INT4) {
-        const uint2 w = *reinterpret_cast<const uint2*>(s_codes + row * C::ROW_BYTES + c * 8);
+        const uint2 w = *reinterpret_cast<const uint2*>(s_codes + swz<C::ROW_BYTES>(row, c * 8));
         i4x8_to_f32(w.x, cv);
         i4x8_to_f32(w.y, cv + 8);
       } else {
-        const uint4 w = *reinterpret_cast<const uint4*>(s_codes + row * C::ROW_BYTES + c * 16);
+        const uint4 w = *reinterpret_cast<const uint4*>(s_codes + swz<C::ROW_BYTES>(row, c * 16));
         i8x4_to_f32(w.x, cv);
         i8x4_to_f32(w.y, cv + 4);
         i8x4_to_f32(w.z, cv + 8);
@@ -580,7 +613,7 @@ __device__ __forceinline__ void step_head(const WinArgs& a, const WinLayout& L, 
       float pa = 0.f, pb = 0.f;
       if (i < P) {
         float kk[16];
-        Num<Act>::template load<16>(s_bk + i * D + c * 16, kk);
+        load_sw<Act, D, 16>(s_bk, i, c * 16, kk);
         if constexpr (C::DIAG) {
           float ll[16];
           Num<float>::load<16>(s_bL + i * D + c * 16, ll);
@@ -628,7 +661,7 @@ __device__ __forceinline__ void step_head(const WinArgs& a, const WinLayout& L, 
     const int v = tid % D, grp = tid / D;
     float aw = 0.f, ar = 0.f;
     for (int i = grp; i < P; i += C::G) {
-      const float u = Num<Buf>::to_f(s_bu[i * D + v]);
+      const float u = Num<Buf>::to_f(s_bu[swz_el<Buf, D>(i, v)]);
       aw = fmaf(ca[i], u, aw);
       ar = fmaf(cb[i], u, ar);
     }
@@ -656,12 +689,12 @@ __device__ __forceinline__ void step_head(const WinArgs& a, const WinLayout& L, 
     const float ur = Num<Buf>::to_f(ub);
     static_cast<Act*>(a.o)[(size_t)head * D + v] = Num<Act>::from_f(rr + ur * misc[0]);
     if (!flush) {
-      static_cast<Buf*>(a.buf_u)[((size_t)head * W + P) * D + v] = ub;
-      static_cast<Act*>(a.buf_k)[((size_t)head * W + P) * D + v] = s_k[v];
+      static_cast<Buf*>(a.buf_u)[(size_t)head * W * D + swz_el<Buf, D>(P, v)] = ub;
+      static_cast<Act*>(a.buf_k)[(size_t)head * W * D + swz_el<Act, D>(P, v)] = s_k[v];
       if constexpr (C::DIAG) a.buf_L[((size_t)head * W + P) * D + v] = Lt[v];
     } else {
-      s_bu[P * D + v] = ub;
-      s_bk[P * D + v] = s_k[v];
+      s_bu[swz_el<Buf, D>(P, v)] = ub;
+      s_bk[swz_el<Act, D>(P, v)] = s_k[v];
       if constexpr (C::DIAG) s_bL[P * D + v] = Lt[v];
     }
   }
@@ -707,6 +740,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     if constexpr (!C::DIAG) hg[i] = a.g[h0 + i];
     hb[i] = a.beta[h0 + i];
   }
+  for (uint32_t e = tid; e < tc_scratch_bytes((a.W + 15) & ~15) / 4; e += C::NT)
+    reinterpret_cast<uint32_t*>(sm + L.tc)[e] = 0u;  // unused rows of the mma operands stay 0
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L.bars);
   if (tid == 0) {
     for (int s = 0; s < nstages; ++s) mbar_init(&bars[s], 1);

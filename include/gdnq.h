@@ -96,6 +96,12 @@ typedef struct {
  *   comp_u   fp32  [B][H][r][D]        value column of each compensator pair (r > 0 only)
  *   pos      int32 [B][H]              pairs already in the window, 0 <= pos < W
  *   status   int32 [1], optional       device word the kernels OR GDN_DEVICE_* bits into
+ * Tiles are stored swizzled: in each per-head [rows][RB-byte] tile of codes, buf_k and buf_u,
+ * the 16-byte chunk c of row i is stored at chunk c ^ x(i), x(i) = i & 7 when RB >= 128, else
+ * (i * RB / 128) & (RB / 16 - 1) (identity for 16-byte rows). A row's bytes keep their order
+ * within a chunk. This lets the kernels copy a head's tiles into shared memory with one bulk
+ * copy each and read eight consecutive rows at one column without bank conflicts.
+ * gdn_state_materialize returns the logical state in plain row-major order.
  * The logical state of a head with P = pos pairs and L = buf_L[P-1] (0 when P == 0) is
  *   S = dequant(codes, scales) Diag(e^L) + sum_c comp_u[c] (e_{comp_idx[c]} e^{L})^T
  *       + sum_{i<P} buf_u[i] (buf_k[i] * e^{L - buf_L[i]})^T.

@@ -24,9 +24,21 @@ def compile_oracle(src: str = SRC, out: str = OUT) -> str:
     return out
 
 
+def _stale() -> bool:
+    return not os.path.exists(OUT) or os.path.getmtime(OUT) < os.path.getmtime(SRC)
+
+
 def build(force: bool = False) -> str:
-    if force or not os.path.exists(OUT) or os.path.getmtime(OUT) < os.path.getmtime(SRC):
-        compile_oracle()
+    if force or _stale():
+        os.makedirs(OUT_DIR, exist_ok=True)
+        import fcntl
+
+        with open(os.path.join(OUT_DIR, ".lock"), "w") as lock:  # one builder at a time
+            fcntl.flock(lock, fcntl.LOCK_EX)
+            if force or _stale():
+                tmp = OUT + f".{os.getpid()}.tmp"
+                compile_oracle(SRC, tmp)
+                os.replace(tmp, OUT)
     return OUT
 
 

@@ -103,14 +103,27 @@ def oracle_run(wl: Workload, heads: np.ndarray, inputs: dict, S0: np.ndarray, fl
 # ---------------------------------------------------------------------------------------------
 # Reading the GPU state back per head
 # ---------------------------------------------------------------------------------------------
+def unswizzle(tiles: np.ndarray) -> np.ndarray:
+    """[n][rows][RB] bytes of swizzled tiles -> row-major bytes. Chunk c (16 bytes) of row i is
+    stored at chunk c ^ x(i): x(i) = i & 7 for rows of 128 bytes or more, else
+    (i * RB / 128) & (RB / 16 - 1) (the layout include/gdnq.h documents)."""
+    n, rows, RB = tiles.shape
+    nch = RB // 16
+    i = np.arange(rows)
+    x = (i & 7) if RB >= 128 else ((i * RB // 128) & (nch - 1))
+    src = np.arange(nch)[None, :] ^ x[:, None]             # [rows][nch] physical chunk
+    t = tiles.reshape(n, rows, nch, 16)
+    return np.take_along_axis(t, src[None, :, :, None], axis=2).reshape(n, rows, RB)
+
+
 def gpu_codes(wl: Workload, st: gdn.GdnState, heads: np.ndarray) -> np.ndarray:
-    """Unpacked int8 codes [n][D][D] of the chosen heads."""
+    """Unpacked int8 codes [n][D][D] of the chosen heads, in row-major order."""
     D = wl.D
+    h = torch.as_tensor(heads, device=st.codes.device)
     if wl.fmt == "int4_g32":
-        packed = st.codes.view(-1, D, D // 2)[torch.as_tensor(heads, device=st.codes.device)]
-        return np.stack([oracle.unpack_int4(p) for p in packed.cpu().numpy()])
-    return st.codes.view(torch.int8).view(-1, D, D)[
-        torch.as_tensor(heads, device=st.codes.device)].cpu().numpy()
+        packed = unswizzle(st.codes.view(-1, D, D // 2)[h].cpu().numpy())
+        return np.stack([oracle.unpack_int4(p) for p in packed])
+    return unswizzle(st.codes.view(-1, D, D)[h].cpu().numpy()).view(np.int8)
 
 
 def gpu_scales(wl: Workload, st: gdn.GdnState, heads: np.ndarray) -> np.ndarray:

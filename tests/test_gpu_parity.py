@@ -33,6 +33,10 @@ SMALL = {
                                                   outliers=True, warmup=16),
     "gdn-d16-bf16-r3": WORKLOADS["gdn-tiny"].with_(name="gdn-d16-bf16", H=3, r=3, act="bf16",
                                                    buf="bf16", T=70, warmup=16),
+    # diagonal gate with a window past the tensor-core flush's limit (FMA path)
+    "kda-int8-w160": KDA.with_(name="kda-w160", B=1, H=2, T=170, W=160, r=2, warmup=32),
+    "gdn-int8-w16": MID.with_(name="gdn-w16", B=2, H=3, T=50, W=16, warmup=32),
+    "gdn-int8-w20": MID.with_(name="gdn-w20", B=2, H=3, T=50, W=20, r=1, warmup=32),
 }
 
 

@@ -83,6 +83,34 @@ __host__ __device__ constexpr uint32_t swz_el(int row, int col) {
   return swz<D * (int)sizeof(T)>(row, col * (int)sizeof(T)) / (uint32_t)sizeof(T);
 }
 
+// Barrier among the 256 computing threads of a CTA (named barrier 1): in the persistent step
+// kernel a 9th warp stages data and never joins; in the other kernels it is every thread.
+constexpr int kComputeThreads = 256;
+
+__device__ __forceinline__ void csync() {
+  asm volatile("bar.sync 1, %0;\n" ::"n"(kComputeThreads) : "memory");
+}
+
+// csync() that also returns whether any computing thread passed a nonzero `pred`.
+__device__ __forceinline__ int csync_or(int pred) {
+  int out;
+  asm volatile(
+      "{\n"
+      " .reg .pred p, q;\n"
+      " setp.ne.s32 p, %1, 0;\n"
+      " barrier.cta.red.or.pred q, 1, %2, p;\n"
+      " selp.s32 %0, 1, 0, q;\n"
+      "}\n"
+      : "=r"(out)
+      : "r"(pred), "n"(kComputeThreads)
+      : "memory");
+  return out;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // e^x through the hardware base-2 exponential (flushes results below 2^-126 to zero).
 __device__ __forceinline__ float fast_exp(float x) {
   float y;

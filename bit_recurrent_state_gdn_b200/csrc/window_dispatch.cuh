@@ -76,7 +76,7 @@ cudaError_t launch_window_cfg(WinOp op, const WinArgs& a, int heads, cudaStream_
       const StepPlan p = plan_step<C>(a.W, a.r, heads);
       e = ensure_smem<window_step_kernel<C>>(p.smem);
       if (e == cudaSuccess)
-        window_step_kernel<C><<<p.grid, kThreads, p.smem, st>>>(a, heads, p.per_cta, p.nstages);
+        window_step_kernel<C><<<p.grid, kStepThreads, p.smem, st>>>(a, heads, p.per_cta, p.nstages);
       break;
     }
     case WinOp::Flush:

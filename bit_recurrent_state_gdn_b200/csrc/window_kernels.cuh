@@ -213,7 +213,7 @@ __device__ __forceinline__ void stage_issue(const WinArgs& a, const WinLayout& L
 // which case every thread returns.
 __device__ __forceinline__ bool stage_wait(const WinArgs& a, uint64_t* bar, uint32_t parity) {
   const int timed_out = mbar_wait_bounded(bar, parity) ? 0 : 1;
-  if (__syncthreads_or(timed_out)) {
+  if (csync_or(timed_out)) {
     if (threadIdx.x == 0) report(a.status, GDN_DEVICE_WAIT_TIMEOUT);
     return false;
   }
@@ -344,7 +344,7 @@ __device__ void requantize_store(const Maker& make, int r, uint8_t* g_codes, flo
 
   if (r > 0) {
     for (int j = tid; j < D; j += C::NT) colmax[j] = 0.f;
-    __syncthreads();
+    csync();
     for (int ps = 0; ps < C::NPASS; ++ps) {
       make(ps, acc);
 #pragma unroll
@@ -357,7 +357,7 @@ __device__ void requantize_store(const Maker& make, int r, uint8_t* g_codes, flo
           atomicMax(reinterpret_cast<unsigned int*>(colmax) + cg * TC + b, __float_as_uint(m));
       }
     }
-    __syncthreads();
+    csync();
     if (warp == 0) {
       for (int c = 0; c < r; ++c) {
         float bv = -1.f;
@@ -379,7 +379,7 @@ __device__ void requantize_store(const Maker& make, int r, uint8_t* g_codes, flo
         __syncwarp();
       }
     }
-    __syncthreads();
+    csync();
   }
 
   for (int ps = 0; ps < C::NPASS; ++ps) {
@@ -544,7 +544,7 @@ __device__ __forceinline__ void step_head(const WinArgs& a, const WinLayout& L, 
     xs[tid] = e * kj;
     ys[tid] = e * qj;
   }
-  __syncthreads();
+  csync();
 
   // ---- phase 1: p = F x, r = F y ---------------------------------------------------------
   {
@@ -654,7 +654,7 @@ __device__ __forceinline__ void step_head(const WinArgs& a, const WinLayout& L, 
       if (lane == 0) misc[0] = s;
     }
   }
-  __syncthreads();
+  csync();
 
   // ---- phase 3: corrections from the buffered write vectors and compensators -------------
   {
@@ -673,7 +673,7 @@ __device__ __forceinline__ void step_head(const WinArgs& a, const WinLayout& L, 
     red[grp * 2 * D + v] = aw;
     red[grp * 2 * D + D + v] = ar;
   }
-  __syncthreads();
+  csync();
 
   // ---- phase 4: write vector, output, append -------------------------------------------
   if (tid < D) {
@@ -708,10 +708,10 @@ __device__ __forceinline__ void step_head(const WinArgs& a, const WinLayout& L, 
   if (!flush) return;
 
   // ---- phase 5: window end -------------------------------------------------------------
-  __syncthreads();
+  csync();
   float* colexp = xs;  // x, y are dead
   prepare_window_end<C>(st, L, P + 1, Lt, Ls, colexp, fac);
-  __syncthreads();
+  csync();
   const WindowTile<C> tile = window_tile<C>(st, L, P + 1, r, colexp, fac);
   requantize_store<C>(tile, r, a.codes + (size_t)head * C::CODE_BYTES,
                       a.scales + (size_t)head * C::NSCALES,
@@ -723,8 +723,10 @@ __device__ __forceinline__ void step_head(const WinArgs& a, const WinLayout& L, 
 // Decode step, persistent: CTA b owns heads [b * per_cta, (b + 1) * per_cta) and walks them in
 // order while up to nstages - 1 later heads are already being copied into their stages.
 // ------------------------------------------------------------------------------------------
+constexpr int kStepThreads = kThreads;
+
 template <class C>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kStepThreads, 2)
     window_step_kernel(const WinArgs a, const int heads, const int per_cta, const int nstages) {
   extern __shared__ __align__(128) uint8_t sm[];
   const WinLayout L = win_layout<C>(a.W, a.r, nstages, per_cta);
@@ -747,7 +749,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int s = 0; s < nstages; ++s) mbar_init(&bars[s], 1);
     fence_barrier_init();
   }
-  __syncthreads();
+  csync();
   if (tid == 0)
     for (int s = 0; s < nstages && s < nh; ++s)
       stage_issue<C>(a, L, sm + L.stage0 + s * L.stage_bytes, &bars[s], h0 + s, hpos[s], true);
@@ -761,11 +763,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     } else if (tid == 0) {
       report(a.status, GDN_DEVICE_BAD_POS);
     }
-    __syncthreads();  // the stage and the per-head scratch are free again
-    if (tid == 0 && n + nstages < nh) {
-      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    // the stage's generic-proxy writes are ordered before the async copies that refill it
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    csync();  // the stage and the per-head scratch are free again
+    if (tid == 0 && n + nstages < nh)
       stage_issue<C>(a, L, st, &bars[s], h0 + n + nstages, hpos[n + nstages], true);
-    }
   }
 }
 
@@ -796,7 +798,7 @@ __global__ void __launch_bounds__(kThreads) window_state_kernel(const WinArgs a)
     fence_barrier_init();
     stage_issue<C>(a, L, st, bar, head, P, false);
   }
-  __syncthreads();
+  csync();
   if (!stage_wait(a, bar, 0)) return;
 
   float* vec = reinterpret_cast<float*>(sm + L.vec);
@@ -810,9 +812,9 @@ __global__ void __launch_bounds__(kThreads) window_state_kernel(const WinArgs a)
   } else {
     Ls = P > 0 ? s_bL[P - 1] : 0.f;
   }
-  __syncthreads();
+  csync();
   prepare_window_end<C>(st, L, P, Lend, Ls, colexp, fac);
-  __syncthreads();
+  csync();
   const WindowTile<C> tile = window_tile<C>(st, L, P, r, colexp, fac);
   if constexpr (MODE == 0) {
     requantize_store<C>(tile, r, a.codes + (size_t)head * C::CODE_BYTES,

@@ -112,6 +112,26 @@ template <class C>
 __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uint8_t* st, int head,
                           int P, float Ls);
 
+// Pair i's coefficients (a, b) as the three-way bf16 split rows of the phase-3 right-hand side.
+__device__ __forceinline__ void put_coef(__nv_bfloat16* Bc, int bcs, int i, float av, float bv) {
+  float h, m, l;
+  split3(av, h, m, l);
+  Bc[0 * bcs + i] = __float2bfloat16_rn(h);
+  Bc[1 * bcs + i] = __float2bfloat16_rn(m);
+  Bc[2 * bcs + i] = __float2bfloat16_rn(l);
+  split3(bv, h, m, l);
+  Bc[3 * bcs + i] = __float2bfloat16_rn(h);
+  Bc[4 * bcs + i] = __float2bfloat16_rn(m);
+  Bc[5 * bcs + i] = __float2bfloat16_rn(l);
+}
+
+// Byte offset of digit (row n, logical k) in the fragment-ordered phase-1 right-hand side: lane
+// (n, q4) finds its eight 32-bit b-registers (b0, b1 of the four 32-column chunks) contiguous.
+__device__ __forceinline__ int digit_off(int n, int k) {
+  const int c = k >> 5, kk = k & 31, half = kk >> 4, q4 = (kk & 15) >> 2, e = kk & 3;
+  return ((n * 4 + q4) * 8 + c * 2 + half) * 4 + e;
+}
+
 template <class C>
 __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm,
                                               uint8_t* st, int head, int P, float g_scalar,
@@ -122,13 +142,14 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
   const int mi = lane >> 3, r8 = lane & 7;
   const int W = a.W, r = a.r, Wp = (W + 3) & ~3, Wr = (W + 15) & ~15, bcs = Wr + 8;
   const bool flush = (P + 1 == W);
+  const int Pp = (P + 15) & ~15;
 
   float* vec = reinterpret_cast<float*>(sm + L.vec);
   float *kt = vec, *qt = vec + D, *xs = vec + 2 * D, *ys = vec + 3 * D, *Lt = vec + 4 * D;
-  float* misc = vec + 7 * D;  // [0..3] k.q partials, [24..27] x chunk scales, [28..31] y
+  float* misc = vec + 7 * D;  // [0..3] k.q partials, [24] x block scale, [25] y block scale
   float* coef = reinterpret_cast<float*>(sm + L.coef);
   float *ca = coef, *cb = coef + (W + r);
-  int8_t* Bt8 = reinterpret_cast<int8_t*>(sm + L.tc);            // [8][144]
+  uint8_t* Bfrag = sm + L.tc;                                      // digits, fragment order
   bf* Bk = reinterpret_cast<bf*>(sm + L.tc + 8 * 144);            // [8][136]
   bf* Bc = reinterpret_cast<bf*>(sm + L.tc + 8 * 144 + 8 * 136 * 2);  // [8][Wr + 8]
 
@@ -144,118 +165,154 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
   const bf* s_v = reinterpret_cast<const bf*>(st + L.v);
   const float* s_g = reinterpret_cast<const float*>(st + L.g);
 
-  // ---- gates; digit columns of phase 1 (warps 0-3: x, chunk w; warps 4-7: y, chunk w-4) ----
   float Ls = 0.f;
   if constexpr (!C::DIAG) Ls = (P > 0 ? s_bL[P - 1] : 0.f) + g_scalar;
+
+  // ---- gates, phase-1 digit columns, the step's key / log-gate appended ------------------
+  // Warps 0-3 take the key side x, warps 4-7 the query side y; warp w owns the 32 columns of
+  // chunk w % 4 (lane l: column 32 (w % 4) + l). Each vector gets one block exponent, found by
+  // every warp of its side from all 128 columns (no cross-warp step): X = rint(v 2^(22-e)),
+  // |X| <= 2^22, three signed 8-bit digits X = d1 2^16 + d2 2^8 + d3.
   {
     const bool isy = warp >= 4;
     const int j = (warp & 3) * 32 + lane;
+    const bf* sv = isy ? s_q : s_k;
+    float m = 0.f, val = 0.f, lj = Ls;
+#pragma unroll
+    for (int mm = 0; mm < 4; ++mm) {
+      const int jj = lane + 32 * mm;
+      float l;
+      if constexpr (C::DIAG) l = (P > 0 ? s_bL[(P - 1) * D + jj] : 0.f) + s_g[jj];
+      else l = Ls;
+      const float v = C::DIAG ? fast_exp(l) * __bfloat162float(sv[jj]) : __bfloat162float(sv[jj]);
+      m = fmaxf(m, fabsf(v));
+      if (mm == (warp & 3)) {  // this lane's own column j
+        val = v;
+        lj = l;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     const float kj = __bfloat162float(s_k[j]), qj = __bfloat162float(s_q[j]);
-    float l;
-    if constexpr (C::DIAG) l = (P > 0 ? s_bL[(P - 1) * D + j] : 0.f) + s_g[j];
-    else l = Ls;
-    const float e = fast_exp(l);
-    float val;
+    const float e = C::DIAG ? fast_exp(lj) : fast_exp(Ls);
     if (!isy) {
       kt[j] = kj;
-      Lt[j] = l;
+      Lt[j] = lj;
       xs[j] = e * kj;
-      val = C::DIAG ? e * kj : kj;  // scalar gate: e^{L_t} is applied after the product
       Bk[j] = s_k[j];
-      float s = kj * qj;
+      float kq = kj * qj;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-      if (lane == 0) misc[warp] = s;
+      for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+      if (lane == 0) misc[warp] = kq;
+      if (!flush) {
+        static_cast<bf*>(a.buf_k)[(size_t)head * W * D + swz_el<bf, D>(P, j)] = s_k[j];
+        if constexpr (C::DIAG) a.buf_L[((size_t)head * W + P) * D + j] = lj;
+      } else {
+        s_bk[swz_el<bf, D>(P, j)] = s_k[j];
+        if constexpr (C::DIAG) s_bL[P * D + j] = lj;
+      }
     } else {
       qt[j] = qj;
       ys[j] = e * qj;
-      val = C::DIAG ? e * qj : qj;
       Bk[136 + j] = s_q[j];
     }
-    float m = fabsf(val);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    int X = 0;
-    float scale = 0.f;
-    if (m >= 0x1p-100f) {  // smaller chunks contribute nothing measurable
-      int e2;
-      frexpf(m, &e2);  // m = f 2^e2, 0.5 <= f < 1
-      X = __float2int_rn(val * ldexpf(1.f, 22 - e2));  // |X| <= 2^22
-      scale = ldexpf(1.f, e2 - 22);
+    float mul = 0.f, scale = 0.f;
+    if (m >= 0x1p-100f) {  // smaller vectors contribute nothing measurable
+      // m = f 2^e2 with 0.5 <= f < 1 (m is normal); powers of two from exponent bits
+      const int e2 = ((__float_as_int(m) >> 23) & 0xFF) - 126;
+      mul = __int_as_float((22 - e2 + 127) << 23);
+      scale = __int_as_float((e2 - 22 + 127) << 23);
     }
+    const int X = __float2int_rn(val * mul);
     const int d3 = (int)(int8_t)(X & 0xFF);
     const int X1 = (X - d3) >> 8;  // exact: X - d3 is a multiple of 256
     const int d2 = (int)(int8_t)(X1 & 0xFF);
     const int d1 = (X1 - d2) >> 8;
-    const int n0 = isy ? 3 : 0, pj = digit_pos<C::INT4>(j);
-    Bt8[(n0 + 0) * 144 + pj] = (int8_t)d1;
-    Bt8[(n0 + 1) * 144 + pj] = (int8_t)d2;
-    Bt8[(n0 + 2) * 144 + pj] = (int8_t)d3;
-    if (lane == 0) misc[24 + (isy ? 4 : 0) + (warp & 3)] = scale;
+    const int n0 = isy ? 3 : 0, k = digit_pos<C::INT4>(j);
+    Bfrag[digit_off(n0 + 0, k)] = (uint8_t)d1;
+    Bfrag[digit_off(n0 + 1, k)] = (uint8_t)d2;
+    Bfrag[digit_off(n0 + 2, k)] = (uint8_t)d3;
+    if (lane == 0 && (warp & 3) == 0) misc[24 + (isy ? 1 : 0)] = scale;
+    if (tid == 0) {
+      if constexpr (!C::DIAG) {
+        if (!flush) a.buf_L[(size_t)head * Wp + P] = Ls;
+        else s_bL[P] = Ls;
+      }
+    }
+    // padding of the phase-3 product to a multiple of 16 pairs: zero rows of U and zero
+    // coefficients (the product must not see stale or non-finite shared memory)
+    for (int e2 = tid; e2 < (Pp - P) * D; e2 += C::NT) s_bu[P * D + e2] = __float2bfloat16_rn(0.f);
+    for (int e2 = tid; e2 < 6 * (Pp - P); e2 += C::NT)
+      Bc[(e2 / (Pp - P)) * bcs + P + e2 % (Pp - P)] = __float2bfloat16_rn(0.f);
   }
-  __syncthreads();
+  csync();
 
-  // ---- phase 1: p = F x, r = F y for rows 16w + gid (+8), held by the quad leaders -------
+  // ---- phase 1: p = F x, r = F y for rows 16w + gid (+8) ----------------------------------
   float pr[2], rr[2];
   {
-    // digit weights of this lane's two columns (2q4, 2q4+1): x = cols 0..2, y = cols 3..5
+    // digit weights of this lane's columns 2q4, 2q4+1: x = columns 0..2, y = columns 3..5
     const float wx0 = q4 == 0 ? 65536.f : (q4 == 1 ? 1.f : 0.f);
     const float wx1 = q4 == 0 ? 256.f : 0.f;
     const float wy0 = q4 == 2 ? 256.f : 0.f;
     const float wy1 = q4 == 1 ? 65536.f : (q4 == 2 ? 1.f : 0.f);
-    float PX[2] = {0.f, 0.f}, PY[2] = {0.f, 0.f};
+    const uint4 bw0 = *reinterpret_cast<const uint4*>(Bfrag + (gid * 4 + q4) * 32);
+    const uint4 bw1 = *reinterpret_cast<const uint4*>(Bfrag + (gid * 4 + q4) * 32 + 16);
+    const uint32_t bw[8] = {bw0.x, bw0.y, bw0.z, bw0.w, bw1.x, bw1.y, bw1.z, bw1.w};
     const uint32_t cb0 = smem_u32(s_codes);
+    float PX[2], PY[2];
+    if constexpr (C::INT4) {
+      PX[0] = PX[1] = PY[0] = PY[1] = 0.f;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t A[4];
-      if constexpr (C::INT4) {
-        uint32_t w0, w1;
+      for (int c = 0; c < 4; ++c) {  // each 32-column chunk is one scale group
+        uint32_t A[4], w0, w1;
         ldsm_x2(cb0 + swz<64>(16 * warp + r8 + 8 * (mi & 1), 16 * c), w0, w1);
         i4x8_to_s8x16(w0, A[0], A[2]);
         i4x8_to_s8x16(w1, A[1], A[3]);
-      } else {
-        ldsm_x4(cb0 + swz<128>(16 * warp + r8 + 8 * (mi & 1), 32 * c + 16 * (mi >> 1)), A);
+        int Cc[4] = {0, 0, 0, 0};
+        mma_s8(Cc, A, bw[2 * c], bw[2 * c + 1]);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float sg = s_scales[(16 * warp + gid + 8 * h) * C::NG + c];
+          const float c0 = (float)Cc[2 * h], c1 = (float)Cc[2 * h + 1];
+          PX[h] = fmaf(sg, wx0 * c0 + wx1 * c1, PX[h]);
+          PY[h] = fmaf(sg, wy0 * c0 + wy1 * c1, PY[h]);
+        }
       }
-      const uint32_t b0 = *reinterpret_cast<const uint32_t*>(Bt8 + gid * 144 + 32 * c + 4 * q4);
-      const uint32_t b1 = *reinterpret_cast<const uint32_t*>(Bt8 + gid * 144 + 32 * c + 16 + 4 * q4);
-      int Cc[4] = {0, 0, 0, 0};
-      mma_s8(Cc, A, b0, b1);
-      float sx = misc[24 + c], sy = misc[28 + c];
-      if constexpr (C::INT4) {
-        sx *= 0.0625f;  // codes entered as 16 x code
-        sy *= 0.0625f;
+    } else {
+      int Cc[4] = {0, 0, 0, 0};  // one exponent per vector: chunks accumulate exactly in int32
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t A[4];
+        ldsm_x4(cb0 + swz<128>(16 * warp + r8 + 8 * (mi & 1), 32 * c + 16 * (mi >> 1)), A);
+        mma_s8(Cc, A, bw[2 * c], bw[2 * c + 1]);
       }
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const float c0 = (float)Cc[2 * h], c1 = (float)Cc[2 * h + 1];
-        float px = sx * (wx0 * c0 + wx1 * c1), py = sy * (wy0 * c0 + wy1 * c1);
-        if constexpr (C::INT4) {
-          const float sg = s_scales[(16 * warp + gid + 8 * h) * C::NG + c];
-          px *= sg;
-          py *= sg;
-        }
-        PX[h] += px;
-        PY[h] += py;
+        PX[h] = wx0 * c0 + wx1 * c1;
+        PY[h] = wy0 * c0 + wy1 * c1;
       }
     }
     const float gam = C::DIAG ? 1.f : fast_exp(Ls);
+    const float sx = misc[24] * gam * (C::INT4 ? 0.0625f : 1.f);  // int4 codes entered as 16 c
+    const float sy = misc[25] * gam * (C::INT4 ? 0.0625f : 1.f);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       PX[h] += __shfl_xor_sync(0xffffffffu, PX[h], 1);
       PX[h] += __shfl_xor_sync(0xffffffffu, PX[h], 2);
       PY[h] += __shfl_xor_sync(0xffffffffu, PY[h], 1);
       PY[h] += __shfl_xor_sync(0xffffffffu, PY[h], 2);
-      const float srow = C::INT4 ? gam : gam * s_scales[16 * warp + gid + 8 * h];
-      pr[h] = PX[h] * srow;
-      rr[h] = PY[h] * srow;
+      const float srow = C::INT4 ? 1.f : s_scales[16 * warp + gid + 8 * h];
+      pr[h] = PX[h] * sx * srow;
+      rr[h] = PY[h] * sy * srow;
     }
   }
 
-  // ---- phase 2: pair coefficients a_i, b_i -------------------------------------------------
+  // ---- phase 2: pair coefficients, written as the split phase-3 right-hand side --------
   if constexpr (!C::DIAG) {
-    const int tiles = (P + 15) >> 4;
+    const int tiles = Pp >> 4;
     for (int tile = warp; tile < tiles; tile += 8) {
-      float Cc[4] = {0.f, 0.f, 0.f, 0.f};
+      float Ce[4] = {0.f, 0.f, 0.f, 0.f}, Co[4] = {0.f, 0.f, 0.f, 0.f};  // even / odd k-steps
       const uint32_t kb = smem_u32(s_bk);
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
@@ -263,18 +320,24 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
         ldsm_x4(kb + swz<256>(16 * tile + r8 + 8 * (mi & 1), 2 * (16 * s + 8 * (mi >> 1))), A);
         const uint32_t b0 = *reinterpret_cast<const uint32_t*>(Bk + gid * 136 + 16 * s + 2 * q4);
         const uint32_t b1 = *reinterpret_cast<const uint32_t*>(Bk + gid * 136 + 16 * s + 8 + 2 * q4);
-        mma_bf16(Cc, A, b0, b1);
+        if (s & 1) mma_bf16(Co, A, b0, b1);
+        else mma_bf16(Ce, A, b0, b1);
       }
-      if (q4 == 0) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int i = 16 * tile + gid + 8 * h;
-          if (i < P) {
-            const float f = fast_exp(Ls - s_bL[i]);
-            ca[i] = Cc[2 * h] * f;
-            cb[i] = Cc[2 * h + 1] * f;
-          }
-        }
+      // the quad leader holds (a, b) of rows gid and gid+8; lane q4 splits one of the four
+      const int ld = lane & ~3;
+      const float a0 = __shfl_sync(0xffffffffu, Ce[0] + Co[0], ld);
+      const float b0 = __shfl_sync(0xffffffffu, Ce[1] + Co[1], ld);
+      const float a1 = __shfl_sync(0xffffffffu, Ce[2] + Co[2], ld);
+      const float b1 = __shfl_sync(0xffffffffu, Ce[3] + Co[3], ld);
+      const float vq = q4 == 0 ? a0 : (q4 == 1 ? b0 : (q4 == 2 ? a1 : b1));
+      const int i = 16 * tile + gid + 8 * (q4 >> 1);
+      if (i < P) {
+        float h, m, l;
+        split3(vq * fast_exp(Ls - s_bL[i]), h, m, l);
+        const int row = (q4 & 1) ? 3 : 0;
+        Bc[(row + 0) * bcs + i] = __float2bfloat16_rn(h);
+        Bc[(row + 1) * bcs + i] = __float2bfloat16_rn(m);
+        Bc[(row + 2) * bcs + i] = __float2bfloat16_rn(l);
       }
     }
   } else {
@@ -311,10 +374,7 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
         pa += __shfl_xor_sync(0xffffffffu, pa, off);
         pb += __shfl_xor_sync(0xffffffffu, pb, off);
       }
-      if (c == 0 && i < P) {
-        ca[i] = pa;
-        cb[i] = pb;
-      }
+      if (c == 0 && i < P) put_coef(Bc, bcs, i, pa, pb);
     }
   }
   if (tid < r) {  // compensator pairs: key e_j entered at L = 0
@@ -322,25 +382,9 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
     ca[W + tid] = xs[j];
     cb[W + tid] = ys[j];
   }
-  const int Pp = (P + 15) & ~15;
-  for (int e = tid; e < (Pp - P) * D; e += C::NT) s_bu[P * D + e] = __float2bfloat16_rn(0.f);
-  __syncthreads();
+  csync();
 
-  // ---- split coefficients into the bf16 right-hand side of phase 3 ----------------------
-  for (int i = tid; i < Pp; i += C::NT) {
-    float h, m, l;
-    split3(i < P ? ca[i] : 0.f, h, m, l);
-    Bc[0 * bcs + i] = __float2bfloat16_rn(h);
-    Bc[1 * bcs + i] = __float2bfloat16_rn(m);
-    Bc[2 * bcs + i] = __float2bfloat16_rn(l);
-    split3(i < P ? cb[i] : 0.f, h, m, l);
-    Bc[3 * bcs + i] = __float2bfloat16_rn(h);
-    Bc[4 * bcs + i] = __float2bfloat16_rn(m);
-    Bc[5 * bcs + i] = __float2bfloat16_rn(l);
-  }
-  __syncthreads();
-
-  // ---- phase 3: w = p + U^T a (+ compensators), r likewise; phase 4 in the quad leaders ---
+  // ---- phase 3: w = p + U^T a (+ compensators), r likewise; then u_t, o_t -----------------
   {
     float Cc[4] = {0.f, 0.f, 0.f, 0.f};
     const uint32_t ub = smem_u32(s_bu);
@@ -364,44 +408,26 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
       Rv[h] += __shfl_xor_sync(0xffffffffu, Rv[h], 1);
       Rv[h] += __shfl_xor_sync(0xffffffffu, Rv[h], 2);
     }
-    if (q4 == 0) {
-      const float kq = misc[0] + misc[1] + misc[2] + misc[3];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int v = 16 * warp + gid + 8 * h;
-        float w = pr[h] + Wv[h], rv = rr[h] + Rv[h];
-        for (int c = 0; c < r; ++c) {
-          const float cu = s_cu[c * D + v];
-          w = fmaf(ca[W + c], cu, w);
-          rv = fmaf(cb[W + c], cu, rv);
-        }
-        const float u = beta * (__bfloat162float(s_v[v]) - w);
-        const bf ubf = __float2bfloat16_rn(u);
-        static_cast<bf*>(a.o)[(size_t)head * D + v] =
-            __float2bfloat16_rn(rv + __bfloat162float(ubf) * kq);
-        if (!flush) static_cast<bf*>(a.buf_u)[(size_t)head * W * D + swz_el<bf, D>(P, v)] = ubf;
-        else s_bu[swz_el<bf, D>(P, v)] = ubf;
+    if (q4 < 2) {  // lane q4 of the quad finishes row 16w + gid + 8 q4
+      const int v = 16 * warp + gid + 8 * q4;
+      float w = (q4 ? pr[1] : pr[0]) + (q4 ? Wv[1] : Wv[0]);
+      float rv = (q4 ? rr[1] : rr[0]) + (q4 ? Rv[1] : Rv[0]);
+      for (int c = 0; c < r; ++c) {
+        const float cu = s_cu[c * D + v];
+        w = fmaf(ca[W + c], cu, w);
+        rv = fmaf(cb[W + c], cu, rv);
       }
+      const float u = beta * (__bfloat162float(s_v[v]) - w);
+      const bf ubf = __float2bfloat16_rn(u);
+      const float kq = misc[0] + misc[1] + misc[2] + misc[3];
+      static_cast<bf*>(a.o)[(size_t)head * D + v] = __float2bfloat16_rn(rv + __bfloat162float(ubf) * kq);
+      if (!flush) static_cast<bf*>(a.buf_u)[(size_t)head * W * D + swz_el<bf, D>(P, v)] = ubf;
+      else s_bu[swz_el<bf, D>(P, v)] = ubf;
     }
   }
-  if (tid < D) {
-    if (!flush) {
-      static_cast<bf*>(a.buf_k)[(size_t)head * W * D + swz_el<bf, D>(P, tid)] = s_k[tid];
-      if constexpr (C::DIAG) a.buf_L[((size_t)head * W + P) * D + tid] = Lt[tid];
-    } else {
-      s_bk[swz_el<bf, D>(P, tid)] = s_k[tid];
-      if constexpr (C::DIAG) s_bL[P * D + tid] = Lt[tid];
-    }
-  }
-  if (tid == 0) {
-    if constexpr (!C::DIAG) {
-      if (!flush) a.buf_L[(size_t)head * Wp + P] = Ls;
-      else s_bL[P] = Ls;
-    }
-    a.pos[head] = flush ? 0 : P + 1;
-  }
+  if (tid == 0) a.pos[head] = flush ? 0 : P + 1;
   if (!flush) return;
-  __syncthreads();
+  csync();
   flush_mma<C>(a, L, sm, st, head, P, Ls);
 }
 
@@ -465,7 +491,7 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
         los[t] = pack_bf16(l0, l1);
       }
     }
-    __syncthreads();
+    csync();
 #pragma unroll
     for (int t = 0; t < kPairs; ++t) {
       const int e = 2 * (tid + t * C::NT);
@@ -476,7 +502,7 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
       }
     }
   }
-  __syncthreads();
+  csync();
 
   // ---- the materialised state, one 64-column half (n-tiles 8hc..8hc+7) at a time -----------
   // acc[n][0..3] = S_W at (v0, j), (v0, j+1), (v1, j), (v1, j+1), j = 64hc + 8n + 2q4
@@ -615,7 +641,7 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
         }
       }
     }
-    __syncthreads();
+    csync();
     if (warp == 0) {
       for (int c = 0; c < r; ++c) {
         float bv = -1.f;
@@ -637,7 +663,7 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
         __syncwarp();
       }
     }
-    __syncthreads();
+    csync();
     if (tid < r) a.comp_idx[(size_t)head * ((r + 3) & ~3) + tid] = sel[tid];
   }
 

@@ -32,6 +32,8 @@ METRIC = "GDN decode head-steps/s (int8 windowed state); achieved HBM GB/s vs B2
 UNIT = "head-steps/s"
 PROFILE = os.path.join(ROOT, "profiles", "window_step_gdn-serving.md")
 KERNEL_SOURCES = ["bit_recurrent_state_gdn_b200/csrc/window_kernels.cuh",
+                  "bit_recurrent_state_gdn_b200/csrc/window_mma.cuh",
+                  "bit_recurrent_state_gdn_b200/csrc/window_dispatch.cuh",
                   "bit_recurrent_state_gdn_b200/csrc/device_util.cuh"]
 FALLBACK_HBM_GBS = 6650.0
 
@@ -47,8 +49,8 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-baselines", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
-    p.add_argument("--cpu-heads", type=int, default=1024)
-    p.add_argument("--ref-heads", type=int, default=256)
+    p.add_argument("--cpu-heads", type=int, default=8192)
+    p.add_argument("--ref-heads", type=int, default=2048)
     return p.parse_args()
 
 
@@ -109,6 +111,31 @@ def kernel_sha() -> str:
         with open(os.path.join(ROOT, p), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
+
+
+# ---------------------------------------------------------------------------------------------
+# Sharding over ranks: every (sequence, head) is independent, so rank r runs its own sequences
+# (the workload's recipe under its own seed) and nothing crosses ranks but the timing
+# ---------------------------------------------------------------------------------------------
+def shard_workload(wl, rank: int):
+    return wl.with_(seed=wl.seed + 7919 * rank)
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time (all ranks take this collective in the same order)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, world: int, max_ms: float) -> float:
+    """Units all ranks processed per second of the slowest rank's time."""
+    return units_per_rank * world / (max_ms / 1e3)
 
 
 # ---------------------------------------------------------------------------------------------
@@ -275,7 +302,7 @@ def main():
     wl0 = WORKLOADS[args.workload]
     if args.batch:
         wl0 = wl0.with_(B=args.batch)
-    wl = wl0.with_(seed=wl0.seed + 7919 * rank)   # disjoint sequences per rank
+    wl = shard_workload(wl0, rank)
     cfg = gdn.make_config(wl.B, wl.H, wl.D, wl.W, wl.r, wl.gate, wl.fmt, wl.act, wl.buf)
 
     # ---- inputs resident in HBM: decode tokens and the fp32 warm-up states ------------------
@@ -323,16 +350,12 @@ def main():
     total_ms = evs[0][0].elapsed_time(evs[-1][2])
     decode_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
     quant_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     status = int(state.status[0].item())
     if status != 0:
         raise RuntimeError(f"device status word {status:#x} after the timed region")
 
-    head_steps = wl.heads * wl.T * args.steps * world
-    value = head_steps / (total_ms / 1e3)
+    value = whole_job_rate(wl.heads * wl.T * args.steps, world, total_ms)
     launches = args.steps * wl.T
     avg_launch_s = decode_ms / 1e3 / launches
     alg_bytes = avg_step_bytes(wl) * wl.heads
@@ -428,13 +451,10 @@ def e2e(args, wl, cfg, inp, S0, state, world, dev):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, world, dev)
     h2d = hS0.numel() * 4 + sum(t.numel() * t.element_size() for t in host.values())
     d2h = ho.numel() * ho.element_size()
-    return {"value": wl.heads * wl.T * n * world / (ms / 1e3), "unit": UNIT,
+    return {"value": whole_job_rate(wl.heads * wl.T * n, world, ms), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
             "api": "gdn_decode_window_steps_host (pinned host buffers, copies pipelined)"}
 

@@ -91,6 +91,11 @@ __device__ __forceinline__ void csync() {
   asm volatile("bar.sync 1, %0;\n" ::"n"(kComputeThreads) : "memory");
 }
 
+// Barrier of warps 0-3 only (named barrier 2), for work split between two warp groups.
+__device__ __forceinline__ void xsync() {
+  asm volatile("bar.sync 2, %0;\n" ::"n"(kComputeThreads / 2) : "memory");
+}
+
 // csync() that also returns whether any computing thread passed a nonzero `pred`.
 __device__ __forceinline__ int csync_or(int pred) {
   int out;

@@ -753,10 +753,16 @@ __global__ void __launch_bounds__(kStepThreads, 2)
   if (tid == 0)
     for (int s = 0; s < nstages && s < nh; ++s)
       stage_issue<C>(a, L, sm + L.stage0 + s * L.stage_bytes, &bars[s], h0 + s, hpos[s], true);
+  if (!stage_wait(a, &bars[0], 0u)) return;
   for (int n = 0; n < nh; ++n) {
-    const int s = n % nstages;
-    uint8_t* st = sm + L.stage0 + s * L.stage_bytes;
-    if (!stage_wait(a, &bars[s], (uint32_t)(n / nstages) & 1u)) return;
+    // refill the stage head n - 1 left (thread 128 leads the warp group with slack at the start
+    // of a head: the pair coefficients are shorter than the gates + frozen-state products)
+    if (nstages > 1 && tid == kStepThreads / 2 && n > 0 && n - 1 + nstages < nh) {
+      const int sp = (n - 1) % nstages;
+      stage_issue<C>(a, L, sm + L.stage0 + sp * L.stage_bytes, &bars[sp], h0 + n - 1 + nstages,
+                     hpos[n - 1 + nstages], true);
+    }
+    uint8_t* st = sm + L.stage0 + (n % nstages) * L.stage_bytes;
     const int P = hpos[n];
     if (P >= 0 && P < a.W) {
       step_head<C>(a, L, sm, st, h0 + n, P, C::DIAG ? 0.f : hg[n], hb[n]);
@@ -765,9 +771,20 @@ __global__ void __launch_bounds__(kStepThreads, 2)
     }
     // the stage's generic-proxy writes are ordered before the async copies that refill it
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-    csync();  // the stage and the per-head scratch are free again
-    if (tid == 0 && n + nstages < nh)
-      stage_issue<C>(a, L, st, &bars[s], h0 + n + nstages, hpos[n + nstages], true);
+    if (nstages == 1) {  // a single stage is refilled only once this head is done with it
+      csync();
+      if (tid == kStepThreads / 2 && n + 1 < nh)
+        stage_issue<C>(a, L, st, &bars[0], h0 + n + 1, hpos[n + 1], true);
+    }
+    // one barrier ends the head (stage and scratch free) and agrees on the next head's copies
+    int timed_out = 0;
+    if (n + 1 < nh)
+      timed_out = mbar_wait_bounded(&bars[(n + 1) % nstages], (uint32_t)((n + 1) / nstages) & 1u)
+                      ? 0 : 1;
+    if (csync_or(timed_out)) {
+      if (tid == 0) report(a.status, GDN_DEVICE_WAIT_TIMEOUT);
+      return;
+    }
   }
 }
 

@@ -145,12 +145,11 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
   const int Pp = (P + 15) & ~15;
 
   float* vec = reinterpret_cast<float*>(sm + L.vec);
-  float *kt = vec, *qt = vec + D, *xs = vec + 2 * D, *ys = vec + 3 * D, *Lt = vec + 4 * D;
+  float* Lt = vec + 4 * D;     // the step's cumulative log-gate per column (the flush reads it)
   float* misc = vec + 7 * D;  // [0..3] k.q partials, [24] x block scale, [25] y block scale
   float* coef = reinterpret_cast<float*>(sm + L.coef);
   float *ca = coef, *cb = coef + (W + r);
   uint8_t* Bfrag = sm + L.tc;                                      // digits, fragment order
-  bf* Bk = reinterpret_cast<bf*>(sm + L.tc + 8 * 144);            // [8][136]
   bf* Bc = reinterpret_cast<bf*>(sm + L.tc + 8 * 144 + 8 * 136 * 2);  // [8][Wr + 8]
 
   const uint8_t* s_codes = st + L.codes;
@@ -168,88 +167,81 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
   float Ls = 0.f;
   if constexpr (!C::DIAG) Ls = (P > 0 ? s_bL[P - 1] : 0.f) + g_scalar;
 
-  // ---- gates, phase-1 digit columns, the step's key / log-gate appended ------------------
-  // Warps 0-3 take the key side x, warps 4-7 the query side y; warp w owns the 32 columns of
-  // chunk w % 4 (lane l: column 32 (w % 4) + l). Each vector gets one block exponent, found by
-  // every warp of its side from all 128 columns (no cross-warp step): X = rint(v 2^(22-e)),
-  // |X| <= 2^22, three signed 8-bit digits X = d1 2^16 + d2 2^8 + d3.
-  {
-    const bool isy = warp >= 4;
-    const int j = (warp & 3) * 32 + lane;
-    const bf* sv = isy ? s_q : s_k;
-    float m = 0.f, val = 0.f, lj = Ls;
+  // Warps 0-3 (group X) take the gates and the frozen-state products (phase 1) while warps 4-7
+  // (group Y) take the pair coefficients (phase 2); both meet before phase 3.
+  float* PR = vec;      // phase-1 results p = F x, r = F y by row
+  float* RR = vec + D;
+  if (warp < 4) {
+    // ---- gates, phase-1 digit columns, the step's key / log-gate appended ----------------
+    // Warp w owns chunk w (lane l: column j = 32 w + l) of both x and y. Each vector gets one
+    // block exponent, found by every warp from all 128 columns (no cross-warp step):
+    // X = rint(v 2^(22-e)), |X| <= 2^22, three signed 8-bit digits X = d1 2^16 + d2 2^8 + d3.
+    const int j = 32 * warp + lane;
+    float mx = 0.f, my = 0.f, vx = 0.f, vy = 0.f, lj = Ls;
 #pragma unroll
     for (int mm = 0; mm < 4; ++mm) {
       const int jj = lane + 32 * mm;
-      float l;
-      if constexpr (C::DIAG) l = (P > 0 ? s_bL[(P - 1) * D + jj] : 0.f) + s_g[jj];
-      else l = Ls;
-      const float v = C::DIAG ? fast_exp(l) * __bfloat162float(sv[jj]) : __bfloat162float(sv[jj]);
-      m = fmaxf(m, fabsf(v));
-      if (mm == (warp & 3)) {  // this lane's own column j
-        val = v;
+      float l = Ls, e = 1.f;
+      if constexpr (C::DIAG) {
+        l = (P > 0 ? s_bL[(P - 1) * D + jj] : 0.f) + s_g[jj];
+        e = fast_exp(l);
+      }
+      const float xv = e * __bfloat162float(s_k[jj]), yv = e * __bfloat162float(s_q[jj]);
+      mx = fmaxf(mx, fabsf(xv));
+      my = fmaxf(my, fabsf(yv));
+      if (mm == warp) {  // this lane's own column j
+        vx = xv;
+        vy = yv;
         lj = l;
       }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     const float kj = __bfloat162float(s_k[j]), qj = __bfloat162float(s_q[j]);
-    const float e = C::DIAG ? fast_exp(lj) : fast_exp(Ls);
-    if (!isy) {
-      kt[j] = kj;
-      Lt[j] = lj;
-      xs[j] = e * kj;
-      Bk[j] = s_k[j];
-      float kq = kj * qj;
+    float kq = kj * qj;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
-      if (lane == 0) misc[warp] = kq;
-      if (!flush) {
-        static_cast<bf*>(a.buf_k)[(size_t)head * W * D + swz_el<bf, D>(P, j)] = s_k[j];
-        if constexpr (C::DIAG) a.buf_L[((size_t)head * W + P) * D + j] = lj;
-      } else {
-        s_bk[swz_el<bf, D>(P, j)] = s_k[j];
-        if constexpr (C::DIAG) s_bL[P * D + j] = lj;
-      }
+    for (int off = 16; off > 0; off >>= 1) {
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      my = fmaxf(my, __shfl_xor_sync(0xffffffffu, my, off));
+      kq += __shfl_xor_sync(0xffffffffu, kq, off);
+    }
+    if (lane == 0) misc[warp] = kq;
+    Lt[j] = lj;
+    if (!flush) {
+      static_cast<bf*>(a.buf_k)[(size_t)head * W * D + swz_el<bf, D>(P, j)] = s_k[j];
+      if constexpr (C::DIAG) a.buf_L[((size_t)head * W + P) * D + j] = lj;
     } else {
-      qt[j] = qj;
-      ys[j] = e * qj;
-      Bk[136 + j] = s_q[j];
+      s_bk[swz_el<bf, D>(P, j)] = s_k[j];
+      if constexpr (C::DIAG) s_bL[P * D + j] = lj;
     }
-    float mul = 0.f, scale = 0.f;
-    if (m >= 0x1p-100f) {  // smaller vectors contribute nothing measurable
-      // m = f 2^e2 with 0.5 <= f < 1 (m is normal); powers of two from exponent bits
-      const int e2 = ((__float_as_int(m) >> 23) & 0xFF) - 126;
-      mul = __int_as_float((22 - e2 + 127) << 23);
-      scale = __int_as_float((e2 - 22 + 127) << 23);
-    }
-    const int X = __float2int_rn(val * mul);
-    const int d3 = (int)(int8_t)(X & 0xFF);
-    const int X1 = (X - d3) >> 8;  // exact: X - d3 is a multiple of 256
-    const int d2 = (int)(int8_t)(X1 & 0xFF);
-    const int d1 = (X1 - d2) >> 8;
-    const int n0 = isy ? 3 : 0, k = digit_pos<C::INT4>(j);
-    Bfrag[digit_off(n0 + 0, k)] = (uint8_t)d1;
-    Bfrag[digit_off(n0 + 1, k)] = (uint8_t)d2;
-    Bfrag[digit_off(n0 + 2, k)] = (uint8_t)d3;
-    if (lane == 0 && (warp & 3) == 0) misc[24 + (isy ? 1 : 0)] = scale;
-    if (tid == 0) {
-      if constexpr (!C::DIAG) {
+    if constexpr (!C::DIAG) {
+      if (tid == 0) {
         if (!flush) a.buf_L[(size_t)head * Wp + P] = Ls;
         else s_bL[P] = Ls;
       }
     }
-    // padding of the phase-3 product to a multiple of 16 pairs: zero rows of U and zero
-    // coefficients (the product must not see stale or non-finite shared memory)
-    for (int e2 = tid; e2 < (Pp - P) * D; e2 += C::NT) s_bu[P * D + e2] = __float2bfloat16_rn(0.f);
-    for (int e2 = tid; e2 < 6 * (Pp - P); e2 += C::NT)
-      Bc[(e2 / (Pp - P)) * bcs + P + e2 % (Pp - P)] = __float2bfloat16_rn(0.f);
-  }
-  csync();
+    const int k = digit_pos<C::INT4>(j);
+#pragma unroll
+    for (int side = 0; side < 2; ++side) {
+      const float m = side ? my : mx, val = side ? vy : vx;
+      float mul = 0.f, scale = 0.f;
+      if (m >= 0x1p-100f) {  // smaller vectors contribute nothing measurable
+        // m = f 2^e2 with 0.5 <= f < 1 (m is normal); powers of two from exponent bits
+        const int e2 = ((__float_as_int(m) >> 23) & 0xFF) - 126;
+        mul = __int_as_float((22 - e2 + 127) << 23);
+        scale = __int_as_float((e2 - 22 + 127) << 23);
+      }
+      const int X = __float2int_rn(val * mul);
+      const int d3 = (int)(int8_t)(X & 0xFF);
+      const int X1 = (X - d3) >> 8;  // exact: X - d3 is a multiple of 256
+      const int d2 = (int)(int8_t)(X1 & 0xFF);
+      const int d1 = (X1 - d2) >> 8;
+      Bfrag[digit_off(3 * side + 0, k)] = (uint8_t)d1;
+      Bfrag[digit_off(3 * side + 1, k)] = (uint8_t)d2;
+      Bfrag[digit_off(3 * side + 2, k)] = (uint8_t)d3;
+      if (tid == 0) misc[24 + side] = scale;
+    }
+    xsync();
 
-  // ---- phase 1: p = F x, r = F y for rows 16w + gid (+8) ----------------------------------
-  float pr[2], rr[2];
-  {
+    // ---- phase 1: p = F x, r = F y for rows 32w + 16mt + gid (+8) --------------------------
     // digit weights of this lane's columns 2q4, 2q4+1: x = columns 0..2, y = columns 3..5
     const float wx0 = q4 == 0 ? 65536.f : (q4 == 1 ? 1.f : 0.f);
     const float wx1 = q4 == 0 ? 256.f : 0.f;
@@ -259,128 +251,149 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
     const uint4 bw1 = *reinterpret_cast<const uint4*>(Bfrag + (gid * 4 + q4) * 32 + 16);
     const uint32_t bw[8] = {bw0.x, bw0.y, bw0.z, bw0.w, bw1.x, bw1.y, bw1.z, bw1.w};
     const uint32_t cb0 = smem_u32(s_codes);
-    float PX[2], PY[2];
-    if constexpr (C::INT4) {
-      PX[0] = PX[1] = PY[0] = PY[1] = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {  // each 32-column chunk is one scale group
-        uint32_t A[4], w0, w1;
-        ldsm_x2(cb0 + swz<64>(16 * warp + r8 + 8 * (mi & 1), 16 * c), w0, w1);
-        i4x8_to_s8x16(w0, A[0], A[2]);
-        i4x8_to_s8x16(w1, A[1], A[3]);
-        int Cc[4] = {0, 0, 0, 0};
-        mma_s8(Cc, A, bw[2 * c], bw[2 * c + 1]);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float sg = s_scales[(16 * warp + gid + 8 * h) * C::NG + c];
-          const float c0 = (float)Cc[2 * h], c1 = (float)Cc[2 * h + 1];
-          PX[h] = fmaf(sg, wx0 * c0 + wx1 * c1, PX[h]);
-          PY[h] = fmaf(sg, wy0 * c0 + wy1 * c1, PY[h]);
-        }
-      }
-    } else {
-      int Cc[4] = {0, 0, 0, 0};  // one exponent per vector: chunks accumulate exactly in int32
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t A[4];
-        ldsm_x4(cb0 + swz<128>(16 * warp + r8 + 8 * (mi & 1), 32 * c + 16 * (mi >> 1)), A);
-        mma_s8(Cc, A, bw[2 * c], bw[2 * c + 1]);
-      }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float c0 = (float)Cc[2 * h], c1 = (float)Cc[2 * h + 1];
-        PX[h] = wx0 * c0 + wx1 * c1;
-        PY[h] = wy0 * c0 + wy1 * c1;
-      }
-    }
     const float gam = C::DIAG ? 1.f : fast_exp(Ls);
     const float sx = misc[24] * gam * (C::INT4 ? 0.0625f : 1.f);  // int4 codes entered as 16 c
     const float sy = misc[25] * gam * (C::INT4 ? 0.0625f : 1.f);
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      PX[h] += __shfl_xor_sync(0xffffffffu, PX[h], 1);
-      PX[h] += __shfl_xor_sync(0xffffffffu, PX[h], 2);
-      PY[h] += __shfl_xor_sync(0xffffffffu, PY[h], 1);
-      PY[h] += __shfl_xor_sync(0xffffffffu, PY[h], 2);
-      const float srow = C::INT4 ? 1.f : s_scales[16 * warp + gid + 8 * h];
-      pr[h] = PX[h] * sx * srow;
-      rr[h] = PY[h] * sy * srow;
-    }
-  }
-
-  // ---- phase 2: pair coefficients, written as the split phase-3 right-hand side --------
-  if constexpr (!C::DIAG) {
-    const int tiles = Pp >> 4;
-    for (int tile = warp; tile < tiles; tile += 8) {
-      float Ce[4] = {0.f, 0.f, 0.f, 0.f}, Co[4] = {0.f, 0.f, 0.f, 0.f};  // even / odd k-steps
-      const uint32_t kb = smem_u32(s_bk);
+    for (int mt = 0; mt < 2; ++mt) {
+      const int row0 = 32 * warp + 16 * mt;
+      float PX[2], PY[2];
+      if constexpr (C::INT4) {
+        PX[0] = PX[1] = PY[0] = PY[1] = 0.f;
 #pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        uint32_t A[4];
-        ldsm_x4(kb + swz<256>(16 * tile + r8 + 8 * (mi & 1), 2 * (16 * s + 8 * (mi >> 1))), A);
-        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(Bk + gid * 136 + 16 * s + 2 * q4);
-        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(Bk + gid * 136 + 16 * s + 8 + 2 * q4);
-        if (s & 1) mma_bf16(Co, A, b0, b1);
-        else mma_bf16(Ce, A, b0, b1);
-      }
-      // the quad leader holds (a, b) of rows gid and gid+8; lane q4 splits one of the four
-      const int ld = lane & ~3;
-      const float a0 = __shfl_sync(0xffffffffu, Ce[0] + Co[0], ld);
-      const float b0 = __shfl_sync(0xffffffffu, Ce[1] + Co[1], ld);
-      const float a1 = __shfl_sync(0xffffffffu, Ce[2] + Co[2], ld);
-      const float b1 = __shfl_sync(0xffffffffu, Ce[3] + Co[3], ld);
-      const float vq = q4 == 0 ? a0 : (q4 == 1 ? b0 : (q4 == 2 ? a1 : b1));
-      const int i = 16 * tile + gid + 8 * (q4 >> 1);
-      if (i < P) {
-        float h, m, l;
-        split3(vq * fast_exp(Ls - s_bL[i]), h, m, l);
-        const int row = (q4 & 1) ? 3 : 0;
-        Bc[(row + 0) * bcs + i] = __float2bfloat16_rn(h);
-        Bc[(row + 1) * bcs + i] = __float2bfloat16_rn(m);
-        Bc[(row + 2) * bcs + i] = __float2bfloat16_rn(l);
-      }
-    }
-  } else {
-    // per-element decay e^{L_t[j] - L_i[j]}: FMA, 8 threads per pair; thread c takes columns
-    // 8c..8c+7 and 64+8c..64+8c+7 (distinct banks across the 8 threads of a pair)
-    const int c = tid & 7;
-    float kr[16], qr[16], lr[16];
+        for (int c = 0; c < 4; ++c) {  // each 32-column chunk is one scale group
+          uint32_t A[4], w0, w1;
+          ldsm_x2(cb0 + swz<64>(row0 + r8 + 8 * (mi & 1), 16 * c), w0, w1);
+          i4x8_to_s8x16(w0, A[0], A[2]);
+          i4x8_to_s8x16(w1, A[1], A[3]);
+          int Cc[4] = {0, 0, 0, 0};
+          mma_s8(Cc, A, bw[2 * c], bw[2 * c + 1]);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const int j = (e < 8 ? 8 * c : 64 + 8 * c) + (e & 7);
-      kr[e] = kt[j];
-      qr[e] = qt[j];
-      lr[e] = Lt[j];
-    }
-    const int npass = (P + 31) >> 5;
-    for (int ps = 0; ps < npass; ++ps) {
-      const int i = ps * 32 + (tid >> 3);
-      float pa = 0.f, pb = 0.f;
-      if (i < P) {
-        float kk[16], ll[16];
-        load_sw<bf, D, 8>(s_bk, i, 8 * c, kk);
-        load_sw<bf, D, 8>(s_bk, i, 64 + 8 * c, kk + 8);
-        Num<float>::load<8>(s_bL + i * D + 8 * c, ll);
-        Num<float>::load<8>(s_bL + i * D + 64 + 8 * c, ll + 8);
+          for (int h = 0; h < 2; ++h) {
+            const float sg = s_scales[(row0 + gid + 8 * h) * C::NG + c];
+            const float c0 = (float)Cc[2 * h], c1 = (float)Cc[2 * h + 1];
+            PX[h] = fmaf(sg, wx0 * c0 + wx1 * c1, PX[h]);
+            PY[h] = fmaf(sg, wy0 * c0 + wy1 * c1, PY[h]);
+          }
+        }
+      } else {
+        int Cc[4] = {0, 0, 0, 0};  // one exponent per vector: chunks accumulate exactly in int32
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float k2 = kk[e] * fast_exp(lr[e] - ll[e]);
-          pa = fmaf(k2, kr[e], pa);
-          pb = fmaf(k2, qr[e], pb);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t A[4];
+          ldsm_x4(cb0 + swz<128>(row0 + r8 + 8 * (mi & 1), 32 * c + 16 * (mi >> 1)), A);
+          mma_s8(Cc, A, bw[2 * c], bw[2 * c + 1]);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float c0 = (float)Cc[2 * h], c1 = (float)Cc[2 * h + 1];
+          PX[h] = wx0 * c0 + wx1 * c1;
+          PY[h] = wy0 * c0 + wy1 * c1;
         }
       }
 #pragma unroll
-      for (int off = 4; off > 0; off >>= 1) {
-        pa += __shfl_xor_sync(0xffffffffu, pa, off);
-        pb += __shfl_xor_sync(0xffffffffu, pb, off);
+      for (int h = 0; h < 2; ++h) {
+        PX[h] += __shfl_xor_sync(0xffffffffu, PX[h], 1);
+        PX[h] += __shfl_xor_sync(0xffffffffu, PX[h], 2);
+        PY[h] += __shfl_xor_sync(0xffffffffu, PY[h], 1);
+        PY[h] += __shfl_xor_sync(0xffffffffu, PY[h], 2);
       }
-      if (c == 0 && i < P) put_coef(Bc, bcs, i, pa, pb);
+      if (q4 < 2) {  // lane q4 of the quad stores row row0 + gid + 8 q4
+        const int v = row0 + gid + 8 * q4;
+        const float srow = C::INT4 ? 1.f : s_scales[v];
+        PR[v] = (q4 ? PX[1] : PX[0]) * sx * srow;
+        RR[v] = (q4 ? PY[1] : PY[0]) * sy * srow;
+      }
     }
-  }
-  if (tid < r) {  // compensator pairs: key e_j entered at L = 0
-    const int j = s_cidx[tid] & (D - 1);
-    ca[W + tid] = xs[j];
-    cb[W + tid] = ys[j];
+  } else {
+    const int ty = tid - 128, wy = warp - 4;
+    // padding of the phase-3 product to a multiple of 16 pairs: zero rows of U and zero
+    // coefficients (the product must not see stale or non-finite shared memory)
+    for (int e2 = ty; e2 < (Pp - P) * D; e2 += 128) s_bu[P * D + e2] = __float2bfloat16_rn(0.f);
+    for (int e2 = ty; e2 < 6 * (Pp - P); e2 += 128)
+      Bc[(e2 / (Pp - P)) * bcs + P + e2 % (Pp - P)] = __float2bfloat16_rn(0.f);
+    if (ty < r) {  // compensator pairs: key e_j entered at L = 0, so their coefficient is x[j]
+      const int j = s_cidx[ty] & (D - 1);
+      float e;
+      if constexpr (C::DIAG) e = fast_exp((P > 0 ? s_bL[(P - 1) * D + j] : 0.f) + s_g[j]);
+      else e = fast_exp(Ls);
+      ca[W + ty] = e * __bfloat162float(s_k[j]);
+      cb[W + ty] = e * __bfloat162float(s_q[j]);
+    }
+
+    // ---- phase 2: pair coefficients, written as the split phase-3 right-hand side ------
+    if constexpr (!C::DIAG) {
+      const int tiles = Pp >> 4;
+      const bf* bsrc = gid == 0 ? s_k : s_q;  // right-hand side columns: 0 = k_t, 1 = q_t
+      for (int tile = wy; tile < tiles; tile += 4) {
+        float Ce[4] = {0.f, 0.f, 0.f, 0.f}, Co[4] = {0.f, 0.f, 0.f, 0.f};  // even / odd k-steps
+        const uint32_t kb = smem_u32(s_bk);
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          uint32_t A[4];
+          ldsm_x4(kb + swz<256>(16 * tile + r8 + 8 * (mi & 1), 2 * (16 * s + 8 * (mi >> 1))), A);
+          uint32_t b0 = 0u, b1 = 0u;
+          if (gid < 2) {
+            b0 = *reinterpret_cast<const uint32_t*>(bsrc + 16 * s + 2 * q4);
+            b1 = *reinterpret_cast<const uint32_t*>(bsrc + 16 * s + 8 + 2 * q4);
+          }
+          if (s & 1) mma_bf16(Co, A, b0, b1);
+          else mma_bf16(Ce, A, b0, b1);
+        }
+        // the quad leader holds (a, b) of rows gid and gid+8; lane q4 splits one of the four
+        const int ld = lane & ~3;
+        const float a0 = __shfl_sync(0xffffffffu, Ce[0] + Co[0], ld);
+        const float b0 = __shfl_sync(0xffffffffu, Ce[1] + Co[1], ld);
+        const float a1 = __shfl_sync(0xffffffffu, Ce[2] + Co[2], ld);
+        const float b1 = __shfl_sync(0xffffffffu, Ce[3] + Co[3], ld);
+        const float vq = q4 == 0 ? a0 : (q4 == 1 ? b0 : (q4 == 2 ? a1 : b1));
+        const int i = 16 * tile + gid + 8 * (q4 >> 1);
+        if (i < P) {
+          float h, m, l;
+          split3(vq * fast_exp(Ls - s_bL[i]), h, m, l);
+          const int row = (q4 & 1) ? 3 : 0;
+          Bc[(row + 0) * bcs + i] = __float2bfloat16_rn(h);
+          Bc[(row + 1) * bcs + i] = __float2bfloat16_rn(m);
+          Bc[(row + 2) * bcs + i] = __float2bfloat16_rn(l);
+        }
+      }
+    } else {
+      // per-element decay e^{L_t[j] - L_i[j]}: FMA, 8 threads per pair; thread c takes columns
+      // 8c..8c+7 and 64+8c..64+8c+7 (distinct banks across the 8 threads of a pair)
+      const int c = ty & 7;
+      float kr[16], qr[16], lr[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int j = (e < 8 ? 8 * c : 64 + 8 * c) + (e & 7);
+        kr[e] = __bfloat162float(s_k[j]);
+        qr[e] = __bfloat162float(s_q[j]);
+        lr[e] = (P > 0 ? s_bL[(P - 1) * D + j] : 0.f) + s_g[j];
+      }
+      const int npass = (P + 15) >> 4;
+      for (int ps = 0; ps < npass; ++ps) {
+        const int i = ps * 16 + (ty >> 3);
+        float pa = 0.f, pb = 0.f;
+        if (i < P) {
+          float kk[16], ll[16];
+          load_sw<bf, D, 8>(s_bk, i, 8 * c, kk);
+          load_sw<bf, D, 8>(s_bk, i, 64 + 8 * c, kk + 8);
+          Num<float>::load<8>(s_bL + i * D + 8 * c, ll);
+          Num<float>::load<8>(s_bL + i * D + 64 + 8 * c, ll + 8);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float k2 = kk[e] * fast_exp(lr[e] - ll[e]);
+            pa = fmaf(k2, kr[e], pa);
+            pb = fmaf(k2, qr[e], pb);
+          }
+        }
+#pragma unroll
+        for (int off = 4; off > 0; off >>= 1) {
+          pa += __shfl_xor_sync(0xffffffffu, pa, off);
+          pb += __shfl_xor_sync(0xffffffffu, pb, off);
+        }
+        if (c == 0 && i < P) put_coef(Bc, bcs, i, pa, pb);
+      }
+    }
   }
   csync();
 
@@ -410,8 +423,8 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
     }
     if (q4 < 2) {  // lane q4 of the quad finishes row 16w + gid + 8 q4
       const int v = 16 * warp + gid + 8 * q4;
-      float w = (q4 ? pr[1] : pr[0]) + (q4 ? Wv[1] : Wv[0]);
-      float rv = (q4 ? rr[1] : rr[0]) + (q4 ? Rv[1] : Rv[0]);
+      float w = PR[v] + (q4 ? Wv[1] : Wv[0]);
+      float rv = RR[v] + (q4 ? Rv[1] : Rv[0]);
       for (int c = 0; c < r; ++c) {
         const float cu = s_cu[c * D + v];
         w = fmaf(ca[W + c], cu, w);

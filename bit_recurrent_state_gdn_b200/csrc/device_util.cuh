@@ -123,6 +123,18 @@ __device__ __forceinline__ float fast_exp(float x) {
   return y;
 }
 
+// rint of the correctly rounded quotient x / s (|x / s| <= 128), given inv = the correctly
+// rounded 1 / s. q = x * inv differs from x / s by at most 2 rounding errors of size
+// 2^-24 * 128 = 2^-17, and the rounded quotient from x / s by one more, so q and the rounded
+// quotient lie on the same side of every half-integer unless q is within 2^-15 of one; only
+// there is the quotient formed by a correctly rounded division.
+__device__ __forceinline__ float rint_quotient(float x, float s, float inv) {
+  const float q = x * inv;
+  const float f = fabsf(q - truncf(q));
+  if (fabsf(f - 0.5f) < 0x1p-14f) return rintf(__fdiv_rn(x, s));
+  return rintf(q);
+}
+
 // ---- exact conversions -------------------------------------------------------------------
 // Four int8 codes (two's complement, byte e = code e) to fp32: bias each byte to b + 128,
 // place it in the mantissa of 2^23 (0x4B0000xx = 2^23 + xx) and subtract 2^23 + 128.

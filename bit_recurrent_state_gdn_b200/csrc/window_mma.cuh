@@ -449,6 +449,15 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
 // compensators, absmax and requantisation, from the accumulators. npairs = P + 1 pairs (the
 // step's pair included) sit in the stage; the gates end at L_W = Lt (per column) / Ls.
 // ------------------------------------------------------------------------------------------
+// 1 << k, hidden from the optimiser: a select over unrolled array elements keyed on it stays a
+// select and is not turned back into a run-time index (which would move the array to local
+// memory).
+__device__ __forceinline__ uint32_t one_hot_opaque(int k) {
+  uint32_t m = 1u << k;
+  asm volatile("" : "+r"(m));
+  return m;
+}
+
 template <class C>
 __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uint8_t* st, int head,
                           int P, float Ls) {
@@ -517,38 +526,39 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
   }
   csync();
 
-  // ---- the materialised state, one 64-column half (n-tiles 8hc..8hc+7) at a time -----------
-  // acc[n][0..3] = S_W at (v0, j), (v0, j+1), (v1, j), (v1, j+1), j = 64hc + 8n + 2q4
+  // ---- the materialised state, all 16 n-tiles of this warp's 16 rows, computed once -------
+  // acc[nt][0..3] = S_W at (v0, j), (v0, j+1), (v1, j), (v1, j+1), j = 8 nt + 2 q4
   const int v0 = 16 * warp + gid, v1 = v0 + 8;
-  const uint32_t ub = smem_u32(s_bu), kb = smem_u32(s_bk);
-  const uint32_t mb = smem_u32(pl_mid), lb = smem_u32(pl_lo);
-  auto tile_half = [&](int hc, float (&acc)[8][4]) {
+  float acc[16][4];
+  {
     const float s0 = C::INT4 ? 0.f : s_scales[v0], s1 = C::INT4 ? 0.f : s_scales[v1];
 #pragma unroll
-    for (int n = 0; n < 8; ++n) {
-      const int j = 64 * hc + 8 * n + 2 * q4;
+    for (int nt = 0; nt < 16; ++nt) {
+      const int j = 8 * nt + 2 * q4;
       float c00, c01, c10, c11, t0 = s0, t1 = s1;
       if constexpr (C::INT4) {
-        const uint8_t b0 = s_codes[swz<64>(v0, j / 2)], b1 = s_codes[swz<64>(v1, j / 2)];
-        c00 = (float)(((int)(b0 << 28)) >> 28);
-        c01 = (float)(((int)(b0 << 24)) >> 28);
-        c10 = (float)(((int)(b1 << 28)) >> 28);
-        c11 = (float)(((int)(b1 << 24)) >> 28);
+        // one byte = columns j (low nibble), j + 1 (high): bias to c + 8, 2^23 trick
+        const uint32_t b0 = s_codes[swz<64>(v0, j / 2)] ^ 0x88u;
+        const uint32_t b1 = s_codes[swz<64>(v1, j / 2)] ^ 0x88u;
+        c00 = __uint_as_float(0x4B000000u | (b0 & 0xFu)) - 8388616.f;
+        c01 = __uint_as_float(0x4B000000u | (b0 >> 4)) - 8388616.f;
+        c10 = __uint_as_float(0x4B000000u | (b1 & 0xFu)) - 8388616.f;
+        c11 = __uint_as_float(0x4B000000u | (b1 >> 4)) - 8388616.f;
         t0 = s_scales[v0 * C::NG + j / 32];
         t1 = s_scales[v1 * C::NG + j / 32];
       } else {
-        const uint16_t h0 = *reinterpret_cast<const uint16_t*>(s_codes + swz<128>(v0, j));
-        const uint16_t h1 = *reinterpret_cast<const uint16_t*>(s_codes + swz<128>(v1, j));
-        c00 = (float)(int8_t)(h0 & 0xFF);
-        c01 = (float)(int8_t)(h0 >> 8);
-        c10 = (float)(int8_t)(h1 & 0xFF);
-        c11 = (float)(int8_t)(h1 >> 8);
+        const uint32_t h0 = *reinterpret_cast<const uint16_t*>(s_codes + swz<128>(v0, j)) ^ 0x8080u;
+        const uint32_t h1 = *reinterpret_cast<const uint16_t*>(s_codes + swz<128>(v1, j)) ^ 0x8080u;
+        c00 = __uint_as_float(__byte_perm(h0, 0x4B000000u, 0x7650)) - 8388736.f;
+        c01 = __uint_as_float(__byte_perm(h0, 0x4B000000u, 0x7651)) - 8388736.f;
+        c10 = __uint_as_float(__byte_perm(h1, 0x4B000000u, 0x7650)) - 8388736.f;
+        c11 = __uint_as_float(__byte_perm(h1, 0x4B000000u, 0x7651)) - 8388736.f;
       }
       const float e0 = colexp[j], e1 = colexp[j + 1];
-      acc[n][0] = t0 * c00 * e0;
-      acc[n][1] = t0 * c01 * e1;
-      acc[n][2] = t1 * c10 * e0;
-      acc[n][3] = t1 * c11 * e1;
+      acc[nt][0] = t0 * c00 * e0;
+      acc[nt][1] = t0 * c01 * e1;
+      acc[nt][2] = t1 * c10 * e0;
+      acc[nt][3] = t1 * c11 * e1;
     }
     // compensator pairs (key e_jc at gate 0), added with selects so that no data-dependent
     // index reaches the accumulator array
@@ -558,16 +568,20 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
       const float ec = colexp[jc];
       const float u0 = mine ? s_cu[c * D + v0] * ec : 0.f;
       const float u1 = mine ? s_cu[c * D + v1] * ec : 0.f;
+      const uint32_t hit = one_hot_opaque(jc >> 3);
 #pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        const bool h = (jc >> 3) == 8 * hc + n;
-        acc[n][0] += (h && !odd) ? u0 : 0.f;
-        acc[n][1] += (h && odd) ? u0 : 0.f;
-        acc[n][2] += (h && !odd) ? u1 : 0.f;
-        acc[n][3] += (h && odd) ? u1 : 0.f;
+      for (int nt = 0; nt < 16; ++nt) {
+        const bool h = (hit >> nt) & 1u;
+        acc[nt][0] += (h && !odd) ? u0 : 0.f;
+        acc[nt][1] += (h && odd) ? u0 : 0.f;
+        acc[nt][2] += (h && !odd) ? u1 : 0.f;
+        acc[nt][3] += (h && odd) ? u1 : 0.f;
       }
     }
-    // rank-Kp update: U^T (v rows, pair k) times Kt (pair k, column j)
+    // rank-Kp update U^T (v rows, pair k) times Kt (pair k, column j); the split left-hand
+    // side of a k-step serves all 16 n-tiles
+    const uint32_t ub = smem_u32(s_bu), kb = smem_u32(s_bk);
+    const uint32_t mb = smem_u32(pl_mid), lb = smem_u32(pl_lo);
     for (int s = 0; s < Kp / 16; ++s) {
       uint32_t A[4];
       ldsm_x4_t(ub + swz<256>(16 * s + r8 + 8 * (mi >> 1), 2 * (16 * warp + 8 * (mi & 1))), A);
@@ -581,9 +595,8 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
         split3_pair(A[3], f2, f3, Ah[3], Am[3], Al[3]);
       }
 #pragma unroll
-      for (int n2 = 0; n2 < 4; ++n2) {
-        const int col = 64 * hc + 16 * n2 + 8 * (mi >> 1);
-        const uint32_t off = swz<256>(16 * s + r8 + 8 * (mi & 1), 2 * col);
+      for (int n2 = 0; n2 < 8; ++n2) {
+        const uint32_t off = swz<256>(16 * s + r8 + 8 * (mi & 1), 2 * (16 * n2 + 8 * (mi >> 1)));
         uint32_t B[4];
         ldsm_x4_t(kb + off, B);
         if constexpr (!C::DIAG) {
@@ -605,53 +618,23 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
         }
       }
     }
-  };
-  // zeroes the picked compensator columns of a half; with `store` also writes them to comp_u
-  auto take_comps = [&](int hc, float (&acc)[8][4], bool store) {
-    float* g_cu = a.comp_u + (size_t)head * r * D;
-    for (int c = 0; c < r; ++c) {
-      const int jc = sel[c];
-      const bool mine = ((jc & 7) >> 1) == q4, odd = jc & 1;
-      float x0 = 0.f, x1 = 0.f;
-      bool here = false;
-#pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        const bool h = mine && (jc >> 3) == 8 * hc + n;
-        const bool he = h && !odd, ho = h && odd;
-        here = here || h;
-        x0 = he ? acc[n][0] : (ho ? acc[n][1] : x0);
-        x1 = he ? acc[n][2] : (ho ? acc[n][3] : x1);
-        acc[n][0] = he ? 0.f : acc[n][0];
-        acc[n][1] = ho ? 0.f : acc[n][1];
-        acc[n][2] = he ? 0.f : acc[n][2];
-        acc[n][3] = ho ? 0.f : acc[n][3];
-      }
-      if (store && here) {
-        g_cu[c * D + v0] = x0;
-        g_cu[c * D + v1] = x1;
-      }
-    }
-  };
+  }
 
-  // ---- pass 1 (compensators only): column max-abs, pick the top r (ties: lower index) ----
+  // ---- compensators: column max-abs, the top r (ties: lower index), taken out exactly -----
   if (r > 0) {
-    for (int hc = 0; hc < 2; ++hc) {
-      float acc[8][4];
-      tile_half(hc, acc);
 #pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        float m0 = fmaxf(fabsf(acc[n][0]), fabsf(acc[n][2]));
-        float m1 = fmaxf(fabsf(acc[n][1]), fabsf(acc[n][3]));
+    for (int nt = 0; nt < 16; ++nt) {
+      float m0 = fmaxf(fabsf(acc[nt][0]), fabsf(acc[nt][2]));
+      float m1 = fmaxf(fabsf(acc[nt][1]), fabsf(acc[nt][3]));
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-          m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, off));
-          m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, off));
-        }
-        if (gid == 0) {
-          unsigned int* cm = reinterpret_cast<unsigned int*>(colmax) + 64 * hc + 8 * n + 2 * q4;
-          atomicMax(cm, __float_as_uint(m0));
-          atomicMax(cm + 1, __float_as_uint(m1));
-        }
+      for (int off = 4; off < 32; off <<= 1) {
+        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, off));
+        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, off));
+      }
+      if (gid == 0) {
+        unsigned int* cm = reinterpret_cast<unsigned int*>(colmax) + 8 * nt + 2 * q4;
+        atomicMax(cm, __float_as_uint(m0));
+        atomicMax(cm + 1, __float_as_uint(m1));
       }
     }
     csync();
@@ -678,84 +661,68 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
     }
     csync();
     if (tid < r) a.comp_idx[(size_t)head * ((r + 3) & ~3) + tid] = sel[tid];
+    float* g_cu = a.comp_u + (size_t)head * r * D;
+    for (int c = 0; c < r; ++c) {
+      const int jc = sel[c];
+      const bool mine = ((jc & 7) >> 1) == q4, odd = jc & 1;
+      float x0 = 0.f, x1 = 0.f;
+      bool here = false;
+      const uint32_t hit = mine ? one_hot_opaque(jc >> 3) : 0u;
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt) {
+        const bool h = (hit >> nt) & 1u;
+        const bool he = h && !odd, ho = h && odd;
+        here = here || h;
+        x0 = he ? acc[nt][0] : (ho ? acc[nt][1] : x0);
+        x1 = he ? acc[nt][2] : (ho ? acc[nt][3] : x1);
+        acc[nt][0] = he ? 0.f : acc[nt][0];
+        acc[nt][1] = ho ? 0.f : acc[nt][1];
+        acc[nt][2] = he ? 0.f : acc[nt][2];
+        acc[nt][3] = ho ? 0.f : acc[nt][3];
+      }
+      if (here) {
+        g_cu[c * D + v0] = x0;
+        g_cu[c * D + v1] = x1;
+      }
+    }
   }
 
-  // ---- pass 2 (int8 row scales span both halves): row max-abs without the picked columns ----
+  // ---- scales and codes into this warp's rows of the stage's code tile ---------------------
+  // (the warp read its old code rows above and no other warp reads them)
   float* g_scales = a.scales + (size_t)head * C::NSCALES;
-  float rs[2] = {0.f, 0.f};
-  if constexpr (!C::INT4) {
-    float m[2] = {0.f, 0.f};
-    for (int hc = 0; hc < 2; ++hc) {
-      float acc[8][4];
-      tile_half(hc, acc);
-      take_comps(hc, acc, true);
+  __syncwarp();
 #pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        m[0] = fmaxf(m[0], fmaxf(fabsf(acc[n][0]), fabsf(acc[n][1])));
-        m[1] = fmaxf(m[1], fmaxf(fabsf(acc[n][2]), fabsf(acc[n][3])));
-      }
-    }
+  for (int h = 0; h < 2; ++h) {
+    const int v = h ? v1 : v0;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      m[h] = fmaxf(m[h], __shfl_xor_sync(0xffffffffu, m[h], 1));
-      m[h] = fmaxf(m[h], __shfl_xor_sync(0xffffffffu, m[h], 2));
-      rs[h] = __fdiv_rn(m[h], (float)QMAX);
-    }
-    if (q4 == 0) {
-      g_scales[v0] = rs[0];
-      g_scales[v1] = rs[1];
-    }
-  }
-
-  // ---- last pass: requantise into this warp's rows of the stage's code tile ---------------
-  for (int hc = 0; hc < 2; ++hc) {
-    float acc[8][4];
-    tile_half(hc, acc);
-    take_comps(hc, acc, C::INT4);
+    for (int gq = 0; gq < (C::INT4 ? 4 : 1); ++gq) {  // int4: groups of 4 n-tiles
+      constexpr int NPG = C::INT4 ? 4 : 16;
+      float m = 0.f;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int v = h ? v1 : v0;
-      if constexpr (C::INT4) {
+      for (int nt = NPG * gq; nt < NPG * gq + NPG; ++nt)
+        m = fmaxf(m, fmaxf(fabsf(acc[nt][2 * h]), fabsf(acc[nt][2 * h + 1])));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      const float sc = __fdiv_rn(m, (float)QMAX);
+      const float inv = sc > 0.f ? __frcp_rn(sc) : 0.f;
+      if (q4 == 0) g_scales[v * C::NG + gq] = sc;
 #pragma unroll
-        for (int gq = 0; gq < 2; ++gq) {  // the two 32-column groups of this half
-          float m = 0.f;
+      for (int nt = NPG * gq; nt < NPG * gq + NPG; ++nt) {
+        int qv[2];
 #pragma unroll
-          for (int n = 4 * gq; n < 4 * gq + 4; ++n)
-            m = fmaxf(m, fmaxf(fabsf(acc[n][2 * h]), fabsf(acc[n][2 * h + 1])));
-          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-          const float sc = __fdiv_rn(m, (float)QMAX);
-          if (q4 == 0) g_scales[v * C::NG + 2 * hc + gq] = sc;
-#pragma unroll
-          for (int n = 4 * gq; n < 4 * gq + 4; ++n) {
-            int qv[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const float t = sc > 0.f ? rintf(__fdiv_rn(acc[n][2 * h + e], sc)) : 0.f;
-              qv[e] = (int)fminf(fmaxf(t, (float)-QMAX), (float)QMAX);
-            }
-            s_codes[swz<64>(v, 32 * hc + 4 * n + q4)] =
-                (uint8_t)((qv[0] & 0xF) | ((qv[1] & 0xF) << 4));
-          }
+        for (int e = 0; e < 2; ++e) {
+          const float t = sc > 0.f ? rint_quotient(acc[nt][2 * h + e], sc, inv) : 0.f;
+          qv[e] = (int)fminf(fmaxf(t, (float)-QMAX), (float)QMAX);
         }
-      } else {
-        const float sc = rs[h];
-#pragma unroll
-        for (int n = 0; n < 8; ++n) {
-          int qv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float t = sc > 0.f ? rintf(__fdiv_rn(acc[n][2 * h + e], sc)) : 0.f;
-            qv[e] = (int)fminf(fmaxf(t, (float)-QMAX), (float)QMAX);
-          }
-          *reinterpret_cast<uint16_t*>(s_codes + swz<128>(v, 64 * hc + 8 * n + 2 * q4)) =
+        if constexpr (C::INT4)
+          s_codes[swz<64>(v, 4 * nt + q4)] = (uint8_t)((qv[0] & 0xF) | ((qv[1] & 0xF) << 4));
+        else
+          *reinterpret_cast<uint16_t*>(s_codes + swz<128>(v, 8 * nt + 2 * q4)) =
               (uint16_t)((qv[0] & 0xFF) | ((qv[1] & 0xFF) << 8));
-        }
       }
     }
-    // the next half re-reads old codes of these rows (other columns): keep this warp in step
-    __syncwarp();
   }
+  __syncwarp();
   // ---- this warp's 16 code rows to HBM, 16 bytes per lane per store -----------------------
   {
     constexpr int RB = C::ROW_BYTES, CH = 16 * RB / 16;  // 16-byte chunks of the warp's rows

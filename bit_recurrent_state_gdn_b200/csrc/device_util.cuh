@@ -96,6 +96,11 @@ __device__ __forceinline__ void xsync() {
   asm volatile("bar.sync 2, %0;\n" ::"n"(kComputeThreads / 2) : "memory");
 }
 
+// Barrier of warps 4-7 only (named barrier 3).
+__device__ __forceinline__ void ysync() {
+  asm volatile("bar.sync 3, %0;\n" ::"n"(kComputeThreads / 2) : "memory");
+}
+
 // csync() that also returns whether any computing thread passed a nonzero `pred`.
 __device__ __forceinline__ int csync_or(int pred) {
   int out;

@@ -168,9 +168,12 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
   if constexpr (!C::DIAG) Ls = (P > 0 ? s_bL[P - 1] : 0.f) + g_scalar;
 
   // Warps 0-3 (group X) take the gates and the frozen-state products (phase 1) while warps 4-7
-  // (group Y) take the pair coefficients (phase 2); both meet before phase 3.
+  // (group Y) take the pair coefficients (phase 2) and the buffer products (phase 3); both meet
+  // before the per-row finish (phase 4).
   float* PR = vec;      // phase-1 results p = F x, r = F y by row
   float* RR = vec + D;
+  float* WV = vec + 5 * D;  // phase-3 results U^T a, U^T b by row
+  float* RV = vec + 6 * D;
   if (warp < 4) {
     // ---- gates, phase-1 digit columns, the step's key / log-gate appended ----------------
     // Warp w owns chunk w (lane l: column j = 32 w + l) of both x and y. Each vector gets one
@@ -394,49 +397,60 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
         if (c == 0 && i < P) put_coef(Bc, bcs, i, pa, pb);
       }
     }
-  }
-  csync();
+    ysync();
 
-  // ---- phase 3: w = p + U^T a (+ compensators), r likewise; then u_t, o_t -----------------
-  {
-    float Cc[4] = {0.f, 0.f, 0.f, 0.f};
+    // ---- phase 3: U^T (a, b) for rows 32 wy + 16 mt + gid (+8) ----------------------------
+    float C0[4] = {0.f, 0.f, 0.f, 0.f}, C1[4] = {0.f, 0.f, 0.f, 0.f};
     const uint32_t ub = smem_u32(s_bu);
     for (int s = 0; s < Pp / 16; ++s) {
-      uint32_t A[4];
-      ldsm_x4_t(ub + swz<256>(16 * s + r8 + 8 * (mi >> 1), 2 * (16 * warp + 8 * (mi & 1))), A);
+      uint32_t A0[4], A1[4];
+      ldsm_x4_t(ub + swz<256>(16 * s + r8 + 8 * (mi >> 1), 2 * (32 * wy + 8 * (mi & 1))), A0);
+      ldsm_x4_t(ub + swz<256>(16 * s + r8 + 8 * (mi >> 1), 2 * (32 * wy + 16 + 8 * (mi & 1))), A1);
       const uint32_t b0 = *reinterpret_cast<const uint32_t*>(Bc + gid * bcs + 16 * s + 2 * q4);
       const uint32_t b1 = *reinterpret_cast<const uint32_t*>(Bc + gid * bcs + 16 * s + 8 + 2 * q4);
-      mma_bf16(Cc, A, b0, b1);
+      mma_bf16(C0, A0, b0, b1);
+      mma_bf16(C1, A1, b0, b1);
     }
     // columns 0..2 belong to w, 3..5 to r
     const float wx0 = q4 <= 1 ? 1.f : 0.f, wx1 = q4 == 0 ? 1.f : 0.f;
     const float wy0 = q4 == 2 ? 1.f : 0.f, wy1 = (q4 == 1 || q4 == 2) ? 1.f : 0.f;
-    float Wv[2], Rv[2];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      Wv[h] = wx0 * Cc[2 * h] + wx1 * Cc[2 * h + 1];
-      Rv[h] = wy0 * Cc[2 * h] + wy1 * Cc[2 * h + 1];
-      Wv[h] += __shfl_xor_sync(0xffffffffu, Wv[h], 1);
-      Wv[h] += __shfl_xor_sync(0xffffffffu, Wv[h], 2);
-      Rv[h] += __shfl_xor_sync(0xffffffffu, Rv[h], 1);
-      Rv[h] += __shfl_xor_sync(0xffffffffu, Rv[h], 2);
-    }
-    if (q4 < 2) {  // lane q4 of the quad finishes row 16w + gid + 8 q4
-      const int v = 16 * warp + gid + 8 * q4;
-      float w = PR[v] + (q4 ? Wv[1] : Wv[0]);
-      float rv = RR[v] + (q4 ? Rv[1] : Rv[0]);
-      for (int c = 0; c < r; ++c) {
-        const float cu = s_cu[c * D + v];
-        w = fmaf(ca[W + c], cu, w);
-        rv = fmaf(cb[W + c], cu, rv);
+    for (int mt = 0; mt < 2; ++mt) {
+      const float* Cc = mt ? C1 : C0;
+      float Wv[2], Rv[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        Wv[h] = wx0 * Cc[2 * h] + wx1 * Cc[2 * h + 1];
+        Rv[h] = wy0 * Cc[2 * h] + wy1 * Cc[2 * h + 1];
+        Wv[h] += __shfl_xor_sync(0xffffffffu, Wv[h], 1);
+        Wv[h] += __shfl_xor_sync(0xffffffffu, Wv[h], 2);
+        Rv[h] += __shfl_xor_sync(0xffffffffu, Rv[h], 1);
+        Rv[h] += __shfl_xor_sync(0xffffffffu, Rv[h], 2);
       }
-      const float u = beta * (__bfloat162float(s_v[v]) - w);
-      const bf ubf = __float2bfloat16_rn(u);
-      const float kq = misc[0] + misc[1] + misc[2] + misc[3];
-      static_cast<bf*>(a.o)[(size_t)head * D + v] = __float2bfloat16_rn(rv + __bfloat162float(ubf) * kq);
-      if (!flush) static_cast<bf*>(a.buf_u)[(size_t)head * W * D + swz_el<bf, D>(P, v)] = ubf;
-      else s_bu[swz_el<bf, D>(P, v)] = ubf;
+      if (q4 < 2) {  // lane q4 of the quad stores row 32 wy + 16 mt + gid + 8 q4
+        const int v = 32 * wy + 16 * mt + gid + 8 * q4;
+        WV[v] = q4 ? Wv[1] : Wv[0];
+        RV[v] = q4 ? Rv[1] : Rv[0];
+      }
     }
+  }
+  csync();
+
+  // ---- phase 4: u_t and o_t, one thread per row v (coalesced stores) ----------------------
+  if (tid < D) {
+    const int v = tid;
+    float w = PR[v] + WV[v], rv = RR[v] + RV[v];
+    for (int c = 0; c < r; ++c) {
+      const float cu = s_cu[c * D + v];
+      w = fmaf(ca[W + c], cu, w);
+      rv = fmaf(cb[W + c], cu, rv);
+    }
+    const float u = beta * (__bfloat162float(s_v[v]) - w);
+    const bf ubf = __float2bfloat16_rn(u);
+    const float kq = misc[0] + misc[1] + misc[2] + misc[3];
+    static_cast<bf*>(a.o)[(size_t)head * D + v] = __float2bfloat16_rn(rv + __bfloat162float(ubf) * kq);
+    if (!flush) static_cast<bf*>(a.buf_u)[(size_t)head * W * D + swz_el<bf, D>(P, v)] = ubf;
+    else s_bu[swz_el<bf, D>(P, v)] = ubf;
   }
   if (tid == 0) a.pos[head] = flush ? 0 : P + 1;
   if (!flush) return;

@@ -172,7 +172,10 @@ __device__ __forceinline__ void report(int32_t* status, int bit) {
 // ------------------------------------------------------------------------------------------
 template <class C>
 __device__ __forceinline__ void stage_issue(const WinArgs& a, const WinLayout& L, uint8_t* st,
-                                            uint64_t* bar, int head, int P, bool with_io) {
+                                            uint64_t* bar, int head, int P, bool with_io,
+                                            int part = -1) {
+  // part -1: every copy; part 0: codes, scales, q, k; part 1: the rest (two issuers, each
+  // arriving once on a barrier that expects two arrivals)
   using Act = typename C::Act;
   using Buf = typename C::Buf;
   constexpr int D = C::D;
@@ -181,31 +184,41 @@ __device__ __forceinline__ void stage_issue(const WinArgs& a, const WinLayout& L
     mbar_arrive_expect_tx(bar, 0);
     return;
   }
+  const bool p0 = part <= 0, p1 = part != 0;
   const uint32_t lbytes = C::DIAG ? 4u * P * D : 4u * ((P + 3) & ~3);
-  uint32_t bytes = C::CODE_BYTES + 4u * C::NSCALES;
-  if (P > 0) bytes += (uint32_t)P * D * (sizeof(Act) + sizeof(Buf)) + lbytes;
-  if (r > 0) bytes += 4u * rp + 4u * r * D;
-  if (with_io) bytes += 3u * D * sizeof(Act) + (C::DIAG ? 4u * D : 0u);
+  uint32_t bytes = 0;
+  if (p0) bytes += C::CODE_BYTES + 4u * C::NSCALES + (with_io ? 2u * D * sizeof(Act) : 0u);
+  if (p1) {
+    if (P > 0) bytes += (uint32_t)P * D * (sizeof(Act) + sizeof(Buf)) + lbytes;
+    if (r > 0) bytes += 4u * rp + 4u * r * D;
+    if (with_io) bytes += D * sizeof(Act) + (C::DIAG ? 4u * D : 0u);
+  }
   mbar_arrive_expect_tx(bar, bytes);
-  bulk_g2s(st + L.codes, a.codes + (size_t)head * C::CODE_BYTES, C::CODE_BYTES, bar);
-  bulk_g2s(st + L.scales, a.scales + (size_t)head * C::NSCALES, 4u * C::NSCALES, bar);
-  if (P > 0) {
-    bulk_g2s(st + L.bk, static_cast<const Act*>(a.buf_k) + (size_t)head * W * D,
-             (uint32_t)P * D * sizeof(Act), bar);
-    bulk_g2s(st + L.bu, static_cast<const Buf*>(a.buf_u) + (size_t)head * W * D,
-             (uint32_t)P * D * sizeof(Buf), bar);
-    bulk_g2s(st + L.bL, a.buf_L + (size_t)head * (C::DIAG ? (size_t)W * D : (size_t)Wp), lbytes,
-             bar);
+  if (p0) {
+    bulk_g2s(st + L.codes, a.codes + (size_t)head * C::CODE_BYTES, C::CODE_BYTES, bar);
+    bulk_g2s(st + L.scales, a.scales + (size_t)head * C::NSCALES, 4u * C::NSCALES, bar);
+    if (with_io) {
+      bulk_g2s(st + L.q, static_cast<const Act*>(a.q) + (size_t)head * D, D * sizeof(Act), bar);
+      bulk_g2s(st + L.k, static_cast<const Act*>(a.k) + (size_t)head * D, D * sizeof(Act), bar);
+    }
   }
-  if (r > 0) {
-    bulk_g2s(st + L.cidx, a.comp_idx + (size_t)head * rp, 4u * rp, bar);
-    bulk_g2s(st + L.cu, a.comp_u + (size_t)head * r * D, 4u * r * D, bar);
-  }
-  if (with_io) {
-    bulk_g2s(st + L.q, static_cast<const Act*>(a.q) + (size_t)head * D, D * sizeof(Act), bar);
-    bulk_g2s(st + L.k, static_cast<const Act*>(a.k) + (size_t)head * D, D * sizeof(Act), bar);
-    bulk_g2s(st + L.v, static_cast<const Act*>(a.v) + (size_t)head * D, D * sizeof(Act), bar);
-    if constexpr (C::DIAG) bulk_g2s(st + L.g, a.g + (size_t)head * D, 4u * D, bar);
+  if (p1) {
+    if (P > 0) {
+      bulk_g2s(st + L.bk, static_cast<const Act*>(a.buf_k) + (size_t)head * W * D,
+               (uint32_t)P * D * sizeof(Act), bar);
+      bulk_g2s(st + L.bu, static_cast<const Buf*>(a.buf_u) + (size_t)head * W * D,
+               (uint32_t)P * D * sizeof(Buf), bar);
+      bulk_g2s(st + L.bL, a.buf_L + (size_t)head * (C::DIAG ? (size_t)W * D : (size_t)Wp), lbytes,
+               bar);
+    }
+    if (r > 0) {
+      bulk_g2s(st + L.cidx, a.comp_idx + (size_t)head * rp, 4u * rp, bar);
+      bulk_g2s(st + L.cu, a.comp_u + (size_t)head * r * D, 4u * r * D, bar);
+    }
+    if (with_io) {
+      bulk_g2s(st + L.v, static_cast<const Act*>(a.v) + (size_t)head * D, D * sizeof(Act), bar);
+      if constexpr (C::DIAG) bulk_g2s(st + L.g, a.g + (size_t)head * D, 4u * D, bar);
+    }
   }
 }
 
@@ -724,6 +737,7 @@ __device__ __forceinline__ void step_head(const WinArgs& a, const WinLayout& L, 
 // order while up to nstages - 1 later heads are already being copied into their stages.
 // ------------------------------------------------------------------------------------------
 constexpr int kStepThreads = kThreads;
+constexpr int kStepIssuer = kStepThreads - 32;  // lane 0 of the last warp issues stage copies
 
 template <class C>
 __global__ void __launch_bounds__(kStepThreads, 2)
@@ -755,9 +769,9 @@ __global__ void __launch_bounds__(kStepThreads, 2)
       stage_issue<C>(a, L, sm + L.stage0 + s * L.stage_bytes, &bars[s], h0 + s, hpos[s], true);
   if (!stage_wait(a, &bars[0], 0u)) return;
   for (int n = 0; n < nh; ++n) {
-    // refill the stage head n - 1 left (thread 128 leads the warp group with slack at the start
-    // of a head: the pair coefficients are shorter than the gates + frozen-state products)
-    if (nstages > 1 && tid == kStepThreads / 2 && n > 0 && n - 1 + nstages < nh) {
+    // refill the stage head n - 1 left; the issuer is lane 0 of the last warp, which has the
+    // least work early in a head (the pair-coefficient tiles go to warps 4, 5, ... in order)
+    if (nstages > 1 && tid == kStepIssuer && n > 0 && n - 1 + nstages < nh) {
       const int sp = (n - 1) % nstages;
       stage_issue<C>(a, L, sm + L.stage0 + sp * L.stage_bytes, &bars[sp], h0 + n - 1 + nstages,
                      hpos[n - 1 + nstages], true);
@@ -773,7 +787,7 @@ __global__ void __launch_bounds__(kStepThreads, 2)
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
     if (nstages == 1) {  // a single stage is refilled only once this head is done with it
       csync();
-      if (tid == kStepThreads / 2 && n + 1 < nh)
+      if (tid == kStepIssuer && n + 1 < nh)
         stage_issue<C>(a, L, st, &bars[0], h0 + n + 1, hpos[n + 1], true);
     }
     // one barrier ends the head (stage and scratch free) and agrees on the next head's copies

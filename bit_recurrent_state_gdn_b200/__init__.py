@@ -11,6 +11,7 @@ from .api import (  # noqa: F401
     gdn_decode_window_step,
     gdn_decode_window_steps,
     gdn_decode_window_steps_host,
+    gdn_decode_window_steps_host_fixed,
     gdn_host_staging_bytes,
     gdn_state_materialize,
     gdn_state_quantize,

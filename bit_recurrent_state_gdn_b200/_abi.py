@@ -51,6 +51,8 @@ SIGNATURES = {
     "gdn_host_staging_bytes": (_sz, [ctypes.POINTER(gdn_config)]),
     "gdn_decode_window_steps_host": (_i32, [ctypes.POINTER(gdn_config), ctypes.POINTER(gdn_state),
                                             _i32] + [_vp] * 7 + [_sz, _vp]),
+    "gdn_decode_window_steps_host_fixed": (_i32, [ctypes.POINTER(gdn_config),
+                                                  ctypes.POINTER(gdn_state), _i32] + [_vp] * 7),
     "gdn_window_flush": (_i32, [ctypes.POINTER(gdn_config), ctypes.POINTER(gdn_state), _vp, _vp]),
     "gdn_state_materialize": (_i32, [ctypes.POINTER(gdn_config), ctypes.POINTER(gdn_state), _vp,
                                      _vp]),

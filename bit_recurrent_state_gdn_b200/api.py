@@ -172,6 +172,20 @@ def gdn_decode_window_steps_host(cfg, state: GdnState, q, k, v, g, beta, o,
         "gdn_decode_window_steps_host")
 
 
+def gdn_decode_window_steps_host_fixed(cfg, state: GdnState, q, k, v, g, beta, o, stream=None):
+    """As gdn_decode_window_steps_host, staging through the library's fixed device array
+    (no staging argument; the call allocates nothing)."""
+    T = q.shape[0]
+    n, act, cpu = T * _heads(cfg) * cfg.d_v, _act(cfg), torch.device("cpu")
+    st = state.c_struct()
+    _check(_abi.load().gdn_decode_window_steps_host_fixed(
+        ctypes.byref(cfg), ctypes.byref(st), T, _ptr(q, "q", act, n, cpu),
+        _ptr(k, "k", act, n, cpu), _ptr(v, "v", act, n, cpu),
+        _ptr(g, "g", torch.float32, T * _gate_numel(cfg), cpu),
+        _ptr(beta, "beta", torch.float32, T * _heads(cfg), cpu), _ptr(o, "o", act, n, cpu),
+        _stream(stream)), "gdn_decode_window_steps_host_fixed")
+
+
 def gdn_window_flush(cfg, state: GdnState, seq_mask: Optional[torch.Tensor] = None, stream=None):
     st = state.c_struct()
     _check(_abi.load().gdn_window_flush(

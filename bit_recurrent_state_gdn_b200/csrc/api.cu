@@ -10,6 +10,10 @@
 #include "launch.h"
 #include "window_kernels.cuh"
 
+// Staging of gdn_decode_window_steps_host_fixed: one fixed array per device, reserved when the
+// module loads (no allocation at call time).
+static __device__ __align__(256) uint8_t g_fixed_staging[GDN_FIXED_STAGING_BYTES];
+
 namespace {
 
 thread_local char g_last_error[512] = "";
@@ -362,6 +366,75 @@ gdn_status gdn_decode_window_steps_host(const gdn_config* cfg, const gdn_state* 
   if (d2h) cudaStreamDestroy(d2h);
   if (st != GDN_OK) return st;
   if (e != cudaSuccess) return cuda_fail(e, "gdn_decode_window_steps_host");
+  return GDN_OK;
+}
+
+gdn_status gdn_decode_window_steps_host_fixed(const gdn_config* cfg, const gdn_state* state,
+                                              int32_t T, const void* host_q, const void* host_k,
+                                              const void* host_v, const float* host_g,
+                                              const float* host_beta, void* host_o,
+                                              gdn_stream_t stream) {
+  g_last_error[0] = 0;
+  gdn_status st = check_config(cfg, Use::Window);
+  if (st != GDN_OK) return st;
+  if (T < 0) return fail(GDN_ERR_INVALID_ARG, "T=%d must be >= 0", T);
+  if (heads_of(cfg) == 0 || T == 0) return GDN_OK;
+  if ((st = check_state(cfg, state)) != GDN_OK) return st;
+  if (!host_q || !host_k || !host_v || !host_g || !host_beta || !host_o)
+    return fail(GDN_ERR_INVALID_ARG, "a host input / output pointer is null");
+  const Slot sl = slot_layout(cfg);
+  if (sl.bytes > GDN_FIXED_STAGING_BYTES)
+    return fail(GDN_ERR_UNSUPPORTED,
+                "gdn_decode_window_steps_host_fixed: one staging slot needs %zu bytes for %lld "
+                "heads, the fixed staging array holds %zu; use gdn_decode_window_steps_host",
+                sl.bytes, (long long)heads_of(cfg), (size_t)GDN_FIXED_STAGING_BYTES);
+  // the array's address on the current device, looked up once per device
+  constexpr int kMaxDevices = 64;
+  static void* fixed_addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "gdn_decode_window_steps_host_fixed: cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail(GDN_ERR_UNSUPPORTED, "device %d beyond the %d this build tracks", dev, kMaxDevices);
+  void* base_v = __atomic_load_n(&fixed_addr[dev], __ATOMIC_ACQUIRE);
+  if (!base_v) {
+    e = cudaGetSymbolAddress(&base_v, g_fixed_staging);
+    if (e != cudaSuccess)
+      return cuda_fail(e, "gdn_decode_window_steps_host_fixed: cudaGetSymbolAddress");
+    __atomic_store_n(&fixed_addr[dev], base_v, __ATOMIC_RELEASE);
+  }
+  uint8_t* base = static_cast<uint8_t*>(base_v);
+  const size_t H = (size_t)heads_of(cfg), D = (size_t)cfg->d_k;
+  const size_t act_step = H * D * act_size(cfg);
+  const size_t g_step = 4 * H * (cfg->gate == GDN_GATE_DIAG ? D : 1);
+  const cudaStream_t cs = (cudaStream_t)stream;
+  gdnq::WinArgs a = make_args(cfg, state);
+  a.q = base + sl.q;
+  a.k = base + sl.k;
+  a.v = base + sl.v;
+  a.g = reinterpret_cast<const float*>(base + sl.g);
+  a.beta = reinterpret_cast<const float*>(base + sl.beta);
+  a.o = base + sl.o;
+  // one slot: on a single stream the copies of step t + 1 follow the step-t kernel and its copy
+  // of o, so nothing is overwritten early
+  for (int32_t t = 0; t < T; ++t) {
+    const uint8_t* hq = static_cast<const uint8_t*>(host_q) + t * act_step;
+    const uint8_t* hk = static_cast<const uint8_t*>(host_k) + t * act_step;
+    const uint8_t* hv = static_cast<const uint8_t*>(host_v) + t * act_step;
+    const uint8_t* hg = reinterpret_cast<const uint8_t*>(host_g) + t * g_step;
+    const uint8_t* hb = reinterpret_cast<const uint8_t*>(host_beta) + t * 4 * H;
+    e = cudaMemcpyAsync(base + sl.q, hq, act_step, cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(base + sl.k, hk, act_step, cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(base + sl.v, hv, act_step, cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(base + sl.g, hg, g_step, cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(base + sl.beta, hb, 4 * H, cudaMemcpyHostToDevice, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_decode_window_steps_host_fixed: copy in");
+    st = launch(gdnq::WinOp::Step, cfg, a, stream, "gdn_decode_window_steps_host_fixed");
+    if (st != GDN_OK) return st;
+    e = cudaMemcpyAsync(static_cast<uint8_t*>(host_o) + t * act_step, base + sl.o, act_step,
+                        cudaMemcpyDeviceToHost, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_decode_window_steps_host_fixed: copy out");
+  }
   return GDN_OK;
 }
 

@@ -190,6 +190,34 @@ gdn_status gdn_decode_window_steps_host(const gdn_config* cfg, const gdn_state* 
                                         size_t staging_bytes, gdn_stream_t stream);
 
 /*
+ * The same T decode steps from host buffers as gdn_decode_window_steps_host, for callers that
+ * may not allocate device memory themselves -- for instance a process whose device memory is
+ * owned by another framework's allocator and fixed at start-up -- and so cannot provide the
+ * staging buffer. (The method's pages describe no such entry point; it is an interface
+ * convenience of this library only.)
+ *   - Staging lives in one fixed device array inside the library, GDN_FIXED_STAGING_BYTES
+ *     (16 MiB) per device, reserved when the library is loaded. The call allocates nothing:
+ *     no device or host memory, no streams, no events.
+ *   - Needs one staging slot, gdn_host_staging_bytes(cfg) / 2 bytes, to fit in
+ *     GDN_FIXED_STAGING_BYTES: about 1 KiB per (sequence, head) pair for bf16 and d = 128, so up
+ *     to roughly 16,000 pairs per call; a larger batch gets GDN_ERR_UNSUPPORTED with the sizes
+ *     in gdn_last_error() and nothing is enqueued.
+ *   - Nothing in the array needs to start at zero: every step overwrites the inputs it uses.
+ *   - Runs serially on `stream` (per step: copy in, the step kernel, copy out), with no overlap
+ *     of copies and kernels; returns after everything is enqueued. host_o is complete once
+ *     `stream` has finished. Pinned host memory is needed for the copies to be asynchronous.
+ *   - All calls on one device share the array: two calls whose work overlaps in time (on
+ *     different streams, or from different host threads) race on it. Serialise them.
+ * Arguments, layouts and errors otherwise as gdn_decode_window_steps_host.
+ */
+#define GDN_FIXED_STAGING_BYTES ((size_t)16 << 20)
+gdn_status gdn_decode_window_steps_host_fixed(const gdn_config* cfg, const gdn_state* state,
+                                              int32_t T, const void* host_q, const void* host_k,
+                                              const void* host_v, const float* host_g,
+                                              const float* host_beta, void* host_o,
+                                              gdn_stream_t stream);
+
+/*
  * Forced window flush: for every head whose sequence is selected (seq_mask == NULL selects all;
  * otherwise device int32 [B], nonzero = selected) and whose pos > 0, materialise the logical
  * state, rebuild compensators and codes as gdn_state_quantize does, and set pos = 0. Heads with

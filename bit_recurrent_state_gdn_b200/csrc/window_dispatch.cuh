@@ -39,31 +39,29 @@ inline int num_sms() {
   return n;
 }
 
-// Shape of a persistent step launch: two CTAs per SM with two stages each when they fit in
-// shared memory, else one CTA per SM with as many stages (up to 4) as fit.
+// Shape of a persistent step launch: two CTAs per SM when two stages of the largest window
+// position fit into half of an SM's shared memory, else one CTA per SM. Each CTA gets all the
+// shared memory that allows and sizes its stages itself (up to kMaxStages).
 struct StepPlan {
-  int grid, per_cta, nstages;
+  int grid, per_cta;
   size_t smem;
 };
 
 template <class C>
 StepPlan plan_step(int W, int r, int heads) {
-  constexpr int kSmemPerSm = 228 * 1024, kSmemPerCta = kMaxSmemPerCta, kReserved = 1024;
+  constexpr int kSmemPerSm = 228 * 1024, kReserved = 1024;
   const int sms = num_sms();
-  auto smem_of = [&](int ns, int pc) { return (size_t)win_layout<C>(W, r, ns, pc).total; };
+  const bool red = !step_uses_mma<C>(W);
   auto per = [&](int ctas) { return std::min(kMaxHeadsPerCta, std::max(1, (heads + ctas - 1) / ctas)); };
   StepPlan p;
-  int bps = 2, ns = 2;
-  if (2 * (smem_of(2, per(2 * sms)) + kReserved) > (size_t)kSmemPerSm) {
-    bps = 1;
-    ns = 1;
-    for (int k = 4; k >= 2; --k)
-      if (smem_of(k, per(sms)) <= (size_t)kSmemPerCta) { ns = k; break; }
-  }
+  const size_t half = (size_t)kSmemPerSm / 2 - kReserved;
+  int bps = 2;
+  if ((size_t)win_layout<C>(W, r, 2, per(2 * sms), -1, red).total > half) bps = 1;
   p.per_cta = per(bps * sms);
   p.grid = (heads + p.per_cta - 1) / p.per_cta;
-  p.nstages = ns;
-  p.smem = smem_of(ns, p.per_cta);
+  p.smem = bps == 2 ? half
+                    : std::min((size_t)kMaxSmemPerCta,
+                               (size_t)win_layout<C>(W, r, kMaxStages, p.per_cta, -1, red).total);
   return p;
 }
 
@@ -76,7 +74,8 @@ cudaError_t launch_window_cfg(WinOp op, const WinArgs& a, int heads, cudaStream_
       const StepPlan p = plan_step<C>(a.W, a.r, heads);
       e = ensure_smem<window_step_kernel<C>>(p.smem);
       if (e == cudaSuccess)
-        window_step_kernel<C><<<p.grid, kStepThreads, p.smem, st>>>(a, heads, p.per_cta, p.nstages);
+        window_step_kernel<C><<<p.grid, kStepThreads, p.smem, st>>>(a, heads, p.per_cta,
+                                                                     (int)p.smem);
       break;
     }
     case WinOp::Flush:

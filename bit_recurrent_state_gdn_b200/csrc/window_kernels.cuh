@@ -81,46 +81,63 @@ struct WinLayout {
   uint32_t bars, stage0, vec, coef, red, tc, harr, total;                 // within the CTA
 };
 
-// Tensor-core scratch: int8 digit matrix of the phase-1 right-hand side [8][144 B], the bf16
-// [8][136] right-hand side of the pair-coefficient products, and the bf16 [8][Wr + 8] split
-// coefficients of the correction products (row strides padded against bank conflicts).
+// Tensor-core scratch: int8 digit matrix of the phase-1 right-hand side [8][144 B] and the bf16
+// [8][Wr + 8] split coefficients of the correction products (row strides padded against bank
+// conflicts).
 __host__ __device__ constexpr uint32_t tc_scratch_bytes(int Wr) {
-  return 8u * 144 + 8u * 136 * 2 + 8u * (Wr + 8) * 2 + 64;
+  return 8u * 144 + 8u * (Wr + 8) * 2 + 64;
 }
 
+// Per-CTA scratch first (barriers, vectors, coefficients, reduction space unless `red` is false,
+// tensor-core scratch, the pos / gate / beta of the CTA's heads), then `nstages` stages whose
+// buffered-pair regions hold `cap` rows (a multiple of 16, at most W rounded up to 16; -1 means
+// that maximum). The kernels only ever read or write pair rows below the stage's cap.
 __host__ __device__ inline WinLayout win_layout(int D, int code_bytes, int nscales, int act_size,
                                                 int buf_size, bool diag, int W, int r,
-                                                int nstages, int per_cta) {
+                                                int nstages, int per_cta, int cap = -1,
+                                                bool red = true) {
   // buffer rows rounded up to 16: the mma k-steps read (zero-filled) rows past the window
   const int Wp = (W + 3) & ~3, rp = (r + 3) & ~3, Wr = (W + 15) & ~15;
+  if (cap < 0) cap = Wr;
   WinLayout L;
+  L.bars = 0;
+  L.vec = 128;
+  L.coef = align128(L.vec + 4u * (7 * D + 64));
+  L.red = align128(L.coef + 4u * (2 * (W + r) + Wr + 4));  // a[W+r], b[W+r], fac[Wr]
+  L.tc = align128(L.red + (red ? 4u * 2 * kThreads : 0u));
+  L.harr = align128(L.tc + tc_scratch_bytes(Wr));
+  L.stage0 = align128(L.harr + 12u * per_cta);
   L.codes = 0;
   L.scales = align128(L.codes + code_bytes);
   L.bk = align128(L.scales + 4u * nscales);
-  L.bu = align128(L.bk + (uint32_t)Wr * D * act_size);
-  L.bL = align128(L.bu + (uint32_t)Wr * D * buf_size);
-  L.cidx = align128(L.bL + 4u * (diag ? (uint32_t)Wr * D : (uint32_t)Wp));
+  L.bu = align128(L.bk + (uint32_t)cap * D * act_size);
+  L.bL = align128(L.bu + (uint32_t)cap * D * buf_size);
+  L.cidx = align128(L.bL + 4u * (diag ? (uint32_t)cap * D : (uint32_t)Wp));
   L.cu = align128(L.cidx + 4u * rp);
   L.q = align128(L.cu + 4u * r * D);
   L.k = align128(L.q + (uint32_t)D * act_size);
   L.v = align128(L.k + (uint32_t)D * act_size);
   L.g = align128(L.v + (uint32_t)D * act_size);
   L.stage_bytes = align128(L.g + (diag ? 4u * D : 0u));
-  L.bars = 0;
-  L.stage0 = 128;
-  L.vec = L.stage0 + (uint32_t)nstages * L.stage_bytes;
-  L.coef = align128(L.vec + 4u * (7 * D + 64));
-  L.red = align128(L.coef + 4u * (2 * (W + r) + Wr + 4));  // a[W+r], b[W+r], fac[Wr]
-  L.tc = align128(L.red + 4u * 2 * kThreads);
-  L.harr = align128(L.tc + tc_scratch_bytes(Wr));
-  L.total = align128(L.harr + 12u * per_cta);
+  L.total = L.stage0 + (uint32_t)nstages * L.stage_bytes;
   return L;
 }
 
 template <class C>
-__host__ __device__ inline WinLayout win_layout(int W, int r, int nstages, int per_cta) {
+__host__ __device__ inline WinLayout win_layout(int W, int r, int nstages, int per_cta,
+                                                int cap = -1, bool red = true) {
   return win_layout(C::D, C::CODE_BYTES, C::NSCALES, (int)sizeof(typename C::Act),
-                    (int)sizeof(typename C::Buf), C::DIAG, W, r, nstages, per_cta);
+                    (int)sizeof(typename C::Buf), C::DIAG, W, r, nstages, per_cta, cap, red);
+}
+
+// Longest window whose diagonal-gate flush builds its split key planes in registers here.
+constexpr int kMmaDiagMaxW = 128;
+
+// Whether a configuration's decode step takes the tensor-core path (which needs no reduction
+// space and whose pair regions may be sized to the furthest window position).
+template <class C>
+__host__ __device__ inline bool step_uses_mma(int W) {
+  return C::MMA && (!C::DIAG || W <= kMmaDiagMaxW);
 }
 
 // Kernel arguments: the state's device pointers and the step's inputs (unused ones null).
@@ -737,27 +754,48 @@ __device__ __forceinline__ void step_head(const WinArgs& a, const WinLayout& L, 
 // order while up to nstages - 1 later heads are already being copied into their stages.
 // ------------------------------------------------------------------------------------------
 constexpr int kStepThreads = kThreads;
+constexpr int kMaxStages = 4;  // stage barriers in the first 64 bytes of shared memory
 constexpr int kStepIssuer = kStepThreads - 32;  // lane 0 of the last warp issues stage copies
 
 template <class C>
 __global__ void __launch_bounds__(kStepThreads, 2)
-    window_step_kernel(const WinArgs a, const int heads, const int per_cta, const int nstages) {
+    window_step_kernel(const WinArgs a, const int heads, const int per_cta, const int smem) {
   extern __shared__ __align__(128) uint8_t sm[];
-  const WinLayout L = win_layout<C>(a.W, a.r, nstages, per_cta);
   const int tid = threadIdx.x;
   const int h0 = blockIdx.x * per_cta;
   const int nh = min(per_cta, heads - h0);
   if (nh <= 0) return;
-  int32_t* hpos = reinterpret_cast<int32_t*>(sm + L.harr);
+  const bool mma = step_uses_mma<C>(a.W);
+  const int Wr = (a.W + 15) & ~15;
+  const WinLayout L0 = win_layout<C>(a.W, a.r, 0, per_cta, Wr, !mma);  // the scratch part
+  int32_t* hpos = reinterpret_cast<int32_t*>(sm + L0.harr);
   float* hg = reinterpret_cast<float*>(hpos + per_cta);
   float* hb = hg + per_cta;
+  int* pmax = reinterpret_cast<int*>(sm + L0.bars + 64);  // after the stage barriers (<= 4)
+  if (tid == 0) *pmax = 0;
+  csync();
+  int mp = 0;
   for (int i = tid; i < nh; i += C::NT) {
-    hpos[i] = a.pos[h0 + i];
+    const int P = a.pos[h0 + i];
+    hpos[i] = P;
+    if (P >= 0 && P < a.W) mp = max(mp, P);
     if constexpr (!C::DIAG) hg[i] = a.g[h0 + i];
     hb[i] = a.beta[h0 + i];
   }
-  for (uint32_t e = tid; e < tc_scratch_bytes((a.W + 15) & ~15) / 4; e += C::NT)
-    reinterpret_cast<uint32_t*>(sm + L.tc)[e] = 0u;  // unused rows of the mma operands stay 0
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mp = max(mp, __shfl_xor_sync(0xffffffffu, mp, off));
+  if ((tid & 31) == 0) atomicMax(pmax, mp);
+  for (uint32_t e = tid; e < tc_scratch_bytes(Wr) / 4; e += C::NT)
+    reinterpret_cast<uint32_t*>(sm + L0.tc)[e] = 0u;  // unused rows of the mma operands stay 0
+  csync();
+  // on the tensor-core path the stages are sized for the furthest window position among this
+  // CTA's heads (row P may be written, the products read up to the next multiple of 16), so a
+  // launch early in its windows keeps more heads' copies in flight
+  const int cap = mma ? min(Wr, (*pmax + 16) & ~15) : Wr;
+  const int nstages =
+      min(kMaxStages, (smem - (int)L0.stage0) /
+                          (int)win_layout<C>(a.W, a.r, 1, per_cta, cap, !mma).stage_bytes);
+  const WinLayout L = win_layout<C>(a.W, a.r, nstages, per_cta, cap, !mma);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L.bars);
   if (tid == 0) {
     for (int s = 0; s < nstages; ++s) mbar_init(&bars[s], 1);

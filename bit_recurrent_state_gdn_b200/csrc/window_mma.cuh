@@ -24,8 +24,6 @@
 
 namespace gdnq {
 
-// Longest window whose diagonal-gate flush builds its split key planes in registers here.
-constexpr int kMmaDiagMaxW = 128;
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
@@ -150,7 +148,7 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
   float* coef = reinterpret_cast<float*>(sm + L.coef);
   float *ca = coef, *cb = coef + (W + r);
   uint8_t* Bfrag = sm + L.tc;                                      // digits, fragment order
-  bf* Bc = reinterpret_cast<bf*>(sm + L.tc + 8 * 144 + 8 * 136 * 2);  // [8][Wr + 8]
+  bf* Bc = reinterpret_cast<bf*>(sm + L.tc + 8 * 144);  // [8][Wr + 8]
 
   const uint8_t* s_codes = st + L.codes;
   const float* s_scales = reinterpret_cast<const float*>(st + L.scales);

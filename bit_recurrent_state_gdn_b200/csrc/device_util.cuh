@@ -133,11 +133,13 @@ __device__ __forceinline__ float fast_exp(float x) {
 // 2^-24 * 128 = 2^-17, and the rounded quotient from x / s by one more, so q and the rounded
 // quotient lie on the same side of every half-integer unless q is within 2^-15 of one; only
 // there is the quotient formed by a correctly rounded division.
+// |q - rint(q)| is the distance to the nearest integer, near 1/2 only near a half-integer; a
+// non-finite q (a reciprocal that overflowed) also takes the division.
 __device__ __forceinline__ float rint_quotient(float x, float s, float inv) {
   const float q = x * inv;
-  const float f = fabsf(q - truncf(q));
-  if (fabsf(f - 0.5f) < 0x1p-14f) return rintf(__fdiv_rn(x, s));
-  return rintf(q);
+  const float r = rintf(q);
+  if (!(fabsf(q - r) <= 0.5f - 0x1p-14f)) return rintf(__fdiv_rn(x, s));
+  return r;
 }
 
 // ---- exact conversions -------------------------------------------------------------------

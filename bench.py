@@ -381,6 +381,10 @@ def main():
         "clocks": clocks,
     }
 
+    # ---- mixed per-head widths: every second head int4, the same inputs ---------------------
+    if not args.no_baselines and wl.fmt == "int8" and wl.D == 128:
+        line["mixed_half_int4"] = mixed_leg(wl, S0, inp, o, peak)
+
     # ---- high-precision-state baselines on the same inputs ---------------------------------
     if not args.no_baselines:
         line["baselines"] = {}
@@ -418,6 +422,35 @@ def main():
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def mixed_leg(wl, S0, inp, o, peak):
+    """The same decode with every second head held as int4 (group 32) in one mixed-format
+    launch; algorithmic bytes averaged over the two formats."""
+    import torch
+
+    import bit_recurrent_state_gdn_b200 as gdn
+
+    cfg = gdn.make_config(wl.B, wl.H, wl.D, wl.W, wl.r, wl.gate, "mixed", wl.act, wl.buf)
+    fmts = ["int8" if h % 2 == 0 else "int4_g32" for h in range(wl.heads)]
+    st = gdn.GdnState.allocate(cfg, head_fmt=fmts)
+    gdn.gdn_state_quantize(cfg, S0, st)
+    for t in range(4):
+        gdn.gdn_decode_window_step(cfg, st, inp["q"][t], inp["k"][t], inp["v"][t], inp["g"][t],
+                                   inp["beta"][t], o[t])
+    gdn.gdn_state_quantize(cfg, S0, st)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    gdn.gdn_decode_window_steps(cfg, st, inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], o)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    per_head = (avg_step_bytes(wl) + avg_step_bytes(wl.with_(fmt="int4_g32"))) / 2
+    gbs = per_head * wl.heads * wl.T / (ms / 1e3) / 1e9
+    return {"value": wl.heads * wl.T / (ms / 1e3), "unit": UNIT, "achieved_gbs": gbs,
+            "frac": gbs / peak, "ms_per_run": ms,
+            "note": "GDN_FMT_MIXED, heads alternately int8 / int4-g32, one launch per step"}
 
 
 def e2e(args, wl, cfg, inp, S0, state, world, dev):

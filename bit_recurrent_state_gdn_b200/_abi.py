@@ -10,7 +10,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdnq.so"
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(5)
 GDN_DEVICE_WAIT_TIMEOUT, GDN_DEVICE_BAD_POS = 0x1, 0x2
 GDN_GATE_SCALAR, GDN_GATE_DIAG = 0, 1
-GDN_FMT_INT8, GDN_FMT_INT4_G32, GDN_FMT_BF16, GDN_FMT_FP32 = 0, 1, 2, 3
+GDN_FMT_INT8, GDN_FMT_INT4_G32, GDN_FMT_BF16, GDN_FMT_FP32, GDN_FMT_MIXED = 0, 1, 2, 3, 4
 GDN_DTYPE_F32, GDN_DTYPE_BF16 = 0, 1
 GDN_MAX_COMPENSATORS = 16
 
@@ -25,7 +25,7 @@ class gdn_config(ctypes.Structure):
 
 
 STATE_FIELDS = ("codes", "scales", "buf_k", "buf_u", "buf_L", "comp_idx", "comp_u", "pos",
-                "status")
+                "status", "head_fmt")
 
 
 class gdn_state(ctypes.Structure):
@@ -33,7 +33,7 @@ class gdn_state(ctypes.Structure):
 
 
 SIZE_FIELDS = ("codes", "scales", "buf_k", "buf_u", "buf_L", "comp_idx", "comp_u", "pos",
-               "smem_step")
+               "smem_step", "head_fmt")
 
 
 class gdn_sizes(ctypes.Structure):

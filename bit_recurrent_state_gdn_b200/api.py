@@ -17,7 +17,7 @@ from . import _abi
 _DT = {"f32": _abi.GDN_DTYPE_F32, "bf16": _abi.GDN_DTYPE_BF16}
 _TORCH_DT = {_abi.GDN_DTYPE_F32: torch.float32, _abi.GDN_DTYPE_BF16: torch.bfloat16}
 _FMT = {"int8": _abi.GDN_FMT_INT8, "int4_g32": _abi.GDN_FMT_INT4_G32, "bf16": _abi.GDN_FMT_BF16,
-        "fp32": _abi.GDN_FMT_FP32}
+        "fp32": _abi.GDN_FMT_FP32, "mixed": _abi.GDN_FMT_MIXED}
 _GATE = {"scalar": _abi.GDN_GATE_SCALAR, "diag": _abi.GDN_GATE_DIAG}
 
 
@@ -82,9 +82,12 @@ class GdnState:
     comp_u: torch.Tensor
     pos: torch.Tensor
     status: torch.Tensor
+    head_fmt: torch.Tensor  # int8 [B*H]: each head's format (mixed-format states only)
 
     @staticmethod
-    def allocate(cfg: _abi.gdn_config, device="cuda") -> "GdnState":
+    def allocate(cfg: _abi.gdn_config, device="cuda", head_fmt=None) -> "GdnState":
+        """Zeroed buffers for cfg. head_fmt (mixed states): one format name ("int8" /
+        "int4_g32") or gdn_state_format value per head, in [B][H] order."""
         sz = gdn_state_sizes(cfg)
         dev = torch.device(device)
 
@@ -97,7 +100,8 @@ class GdnState:
             buf_k=buf(sz.buf_k, torch.uint8), buf_u=buf(sz.buf_u, torch.uint8),
             buf_L=buf(sz.buf_L, torch.float32), comp_idx=buf(sz.comp_idx, torch.int32),
             comp_u=buf(sz.comp_u, torch.float32), pos=buf(sz.pos, torch.int32),
-            status=torch.zeros(4, dtype=torch.int32, device=dev))
+            status=torch.zeros(4, dtype=torch.int32, device=dev),
+            head_fmt=_head_fmt(cfg, head_fmt, sz.head_fmt, dev))
 
     def c_struct(self) -> _abi.gdn_state:
         return _abi.gdn_state(*[getattr(self, n).data_ptr() for n in _abi.STATE_FIELDS])
@@ -112,6 +116,17 @@ class GdnState:
         for n, t in self.tensors().items():
             t.copy_(getattr(other, n))
         return self
+
+
+def _head_fmt(cfg, head_fmt, nbytes, dev) -> torch.Tensor:
+    if cfg.fmt != _abi.GDN_FMT_MIXED:
+        return torch.zeros(1, dtype=torch.int8, device=dev)
+    if head_fmt is None or len(head_fmt) != nbytes:
+        raise ValueError(f"a mixed-format state needs head_fmt with {nbytes} entries")
+    vals = [_FMT[f] if isinstance(f, str) else int(f) for f in head_fmt]
+    if any(v not in (_abi.GDN_FMT_INT8, _abi.GDN_FMT_INT4_G32) for v in vals):
+        raise ValueError("head_fmt entries must be int8 or int4_g32")
+    return torch.tensor(vals, dtype=torch.int8, device=dev)
 
 
 def _heads(cfg):

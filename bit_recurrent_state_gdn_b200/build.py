@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OBJ_DIR = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libgdnq.so")
-SOURCES = ["api.cu", "window_int8.cu", "window_int4.cu", "baseline.cu"]
+SOURCES = ["api.cu", "window_int8.cu", "window_int4.cu", "window_mixed.cu", "baseline.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -52,7 +52,7 @@ gdn_status check_config(const gdn_config* c, Use use) {
   if (heads_of(c) > INT32_MAX) return fail(GDN_ERR_INVALID_ARG, "B*H exceeds 2^31-1");
   if (c->gate != GDN_GATE_SCALAR && c->gate != GDN_GATE_DIAG)
     return fail(GDN_ERR_INVALID_ARG, "gate=%d is not a gdn_gate_kind", c->gate);
-  if (c->fmt < GDN_FMT_INT8 || c->fmt > GDN_FMT_FP32)
+  if (c->fmt < GDN_FMT_INT8 || c->fmt > GDN_FMT_MIXED)
     return fail(GDN_ERR_INVALID_ARG, "fmt=%d is not a gdn_state_format", c->fmt);
   if (c->act_dtype != GDN_DTYPE_F32 && c->act_dtype != GDN_DTYPE_BF16)
     return fail(GDN_ERR_INVALID_ARG, "act_dtype=%d is not a gdn_dtype", c->act_dtype);
@@ -65,8 +65,8 @@ gdn_status check_config(const gdn_config* c, Use use) {
       return fail(GDN_ERR_INVALID_ARG, "baseline step needs fmt FP32 or BF16");
     return GDN_OK;
   }
-  if (c->fmt != GDN_FMT_INT8 && c->fmt != GDN_FMT_INT4_G32)
-    return fail(GDN_ERR_INVALID_ARG, "windowed state needs fmt INT8 or INT4_G32");
+  if (c->fmt != GDN_FMT_INT8 && c->fmt != GDN_FMT_INT4_G32 && c->fmt != GDN_FMT_MIXED)
+    return fail(GDN_ERR_INVALID_ARG, "windowed state needs fmt INT8, INT4_G32 or MIXED");
   if (c->buf_dtype != GDN_DTYPE_F32 && c->buf_dtype != GDN_DTYPE_BF16)
     return fail(GDN_ERR_INVALID_ARG, "buf_dtype=%d is not a gdn_dtype", c->buf_dtype);
   if (c->W < 1) return fail(GDN_ERR_INVALID_ARG, "W=%d must be >= 1", c->W);
@@ -76,8 +76,8 @@ gdn_status check_config(const gdn_config* c, Use use) {
     return fail(GDN_ERR_UNSUPPORTED, "r=%d exceeds %d", c->r, GDN_MAX_COMPENSATORS);
   if (c->fmt == GDN_FMT_INT4_G32 && c->d_k % 32 != 0)
     return fail(GDN_ERR_UNSUPPORTED, "int4 with group 32 needs d_k %% 32 == 0");
-  if (c->fmt == GDN_FMT_INT4_G32 && c->d_k != 128)
-    return fail(GDN_ERR_UNSUPPORTED, "int4 state is built for d_k = 128");
+  if ((c->fmt == GDN_FMT_INT4_G32 || c->fmt == GDN_FMT_MIXED) && c->d_k != 128)
+    return fail(GDN_ERR_UNSUPPORTED, "int4 and mixed states are built for d_k = 128");
   if (c->W > (1 << 20)) return fail(GDN_ERR_UNSUPPORTED, "W=%d is too large", c->W);
   const size_t smem = gdnq::window_smem_bytes(*c);
   if (smem > (size_t)gdnq::kMaxSmemPerCta)
@@ -92,10 +92,10 @@ struct PerHead {
 
 PerHead per_head_bytes(const gdn_config* c) {
   const size_t D = (size_t)c->d_k;
-  const bool int4 = c->fmt == GDN_FMT_INT4_G32;
-  PerHead p;
+  const bool int4 = c->fmt == GDN_FMT_INT4_G32, mixed = c->fmt == GDN_FMT_MIXED;
+  PerHead p;  // a mixed state gives every head the larger slot of each buffer
   p.codes = int4 ? D * D / 2 : D * D;
-  p.scales = 4 * (int4 ? D * (D / 32) : D);
+  p.scales = 4 * (int4 || mixed ? D * (D / 32) : D);
   p.buf_k = (size_t)c->W * D * act_size(c);
   p.buf_u = (size_t)c->W * D * buf_size(c);
   p.buf_L = 4 * (c->gate == GDN_GATE_DIAG ? (size_t)c->W * D : (size_t)round4(c->W));
@@ -119,6 +119,8 @@ gdn_status check_state(const gdn_config* c, const gdn_state* s) {
   }
   if (s->status && (reinterpret_cast<uintptr_t>(s->status) & 3u) != 0)
     return fail(GDN_ERR_INVALID_ARG, "state.status is not 4-byte aligned");
+  if (c->fmt == GDN_FMT_MIXED && !s->head_fmt)
+    return fail(GDN_ERR_INVALID_ARG, "state.head_fmt is null for a mixed-format state");
   return GDN_OK;
 }
 
@@ -152,6 +154,10 @@ gdnq::WinArgs make_args(const gdn_config* c, const gdn_state* s) {
   a.comp_u = s->comp_u;
   a.pos = s->pos;
   a.status = s->status;
+  const PerHead ph = per_head_bytes(c);
+  a.code_stride = (uint32_t)ph.codes;
+  a.scale_stride = (uint32_t)(ph.scales / 4);
+  a.head_fmt = c->fmt == GDN_FMT_MIXED ? s->head_fmt : nullptr;
   a.H = c->H;
   a.W = c->W;
   a.r = c->r;
@@ -163,6 +169,8 @@ gdn_status launch(gdnq::WinOp op, const gdn_config* c, const gdnq::WinArgs& a,
   const int heads = (int)heads_of(c);
   cudaError_t e = c->fmt == GDN_FMT_INT4_G32
                       ? gdnq::launch_window_int4(op, *c, a, heads, (cudaStream_t)stream)
+                  : c->fmt == GDN_FMT_MIXED
+                      ? gdnq::launch_window_mixed(op, *c, a, heads, (cudaStream_t)stream)
                       : gdnq::launch_window_int8(op, *c, a, heads, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, where);
   return GDN_OK;
@@ -196,9 +204,9 @@ namespace gdnq {
 
 size_t window_smem_bytes(const gdn_config& c) {
   const int D = c.d_k;
-  const bool int4 = c.fmt == GDN_FMT_INT4_G32;
+  const bool int4 = c.fmt == GDN_FMT_INT4_G32, mixed = c.fmt == GDN_FMT_MIXED;
   const int code_bytes = int4 ? D * D / 2 : D * D;
-  const int nscales = int4 ? D * (D / 32) : D;
+  const int nscales = int4 || mixed ? D * (D / 32) : D;
   return win_layout(D, code_bytes, nscales, (int)act_size(&c), (int)buf_size(&c),
                     c.gate == GDN_GATE_DIAG, c.W, c.r, 1, kMaxHeadsPerCta)
       .total;
@@ -237,6 +245,7 @@ gdn_status gdn_state_sizes(const gdn_config* cfg, gdn_sizes* out) {
   out->comp_u = cfg->r > 0 ? n * p.comp_u : 0;
   out->pos = n * 4;
   out->smem_step = gdnq::window_smem_bytes(*cfg);
+  out->head_fmt = cfg->fmt == GDN_FMT_MIXED ? n : 0;
   return GDN_OK;
 }
 

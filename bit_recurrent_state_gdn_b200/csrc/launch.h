@@ -28,6 +28,8 @@ cudaError_t launch_window_int8(WinOp op, const gdn_config& cfg, const WinArgs& a
                                cudaStream_t stream);
 cudaError_t launch_window_int4(WinOp op, const gdn_config& cfg, const WinArgs& a, int heads,
                                cudaStream_t stream);
+cudaError_t launch_window_mixed(WinOp op, const gdn_config& cfg, const WinArgs& a, int heads,
+                                cudaStream_t stream);
 cudaError_t launch_baseline(const gdn_config& cfg, const BaseArgs& a, int heads,
                             cudaStream_t stream);
 

@@ -47,7 +47,7 @@ struct StepPlan {
   size_t smem;
 };
 
-template <class C>
+template <class C, bool MIX>
 StepPlan plan_step(int W, int r, int heads) {
   constexpr int kSmemPerSm = 228 * 1024, kReserved = 1024;
   const int sms = num_sms();
@@ -56,60 +56,66 @@ StepPlan plan_step(int W, int r, int heads) {
   StepPlan p;
   const size_t half = (size_t)kSmemPerSm / 2 - kReserved;
   int bps = 2;
-  if ((size_t)win_layout<C>(W, r, 2, per(2 * sms), -1, red).total > half) bps = 1;
+  if ((size_t)win_layout_mix<C, MIX>(W, r, 2, per(2 * sms), -1, red).total > half) bps = 1;
   p.per_cta = per(bps * sms);
   p.grid = (heads + p.per_cta - 1) / p.per_cta;
   p.smem = bps == 2 ? half
                     : std::min((size_t)kMaxSmemPerCta,
-                               (size_t)win_layout<C>(W, r, kMaxStages, p.per_cta, -1, red).total);
+                               (size_t)win_layout_mix<C, MIX>(W, r, kMaxStages, p.per_cta, -1,
+                                                              red).total);
   return p;
 }
 
-template <class C>
+template <class C, bool MIX = false>
 cudaError_t launch_window_cfg(WinOp op, const WinArgs& a, int heads, cudaStream_t st) {
-  const size_t smem1 = win_layout<C>(a.W, a.r, 1, 0).total;
+  size_t smem1 = win_layout<C>(a.W, a.r, 1, 0).total;
+  if constexpr (MIX) smem1 = std::max(smem1, (size_t)win_layout<Int4Of<C>>(a.W, a.r, 1, 0).total);
   cudaError_t e = cudaSuccess;
   switch (op) {
     case WinOp::Step: {
-      const StepPlan p = plan_step<C>(a.W, a.r, heads);
-      e = ensure_smem<window_step_kernel<C>>(p.smem);
+      const StepPlan p = plan_step<C, MIX>(a.W, a.r, heads);
+      e = ensure_smem<window_step_kernel<C, MIX>>(p.smem);
       if (e == cudaSuccess)
-        window_step_kernel<C><<<p.grid, kStepThreads, p.smem, st>>>(a, heads, p.per_cta,
-                                                                     (int)p.smem);
+        window_step_kernel<C, MIX><<<p.grid, kStepThreads, p.smem, st>>>(a, heads, p.per_cta,
+                                                                          (int)p.smem);
       break;
     }
     case WinOp::Flush:
-      e = ensure_smem<window_state_kernel<C, 0>>(smem1);
-      if (e == cudaSuccess) window_state_kernel<C, 0><<<heads, kThreads, smem1, st>>>(a);
+      e = ensure_smem<window_state_kernel<C, 0, MIX>>(smem1);
+      if (e == cudaSuccess) window_state_kernel<C, 0, MIX><<<heads, kThreads, smem1, st>>>(a);
       break;
     case WinOp::Materialize:
-      e = ensure_smem<window_state_kernel<C, 1>>(smem1);
-      if (e == cudaSuccess) window_state_kernel<C, 1><<<heads, kThreads, smem1, st>>>(a);
+      e = ensure_smem<window_state_kernel<C, 1, MIX>>(smem1);
+      if (e == cudaSuccess) window_state_kernel<C, 1, MIX><<<heads, kThreads, smem1, st>>>(a);
       break;
     case WinOp::Quantize:
-      quantize_kernel<C><<<heads, kThreads, 0, st>>>(a);
+      quantize_kernel<C, MIX><<<heads, kThreads, 0, st>>>(a);
       break;
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-template <int D, bool DIAG, bool INT4>
+// MIX: int8 and int4 heads in one launch (INT4 is then false: the int8 configuration, whose
+// int4 companion Int4Of<> takes the int4 heads).
+template <int D, bool DIAG, bool INT4, bool MIX = false>
 cudaError_t launch_window_types(WinOp op, const gdn_config& cfg, const WinArgs& a, int heads,
                                 cudaStream_t st) {
   using bf = __nv_bfloat16;
   const bool af = cfg.act_dtype == GDN_DTYPE_F32, bfp = cfg.buf_dtype == GDN_DTYPE_F32;
-  if (af && bfp) return launch_window_cfg<WinCfg<D, DIAG, INT4, float, float>>(op, a, heads, st);
-  if (af) return launch_window_cfg<WinCfg<D, DIAG, INT4, float, bf>>(op, a, heads, st);
-  if (bfp) return launch_window_cfg<WinCfg<D, DIAG, INT4, bf, float>>(op, a, heads, st);
-  return launch_window_cfg<WinCfg<D, DIAG, INT4, bf, bf>>(op, a, heads, st);
+  if (af && bfp)
+    return launch_window_cfg<WinCfg<D, DIAG, INT4, float, float>, MIX>(op, a, heads, st);
+  if (af) return launch_window_cfg<WinCfg<D, DIAG, INT4, float, bf>, MIX>(op, a, heads, st);
+  if (bfp) return launch_window_cfg<WinCfg<D, DIAG, INT4, bf, float>, MIX>(op, a, heads, st);
+  return launch_window_cfg<WinCfg<D, DIAG, INT4, bf, bf>, MIX>(op, a, heads, st);
 }
 
-template <int D, bool INT4>
+template <int D, bool INT4, bool MIX = false>
 cudaError_t launch_window_gate(WinOp op, const gdn_config& cfg, const WinArgs& a, int heads,
                                cudaStream_t st) {
-  if (cfg.gate == GDN_GATE_DIAG) return launch_window_types<D, true, INT4>(op, cfg, a, heads, st);
-  return launch_window_types<D, false, INT4>(op, cfg, a, heads, st);
+  if (cfg.gate == GDN_GATE_DIAG)
+    return launch_window_types<D, true, INT4, MIX>(op, cfg, a, heads, st);
+  return launch_window_types<D, false, INT4, MIX>(op, cfg, a, heads, st);
 }
 
 }  // namespace gdnq

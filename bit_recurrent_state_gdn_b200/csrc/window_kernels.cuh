@@ -130,6 +130,23 @@ __host__ __device__ inline WinLayout win_layout(int W, int r, int nstages, int p
                     (int)sizeof(typename C::Buf), C::DIAG, W, r, nstages, per_cta, cap, red);
 }
 
+// The int4 (group 32) configuration that shares C's head size, gate and dtypes, and the shared-
+// memory layout that holds a head of either format (codes of the int8 size, scales of the int4
+// size) when MIX is set.
+template <class C>
+using Int4Of = WinCfg<C::D, C::DIAG, true, typename C::Act, typename C::Buf>;
+
+template <class C, bool MIX>
+__host__ __device__ inline WinLayout win_layout_mix(int W, int r, int nstages, int per_cta,
+                                                    int cap = -1, bool red = true) {
+  if constexpr (!MIX) {
+    return win_layout<C>(W, r, nstages, per_cta, cap, red);
+  } else {
+    return win_layout(C::D, C::CODE_BYTES, Int4Of<C>::NSCALES, (int)sizeof(typename C::Act),
+                      (int)sizeof(typename C::Buf), C::DIAG, W, r, nstages, per_cta, cap, red);
+  }
+}
+
 // Longest window whose diagonal-gate flush builds its split key planes in registers here.
 constexpr int kMmaDiagMaxW = 128;
 
@@ -160,8 +177,16 @@ struct WinArgs {
   const float* S_in;       // quantize: fp32 states
   float* S_out;            // materialise: fp32 states
   const int32_t* seq_mask; // forced flush: [B] or null
+  const int8_t* head_fmt;  // mixed formats: gdn_state_format of each head, else null
+  uint32_t code_stride;    // bytes of codes per head
+  uint32_t scale_stride;   // scales (floats) per head
   int H, W, r;
 };
+
+// Whether a head of a mixed-format state is held as int4 (group 32).
+__device__ __forceinline__ bool head_is_int4(const WinArgs& a, int head) {
+  return a.head_fmt != nullptr && a.head_fmt[head] == GDN_FMT_INT4_G32;
+}
 
 // N consecutive logical elements (from column col0) of row `row` of a swizzled [rows][D] tile
 // of T, as fp32.
@@ -212,8 +237,8 @@ __device__ __forceinline__ void stage_issue(const WinArgs& a, const WinLayout& L
   }
   mbar_arrive_expect_tx(bar, bytes);
   if (p0) {
-    bulk_g2s(st + L.codes, a.codes + (size_t)head * C::CODE_BYTES, C::CODE_BYTES, bar);
-    bulk_g2s(st + L.scales, a.scales + (size_t)head * C::NSCALES, 4u * C::NSCALES, bar);
+    bulk_g2s(st + L.codes, a.codes + (size_t)head * a.code_stride, C::CODE_BYTES, bar);
+    bulk_g2s(st + L.scales, a.scales + (size_t)head * a.scale_stride, 4u * C::NSCALES, bar);
     if (with_io) {
       bulk_g2s(st + L.q, static_cast<const Act*>(a.q) + (size_t)head * D, D * sizeof(Act), bar);
       bulk_g2s(st + L.k, static_cast<const Act*>(a.k) + (size_t)head * D, D * sizeof(Act), bar);
@@ -743,8 +768,8 @@ __device__ __forceinline__ void step_head(const WinArgs& a, const WinLayout& L, 
   prepare_window_end<C>(st, L, P + 1, Lt, Ls, colexp, fac);
   csync();
   const WindowTile<C> tile = window_tile<C>(st, L, P + 1, r, colexp, fac);
-  requantize_store<C>(tile, r, a.codes + (size_t)head * C::CODE_BYTES,
-                      a.scales + (size_t)head * C::NSCALES,
+  requantize_store<C>(tile, r, a.codes + (size_t)head * a.code_stride,
+                      a.scales + (size_t)head * a.scale_stride,
                       a.comp_idx + (size_t)head * ((r + 3) & ~3), a.comp_u + (size_t)head * r * D,
                       ys, reinterpret_cast<int32_t*>(misc + 4));
 }
@@ -757,7 +782,7 @@ constexpr int kStepThreads = kThreads;
 constexpr int kMaxStages = 4;  // stage barriers in the first 64 bytes of shared memory
 constexpr int kStepIssuer = kStepThreads - 32;  // lane 0 of the last warp issues stage copies
 
-template <class C>
+template <class C, bool MIX>
 __global__ void __launch_bounds__(kStepThreads, 2)
     window_step_kernel(const WinArgs a, const int heads, const int per_cta, const int smem) {
   extern __shared__ __align__(128) uint8_t sm[];
@@ -767,7 +792,7 @@ __global__ void __launch_bounds__(kStepThreads, 2)
   if (nh <= 0) return;
   const bool mma = step_uses_mma<C>(a.W);
   const int Wr = (a.W + 15) & ~15;
-  const WinLayout L0 = win_layout<C>(a.W, a.r, 0, per_cta, Wr, !mma);  // the scratch part
+  const WinLayout L0 = win_layout_mix<C, MIX>(a.W, a.r, 0, per_cta, Wr, !mma);  // the scratch part
   int32_t* hpos = reinterpret_cast<int32_t*>(sm + L0.harr);
   float* hg = reinterpret_cast<float*>(hpos + per_cta);
   float* hb = hg + per_cta;
@@ -794,8 +819,18 @@ __global__ void __launch_bounds__(kStepThreads, 2)
   const int cap = mma ? min(Wr, (*pmax + 16) & ~15) : Wr;
   const int nstages =
       min(kMaxStages, (smem - (int)L0.stage0) /
-                          (int)win_layout<C>(a.W, a.r, 1, per_cta, cap, !mma).stage_bytes);
-  const WinLayout L = win_layout<C>(a.W, a.r, nstages, per_cta, cap, !mma);
+                          (int)win_layout_mix<C, MIX>(a.W, a.r, 1, per_cta, cap, !mma).stage_bytes);
+  const WinLayout L = win_layout_mix<C, MIX>(a.W, a.r, nstages, per_cta, cap, !mma);
+  // a head's stage copies and step in its own format (both fit the mixed layout)
+  auto issue = [&](uint8_t* st, uint64_t* bar, int head, int P) {
+    if constexpr (MIX) {
+      if (head_is_int4(a, head)) {
+        stage_issue<Int4Of<C>>(a, L, st, bar, head, P, true);
+        return;
+      }
+    }
+    stage_issue<C>(a, L, st, bar, head, P, true);
+  };
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L.bars);
   if (tid == 0) {
     for (int s = 0; s < nstages; ++s) mbar_init(&bars[s], 1);
@@ -804,20 +839,27 @@ __global__ void __launch_bounds__(kStepThreads, 2)
   csync();
   if (tid == 0)
     for (int s = 0; s < nstages && s < nh; ++s)
-      stage_issue<C>(a, L, sm + L.stage0 + s * L.stage_bytes, &bars[s], h0 + s, hpos[s], true);
+      issue(sm + L.stage0 + s * L.stage_bytes, &bars[s], h0 + s, hpos[s]);
   if (!stage_wait(a, &bars[0], 0u)) return;
   for (int n = 0; n < nh; ++n) {
     // refill the stage head n - 1 left; the issuer is lane 0 of the last warp, which has the
     // least work early in a head (the pair-coefficient tiles go to warps 4, 5, ... in order)
     if (nstages > 1 && tid == kStepIssuer && n > 0 && n - 1 + nstages < nh) {
       const int sp = (n - 1) % nstages;
-      stage_issue<C>(a, L, sm + L.stage0 + sp * L.stage_bytes, &bars[sp], h0 + n - 1 + nstages,
-                     hpos[n - 1 + nstages], true);
+      issue(sm + L.stage0 + sp * L.stage_bytes, &bars[sp], h0 + n - 1 + nstages,
+            hpos[n - 1 + nstages]);
     }
     uint8_t* st = sm + L.stage0 + (n % nstages) * L.stage_bytes;
     const int P = hpos[n];
     if (P >= 0 && P < a.W) {
-      step_head<C>(a, L, sm, st, h0 + n, P, C::DIAG ? 0.f : hg[n], hb[n]);
+      bool done = false;
+      if constexpr (MIX) {
+        if (head_is_int4(a, h0 + n)) {
+          step_head<Int4Of<C>>(a, L, sm, st, h0 + n, P, C::DIAG ? 0.f : hg[n], hb[n]);
+          done = true;
+        }
+      }
+      if (!done) step_head<C>(a, L, sm, st, h0 + n, P, C::DIAG ? 0.f : hg[n], hb[n]);
     } else if (tid == 0) {
       report(a.status, GDN_DEVICE_BAD_POS);
     }
@@ -825,8 +867,7 @@ __global__ void __launch_bounds__(kStepThreads, 2)
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
     if (nstages == 1) {  // a single stage is refilled only once this head is done with it
       csync();
-      if (tid == kStepIssuer && n + 1 < nh)
-        stage_issue<C>(a, L, st, &bars[0], h0 + n + 1, hpos[n + 1], true);
+      if (tid == kStepIssuer && n + 1 < nh) issue(st, &bars[0], h0 + n + 1, hpos[n + 1]);
     }
     // one barrier ends the head (stage and scratch free) and agrees on the next head's copies
     int timed_out = 0;
@@ -845,11 +886,10 @@ __global__ void __launch_bounds__(kStepThreads, 2)
 // One CTA per head, one stage.
 // ------------------------------------------------------------------------------------------
 template <class C, int MODE>
-__global__ void __launch_bounds__(kThreads) window_state_kernel(const WinArgs a) {
+__device__ __forceinline__ void window_state_body(const WinArgs& a, uint8_t* sm, int head) {
   constexpr int D = C::D;
-  extern __shared__ __align__(128) uint8_t sm[];
   const WinLayout L = win_layout<C>(a.W, a.r, 1, 0);
-  const int head = blockIdx.x, tid = threadIdx.x;
+  const int tid = threadIdx.x;
   const int W = a.W, r = a.r;
   const int P = a.pos[head];
   if (P < 0 || P >= W) {
@@ -886,8 +926,8 @@ __global__ void __launch_bounds__(kThreads) window_state_kernel(const WinArgs a)
   csync();
   const WindowTile<C> tile = window_tile<C>(st, L, P, r, colexp, fac);
   if constexpr (MODE == 0) {
-    requantize_store<C>(tile, r, a.codes + (size_t)head * C::CODE_BYTES,
-                        a.scales + (size_t)head * C::NSCALES,
+    requantize_store<C>(tile, r, a.codes + (size_t)head * a.code_stride,
+                        a.scales + (size_t)head * a.scale_stride,
                         a.comp_idx + (size_t)head * ((r + 3) & ~3),
                         a.comp_u + (size_t)head * r * D, colmax, sel);
     if (tid == 0) a.pos[head] = 0;
@@ -907,22 +947,47 @@ __global__ void __launch_bounds__(kThreads) window_state_kernel(const WinArgs a)
   }
 }
 
+// One CTA per head. With MIX, a head whose head_fmt is INT4_G32 takes the int4 configuration.
+template <class C, int MODE, bool MIX>
+__global__ void __launch_bounds__(kThreads) window_state_kernel(const WinArgs a) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  const int head = blockIdx.x;
+  if constexpr (MIX) {
+    if (head_is_int4(a, head)) {
+      window_state_body<Int4Of<C>, MODE>(a, sm, head);
+      return;
+    }
+  }
+  window_state_body<C, MODE>(a, sm, head);
+}
+
 // ------------------------------------------------------------------------------------------
 // Initial quantization of fp32 states.
 // ------------------------------------------------------------------------------------------
 template <class C>
-__global__ void __launch_bounds__(kThreads) quantize_kernel(const WinArgs a) {
+__device__ __forceinline__ void quantize_body(const WinArgs& a, int head) {
   constexpr int D = C::D;
   __shared__ float colmax[D];
   __shared__ int32_t sel[GDN_MAX_COMPENSATORS];
-  const int head = blockIdx.x;
   DenseTile<C> tile;
   tile.S = a.S_in + (size_t)head * D * D;
-  requantize_store<C>(tile, a.r, a.codes + (size_t)head * C::CODE_BYTES,
-                      a.scales + (size_t)head * C::NSCALES,
+  requantize_store<C>(tile, a.r, a.codes + (size_t)head * a.code_stride,
+                      a.scales + (size_t)head * a.scale_stride,
                       a.comp_idx + (size_t)head * ((a.r + 3) & ~3),
                       a.comp_u + (size_t)head * a.r * D, colmax, sel);
   if (threadIdx.x == 0) a.pos[head] = 0;
+}
+
+template <class C, bool MIX>
+__global__ void __launch_bounds__(kThreads) quantize_kernel(const WinArgs a) {
+  const int head = blockIdx.x;
+  if constexpr (MIX) {
+    if (head_is_int4(a, head)) {
+      quantize_body<Int4Of<C>>(a, head);
+      return;
+    }
+  }
+  quantize_body<C>(a, head);
 }
 
 }  // namespace gdnq

@@ -701,7 +701,7 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
 
   // ---- scales and codes into this warp's rows of the stage's code tile ---------------------
   // (the warp read its old code rows above and no other warp reads them)
-  float* g_scales = a.scales + (size_t)head * C::NSCALES;
+  float* g_scales = a.scales + (size_t)head * a.scale_stride;
   __syncwarp();
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
@@ -738,7 +738,7 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
   // ---- this warp's 16 code rows to HBM, 16 bytes per lane per store -----------------------
   {
     constexpr int RB = C::ROW_BYTES, CH = 16 * RB / 16;  // 16-byte chunks of the warp's rows
-    uint8_t* g_codes = a.codes + (size_t)head * C::CODE_BYTES + 16 * warp * RB;
+    uint8_t* g_codes = a.codes + (size_t)head * a.code_stride + 16 * warp * RB;
     const uint8_t* src = s_codes + 16 * warp * RB;
 #pragma unroll
     for (int ch = lane; ch < CH; ch += 32)

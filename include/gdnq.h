@@ -60,7 +60,8 @@ typedef enum {
     GDN_FMT_INT8 = 0,     /* int8 codes, one fp32 scale per state row */
     GDN_FMT_INT4_G32 = 1, /* packed int4 codes, one fp32 scale per row and 32 key channels */
     GDN_FMT_BF16 = 2,     /* plain bf16 state (baseline step only) */
-    GDN_FMT_FP32 = 3      /* plain fp32 state (baseline step only) */
+    GDN_FMT_FP32 = 3,     /* plain fp32 state (baseline step only) */
+    GDN_FMT_MIXED = 4     /* INT8 or INT4_G32 per head, as gdn_state.head_fmt says (d = 128) */
 } gdn_state_format;
 
 typedef enum { GDN_DTYPE_F32 = 0, GDN_DTYPE_BF16 = 1 } gdn_dtype;
@@ -96,6 +97,15 @@ typedef struct {
  *   comp_u   fp32  [B][H][r][D]        value column of each compensator pair (r > 0 only)
  *   pos      int32 [B][H]              pairs already in the window, 0 <= pos < W
  *   status   int32 [1], optional       device word the kernels OR GDN_DEVICE_* bits into
+ *   head_fmt int8  [B][H]              (GDN_FMT_MIXED only) GDN_FMT_INT8 or GDN_FMT_INT4_G32 for
+ *                                       each head; read by every call, written by none
+ * With GDN_FMT_MIXED ("Low-Bit GDN Recurrent-State Quantization ...", Abstract: bit widths
+ * allocated per head under a model-wide budget) every head has the slot of the larger format:
+ *   codes    uint8 [B][H][D][D]        an INT8 head fills its slot as above; an INT4_G32 head
+ *                                       uses its first D*D/2 bytes, laid out as for INT4_G32
+ *   scales   fp32  [B][H][D][D/32]     an INT4_G32 head fills its slot; an INT8 head uses its
+ *                                       first D floats
+ * and every entry point treats each head exactly as a call with that head's format would.
  * Tiles are stored swizzled: in each per-head [rows][RB-byte] tile of codes, buf_k and buf_u,
  * the 16-byte chunk c of row i is stored at chunk c ^ x(i), x(i) = i & 7 when RB >= 128, else
  * (i * RB / 128) & (RB / 16 - 1) (identity for 16-byte rows). A row's bytes keep their order
@@ -117,6 +127,7 @@ typedef struct {
     float* comp_u;
     int32_t* pos;
     int32_t* status;
+    const int8_t* head_fmt;
 } gdn_state;
 
 /* Byte sizes of each buffer of gdn_state for the whole batch (0 where unused), and the dynamic
@@ -124,6 +135,7 @@ typedef struct {
 typedef struct {
     size_t codes, scales, buf_k, buf_u, buf_L, comp_idx, comp_u, pos;
     size_t smem_step;
+    size_t head_fmt;
 } gdn_sizes;
 
 /* Checks cfg and fills *out. Host-only: touches no device. Errors: GDN_ERR_INVALID_ARG for a

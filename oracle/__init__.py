@@ -9,6 +9,11 @@ function of the method lives in the C file, which states what it restates from t
 ("LeapQuant: Efficient Linear Attention with Accurate Recurrent State Quantization", Abstract;
 "Low-Bit GDN Recurrent-State Quantization: ... Pure-Write Sliding Windows", Abstract).
 
+Parity unpinned against the pages (pinned only to the mathematics): the FP8 format of the
+pure-write pairs (e4m3, one fp32 scale absmax / 448 per vector). The page says "FP8 vector
+pairs" and nothing more; the tests pin the e4m3 rounding to torch's float8_e4m3fn and the
+window's algebra to the plain recurrence, not the format choice.
+
 Parity unpinned: the compensator column-selection rule (top-r columns by max-abs). The pages
 name compensator tokens but give no selection rule and no numbers; the tests pin only that the
 taken-out columns plus the residual reproduce the state exactly.
@@ -76,6 +81,12 @@ def load(path: Optional[str] = None):
     lib.orc_o1_run.argtypes = [_int] * 7 + [_vp] * 8
     lib.orc_o2_run.restype = _int
     lib.orc_o2_run.argtypes = [_int] * 9 + [_vp] * 18
+    lib.orc_round_e4m3.restype = ctypes.c_double
+    lib.orc_round_e4m3.argtypes = [ctypes.c_double]
+    lib.orc_fp8_vector.restype = ctypes.c_double
+    lib.orc_fp8_vector.argtypes = [_int, _int, _d, _d]
+    lib.orc_pw_run.restype = _int
+    lib.orc_pw_run.argtypes = [_int] * 9 + [_vp] * 12
     if path == _build.OUT:
         _lib, _lib_path = lib, path
     return lib
@@ -232,4 +243,52 @@ def o2_run(q, k, v, g, beta, W: int, r: int = 0, fmt: str = "int8", S0=None,
         _p(v), _p(g), _p(beta), _p(fm), _p(res.o), _p(res.codes), _p(res.scales),
         _p(res.cidx) if r > 0 else None, _p(res.cu) if r > 0 else None, _p(res.pos),
         _p(res.bk), _p(res.bu), _p(res.bL), _p(res.S), _p(res.ties))
+    return res
+
+
+# ---------------------------------------------------------------------------------------------
+# PW: the pure-write sliding window
+# ---------------------------------------------------------------------------------------------
+def round_e4m3(x: float, lib=None) -> float:
+    return (lib or load()).orc_round_e4m3(float(x))
+
+
+def fp8_vector(x: np.ndarray, prec32: bool = False, lib=None):
+    """FP8 round trip of a vector with one scale. Returns (values, scale)."""
+    lib = lib or load()
+    x = _f64(x).ravel()
+    out = np.zeros_like(x)
+    s = lib.orc_fp8_vector(x.size, int(prec32), x, out)
+    return out, s
+
+
+@dataclass
+class PWResult:
+    o: np.ndarray          # [T][nh][D] fp64, before storage rounding
+    codes: np.ndarray      # [nh][D][D] int8 history codes (int4 unpacked, in [-7, 7])
+    scales: np.ndarray     # [nh][D][groups]
+    px: np.ndarray         # [nh][Wp][D] pair value vectors as stored, by ring slot
+    py: np.ndarray         # [nh][Wp][D] pair key vectors as stored, by ring slot
+    S: np.ndarray          # [nh][D][D] logical state: history + the pairs in the window
+
+
+def pw_run(q, k, v, g, beta, Wp: int, fmt: str = "int8", S0=None, quant: bool = True,
+           fp8: bool = True, prec32: bool = False, lib=None) -> PWResult:
+    """Pure-write sliding window of Wp FP8 pairs over a low-bit history (``quant``; else an
+    exact history). ``prec32`` mirrors GPU storage and single-precision decisions."""
+    lib = lib or load()
+    q, k, v, beta = _f64(q), _f64(k), _f64(v), _f64(beta)
+    T, nh, D = k.shape
+    g, Dg = _gate(g, T, nh, D)
+    S0 = _f64(S0)
+    f = _FMT[fmt]
+    ng = lib.orc_num_groups(FMT_INT4 if f == FMT_INT4 else FMT_INT8, D)
+    res = PWResult(o=np.zeros((T, nh, D)), codes=np.zeros((nh, D, D), np.int8),
+                   scales=np.zeros((nh, D, ng)), px=np.zeros((nh, Wp, D)),
+                   py=np.zeros((nh, Wp, D)), S=np.zeros((nh, D, D)))
+    rc = lib.orc_pw_run(D, T, Wp, f, nh, Dg, int(quant), int(fp8), int(prec32), _p(S0), _p(q),
+                        _p(k), _p(v), _p(g), _p(beta), _p(res.o), _p(res.codes),
+                        _p(res.scales), _p(res.px), _p(res.py), _p(res.S))
+    if rc != 0:
+        raise ValueError("pw_run: bad window length or history format")
     return res

@@ -21,7 +21,9 @@
  *            no mechanism).
  *   [PW] "Low-Bit GDN Recurrent-State Quantization: Global Gradient-aware Allocation and
  *        Pure-Write Sliding Windows", Abstract: quantized write-back errors feed into later
- *        steps (why quantize-every-step, the window length 1 case, degrades).
+ *        steps (why quantize-every-step, the window length 1 case, degrades); recent pure
+ *        writes are kept as FP8 vector pairs, carried through the full transition, and merged
+ *        into the low-bit history only once they leave the window.
  *
  * The recurrence, for one (sequence, head), state S in R^{d_v x d_k} (row i = value channel,
  * column j = key channel), gate a_t in R^{d_k} (GDN: all entries equal; KDA: per key channel):
@@ -30,7 +32,7 @@
  *
  * The gate enters as its logarithm g_t = log a_t, so products of gates over a window are sums.
  *
- * Three formulations live here; none calls another's step code:
+ * Four formulations live here; none calls another's step code:
  *   plain  -- the recurrence in fp64, optionally rounding the stored state to fp32 / bf16 after
  *             each step (the high-precision-state baselines and the fp32 warm-up);
  *   O1     -- the recurrence applied literally as matrix products (D x D transition matrix),
@@ -38,6 +40,8 @@
  *   O2     -- the buffered form: frozen low-bit state + buffered pairs (k_i, u_i, L_i) +
  *             compensator pairs, flushed (materialised, requantised) when the window fills.
  *             Optional storage roundings mirror what a GPU stores between steps.
+ *   PW     -- the pure-write sliding window [PW]: a low-bit history requantised every step plus
+ *             the last Wp pure writes as FP8 pairs (its readings are stated where it starts).
  *
  * Readings of the pages where they are silent (each one is listed in the design notes):
  *   - quantizer: symmetric absmax, s = absmax / 127 (int8, one scale per row) or absmax / 7
@@ -520,4 +524,206 @@ int orc_o2_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int round_st
         free(s.bk); free(s.bu); free(s.bL); free(Sx); free(vec);
     }
     return ties;
+}
+
+
+/* ------------------------------------------------------------------------------------------
+ * PW: the pure-write sliding window ("Low-Bit GDN Recurrent-State Quantization: Global
+ * Gradient-aware Allocation and Pure-Write Sliding Windows", Abstract). The state is a low-bit
+ * history H plus the pure writes of the last Wp steps, each kept apart as a pair of FP8 vectors
+ * (x, y) standing for the rank-one matrix x y^T. The pure write of step t is its state-free term
+ * beta_t v_t k_t^T, so a pair starts as x = beta_t v_t, y = k_t. The full transition
+ * Z -> Z Diag(a) (I - beta k k^T) applied to x y^T only changes the key side,
+ *     y -> (I - beta k k^T) Diag(a) y = a.y - beta <k, a.y> k,
+ * so a pair stays a pair while it is carried through later steps. A pair leaves the window Wp
+ * steps after its write and is then added to the history, which is requantised. Since the
+ * history also takes the transition every step, it is requantised every step (the low-bit
+ * write-back that the window keeps recent writes out of).
+ *
+ * Readings (the page gives no more than the sentence above; each is listed in the design notes):
+ *   - FP8 is e4m3 (the finite variant: 4 exponent bits, bias 7, 3 mantissa bits, largest 448)
+ *     with one fp32 scale per vector, s = absmax / 448; stored t = e4m3(x / s), value s * t.
+ *   - Step t: the pair written at t - Wp (if any) is added to the history first; the history
+ *     then takes step t's transition; the pairs still in the window take it on their key side;
+ *     the new pair (beta v, k) enters. Wp = 0: the write joins the history at once (this is
+ *     quantize-every-step write-back).
+ *   - o_t = S_t q_t from the step's results before they are stored (the history before its
+ *     requantisation, the carried keys and the new pair before FP8 rounding): the rounding at
+ *     the write reaches the output from the next step on, as in the window form.
+ * quant = 0 keeps the history exact; fp8 = 0 keeps pairs exact. prec32 rounds what a GPU stores
+ * (the write vector beta v, carried keys, merged history entries) to fp32 and takes the
+ * quantizer's and the FP8 decisions in single precision.
+ * ---------------------------------------------------------------------------------------- */
+
+/* Nearest e4m3 value, ties to even, saturating at +-448. From the format's definition: normal
+ * values 2^(E-7) (1 + m/8) for E = 1..15 (E = 15, m = 7 is NaN, so 448 = 2^8 * 1.75 is the
+ * largest), subnormals 2^-6 (m/8); the spacing in x's binade [2^(e-1), 2^e) is 2^(e-4), never
+ * finer than the subnormal spacing 2^-9. */
+double orc_round_e4m3(double x) {
+    if (x == 0.0 || !isfinite(x)) return x;
+    double m = fabs(x);
+    if (m >= 448.0) return copysign(448.0, x);
+    int e;
+    frexp(m, &e);                          /* m = f 2^e, 0.5 <= f < 1 */
+    int qexp = e - 4;
+    if (qexp < -9) qexp = -9;
+    double quantum = ldexp(1.0, qexp);
+    double r = rint(m / quantum) * quantum; /* 448 < r only for m in (448, 464): excluded above */
+    return copysign(r, x);
+}
+
+/* FP8 round trip of an n-vector with one scale: s = absmax / 448, out = s * e4m3(x / s).
+ * Returns the scale. prec32: x is first rounded to fp32 and each decision is taken in fp32. */
+double orc_fp8_vector(int n, int prec32, const double* x, double* out) {
+    double m = 0.0;
+    for (int j = 0; j < n; ++j) m = fmax(m, fabs(prec32 ? orc_round_f32(x[j]) : x[j]));
+    double s = m / 448.0;
+    if (prec32) s = orc_round_f32(s);
+    for (int j = 0; j < n; ++j) {
+        if (s == 0.0) { out[j] = 0.0; continue; }
+        double t = (prec32 ? orc_round_f32(x[j]) : x[j]) / s;
+        if (prec32) t = orc_round_f32(t);
+        double y = s * orc_round_e4m3(t);
+        out[j] = prec32 ? orc_round_f32(y) : y;
+    }
+    return s;
+}
+
+int orc_pw_run(int D, int T, int Wp, int fmt, int nh, int Dg, int quant, int fp8, int prec32,
+               const double* S0, const double* q, const double* k, const double* v,
+               const double* g, const double* beta, double* o, int8_t* codes_out,
+               double* scales_out, double* px_out, double* py_out, double* S_out) {
+    if (Wp < 0 || (quant && fmt != ORC_FMT_INT8 && fmt != ORC_FMT_INT4)) return -1;
+    const int qfmt = fmt == ORC_FMT_INT4 ? ORC_FMT_INT4 : ORC_FMT_INT8;
+    const int ng = orc_num_groups(qfmt, D);
+#pragma omp parallel for schedule(dynamic)
+    for (int h = 0; h < nh; ++h) {
+        const size_t DD = (size_t)D * D;
+        const int ns = Wp > 0 ? Wp : 1;
+        double* H = (double*)malloc(sizeof(double) * DD);   /* history as stored (dequantised) */
+        int8_t* codes = (int8_t*)calloc(DD, 1);
+        double* scales = (double*)calloc((size_t)D * ng, sizeof(double));
+        double* px = (double*)calloc((size_t)ns * D, sizeof(double)); /* pair x, by ring slot */
+        double* py = (double*)calloc((size_t)ns * D, sizeof(double)); /* pair y, by ring slot */
+        double* pyn = (double*)malloc(sizeof(double) * (size_t)ns * D);  /* carried keys */
+        double* a = (double*)malloc(sizeof(double) * D);
+        double* w = (double*)malloc(sizeof(double) * D);
+        double* x = (double*)malloc(sizeof(double) * D);
+        if (S0) memcpy(H, S0 + h * DD, sizeof(double) * DD);
+        else memset(H, 0, sizeof(double) * DD);
+        if (quant) {
+            orc_quantize(D, qfmt, prec32, H, codes, scales);
+            orc_dequantize(D, qfmt, codes, scales, H);
+        }
+        for (int t = 0; t < T; ++t) {
+            const size_t th = (size_t)t * nh + h;
+            const double* kt = k + th * D;
+            const double* qt = q + th * D;
+            const double* vt = v + th * D;
+            const double* gt = g + th * Dg;
+            const double bt = beta[th];
+            for (int j = 0; j < D; ++j) a[j] = exp(gate_log(gt, Dg, j));
+            const int slot = Wp > 0 ? t % Wp : 0;
+            /* the pair written Wp steps ago leaves the window: into the history */
+            if (Wp > 0 && t >= Wp)
+                for (int i = 0; i < D; ++i)
+                    for (int j = 0; j < D; ++j)
+                        H[(size_t)i * D + j] += px[(size_t)slot * D + i] * py[(size_t)slot * D + j];
+            /* history: H <- H Diag(a) (I - beta k k^T) */
+            for (int i = 0; i < D; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < D; ++j) {
+                    H[(size_t)i * D + j] *= a[j];
+                    acc += H[(size_t)i * D + j] * kt[j];
+                }
+                w[i] = acc;
+            }
+            for (int i = 0; i < D; ++i)
+                for (int j = 0; j < D; ++j) H[(size_t)i * D + j] -= bt * w[i] * kt[j];
+            /* pairs still in the window (written at t-Wp+1 .. t-1): key side of the transition */
+            const int carried = Wp > 0 ? (t < Wp - 1 ? t : Wp - 1) : 0;
+            for (int p = 1; p <= carried; ++p) {
+                const int sl = (t - p) % Wp;
+                const double* y = py + (size_t)sl * D;
+                double* yn = pyn + (size_t)sl * D;
+                double ky = 0.0;
+                for (int j = 0; j < D; ++j) ky += kt[j] * a[j] * y[j];
+                for (int j = 0; j < D; ++j) yn[j] = a[j] * y[j] - bt * ky * kt[j];
+            }
+            /* the pure write of this step */
+            for (int i = 0; i < D; ++i) {
+                x[i] = bt * vt[i];
+                if (prec32) x[i] = orc_round_f32(x[i]);
+            }
+            if (Wp == 0)
+                for (int i = 0; i < D; ++i)
+                    for (int j = 0; j < D; ++j) H[(size_t)i * D + j] += x[i] * kt[j];
+            /* o_t = S_t q_t, before storage rounding */
+            if (o) {
+                double* ot = o + th * D;
+                for (int i = 0; i < D; ++i) {
+                    double acc = 0.0;
+                    for (int j = 0; j < D; ++j) acc += H[(size_t)i * D + j] * qt[j];
+                    ot[i] = acc;
+                }
+                for (int p = 1; p <= carried; ++p) {
+                    const int sl = (t - p) % Wp;
+                    double yq = 0.0;
+                    for (int j = 0; j < D; ++j) yq += pyn[(size_t)sl * D + j] * qt[j];
+                    for (int i = 0; i < D; ++i) ot[i] += px[(size_t)sl * D + i] * yq;
+                }
+                if (Wp > 0) {
+                    double kq = 0.0;
+                    for (int j = 0; j < D; ++j) kq += kt[j] * qt[j];
+                    for (int i = 0; i < D; ++i) ot[i] += x[i] * kq;
+                }
+            }
+            /* storage: history requantised (or fp32), carried keys and the new pair rounded */
+            if (quant) {
+                if (prec32)
+                    for (size_t e = 0; e < DD; ++e) H[e] = orc_round_f32(H[e]);
+                orc_quantize(D, qfmt, prec32, H, codes, scales);
+                orc_dequantize(D, qfmt, codes, scales, H);
+            } else if (prec32) {
+                for (size_t e = 0; e < DD; ++e) H[e] = orc_round_f32(H[e]);
+            }
+            for (int p = 1; p <= carried; ++p) {
+                const int sl = (t - p) % Wp;
+                double* y = py + (size_t)sl * D;
+                const double* yn = pyn + (size_t)sl * D;
+                if (fp8) orc_fp8_vector(D, prec32, yn, y);
+                else
+                    for (int j = 0; j < D; ++j) y[j] = prec32 ? orc_round_f32(yn[j]) : yn[j];
+            }
+            if (Wp > 0) {
+                double* xs = px + (size_t)slot * D;
+                double* ys = py + (size_t)slot * D;
+                if (fp8) {
+                    orc_fp8_vector(D, prec32, x, xs);
+                    orc_fp8_vector(D, prec32, kt, ys);
+                } else {
+                    memcpy(xs, x, sizeof(double) * D);
+                    for (int j = 0; j < D; ++j) ys[j] = prec32 ? orc_round_f32(kt[j]) : kt[j];
+                }
+            }
+        }
+        if (codes_out) memcpy(codes_out + h * DD, codes, DD);
+        if (scales_out) memcpy(scales_out + (size_t)h * D * ng, scales, sizeof(double) * (size_t)D * ng);
+        if (px_out && Wp > 0) memcpy(px_out + (size_t)h * Wp * D, px, sizeof(double) * (size_t)Wp * D);
+        if (py_out && Wp > 0) memcpy(py_out + (size_t)h * Wp * D, py, sizeof(double) * (size_t)Wp * D);
+        if (S_out) {
+            double* S = S_out + h * DD;
+            memcpy(S, H, sizeof(double) * DD);
+            const int live = T < Wp ? T : Wp;  /* pairs written at T-live .. T-1 */
+            for (int p = 1; p <= live; ++p) {
+                const int sl = (T - p) % Wp;
+                for (int i = 0; i < D; ++i)
+                    for (int j = 0; j < D; ++j)
+                        S[(size_t)i * D + j] += px[(size_t)sl * D + i] * py[(size_t)sl * D + j];
+            }
+        }
+        free(H); free(codes); free(scales); free(px); free(py); free(pyn);
+        free(a); free(w); free(x);
+    }
+    return 0;
 }

@@ -11,7 +11,8 @@ Kinds of pin used here:
     the delta-rule write identity at the written key;
   - agreement of independent formulations (literal matrix form, distributive plain form,
     buffered windows) where the mathematics says they are equal;
-  - library routines for special cases: numpy rint / argsort, torch's bf16 conversion.
+  - library routines for special cases: numpy rint / argsort, torch's bf16 and float8_e4m3fn
+    conversions.
 """
 from __future__ import annotations
 
@@ -398,6 +399,116 @@ def pin_storage_roundings(lib):
     close(res.o, exact.o, 2e-2, "storage roundings stay small")
 
 
+# ---------------------------------------------------------------------------------------------
+# PW: the pure-write sliding window
+# ---------------------------------------------------------------------------------------------
+def pin_golden_pure_write_window(lib):
+    gd = read("pure_write_window_2x2.txt")
+    D, T, Wp = 2, 3, 2
+    q, k, v = (gd[n].reshape(T, 1, D) for n in ("q", "k", "v"))
+    g = np.log(gd["a"]).reshape(T, 1)
+    beta = gd["beta"].reshape(T, 1)
+    S0 = gd["S0"].reshape(1, D, D)
+    res = oracle.pw_run(q, k, v, g, beta, Wp=Wp, S0=S0, lib=lib)
+    assert np.allclose(res.o.ravel(), gd["o"], atol=1e-12), ("PW o", res.o.ravel())
+    assert np.allclose(res.S.ravel(), gd["S3"], atol=1e-12), ("PW S3", res.S.ravel())
+    r2 = oracle.pw_run(q[:2], k[:2], v[:2], g[:2], beta[:2], Wp=Wp, S0=S0, lib=lib)
+    H2 = (r2.codes[0] * r2.scales[0]).ravel()       # int8: one scale per row
+    assert np.allclose(H2, gd["H2"], atol=1e-12), ("PW H2", H2)
+
+
+def pin_e4m3_rounding(lib):
+    """e4m3 against torch's float8_e4m3fn conversion (round to nearest even) on normals,
+    subnormals, exact ties and the largest finite value; the FP8 vector round trip against
+    s * e4m3(x / s) with s = absmax / 448 done through torch."""
+    rng = np.random.default_rng(12)
+    x = np.concatenate([
+        rng.uniform(-447.0, 447.0, 3000),
+        np.clip(rng.standard_normal(2000) * 2.0 ** rng.uniform(-12, 8, 2000), -460.0, 460.0),
+        np.array([2.0**-9, 2.0**-10, 3 * 2.0**-10, 5 * 2.0**-10, 1 + 2.0**-4, 1 + 3 * 2.0**-4,
+                  -(1 + 2.0**-4), 2.0**-6 * (1 + 2.0**-4), 17.0 * 2.0**-10, 448.0, -448.0,
+                  464.0 - 2.0**-6, 0.0]),
+    ]).astype(np.float32)
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([lib.orc_round_e4m3(float(t)) for t in x])
+    assert np.array_equal(got, want), np.flatnonzero(got != want)[:10]
+    # past 464 torch's conversion gives NaN; the saturating reading (a GPU's satfinite
+    # conversion) keeps the largest finite value
+    assert lib.orc_round_e4m3(500.0) == 448.0 and lib.orc_round_e4m3(-1e6) == -448.0
+    for n in (5, 128):
+        vec = rng.standard_normal(n) * 10.0 ** rng.uniform(-3, 3)
+        out, s = oracle.fp8_vector(vec, lib=lib)
+        ref_s = np.abs(vec).max() / 448.0
+        t = torch.from_numpy(vec / ref_s).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+        assert s == ref_s and np.allclose(out, ref_s * t, rtol=1e-15, atol=0), (n, out)
+        j = int(np.argmax(np.abs(vec)))
+        assert abs(out[j] - vec[j]) <= 1e-14 * abs(vec[j])   # the absmax entry is kept
+    out, s = oracle.fp8_vector(np.zeros(4), lib=lib)
+    assert s == 0.0 and not out.any()
+
+
+def pin_pw_exact_is_plain(lib):
+    """With an exact history and exact pairs the window only moves terms between two stores:
+    outputs and final state are the plain recurrence's, for every window length and gate."""
+    for gate, seed in (("scalar", 51), ("diag", 52)):
+        q, k, v, g, beta = rand_inputs(seed, 9, 2, 6, gate)
+        S0 = np.random.default_rng(seed).standard_normal((2, 6, 6))
+        o_ref, S_ref = oracle.plain_run(q, k, v, g, beta, S0=S0, lib=lib)
+        for Wp in (0, 1, 3, 12):
+            res = oracle.pw_run(q, k, v, g, beta, Wp=Wp, S0=S0, quant=False, fp8=False, lib=lib)
+            close(res.o, o_ref, 1e-12, f"PW exact o ({gate}, Wp={Wp})")
+            close(res.S, S_ref, 1e-12, f"PW exact S ({gate}, Wp={Wp})")
+
+
+def pin_pw_no_window_is_every_step_quantization(lib):
+    """Wp = 0: each write joins the history at once, which is then requantised: the literal
+    matrix form requantised after every step (window length 1)."""
+    for fmt, D in (("int8", 8), ("int4_g32", 32)):
+        for gate in ("scalar", "diag"):
+            q, k, v, g, beta = rand_inputs(61, 7, 2, D, gate)
+            S0 = np.random.default_rng(62).standard_normal((2, D, D))
+            o1, S1, _ = oracle.o1_run(q, k, v, g, beta, W=1, fmt=fmt, S0=S0, lib=lib)
+            res = oracle.pw_run(q, k, v, g, beta, Wp=0, fmt=fmt, S0=S0, lib=lib)
+            close(res.o, o1, 1e-12, f"PW Wp=0 o ({fmt}, {gate})")
+            close(res.S, S1, 1e-12, f"PW Wp=0 S ({fmt}, {gate})")
+
+
+def pin_pw_superposition(lib):
+    """When no pair leaves the window (Wp >= T) the writes never meet the quantizer: the state
+    is the history's own quantised evolution (the every-step-quantised recurrence with v = 0)
+    plus every write carried exactly (the plain recurrence from a zero state). The recurrence
+    is linear in S, so the outputs add up the same way."""
+    for gate in ("scalar", "diag"):
+        q, k, v, g, beta = rand_inputs(71, 6, 2, 8, gate)
+        S0 = np.random.default_rng(72).standard_normal((2, 8, 8))
+        oh, Sh, _ = oracle.o1_run(q, k, np.zeros_like(v), g, beta, W=1, fmt="int8", S0=S0,
+                                  lib=lib)
+        ow, Sw = oracle.plain_run(q, k, v, g, beta, lib=lib)
+        res = oracle.pw_run(q, k, v, g, beta, Wp=6, fmt="int8", S0=S0, fp8=False, lib=lib)
+        close(res.o, oh + ow, 1e-12, f"PW superposition o ({gate})")
+        close(res.S, Sh + Sw, 1e-12, f"PW superposition S ({gate})")
+
+
+def pin_pw_window_timing(lib):
+    """A write below half a quantization step of its row is visible in the outputs exactly
+    while it is in the window (steps tau .. tau + Wp - 1), and on the step it joins the history
+    (that step's output precedes the requantisation, which then rounds it away)."""
+    D, T, tau, eps = 2, 12, 2, 1e-3
+    S0 = np.array([[[1.0, 0.0], [1.0, 0.0]]])     # column 1 empty
+    q = np.tile(np.array([0.0, 1.0]), (T, 1, 1))   # read column 1
+    k = np.tile(np.array([0.0, 1.0]), (T, 1, 1))
+    v = np.zeros((T, 1, D))
+    v[tau, 0] = [eps, 0.0]
+    g = np.zeros((T, 1))                            # a = 1
+    beta = np.zeros((T, 1))
+    beta[tau] = 1.0                                 # the one write; otherwise no transition
+    for Wp in (0, 1, 3):
+        res = oracle.pw_run(q, k, v, g, beta, Wp=Wp, S0=S0, lib=lib)
+        want = np.zeros((T, 1, D))
+        want[tau: tau + Wp + 1, 0, 0] = eps
+        assert np.allclose(res.o, want, rtol=1e-12, atol=1e-18), (Wp, res.o[:, 0, 0])
+
+
 PINS = [
     pin_golden_delta_rule_kda,
     pin_golden_window_int8,
@@ -416,4 +527,10 @@ PINS = [
     pin_literal_equals_buffered_quantized,
     pin_compensator_decomposition,
     pin_storage_roundings,
+    pin_golden_pure_write_window,
+    pin_e4m3_rounding,
+    pin_pw_exact_is_plain,
+    pin_pw_no_window_is_every_step_quantization,
+    pin_pw_superposition,
+    pin_pw_window_timing,
 ]

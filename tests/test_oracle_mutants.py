@@ -82,6 +82,36 @@ MUTANTS = [
     ("bf16: one mantissa bit too many",
      "int qexp = e - 8;",
      "int qexp = e - 9;"),
+    ("PW: pair leaves the window one step late",
+     "if (Wp > 0 && t >= Wp)",
+     "if (Wp > 0 && t > Wp)"),
+    ("PW: carried keys not erased by later writes",
+     "yn[j] = a[j] * y[j] - bt * ky * kt[j];",
+     "yn[j] = a[j] * y[j];"),
+    ("PW: carried keys not gated",
+     "yn[j] = a[j] * y[j] - bt * ky * kt[j];",
+     "yn[j] = y[j] - bt * ky * kt[j];"),
+    ("PW: new write missing from the output",
+     "for (int i = 0; i < D; ++i) ot[i] += x[i] * kq;",
+     "for (int i = 0; i < D; ++i) ot[i] += 0.0 * x[i] * kq;"),
+    ("PW: carried pairs read with the key instead of the query",
+     "for (int j = 0; j < D; ++j) yq += pyn[(size_t)sl * D + j] * qt[j];",
+     "for (int j = 0; j < D; ++j) yq += pyn[(size_t)sl * D + j] * kt[j];"),
+    ("PW: history requantised only when a pair joins it",
+     "            if (quant) {\n                if (prec32)",
+     "            if (quant && (Wp == 0 || t >= Wp)) {\n                if (prec32)"),
+    ("PW: write vector without beta",
+     "x[i] = bt * vt[i];",
+     "x[i] = vt[i];"),
+    ("e4m3: one mantissa bit too many",
+     "int qexp = e - 4;",
+     "int qexp = e - 5;"),
+    ("e4m3: subnormal spacing too fine",
+     "if (qexp < -9) qexp = -9;",
+     "if (qexp < -10) qexp = -10;"),
+    ("FP8 vector: scale for a largest value of 240",
+     "double s = m / 448.0;",
+     "double s = m / 240.0;"),
 ]
 
 

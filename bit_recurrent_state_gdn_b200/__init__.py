@@ -1,6 +1,6 @@
 """Windowed low-bit recurrent-state GDN / KDA decode for B200 (sm_100a).
 
-Python face of libgdnq (include/gdnq.h): the functions here carry the C ABI's names and only
+Python face of libgdnq (include/gdnq.h, include/gdnq_pw.h): the functions here carry the C ABI's names and only
 marshal arguments -- torch tensors to device pointers, the current CUDA stream, status codes to
 exceptions. Every step of the computation runs in the library's CUDA kernels.
 """
@@ -18,4 +18,13 @@ from .api import (  # noqa: F401
     gdn_state_sizes,
     gdn_window_flush,
     make_config,
+)
+from .pw import (  # noqa: F401
+    PwState,
+    gdn_pw_decode_step,
+    gdn_pw_decode_steps,
+    gdn_pw_materialize,
+    gdn_pw_quantize,
+    gdn_pw_state_sizes,
+    make_pw_config,
 )

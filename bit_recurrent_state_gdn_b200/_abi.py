@@ -1,4 +1,4 @@
-"""ctypes declarations of libgdnq's C ABI (include/gdnq.h). Loading fails loudly when the
+"""ctypes declarations of libgdnq's C ABI (include/gdnq.h, include/gdnq_pw.h). Loading fails loudly when the
 library has not been built: there is no fallback path."""
 from __future__ import annotations
 
@@ -13,6 +13,7 @@ GDN_GATE_SCALAR, GDN_GATE_DIAG = 0, 1
 GDN_FMT_INT8, GDN_FMT_INT4_G32, GDN_FMT_BF16, GDN_FMT_FP32, GDN_FMT_MIXED = 0, 1, 2, 3, 4
 GDN_DTYPE_F32, GDN_DTYPE_BF16 = 0, 1
 GDN_MAX_COMPENSATORS = 16
+GDN_PW_MAX_WINDOW = 16
 
 _i32 = ctypes.c_int32
 _vp = ctypes.c_void_p
@@ -40,7 +41,27 @@ class gdn_sizes(ctypes.Structure):
     _fields_ = [(n, _sz) for n in SIZE_FIELDS]
 
 
-# name -> (restype, argtypes); every symbol include/gdnq.h declares
+class gdn_pw_config(ctypes.Structure):
+    _fields_ = [(n, _i32) for n in ("B", "H", "d", "Wp", "gate", "fmt", "act_dtype")]
+
+
+PW_STATE_FIELDS = ("codes", "scales", "pairs", "pscales", "count", "status")
+
+
+class gdn_pw_state(ctypes.Structure):
+    _fields_ = [(n, _vp) for n in PW_STATE_FIELDS]
+
+
+PW_SIZE_FIELDS = ("codes", "scales", "pairs", "pscales", "count")
+
+
+class gdn_pw_sizes(ctypes.Structure):
+    _fields_ = [(n, _sz) for n in PW_SIZE_FIELDS]
+
+
+_PWC, _PWS = ctypes.POINTER(gdn_pw_config), ctypes.POINTER(gdn_pw_state)
+
+# name -> (restype, argtypes); every symbol include/gdnq.h and include/gdnq_pw.h declare
 SIGNATURES = {
     "gdn_state_sizes": (_i32, [ctypes.POINTER(gdn_config), ctypes.POINTER(gdn_sizes)]),
     "gdn_state_quantize": (_i32, [ctypes.POINTER(gdn_config), _vp, ctypes.POINTER(gdn_state), _vp]),
@@ -57,6 +78,11 @@ SIGNATURES = {
     "gdn_state_materialize": (_i32, [ctypes.POINTER(gdn_config), ctypes.POINTER(gdn_state), _vp,
                                      _vp]),
     "gdn_baseline_step": (_i32, [ctypes.POINTER(gdn_config)] + [_vp] * 8),
+    "gdn_pw_state_sizes": (_i32, [_PWC, ctypes.POINTER(gdn_pw_sizes)]),
+    "gdn_pw_quantize": (_i32, [_PWC, _vp, _PWS, _vp]),
+    "gdn_pw_decode_step": (_i32, [_PWC, _PWS] + [_vp] * 7),
+    "gdn_pw_decode_steps": (_i32, [_PWC, _PWS, _i32] + [_vp] * 7),
+    "gdn_pw_materialize": (_i32, [_PWC, _PWS, _vp, _vp]),
     "gdn_status_string": (ctypes.c_char_p, [_i32]),
     "gdn_last_error": (ctypes.c_char_p, []),
 }

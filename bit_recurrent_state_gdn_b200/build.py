@@ -19,7 +19,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OBJ_DIR = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libgdnq.so")
-SOURCES = ["api.cu", "window_int8.cu", "window_int4.cu", "window_mixed.cu", "baseline.cu"]
+SOURCES = ["api.cu", "window_int8.cu", "window_int4.cu", "window_mixed.cu", "baseline.cu",
+           "pw.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -40,7 +41,7 @@ def _flags(ptxas_info: bool) -> list[str]:
 
 def _deps() -> list[str]:
     files = [os.path.join(CSRC, n) for n in os.listdir(CSRC)]
-    return files + [os.path.join(INCLUDE, "gdnq.h")]
+    return files + [os.path.join(INCLUDE, n) for n in ("gdnq.h", "gdnq_pw.h")]
 
 
 def _stale() -> bool:

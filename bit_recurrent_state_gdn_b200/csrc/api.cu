@@ -7,7 +7,9 @@
 
 #include "baseline_kernels.cuh"
 #include "gdnq.h"
+#include "gdnq_pw.h"
 #include "launch.h"
+#include "pw_kernels.cuh"
 #include "window_kernels.cuh"
 
 // Staging of gdn_decode_window_steps_host_fixed: one fixed array per device, reserved when the
@@ -213,6 +215,91 @@ size_t window_smem_bytes(const gdn_config& c) {
 }
 
 }  // namespace gdnq
+
+
+// ---- pure-write sliding window ----------------------------------------------------------------
+namespace {
+
+int64_t pw_heads(const gdn_pw_config* c) { return (int64_t)c->B * (int64_t)c->H; }
+size_t pw_act_size(const gdn_pw_config* c) { return c->act_dtype == GDN_DTYPE_F32 ? 4 : 2; }
+
+gdn_status check_pw_config(const gdn_pw_config* c) {
+  if (!c) return fail(GDN_ERR_INVALID_ARG, "cfg is null");
+  if (c->B < 0 || c->H < 0) return fail(GDN_ERR_INVALID_ARG, "B=%d, H=%d must be >= 0", c->B, c->H);
+  if (pw_heads(c) > INT32_MAX) return fail(GDN_ERR_INVALID_ARG, "B*H exceeds 2^31-1");
+  if (c->gate != GDN_GATE_SCALAR && c->gate != GDN_GATE_DIAG)
+    return fail(GDN_ERR_INVALID_ARG, "gate=%d is not a gdn_gate_kind", c->gate);
+  if (c->fmt != GDN_FMT_INT8 && c->fmt != GDN_FMT_INT4_G32)
+    return fail(GDN_ERR_INVALID_ARG, "the history needs fmt INT8 or INT4_G32 (got %d)", c->fmt);
+  if (c->act_dtype != GDN_DTYPE_F32 && c->act_dtype != GDN_DTYPE_BF16)
+    return fail(GDN_ERR_INVALID_ARG, "act_dtype=%d is not a gdn_dtype", c->act_dtype);
+  if (c->d < 1) return fail(GDN_ERR_INVALID_ARG, "d=%d", c->d);
+  if (c->d != 128) return fail(GDN_ERR_UNSUPPORTED, "head size %d is not built (128)", c->d);
+  if (c->Wp < 0) return fail(GDN_ERR_INVALID_ARG, "Wp=%d must be >= 0", c->Wp);
+  if (c->Wp > GDN_PW_MAX_WINDOW)
+    return fail(GDN_ERR_UNSUPPORTED, "Wp=%d exceeds %d", c->Wp, GDN_PW_MAX_WINDOW);
+  return GDN_OK;
+}
+
+struct PwPerHead {
+  size_t codes, scales, pairs, pscales;
+};
+
+PwPerHead pw_per_head(const gdn_pw_config* c) {
+  const size_t D = (size_t)c->d;
+  const bool int4 = c->fmt == GDN_FMT_INT4_G32;
+  PwPerHead p;
+  p.codes = int4 ? D * D / 2 : D * D;
+  p.scales = 4 * (int4 ? D * (D / 32) : D);
+  p.pairs = 2 * (size_t)c->Wp * D;
+  p.pscales = 8 * (size_t)round4(c->Wp);
+  return p;
+}
+
+gdn_status check_pw_state(const gdn_pw_config* c, const gdn_pw_state* s) {
+  if (!s) return fail(GDN_ERR_INVALID_ARG, "state is null");
+  gdn_status st;
+  if ((st = need_ptr(s->codes, "state.codes")) != GDN_OK) return st;
+  if ((st = need_ptr(s->scales, "state.scales")) != GDN_OK) return st;
+  if ((st = need_ptr(s->count, "state.count", 4)) != GDN_OK) return st;
+  if (c->Wp > 0) {
+    if ((st = need_ptr(s->pairs, "state.pairs")) != GDN_OK) return st;
+    if ((st = need_ptr(s->pscales, "state.pscales")) != GDN_OK) return st;
+  }
+  if (s->status && (reinterpret_cast<uintptr_t>(s->status) & 3u) != 0)
+    return fail(GDN_ERR_INVALID_ARG, "state.status is not 4-byte aligned");
+  return GDN_OK;
+}
+
+gdnq::PwArgs make_pw_args(const gdn_pw_config* c, const gdn_pw_state* s) {
+  gdnq::PwArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.codes = static_cast<uint8_t*>(s->codes);
+  a.scales = s->scales;
+  a.pairs = s->pairs;
+  a.pscales = s->pscales;
+  a.count = s->count;
+  a.status = s->status;
+  a.Wp = c->Wp;
+  return a;
+}
+
+// The window configuration whose quantize kernel writes the same history layout.
+gdn_config pw_as_window(const gdn_pw_config* c) {
+  gdn_config w;
+  std::memset(&w, 0, sizeof w);
+  w.B = c->B;
+  w.H = c->H;
+  w.d_k = w.d_v = c->d;
+  w.W = 1;
+  w.r = 0;
+  w.gate = c->gate;
+  w.fmt = c->fmt;
+  w.act_dtype = w.buf_dtype = c->act_dtype;
+  return w;
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -486,6 +573,97 @@ gdn_status gdn_baseline_step(const gdn_config* cfg, void* S, const void* q, cons
   gdnq::BaseArgs a{S, q, k, v, g, beta, o};
   cudaError_t e = gdnq::launch_baseline(*cfg, a, (int)heads_of(cfg), (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "gdn_baseline_step");
+  return GDN_OK;
+}
+
+gdn_status gdn_pw_state_sizes(const gdn_pw_config* cfg, gdn_pw_sizes* out) {
+  g_last_error[0] = 0;
+  if (!out) return fail(GDN_ERR_INVALID_ARG, "out is null");
+  gdn_status st = check_pw_config(cfg);
+  if (st != GDN_OK) return st;
+  const PwPerHead p = pw_per_head(cfg);
+  const size_t n = (size_t)pw_heads(cfg);
+  out->codes = n * p.codes;
+  out->scales = n * p.scales;
+  out->pairs = n * p.pairs;
+  out->pscales = cfg->Wp > 0 ? n * p.pscales : 0;
+  out->count = n * 4;
+  return GDN_OK;
+}
+
+gdn_status gdn_pw_quantize(const gdn_pw_config* cfg, const float* S, const gdn_pw_state* state,
+                           gdn_stream_t stream) {
+  g_last_error[0] = 0;
+  gdn_status st = check_pw_config(cfg);
+  if (st != GDN_OK) return st;
+  if (pw_heads(cfg) == 0) return GDN_OK;
+  if ((st = check_pw_state(cfg, state)) != GDN_OK) return st;
+  if ((st = need_ptr(S, "S")) != GDN_OK) return st;
+  const gdn_config w = pw_as_window(cfg);
+  gdnq::WinArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.codes = static_cast<uint8_t*>(state->codes);
+  a.scales = state->scales;
+  a.pos = state->count;  // the quantize kernel empties the window: count = 0
+  a.status = state->status;
+  a.S_in = S;
+  const PwPerHead ph = pw_per_head(cfg);
+  a.code_stride = (uint32_t)ph.codes;
+  a.scale_stride = (uint32_t)(ph.scales / 4);
+  a.H = cfg->H;
+  a.W = 1;
+  a.r = 0;
+  return launch(gdnq::WinOp::Quantize, &w, a, stream, "gdn_pw_quantize");
+}
+
+gdn_status gdn_pw_decode_step(const gdn_pw_config* cfg, const gdn_pw_state* state, const void* q,
+                              const void* k, const void* v, const float* g, const float* beta,
+                              void* o, gdn_stream_t stream) {
+  return gdn_pw_decode_steps(cfg, state, 1, q, k, v, g, beta, o, stream);
+}
+
+gdn_status gdn_pw_decode_steps(const gdn_pw_config* cfg, const gdn_pw_state* state, int32_t T,
+                               const void* q, const void* k, const void* v, const float* g,
+                               const float* beta, void* o, gdn_stream_t stream) {
+  g_last_error[0] = 0;
+  gdn_status st = check_pw_config(cfg);
+  if (st != GDN_OK) return st;
+  if (T < 0) return fail(GDN_ERR_INVALID_ARG, "T=%d must be >= 0", T);
+  if (pw_heads(cfg) == 0 || T == 0) return GDN_OK;
+  if ((st = check_pw_state(cfg, state)) != GDN_OK) return st;
+  const gdn_config w = pw_as_window(cfg);
+  if ((st = check_inputs(&w, q, k, v, g, beta, o, true)) != GDN_OK) return st;
+  const size_t H = (size_t)pw_heads(cfg), D = (size_t)cfg->d;
+  const size_t act_step = H * D * pw_act_size(cfg);
+  const size_t g_step = H * (cfg->gate == GDN_GATE_DIAG ? D : 1);
+  gdnq::PwArgs a = make_pw_args(cfg, state);
+  for (int32_t t = 0; t < T; ++t) {
+    a.q = static_cast<const uint8_t*>(q) + t * act_step;
+    a.k = static_cast<const uint8_t*>(k) + t * act_step;
+    a.v = static_cast<const uint8_t*>(v) + t * act_step;
+    a.g = g + t * g_step;
+    a.beta = beta + t * H;
+    a.o = static_cast<uint8_t*>(o) + t * act_step;
+    const cudaError_t e =
+        gdnq::launch_pw(gdnq::PwOp::Step, *cfg, a, (int)H, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "gdn_pw_decode_step");
+  }
+  return GDN_OK;
+}
+
+gdn_status gdn_pw_materialize(const gdn_pw_config* cfg, const gdn_pw_state* state, float* S,
+                              gdn_stream_t stream) {
+  g_last_error[0] = 0;
+  gdn_status st = check_pw_config(cfg);
+  if (st != GDN_OK) return st;
+  if (pw_heads(cfg) == 0) return GDN_OK;
+  if ((st = check_pw_state(cfg, state)) != GDN_OK) return st;
+  if ((st = need_ptr(S, "S")) != GDN_OK) return st;
+  gdnq::PwArgs a = make_pw_args(cfg, state);
+  a.S_out = S;
+  const cudaError_t e = gdnq::launch_pw(gdnq::PwOp::Materialize, *cfg, a, (int)pw_heads(cfg),
+                                        (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "gdn_pw_materialize");
   return GDN_OK;
 }
 

@@ -142,6 +142,54 @@ __device__ __forceinline__ float rint_quotient(float x, float s, float inv) {
   return r;
 }
 
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic, round to nearest) -------------------------
+struct F2 {
+  uint64_t v;
+};
+__device__ __forceinline__ F2 f2(float lo, float hi) {
+  F2 r;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(r.v) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_get(F2 a, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(lo), "=f"(hi) : "l"(a.v));
+}
+__device__ __forceinline__ F2 f2_fma(F2 a, F2 b, F2 c) {
+  F2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(d.v) : "l"(a.v), "l"(b.v), "l"(c.v));
+  return d;
+}
+__device__ __forceinline__ F2 f2_mul(F2 a, F2 b) {
+  F2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;\n" : "=l"(d.v) : "l"(a.v), "l"(b.v));
+  return d;
+}
+__device__ __forceinline__ F2 f2_add(F2 a, F2 b) {
+  F2 d;
+  asm("add.rn.f32x2 %0, %1, %2;\n" : "=l"(d.v) : "l"(a.v), "l"(b.v));
+  return d;
+}
+
+// Correctly rounded quotients x / s of a pair, from inv = the correctly rounded 1 / s and
+// ninv_s = -s: q1 = x * inv is within one ulp of x / s, the remainder x - q1 s is exact in one
+// fma, and q1 + remainder * inv rounded once is the correctly rounded quotient (Markstein's
+// correction: P. Markstein, IBM J. Res. Dev. 34(1), 1990; also Muller et al., Handbook of
+// Floating-Point Arithmetic, the theorem on correcting a quotient with an fma). Valid while
+// x / s and 1 / s are normal and finite.
+__device__ __forceinline__ F2 f2_quot(F2 x, F2 inv, F2 neg_s) {
+  const F2 q1 = f2_mul(x, inv);
+  const F2 r = f2_fma(q1, neg_s, x);
+  return f2_fma(r, inv, q1);
+}
+
+// The correctly rounded quotient x / d for a constant divisor d, given inv_d = the correctly
+// rounded 1 / d (the same correction, scalar). Valid while x / d is normal or zero.
+__device__ __forceinline__ float quot_const(float x, float d, float inv_d) {
+  const float q1 = x * inv_d;
+  const float r = fmaf(-q1, d, x);
+  return fmaf(r, inv_d, q1);
+}
+
 // ---- exact conversions -------------------------------------------------------------------
 // Four int8 codes (two's complement, byte e = code e) to fp32: bias each byte to b + 128,
 // place it in the mantissa of 2^23 (0x4B0000xx = 2^23 + xx) and subtract 2^23 + 128.
@@ -162,6 +210,30 @@ __device__ __forceinline__ void i4x8_to_f32(uint32_t w, float* f) {
   for (int m = 0; m < 4; ++m) {
     f[2 * m] = __uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650 + m)) - 8388616.f;
     f[2 * m + 1] = __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650 + m)) - 8388616.f;
+  }
+}
+
+// The same two conversions with the bias subtractions done on packed pairs.
+__device__ __forceinline__ void i8x4_to_f32_2(uint32_t w, float* f) {
+  const uint32_t x = w ^ 0x80808080u;
+  const F2 bias = f2(-8388736.f, -8388736.f);
+  const F2 a = f2_add(f2(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7650)),
+                         __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7651))), bias);
+  const F2 b = f2_add(f2(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7652)),
+                         __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7653))), bias);
+  f2_get(a, f[0], f[1]);
+  f2_get(b, f[2], f[3]);
+}
+
+__device__ __forceinline__ void i4x8_to_f32_2(uint32_t w, float* f) {
+  const uint32_t x = w ^ 0x88888888u;
+  const uint32_t lo = x & 0x0F0F0F0Fu, hi = (x >> 4) & 0x0F0F0F0Fu;
+  const F2 bias = f2(-8388616.f, -8388616.f);
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const F2 v = f2_add(f2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650 + m)),
+                           __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650 + m))), bias);
+    f2_get(v, f[2 * m], f[2 * m + 1]);
   }
 }
 

@@ -4,11 +4,13 @@
 #include <cuda_runtime.h>
 
 #include "gdnq.h"
+#include "gdnq_pw.h"
 
 namespace gdnq {
 
 struct WinArgs;
 struct BaseArgs;
+struct PwArgs;
 
 enum class WinOp { Step, Flush, Materialize, Quantize };
 
@@ -30,6 +32,11 @@ cudaError_t launch_window_int4(WinOp op, const gdn_config& cfg, const WinArgs& a
                                cudaStream_t stream);
 cudaError_t launch_window_mixed(WinOp op, const gdn_config& cfg, const WinArgs& a, int heads,
                                 cudaStream_t stream);
+// Pure-write sliding window: the persistent decode step, or the materialisation (one CTA per
+// head), over `heads` heads.
+enum class PwOp { Step, Materialize };
+cudaError_t launch_pw(PwOp op, const gdn_pw_config& cfg, const PwArgs& a, int heads,
+                      cudaStream_t stream);
 cudaError_t launch_baseline(const gdn_config& cfg, const BaseArgs& a, int heads,
                             cudaStream_t stream);
 

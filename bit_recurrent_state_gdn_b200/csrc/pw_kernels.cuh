@@ -1,0 +1,690 @@
+// Pure-write sliding window kernels ("Low-Bit GDN Recurrent-State Quantization: Global
+// Gradient-aware Allocation and Pure-Write Sliding Windows", Abstract): a low-bit history that
+// takes every step's transition and is requantised every step, plus the last Wp pure writes as
+// FP8 (e4m3) vector pairs carried through the transition on their key side.
+//
+// The decode step is one persistent kernel: each CTA walks a contiguous range of heads, one
+// thread bulk-copies each head's history tile, pairs and inputs into a ring of shared-memory
+// stages ahead of the compute, and the new history tile is written back from the same stage
+// with a bulk store. Within a head the work is elementwise plus length-D dot products, so it
+// runs on the FP32 pipes; 256 threads split the rows two to a row, each thread holding its half
+// row of the new history in registers between the absmax and the requantisation.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
+#include "device_util.cuh"
+#include "gdnq_pw.h"
+#include "mma_util.cuh"
+
+namespace gdnq {
+
+constexpr int kPwThreads = 256;
+constexpr int kPwIssuer = kPwThreads - 1;  // lane 31 of the last warp stages the copies
+constexpr int kPwMaxStages = 4;
+constexpr int kPwMaxHeadsPerCta = 1024;
+
+// CTAs per SM the step kernel is built for: an int4 history leaves registers for three.
+template <class P>
+constexpr int pw_ctas_per_sm() {
+  return P::INT4 ? 3 : 2;
+}
+
+template <bool DIAG_, bool INT4_, typename Act_>
+struct PwCfg {
+  static constexpr int D = 128;
+  static constexpr bool DIAG = DIAG_;
+  static constexpr bool INT4 = INT4_;
+  using Act = Act_;
+  static constexpr int QMAX = INT4 ? 7 : 127;
+  static constexpr int GS = INT4 ? 32 : D;  // columns per scale
+  static constexpr int NG = D / GS;
+  static constexpr int ROW_BYTES = INT4 ? D / 2 : D;
+  static constexpr int CODE_BYTES = D * ROW_BYTES;
+  static constexpr int NSCALES = D * NG;
+  static constexpr int COLS = D / 2;  // columns per thread (two threads per row)
+  static_assert(kPwThreads == 2 * D, "two threads per history row");
+};
+
+struct PwArgs {
+  uint8_t* codes;
+  float* scales;
+  uint8_t* pairs;
+  float* pscales;
+  int32_t* count;
+  int32_t* status;
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;
+  const float* beta;
+  void* o;
+  float* S_out;
+  int Wp;
+};
+
+__device__ __forceinline__ void pw_report(int32_t* status, int bit) {
+  if (status) atomicOr(status, bit);
+}
+
+// Shared-memory layout (byte offsets). A stage holds one head's history tile (codes, scales),
+// its pairs and pair scales, and the step's q, k, v (and g for the diagonal gate). After the
+// stages: per-head fp32 vectors, a few scalars and pair coefficients, the CTA's per-head
+// count / g / beta, and the stage barriers.
+struct PwLayout {
+  uint32_t codes, scales, pairs, pscales, q, k, v, g, stage_bytes;
+  uint32_t vec, frag, meta, bars, total;
+};
+
+constexpr int kPwVecs = 9;      // k, q, a, a.k, a.q, a.y_o, x_o, p, r
+constexpr int kPwScalars = 64;  // [0] <k,q>, [1] <y_o,a.k>, [2] <y_o,a.q>, [3] a (scalar gate),
+                                // [4..5] digit units,
+                                // [16..31] pair coefficients
+constexpr int kPwFragBytes = 1024;  // the digit right-hand side of the tensor-core mat-vec
+
+__host__ __device__ constexpr uint32_t pw_align(uint32_t x, uint32_t a) {
+  return (x + a - 1) & ~(a - 1);
+}
+
+template <class P>
+__host__ __device__ inline PwLayout pw_layout(int Wp, int nstages, int per_cta) {
+  PwLayout L;
+  const uint32_t Wr = (uint32_t)((Wp + 3) & ~3);
+  const uint32_t act = (uint32_t)(P::D * sizeof(typename P::Act));
+  uint32_t o = 0;
+  L.codes = o;
+  o += P::CODE_BYTES;
+  L.scales = o;
+  o += 4u * P::NSCALES;
+  L.pairs = o;
+  o += 2u * (uint32_t)Wp * P::D;
+  L.pscales = o;
+  o += 8u * Wr;
+  L.q = o;
+  o += act;
+  L.k = o;
+  o += act;
+  L.v = o;
+  o += act;
+  L.g = o;
+  if (P::DIAG) o += 4u * P::D;
+  L.stage_bytes = pw_align(o, 128);
+  o = (uint32_t)nstages * L.stage_bytes;
+  L.vec = o;
+  o += 4u * (kPwVecs * P::D + kPwScalars);
+  L.frag = o;
+  o += kPwFragBytes;
+  L.meta = o;
+  o += pw_align(12u * (uint32_t)per_cta, 16);
+  L.bars = o;
+  o += 8u * kPwMaxStages;
+  L.total = pw_align(o, 128);
+  return L;
+}
+
+// ---- bulk stores (shared -> global), completed per bulk group ----------------------------
+__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(dst),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
+}
+// Waits until every committed bulk store has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
+}
+// Waits until every committed bulk store has completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
+}
+
+// ---- e4m3 ----------------------------------------------------------------------------------
+// Four e4m3 codes (byte e = element e) to fp32, through the exact e4m3 -> f16 conversion.
+__device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float* f) {
+  const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xFFFFu), __NV_E4M3);
+  const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
+  const float2 a = __half22float2(__half2(lo)), b = __half22float2(__half2(hi));
+  f[0] = a.x;
+  f[1] = a.y;
+  f[2] = b.x;
+  f[3] = b.y;
+}
+
+// Four fp32 values to e4m3 codes (round to nearest even, saturating), byte e = element e.
+__device__ __forceinline__ uint32_t f32x4_to_e4m3(const float* t) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(t[0], t[1]), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(t[2], t[3]), __NV_SATFINITE, __NV_E4M3);
+  return (lo & 0xFFFFu) | (hi << 16);
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
+  return x;
+}
+
+// A warp stores a D = 128 vector (4 elements per lane) as e4m3 codes with one scale:
+// s = absmax / 448 and codes e4m3(x / s), both quotients correctly rounded (a zero vector gets
+// s = 0 and codes 0).
+__device__ __forceinline__ void pw_store_fp8(const float* x, uint8_t* dst, float* dst_scale) {
+  const float m = warp_max(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3]))));
+  const float s = m >= 0x1p-100f ? quot_const(m, 448.f, 1.f / 448.f) : __fdiv_rn(m, 448.f);
+  float t[4] = {0.f, 0.f, 0.f, 0.f};
+  if (s >= 0x1p-125f) {
+    const float inv = __frcp_rn(s);
+    const F2 inv2 = f2(inv, inv), ns = f2(-s, -s);
+    f2_get(f2_quot(f2(x[0], x[1]), inv2, ns), t[0], t[1]);
+    f2_get(f2_quot(f2(x[2], x[3]), inv2, ns), t[2], t[3]);
+  } else if (s > 0.f) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) t[e] = __fdiv_rn(x[e], s);
+  }
+  *reinterpret_cast<uint32_t*>(dst + 4 * (threadIdx.x & 31)) = f32x4_to_e4m3(t);
+  if ((threadIdx.x & 31) == 0) *dst_scale = s;
+}
+
+template <class P>
+__device__ __forceinline__ void pw_issue(const PwArgs& a, const PwLayout& L, uint8_t* st,
+                                         uint64_t* bar, int head) {
+  constexpr int D = P::D;
+  using Act = typename P::Act;
+  const int Wp = a.Wp, Wr = (Wp + 3) & ~3;
+  const uint32_t act = D * sizeof(Act);
+  uint32_t bytes = P::CODE_BYTES + 4u * P::NSCALES + 3u * act + (P::DIAG ? 4u * D : 0u);
+  if (Wp > 0) bytes += 2u * Wp * D + 8u * Wr;
+  mbar_arrive_expect_tx(bar, bytes);
+  bulk_g2s(st + L.codes, a.codes + (size_t)head * P::CODE_BYTES, P::CODE_BYTES, bar);
+  bulk_g2s(st + L.scales, a.scales + (size_t)head * P::NSCALES, 4u * P::NSCALES, bar);
+  if (Wp > 0) {
+    bulk_g2s(st + L.pairs, a.pairs + (size_t)head * 2 * Wp * D, 2u * Wp * D, bar);
+    bulk_g2s(st + L.pscales, a.pscales + (size_t)head * 2 * Wr, 8u * Wr, bar);
+  }
+  bulk_g2s(st + L.q, static_cast<const Act*>(a.q) + (size_t)head * D, act, bar);
+  bulk_g2s(st + L.k, static_cast<const Act*>(a.k) + (size_t)head * D, act, bar);
+  bulk_g2s(st + L.v, static_cast<const Act*>(a.v) + (size_t)head * D, act, bar);
+  if constexpr (P::DIAG) bulk_g2s(st + L.g, a.g + (size_t)head * D, 4u * D, bar);
+}
+
+__device__ __forceinline__ bool pw_count_ok(int cnt, int Wp) {
+  return Wp == 0 ? cnt == 0 : (cnt >= 0 && cnt < 2 * Wp);
+}
+
+// One head's step. All 256 threads; `st` holds the head's staged data. On return the stage
+// holds the new history tile (codes, scales) for the bulk store; pairs, o and count are stored.
+//   phase 0  fp32 vectors k, q, a, a.k, a.q                                   (threads 0..127)
+//   phase 1  warps 0-3: a.k and a.q as exact integer digits for the tensor cores; all warps,
+//            last first: the new pair, the leaving pair, the carried pairs (FP8 round trips)
+//   phase 2  warp w, rows 16w..16w+15: p = (dequant H) a.k and r = (dequant H) a.q on the
+//            integer tensor cores (mma.m16n8k32.s8, exact int32 sums of code x digit), then two
+//            threads per row form the new row, its absmax per scale group and its codes.
+template <class P>
+__device__ __forceinline__ void pw_head(const PwArgs& a, const PwLayout& L, uint8_t* sm,
+                                        uint8_t* st, int head, int cnt, float gs, float bt) {
+  constexpr int D = P::D;
+  using Act = typename P::Act;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int Wp = a.Wp, Wr = (Wp + 3) & ~3;
+  float* vec = reinterpret_cast<float*>(sm + L.vec);
+  float *kf = vec, *qf = vec + D, *A = vec + 2 * D, *ak = vec + 3 * D, *aq = vec + 4 * D;
+  float *Y = vec + 5 * D, *xo = vec + 6 * D, *PR = vec + 7 * D, *RR = vec + 8 * D;
+  float* sc = vec + 9 * D;
+  float* cp = sc + 16;
+  uint8_t* Bfrag = sm + L.frag;
+  const Act* sq = reinterpret_cast<const Act*>(st + L.q);
+  const Act* sk = reinterpret_cast<const Act*>(st + L.k);
+  const Act* sv = reinterpret_cast<const Act*>(st + L.v);
+  const uint8_t* spx = st + L.pairs;                   // [0][slot][D]
+  const uint8_t* spy = st + L.pairs + (size_t)Wp * D;  // [1][slot][D]
+  const float* ssx = reinterpret_cast<const float*>(st + L.pscales);
+  const float* ssy = ssx + Wr;
+  const int full = (Wp > 0 && cnt >= Wp) ? 1 : 0;
+  const int fill = min(cnt, Wp);
+  const int carried = fill - full;
+  const int slot_new = Wp > 0 ? (cnt >= Wp ? cnt - Wp : cnt) : 0;
+
+  // ---- phase 0 ------------------------------------------------------------------------------
+  if (tid < D) {
+    const float kj = Num<Act>::to_f(sk[tid]), qj = Num<Act>::to_f(sq[tid]);
+    float aj;
+    if constexpr (P::DIAG) {
+      aj = expf(reinterpret_cast<const float*>(st + L.g)[tid]);
+    } else {
+      aj = expf(gs);  // one value, formed the same way by every thread
+      if (tid == 0) sc[3] = aj;
+    }
+    kf[tid] = kj;
+    qf[tid] = qj;
+    A[tid] = aj;
+    ak[tid] = aj * kj;
+    aq[tid] = aj * qj;
+  }
+  __syncthreads();
+
+  // ---- phase 1 ------------------------------------------------------------------------------
+  if (warp < 4) {
+    // one block exponent per vector, found by every warp from all 128 columns
+    float mx = 0.f, my = 0.f;
+#pragma unroll
+    for (int mm = 0; mm < 4; ++mm) {
+      mx = fmaxf(mx, fabsf(ak[lane + 32 * mm]));
+      my = fmaxf(my, fabsf(aq[lane + 32 * mm]));
+    }
+    mx = warp_max(mx);
+    my = warp_max(my);
+    const float ux = put_digits<P::INT4>(Bfrag, 0, tid, ak[tid], mx);
+    const float uy = put_digits<P::INT4>(Bfrag, 3, tid, aq[tid], my);
+    if (tid == 0) {
+      sc[4] = ux;
+      sc[5] = uy;
+    }
+  }
+  const int j0 = 4 * lane;
+  uint8_t* gpx = a.pairs + (size_t)head * 2 * Wp * D;
+  uint8_t* gpy = gpx + (size_t)Wp * D;
+  float* gsx = a.pscales + (size_t)head * 2 * Wr;
+  float* gsy = gsx + Wr;
+  for (int task = 7 - warp; task < carried + 2; task += kPwThreads / 32) {
+    if (task == 0) {  // <k, q> and the new pair (beta v, k)
+      float kq = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) kq += kf[j0 + e] * qf[j0 + e];
+      kq = warp_sum(kq);
+      if (lane == 0) sc[0] = kq;
+      if (Wp > 0) {
+        float x[4], y[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          x[e] = bt * Num<Act>::to_f(sv[j0 + e]);
+          y[e] = kf[j0 + e];
+        }
+        pw_store_fp8(x, gpx + (size_t)slot_new * D, gsx + slot_new);
+        pw_store_fp8(y, gpy + (size_t)slot_new * D, gsy + slot_new);
+      }
+    } else if (task == 1) {  // the pair leaving the window joins the history (or nothing)
+      float yak = 0.f, yaq = 0.f;
+      if (full) {
+        float x[4], y[4];
+        e4m3x4_to_f32(*reinterpret_cast<const uint32_t*>(spx + (size_t)slot_new * D + j0), x);
+        e4m3x4_to_f32(*reinterpret_cast<const uint32_t*>(spy + (size_t)slot_new * D + j0), y);
+        const float sx = ssx[slot_new], sy = ssy[slot_new];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float yv = sy * y[e];
+          xo[j0 + e] = sx * x[e];
+          Y[j0 + e] = A[j0 + e] * yv;
+          yak += yv * ak[j0 + e];
+          yaq += yv * aq[j0 + e];
+        }
+        yak = warp_sum(yak);
+        yaq = warp_sum(yaq);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) xo[j0 + e] = Y[j0 + e] = 0.f;
+      }
+      if (lane == 0) {
+        sc[1] = yak;
+        sc[2] = yaq;
+      }
+    } else {  // a carried pair: key side through the transition
+      const int p = task - 1;  // written p writes ago
+      int sl = slot_new - p;
+      if (sl < 0) sl += Wp;
+      float y[4], yn[4];
+      e4m3x4_to_f32(*reinterpret_cast<const uint32_t*>(spy + (size_t)sl * D + j0), y);
+      const float sy = ssy[sl];
+      float d = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        y[e] = A[j0 + e] * (sy * y[e]);
+        d += kf[j0 + e] * y[e];
+      }
+      d = bt * warp_sum(d);
+      float cq = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        yn[e] = y[e] - d * kf[j0 + e];
+        cq += yn[e] * qf[j0 + e];
+      }
+      cq = warp_sum(cq);
+      if (lane == 0) cp[sl] = cq;
+      pw_store_fp8(yn, gpy + (size_t)sl * D, gsy + sl);
+    }
+  }
+  __syncthreads();
+
+  // ---- phase 2a: p, r of rows 16w..16w+15 on the tensor cores --------------------------------
+  uint8_t* crow = st + L.codes;
+  float* sscale = reinterpret_cast<float*>(st + L.scales);
+  {
+    const int gid = lane >> 2, q4 = lane & 3, r8 = lane & 7, mi = lane >> 3;
+    const int row0 = 16 * warp;
+    // digit weights of this lane's accumulator columns 2q4, 2q4 + 1: x = columns 0..2,
+    // y = columns 3..5 (d1 2^16 + d2 2^8 + d3)
+    const float wx0 = q4 == 0 ? 65536.f : (q4 == 1 ? 1.f : 0.f);
+    const float wx1 = q4 == 0 ? 256.f : 0.f;
+    const float wy0 = q4 == 2 ? 256.f : 0.f;
+    const float wy1 = q4 == 1 ? 65536.f : (q4 == 2 ? 1.f : 0.f);
+    const uint4 bw0 = *reinterpret_cast<const uint4*>(Bfrag + (gid * 4 + q4) * 32);
+    const uint4 bw1 = *reinterpret_cast<const uint4*>(Bfrag + (gid * 4 + q4) * 32 + 16);
+    const uint32_t bw[8] = {bw0.x, bw0.y, bw0.z, bw0.w, bw1.x, bw1.y, bw1.z, bw1.w};
+    const uint32_t cb0 = smem_u32(crow);
+    float PX[2], PY[2];
+    if constexpr (P::INT4) {
+      PX[0] = PX[1] = PY[0] = PY[1] = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {  // each 32-column chunk is one scale group
+        uint32_t Af[4], w0, w1;
+        ldsm_x2(cb0 + swz<64>(row0 + r8 + 8 * (mi & 1), 16 * c), w0, w1);
+        i4x8_to_s8x16(w0, Af[0], Af[2]);
+        i4x8_to_s8x16(w1, Af[1], Af[3]);
+        int Cc[4] = {0, 0, 0, 0};
+        mma_s8(Cc, Af, bw[2 * c], bw[2 * c + 1]);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const float sg = sscale[(row0 + gid + 8 * hh) * P::NG + c];
+          const float c0 = (float)Cc[2 * hh], c1 = (float)Cc[2 * hh + 1];
+          PX[hh] = fmaf(sg, wx0 * c0 + wx1 * c1, PX[hh]);
+          PY[hh] = fmaf(sg, wy0 * c0 + wy1 * c1, PY[hh]);
+        }
+      }
+    } else {
+      int Cc[4] = {0, 0, 0, 0};  // one exponent per vector: chunks accumulate exactly in int32
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t Af[4];
+        ldsm_x4(cb0 + swz<128>(row0 + r8 + 8 * (mi & 1), 32 * c + 16 * (mi >> 1)), Af);
+        mma_s8(Cc, Af, bw[2 * c], bw[2 * c + 1]);
+      }
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const float c0 = (float)Cc[2 * hh], c1 = (float)Cc[2 * hh + 1];
+        PX[hh] = wx0 * c0 + wx1 * c1;
+        PY[hh] = wy0 * c0 + wy1 * c1;
+      }
+    }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      PX[hh] += __shfl_xor_sync(0xffffffffu, PX[hh], 1);
+      PX[hh] += __shfl_xor_sync(0xffffffffu, PX[hh], 2);
+      PY[hh] += __shfl_xor_sync(0xffffffffu, PY[hh], 1);
+      PY[hh] += __shfl_xor_sync(0xffffffffu, PY[hh], 2);
+    }
+    if (q4 < 2) {  // lane q4 of the quad stores row row0 + gid + 8 q4
+      const int v = row0 + gid + 8 * q4;
+      const float srow = P::INT4 ? 0.0625f : sscale[v];  // int4 codes entered as 16 c
+      PR[v] = (q4 ? PX[1] : PX[0]) * sc[4] * srow;
+      RR[v] = (q4 ? PY[1] : PY[0]) * sc[5] * srow;
+    }
+  }
+  __syncwarp();
+
+  // ---- phase 2b: the new rows -----------------------------------------------------------------
+  // thread (i, h): 8-byte code blocks m = 0..NM-1 of row i at logical bytes 16m + 8h, i.e.
+  // columns BSTEP m + BW h .. + BW - 1 (interleaved, so the two threads of a row read vector
+  // entries in different banks)
+  const int i = tid >> 1, h = tid & 1;
+  const float a_s = P::DIAG ? 1.f : sc[3];
+  constexpr int NM = P::INT4 ? 4 : 8;      // blocks per thread
+  constexpr int BW = P::INT4 ? 16 : 8;     // columns per block
+  constexpr int BSTEP = 2 * BW;            // column step between a thread's blocks
+  constexpr int GB = P::INT4 ? 1 : NM;     // blocks per scale group
+  constexpr int NGRP = NM / GB;            // scale groups per thread
+  const float xoi = xo[i], kq = sc[0];
+  const float vi = Num<Act>::to_f(sv[i]);
+  const float p = fmaf(xoi, sc[1], PR[i]);
+  const float rq = fmaf(xoi, sc[2], RR[i]);
+  // H'[i][j] = a_j (s c_ij + x_o,i y_o,j) - beta p k_j  (+ beta v_i k_j when Wp = 0)
+  const float nb = Wp == 0 ? bt * (vi - p) : -bt * p;
+
+  // output: o_i = rq + beta (v_i - p) <k, q> + sum over carried pairs x_p,i c_p (the two
+  // threads of the row take alternate pairs)
+  {
+    float oi = h == 0 ? fmaf(bt * (vi - p), kq, rq) : 0.f;
+    for (int pp = 1 + h; pp <= carried; pp += 2) {
+      int sl = slot_new - pp;
+      if (sl < 0) sl += Wp;
+      const __half_raw hr =
+          __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)spx[(size_t)sl * D + i], __NV_E4M3);
+      oi = fmaf(ssx[sl] * __half2float(__half(hr)), cp[sl], oi);
+    }
+    oi += __shfl_xor_sync(0xffffffffu, oi, 1);
+    if (h == 0) static_cast<Act*>(a.o)[(size_t)head * D + i] = Num<Act>::from_f(oi);
+  }
+
+  uint32_t w[2 * NM];
+#pragma unroll
+  for (int m = 0; m < NM; ++m) {
+    const uint2 t = *reinterpret_cast<const uint2*>(crow + swz<P::ROW_BYTES>(i, 16 * m + 8 * h));
+    w[2 * m] = t.x;
+    w[2 * m + 1] = t.y;
+  }
+  const F2 nb2 = f2(nb, nb), xo2 = f2(xoi, xoi);
+  const F2 magic2 = f2(12582912.f, 12582912.f);  // 1.5 2^23: adding it rounds to an integer
+  float* srow = sscale + (size_t)i * P::NG;
+#pragma unroll
+  for (int gi = 0; gi < NGRP; ++gi) {
+    const float s = srow[P::INT4 ? gi : 0];
+    const F2 as2 = f2(a_s * s, a_s * s);
+    float Hg[GB * BW];
+    float mx = 0.f;
+#pragma unroll
+    for (int mb = 0; mb < GB; ++mb) {
+      const int m = gi * GB + mb;
+      const int jb = BSTEP * m + BW * h;
+      float f[BW];
+      if constexpr (P::INT4) {
+        i4x8_to_f32_2(w[2 * m], f);
+        i4x8_to_f32_2(w[2 * m + 1], f + 8);
+      } else {
+        i8x4_to_f32_2(w[2 * m], f);
+        i8x4_to_f32_2(w[2 * m + 1], f + 4);
+      }
+#pragma unroll
+      for (int e = 0; e < BW; e += 4) {
+        const float4 K4 = *reinterpret_cast<const float4*>(kf + jb + e);
+        const float4 Y4 = *reinterpret_cast<const float4*>(Y + jb + e);
+        F2 c01 = f2(f[e], f[e + 1]), c23 = f2(f[e + 2], f[e + 3]);
+        F2 s01 = as2, s23 = as2;
+        if constexpr (P::DIAG) {
+          const float4 A4 = *reinterpret_cast<const float4*>(A + jb + e);
+          s01 = f2_mul(f2(s, s), f2(A4.x, A4.y));
+          s23 = f2_mul(f2(s, s), f2(A4.z, A4.w));
+        }
+        const F2 h01 = f2_fma(s01, c01, f2_fma(xo2, f2(Y4.x, Y4.y), f2_mul(nb2, f2(K4.x, K4.y))));
+        const F2 h23 = f2_fma(s23, c23, f2_fma(xo2, f2(Y4.z, Y4.w), f2_mul(nb2, f2(K4.z, K4.w))));
+        float* hv = Hg + mb * BW + e;
+        f2_get(h01, hv[0], hv[1]);
+        f2_get(h23, hv[2], hv[3]);
+        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(hv[0]), fabsf(hv[1])), fmaxf(fabsf(hv[2]), fabsf(hv[3]))));
+      }
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));  // the row's (group's) other half
+    const float s2 = mx >= 0x1p-100f ? quot_const(mx, (float)P::QMAX, 1.f / (float)P::QMAX)
+                                     : __fdiv_rn(mx, (float)P::QMAX);
+    if (h == 0) srow[P::INT4 ? gi : 0] = s2;
+    if (s2 >= 0x1p-125f) {  // 1 / s2 finite and normal: corrected reciprocal quotients
+      const float inv = __frcp_rn(s2);
+      const F2 inv2 = f2(inv, inv), ns2 = f2(-s2, -s2);
+#pragma unroll
+      for (int mb = 0; mb < GB; ++mb) {
+        const int m = gi * GB + mb;
+        uint32_t b[BW];  // low byte = the code (two's complement) from 1.5 2^23 + rint(q)
+#pragma unroll
+        for (int e = 0; e < BW; e += 2) {
+          const F2 y = f2_add(f2_quot(f2(Hg[mb * BW + e], Hg[mb * BW + e + 1]), inv2, ns2), magic2);
+          float y0, y1;
+          f2_get(y, y0, y1);
+          b[e] = __float_as_uint(y0);
+          b[e + 1] = __float_as_uint(y1);
+        }
+        if constexpr (P::INT4) {  // 16 nibbles: column e at bits 4e of the block's two words
+#pragma unroll
+          for (int wd = 0; wd < 2; ++wd) {
+            const uint32_t* bb = b + 8 * wd;
+            const uint32_t ev = __byte_perm(__byte_perm(bb[0], bb[2], 0x0040),
+                                            __byte_perm(bb[4], bb[6], 0x0040), 0x5410);
+            const uint32_t od = __byte_perm(__byte_perm(bb[1], bb[3], 0x0040),
+                                            __byte_perm(bb[5], bb[7], 0x0040), 0x5410);
+            w[2 * m + wd] = (ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u);
+          }
+        } else {
+#pragma unroll
+          for (int wd = 0; wd < 2; ++wd) {
+            const uint32_t* bb = b + 4 * wd;
+            w[2 * m + wd] = __byte_perm(__byte_perm(bb[0], bb[1], 0x0040),
+                                        __byte_perm(bb[2], bb[3], 0x0040), 0x5410);
+          }
+        }
+      }
+    } else {  // a zero group, or one so small that 1 / s2 overflows: IEEE division
+#pragma unroll
+      for (int mb = 0; mb < GB; ++mb) {
+        const int m = gi * GB + mb;
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int e = 0; e < BW; ++e) {
+          const int c = s2 > 0.f ? (int)rintf(__fdiv_rn(Hg[mb * BW + e], s2)) : 0;
+          if constexpr (P::INT4) {
+            const uint32_t nib = (uint32_t)(c & 0xF) << (4 * (e & 7));
+            if (e < 8) lo |= nib;
+            else hi |= nib;
+          } else {
+            const uint32_t byte = (uint32_t)(c & 0xFF) << (8 * (e & 3));
+            if (e < 4) lo |= byte;
+            else hi |= byte;
+          }
+        }
+        w[2 * m] = lo;
+        w[2 * m + 1] = hi;
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < NM; ++m)
+    *reinterpret_cast<uint2*>(crow + swz<P::ROW_BYTES>(i, 16 * m + 8 * h)) =
+        make_uint2(w[2 * m], w[2 * m + 1]);
+  if (tid == 0) a.count[head] = Wp == 0 ? 0 : (cnt + 1 < 2 * Wp ? cnt + 1 : Wp);
+}
+
+// Persistent decode step: CTA b takes heads [b * per_cta, (b + 1) * per_cta).
+template <class P>
+__global__ void __launch_bounds__(kPwThreads, pw_ctas_per_sm<P>())
+    pw_step_kernel(const PwArgs a, const int heads, const int per_cta, const int nstages) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  const int tid = threadIdx.x;
+  const int h0 = blockIdx.x * per_cta;
+  const int nh = min(per_cta, heads - h0);
+  if (nh <= 0) return;
+  const PwLayout L = pw_layout<P>(a.Wp, nstages, per_cta);
+  int32_t* hcnt = reinterpret_cast<int32_t*>(sm + L.meta);
+  float* hg = reinterpret_cast<float*>(hcnt + per_cta);
+  float* hb = hg + per_cta;
+  for (int n = tid; n < nh; n += kPwThreads) {
+    hcnt[n] = a.count[h0 + n];
+    if constexpr (!P::DIAG) hg[n] = a.g[h0 + n];
+    hb[n] = a.beta[h0 + n];
+  }
+  // digit columns 6 and 7 of the tensor-core right-hand side are never written: zero once
+  for (int e = tid; e < kPwFragBytes / 4; e += kPwThreads)
+    reinterpret_cast<uint32_t*>(sm + L.frag)[e] = 0u;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L.bars);
+  if (tid == 0) {
+    for (int s = 0; s < nstages; ++s) mbar_init(&bars[s], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (tid == kPwIssuer)
+    for (int s = 0; s < nstages && s < nh; ++s)
+      pw_issue<P>(a, L, sm + s * L.stage_bytes, &bars[s], h0 + s);
+  for (int n = 0; n < nh; ++n) {
+    // refill the stage head n - 1 used, once its history tile has been read out
+    if (tid == kPwIssuer && n > 0 && n - 1 + nstages < nh) {
+      const int sp = (n - 1) % nstages;
+      bulk_wait_read_all();
+      pw_issue<P>(a, L, sm + sp * L.stage_bytes, &bars[sp], h0 + n - 1 + nstages);
+    }
+    const int timed_out =
+        mbar_wait_bounded(&bars[n % nstages], (uint32_t)(n / nstages) & 1u) ? 0 : 1;
+    if (__syncthreads_or(timed_out)) {
+      // give the copies still in flight (heads n .. n + nstages - 1) a bounded wait each
+      // before the CTA's shared memory goes away
+      if (tid == 0) {
+        pw_report(a.status, GDN_DEVICE_WAIT_TIMEOUT);
+        for (int m = n; m < nh && m < n + nstages; ++m)
+          (void)mbar_wait_bounded(&bars[m % nstages], (uint32_t)(m / nstages) & 1u);
+      }
+      break;
+    }
+    uint8_t* st = sm + (n % nstages) * L.stage_bytes;
+    const int cnt = hcnt[n];
+    const bool ok = pw_count_ok(cnt, a.Wp);
+    if (ok) pw_head<P>(a, L, sm, st, h0 + n, cnt, P::DIAG ? 0.f : hg[n], hb[n]);
+    else if (tid == 0) pw_report(a.status, GDN_DEVICE_BAD_POS);
+    // the stage's generic-proxy writes are ordered before the bulk store that reads them and
+    // the copies that later refill it
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    __syncthreads();
+    if (ok && tid == kPwIssuer) {
+      const int head = h0 + n;
+      bulk_s2g(a.codes + (size_t)head * P::CODE_BYTES, st + L.codes, P::CODE_BYTES);
+      bulk_s2g(a.scales + (size_t)head * P::NSCALES, st + L.scales, 4u * P::NSCALES);
+      bulk_commit();
+    }
+  }
+  if (tid == kPwIssuer) bulk_wait_all();
+}
+
+// Logical state: history plus the pairs in the window. One CTA per head.
+template <class P>
+__global__ void __launch_bounds__(kPwThreads) pw_materialize_kernel(const PwArgs a) {
+  constexpr int D = P::D;
+  __shared__ float xs[GDN_PW_MAX_WINDOW][D];
+  __shared__ float ys[GDN_PW_MAX_WINDOW][D];
+  const int head = blockIdx.x, tid = threadIdx.x;
+  const int Wp = a.Wp, Wr = (Wp + 3) & ~3;
+  const int cnt = a.count[head];
+  if (!pw_count_ok(cnt, Wp)) {
+    if (tid == 0) pw_report(a.status, GDN_DEVICE_BAD_POS);
+    return;
+  }
+  const int fill = min(cnt, Wp);  // slots 0 .. fill-1 hold pairs (all of them once full)
+  const uint8_t* gp = a.pairs + (size_t)head * 2 * Wp * D;
+  const float* gs = a.pscales + (size_t)head * 2 * Wr;
+  for (int e = tid; e < fill * D; e += kPwThreads) {
+    const int sl = e / D, j = e % D;
+    const __half_raw hx = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)gp[(size_t)sl * D + j], __NV_E4M3);
+    const __half_raw hy =
+        __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)gp[(size_t)(Wp + sl) * D + j], __NV_E4M3);
+    xs[sl][j] = gs[sl] * __half2float(__half(hx));
+    ys[sl][j] = gs[Wr + sl] * __half2float(__half(hy));
+  }
+  __syncthreads();
+  const uint8_t* codes = a.codes + (size_t)head * P::CODE_BYTES;
+  const float* scales = a.scales + (size_t)head * P::NSCALES;
+  float* out = a.S_out + (size_t)head * D * D;
+  for (int e = tid; e < D * D; e += kPwThreads) {
+    const int i = e / D, j = e % D;
+    float c;
+    if constexpr (P::INT4) {
+      const uint8_t b = codes[swz<P::ROW_BYTES>(i, j / 2)];
+      const int nib = (j & 1) ? (b >> 4) : (b & 0xF);
+      c = (float)(nib >= 8 ? nib - 16 : nib);
+    } else {
+      c = (float)(int8_t)codes[swz<P::ROW_BYTES>(i, j)];
+    }
+    float x = scales[i * P::NG + j / P::GS] * c;
+    for (int sl = 0; sl < fill; ++sl) x = fmaf(xs[sl][i], ys[sl][j], x);
+    out[e] = x;
+  }
+}
+
+}  // namespace gdnq

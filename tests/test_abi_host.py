@@ -1,7 +1,8 @@
-"""The C ABI on the host: the library loads, exports every symbol include/gdnq.h declares, sizes
+"""The C ABI on the host: the library loads, exports every symbol include/*.h declares, sizes
 its buffers, and rejects bad arguments before touching a device. Every call here fails argument
 checks (or is an empty batch), so no kernel is launched and no pointer is dereferenced."""
 import ctypes
+import glob
 import os
 import re
 
@@ -11,7 +12,7 @@ import bit_recurrent_state_gdn_b200 as gdn
 from bit_recurrent_state_gdn_b200 import _abi, build
 from workloads import WORKLOADS
 
-HEADER = os.path.join(os.path.dirname(build.PKG), "include", "gdnq.h")
+HEADERS = sorted(glob.glob(os.path.join(os.path.dirname(build.PKG), "include", "*.h")))
 
 
 @pytest.fixture(scope="module")
@@ -21,14 +22,17 @@ def lib():
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(gdn_[a-z_]+)\s*\(", text)))
+    names = set()
+    for h in HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"\b(gdn_[a-z_]+)\s*\(", text))
+    return sorted(names)
 
 
 def test_every_declared_symbol_is_exported_and_bound(lib):
+    assert len(HEADERS) >= 2
     names = declared_functions()
-    assert len(names) >= 11
+    assert len(names) >= 16
     for n in names:
         assert hasattr(lib, n), f"{n} not exported"
         assert n in _abi.SIGNATURES, f"{n} not bound in the Python layer"
@@ -190,3 +194,64 @@ def test_baseline_format_checks(lib):
 def test_python_layer_raises_with_detail(lib):
     with pytest.raises(gdn.GdnError, match="GDN_ERR_UNSUPPORTED.*head size"):
         gdn.gdn_state_sizes(_cfg(D=64))
+
+
+# ---- pure-write sliding window ----------------------------------------------------------------
+def _pw(**kw):
+    base = dict(B=2, H=3, D=128, Wp=8, gate="scalar", fmt="int4_g32", act="bf16")
+    base.update(kw)
+    return gdn.make_pw_config(**base)
+
+
+@pytest.mark.parametrize("fmt,Wp", [("int8", 8), ("int4_g32", 8), ("int4_g32", 0), ("int8", 5)])
+def test_pw_state_sizes(fmt, Wp, lib):
+    cfg = _pw(fmt=fmt, Wp=Wp)
+    s = gdn.gdn_pw_state_sizes(cfg)
+    n, D = 6, 128
+    if fmt == "int8":
+        assert s.codes == n * D * D and s.scales == n * D * 4
+    else:
+        assert s.codes == n * D * D // 2 and s.scales == n * D * 4 * 4
+    assert s.pairs == n * 2 * Wp * D
+    assert s.pscales == (n * 8 * ((Wp + 3) // 4 * 4) if Wp else 0)
+    assert s.count == n * 4
+
+
+PW_BAD = [
+    ("Wp<0", dict(Wp=-1), _abi.GDN_ERR_INVALID_ARG),
+    ("Wp>max", dict(Wp=17), _abi.GDN_ERR_UNSUPPORTED),
+    ("D=64", dict(D=64), _abi.GDN_ERR_UNSUPPORTED),
+    ("fmt mixed", dict(fmt="mixed"), _abi.GDN_ERR_INVALID_ARG),
+    ("fmt fp32", dict(fmt="fp32"), _abi.GDN_ERR_INVALID_ARG),
+    ("B<0", dict(B=-1), _abi.GDN_ERR_INVALID_ARG),
+]
+
+
+@pytest.mark.parametrize("name,kw,status", PW_BAD, ids=[b[0] for b in PW_BAD])
+def test_pw_bad_configs(name, kw, status, lib):
+    out = _abi.gdn_pw_sizes()
+    assert lib.gdn_pw_state_sizes(ctypes.byref(_pw(**kw)), ctypes.byref(out)) == status
+    assert lib.gdn_last_error() != b""
+
+
+def test_pw_calls_reject_missing_buffers(lib):
+    cfg = _pw()
+    st = _abi.gdn_pw_state()  # all null
+    assert lib.gdn_pw_quantize(ctypes.byref(cfg), None, ctypes.byref(st), None) == \
+        _abi.GDN_ERR_INVALID_ARG
+    assert lib.gdn_pw_decode_steps(ctypes.byref(cfg), ctypes.byref(st), 1, *([None] * 7)) == \
+        _abi.GDN_ERR_INVALID_ARG
+    assert lib.gdn_pw_materialize(ctypes.byref(cfg), ctypes.byref(st), None, None) == \
+        _abi.GDN_ERR_INVALID_ARG
+    assert lib.gdn_pw_decode_steps(ctypes.byref(cfg), ctypes.byref(st), -1, *([None] * 7)) == \
+        _abi.GDN_ERR_INVALID_ARG
+
+
+def test_pw_empty_batch_and_zero_steps_are_noops(lib):
+    st = _abi.gdn_pw_state()
+    empty = _pw(B=0)
+    assert lib.gdn_pw_quantize(ctypes.byref(empty), None, ctypes.byref(st), None) == _abi.GDN_OK
+    assert lib.gdn_pw_decode_steps(ctypes.byref(empty), ctypes.byref(st), 3, *([None] * 7)) == \
+        _abi.GDN_OK
+    assert lib.gdn_pw_decode_steps(ctypes.byref(_pw()), ctypes.byref(st), 0, *([None] * 7)) == \
+        _abi.GDN_OK

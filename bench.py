@@ -34,7 +34,13 @@ PROFILE = os.path.join(ROOT, "profiles", "window_step_gdn-serving.md")
 KERNEL_SOURCES = ["bit_recurrent_state_gdn_b200/csrc/window_kernels.cuh",
                   "bit_recurrent_state_gdn_b200/csrc/window_mma.cuh",
                   "bit_recurrent_state_gdn_b200/csrc/window_dispatch.cuh",
-                  "bit_recurrent_state_gdn_b200/csrc/device_util.cuh"]
+                  "bit_recurrent_state_gdn_b200/csrc/device_util.cuh",
+                  "bit_recurrent_state_gdn_b200/csrc/mma_util.cuh"]
+PW_PROFILE = os.path.join(ROOT, "profiles", "pw_step_gdn-serving.md")
+PW_KERNEL_SOURCES = ["bit_recurrent_state_gdn_b200/csrc/pw_kernels.cuh",
+                     "bit_recurrent_state_gdn_b200/csrc/pw.cu",
+                     "bit_recurrent_state_gdn_b200/csrc/device_util.cuh",
+                     "bit_recurrent_state_gdn_b200/csrc/mma_util.cuh"]
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -51,6 +57,8 @@ def parse_args():
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--cpu-heads", type=int, default=8192)
     p.add_argument("--ref-heads", type=int, default=2048)
+    p.add_argument("--pw-only", action="store_true",
+                   help="run only the pure-write window legs (profiling captures)")
     return p.parse_args()
 
 
@@ -91,23 +99,23 @@ def peak_hbm():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profiled_traffic():
-    """Per-launch DRAM bytes of the window-step kernel from the committed ncu summary, if the
-    kernel source still matches the one profiled; else None."""
+def profiled_traffic(profile=PROFILE, sources=KERNEL_SOURCES, key="traffic_bytes_per_launch"):
+    """Per-launch DRAM bytes of a kernel from its committed ncu summary, if the kernel source
+    still matches the one profiled; else None."""
     try:
-        text = open(PROFILE).read()
+        text = open(profile).read()
     except OSError:
         return None, None
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m = re.search(key + r":\s*([0-9.eE+]+)", text)
     s = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
-    if not m or not s or s.group(1) != kernel_sha():
+    if not m or not s or s.group(1) != kernel_sha(sources):
         return None, None
-    return float(m.group(1)), os.path.relpath(PROFILE, ROOT)
+    return float(m.group(1)), os.path.relpath(profile, ROOT)
 
 
-def kernel_sha() -> str:
+def kernel_sha(sources=KERNEL_SOURCES) -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in sources:
         with open(os.path.join(ROOT, p), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -317,6 +325,15 @@ def main():
     state = gdn.GdnState.allocate(cfg, dev)
     o = torch.empty_like(inp["q"])
     torch.cuda.synchronize()
+    if args.pw_only:
+        peak, _ = peak_hbm()
+        pw = {f: pw_leg(wl.with_(fmt=f), 8, S0, inp, o, peak) for f in ("int4_g32", "int8")}
+        if rank == 0:
+            print(json.dumps({"pure_write_s8": pw, "config": bench_config(wl0, world)}),
+                  flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
 
     def one_step(ev=None):
         if ev is not None:
@@ -385,6 +402,11 @@ def main():
     if not args.no_baselines and wl.fmt == "int8" and wl.D == 128:
         line["mixed_half_int4"] = mixed_leg(wl, S0, inp, o, peak)
 
+    # ---- pure-write sliding window (PW-S8) over int4 and int8 histories, the same inputs ----
+    if not args.no_baselines and wl.D == 128:
+        line["pure_write_s8"] = {f: pw_leg(wl.with_(fmt=f), 8, S0, inp, o, peak)
+                                 for f in ("int4_g32", "int8")}
+
     # ---- high-precision-state baselines on the same inputs ---------------------------------
     if not args.no_baselines:
         line["baselines"] = {}
@@ -451,6 +473,52 @@ def mixed_leg(wl, S0, inp, o, peak):
     return {"value": wl.heads * wl.T / (ms / 1e3), "unit": UNIT, "achieved_gbs": gbs,
             "frac": gbs / peak, "ms_per_run": ms,
             "note": "GDN_FMT_MIXED, heads alternately int8 / int4-g32, one launch per step"}
+
+
+def pw_step_bytes(wl, Wp: int) -> int:
+    """Algorithmic bytes of one pure-write window step per head with a full window: the history
+    (codes + scales) read and written, the Wp pairs (e4m3 x and y, fp32 scales) read, the Wp - 1
+    carried keys and the new pair written with their scales, q / k / v / g / beta / count read,
+    o and count written."""
+    D = wl.D
+    act = 4 if wl.act == "f32" else 2
+    hist = (D * D // 2 + 4 * D * (D // 32)) if wl.fmt == "int4_g32" else (D * D + 4 * D)
+    g = 4 * D if wl.gate == "diag" else 4
+    read = hist + 2 * Wp * D + 8 * Wp + 3 * D * act + g + 4 + 4
+    write = hist + ((Wp + 1) * D + 4 * (Wp + 1) if Wp else 0) + D * act + 4
+    return read + write
+
+
+def pw_leg(wl, Wp, S0, inp, o, peak):
+    """The pure-write sliding window decode on the same inputs: the history quantized from the
+    same initial states, then the T steps, one launch each, timed with CUDA events."""
+    import torch
+
+    import bit_recurrent_state_gdn_b200 as gdn
+
+    cfg = gdn.make_pw_config(wl.B, wl.H, wl.D, Wp, wl.gate, wl.fmt, wl.act)
+    st = gdn.PwState.allocate(cfg)
+    gdn.gdn_pw_quantize(cfg, S0, st)
+    gdn.gdn_pw_decode_steps(cfg, st, inp["q"][:4], inp["k"][:4], inp["v"][:4], inp["g"][:4],
+                            inp["beta"][:4], o[:4])
+    gdn.gdn_pw_quantize(cfg, S0, st)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    gdn.gdn_pw_decode_steps(cfg, st, inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], o)
+    e1.record()
+    torch.cuda.synchronize()
+    if int(st.status[0].item()) != 0:
+        raise RuntimeError("pure-write window: device status word set")
+    ms = e0.elapsed_time(e1)
+    gbs = pw_step_bytes(wl, Wp) * wl.heads * wl.T / (ms / 1e3) / 1e9
+    traffic, src = profiled_traffic(PW_PROFILE, PW_KERNEL_SOURCES,
+                                    f"traffic_bytes_per_head_{wl.fmt}")
+    return {"value": wl.heads * wl.T / (ms / 1e3), "unit": UNIT, "achieved_gbs": gbs,
+            "frac": gbs / peak, "avg_launch_us": ms * 1e3 / wl.T, "ms_per_run": ms,
+            "bytes_per_head_step": pw_step_bytes(wl, Wp), "Wp": Wp,
+            "traffic": None if traffic is None else traffic * wl.heads, "traffic_source": src,
+            "kernel": "pw_step_kernel (history requantised every step, FP8 pairs)"}
 
 
 def e2e(args, wl, cfg, inp, S0, state, world, dev):

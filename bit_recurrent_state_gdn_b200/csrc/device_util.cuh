@@ -237,6 +237,27 @@ __device__ __forceinline__ void i4x8_to_f32_2(uint32_t w, float* f) {
   }
 }
 
+// Packed-pair forms: int8 codes of one word as (c0, c1), (c2, c3); int4 codes of one word as
+// (c0, c1) .. (c6, c7).
+__device__ __forceinline__ void i8x4_to_f2(uint32_t w, F2* out) {
+  const uint32_t x = w ^ 0x80808080u;
+  const F2 bias = f2(-8388736.f, -8388736.f);
+  out[0] = f2_add(f2(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7650)),
+                     __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7651))), bias);
+  out[1] = f2_add(f2(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7652)),
+                     __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7653))), bias);
+}
+
+__device__ __forceinline__ void i4x8_to_f2(uint32_t w, F2* out) {
+  const uint32_t x = w ^ 0x88888888u;
+  const uint32_t lo = x & 0x0F0F0F0Fu, hi = (x >> 4) & 0x0F0F0F0Fu;
+  const F2 bias = f2(-8388616.f, -8388616.f);
+#pragma unroll
+  for (int m = 0; m < 4; ++m)
+    out[m] = f2_add(f2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650 + m)),
+                       __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650 + m))), bias);
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 

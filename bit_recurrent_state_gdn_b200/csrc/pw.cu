@@ -22,8 +22,9 @@ cudaError_t pw_launch_cfg(PwOp op, const PwArgs& a, int heads, cudaStream_t st) 
   if (per_cta > kPwMaxHeadsPerCta) per_cta = kPwMaxHeadsPerCta;
   const int grid = (heads + per_cta - 1) / per_cta;
   const size_t budget = (size_t)228 * 1024 / cps - 1024;
+  // at least two stages (the loop's refill order needs them; two always fit)
   int nstages = kPwMaxStages;
-  while (nstages > 1 && pw_layout<P>(a.Wp, nstages, per_cta).total > budget) --nstages;
+  while (nstages > 2 && pw_layout<P>(a.Wp, nstages, per_cta).total > budget) --nstages;
   const size_t smem = pw_layout<P>(a.Wp, nstages, per_cta).total;
   cudaError_t e = ensure_smem<pw_step_kernel<P>>(smem);
   if (e != cudaSuccess) return e;

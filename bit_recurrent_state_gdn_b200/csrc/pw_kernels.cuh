@@ -77,7 +77,7 @@ struct PwLayout {
   uint32_t vec, frag, meta, bars, total;
 };
 
-constexpr int kPwVecs = 9;      // k, q, a, a.k, a.q, a.y_o, x_o, p, r
+constexpr int kPwVecs = 9;      // k, -, a, -, -, a.y_o, x_o, p, r
 constexpr int kPwScalars = 64;  // [0] <k,q>, [1] <y_o,a.k>, [2] <y_o,a.q>, [3] a (scalar gate),
                                 // [4..5] digit units,
                                 // [16..31] pair coefficients
@@ -136,6 +136,10 @@ __device__ __forceinline__ void bulk_commit() {
 __device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
 }
+// Waits until every committed bulk store but the newest has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_newest_pending() {
+  asm volatile("cp.async.bulk.wait_group.read 1;\n" ::: "memory");
+}
 // Waits until every committed bulk store has completed.
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
@@ -160,36 +164,46 @@ __device__ __forceinline__ uint32_t f32x4_to_e4m3(const float* t) {
   return (lo & 0xFFFFu) | (hi << 16);
 }
 
-__device__ __forceinline__ float warp_sum(float x) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-  return x;
-}
-
 __device__ __forceinline__ float warp_max(float x) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
   return x;
 }
 
-// A warp stores a D = 128 vector (4 elements per lane) as e4m3 codes with one scale:
-// s = absmax / 448 and codes e4m3(x / s), both quotients correctly rounded (a zero vector gets
-// s = 0 and codes 0).
-__device__ __forceinline__ void pw_store_fp8(const float* x, uint8_t* dst, float* dst_scale) {
-  const float m = warp_max(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3]))));
+// Sum / max over the 16 lanes of a half-warp (mask: that half's lanes).
+__device__ __forceinline__ float hw_sum(float x, unsigned mask) {
+#pragma unroll
+  for (int off = 8; off > 0; off >>= 1) x += __shfl_xor_sync(mask, x, off);
+  return x;
+}
+__device__ __forceinline__ float hw_max(float x, unsigned mask) {
+#pragma unroll
+  for (int off = 8; off > 0; off >>= 1) x = fmaxf(x, __shfl_xor_sync(mask, x, off));
+  return x;
+}
+
+// A half-warp stores a D = 128 vector (8 elements per lane, lane l16 holds 8 l16 .. 8 l16 + 7)
+// as e4m3 codes with one scale: s = absmax / 448 and codes e4m3(x / s), both quotients
+// correctly rounded (a zero vector gets s = 0 and codes 0).
+__device__ __forceinline__ void pw_store_fp8(const float* x, uint8_t* dst, float* dst_scale,
+                                             int l16, unsigned mask) {
+  float m = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(x[e]));
+  m = hw_max(m, mask);
   const float s = m >= 0x1p-100f ? quot_const(m, 448.f, 1.f / 448.f) : __fdiv_rn(m, 448.f);
-  float t[4] = {0.f, 0.f, 0.f, 0.f};
+  float t[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (s >= 0x1p-125f) {
     const float inv = __frcp_rn(s);
     const F2 inv2 = f2(inv, inv), ns = f2(-s, -s);
-    f2_get(f2_quot(f2(x[0], x[1]), inv2, ns), t[0], t[1]);
-    f2_get(f2_quot(f2(x[2], x[3]), inv2, ns), t[2], t[3]);
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) f2_get(f2_quot(f2(x[e], x[e + 1]), inv2, ns), t[e], t[e + 1]);
   } else if (s > 0.f) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) t[e] = __fdiv_rn(x[e], s);
+    for (int e = 0; e < 8; ++e) t[e] = __fdiv_rn(x[e], s);
   }
-  *reinterpret_cast<uint32_t*>(dst + 4 * (threadIdx.x & 31)) = f32x4_to_e4m3(t);
-  if ((threadIdx.x & 31) == 0) *dst_scale = s;
+  *reinterpret_cast<uint2*>(dst + 8 * l16) = make_uint2(f32x4_to_e4m3(t), f32x4_to_e4m3(t + 4));
+  if (l16 == 0) *dst_scale = s;
 }
 
 template <class P>
@@ -234,7 +248,7 @@ __device__ __forceinline__ void pw_head(const PwArgs& a, const PwLayout& L, uint
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Wp = a.Wp, Wr = (Wp + 3) & ~3;
   float* vec = reinterpret_cast<float*>(sm + L.vec);
-  float *kf = vec, *qf = vec + D, *A = vec + 2 * D, *ak = vec + 3 * D, *aq = vec + 4 * D;
+  float *kf = vec, *A = vec + 2 * D;
   float *Y = vec + 5 * D, *xo = vec + 6 * D, *PR = vec + 7 * D, *RR = vec + 8 * D;
   float* sc = vec + 9 * D;
   float* cp = sc + 16;
@@ -251,112 +265,135 @@ __device__ __forceinline__ void pw_head(const PwArgs& a, const PwLayout& L, uint
   const int carried = fill - full;
   const int slot_new = Wp > 0 ? (cnt >= Wp ? cnt - Wp : cnt) : 0;
 
-  // ---- phase 0 ------------------------------------------------------------------------------
-  if (tid < D) {
-    const float kj = Num<Act>::to_f(sk[tid]), qj = Num<Act>::to_f(sq[tid]);
-    float aj;
-    if constexpr (P::DIAG) {
-      aj = expf(reinterpret_cast<const float*>(st + L.g)[tid]);
-    } else {
-      aj = expf(gs);  // one value, formed the same way by every thread
-      if (tid == 0) sc[3] = aj;
-    }
-    kf[tid] = kj;
-    qf[tid] = qj;
-    A[tid] = aj;
-    ak[tid] = aj * kj;
-    aq[tid] = aj * qj;
-  }
-  __syncthreads();
+  const float* sgd = reinterpret_cast<const float*>(st + L.g);  // per-channel log-gate (diag)
+  const float a_scalar = P::DIAG ? 1.f : expf(gs);  // formed the same way by every thread
 
   // ---- phase 1 ------------------------------------------------------------------------------
-  if (warp < 4) {
-    // one block exponent per vector, found by every warp from all 128 columns
-    float mx = 0.f, my = 0.f;
+  // warps 0-1: the fp32 vectors k, a (for the row phase) and a.k, a.q as exact integer digits for
+  // the tensor cores (lane: columns lane + 32 mm, the block maxima over all 128 columns)
+  if (warp < 2) {
+    float akv[4], aqv[4], mx = 0.f, my = 0.f;
 #pragma unroll
     for (int mm = 0; mm < 4; ++mm) {
-      mx = fmaxf(mx, fabsf(ak[lane + 32 * mm]));
-      my = fmaxf(my, fabsf(aq[lane + 32 * mm]));
+      const int j = lane + 32 * mm;
+      const float kj = Num<Act>::to_f(sk[j]), qj = Num<Act>::to_f(sq[j]);
+      const float aj = P::DIAG ? expf(sgd[j]) : a_scalar;
+      akv[mm] = aj * kj;
+      aqv[mm] = aj * qj;
+      mx = fmaxf(mx, fabsf(akv[mm]));
+      my = fmaxf(my, fabsf(aqv[mm]));
+      if (mm == warp || mm == warp + 2) {  // this thread's two columns
+        kf[j] = kj;
+        A[j] = aj;
+      }
     }
     mx = warp_max(mx);
     my = warp_max(my);
-    const float ux = put_digits<P::INT4>(Bfrag, 0, tid, ak[tid], mx);
-    const float uy = put_digits<P::INT4>(Bfrag, 3, tid, aq[tid], my);
-    if (tid == 0) {
-      sc[4] = ux;
-      sc[5] = uy;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int j = lane + 32 * (warp + 2 * c);  // (static register indices: no local array)
+      const float xv = warp == 0 ? akv[2 * c] : akv[2 * c + 1];
+      const float yv = warp == 0 ? aqv[2 * c] : aqv[2 * c + 1];
+      const float ux = put_digits<P::INT4>(Bfrag, 0, j, xv, mx);
+      const float uy = put_digits<P::INT4>(Bfrag, 3, j, yv, my);
+      if (j == 0) {
+        sc[3] = a_scalar;
+        sc[4] = ux;
+        sc[5] = uy;
+      }
     }
   }
-  const int j0 = 4 * lane;
-  uint8_t* gpx = a.pairs + (size_t)head * 2 * Wp * D;
-  uint8_t* gpy = gpx + (size_t)Wp * D;
-  float* gsx = a.pscales + (size_t)head * 2 * Wr;
-  float* gsy = gsx + Wr;
-  for (int task = 7 - warp; task < carried + 2; task += kPwThreads / 32) {
-    if (task == 0) {  // <k, q> and the new pair (beta v, k)
-      float kq = 0.f;
+  // pair tasks on half-warps, the last half-warp first: task 0 <k, q> and the new pair, 1 the
+  // leaving pair (or zeros), 2.. the carried pairs. Lane l16 of a half-warp holds columns
+  // 8 l16 .. 8 l16 + 7.
+  {
+    const int hw = tid >> 4, l16 = lane & 15;
+    const unsigned mask = 0xFFFFu << (lane & 16);
+    const int j0 = 8 * l16;
+    uint8_t* gpx = a.pairs + (size_t)head * 2 * Wp * D;
+    uint8_t* gpy = gpx + (size_t)Wp * D;
+    float* gsx = a.pscales + (size_t)head * 2 * Wr;
+    float* gsy = gsx + Wr;
+    auto act8 = [&](const Act* v, float* out) { Num<Act>::template load<8>(v + j0, out); };
+    auto gate8 = [&](float* out) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) kq += kf[j0 + e] * qf[j0 + e];
-      kq = warp_sum(kq);
-      if (lane == 0) sc[0] = kq;
-      if (Wp > 0) {
-        float x[4], y[4];
+      for (int e = 0; e < 8; ++e) out[e] = P::DIAG ? expf(sgd[j0 + e]) : a_scalar;
+    };
+    auto fp8x8 = [&](const uint8_t* src, float sv8, float* out) {
+      const uint2 wv = *reinterpret_cast<const uint2*>(src + j0);
+      e4m3x4_to_f32(wv.x, out);
+      e4m3x4_to_f32(wv.y, out + 4);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          x[e] = bt * Num<Act>::to_f(sv[j0 + e]);
-          y[e] = kf[j0 + e];
+      for (int e = 0; e < 8; ++e) out[e] *= sv8;
+    };
+    for (int task = 15 - hw; task < carried + 2; task += 16) {
+      float kv[8];
+      act8(sk, kv);
+      if (task == 0) {
+        float qv[8];
+        act8(sq, qv);
+        float kq = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) kq = fmaf(kv[e], qv[e], kq);
+        kq = hw_sum(kq, mask);
+        if (l16 == 0) sc[0] = kq;
+        if (Wp > 0) {
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = bt * Num<Act>::to_f(sv[j0 + e]);
+          pw_store_fp8(x, gpx + (size_t)slot_new * D, gsx + slot_new, l16, mask);
+          pw_store_fp8(kv, gpy + (size_t)slot_new * D, gsy + slot_new, l16, mask);
         }
-        pw_store_fp8(x, gpx + (size_t)slot_new * D, gsx + slot_new);
-        pw_store_fp8(y, gpy + (size_t)slot_new * D, gsy + slot_new);
-      }
-    } else if (task == 1) {  // the pair leaving the window joins the history (or nothing)
-      float yak = 0.f, yaq = 0.f;
-      if (full) {
-        float x[4], y[4];
-        e4m3x4_to_f32(*reinterpret_cast<const uint32_t*>(spx + (size_t)slot_new * D + j0), x);
-        e4m3x4_to_f32(*reinterpret_cast<const uint32_t*>(spy + (size_t)slot_new * D + j0), y);
-        const float sx = ssx[slot_new], sy = ssy[slot_new];
+      } else if (task == 1) {
+        float yak = 0.f, yaq = 0.f;
+        if (full) {
+          float x[8], y[8], av[8], qv[8];
+          fp8x8(spx + (size_t)slot_new * D, ssx[slot_new], x);
+          fp8x8(spy + (size_t)slot_new * D, ssy[slot_new], y);
+          gate8(av);
+          act8(sq, qv);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float yv = sy * y[e];
-          xo[j0 + e] = sx * x[e];
-          Y[j0 + e] = A[j0 + e] * yv;
-          yak += yv * ak[j0 + e];
-          yaq += yv * aq[j0 + e];
+          for (int e = 0; e < 8; ++e) {
+            xo[j0 + e] = x[e];
+            Y[j0 + e] = av[e] * y[e];
+            yak = fmaf(y[e], av[e] * kv[e], yak);
+            yaq = fmaf(y[e], av[e] * qv[e], yaq);
+          }
+          yak = hw_sum(yak, mask);
+          yaq = hw_sum(yaq, mask);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xo[j0 + e] = Y[j0 + e] = 0.f;
         }
-        yak = warp_sum(yak);
-        yaq = warp_sum(yaq);
-      } else {
+        if (l16 == 0) {
+          sc[1] = yak;
+          sc[2] = yaq;
+        }
+      } else {  // a carried pair: key side through the transition
+        const int p = task - 1;  // written p writes ago
+        int sl = slot_new - p;
+        if (sl < 0) sl += Wp;
+        float y[8], av[8], qv[8];
+        fp8x8(spy + (size_t)sl * D, ssy[sl], y);
+        gate8(av);
+        act8(sq, qv);
+        float d = 0.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) xo[j0 + e] = Y[j0 + e] = 0.f;
-      }
-      if (lane == 0) {
-        sc[1] = yak;
-        sc[2] = yaq;
-      }
-    } else {  // a carried pair: key side through the transition
-      const int p = task - 1;  // written p writes ago
-      int sl = slot_new - p;
-      if (sl < 0) sl += Wp;
-      float y[4], yn[4];
-      e4m3x4_to_f32(*reinterpret_cast<const uint32_t*>(spy + (size_t)sl * D + j0), y);
-      const float sy = ssy[sl];
-      float d = 0.f;
+        for (int e = 0; e < 8; ++e) {
+          y[e] = av[e] * y[e];
+          d = fmaf(kv[e], y[e], d);
+        }
+        d = bt * hw_sum(d, mask);
+        float cq = 0.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        y[e] = A[j0 + e] * (sy * y[e]);
-        d += kf[j0 + e] * y[e];
+        for (int e = 0; e < 8; ++e) {
+          y[e] = fmaf(-d, kv[e], y[e]);
+          cq = fmaf(y[e], qv[e], cq);
+        }
+        cq = hw_sum(cq, mask);
+        if (l16 == 0) cp[sl] = cq;
+        pw_store_fp8(y, gpy + (size_t)sl * D, gsy + sl, l16, mask);
       }
-      d = bt * warp_sum(d);
-      float cq = 0.f;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        yn[e] = y[e] - d * kf[j0 + e];
-        cq += yn[e] * qf[j0 + e];
-      }
-      cq = warp_sum(cq);
-      if (lane == 0) cp[sl] = cq;
-      pw_store_fp8(yn, gpy + (size_t)sl * D, gsy + sl);
     }
   }
   __syncthreads();
@@ -470,41 +507,43 @@ __device__ __forceinline__ void pw_head(const PwArgs& a, const PwLayout& L, uint
   const F2 nb2 = f2(nb, nb), xo2 = f2(xoi, xoi);
   const F2 magic2 = f2(12582912.f, 12582912.f);  // 1.5 2^23: adding it rounds to an integer
   float* srow = sscale + (size_t)i * P::NG;
+  constexpr int NP = GB * BW / 2;  // column pairs per thread and scale group
 #pragma unroll
   for (int gi = 0; gi < NGRP; ++gi) {
     const float s = srow[P::INT4 ? gi : 0];
     const F2 as2 = f2(a_s * s, a_s * s);
-    float Hg[GB * BW];
+    F2 Hg[NP];
     float mx = 0.f;
 #pragma unroll
     for (int mb = 0; mb < GB; ++mb) {
       const int m = gi * GB + mb;
       const int jb = BSTEP * m + BW * h;
-      float f[BW];
+      F2 c[BW / 2];
       if constexpr (P::INT4) {
-        i4x8_to_f32_2(w[2 * m], f);
-        i4x8_to_f32_2(w[2 * m + 1], f + 8);
+        i4x8_to_f2(w[2 * m], c);
+        i4x8_to_f2(w[2 * m + 1], c + 4);
       } else {
-        i8x4_to_f32_2(w[2 * m], f);
-        i8x4_to_f32_2(w[2 * m + 1], f + 4);
+        i8x4_to_f2(w[2 * m], c);
+        i8x4_to_f2(w[2 * m + 1], c + 2);
       }
 #pragma unroll
       for (int e = 0; e < BW; e += 4) {
         const float4 K4 = *reinterpret_cast<const float4*>(kf + jb + e);
         const float4 Y4 = *reinterpret_cast<const float4*>(Y + jb + e);
-        F2 c01 = f2(f[e], f[e + 1]), c23 = f2(f[e + 2], f[e + 3]);
         F2 s01 = as2, s23 = as2;
         if constexpr (P::DIAG) {
           const float4 A4 = *reinterpret_cast<const float4*>(A + jb + e);
           s01 = f2_mul(f2(s, s), f2(A4.x, A4.y));
           s23 = f2_mul(f2(s, s), f2(A4.z, A4.w));
         }
-        const F2 h01 = f2_fma(s01, c01, f2_fma(xo2, f2(Y4.x, Y4.y), f2_mul(nb2, f2(K4.x, K4.y))));
-        const F2 h23 = f2_fma(s23, c23, f2_fma(xo2, f2(Y4.z, Y4.w), f2_mul(nb2, f2(K4.z, K4.w))));
-        float* hv = Hg + mb * BW + e;
-        f2_get(h01, hv[0], hv[1]);
-        f2_get(h23, hv[2], hv[3]);
-        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(hv[0]), fabsf(hv[1])), fmaxf(fabsf(hv[2]), fabsf(hv[3]))));
+        const int q = (mb * BW + e) / 2;
+        Hg[q] = f2_fma(s01, c[e / 2], f2_fma(xo2, f2(Y4.x, Y4.y), f2_mul(nb2, f2(K4.x, K4.y))));
+        Hg[q + 1] =
+            f2_fma(s23, c[e / 2 + 1], f2_fma(xo2, f2(Y4.z, Y4.w), f2_mul(nb2, f2(K4.z, K4.w))));
+        float h0, h1, h2, h3;
+        f2_get(Hg[q], h0, h1);
+        f2_get(Hg[q + 1], h2, h3);
+        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))));
       }
     }
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));  // the row's (group's) other half
@@ -520,7 +559,7 @@ __device__ __forceinline__ void pw_head(const PwArgs& a, const PwLayout& L, uint
         uint32_t b[BW];  // low byte = the code (two's complement) from 1.5 2^23 + rint(q)
 #pragma unroll
         for (int e = 0; e < BW; e += 2) {
-          const F2 y = f2_add(f2_quot(f2(Hg[mb * BW + e], Hg[mb * BW + e + 1]), inv2, ns2), magic2);
+          const F2 y = f2_add(f2_quot(Hg[(mb * BW + e) / 2], inv2, ns2), magic2);
           float y0, y1;
           f2_get(y, y0, y1);
           b[e] = __float_as_uint(y0);
@@ -551,16 +590,22 @@ __device__ __forceinline__ void pw_head(const PwArgs& a, const PwLayout& L, uint
         const int m = gi * GB + mb;
         uint32_t lo = 0, hi = 0;
 #pragma unroll
-        for (int e = 0; e < BW; ++e) {
-          const int c = s2 > 0.f ? (int)rintf(__fdiv_rn(Hg[mb * BW + e], s2)) : 0;
-          if constexpr (P::INT4) {
-            const uint32_t nib = (uint32_t)(c & 0xF) << (4 * (e & 7));
-            if (e < 8) lo |= nib;
-            else hi |= nib;
-          } else {
-            const uint32_t byte = (uint32_t)(c & 0xFF) << (8 * (e & 3));
-            if (e < 4) lo |= byte;
-            else hi |= byte;
+        for (int e = 0; e < BW; e += 2) {
+          float hv[2];
+          f2_get(Hg[(mb * BW + e) / 2], hv[0], hv[1]);
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int c = s2 > 0.f ? (int)rintf(__fdiv_rn(hv[u], s2)) : 0;
+            const int ee = e + u;
+            if constexpr (P::INT4) {
+              const uint32_t nib = (uint32_t)(c & 0xF) << (4 * (ee & 7));
+              if (ee < 8) lo |= nib;
+              else hi |= nib;
+            } else {
+              const uint32_t byte = (uint32_t)(c & 0xFF) << (8 * (ee & 3));
+              if (ee < 4) lo |= byte;
+              else hi |= byte;
+            }
           }
         }
         w[2 * m] = lo;
@@ -605,24 +650,27 @@ __global__ void __launch_bounds__(kPwThreads, pw_ctas_per_sm<P>())
   if (tid == kPwIssuer)
     for (int s = 0; s < nstages && s < nh; ++s)
       pw_issue<P>(a, L, sm + s * L.stage_bytes, &bars[s], h0 + s);
-  for (int n = 0; n < nh; ++n) {
-    // refill the stage head n - 1 used, once its history tile has been read out
-    if (tid == kPwIssuer && n > 0 && n - 1 + nstages < nh) {
-      const int sp = (n - 1) % nstages;
-      bulk_wait_read_all();
-      pw_issue<P>(a, L, sm + sp * L.stage_bytes, &bars[sp], h0 + n - 1 + nstages);
+  // every head ends with one barrier, which also agrees that the next head's stage has landed
+  auto give_up = [&](int n) {
+    // give the copies still in flight (heads n .. n + nstages - 1) a bounded wait each before
+    // the CTA's shared memory goes away
+    if (tid == 0) {
+      pw_report(a.status, GDN_DEVICE_WAIT_TIMEOUT);
+      for (int m = n; m < nh && m < n + nstages; ++m)
+        (void)mbar_wait_bounded(&bars[m % nstages], (uint32_t)(m / nstages) & 1u);
     }
-    const int timed_out =
-        mbar_wait_bounded(&bars[n % nstages], (uint32_t)(n / nstages) & 1u) ? 0 : 1;
-    if (__syncthreads_or(timed_out)) {
-      // give the copies still in flight (heads n .. n + nstages - 1) a bounded wait each
-      // before the CTA's shared memory goes away
-      if (tid == 0) {
-        pw_report(a.status, GDN_DEVICE_WAIT_TIMEOUT);
-        for (int m = n; m < nh && m < n + nstages; ++m)
-          (void)mbar_wait_bounded(&bars[m % nstages], (uint32_t)(m / nstages) & 1u);
-      }
-      break;
+  };
+  if (__syncthreads_or(mbar_wait_bounded(&bars[0], 0u) ? 0 : 1)) {
+    give_up(0);
+    return;
+  }
+  for (int n = 0; n < nh; ++n) {
+    // with three stages or more, refill the stage of head n - 2, whose history tile has been
+    // read out by now (the store of head n - 1 may still be reading its own stage)
+    if (tid == kPwIssuer && nstages > 2 && n >= 2 && n - 2 + nstages < nh) {
+      bulk_wait_read_newest_pending();
+      const int sp = (n - 2) % nstages;
+      pw_issue<P>(a, L, sm + sp * L.stage_bytes, &bars[sp], h0 + n - 2 + nstages);
     }
     uint8_t* st = sm + (n % nstages) * L.stage_bytes;
     const int cnt = hcnt[n];
@@ -632,12 +680,26 @@ __global__ void __launch_bounds__(kPwThreads, pw_ctas_per_sm<P>())
     // the stage's generic-proxy writes are ordered before the bulk store that reads them and
     // the copies that later refill it
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-    __syncthreads();
-    if (ok && tid == kPwIssuer) {
-      const int head = h0 + n;
-      bulk_s2g(a.codes + (size_t)head * P::CODE_BYTES, st + L.codes, P::CODE_BYTES);
-      bulk_s2g(a.scales + (size_t)head * P::NSCALES, st + L.scales, 4u * P::NSCALES);
-      bulk_commit();
+    int timed_out = 0;
+    if (n + 1 < nh)
+      timed_out = mbar_wait_bounded(&bars[(n + 1) % nstages], (uint32_t)((n + 1) / nstages) & 1u)
+                      ? 0 : 1;
+    if (__syncthreads_or(timed_out)) {
+      give_up(n + 1);
+      break;
+    }
+    if (tid == kPwIssuer) {
+      if (ok) {
+        const int head = h0 + n;
+        bulk_s2g(a.codes + (size_t)head * P::CODE_BYTES, st + L.codes, P::CODE_BYTES);
+        bulk_s2g(a.scales + (size_t)head * P::NSCALES, st + L.scales, 4u * P::NSCALES);
+      }
+      bulk_commit();  // (an empty group for a skipped head keeps one group per head)
+      // with two stages the stage of head n is refilled as soon as it has been read out
+      if (nstages == 2 && n + 2 < nh) {
+        bulk_wait_read_all();
+        pw_issue<P>(a, L, st, &bars[n % 2], h0 + n + 2);
+      }
     }
   }
   if (tid == kPwIssuer) bulk_wait_all();

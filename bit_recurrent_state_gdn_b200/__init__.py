@@ -1,6 +1,6 @@
 """Windowed low-bit recurrent-state GDN / KDA decode for B200 (sm_100a).
 
-Python face of libgdnq (include/gdnq.h, include/gdnq_pw.h): the functions here carry the C ABI's names and only
+Python face of libgdnq (include/gdnq.h, gdnq_pw.h, gdnq_prefill.h): the functions here carry the C ABI's names and only
 marshal arguments -- torch tensors to device pointers, the current CUDA stream, status codes to
 exceptions. Every step of the computation runs in the library's CUDA kernels.
 """
@@ -28,3 +28,4 @@ from .pw import (  # noqa: F401
     gdn_pw_state_sizes,
     make_pw_config,
 )
+from .prefill import gdn_prefill  # noqa: F401,E402

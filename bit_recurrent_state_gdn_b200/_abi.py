@@ -1,4 +1,4 @@
-"""ctypes declarations of libgdnq's C ABI (include/gdnq.h, include/gdnq_pw.h). Loading fails loudly when the
+"""ctypes declarations of libgdnq's C ABI (include/gdnq.h, gdnq_pw.h, gdnq_prefill.h). Loading fails loudly when the
 library has not been built: there is no fallback path."""
 from __future__ import annotations
 
@@ -61,7 +61,7 @@ class gdn_pw_sizes(ctypes.Structure):
 
 _PWC, _PWS = ctypes.POINTER(gdn_pw_config), ctypes.POINTER(gdn_pw_state)
 
-# name -> (restype, argtypes); every symbol include/gdnq.h and include/gdnq_pw.h declare
+# name -> (restype, argtypes); every symbol the headers under include/ declare
 SIGNATURES = {
     "gdn_state_sizes": (_i32, [ctypes.POINTER(gdn_config), ctypes.POINTER(gdn_sizes)]),
     "gdn_state_quantize": (_i32, [ctypes.POINTER(gdn_config), _vp, ctypes.POINTER(gdn_state), _vp]),
@@ -83,6 +83,7 @@ SIGNATURES = {
     "gdn_pw_decode_step": (_i32, [_PWC, _PWS] + [_vp] * 7),
     "gdn_pw_decode_steps": (_i32, [_PWC, _PWS, _i32] + [_vp] * 7),
     "gdn_pw_materialize": (_i32, [_PWC, _PWS, _vp, _vp]),
+    "gdn_prefill": (_i32, [ctypes.POINTER(gdn_config), _i32] + [_vp] * 8),
     "gdn_status_string": (ctypes.c_char_p, [_i32]),
     "gdn_last_error": (ctypes.c_char_p, []),
 }

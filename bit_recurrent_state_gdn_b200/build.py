@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 OBJ_DIR = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libgdnq.so")
 SOURCES = ["api.cu", "window_int8.cu", "window_int4.cu", "window_mixed.cu", "baseline.cu",
-           "pw.cu"]
+           "pw.cu", "prefill.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -41,7 +41,7 @@ def _flags(ptxas_info: bool) -> list[str]:
 
 def _deps() -> list[str]:
     files = [os.path.join(CSRC, n) for n in os.listdir(CSRC)]
-    return files + [os.path.join(INCLUDE, n) for n in ("gdnq.h", "gdnq_pw.h")]
+    return files + [os.path.join(INCLUDE, n) for n in ("gdnq.h", "gdnq_pw.h", "gdnq_prefill.h")]
 
 
 def _stale() -> bool:

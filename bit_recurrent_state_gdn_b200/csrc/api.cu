@@ -7,8 +7,10 @@
 
 #include "baseline_kernels.cuh"
 #include "gdnq.h"
+#include "gdnq_prefill.h"
 #include "gdnq_pw.h"
 #include "launch.h"
+#include "prefill_args.h"
 #include "pw_kernels.cuh"
 #include "window_kernels.cuh"
 
@@ -664,6 +666,54 @@ gdn_status gdn_pw_materialize(const gdn_pw_config* cfg, const gdn_pw_state* stat
   const cudaError_t e = gdnq::launch_pw(gdnq::PwOp::Materialize, *cfg, a, (int)pw_heads(cfg),
                                         (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "gdn_pw_materialize");
+  return GDN_OK;
+}
+
+gdn_status gdn_prefill(const gdn_config* cfg, int32_t L, const void* q, const void* k,
+                       const void* v, const float* g, const float* beta, void* o, float* S,
+                       gdn_stream_t stream) {
+  g_last_error[0] = 0;
+  if (!cfg) return fail(GDN_ERR_INVALID_ARG, "cfg is null");
+  if (cfg->B < 0 || cfg->H < 0)
+    return fail(GDN_ERR_INVALID_ARG, "B=%d, H=%d must be >= 0", cfg->B, cfg->H);
+  if (heads_of(cfg) > INT32_MAX) return fail(GDN_ERR_INVALID_ARG, "B*H exceeds 2^31-1");
+  if (cfg->gate != GDN_GATE_SCALAR && cfg->gate != GDN_GATE_DIAG)
+    return fail(GDN_ERR_INVALID_ARG, "gate=%d is not a gdn_gate_kind", cfg->gate);
+  if (cfg->act_dtype != GDN_DTYPE_F32 && cfg->act_dtype != GDN_DTYPE_BF16)
+    return fail(GDN_ERR_INVALID_ARG, "act_dtype=%d is not a gdn_dtype", cfg->act_dtype);
+  if (cfg->d_k < 1 || cfg->d_v < 1)
+    return fail(GDN_ERR_INVALID_ARG, "d_k=%d, d_v=%d", cfg->d_k, cfg->d_v);
+  if (cfg->d_k != 128 || cfg->d_v != 128)
+    return fail(GDN_ERR_UNSUPPORTED, "prefill is built for d_k = d_v = 128");
+  if (cfg->gate != GDN_GATE_SCALAR)
+    return fail(GDN_ERR_UNSUPPORTED, "prefill is built for the scalar (GDN) gate");
+  if (cfg->act_dtype != GDN_DTYPE_BF16)
+    return fail(GDN_ERR_UNSUPPORTED, "prefill is built for bf16 activations");
+  if (L < 0) return fail(GDN_ERR_INVALID_ARG, "L=%d must be >= 0", L);
+  if (heads_of(cfg) == 0) return GDN_OK;
+  if ((size_t)heads_of(cfg) * (size_t)L * 128 > (size_t)INT64_MAX / 4)
+    return fail(GDN_ERR_INVALID_ARG, "B*H*L is too large");
+  gdn_status st;
+  if ((st = need_ptr(S, "S")) != GDN_OK) return st;
+  if (L > 0) {
+    if ((st = need_ptr(q, "q")) != GDN_OK) return st;
+    if ((st = need_ptr(k, "k")) != GDN_OK) return st;
+    if ((st = need_ptr(v, "v")) != GDN_OK) return st;
+    if ((st = need_ptr(g, "g", 4)) != GDN_OK) return st;
+    if ((st = need_ptr(beta, "beta", 4)) != GDN_OK) return st;
+    if ((st = need_ptr(o, "o", 4)) != GDN_OK) return st;
+  }
+  gdnq::PfArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.g = g;
+  a.beta = beta;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.S = S;
+  a.L = L;
+  const cudaError_t e = gdnq::launch_prefill(a, (int)heads_of(cfg), (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "gdn_prefill");
   return GDN_OK;
 }
 

@@ -182,8 +182,9 @@ __device__ __forceinline__ F2 f2_quot(F2 x, F2 inv, F2 neg_s) {
   return f2_fma(r, inv, q1);
 }
 
-// The correctly rounded quotient x / d for a constant divisor d, given inv_d = the correctly
-// rounded 1 / d (the same correction, scalar). Valid while x / d is normal or zero.
+// The correctly rounded quotient x / d given inv_d = the correctly rounded 1 / d (the same
+// correction, scalar; d a constant or not). Valid while x / d is normal or zero and 1 / d is
+// finite and normal.
 __device__ __forceinline__ float quot_const(float x, float d, float inv_d) {
   const float q1 = x * inv_d;
   const float r = fmaf(-q1, d, x);

@@ -11,6 +11,7 @@ namespace gdnq {
 struct WinArgs;
 struct BaseArgs;
 struct PwArgs;
+struct PfArgs;
 
 enum class WinOp { Step, Flush, Materialize, Quantize };
 
@@ -37,6 +38,9 @@ cudaError_t launch_window_mixed(WinOp op, const gdn_config& cfg, const WinArgs& 
 enum class PwOp { Step, Materialize };
 cudaError_t launch_pw(PwOp op, const gdn_pw_config& cfg, const PwArgs& a, int heads,
                       cudaStream_t stream);
+// Chunkwise prefill: one CTA per head.
+cudaError_t launch_prefill(const PfArgs& a, int heads, cudaStream_t stream);
+size_t prefill_smem_bytes();
 cudaError_t launch_baseline(const gdn_config& cfg, const BaseArgs& a, int heads,
                             cudaStream_t stream);
 

@@ -1,0 +1,19 @@
+// Arguments of the chunkwise prefill kernel (shared by the kernel and the C ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+
+namespace gdnq {
+
+struct PfArgs {
+  const __nv_bfloat16* q;  // [heads][L][128]
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const float* g;          // [heads][L]
+  const float* beta;
+  __nv_bfloat16* o;        // [heads][L][128]
+  float* S;                // [heads][128][128], in place
+  int L;
+};
+
+}  // namespace gdnq

@@ -1,0 +1,50 @@
+/*
+ * gdnq_prefill.h -- C ABI of libgdnq, part 3: chunkwise-parallel GDN prefill, the step that
+ * produces the recurrent state decode starts from, for NVIDIA B200 (sm_100a).
+ *
+ * The method ("LinQuant: Functional Invariances for Low-Precision Linear Recurrences",
+ * Abstract: a linear recurrence's prefill evaluated chunk by chunk as dense matrix products):
+ * the L tokens of a prompt run through the gated delta rule of gdnq.h,
+ *     S_t = S_{t-1} a_t (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,     o_t = S_t q_t,
+ * for every (sequence, head), in chunks of 64 tokens whose intra-chunk part is a handful of
+ * 64 x 64 and 64 x 128 products (the UT / WY form of the delta rule); only the state passes
+ * from one chunk to the next. The final state can then be quantized for decode with
+ * gdn_state_quantize.
+ *
+ * Conventions are those of gdnq.h (device pointers, caller-owned buffers, asynchronous work on
+ * `stream`, argument checks before anything is enqueued, B * H == 0 a valid empty batch).
+ */
+#ifndef GDNQ_PREFILL_H
+#define GDNQ_PREFILL_H
+
+#include "gdnq.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/*
+ * L prompt tokens of every head, in place on S.
+ *   cfg     B, H, d_k = d_v = 128, gate GDN_GATE_SCALAR, act_dtype GDN_DTYPE_BF16 (this build);
+ *           W, r, fmt and buf_dtype are ignored.
+ *   L       tokens per sequence, >= 0 (any length: a last partial chunk is padded inside the
+ *           kernel with tokens that change nothing).
+ *   q, k, v device bf16 [B][H][L][D] (head-major: each head's tokens contiguous), 16-byte
+ *           aligned; k and q as the decode step takes them (the layer's normalisation applied).
+ *   g       device fp32 [B][H][L], the log of the scalar gate; beta device fp32 [B][H][L].
+ *   o       device bf16 [B][H][L][D], written for every token.
+ *   S       device fp32 [B][H][D][D], 16-byte aligned: the state before the prompt on entry, after
+ *           it on return (row = value channel, column = key channel).
+ * Arithmetic: products on tensor cores with fp32 accumulation; q, k, v enter exactly, every
+ * fp32 operand (the state, the chunk's triangular inverse, the corrected values, the decayed
+ * scores, the write vectors) as the sum of two bf16 parts; the triangular inverse in fp32.
+ */
+gdn_status gdn_prefill(const gdn_config* cfg, int32_t L, const void* q, const void* k,
+                       const void* v, const float* g, const float* beta, void* o, float* S,
+                       gdn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDNQ_PREFILL_H */

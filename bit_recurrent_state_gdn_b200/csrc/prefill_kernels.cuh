@@ -54,6 +54,26 @@ struct PfLayout {
   static constexpr uint32_t TOTAL = GATE + 4 * kPfC * 4;
 };
 
+// 16-byte asynchronous global -> shared copy; src_bytes = 0 fills the 16 bytes with zeros.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
+// One 64 x 128 bf16 tile of chunk rows [c0, c0 + 64) of a head (rows >= n zero) into a padded
+// shared tile, as asynchronous copies (4 per thread).
+__device__ __forceinline__ void load_tile_async(__nv_bfloat16* dst, const __nv_bfloat16* src,
+                                                size_t row0, int n) {
+  for (int e = threadIdx.x; e < kPfC * 16; e += kPfThreads) {
+    const int r = e >> 4, ch = e & 15;
+    const __nv_bfloat16* g = src + (row0 + (r < n ? r : 0)) * kPfD + 8 * ch;
+    cp_async16(dst + r * kLd128 + 8 * ch, g, r < n ? 16 : 0);
+  }
+}
+
 __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
   hi = __float2bfloat16_rn(x);
   lo = __float2bfloat16_rn(x - __bfloat162float(hi));
@@ -123,7 +143,8 @@ __device__ __forceinline__ void store_split(const float (&acc)[NT][4], __nv_bflo
 
 // R = (I + A)^{-1} for the strictly lower triangular 64 x 64 A (fp32, stride kLdF), blocked in
 // 16 x 16: diagonal blocks by forward substitution (one lane per column), then
-// R_ij = -R_ii sum_{j <= k < i} A_ik R_kj level by level (i - j = 1, 2, 3).
+// R_ij = -R_ii sum_{j <= k < i} A_ik R_kj level by level (i - j = 1, 2, 3), each level spread
+// over all threads. xs: 3 x 256 floats of scratch.
 __device__ __forceinline__ void unit_lower_inverse(const float* A, float* R, float* xs) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // diagonal blocks: warps 0-1, lanes 0-15 / 16-31 take blocks 2 warp and 2 warp + 1
@@ -141,35 +162,27 @@ __device__ __forceinline__ void unit_lower_inverse(const float* A, float* R, flo
     for (int t = 0; t < 16; ++t) R[(o + t) * kLdF + o + c] = rc[t];
   }
   __syncthreads();
-  // off-diagonal blocks, one warp per block: lane = (row half h, column c): rows 8h..8h+7
+  // off-diagonal blocks, every thread: level lvl has the blocks (j + lvl, j), j < 4 - lvl;
+  // first X_j = sum_{j <= kb < i} A_{i,kb} R_{kb,j}, then R_ij = -R_ii X_j
   for (int lvl = 1; lvl < 4; ++lvl) {
-    const int nb = 4 - lvl;  // blocks (j + lvl, j), j = 0 .. nb - 1
-    if (warp < nb) {
-      const int j = warp, i = j + lvl;
-      const int c = lane & 15, h = lane >> 4;
-      float* X = xs + 256 * warp;
-      // X = sum_{k = j}^{i-1} A_ik R_kj  (rows 8h..8h+7, column c)
+    const int nb = 4 - lvl;
+    for (int e = tid; e < 256 * nb; e += kPfThreads) {
+      const int j = e >> 8, i = j + lvl, r = (e >> 4) & 15, c = e & 15;
+      float sum = 0.f;
+      for (int kb = j; kb < i; ++kb) {
 #pragma unroll
-      for (int rr = 0; rr < 8; ++rr) {
-        const int r = 8 * h + rr;
-        float sum = 0.f;
-        for (int kb = j; kb < i; ++kb) {
-#pragma unroll
-          for (int s = 0; s < 16; ++s)
-            sum = fmaf(A[(16 * i + r) * kLdF + 16 * kb + s], R[(16 * kb + s) * kLdF + 16 * j + c], sum);
-        }
-        X[r * 16 + c] = sum;
+        for (int s = 0; s < 16; ++s)
+          sum = fmaf(A[(16 * i + r) * kLdF + 16 * kb + s], R[(16 * kb + s) * kLdF + 16 * j + c], sum);
       }
-      __syncwarp();
-      // R_ij = -R_ii X
+      xs[e] = sum;
+    }
+    __syncthreads();
+    for (int e = tid; e < 256 * nb; e += kPfThreads) {
+      const int j = e >> 8, i = j + lvl, r = (e >> 4) & 15, c = e & 15;
+      float sum = 0.f;
 #pragma unroll
-      for (int rr = 0; rr < 8; ++rr) {
-        const int r = 8 * h + rr;
-        float sum = 0.f;
-#pragma unroll
-        for (int s = 0; s < 16; ++s) sum = fmaf(R[(16 * i + r) * kLdF + 16 * i + s], X[s * 16 + c], sum);
-        R[(16 * i + r) * kLdF + 16 * j + c] = -sum;
-      }
+      for (int s = 0; s < 16; ++s) sum = fmaf(R[(16 * i + r) * kLdF + 16 * i + s], xs[(j << 8) + s * 16 + c], sum);
+      R[(16 * i + r) * kLdF + 16 * j + c] = -sum;
     }
     __syncthreads();
   }
@@ -219,15 +232,16 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const PfArgs a) 
   const int m0 = 16 * mt;
   for (int c0 = 0; c0 < L; c0 += kPfC) {
     const int n = min(kPfC, L - c0);
-    // ---- load the chunk (rows past the end are zero: beta = 0, g = 0 leave S unchanged) ----
-    for (int e = tid; e < 3 * kPfC * 16; e += kPfThreads) {
-      const int mat = e >> 10, r = (e >> 4) & (kPfC - 1), ch = e & 15;
-      const bf* src = mat == 0 ? a.q : (mat == 1 ? a.k : a.v);
-      uint4 val = make_uint4(0u, 0u, 0u, 0u);
-      if (r < n) val = *reinterpret_cast<const uint4*>(src + ((size_t)head * L + c0 + r) * kPfD + 8 * ch);
-      bf* dst = mat == 0 ? Qs : (mat == 1 ? Ks : Vs);
-      *reinterpret_cast<uint4*>(dst + r * kLd128 + 8 * ch) = val;
+    // ---- the chunk's tiles (rows past the end are zero: beta = 0, g = 0 leave S unchanged):
+    // K now, Q and V were prefetched during the previous chunk (the first chunk loads all three)
+    const size_t row0 = (size_t)head * L + c0;
+    if (c0 == 0) {
+      load_tile_async(Qs, a.q, row0, n);
+      load_tile_async(Vs, a.v, row0, n);
     }
+    load_tile_async(Ks, a.k, row0, n);
+    cp_async_commit();
+    const int c1 = c0 + kPfC, n1 = min(kPfC, L - c1);  // the next chunk
     if (warp == 0) {  // cumulative log-gate over the chunk, two tokens per lane
       const int t0 = 2 * lane;
       const float g0 = t0 < n ? a.g[(size_t)head * L + c0 + t0] : 0.f;
@@ -250,6 +264,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const PfArgs a) 
       bet[t0] = t0 < n ? a.beta[(size_t)head * L + c0 + t0] : 0.f;
       bet[t0 + 1] = t0 + 1 < n ? a.beta[(size_t)head * L + c0 + t0 + 1] : 0.f;
     }
+    cp_async_wait_all();
     __syncthreads();
 
     // ---- A = beta_t e^{G_t - G_s} K K^T (s < t); V' = V - Diag(e^G) K S^T --------------------
@@ -262,7 +277,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const PfArgs a) 
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int t = m0 + gid + 8 * (e >> 1), s = 32 * nh + 8 * nt + 2 * q4 + (e & 1);
-          Af[t * kLdF + s] = s < t ? bet[t] * expf(Gs[t] - Gs[s]) * acc[nt][e] : 0.f;
+          Af[t * kLdF + s] = s < t ? bet[t] * __expf(Gs[t] - Gs[s]) * acc[nt][e] : 0.f;
         }
       float ks[8][4];
       zero_acc(ks);
@@ -273,6 +288,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const PfArgs a) 
       });
     }
     __syncthreads();
+    if (n1 > 0) {  // V is read out: the next chunk's V
+      load_tile_async(Vs, a.v, row0 + kPfC, n1);
+      cp_async_commit();
+    }
 
     // ---- T = (I + A)^{-1} Diag(beta), split ---------------------------------------------------
     unit_lower_inverse(Af, Rf, xs);
@@ -300,10 +319,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const PfArgs a) 
     float pacc[4][4];
     zero_acc(pacc);
     warp_mma<4, 8, false, false>(pacc, q_b, kLd128, m0, k_b, kLd128, 32 * nh, 0);
-    __syncthreads();  // V' and T are read out
+    __syncthreads();  // V', T and Q are read out
+    if (n1 > 0) {  // the next chunk's Q
+      load_tile_async(Qs, a.q, row0 + kPfC, n1);
+      cp_async_commit();
+    }
     store_split(uacc, Xhi, Xlo, kLd128, m0, 64 * nh, [](int, int, float x) { return x; });
     store_split(pacc, Thi, Tlo, kLd64, m0, 32 * nh, [&](int t, int s, float x) {
-      return s <= t ? expf(Gs[t] - Gs[s]) * x : 0.f;
+      return s <= t ? __expf(Gs[t] - Gs[s]) * x : 0.f;
     });
     __syncthreads();
 

@@ -59,6 +59,9 @@ def parse_args():
     p.add_argument("--ref-heads", type=int, default=2048)
     p.add_argument("--pw-only", action="store_true",
                    help="run only the pure-write window legs (profiling captures)")
+    p.add_argument("--prefill-only", action="store_true",
+                   help="run only the chunkwise prefill leg (profiling captures)")
+    p.add_argument("--prefill-batch", type=int, default=None, help="override the prefill B")
     return p.parse_args()
 
 
@@ -293,6 +296,14 @@ def main():
     if args.impl == "reference":
         reference_arm(args, rank, world)
         return
+    if args.prefill_only:
+        import torch
+
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        line = {"prefill": prefill_leg(args, torch.device("cuda"))}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return
 
     import numpy as np
     import torch
@@ -407,6 +418,10 @@ def main():
         line["pure_write_s8"] = {f: pw_leg(wl.with_(fmt=f), 8, S0, inp, o, peak)
                                  for f in ("int4_g32", "int8")}
 
+    # ---- chunkwise prefill of a prompt batch (its own workload) ----------------------------
+    if not args.no_baselines and world == 1:
+        line["prefill"] = prefill_leg(args, dev)
+
     # ---- high-precision-state baselines on the same inputs ---------------------------------
     if not args.no_baselines:
         line["baselines"] = {}
@@ -487,6 +502,68 @@ def pw_step_bytes(wl, Wp: int) -> int:
     read = hist + 2 * Wp * D + 8 * Wp + 3 * D * act + g + 4 + 4
     write = hist + ((Wp + 1) * D + 4 * (Wp + 1) if Wp else 0) + D * act + 4
     return read + write
+
+
+def prefill_flops_per_chunk(C: int = 64, D: int = 128) -> int:
+    """The UT-form products of one chunk with single-precision operands: K K^T, Q K^T (C x C x D),
+    K S^T, Q S^T (C x D x D), T V', P U (C x C x D) and the state update U^T K (D x C x D)."""
+    return 2 * (4 * C * C * D + 2 * C * D * D + D * C * D)
+
+
+def peak_bf16():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured bf16_tflops (burst)"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback"
+
+
+def prefill_leg(args, dev, reps: int = 5):
+    """gdn_prefill over the gdn-prefill workload (B x H heads, L-token prompts, zero initial
+    state): the median of `reps` launches after two untimed ones, CUDA events."""
+    import torch
+
+    import bit_recurrent_state_gdn_b200 as gdn
+
+    wl = WORKLOADS["gdn-prefill"]
+    if args.prefill_batch:
+        wl = wl.with_(B=args.prefill_batch)
+    L = wl.T
+    inp = decode_inputs(wl, dev)
+    hm = {n: t.permute(1, 2, 0, *range(3, t.dim())).contiguous() for n, t in inp.items()}
+    del inp
+    cfg = gdn.make_config(wl.B, wl.H, wl.D, gate="scalar", act="bf16")
+    o = torch.empty_like(hm["q"])
+    S = torch.zeros((wl.B, wl.H, wl.D, wl.D), dtype=torch.float32, device=dev)
+    for _ in range(2):
+        gdn.gdn_prefill(cfg, hm["q"], hm["k"], hm["v"], hm["g"], hm["beta"], o, S)
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(reps):
+        S.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        gdn.gdn_prefill(cfg, hm["q"], hm["k"], hm["v"], hm["g"], hm["beta"], o, S)
+        e1.record()
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    t = sorted(ms)[len(ms) // 2]
+    if not bool(torch.isfinite(S).all()):
+        raise RuntimeError("prefill: non-finite state")
+    chunks = wl.heads * ((L + 63) // 64)
+    flops = chunks * prefill_flops_per_chunk()
+    tf = flops / (t / 1e3) / 1e12
+    peak, src = peak_bf16()
+    return {"value": wl.heads * L / (t / 1e3), "unit": "head-tokens/s", "ms_per_launch": t,
+            "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "L": L, "D": wl.D,
+                       "gate": "scalar", "act": "bf16", "chunk": 64},
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tf / peak, "peak_source": src,
+                         "flops_per_launch": flops,
+                         "note": "UT-form products at single precision; the kernel issues "
+                                 "twice that on mma.sync (hi/lo bf16 splits)"},
+            "kernel": "prefill_kernel (one CTA per head, 64-token chunks)"}
 
 
 def pw_leg(wl, Wp, S0, inp, o, peak):

@@ -42,6 +42,9 @@ WORKLOADS = {
                               seed=1004),
     # serving-scale batch (the throughput workload)
     "gdn-serving": Workload("gdn-serving", B=1024, H=32, D=128, T=256, W=64, seed=1005),
+    # prompt prefill before decode: T = prompt length L, one chunkwise launch over all of it
+    "gdn-prefill": Workload("gdn-prefill", B=8, H=32, D=128, T=4096, W=64, warmup=0,
+                            seed=1006),
 }
 
 

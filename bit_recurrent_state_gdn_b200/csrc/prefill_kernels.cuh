@@ -13,7 +13,8 @@
 // over the chunk: (I + A) U = Diag(beta) V').
 //
 // One CTA per head, 256 threads, the state in registers as mma accumulators (warp w: rows
-// 16w..16w+15). The products run on mma.sync bf16 with fp32 accumulation; q, k, v are exact in
+// 16w..16w+15), which also serve, split into hi / lo bf16 on the fly, as the B operand of the
+// products with S^T (warp w computes their columns 16w..16w+15). The products run on mma.sync bf16 with fp32 accumulation; q, k, v are exact in
 // bf16, and every fp32 operand (S, T, V', P, U) is split into hi + lo bf16 parts, so products
 // carry about 16 significant bits of each fp32 operand. The triangular inverse is blocked
 // (16 x 16 diagonal blocks by forward substitution, off-diagonal blocks by three levels of
@@ -39,18 +40,17 @@ constexpr int kLdF = 65;     // fp32 row stride of 64 x 64 fp32 tiles
 // Shared memory (bytes)
 struct PfLayout {
   static constexpr uint32_t Q = 0;
-  static constexpr uint32_t K = Q + kPfC * kLd128 * 2;
-  static constexpr uint32_t V = K + kPfC * kLd128 * 2;
-  static constexpr uint32_t S_HI = V + kPfC * kLd128 * 2;
-  static constexpr uint32_t S_LO = S_HI + kPfD * kLd128 * 2;
-  static constexpr uint32_t X_HI = S_LO + kPfD * kLd128 * 2;  // V', then U, then e^{G_C-G} U
+  static constexpr uint32_t K0 = Q + kPfC * kLd128 * 2;        // K of even chunks
+  static constexpr uint32_t K1 = K0 + kPfC * kLd128 * 2;       // K of odd chunks
+  static constexpr uint32_t V = K1 + kPfC * kLd128 * 2;
+  static constexpr uint32_t X_HI = V + kPfC * kLd128 * 2;      // V', then U, then e^{G_C-G} U
   static constexpr uint32_t X_LO = X_HI + kPfC * kLd128 * 2;
-  static constexpr uint32_t T_HI = X_LO + kPfC * kLd128 * 2;  // T, then P
+  static constexpr uint32_t T_HI = X_LO + kPfC * kLd128 * 2;   // T, then P
   static constexpr uint32_t T_LO = T_HI + kPfC * kLd64 * 2;
-  static constexpr uint32_t AF = T_LO + kPfC * kLd64 * 2;     // A (fp32)
-  static constexpr uint32_t RF = AF + kPfC * kLdF * 4;        // R = (I + A)^{-1} (fp32)
-  static constexpr uint32_t XS = RF + kPfC * kLdF * 4;        // 8 warps x 16 x 16 fp32 scratch
-  static constexpr uint32_t GATE = XS + 8 * 256 * 4;          // G, e^G, e^{G_C - G}, beta
+  static constexpr uint32_t AF = T_LO + kPfC * kLd64 * 2;      // A (fp32)
+  static constexpr uint32_t RF = AF + kPfC * kLdF * 4;         // R = (I + A)^{-1} (fp32)
+  static constexpr uint32_t XS = RF + kPfC * kLdF * 4;         // 3 x 256 fp32 scratch
+  static constexpr uint32_t GATE = XS + 3 * 256 * 4;           // G, e^G, e^{G_C - G}, beta
   static constexpr uint32_t TOTAL = GATE + 4 * kPfC * 4;
 };
 
@@ -188,6 +188,64 @@ __device__ __forceinline__ void unit_lower_inverse(const float* A, float* R, flo
   }
 }
 
+// acc[2 mt + nn] (rows 16 mt.., columns 8 nn.. of this warp's 16-column slab v0..v0+15)
+// += A (64 x 128, a bf16 tile at a_base) * S^T restricted to the slab, S in this warp's
+// accumulators: the accumulator layout of the warp's state rows v0..v0+15 is the B-fragment
+// layout of those columns of S^T, so each B register is two accumulator entries, split into
+// hi and lo bf16 on the fly.
+__device__ __forceinline__ void mma_state_slab(float (&acc)[8][4], uint32_t a_base,
+                                               const float (&sacc)[16][4]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    uint32_t bh[2][2], bl[2][2];
+#pragma unroll
+    for (int nn = 0; nn < 2; ++nn)
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const float x0 = sacc[2 * ks + half][2 * nn], x1 = sacc[2 * ks + half][2 * nn + 1];
+        const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
+        bh[nn][half] = pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
+        bl[nn][half] = pack_bf16(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
+      }
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      uint32_t a[4];
+      ldsm_x4(a_base + 2u * ((16 * mt + (lane & 15)) * kLd128 + 16 * ks + 8 * (lane >> 4)), a);
+#pragma unroll
+      for (int nn = 0; nn < 2; ++nn) {
+        mma_bf16(acc[2 * mt + nn], a, bh[nn][0], bh[nn][1]);
+        mma_bf16(acc[2 * mt + nn], a, bl[nn][0], bl[nn][1]);
+      }
+    }
+  }
+}
+
+// A slab accumulator (tiles 2 mt + nn: rows 16 mt.., columns v0 + 8 nn..) into hi / lo tiles
+// after f(row, column, value).
+template <class F>
+__device__ __forceinline__ void store_split_slab(const float (&acc)[8][4], __nv_bfloat16* hi,
+                                                 __nv_bfloat16* lo, int ld, int v0, F f) {
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    const float(&t2)[2][4] = *reinterpret_cast<const float(*)[2][4]>(&acc[2 * mt]);
+    store_split(t2, hi, lo, ld, 16 * mt, v0, f);
+  }
+}
+
+// acc (slab) += A (64 x 64 hi / lo tiles, rows t) * B (64 x 128 hi / lo tiles stored [s][v],
+// columns v0..v0+15): the three-term split product.
+__device__ __forceinline__ void mma_slab_split3(float (&acc)[8][4], uint32_t ahi, uint32_t alo,
+                                                uint32_t bhi, uint32_t blo, int v0) {
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    float(&t2)[2][4] = *reinterpret_cast<float(*)[2][4]>(&acc[2 * mt]);
+    warp_mma<2, 4, false, true>(t2, ahi, kLd64, 16 * mt, bhi, kLd128, v0, 0);
+    warp_mma<2, 4, false, true>(t2, ahi, kLd64, 16 * mt, blo, kLd128, v0, 0);
+    warp_mma<2, 4, false, true>(t2, alo, kLd64, 16 * mt, bhi, kLd128, v0, 0);
+  }
+}
+
 __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const PfArgs a) {
   using bf = __nv_bfloat16;
   extern __shared__ __align__(128) uint8_t sm[];
@@ -195,10 +253,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const PfArgs a) 
   const int gid = lane >> 2, q4 = lane & 3;
   const int L = a.L;
   bf* Qs = reinterpret_cast<bf*>(sm + PfLayout::Q);
-  bf* Ks = reinterpret_cast<bf*>(sm + PfLayout::K);
+  bf* K0s = reinterpret_cast<bf*>(sm + PfLayout::K0);
+  bf* K1s = reinterpret_cast<bf*>(sm + PfLayout::K1);
   bf* Vs = reinterpret_cast<bf*>(sm + PfLayout::V);
-  bf* Shi = reinterpret_cast<bf*>(sm + PfLayout::S_HI);
-  bf* Slo = reinterpret_cast<bf*>(sm + PfLayout::S_LO);
   bf* Xhi = reinterpret_cast<bf*>(sm + PfLayout::X_HI);
   bf* Xlo = reinterpret_cast<bf*>(sm + PfLayout::X_LO);
   bf* Thi = reinterpret_cast<bf*>(sm + PfLayout::T_HI);
@@ -210,42 +267,41 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const PfArgs a) 
   float* eG = Gs + kPfC;   // e^{G_t}
   float* eGC = eG + kPfC;  // e^{G_C - G_t}
   float* bet = eGC + kPfC;
-  const uint32_t q_b = smem_u32(Qs), k_b = smem_u32(Ks), shi_b = smem_u32(Shi), slo_b = smem_u32(Slo);
+  const uint32_t q_b = smem_u32(Qs);
   const uint32_t xhi_b = smem_u32(Xhi), xlo_b = smem_u32(Xlo), thi_b = smem_u32(Thi), tlo_b = smem_u32(Tlo);
 
-  // the state: warp w holds rows 16w..16w+15, all 128 columns, in accumulator layout
+  // the state: warp w holds rows 16w..16w+15, all 128 columns, in accumulator layout; it also
+  // computes every chunk product whose columns are value channels for the slab v0..v0+15
   float sacc[16][4];
   float* Sg = a.S + (size_t)head * kPfD * kPfD;
-  {
-    const int v0 = 16 * warp + gid;
+  const int v0 = 16 * warp;
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      const int j = 8 * nt + 2 * q4;
-      const float2 r0 = *reinterpret_cast<const float2*>(Sg + v0 * kPfD + j);
-      const float2 r1 = *reinterpret_cast<const float2*>(Sg + (v0 + 8) * kPfD + j);
-      sacc[nt][0] = r0.x; sacc[nt][1] = r0.y; sacc[nt][2] = r1.x; sacc[nt][3] = r1.y;
-    }
-    store_split(sacc, Shi, Slo, kLd128, 16 * warp, 0, [](int, int, float x) { return x; });
+  for (int nt = 0; nt < 16; ++nt) {
+    const int j = 8 * nt + 2 * q4;
+    const float2 r0 = *reinterpret_cast<const float2*>(Sg + (v0 + gid) * kPfD + j);
+    const float2 r1 = *reinterpret_cast<const float2*>(Sg + (v0 + gid + 8) * kPfD + j);
+    sacc[nt][0] = r0.x; sacc[nt][1] = r0.y; sacc[nt][2] = r1.x; sacc[nt][3] = r1.y;
   }
 
-  const int mt = warp & 3, nh = warp >> 2;  // chunk-row tile and column half of this warp
+  const int mt = warp & 3, nh = warp >> 2;  // the C x C products: row tile and column half
   const int m0 = 16 * mt;
-  for (int c0 = 0; c0 < L; c0 += kPfC) {
-    const int n = min(kPfC, L - c0);
-    // ---- the chunk's tiles (rows past the end are zero: beta = 0, g = 0 leave S unchanged):
-    // K now, Q and V were prefetched during the previous chunk (the first chunk loads all three)
-    const size_t row0 = (size_t)head * L + c0;
-    if (c0 == 0) {
-      load_tile_async(Qs, a.q, row0, n);
-      load_tile_async(Vs, a.v, row0, n);
-    }
-    load_tile_async(Ks, a.k, row0, n);
+  if (L > 0) {  // the first chunk's tiles
+    const int n = min(kPfC, L);
+    load_tile_async(Qs, a.q, (size_t)head * L, n);
+    load_tile_async(Vs, a.v, (size_t)head * L, n);
+    load_tile_async(K0s, a.k, (size_t)head * L, n);
     cp_async_commit();
-    const int c1 = c0 + kPfC, n1 = min(kPfC, L - c1);  // the next chunk
+  }
+  for (int c0 = 0, ci = 0; c0 < L; c0 += kPfC, ++ci) {
+    const int n = min(kPfC, L - c0);
+    const size_t row0 = (size_t)head * L + c0;
+    const int n1 = min(kPfC, L - c0 - kPfC);  // the next chunk (<= 0: none)
+    bf* Ks = (ci & 1) ? K1s : K0s;
+    const uint32_t k_b = smem_u32(Ks);
     if (warp == 0) {  // cumulative log-gate over the chunk, two tokens per lane
       const int t0 = 2 * lane;
-      const float g0 = t0 < n ? a.g[(size_t)head * L + c0 + t0] : 0.f;
-      const float g1 = t0 + 1 < n ? a.g[(size_t)head * L + c0 + t0 + 1] : 0.f;
+      const float g0 = t0 < n ? a.g[row0 + t0] : 0.f;
+      const float g1 = t0 + 1 < n ? a.g[row0 + t0 + 1] : 0.f;
       float incl = g0 + g1;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -261,11 +317,16 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const PfArgs a) 
       eG[t0 + 1] = expf(G1);
       eGC[t0] = expf(GC - G0);
       eGC[t0 + 1] = expf(GC - G1);
-      bet[t0] = t0 < n ? a.beta[(size_t)head * L + c0 + t0] : 0.f;
-      bet[t0 + 1] = t0 + 1 < n ? a.beta[(size_t)head * L + c0 + t0 + 1] : 0.f;
+      bet[t0] = t0 < n ? a.beta[row0 + t0] : 0.f;
+      bet[t0 + 1] = t0 + 1 < n ? a.beta[row0 + t0 + 1] : 0.f;
     }
-    cp_async_wait_all();
+    cp_async_wait_all();  // this chunk's Q, K, V (rows past the end are zero)
     __syncthreads();
+    if (n1 > 0) {  // the next chunk's K, into the other buffer (its last reader, the previous
+                   // chunk's state update, is behind the barrier above)
+      load_tile_async((ci & 1) ? K0s : K1s, a.k, row0 + kPfC, n1);
+      cp_async_commit();
+    }
 
     // ---- A = beta_t e^{G_t - G_s} K K^T (s < t); V' = V - Diag(e^G) K S^T --------------------
     {
@@ -281,9 +342,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const PfArgs a) 
         }
       float ks[8][4];
       zero_acc(ks);
-      warp_mma<8, 8, false, false>(ks, k_b, kLd128, m0, shi_b, kLd128, 64 * nh, 0);
-      warp_mma<8, 8, false, false>(ks, k_b, kLd128, m0, slo_b, kLd128, 64 * nh, 0);
-      store_split(ks, Xhi, Xlo, kLd128, m0, 64 * nh, [&](int t, int vv, float x) {
+      mma_state_slab(ks, k_b, sacc);
+      store_split_slab(ks, Xhi, Xlo, kLd128, v0, [&](int t, int vv, float x) {
         return __bfloat162float(Vs[t * kLd128 + vv]) - eG[t] * x;
       });
     }
@@ -301,21 +361,16 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const PfArgs a) 
     }
     __syncthreads();
 
-    // ---- U = T V'; P = M .* Q K^T; O = Diag(e^G) Q S^T ----------------------------------------
+    // ---- U = T V'; O = Diag(e^G) Q S^T (slabs); P = M .* Q K^T --------------------------------
     float uacc[8][4], oacc[8][4];
-    {
-      zero_acc(uacc);
-      warp_mma<8, 4, false, true>(uacc, thi_b, kLd64, m0, xhi_b, kLd128, 64 * nh, 0);
-      warp_mma<8, 4, false, true>(uacc, thi_b, kLd64, m0, xlo_b, kLd128, 64 * nh, 0);
-      warp_mma<8, 4, false, true>(uacc, tlo_b, kLd64, m0, xhi_b, kLd128, 64 * nh, 0);
-      zero_acc(oacc);
-      warp_mma<8, 8, false, false>(oacc, q_b, kLd128, m0, shi_b, kLd128, 64 * nh, 0);
-      warp_mma<8, 8, false, false>(oacc, q_b, kLd128, m0, slo_b, kLd128, 64 * nh, 0);
+    zero_acc(uacc);
+    mma_slab_split3(uacc, thi_b, tlo_b, xhi_b, xlo_b, v0);
+    zero_acc(oacc);
+    mma_state_slab(oacc, q_b, sacc);
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
+    for (int tt = 0; tt < 8; ++tt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) oacc[nt][e] *= eG[m0 + gid + 8 * (e >> 1)];
-    }
+      for (int e = 0; e < 4; ++e) oacc[tt][e] *= eG[16 * (tt >> 1) + gid + 8 * (e >> 1)];
     float pacc[4][4];
     zero_acc(pacc);
     warp_mma<4, 8, false, false>(pacc, q_b, kLd128, m0, k_b, kLd128, 32 * nh, 0);
@@ -324,32 +379,30 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const PfArgs a) 
       load_tile_async(Qs, a.q, row0 + kPfC, n1);
       cp_async_commit();
     }
-    store_split(uacc, Xhi, Xlo, kLd128, m0, 64 * nh, [](int, int, float x) { return x; });
+    store_split_slab(uacc, Xhi, Xlo, kLd128, v0, [](int, int, float x) { return x; });
     store_split(pacc, Thi, Tlo, kLd64, m0, 32 * nh, [&](int t, int s, float x) {
       return s <= t ? __expf(Gs[t] - Gs[s]) * x : 0.f;
     });
     __syncthreads();
 
     // ---- O += P U; outputs ----------------------------------------------------------------------
-    warp_mma<8, 4, false, true>(oacc, thi_b, kLd64, m0, xhi_b, kLd128, 64 * nh, 0);
-    warp_mma<8, 4, false, true>(oacc, thi_b, kLd64, m0, xlo_b, kLd128, 64 * nh, 0);
-    warp_mma<8, 4, false, true>(oacc, tlo_b, kLd64, m0, xhi_b, kLd128, 64 * nh, 0);
+    mma_slab_split3(oacc, thi_b, tlo_b, xhi_b, xlo_b, v0);
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+    for (int tt = 0; tt < 8; ++tt)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
-        const int t = m0 + gid + 8 * hh, vv = 64 * nh + 8 * nt + 2 * q4;
+        const int t = 16 * (tt >> 1) + gid + 8 * hh, vv = v0 + 8 * (tt & 1) + 2 * q4;
         if (t < n) {
           __nv_bfloat162 ov;
-          ov.x = __float2bfloat16_rn(oacc[nt][2 * hh]);
-          ov.y = __float2bfloat16_rn(oacc[nt][2 * hh + 1]);
-          *reinterpret_cast<__nv_bfloat162*>(a.o + ((size_t)head * L + c0 + t) * kPfD + vv) = ov;
+          ov.x = __float2bfloat16_rn(oacc[tt][2 * hh]);
+          ov.y = __float2bfloat16_rn(oacc[tt][2 * hh + 1]);
+          *reinterpret_cast<__nv_bfloat162*>(a.o + (row0 + t) * kPfD + vv) = ov;
         }
       }
     __syncthreads();  // U is read out
 
     // ---- S = e^{G_C} S + (Diag(e^{G_C - G}) U)^T K -------------------------------------------
-    store_split(uacc, Xhi, Xlo, kLd128, m0, 64 * nh, [&](int t, int, float x) { return eGC[t] * x; });
+    store_split_slab(uacc, Xhi, Xlo, kLd128, v0, [&](int t, int, float x) { return eGC[t] * x; });
     __syncthreads();
     {
       const float eC = eG[kPfC - 1];
@@ -358,21 +411,17 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const PfArgs a) 
 #pragma unroll
         for (int e = 0; e < 4; ++e) sacc[nt][e] *= eC;
       // A = (e^{G_C - G} U)^T: stored [t][v] = [k][m]; B = K stored [t][j] = [k][n]
-      warp_mma<16, 4, true, true>(sacc, xhi_b, kLd128, 16 * warp, k_b, kLd128, 0, 0);
-      warp_mma<16, 4, true, true>(sacc, xlo_b, kLd128, 16 * warp, k_b, kLd128, 0, 0);
+      warp_mma<16, 4, true, true>(sacc, xhi_b, kLd128, v0, k_b, kLd128, 0, 0);
+      warp_mma<16, 4, true, true>(sacc, xlo_b, kLd128, v0, k_b, kLd128, 0, 0);
     }
-    __syncthreads();  // every warp is done with S's split and K
-    store_split(sacc, Shi, Slo, kLd128, 16 * warp, 0, [](int, int, float x) { return x; });
+    __syncthreads();  // every warp is done with X and this chunk's K
   }
   // ---- the final state ---------------------------------------------------------------------
-  {
-    const int v0 = 16 * warp + gid;
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      const int j = 8 * nt + 2 * q4;
-      *reinterpret_cast<float2*>(Sg + v0 * kPfD + j) = make_float2(sacc[nt][0], sacc[nt][1]);
-      *reinterpret_cast<float2*>(Sg + (v0 + 8) * kPfD + j) = make_float2(sacc[nt][2], sacc[nt][3]);
-    }
+  for (int nt = 0; nt < 16; ++nt) {
+    const int j = 8 * nt + 2 * q4;
+    *reinterpret_cast<float2*>(Sg + (v0 + gid) * kPfD + j) = make_float2(sacc[nt][0], sacc[nt][1]);
+    *reinterpret_cast<float2*>(Sg + (v0 + gid + 8) * kPfD + j) = make_float2(sacc[nt][2], sacc[nt][3]);
   }
 }
 

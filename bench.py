@@ -338,7 +338,8 @@ def main():
     torch.cuda.synchronize()
     if args.pw_only:
         peak, _ = peak_hbm()
-        pw = {f: pw_leg(wl.with_(fmt=f), 8, S0, inp, o, peak) for f in ("int4_g32", "int8")}
+        pw = {f: pw_leg(wl.with_(fmt=f), 8, S0, inp, o, peak, cpu=not args.no_cpu)
+              for f in ("int4_g32", "int8")}
         if rank == 0:
             print(json.dumps({"pure_write_s8": pw, "config": bench_config(wl0, world)}),
                   flush=True)
@@ -415,8 +416,10 @@ def main():
 
     # ---- pure-write sliding window (PW-S8) over int4 and int8 histories, the same inputs ----
     if not args.no_baselines and wl.D == 128:
-        line["pure_write_s8"] = {f: pw_leg(wl.with_(fmt=f), 8, S0, inp, o, peak)
-                                 for f in ("int4_g32", "int8")}
+        line["pure_write_s8"] = {
+            f: pw_leg(wl.with_(fmt=f), 8, S0, inp, o, peak,
+                      cpu=not args.no_cpu and world == 1 and rank == 0)
+            for f in ("int4_g32", "int8")}
 
     # ---- chunkwise prefill of a prompt batch (its own workload) ----------------------------
     if not args.no_baselines and world == 1:
@@ -532,7 +535,6 @@ def prefill_leg(args, dev, reps: int = 5):
     L = wl.T
     inp = decode_inputs(wl, dev)
     hm = {n: t.permute(1, 2, 0, *range(3, t.dim())).contiguous() for n, t in inp.items()}
-    del inp
     cfg = gdn.make_config(wl.B, wl.H, wl.D, gate="scalar", act="bf16")
     o = torch.empty_like(hm["q"])
     S = torch.zeros((wl.B, wl.H, wl.D, wl.D), dtype=torch.float32, device=dev)
@@ -555,7 +557,9 @@ def prefill_leg(args, dev, reps: int = 5):
     flops = chunks * prefill_flops_per_chunk()
     tf = flops / (t / 1e3) / 1e12
     peak, src = peak_bf16()
+    cpu = None if args.no_cpu else prefill_cpu_baseline(wl, inp, dev)
     return {"value": wl.heads * L / (t / 1e3), "unit": "head-tokens/s", "ms_per_launch": t,
+            "cpu_baseline": cpu,
             "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "L": L, "D": wl.D,
                        "gate": "scalar", "act": "bf16", "chunk": 64},
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
@@ -566,7 +570,7 @@ def prefill_leg(args, dev, reps: int = 5):
             "kernel": "prefill_kernel (one CTA per head, 64-token chunks)"}
 
 
-def pw_leg(wl, Wp, S0, inp, o, peak):
+def pw_leg(wl, Wp, S0, inp, o, peak, cpu=False):
     """The pure-write sliding window decode on the same inputs: the history quantized from the
     same initial states, then the T steps, one launch each, timed with CUDA events."""
     import torch
@@ -592,6 +596,7 @@ def pw_leg(wl, Wp, S0, inp, o, peak):
     traffic, src = profiled_traffic(PW_PROFILE, PW_KERNEL_SOURCES,
                                     f"traffic_bytes_per_head_{wl.fmt}")
     return {"value": wl.heads * wl.T / (ms / 1e3), "unit": UNIT, "achieved_gbs": gbs,
+            "cpu_baseline": pw_cpu_baseline(wl, Wp, inp, S0.device) if cpu else None,
             "frac": gbs / peak, "avg_launch_us": ms * 1e3 / wl.T, "ms_per_run": ms,
             "bytes_per_head_step": pw_step_bytes(wl, Wp), "Wp": Wp,
             "traffic": None if traffic is None else traffic * wl.heads, "traffic_source": src,
@@ -637,11 +642,12 @@ def e2e(args, wl, cfg, inp, S0, state, world, dev):
             "api": "gdn_decode_window_steps_host (pinned host buffers, copies pipelined)"}
 
 
-def cpu_baseline(args, wl, inp, dev):
+def oracle_sample(wl, inp, n_seq, dev):
+    """The first n_seq sequences' inputs as float64 numpy ([T][n][...]) and their initial states
+    made by the oracle's own fp32-storage warm-up recurrence (nothing from the GPU)."""
     import numpy as np
     import torch
 
-    n_seq = max(1, min(wl.B, args.cpu_heads // wl.H))
     heads = np.arange(n_seq * wl.H)
     idx = torch.as_tensor(heads, device=dev)
 
@@ -649,7 +655,9 @@ def cpu_baseline(args, wl, inp, dev):
         flat = x.reshape(T, wl.heads, *x.shape[3:])
         return flat.index_select(1, idx).double().cpu().numpy()
 
-    d = {n: pick(x, wl.T) for n, x in inp.items()}
+    d = {n: pick(x, x.shape[0]) for n, x in inp.items()}
+    if wl.warmup == 0:
+        return d, np.zeros((len(heads), wl.D, wl.D))
     scales = outlier_scales(wl, dev)
     warm = {n: [] for n in ("q", "k", "v", "g", "beta")}
     for t in range(wl.warmup):
@@ -659,11 +667,46 @@ def cpu_baseline(args, wl, inp, dev):
             warm[n].append(x.reshape(wl.heads, *x.shape[2:]).index_select(0, idx).double()
                            .cpu().numpy())
     warm = {n: np.stack(v) for n, v in warm.items()}
-    S0 = oracle_warm_state(wl, warm)
+    return d, oracle_warm_state(wl, warm)
+
+
+def cpu_baseline(args, wl, inp, dev):
+    n_seq = max(1, min(wl.B, args.cpu_heads // wl.H))
+    d, S0 = oracle_sample(wl, inp, n_seq, dev)
     hs, dt, cores = time_oracle(wl, d["q"], d["k"], d["v"], d["g"], d["beta"], S0)
     return {"value": hs, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{len(heads)} heads (sequences 0..{n_seq - 1}, all {wl.H} heads) x "
+            "sample": f"{n_seq * wl.H} heads (sequences 0..{n_seq - 1}, all {wl.H} heads) x "
                       f"{wl.T} steps of the same inputs, {dt:.1f} s"}
+
+
+def pw_cpu_baseline(wl, Wp, inp, dev, n_seq: int = 4):
+    """The oracle's pure-write window (GPU storage roundings on) on the first n_seq sequences."""
+    import oracle
+
+    d, S0 = oracle_sample(wl, inp, n_seq, dev)
+    T, n = d["q"].shape[0], d["q"].shape[1]
+    t0 = time.perf_counter()
+    oracle.pw_run(d["q"], d["k"], d["v"], d["g"], d["beta"], Wp=Wp, fmt=wl.fmt, S0=S0,
+                  prec32=True)
+    dt = time.perf_counter() - t0
+    return {"value": n * T / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} heads (sequences 0..{n_seq - 1}) x {T} steps, {dt:.1f} s"}
+
+
+def prefill_cpu_baseline(wl, inp, dev, n_heads: int = 16):
+    """The oracle's plain fp64 recurrence over the first n_heads heads' prompts."""
+    import oracle
+    import torch
+
+    idx = torch.arange(n_heads, device=dev)
+    d = {n: x.reshape(x.shape[0], wl.heads, *x.shape[3:]).index_select(1, idx).double().cpu()
+         .numpy() for n, x in inp.items()}
+    t0 = time.perf_counter()
+    oracle.plain_run(d["q"], d["k"], d["v"], d["g"], d["beta"])
+    dt = time.perf_counter() - t0
+    L = d["q"].shape[0]
+    return {"value": n_heads * L / dt, "unit": "head-tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{n_heads} heads x {L} tokens, {dt:.1f} s"}
 
 
 if __name__ == "__main__":

@@ -255,3 +255,24 @@ def test_pw_empty_batch_and_zero_steps_are_noops(lib):
         _abi.GDN_OK
     assert lib.gdn_pw_decode_steps(ctypes.byref(_pw()), ctypes.byref(st), 0, *([None] * 7)) == \
         _abi.GDN_OK
+
+
+# ---- chunkwise prefill ------------------------------------------------------------------------
+PF_BAD = [
+    ("diag gate", dict(gate="diag"), 8, _abi.GDN_ERR_UNSUPPORTED),
+    ("fp32 activations", dict(act="f32"), 8, _abi.GDN_ERR_UNSUPPORTED),
+    ("D=16", dict(D=16), 8, _abi.GDN_ERR_UNSUPPORTED),
+    ("L<0", dict(), -1, _abi.GDN_ERR_INVALID_ARG),
+    ("null buffers", dict(), 8, _abi.GDN_ERR_INVALID_ARG),
+]
+
+
+@pytest.mark.parametrize("name,kw,L,status", PF_BAD, ids=[b[0] for b in PF_BAD])
+def test_prefill_rejects_bad_arguments(name, kw, L, status, lib):
+    cfg = _cfg(**kw)
+    assert lib.gdn_prefill(ctypes.byref(cfg), L, *([None] * 8)) == status
+    assert lib.gdn_last_error() != b""
+
+
+def test_prefill_empty_batch_is_a_noop(lib):
+    assert lib.gdn_prefill(ctypes.byref(_cfg(B=0)), 100, *([None] * 8)) == _abi.GDN_OK

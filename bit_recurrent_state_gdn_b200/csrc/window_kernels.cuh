@@ -384,7 +384,7 @@ struct DenseTile {
 // Requantisation of the state that `make` produces: compensator columns (top r by max-abs,
 // ties to the lower index) go to comp_u / comp_idx in fp32 and are zeroed; each row (int4: each
 // 32-column group) gets s = absmax / QMAX and codes rint(x / s) clamped to [-QMAX, QMAX], both
-// with IEEE single division. Codes, scales and compensators are written straight to HBM; the
+// quotients correctly rounded as IEEE single division rounds them. Codes, scales and compensators are written straight to HBM; the
 // tile maker may still read the staged old state because rows of later passes are untouched
 // and the old compensators live in shared memory. `colmax` (D floats) and `sel` (r ints) are
 // shared scratch. Called by all threads.
@@ -463,11 +463,17 @@ __device__ void requantize_store(const Maker& make, int r, uint8_t* g_codes, flo
       constexpr int span = C::GS / TC;
 #pragma unroll
       for (int off = span / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      const float s = __fdiv_rn(m, (float)QMAX);
+      // s = fp32(m / QMAX) and the codes' quotients, correctly rounded from a reciprocal with
+      // one fma correction (IEEE division only for tiny or zero scales)
+      const float s = m >= 0x1p-100f ? quot_const(m, (float)QMAX, 1.f / (float)QMAX)
+                                     : __fdiv_rn(m, (float)QMAX);
+      const bool fast = s >= 0x1p-125f;
+      const float inv = fast ? __frcp_rn(s) : 0.f;
       int q[TC];
 #pragma unroll
       for (int b = 0; b < TC; ++b) {
-        float t = s > 0.f ? rintf(__fdiv_rn(acc[a][b], s)) : 0.f;
+        float t = fast ? rintf(quot_const(acc[a][b], s, inv))
+                       : (s > 0.f ? rintf(__fdiv_rn(acc[a][b], s)) : 0.f);
         t = fminf(fmaxf(t, (float)-QMAX), (float)QMAX);
         q[b] = (int)t;
       }

@@ -383,6 +383,10 @@ def main():
     status = int(state.status[0].item())
     if status != 0:
         raise RuntimeError(f"device status word {status:#x} after the timed region")
+    # the quality figure uses this step's outputs, before the legs below reuse the buffer
+    quality = None
+    if not args.no_cpu and world == 1 and rank == 0:
+        quality = quality_figure(wl, inp, o, dev)
 
     value = whole_job_rate(wl.heads * wl.T * args.steps, world, total_ms)
     launches = args.steps * wl.T
@@ -457,6 +461,7 @@ def main():
     # ---- the oracle on the host cores (rank 0, one GPU) ------------------------------------
     if not args.no_cpu and world == 1 and rank == 0:
         line["cpu_baseline"] = cpu_baseline(args, wl, inp, dev)
+        line["quality"] = quality
 
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -677,6 +682,24 @@ def cpu_baseline(args, wl, inp, dev):
     return {"value": hs, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{n_seq * wl.H} heads (sequences 0..{n_seq - 1}, all {wl.H} heads) x "
                       f"{wl.T} steps of the same inputs, {dt:.1f} s"}
+
+
+def quality_figure(wl, inp, o, dev, n_seq: int = 8):
+    """Output error of the windowed int8 decode against the unquantized fp64 recurrence (the
+    oracle's plain run from the oracle's own warm-up states), on the first n_seq sequences: the
+    cost of the low-bit state, not a parity bar."""
+    import numpy as np
+
+    import oracle
+
+    d, S0 = oracle_sample(wl, inp, n_seq, dev)
+    ref, _ = oracle.plain_run(d["q"], d["k"], d["v"], d["g"], d["beta"], S0=S0, want_o=True)
+    n = n_seq * wl.H
+    got = o.reshape(wl.T, wl.heads, wl.D)[:, :n].double().cpu().numpy()
+    err = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+    return {"o_rel_l2_vs_fp64_recurrence": err, "heads": n, "steps": wl.T,
+            "note": "int8 windowed state (W = %d) against the fp64 recurrence with no "
+                    "quantization; GPU outputs in bf16" % wl.W}
 
 
 def pw_cpu_baseline(wl, Wp, inp, dev, n_seq: int = 4):

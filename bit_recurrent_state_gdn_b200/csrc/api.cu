@@ -685,8 +685,6 @@ gdn_status gdn_prefill(const gdn_config* cfg, int32_t L, const void* q, const vo
     return fail(GDN_ERR_INVALID_ARG, "d_k=%d, d_v=%d", cfg->d_k, cfg->d_v);
   if (cfg->d_k != 128 || cfg->d_v != 128)
     return fail(GDN_ERR_UNSUPPORTED, "prefill is built for d_k = d_v = 128");
-  if (cfg->gate != GDN_GATE_SCALAR)
-    return fail(GDN_ERR_UNSUPPORTED, "prefill is built for the scalar (GDN) gate");
   if (cfg->act_dtype != GDN_DTYPE_BF16)
     return fail(GDN_ERR_UNSUPPORTED, "prefill is built for bf16 activations");
   if (L < 0) return fail(GDN_ERR_INVALID_ARG, "L=%d must be >= 0", L);
@@ -699,7 +697,7 @@ gdn_status gdn_prefill(const gdn_config* cfg, int32_t L, const void* q, const vo
     if ((st = need_ptr(q, "q")) != GDN_OK) return st;
     if ((st = need_ptr(k, "k")) != GDN_OK) return st;
     if ((st = need_ptr(v, "v")) != GDN_OK) return st;
-    if ((st = need_ptr(g, "g", 4)) != GDN_OK) return st;
+    if ((st = need_ptr(g, "g", cfg->gate == GDN_GATE_DIAG ? 16 : 4)) != GDN_OK) return st;
     if ((st = need_ptr(beta, "beta", 4)) != GDN_OK) return st;
     if ((st = need_ptr(o, "o", 4)) != GDN_OK) return st;
   }
@@ -712,7 +710,8 @@ gdn_status gdn_prefill(const gdn_config* cfg, int32_t L, const void* q, const vo
   a.o = static_cast<__nv_bfloat16*>(o);
   a.S = S;
   a.L = L;
-  const cudaError_t e = gdnq::launch_prefill(a, (int)heads_of(cfg), (cudaStream_t)stream);
+  const cudaError_t e = gdnq::launch_prefill(a, (int)heads_of(cfg), cfg->gate == GDN_GATE_DIAG,
+                                             (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "gdn_prefill");
   return GDN_OK;
 }

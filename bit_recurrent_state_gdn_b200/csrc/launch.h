@@ -38,9 +38,9 @@ cudaError_t launch_window_mixed(WinOp op, const gdn_config& cfg, const WinArgs& 
 enum class PwOp { Step, Materialize };
 cudaError_t launch_pw(PwOp op, const gdn_pw_config& cfg, const PwArgs& a, int heads,
                       cudaStream_t stream);
-// Chunkwise prefill: one CTA per head.
-cudaError_t launch_prefill(const PfArgs& a, int heads, cudaStream_t stream);
-size_t prefill_smem_bytes();
+// Chunkwise prefill: one CTA per head; diag selects the per-key-channel gate (g [heads][L][128]).
+cudaError_t launch_prefill(const PfArgs& a, int heads, bool diag, cudaStream_t stream);
+size_t prefill_smem_bytes(bool diag);
 cudaError_t launch_baseline(const gdn_config& cfg, const BaseArgs& a, int heads,
                             cudaStream_t stream);
 

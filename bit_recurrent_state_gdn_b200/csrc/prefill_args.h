@@ -9,7 +9,7 @@ struct PfArgs {
   const __nv_bfloat16* q;  // [heads][L][128]
   const __nv_bfloat16* k;
   const __nv_bfloat16* v;
-  const float* g;          // [heads][L]
+  const float* g;          // [heads][L] (scalar gate) or [heads][L][128] (per-channel gate)
   const float* beta;
   __nv_bfloat16* o;        // [heads][L][128]
   float* S;                // [heads][128][128], in place

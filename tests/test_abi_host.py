@@ -259,7 +259,7 @@ def test_pw_empty_batch_and_zero_steps_are_noops(lib):
 
 # ---- chunkwise prefill ------------------------------------------------------------------------
 PF_BAD = [
-    ("diag gate", dict(gate="diag"), 8, _abi.GDN_ERR_UNSUPPORTED),
+    ("diag gate, null buffers", dict(gate="diag"), 8, _abi.GDN_ERR_INVALID_ARG),
     ("fp32 activations", dict(act="f32"), 8, _abi.GDN_ERR_UNSUPPORTED),
     ("D=16", dict(D=16), 8, _abi.GDN_ERR_UNSUPPORTED),
     ("L<0", dict(), -1, _abi.GDN_ERR_INVALID_ARG),
@@ -272,6 +272,16 @@ def test_prefill_rejects_bad_arguments(name, kw, L, status, lib):
     cfg = _cfg(**kw)
     assert lib.gdn_prefill(ctypes.byref(cfg), L, *([None] * 8)) == status
     assert lib.gdn_last_error() != b""
+
+
+def test_prefill_diag_gate_wants_16_byte_aligned_gates(lib):
+    """The per-channel gate rows are copied 16 bytes at a time: an 8-byte aligned g is refused
+    before anything is enqueued (the other pointers are aligned placeholders, never touched)."""
+    p = ctypes.c_void_p(1 << 20)
+    args = [p, p, p, ctypes.c_void_p((1 << 20) + 8), p, p, p]
+    cfg = _cfg(gate="diag")
+    assert lib.gdn_prefill(ctypes.byref(cfg), 8, *args, None) == _abi.GDN_ERR_INVALID_ARG
+    assert b"g is not 16-byte aligned" in lib.gdn_last_error()
 
 
 def test_prefill_empty_batch_is_a_noop(lib):

@@ -1,7 +1,9 @@
 """Chunkwise prefill (include/gdnq_prefill.h) against the oracle's plain fp64 recurrence on the
 same seeded inputs: every output and the final state, for one chunk, several chunks with a
 ragged tail, a single token, an empty prompt, a zero and a warmed-up initial state, prompts
-split over two calls, and a 128-head batch on sampled heads. All calls go through the C ABI."""
+split over calls, and a 128-head batch on sampled heads, with the scalar (GDN) gate and with
+the per-key-channel (KDA) gate (plus strong per-channel decays at the kernel's documented
+bound). All calls go through the C ABI."""
 import numpy as np
 import pytest
 import torch
@@ -16,6 +18,7 @@ from workloads import WORKLOADS, decode_inputs
 pytestmark = pytest.mark.gpu
 
 MID = WORKLOADS["gdn-mid"]
+KDA = WORKLOADS["kda"].with_(r=0)
 S_TOL = 2e-3  # final state, rel-L2 (the outputs' bar)
 
 CASES = {
@@ -24,6 +27,12 @@ CASES = {
     "zero-state": MID.with_(name="pf-zero", B=1, H=2, T=150, warmup=0),
     "single-token": MID.with_(name="pf-1", B=1, H=2, T=1, warmup=32),
     "long": MID.with_(name="pf-1000", B=1, H=2, T=1000, warmup=48),
+    # per-key-channel gate (16-token chunks): one chunk, ragged tail, zero state, one token, long
+    "kda-one-chunk": KDA.with_(name="kpf-16", B=1, H=3, T=16, warmup=32),
+    "kda-ragged": KDA.with_(name="kpf-200", B=2, H=2, T=200, warmup=32),
+    "kda-zero-state": KDA.with_(name="kpf-zero", B=1, H=2, T=37, warmup=0),
+    "kda-single-token": KDA.with_(name="kpf-1", B=1, H=2, T=1, warmup=32),
+    "kda-long": KDA.with_(name="kpf-1000", B=1, H=2, T=1000, warmup=48),
 }
 
 
@@ -33,7 +42,7 @@ def head_major(x):
 
 
 def pf_run(wl, inp, S0, cuts=None):
-    cfg = gdn.make_config(wl.B, wl.H, wl.D, gate="scalar", act="bf16")
+    cfg = gdn.make_config(wl.B, wl.H, wl.D, gate=wl.gate, act="bf16")
     S = S0.clone()
     L = inp["q"].shape[0]
     o = torch.empty((wl.B, wl.H, L, wl.D), dtype=torch.bfloat16, device="cuda")
@@ -69,17 +78,33 @@ def test_prefill_parity(name):
     assert o_rel <= O_TOL and s_rel <= S_TOL, (o_rel, s_rel)
 
 
-def test_prefill_split_over_calls_carries_the_state():
-    wl = CASES["ragged"]
+@pytest.mark.parametrize("name", ["ragged", "kda-ragged"])
+def test_prefill_split_over_calls_carries_the_state(name):
+    wl = CASES[name]
     inp = decode_inputs(wl, "cuda")
     S0 = gpu_warmup(wl)
-    o, S = pf_run(wl, inp, S0, cuts=[0, 70, 131, 200])  # chunk boundaries inside the calls
+    o, S = pf_run(wl, inp, S0, cuts=[0, 5, 70, 131, 200])  # chunk boundaries inside the calls
     o_rel, s_rel = compare(wl, inp, o, S, np.arange(wl.heads))
     assert o_rel <= O_TOL and s_rel <= S_TOL, (o_rel, s_rel)
 
 
-def test_prefill_batch_sampled_heads():
-    wl = MID.with_(name="pf-batch", B=4, H=32, T=512, warmup=32)
+def test_kda_prefill_strong_decays():
+    """Per-channel log-gates three times the recipe's, floored at -10 per token: 8-token sums
+    reach -80, the bound up to which the chunk's decay factors e^{+-(G_t - G_r)} stay finite."""
+    wl = KDA.with_(name="kpf-strong", B=1, H=4, T=160, warmup=32)
+    inp = decode_inputs(wl, "cuda")
+    inp["g"] = (3.0 * inp["g"]).clamp_min(-10.0)
+    inp["g"][5:13, :, :, :7] = -10.0  # a run of 8 tokens at the floor on a few channels
+    o, S = pf_run(wl, inp, gpu_warmup(wl))
+    o_rel, s_rel = compare(wl, inp, o, S, np.arange(wl.heads))
+    print("strong", o_rel, s_rel)
+    assert np.isfinite(o_rel) and np.isfinite(s_rel)
+    assert o_rel <= O_TOL and s_rel <= S_TOL, (o_rel, s_rel)
+
+
+@pytest.mark.parametrize("base", ["gdn", "kda"])
+def test_prefill_batch_sampled_heads(base):
+    wl = (MID if base == "gdn" else KDA).with_(name="pf-batch", B=4, H=32, T=512, warmup=32)
     inp = decode_inputs(wl, "cuda")
     o, S = pf_run(wl, inp, gpu_warmup(wl))
     heads = sample_heads(wl, 24, seed=3)
@@ -88,27 +113,32 @@ def test_prefill_batch_sampled_heads():
     assert o_rel <= O_TOL and s_rel <= S_TOL, (o_rel, s_rel)
 
 
-def test_empty_prompt_leaves_the_state():
-    wl = CASES["one-chunk"]
-    cfg = gdn.make_config(wl.B, wl.H, wl.D)
+@pytest.mark.parametrize("name", ["one-chunk", "kda-one-chunk"])
+def test_empty_prompt_leaves_the_state(name):
+    wl = CASES[name]
+    cfg = gdn.make_config(wl.B, wl.H, wl.D, gate=wl.gate)
     S0 = gpu_warmup(wl)
     S = S0.clone()
     z = torch.empty((wl.B, wl.H, 0, wl.D), dtype=torch.bfloat16, device="cuda")
     zf = torch.empty((wl.B, wl.H, 0), dtype=torch.float32, device="cuda")
-    gdn.gdn_prefill(cfg, z, z, z, zf, zf, z, S)
+    zg = torch.empty((wl.B, wl.H, 0, wl.D) if wl.gate == "diag" else (wl.B, wl.H, 0),
+                     dtype=torch.float32, device="cuda")
+    gdn.gdn_prefill(cfg, z, z, z, zg, zf, z, S)
     torch.cuda.synchronize()
     assert torch.equal(S, S0)
 
 
-def test_prefill_then_window_decode():
+@pytest.mark.parametrize("base", ["gdn", "kda"])
+def test_prefill_then_window_decode(base):
     """The state a prefill leaves, quantized, starts the windowed decode: the decode's outputs
     match the oracle running the same prompt and decode tokens through the plain recurrence
     then the windowed form."""
-    wl = MID.with_(name="pf-decode", B=1, H=4, T=64, W=64, warmup=0)
-    prompt = MID.with_(name="pf-prompt", B=1, H=4, T=300, warmup=0, seed=4242)
+    wb = MID if base == "gdn" else KDA
+    wl = wb.with_(name="pf-decode", B=1, H=4, T=64, W=64, warmup=0)
+    prompt = wb.with_(name="pf-prompt", B=1, H=4, T=300, warmup=0, seed=4242)
     pin = decode_inputs(prompt, "cuda")
     _, S = pf_run(prompt, pin, torch.zeros((1, 4, 128, 128), device="cuda"))
-    cfg = gdn.make_config(wl.B, wl.H, wl.D, wl.W, 0, "scalar", "int8", "bf16", "bf16")
+    cfg = gdn.make_config(wl.B, wl.H, wl.D, wl.W, 0, wl.gate, "int8", "bf16", "bf16")
     st = gdn.GdnState.allocate(cfg)
     gdn.gdn_state_quantize(cfg, S, st)
     inp = decode_inputs(wl, "cuda")

@@ -78,9 +78,13 @@ def load(path: Optional[str] = None):
     lib.orc_plain_run.restype = None
     lib.orc_plain_run.argtypes = [_int] * 5 + [_vp] * 8
     lib.orc_o1_run.restype = _int
-    lib.orc_o1_run.argtypes = [_int] * 7 + [_vp] * 8
+    lib.orc_o1_run.argtypes = [_int] * 8 + [_vp] * 8
     lib.orc_o2_run.restype = _int
-    lib.orc_o2_run.argtypes = [_int] * 9 + [_vp] * 18
+    lib.orc_o2_run.argtypes = [_int] * 10 + [_vp] * 19
+    lib.orc_smooth_exponent.restype = _int
+    lib.orc_smooth_exponent.argtypes = [ctypes.c_double]
+    lib.orc_window_end.restype = _int
+    lib.orc_window_end.argtypes = [_int] * 5 + [_vp] * 6
     lib.orc_round_e4m3.restype = ctypes.c_double
     lib.orc_round_e4m3.argtypes = [ctypes.c_double]
     lib.orc_fp8_vector.restype = ctypes.c_double
@@ -167,6 +171,40 @@ def select_columns(S: np.ndarray, r: int, lib=None):
 # ---------------------------------------------------------------------------------------------
 # The three formulations
 # ---------------------------------------------------------------------------------------------
+def smooth_exponent(colmax: float, lib=None) -> int:
+    """e = floor(floor(log2 colmax) / 2) clamped to [-63, 63]; 0 for a zero column."""
+    return (lib or load()).orc_smooth_exponent(float(colmax))
+
+
+@dataclass
+class WindowEnd:
+    residual: np.ndarray   # [D][D] the rescaled residual that was quantized
+    codes: np.ndarray      # [D][D] int8
+    scales: np.ndarray     # [D][groups]
+    cidx: np.ndarray       # [r]
+    cu: np.ndarray         # [r][D] compensator columns (value side)
+    sexp: np.ndarray       # [D] int8 smoothing exponents
+    near_tie: int
+
+
+def window_end(S: np.ndarray, fmt: str = "int8", r: int = 0, smooth: bool = False,
+               prec32: bool = False, lib=None) -> WindowEnd:
+    """The window-end operation on one [D][D] state: compensators out, residual smoothing,
+    quantization. The state it leaves is dequant(codes, scales) Diag(2^sexp) plus the
+    compensator columns."""
+    lib = lib or load()
+    R = _f64(S).copy()
+    D = R.shape[0]
+    f = _FMT[fmt]
+    ng = lib.orc_num_groups(FMT_INT8 if f == FMT_NONE else f, D)
+    out = WindowEnd(R, np.zeros((D, D), np.int8), np.zeros((D, ng)), np.zeros(max(r, 1), np.int32),
+                    np.zeros((max(r, 1), D)), np.zeros(D, np.int8), 0)
+    out.near_tie = lib.orc_window_end(D, f, r, int(prec32), int(smooth), _p(R), _p(out.codes),
+                                      _p(out.scales), _p(out.cidx), _p(out.cu), _p(out.sexp))
+    out.cidx, out.cu = out.cidx[:r], out.cu[:r]
+    return out
+
+
 def _gate(g, T, nh, D):
     g = _f64(g)
     if g.ndim == 2:
@@ -188,9 +226,10 @@ def plain_run(q, k, v, g, beta, S0=None, state_round: str = "none", want_o: bool
     return o, S
 
 
-def o1_run(q, k, v, g, beta, W: int, r: int = 0, fmt: str = "int8", S0=None, lib=None):
-    """Literal matrix-form recurrence with window-end requantisation (fp64 decisions).
-    Returns (o, S_T, near_ties)."""
+def o1_run(q, k, v, g, beta, W: int, r: int = 0, fmt: str = "int8", S0=None,
+           smooth: bool = False, lib=None):
+    """Literal matrix-form recurrence with window-end requantisation (fp64 decisions; ``smooth``
+    adds the residual smoothing). Returns (o, S_T, near_ties)."""
     lib = lib or load()
     q, k, v, beta = _f64(q), _f64(k), _f64(v), _f64(beta)
     T, nh, D = k.shape
@@ -198,8 +237,8 @@ def o1_run(q, k, v, g, beta, W: int, r: int = 0, fmt: str = "int8", S0=None, lib
     S0 = _f64(S0)
     o = np.zeros((T, nh, D))
     S = np.zeros((nh, D, D))
-    ties = lib.orc_o1_run(D, T, W, r, _FMT[fmt], nh, Dg, _p(S0), _p(q), _p(k), _p(v), _p(g),
-                          _p(beta), _p(o), _p(S))
+    ties = lib.orc_o1_run(D, T, W, r, _FMT[fmt], nh, Dg, int(smooth), _p(S0), _p(q), _p(k),
+                          _p(v), _p(g), _p(beta), _p(o), _p(S))
     return o, S, ties
 
 
@@ -217,13 +256,15 @@ class O2Result:
     S: np.ndarray          # [nh][D][D] logical state at the end
     near_ties: int
     ties: np.ndarray       # [nh] near ties per head
+    sexp: np.ndarray       # [nh][D] int8 smoothing exponents (zeros without smoothing)
 
 
 def o2_run(q, k, v, g, beta, W: int, r: int = 0, fmt: str = "int8", S0=None,
            round_storage: bool = False, buf_round: str = "bf16", flush_mask=None,
-           lib=None) -> O2Result:
+           smooth: bool = False, lib=None) -> O2Result:
     """Buffered-window form. ``round_storage`` mirrors GPU storage (fp32 state / L / scales,
-    ``buf_round`` write vectors, fp32 quantizer decisions)."""
+    ``buf_round`` write vectors, fp32 quantizer decisions); ``smooth`` adds the residual
+    smoothing at every quantization."""
     lib = lib or load()
     q, k, v, beta = _f64(q), _f64(k), _f64(v), _f64(beta)
     T, nh, D = k.shape
@@ -236,13 +277,14 @@ def o2_run(q, k, v, g, beta, W: int, r: int = 0, fmt: str = "int8", S0=None,
         scales=np.zeros((nh, D, ng)), cidx=np.zeros((nh, max(r, 0)), np.int32),
         cu=np.zeros((nh, max(r, 0), D)), pos=np.zeros(nh, np.int32),
         bk=np.zeros((nh, W, D)), bu=np.zeros((nh, W, D)), bL=np.zeros((nh, W, D)),
-        S=np.zeros((nh, D, D)), near_ties=0, ties=np.zeros(nh, np.int32))
+        S=np.zeros((nh, D, D)), near_ties=0, ties=np.zeros(nh, np.int32),
+        sexp=np.zeros((nh, D), np.int8))
     fm = None if flush_mask is None else np.ascontiguousarray(flush_mask, np.uint8).reshape(T, nh)
     res.near_ties = lib.orc_o2_run(
-        D, T, W, r, f, nh, Dg, int(round_storage), _ROUND[buf_round], _p(S0), _p(q), _p(k),
-        _p(v), _p(g), _p(beta), _p(fm), _p(res.o), _p(res.codes), _p(res.scales),
+        D, T, W, r, f, nh, Dg, int(round_storage), _ROUND[buf_round], int(smooth), _p(S0),
+        _p(q), _p(k), _p(v), _p(g), _p(beta), _p(fm), _p(res.o), _p(res.codes), _p(res.scales),
         _p(res.cidx) if r > 0 else None, _p(res.cu) if r > 0 else None, _p(res.pos),
-        _p(res.bk), _p(res.bu), _p(res.bL), _p(res.S), _p(res.ties))
+        _p(res.bk), _p(res.bu), _p(res.bL), _p(res.S), _p(res.ties), _p(res.sexp))
     return res
 
 

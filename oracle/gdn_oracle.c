@@ -17,8 +17,12 @@
  *            high-precision updates;
  *          - a few high-precision "compensator tokens" keep the state's largest outliers and
  *            take the same update path as real tokens;
- *          - the residual is smoothed before quantization (NOT restated here: the page gives
- *            no mechanism).
+ *          - the residual is smoothed before quantization. The page gives no mechanism; the
+ *            reading restated here (window_end's smooth option) is a per-key-column power-of-
+ *            two rescaling before the per-row quantizer, the factor about the square root of
+ *            the column's max-abs. Parity unpinned against the pages (they give no rule and no
+ *            numbers for it); its arithmetic is pinned by a hand-worked fixture, the exponent's
+ *            closed form, exactness without quantization and O1 = O2.
  *   [PW] "Low-Bit GDN Recurrent-State Quantization: Global Gradient-aware Allocation and
  *        Pure-Write Sliding Windows", Abstract: quantized write-back errors feed into later
  *        steps (why quantize-every-step, the window length 1 case, degrades); recent pure
@@ -200,19 +204,62 @@ int orc_select_columns(int D, int r, const double* S, int* idx) {
     return near;
 }
 
+/* ------------------------------------------------------------------------------------------
+ * Residual smoothing ("LeapQuant: Efficient Linear Attention with Accurate Recurrent State
+ * Quantization", Abstract: the residual left after the compensators is smoothed before it is
+ * quantized). The page names the step and no mechanism; the reading taken here is a per-key-
+ * column rescaling of the residual R before the per-row quantizer, R = R' Diag(m), with
+ * m_j = 2^{e_j} and e_j = floor(E_j / 2), E_j the binary exponent of column j's max-abs
+ * (m_j ~ sqrt(colmax_j): the usual half-way migration of a column's range), e_j = 0 for a zero
+ * column, e_j clamped to [-63, 63]. Powers of two make the rescaling exact, so the only rounding
+ * left is the quantizer's; the frozen state is dequant(codes, scales) Diag(m), and a step's
+ * products with it take m .* x.
+ * ---------------------------------------------------------------------------------------- */
+int orc_smooth_exponent(double colmax) {
+    if (!(colmax > 0.0)) return 0;
+    int x;
+    frexp(colmax, &x);           /* colmax = f 2^x, f in [1/2, 1) */
+    int E = x - 1;               /* floor(log2 colmax) */
+    int e = E >= 0 ? E / 2 : -((1 - E) / 2);  /* floor(E / 2) */
+    if (e < -63) e = -63;
+    if (e > 63) e = 63;
+    return e;
+}
+
 /* Window-end operation on a full state S (overwritten by the residual): take out r compensator
- * columns exactly, then quantize the residual. fmt == NONE keeps the residual unquantized in S.
- * Returns the near-tie flag of the column choice. */
-static int window_end(int D, int fmt, int r, int prec32, double* S, int8_t* codes, double* scales,
-                      int* cidx, double* cu) {
+ * columns exactly, then (smooth) rescale the residual's columns by 2^{-e_j} into sexp, then
+ * quantize the residual. fmt == NONE keeps the (rescaled) residual unquantized in S. Returns the
+ * near-tie flag of the column choice. sexp may be NULL when smooth is 0. */
+static int window_end(int D, int fmt, int r, int prec32, int smooth, double* S, int8_t* codes,
+                      double* scales, int* cidx, double* cu, int8_t* sexp) {
     int near = orc_select_columns(D, r, S, cidx);
     for (int c = 0; c < r; ++c)
         for (int i = 0; i < D; ++i) {
             cu[(size_t)c * D + i] = S[(size_t)i * D + cidx[c]];
             S[(size_t)i * D + cidx[c]] = 0.0;
         }
+    if (smooth) {
+        for (int j = 0; j < D; ++j) {
+            double m = 0.0;
+            for (int i = 0; i < D; ++i) m = fmax(m, fabs(S[(size_t)i * D + j]));
+            sexp[j] = (int8_t)orc_smooth_exponent(m);
+            for (int i = 0; i < D; ++i) S[(size_t)i * D + j] = ldexp(S[(size_t)i * D + j], -sexp[j]);
+        }
+    }
     if (fmt != ORC_FMT_NONE) orc_quantize(D, fmt, prec32, S, codes, scales);
     return near;
+}
+
+/* Columns j of S [D][D] times 2^{sexp[j]} (undoes the smoothing; exact). */
+static void unsmooth(int D, const int8_t* sexp, double* S) {
+    for (int i = 0; i < D; ++i)
+        for (int j = 0; j < D; ++j) S[(size_t)i * D + j] = ldexp(S[(size_t)i * D + j], sexp[j]);
+}
+
+/* The window-end operation on its own (pins): S is overwritten by the (rescaled) residual. */
+int orc_window_end(int D, int fmt, int r, int prec32, int smooth, double* S, int8_t* codes,
+                   double* scales, int* cidx, double* cu, int8_t* sexp) {
+    return window_end(D, fmt, r, prec32, smooth, S, codes, scales, cidx, cu, sexp);
 }
 
 static double gate_log(const double* g, int Dg, int j) { return Dg == 1 ? g[0] : g[j]; }
@@ -276,15 +323,18 @@ void orc_plain_run(int D, int T, int nh, int Dg, int state_round, const double* 
  * W-th step, S <- dequant(quant(S - C)) + C, where C holds the r compensator columns of S
  * (fmt NONE: S is left as it is). All decisions in fp64. Returns the number of near ties.
  * ---------------------------------------------------------------------------------------- */
-static int dense_window_end(int D, int fmt, int r, double* S) {
-    if (fmt == ORC_FMT_NONE && r == 0) return 0;
+static int dense_window_end(int D, int fmt, int r, int smooth, double* S) {
+    if (fmt == ORC_FMT_NONE && r == 0 && !smooth) return 0;
     int ng = orc_num_groups(fmt == ORC_FMT_NONE ? ORC_FMT_INT8 : fmt, D);
     int8_t* codes = (int8_t*)malloc((size_t)D * D);
     double* scales = (double*)malloc(sizeof(double) * (size_t)D * ng);
     int* cidx = (int*)malloc(sizeof(int) * (size_t)(r > 0 ? r : 1));
     double* cu = (double*)malloc(sizeof(double) * (size_t)(r > 0 ? r : 1) * D);
-    int near = window_end(D, fmt, r, 0, S, codes, scales, cidx, cu);
+    int8_t* sexp = (int8_t*)calloc((size_t)D, 1);
+    int near = window_end(D, fmt, r, 0, smooth, S, codes, scales, cidx, cu, sexp);
     if (fmt != ORC_FMT_NONE) orc_dequantize(D, fmt, codes, scales, S);
+    if (smooth) unsmooth(D, sexp, S);
+    free(sexp);
     for (int c = 0; c < r; ++c)
         for (int i = 0; i < D; ++i) S[(size_t)i * D + cidx[c]] += cu[(size_t)c * D + i];
     free(codes);
@@ -294,7 +344,7 @@ static int dense_window_end(int D, int fmt, int r, double* S) {
     return near;
 }
 
-int orc_o1_run(int D, int T, int W, int r, int fmt, int nh, int Dg, const double* S0,
+int orc_o1_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int smooth, const double* S0,
                const double* q, const double* k, const double* v, const double* g,
                const double* beta, double* o, double* S_out) {
     int ties = 0;
@@ -306,7 +356,7 @@ int orc_o1_run(int D, int T, int W, int r, int fmt, int nh, int Dg, const double
         double* N = (double*)malloc(sizeof(double) * DD);
         if (S0) memcpy(S, S0 + (size_t)h * DD, sizeof(double) * DD);
         else memset(S, 0, sizeof(double) * DD);
-        ties += dense_window_end(D, fmt, r, S);
+        ties += dense_window_end(D, fmt, r, smooth, S);
         for (int t = 0; t < T; ++t) {
             const double* kt = k + ((size_t)t * nh + h) * D;
             const double* qt = q + ((size_t)t * nh + h) * D;
@@ -332,7 +382,7 @@ int orc_o1_run(int D, int T, int W, int r, int fmt, int nh, int Dg, const double
                     ot[i] = acc;
                 }
             }
-            if ((t + 1) % W == 0) ties += dense_window_end(D, fmt, r, S);
+            if ((t + 1) % W == 0) ties += dense_window_end(D, fmt, r, smooth, S);
         }
         if (S_out) memcpy(S_out + (size_t)h * DD, S, sizeof(double) * DD);
         free(S);
@@ -359,6 +409,8 @@ int orc_o1_run(int D, int T, int W, int r, int fmt, int nh, int Dg, const double
  *   = S Diag(a) + beta (v - S Diag(a) k) k^T.
  * When P reaches W (or a flush is forced after the step) the logical state is materialised and
  * the window-end operation (compensators out, residual quantized) makes the next F.
+ * smooth = 1 adds the residual smoothing of window_end: F = dequant(codes, scales) Diag(2^e),
+ * so every product with F (steps, materialisation) sees the smoothing undone exactly.
  *
  * round_storage = 1 mirrors what a GPU keeps between steps: the initial state and the
  * materialised state are fp32, L is fp32, u_t is rounded to buf_round (bf16 / fp32), and the
@@ -366,17 +418,18 @@ int orc_o1_run(int D, int T, int W, int r, int fmt, int nh, int Dg, const double
  *
  * Outputs (any may be NULL): o [T][nh][D]; codes [nh][D][D]; scales [nh][D][groups];
  * cidx [nh][r]; cu [nh][r][D]; pos [nh]; bk, bu, bL [nh][W][D]; S_out [nh][D][D] (the logical
- * state at the end); ties_out [nh] (near ties met per head); flush_mask [T][nh] forces a flush
+ * state at the end); ties_out [nh] (near ties met per head); sexp_out [nh][D] (the smoothing
+ * exponents of the last quantization); flush_mask [T][nh] forces a flush
  * after step t of head h when nonzero. Returns the number of near ties met in compensator
  * choices.
  * ---------------------------------------------------------------------------------------- */
 typedef struct {
-    int D, W, r, fmt, Dg, round_storage, buf_round;
+    int D, W, r, fmt, Dg, round_storage, buf_round, smooth;
 } o2_cfg;
 
 typedef struct {
     double *F, *scales, *cu, *bk, *bu, *bL;
-    int8_t* codes;
+    int8_t *codes, *sexp;
     int* cidx;
     int P;
 } o2_head;
@@ -406,9 +459,11 @@ static int o2_set_frozen(const o2_cfg* c, o2_head* s, double* S) {
     int D = c->D;
     if (c->round_storage)
         for (size_t e = 0; e < (size_t)D * D; ++e) S[e] = orc_round_f32(S[e]);
-    int near = window_end(D, c->fmt, c->r, c->round_storage, S, s->codes, s->scales, s->cidx, s->cu);
+    int near = window_end(D, c->fmt, c->r, c->round_storage, c->smooth, S, s->codes, s->scales,
+                          s->cidx, s->cu, s->sexp);
     if (c->fmt != ORC_FMT_NONE) orc_dequantize(D, c->fmt, s->codes, s->scales, s->F);
     else memcpy(s->F, S, sizeof(double) * (size_t)D * D);
+    if (c->smooth) unsmooth(D, s->sexp, s->F);
     s->P = 0;
     return near;
 }
@@ -473,11 +528,12 @@ static void o2_step(const o2_cfg* c, o2_head* s, const double* qt, const double*
 }
 
 int orc_o2_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int round_storage,
-               int buf_round, const double* S0, const double* q, const double* k, const double* v,
+               int buf_round, int smooth, const double* S0, const double* q, const double* k, const double* v,
                const double* g, const double* beta, const uint8_t* flush_mask, double* o,
                int8_t* codes_out, double* scales_out, int* cidx_out, double* cu_out, int* pos_out,
-               double* bk_out, double* bu_out, double* bL_out, double* S_out, int* ties_out) {
-    o2_cfg c = {D, W, r, fmt, Dg, round_storage, buf_round};
+               double* bk_out, double* bu_out, double* bL_out, double* S_out, int* ties_out,
+               int8_t* sexp_out) {
+    o2_cfg c = {D, W, r, fmt, Dg, round_storage, buf_round, smooth};
     int ng = orc_num_groups(fmt == ORC_FMT_NONE ? ORC_FMT_INT8 : fmt, D);
     int ties = 0;
 #pragma omp parallel for schedule(dynamic) reduction(+ : ties)
@@ -487,6 +543,7 @@ int orc_o2_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int round_st
         s.F = (double*)calloc(DD, sizeof(double));
         s.scales = (double*)calloc((size_t)D * ng, sizeof(double));
         s.codes = (int8_t*)calloc(DD, 1);
+        s.sexp = (int8_t*)calloc((size_t)D, 1);
         s.cidx = (int*)calloc((size_t)(r > 0 ? r : 1), sizeof(int));
         s.cu = (double*)calloc((size_t)(r > 0 ? r : 1) * D, sizeof(double));
         s.bk = (double*)calloc((size_t)W * D, sizeof(double));
@@ -513,6 +570,7 @@ int orc_o2_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int round_st
         if (cidx_out && r > 0) memcpy(cidx_out + (size_t)h * r, s.cidx, sizeof(int) * (size_t)r);
         if (cu_out && r > 0) memcpy(cu_out + (size_t)h * r * D, s.cu, sizeof(double) * (size_t)r * D);
         if (pos_out) pos_out[h] = s.P;
+        if (sexp_out) memcpy(sexp_out + (size_t)h * D, s.sexp, (size_t)D);
         if (bk_out) memcpy(bk_out + (size_t)h * W * D, s.bk, sizeof(double) * (size_t)W * D);
         if (bu_out) memcpy(bu_out + (size_t)h * W * D, s.bu, sizeof(double) * (size_t)W * D);
         if (bL_out) memcpy(bL_out + (size_t)h * W * D, s.bL, sizeof(double) * (size_t)W * D);
@@ -520,7 +578,7 @@ int orc_o2_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int round_st
             o2_current_L(&c, &s, Lt);
             o2_materialize(&c, &s, Lt, S_out + h * DD);
         }
-        free(s.F); free(s.scales); free(s.codes); free(s.cidx); free(s.cu);
+        free(s.F); free(s.scales); free(s.codes); free(s.sexp); free(s.cidx); free(s.cu);
         free(s.bk); free(s.bu); free(s.bL); free(Sx); free(vec);
     }
     return ties;

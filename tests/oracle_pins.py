@@ -400,6 +400,122 @@ def pin_storage_roundings(lib):
 
 
 # ---------------------------------------------------------------------------------------------
+# Residual smoothing (reading: per-column power-of-two factors m_j = 2^floor(E_j / 2))
+# ---------------------------------------------------------------------------------------------
+def pin_golden_smoothing(lib):
+    gd = read("smoothing_4x4.txt")
+    S = gd["S"].reshape(4, 4)
+    we = oracle.window_end(S, "int8", r=0, smooth=True, lib=lib)
+    assert list(we.sexp) == [int(x) for x in gd["sexp"]], we.sexp
+    assert np.array_equal(we.codes.ravel(), gd["codes"].astype(np.int8)), we.codes
+    assert np.allclose(we.scales.ravel() * 127, gd["absmax"], rtol=1e-15, atol=0), we.scales
+    we1 = oracle.window_end(S, "int8", r=1, smooth=True, lib=lib)
+    assert list(we1.cidx) == [0] and np.array_equal(we1.cu[0], gd["comp_u_r1"])
+    assert list(we1.sexp) == [int(x) for x in gd["sexp_r1"]], we1.sexp
+    assert np.array_equal(we1.codes.ravel(), gd["codes_r1"].astype(np.int8)), we1.codes
+    assert np.allclose(we1.scales.ravel() * 127, gd["absmax_r1"], rtol=1e-15, atol=0)
+    # the same as the initial quantization of the buffered form: the state it keeps is
+    # dequant(codes, scales) Diag(2^e) plus the compensator column
+    e0 = np.zeros((0, 1, 4))
+    res = oracle.o2_run(e0, e0, e0, np.zeros((0, 1)), np.zeros((0, 1)), W=4, r=1, fmt="int8",
+                        S0=S.reshape(1, 4, 4), smooth=True, lib=lib)
+    assert np.array_equal(res.codes[0], we1.codes) and list(res.sexp[0]) == list(we1.sexp)
+    kept = gd["codes_r1"].reshape(4, 4) * (gd["absmax_r1"].reshape(4, 1) / 127.0)
+    kept = kept * 2.0 ** gd["sexp_r1"].reshape(1, 4)
+    kept[:, 0] += gd["comp_u_r1"]
+    assert np.allclose(res.S[0], kept, rtol=1e-15, atol=1e-300), res.S[0]
+
+
+def pin_smooth_exponent(lib):
+    """Hand values of e = floor(floor(log2 m) / 2) clamped to [-63, 63], and m_j = 2^e against
+    the square root it stands for: 2^e <= sqrt(colmax) < 2^(e+1)."""
+    cases = [(0.0, 0), (1.0, 0), (2.0, 0), (3.99, 0), (4.0, 1), (15.9, 1), (16.0, 2),
+             (0.5, -1), (0.3, -1), (0.25, -1), (0.2, -2), (2.0 ** 200, 63), (2.0 ** -200, -63),
+             (2.0 ** -127, -63), (2.0 ** -126, -63), (2.0 ** -125, -63), (2.0 ** -124, -62)]
+    for m, e in cases:
+        got = oracle.smooth_exponent(m, lib=lib)
+        assert got == e, (m, got, e)
+    rng = np.random.default_rng(3)
+    for m in 10.0 ** rng.uniform(-30, 30, size=400):
+        e = oracle.smooth_exponent(m, lib=lib)
+        assert 2.0 ** e <= np.sqrt(m) < 2.0 ** (e + 1), (m, e)
+
+
+def pin_smoothing_properties(lib):
+    """On states with outlier key columns: the exponents follow the residual's column max-abs
+    (compensator columns excluded), the kept state is within half a quantization step (times
+    the column's factor) of the input, a uniform band of column maxima gives the unsmoothed
+    codes, and smoothing lowers the reconstruction error (what the page claims for it)."""
+    rng = np.random.default_rng(17)
+    D = 64
+    for fmt in ("int8", "int4_g32"):
+        for r in (0, 3):
+            S = rng.standard_normal((D, D)) * rng.uniform(0.05, 3.0, size=(D, 1))
+            S[:, [3, 20, 41]] *= 20.0
+            S[:, 50:] *= 0.05
+            S = S.astype(np.float32).astype(np.float64)
+            plain = oracle.window_end(S, fmt, r=r, smooth=False, lib=lib)
+            sm = oracle.window_end(S, fmt, r=r, smooth=True, lib=lib)
+            assert list(plain.cidx) == list(sm.cidx)
+            R = S.copy()
+            R[:, sm.cidx] = 0.0
+            cm = np.abs(R).max(axis=0)
+            m = 2.0 ** sm.sexp.astype(np.float64)
+            nz = cm > 0
+            assert np.all((m[nz] <= np.sqrt(cm[nz])) & (np.sqrt(cm[nz]) < 2 * m[nz]))
+            assert np.all(sm.sexp[~nz] == 0)
+            deq = oracle.dequantize(sm.codes, sm.scales, fmt, lib=lib) * m
+            step = np.repeat(sm.scales, D // sm.scales.shape[1], axis=1) * m
+            assert np.all(np.abs(R - deq) <= step / 2 * (1 + 1e-12))
+            kept = deq.copy()
+            kept[:, sm.cidx] += sm.cu.T
+            kept_p = oracle.dequantize(plain.codes, plain.scales, fmt, lib=lib)
+            kept_p[:, plain.cidx] += plain.cu.T
+            assert rel(kept, S) < rel(kept_p, S), (fmt, r, rel(kept, S), rel(kept_p, S))
+    # column maxima all in [4, 16): every e is 1, codes as without smoothing, scales halved
+    S = rng.uniform(-1, 1, size=(D, D))
+    S *= (4.0 + 11.9 * rng.uniform(size=D))[None, :] / np.abs(S).max(axis=0)
+    for fmt in ("int8", "int4_g32"):
+        plain = oracle.window_end(S, fmt, smooth=False, lib=lib)
+        sm = oracle.window_end(S, fmt, smooth=True, lib=lib)
+        assert np.all(sm.sexp == 1)
+        assert np.array_equal(sm.codes, plain.codes)
+        assert np.array_equal(sm.scales * 2.0, plain.scales)
+
+
+def pin_smoothing_unquantized_is_exact(lib):
+    """Without quantization the smoothing is undone exactly: the buffered form with and without
+    it gives bit-identical outputs and states."""
+    T, nh, D = 9, 2, 16
+    for gate in ("scalar", "diag"):
+        q, k, v, g, beta = rand_inputs(61, T, nh, D, gate, outlier=True)
+        S0 = np.random.default_rng(5).standard_normal((nh, D, D)) * 3.0
+        a = oracle.o2_run(q, k, v, g, beta, W=4, r=2, fmt="none", S0=S0, smooth=True, lib=lib)
+        b = oracle.o2_run(q, k, v, g, beta, W=4, r=2, fmt="none", S0=S0, smooth=False, lib=lib)
+        assert np.array_equal(a.o, b.o) and np.array_equal(a.S, b.S), gate
+        assert np.any(a.sexp != 0)
+
+
+def pin_smoothed_literal_equals_buffered(lib):
+    """O1 (dense, requantised every W steps) equals O2 (frozen low-bit state + buffer) with
+    residual smoothing too, for int8 and int4, with and without compensators."""
+    for fmt, D in (("int8", 8), ("int4_g32", 32)):
+        T, nh = 11, 2
+        for gate in ("scalar", "diag"):
+            q, k, v, g, beta = rand_inputs(71 + D, T, nh, D, gate, outlier=True)
+            S0 = np.random.default_rng(D + 1).standard_normal((nh, D, D))
+            S0[:, :, 1] *= 25.0
+            for W in (1, 3, 8):
+                for r in (0, 2):
+                    o1, S1, _ = oracle.o1_run(q, k, v, g, beta, W=W, r=r, fmt=fmt, S0=S0,
+                                              smooth=True, lib=lib)
+                    res = oracle.o2_run(q, k, v, g, beta, W=W, r=r, fmt=fmt, S0=S0, smooth=True,
+                                        lib=lib)
+                    close(res.o, o1, 1e-10, f"smoothed O1 vs O2 {fmt} {gate} W={W} r={r}")
+                    close(res.S, S1, 1e-10, f"smoothed O1 vs O2 state {fmt} {gate} W={W} r={r}")
+
+
+# ---------------------------------------------------------------------------------------------
 # PW: the pure-write sliding window
 # ---------------------------------------------------------------------------------------------
 def pin_golden_pure_write_window(lib):
@@ -527,6 +643,11 @@ PINS = [
     pin_literal_equals_buffered_quantized,
     pin_compensator_decomposition,
     pin_storage_roundings,
+    pin_golden_smoothing,
+    pin_smooth_exponent,
+    pin_smoothing_properties,
+    pin_smoothing_unquantized_is_exact,
+    pin_smoothed_literal_equals_buffered,
     pin_golden_pure_write_window,
     pin_e4m3_rounding,
     pin_pw_exact_is_plain,

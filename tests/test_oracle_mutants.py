@@ -29,8 +29,8 @@ MUTANTS = [
      "exp(gate_log(gt, Dg, j)) * ((j == l",
      "exp(gate_log(gt, Dg, l)) * ((j == l"),
     ("O1: window end one step early",
-     "if ((t + 1) % W == 0) ties += dense_window_end(D, fmt, r, S);",
-     "if (t % W == 0) ties += dense_window_end(D, fmt, r, S);"),
+     "if ((t + 1) % W == 0) ties += dense_window_end(D, fmt, r, smooth, S);",
+     "if (t % W == 0) ties += dense_window_end(D, fmt, r, smooth, S);"),
     ("O2: beta dropped from the write vector",
      "double u = bt * (vt[i] - w[i]);",
      "double u = (vt[i] - w[i]);"),
@@ -58,6 +58,21 @@ MUTANTS = [
     ("O2: frozen state not decayed at materialisation",
      "S[(size_t)i * D + j] = s->F[(size_t)i * D + j] * exp(L[j]);",
      "S[(size_t)i * D + j] = s->F[(size_t)i * D + j];"),
+    ("smoothing: factor not undone on the frozen state",
+     "    if (c->smooth) unsmooth(D, s->sexp, s->F);",
+     "    if (0) unsmooth(D, s->sexp, s->F);"),
+    ("smoothing: exponent not halved",
+     "int e = E >= 0 ? E / 2 : -((1 - E) / 2);  /* floor(E / 2) */",
+     "int e = E;"),
+    ("smoothing: exponent rounded toward zero",
+     "int e = E >= 0 ? E / 2 : -((1 - E) / 2);  /* floor(E / 2) */",
+     "int e = E / 2;"),
+    ("smoothing: factors from row maxima",
+     "for (int i = 0; i < D; ++i) m = fmax(m, fabs(S[(size_t)i * D + j]));\n            sexp[j]",
+     "for (int i = 0; i < D; ++i) m = fmax(m, fabs(S[(size_t)j * D + i]));\n            sexp[j]"),
+    ("smoothing: residual scaled up instead of down",
+     "S[(size_t)i * D + j] = ldexp(S[(size_t)i * D + j], -sexp[j]);",
+     "S[(size_t)i * D + j] = ldexp(S[(size_t)i * D + j], sexp[j]);"),
     ("quantizer: int8 range 128",
      "return fmt == ORC_FMT_INT4 ? 7 : 127;",
      "return fmt == ORC_FMT_INT4 ? 7 : 128;"),

@@ -76,6 +76,7 @@ def step_bytes(wl, P: int) -> int:
     lbytes = 4 * D if wl.gate == "diag" else 4
     codes = D * D // 2 if wl.fmt == "int4_g32" else D * D
     scales = 4 * D * (D // 32 if wl.fmt == "int4_g32" else 1)
+    scales += D if wl.smooth else 0  # residual smoothing: one exponent byte per key column
     comps = r * (4 + 4 * D)
     pair = D * act + D * buf + lbytes
     io_ = 4 * D * act + (4 * D if wl.gate == "diag" else 4) + 4 + 8  # q k v o, g, beta, pos r/w
@@ -300,7 +301,8 @@ def main():
         import torch
 
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-        line = {"prefill": prefill_leg(args, torch.device("cuda"))}
+        dev = torch.device("cuda")
+        line = {"prefill": prefill_leg(args, dev), "prefill_kda": prefill_leg(args, dev, "kda-prefill")}
         if rank == 0:
             print(json.dumps(line), flush=True)
         return
@@ -418,6 +420,11 @@ def main():
     if not args.no_baselines and wl.fmt == "int8" and wl.D == 128:
         line["mixed_half_int4"] = mixed_leg(wl, S0, inp, o, peak)
 
+    # ---- residual smoothing at every quantization, the same inputs ---------------------------
+    if not args.no_baselines and wl.fmt in ("int8", "int4_g32"):
+        line["smoothing"] = smoothing_leg(wl, S0, inp, o, peak, dev,
+                                          cpu=not args.no_cpu and world == 1 and rank == 0)
+
     # ---- pure-write sliding window (PW-S8) over int4 and int8 histories, the same inputs ----
     if not args.no_baselines and wl.D == 128:
         line["pure_write_s8"] = {
@@ -428,6 +435,7 @@ def main():
     # ---- chunkwise prefill of a prompt batch (its own workload) ----------------------------
     if not args.no_baselines and world == 1:
         line["prefill"] = prefill_leg(args, dev)
+        line["prefill_kda"] = prefill_leg(args, dev, "kda-prefill")
 
     # ---- high-precision-state baselines on the same inputs ---------------------------------
     if not args.no_baselines:
@@ -498,6 +506,42 @@ def mixed_leg(wl, S0, inp, o, peak):
             "note": "GDN_FMT_MIXED, heads alternately int8 / int4-g32, one launch per step"}
 
 
+def smoothing_leg(wl, S0, inp, o, peak, dev, cpu: bool):
+    """The same decode with residual smoothing at every quantization (per-key-column power-of-
+    two factors), timed like the mixed leg; with cpu, its output error against the unquantized
+    fp64 recurrence on the quality figure's sample."""
+    import torch
+
+    import bit_recurrent_state_gdn_b200 as gdn
+
+    ws = wl.with_(smooth=True)
+    cfg = gdn.make_config(ws.B, ws.H, ws.D, ws.W, ws.r, ws.gate, ws.fmt, ws.act, ws.buf,
+                          smooth=True)
+    st = gdn.GdnState.allocate(cfg)
+    gdn.gdn_state_quantize(cfg, S0, st)
+    for t in range(4):
+        gdn.gdn_decode_window_step(cfg, st, inp["q"][t], inp["k"][t], inp["v"][t], inp["g"][t],
+                                   inp["beta"][t], o[t])
+    gdn.gdn_state_quantize(cfg, S0, st)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    gdn.gdn_decode_window_steps(cfg, st, inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], o)
+    e1.record()
+    torch.cuda.synchronize()
+    if int(st.status[0].item()) != 0:
+        raise RuntimeError("smoothing leg: device status word set")
+    ms = e0.elapsed_time(e1)
+    gbs = avg_step_bytes(ws) * ws.heads * ws.T / (ms / 1e3) / 1e9
+    out = {"value": ws.heads * ws.T / (ms / 1e3), "unit": UNIT, "achieved_gbs": gbs,
+           "frac": gbs / peak, "ms_per_run": ms,
+           "note": "GDN_SMOOTH_POW2_COLUMNS: residual columns scaled by 2^-floor(E/2) before "
+                   "the row quantizer, E the exponent of the column's max-abs"}
+    if cpu:
+        out["quality"] = quality_figure(ws, inp, o, dev)
+    return out
+
+
 def pw_step_bytes(wl, Wp: int) -> int:
     """Algorithmic bytes of one pure-write window step per head with a full window: the history
     (codes + scales) read and written, the Wp pairs (e4m3 x and y, fp32 scales) read, the Wp - 1
@@ -527,20 +571,20 @@ def peak_bf16():
         return 1590.0, "fallback"
 
 
-def prefill_leg(args, dev, reps: int = 5):
-    """gdn_prefill over the gdn-prefill workload (B x H heads, L-token prompts, zero initial
-    state): the median of `reps` launches after two untimed ones, CUDA events."""
+def prefill_leg(args, dev, name: str = "gdn-prefill", reps: int = 5):
+    """gdn_prefill over a prompt workload (B x H heads, L-token prompts, zero initial state):
+    the median of `reps` launches after two untimed ones, CUDA events."""
     import torch
 
     import bit_recurrent_state_gdn_b200 as gdn
 
-    wl = WORKLOADS["gdn-prefill"]
+    wl = WORKLOADS[name]
     if args.prefill_batch:
         wl = wl.with_(B=args.prefill_batch)
     L = wl.T
     inp = decode_inputs(wl, dev)
     hm = {n: t.permute(1, 2, 0, *range(3, t.dim())).contiguous() for n, t in inp.items()}
-    cfg = gdn.make_config(wl.B, wl.H, wl.D, gate="scalar", act="bf16")
+    cfg = gdn.make_config(wl.B, wl.H, wl.D, gate=wl.gate, act="bf16")
     o = torch.empty_like(hm["q"])
     S = torch.zeros((wl.B, wl.H, wl.D, wl.D), dtype=torch.float32, device=dev)
     for _ in range(2):
@@ -557,22 +601,25 @@ def prefill_leg(args, dev, reps: int = 5):
         ms.append(e0.elapsed_time(e1))
     t = sorted(ms)[len(ms) // 2]
     if not bool(torch.isfinite(S).all()):
-        raise RuntimeError("prefill: non-finite state")
-    chunks = wl.heads * ((L + 63) // 64)
-    flops = chunks * prefill_flops_per_chunk()
+        raise RuntimeError(f"prefill {wl.name}: non-finite state")
+    C = 16 if wl.gate == "diag" else 64
+    chunks = wl.heads * ((L + C - 1) // C)
+    flops = chunks * prefill_flops_per_chunk(C)
     tf = flops / (t / 1e3) / 1e12
     peak, src = peak_bf16()
     cpu = None if args.no_cpu else prefill_cpu_baseline(wl, inp, dev)
+    kernel = ("prefill_kda_kernel (one CTA per head, two per SM, 16-token chunks)"
+              if wl.gate == "diag" else "prefill_kernel (one CTA per head, 64-token chunks)")
     return {"value": wl.heads * L / (t / 1e3), "unit": "head-tokens/s", "ms_per_launch": t,
             "cpu_baseline": cpu,
             "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "L": L, "D": wl.D,
-                       "gate": "scalar", "act": "bf16", "chunk": 64},
+                       "gate": wl.gate, "act": "bf16", "chunk": C},
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
                          "frac": tf / peak, "peak_source": src,
                          "flops_per_launch": flops,
                          "note": "UT-form products at single precision; the kernel issues "
-                                 "twice that on mma.sync (hi/lo bf16 splits)"},
-            "kernel": "prefill_kernel (one CTA per head, 64-token chunks)"}
+                                 "up to three times that on mma.sync (hi/lo bf16 splits)"},
+            "kernel": kernel}
 
 
 def pw_leg(wl, Wp, S0, inp, o, peak, cpu=False):
@@ -698,8 +745,9 @@ def quality_figure(wl, inp, o, dev, n_seq: int = 8):
     got = o.reshape(wl.T, wl.heads, wl.D)[:, :n].double().cpu().numpy()
     err = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
     return {"o_rel_l2_vs_fp64_recurrence": err, "heads": n, "steps": wl.T,
-            "note": "int8 windowed state (W = %d) against the fp64 recurrence with no "
-                    "quantization; GPU outputs in bf16" % wl.W}
+            "note": "%s windowed state (W = %d%s) against the fp64 recurrence with no "
+                    "quantization; GPU outputs in bf16"
+                    % (wl.fmt, wl.W, ", residual smoothing" if wl.smooth else "")}
 
 
 def pw_cpu_baseline(wl, Wp, inp, dev, n_seq: int = 4):

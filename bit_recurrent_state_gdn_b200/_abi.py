@@ -10,6 +10,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgdnq.so"
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(5)
 GDN_DEVICE_WAIT_TIMEOUT, GDN_DEVICE_BAD_POS = 0x1, 0x2
 GDN_GATE_SCALAR, GDN_GATE_DIAG = 0, 1
+GDN_SMOOTH_NONE, GDN_SMOOTH_POW2_COLUMNS = 0, 1
 GDN_FMT_INT8, GDN_FMT_INT4_G32, GDN_FMT_BF16, GDN_FMT_FP32, GDN_FMT_MIXED = 0, 1, 2, 3, 4
 GDN_DTYPE_F32, GDN_DTYPE_BF16 = 0, 1
 GDN_MAX_COMPENSATORS = 16
@@ -22,11 +23,12 @@ _sz = ctypes.c_size_t
 
 class gdn_config(ctypes.Structure):
     _fields_ = [(n, _i32) for n in
-                ("B", "H", "d_k", "d_v", "W", "r", "gate", "fmt", "act_dtype", "buf_dtype")]
+                ("B", "H", "d_k", "d_v", "W", "r", "gate", "fmt", "act_dtype", "buf_dtype",
+                 "smooth")]
 
 
 STATE_FIELDS = ("codes", "scales", "buf_k", "buf_u", "buf_L", "comp_idx", "comp_u", "pos",
-                "status", "head_fmt")
+                "status", "head_fmt", "smooth_exp")
 
 
 class gdn_state(ctypes.Structure):
@@ -34,7 +36,7 @@ class gdn_state(ctypes.Structure):
 
 
 SIZE_FIELDS = ("codes", "scales", "buf_k", "buf_u", "buf_L", "comp_idx", "comp_u", "pos",
-               "smem_step", "head_fmt")
+               "smem_step", "head_fmt", "smooth_exp")
 
 
 class gdn_sizes(ctypes.Structure):

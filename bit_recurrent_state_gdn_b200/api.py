@@ -31,8 +31,11 @@ class GdnError(RuntimeError):
 
 
 def make_config(B: int, H: int, D: int, W: int = 1, r: int = 0, gate: str = "scalar",
-                fmt: str = "int8", act: str = "bf16", buf: str = "bf16") -> _abi.gdn_config:
-    return _abi.gdn_config(B, H, D, D, W, r, _GATE[gate], _FMT[fmt], _DT[act], _DT[buf])
+                fmt: str = "int8", act: str = "bf16", buf: str = "bf16",
+                smooth: bool = False) -> _abi.gdn_config:
+    """smooth: residual smoothing (per-key-column power-of-two factors) at every quantization."""
+    return _abi.gdn_config(B, H, D, D, W, r, _GATE[gate], _FMT[fmt], _DT[act], _DT[buf],
+                           _abi.GDN_SMOOTH_POW2_COLUMNS if smooth else _abi.GDN_SMOOTH_NONE)
 
 
 def _check(status: int, where: str):
@@ -83,6 +86,7 @@ class GdnState:
     pos: torch.Tensor
     status: torch.Tensor
     head_fmt: torch.Tensor  # int8 [B*H]: each head's format (mixed-format states only)
+    smooth_exp: torch.Tensor  # int8 [B*H*D]: smoothing exponents (smoothed states only)
 
     @staticmethod
     def allocate(cfg: _abi.gdn_config, device="cuda", head_fmt=None) -> "GdnState":
@@ -101,7 +105,8 @@ class GdnState:
             buf_L=buf(sz.buf_L, torch.float32), comp_idx=buf(sz.comp_idx, torch.int32),
             comp_u=buf(sz.comp_u, torch.float32), pos=buf(sz.pos, torch.int32),
             status=torch.zeros(4, dtype=torch.int32, device=dev),
-            head_fmt=_head_fmt(cfg, head_fmt, sz.head_fmt, dev))
+            head_fmt=_head_fmt(cfg, head_fmt, sz.head_fmt, dev),
+            smooth_exp=torch.zeros(max(sz.smooth_exp, 16), dtype=torch.int8, device=dev))
 
     def c_struct(self) -> _abi.gdn_state:
         return _abi.gdn_state(*[getattr(self, n).data_ptr() for n in _abi.STATE_FIELDS])

@@ -19,7 +19,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OBJ_DIR = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libgdnq.so")
-SOURCES = ["api.cu", "window_int8.cu", "window_int4.cu", "window_mixed.cu", "baseline.cu",
+SOURCES = ["api.cu", "window_int8.cu", "window_int4.cu", "window_mixed.cu", "window_int8_smooth.cu",
+           "window_int4_smooth.cu", "baseline.cu",
            "pw.cu", "prefill.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

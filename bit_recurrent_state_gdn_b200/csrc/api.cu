@@ -78,6 +78,10 @@ gdn_status check_config(const gdn_config* c, Use use) {
     return fail(GDN_ERR_INVALID_ARG, "r=%d must lie in [0, d_k]", c->r);
   if (c->r > GDN_MAX_COMPENSATORS)
     return fail(GDN_ERR_UNSUPPORTED, "r=%d exceeds %d", c->r, GDN_MAX_COMPENSATORS);
+  if (c->smooth != GDN_SMOOTH_NONE && c->smooth != GDN_SMOOTH_POW2_COLUMNS)
+    return fail(GDN_ERR_INVALID_ARG, "smooth=%d is not a gdn_smoothing", c->smooth);
+  if (c->smooth != GDN_SMOOTH_NONE && c->fmt == GDN_FMT_MIXED)
+    return fail(GDN_ERR_UNSUPPORTED, "residual smoothing is built for INT8 and INT4_G32 states");
   if (c->fmt == GDN_FMT_INT4_G32 && c->d_k % 32 != 0)
     return fail(GDN_ERR_UNSUPPORTED, "int4 with group 32 needs d_k %% 32 == 0");
   if ((c->fmt == GDN_FMT_INT4_G32 || c->fmt == GDN_FMT_MIXED) && c->d_k != 128)
@@ -125,6 +129,8 @@ gdn_status check_state(const gdn_config* c, const gdn_state* s) {
     return fail(GDN_ERR_INVALID_ARG, "state.status is not 4-byte aligned");
   if (c->fmt == GDN_FMT_MIXED && !s->head_fmt)
     return fail(GDN_ERR_INVALID_ARG, "state.head_fmt is null for a mixed-format state");
+  if (c->smooth != GDN_SMOOTH_NONE && (st = need_ptr(s->smooth_exp, "state.smooth_exp")) != GDN_OK)
+    return st;
   return GDN_OK;
 }
 
@@ -162,6 +168,7 @@ gdnq::WinArgs make_args(const gdn_config* c, const gdn_state* s) {
   a.code_stride = (uint32_t)ph.codes;
   a.scale_stride = (uint32_t)(ph.scales / 4);
   a.head_fmt = c->fmt == GDN_FMT_MIXED ? s->head_fmt : nullptr;
+  a.smooth_exp = c->smooth != GDN_SMOOTH_NONE ? s->smooth_exp : nullptr;
   a.H = c->H;
   a.W = c->W;
   a.r = c->r;
@@ -171,11 +178,15 @@ gdnq::WinArgs make_args(const gdn_config* c, const gdn_state* s) {
 gdn_status launch(gdnq::WinOp op, const gdn_config* c, const gdnq::WinArgs& a,
                   gdn_stream_t stream, const char* where) {
   const int heads = (int)heads_of(c);
+  const bool sm = c->smooth != GDN_SMOOTH_NONE;
+  const cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = c->fmt == GDN_FMT_INT4_G32
-                      ? gdnq::launch_window_int4(op, *c, a, heads, (cudaStream_t)stream)
+                      ? (sm ? gdnq::launch_window_int4_smooth(op, *c, a, heads, st)
+                            : gdnq::launch_window_int4(op, *c, a, heads, st))
                   : c->fmt == GDN_FMT_MIXED
-                      ? gdnq::launch_window_mixed(op, *c, a, heads, (cudaStream_t)stream)
-                      : gdnq::launch_window_int8(op, *c, a, heads, (cudaStream_t)stream);
+                      ? gdnq::launch_window_mixed(op, *c, a, heads, st)
+                      : (sm ? gdnq::launch_window_int8_smooth(op, *c, a, heads, st)
+                            : gdnq::launch_window_int8(op, *c, a, heads, st));
   if (e != cudaSuccess) return cuda_fail(e, where);
   return GDN_OK;
 }
@@ -212,7 +223,8 @@ size_t window_smem_bytes(const gdn_config& c) {
   const int code_bytes = int4 ? D * D / 2 : D * D;
   const int nscales = int4 || mixed ? D * (D / 32) : D;
   return win_layout(D, code_bytes, nscales, (int)act_size(&c), (int)buf_size(&c),
-                    c.gate == GDN_GATE_DIAG, c.W, c.r, 1, kMaxHeadsPerCta)
+                    c.gate == GDN_GATE_DIAG, c.W, c.r, 1, kMaxHeadsPerCta, -1, true,
+                    c.smooth != GDN_SMOOTH_NONE)
       .total;
 }
 
@@ -335,6 +347,7 @@ gdn_status gdn_state_sizes(const gdn_config* cfg, gdn_sizes* out) {
   out->pos = n * 4;
   out->smem_step = gdnq::window_smem_bytes(*cfg);
   out->head_fmt = cfg->fmt == GDN_FMT_MIXED ? n : 0;
+  out->smooth_exp = cfg->smooth != GDN_SMOOTH_NONE ? n * (size_t)cfg->d_k : 0;
   return GDN_OK;
 }
 

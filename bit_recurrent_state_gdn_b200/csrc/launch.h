@@ -33,6 +33,11 @@ cudaError_t launch_window_int4(WinOp op, const gdn_config& cfg, const WinArgs& a
                                cudaStream_t stream);
 cudaError_t launch_window_mixed(WinOp op, const gdn_config& cfg, const WinArgs& a, int heads,
                                 cudaStream_t stream);
+// The same with residual smoothing (cfg.smooth != GDN_SMOOTH_NONE).
+cudaError_t launch_window_int8_smooth(WinOp op, const gdn_config& cfg, const WinArgs& a,
+                                      int heads, cudaStream_t stream);
+cudaError_t launch_window_int4_smooth(WinOp op, const gdn_config& cfg, const WinArgs& a,
+                                      int heads, cudaStream_t stream);
 // Pure-write sliding window: the persistent decode step, or the materialisation (one CTA per
 // head), over `heads` heads.
 enum class PwOp { Step, Materialize };

@@ -98,24 +98,26 @@ cudaError_t launch_window_cfg(WinOp op, const WinArgs& a, int heads, cudaStream_
 
 // MIX: int8 and int4 heads in one launch (INT4 is then false: the int8 configuration, whose
 // int4 companion Int4Of<> takes the int4 heads).
-template <int D, bool DIAG, bool INT4, bool MIX = false>
+template <int D, bool DIAG, bool INT4, bool MIX = false, bool SMOOTH = false>
 cudaError_t launch_window_types(WinOp op, const gdn_config& cfg, const WinArgs& a, int heads,
                                 cudaStream_t st) {
   using bf = __nv_bfloat16;
   const bool af = cfg.act_dtype == GDN_DTYPE_F32, bfp = cfg.buf_dtype == GDN_DTYPE_F32;
   if (af && bfp)
-    return launch_window_cfg<WinCfg<D, DIAG, INT4, float, float>, MIX>(op, a, heads, st);
-  if (af) return launch_window_cfg<WinCfg<D, DIAG, INT4, float, bf>, MIX>(op, a, heads, st);
-  if (bfp) return launch_window_cfg<WinCfg<D, DIAG, INT4, bf, float>, MIX>(op, a, heads, st);
-  return launch_window_cfg<WinCfg<D, DIAG, INT4, bf, bf>, MIX>(op, a, heads, st);
+    return launch_window_cfg<WinCfg<D, DIAG, INT4, float, float, SMOOTH>, MIX>(op, a, heads, st);
+  if (af)
+    return launch_window_cfg<WinCfg<D, DIAG, INT4, float, bf, SMOOTH>, MIX>(op, a, heads, st);
+  if (bfp)
+    return launch_window_cfg<WinCfg<D, DIAG, INT4, bf, float, SMOOTH>, MIX>(op, a, heads, st);
+  return launch_window_cfg<WinCfg<D, DIAG, INT4, bf, bf, SMOOTH>, MIX>(op, a, heads, st);
 }
 
-template <int D, bool INT4, bool MIX = false>
+template <int D, bool INT4, bool MIX = false, bool SMOOTH = false>
 cudaError_t launch_window_gate(WinOp op, const gdn_config& cfg, const WinArgs& a, int heads,
                                cudaStream_t st) {
   if (cfg.gate == GDN_GATE_DIAG)
-    return launch_window_types<D, true, INT4, MIX>(op, cfg, a, heads, st);
-  return launch_window_types<D, false, INT4, MIX>(op, cfg, a, heads, st);
+    return launch_window_types<D, true, INT4, MIX, SMOOTH>(op, cfg, a, heads, st);
+  return launch_window_types<D, false, INT4, MIX, SMOOTH>(op, cfg, a, heads, st);
 }
 
 }  // namespace gdnq

@@ -34,11 +34,13 @@ namespace gdnq {
 
 constexpr int kThreads = 256;
 
-template <int D_, bool DIAG_, bool INT4_, typename Act_, typename Buf_>
+template <int D_, bool DIAG_, bool INT4_, typename Act_, typename Buf_, bool SMOOTH_ = false>
 struct WinCfg {
   static constexpr int D = D_;
   static constexpr bool DIAG = DIAG_;
   static constexpr bool INT4 = INT4_;
+  // residual smoothing: frozen state dequant(codes, scales) Diag(2^e), e per key column
+  static constexpr bool SMOOTH = SMOOTH_;
   using Act = Act_;
   using Buf = Buf_;
   static constexpr int NT = kThreads;
@@ -77,7 +79,7 @@ __host__ __device__ constexpr uint32_t align128(uint32_t x) { return (x + 127u) 
 // coefficients, reduction space) and, for the persistent step kernel, the pos / gate / beta of
 // its whole head range.
 struct WinLayout {
-  uint32_t codes, scales, bk, bu, bL, cidx, cu, q, k, v, g, stage_bytes;  // within a stage
+  uint32_t codes, scales, bk, bu, bL, cidx, cu, q, k, v, g, sexp, stage_bytes;  // within a stage
   uint32_t bars, stage0, vec, coef, red, tc, harr, total;                 // within the CTA
 };
 
@@ -91,11 +93,12 @@ __host__ __device__ constexpr uint32_t tc_scratch_bytes(int Wr) {
 // Per-CTA scratch first (barriers, vectors, coefficients, reduction space unless `red` is false,
 // tensor-core scratch, the pos / gate / beta of the CTA's heads), then `nstages` stages whose
 // buffered-pair regions hold `cap` rows (a multiple of 16, at most W rounded up to 16; -1 means
-// that maximum). The kernels only ever read or write pair rows below the stage's cap.
+// that maximum). The kernels only ever read or write pair rows below the stage's cap. With
+// `smooth` a stage also holds the head's D smoothing exponents.
 __host__ __device__ inline WinLayout win_layout(int D, int code_bytes, int nscales, int act_size,
                                                 int buf_size, bool diag, int W, int r,
                                                 int nstages, int per_cta, int cap = -1,
-                                                bool red = true) {
+                                                bool red = true, bool smooth = false) {
   // buffer rows rounded up to 16: the mma k-steps read (zero-filled) rows past the window
   const int Wp = (W + 3) & ~3, rp = (r + 3) & ~3, Wr = (W + 15) & ~15;
   if (cap < 0) cap = Wr;
@@ -118,7 +121,8 @@ __host__ __device__ inline WinLayout win_layout(int D, int code_bytes, int nscal
   L.k = align128(L.q + (uint32_t)D * act_size);
   L.v = align128(L.k + (uint32_t)D * act_size);
   L.g = align128(L.v + (uint32_t)D * act_size);
-  L.stage_bytes = align128(L.g + (diag ? 4u * D : 0u));
+  L.sexp = align128(L.g + (diag ? 4u * D : 0u));
+  L.stage_bytes = align128(L.sexp + (smooth ? (uint32_t)D : 0u));
   L.total = L.stage0 + (uint32_t)nstages * L.stage_bytes;
   return L;
 }
@@ -127,7 +131,8 @@ template <class C>
 __host__ __device__ inline WinLayout win_layout(int W, int r, int nstages, int per_cta,
                                                 int cap = -1, bool red = true) {
   return win_layout(C::D, C::CODE_BYTES, C::NSCALES, (int)sizeof(typename C::Act),
-                    (int)sizeof(typename C::Buf), C::DIAG, W, r, nstages, per_cta, cap, red);
+                    (int)sizeof(typename C::Buf), C::DIAG, W, r, nstages, per_cta, cap, red,
+                    C::SMOOTH);
 }
 
 // The int4 (group 32) configuration that shares C's head size, gate and dtypes, and the shared-
@@ -181,7 +186,19 @@ struct WinArgs {
   uint32_t code_stride;    // bytes of codes per head
   uint32_t scale_stride;   // scales (floats) per head
   int H, W, r;
+  int8_t* smooth_exp;      // residual smoothing: [heads][D] column exponents, else null
 };
+
+// 2^e for an integer e in [-126, 127], from the exponent bits (exact).
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
+
+// Residual smoothing exponent of a column whose max-abs is m: floor(floor(log2 m) / 2) clamped
+// to [-63, 63] (a subnormal m counts as 2^-127); 0 for m <= 0 (a zero or a taken column).
+__device__ __forceinline__ int smooth_exponent(float m) {
+  if (!(m > 0.f)) return 0;
+  const int E = (int)(__float_as_uint(m) >> 23) - 127;
+  return max(-63, min(63, E >> 1));  // arithmetic shift: floor(E / 2)
+}
 
 // Whether a head of a mixed-format state is held as int4 (group 32).
 __device__ __forceinline__ bool head_is_int4(const WinArgs& a, int head) {
@@ -230,6 +247,9 @@ __device__ __forceinline__ void stage_issue(const WinArgs& a, const WinLayout& L
   const uint32_t lbytes = C::DIAG ? 4u * P * D : 4u * ((P + 3) & ~3);
   uint32_t bytes = 0;
   if (p0) bytes += C::CODE_BYTES + 4u * C::NSCALES + (with_io ? 2u * D * sizeof(Act) : 0u);
+  if constexpr (C::SMOOTH) {
+    if (p0) bytes += (uint32_t)D;
+  }
   if (p1) {
     if (P > 0) bytes += (uint32_t)P * D * (sizeof(Act) + sizeof(Buf)) + lbytes;
     if (r > 0) bytes += 4u * rp + 4u * r * D;
@@ -239,6 +259,7 @@ __device__ __forceinline__ void stage_issue(const WinArgs& a, const WinLayout& L
   if (p0) {
     bulk_g2s(st + L.codes, a.codes + (size_t)head * a.code_stride, C::CODE_BYTES, bar);
     bulk_g2s(st + L.scales, a.scales + (size_t)head * a.scale_stride, 4u * C::NSCALES, bar);
+    if constexpr (C::SMOOTH) bulk_g2s(st + L.sexp, a.smooth_exp + (size_t)head * D, (uint32_t)D, bar);
     if (with_io) {
       bulk_g2s(st + L.q, static_cast<const Act*>(a.q) + (size_t)head * D, D * sizeof(Act), bar);
       bulk_g2s(st + L.k, static_cast<const Act*>(a.k) + (size_t)head * D, D * sizeof(Act), bar);
@@ -296,15 +317,20 @@ struct WindowTile {
   const int32_t* cidx;
   const float* cu;
   const float* colexp;
+  const int8_t* sexp;  // smoothing exponents of the frozen codes (SMOOTH only)
   int npairs, r;
 
   __device__ __forceinline__ void operator()(int ps, float (&acc)[C::TR][C::TC]) const {
     constexpr int D = C::D, TC = C::TC, TR = C::TR;
     const int tid = threadIdx.x, cg = tid % C::CG, rg = tid / C::CG;
     const int c0 = cg * TC;
-    float ce[TC];
+    float ce[TC], cf[TC];  // column decay; the frozen codes' factor (decay times 2^e)
 #pragma unroll
-    for (int b = 0; b < TC; ++b) ce[b] = colexp[c0 + b];
+    for (int b = 0; b < TC; ++b) {
+      ce[b] = colexp[c0 + b];
+      cf[b] = ce[b];
+      if constexpr (C::SMOOTH) cf[b] *= pow2i(sexp[c0 + b]);
+    }
 #pragma unroll
     for (int a = 0; a < TR; ++a) {
       const int row = ps * C::RPASS + rg * TR + a;
@@ -324,7 +350,7 @@ struct WindowTile {
       }
       const float s = scales[row * C::NG + c0 / C::GS];
 #pragma unroll
-      for (int b = 0; b < TC; ++b) acc[a][b] = s * cv[b] * ce[b];
+      for (int b = 0; b < TC; ++b) acc[a][b] = s * cv[b] * cf[b];
     }
     for (int c = 0; c < r; ++c) {
       const int j = cidx[c];
@@ -387,17 +413,21 @@ struct DenseTile {
 // quotients correctly rounded as IEEE single division rounds them. Codes, scales and compensators are written straight to HBM; the
 // tile maker may still read the staged old state because rows of later passes are untouched
 // and the old compensators live in shared memory. `colmax` (D floats) and `sel` (r ints) are
-// shared scratch. Called by all threads.
+// shared scratch. Called by all threads. With residual smoothing (C::SMOOTH) the columns' max-abs
+// are always taken; after the compensator choice column j gets e_j = smooth_exponent(max-abs of
+// the residual column) (0 for a taken column), written to g_sexp, and the residual is quantized
+// times 2^-e_j.
 // ------------------------------------------------------------------------------------------
 template <class C, class Maker>
 __device__ void requantize_store(const Maker& make, int r, uint8_t* g_codes, float* g_scales,
-                                 int32_t* g_cidx, float* g_cu, float* colmax, int32_t* sel) {
+                                 int32_t* g_cidx, float* g_cu, float* colmax, int32_t* sel,
+                                 int8_t* g_sexp = nullptr) {
   constexpr int D = C::D, TR = C::TR, TC = C::TC, QMAX = C::QMAX;
   const int tid = threadIdx.x, cg = tid % C::CG, rg = tid / C::CG;
   const int lane = tid & 31, warp = tid >> 5;
   float acc[TR][TC];
 
-  if (r > 0) {
+  if (r > 0 || C::SMOOTH) {
     for (int j = tid; j < D; j += C::NT) colmax[j] = 0.f;
     csync();
     for (int ps = 0; ps < C::NPASS; ++ps) {
@@ -435,6 +465,14 @@ __device__ void requantize_store(const Maker& make, int r, uint8_t* g_codes, flo
       }
     }
     csync();
+    if constexpr (C::SMOOTH) {  // colmax[j] becomes the column's factor 2^-e_j
+      for (int j = tid; j < D; j += C::NT) {
+        const int e = smooth_exponent(colmax[j]);
+        g_sexp[j] = (int8_t)e;
+        colmax[j] = pow2i(-e);
+      }
+      csync();
+    }
   }
 
   for (int ps = 0; ps < C::NPASS; ++ps) {
@@ -451,6 +489,14 @@ __device__ void requantize_store(const Maker& make, int r, uint8_t* g_codes, flo
               acc[a][b] = 0.f;
             }
           }
+      }
+    }
+    if constexpr (C::SMOOTH) {
+#pragma unroll
+      for (int b = 0; b < TC; ++b) {
+        const float f = colmax[cg * TC + b];
+#pragma unroll
+        for (int a = 0; a < TR; ++a) acc[a][b] *= f;
       }
     }
 #pragma unroll
@@ -541,6 +587,7 @@ __device__ __forceinline__ WindowTile<C> window_tile(const uint8_t* st, const Wi
   t.cidx = reinterpret_cast<const int32_t*>(st + L.cidx);
   t.cu = reinterpret_cast<const float*>(st + L.cu);
   t.colexp = colexp;
+  t.sexp = reinterpret_cast<const int8_t*>(st + L.sexp);
   t.npairs = npairs;
   t.r = r;
   return t;
@@ -615,6 +662,11 @@ __device__ __forceinline__ void step_head(const WinArgs& a, const WinLayout& L, 
     for (int e = 0; e < 16; ++e) {
       xr[e] = xs[c * 16 + e];
       yr[e] = ys[c * 16 + e];
+      if constexpr (C::SMOOTH) {  // F = dequant Diag(2^e): the codes meet 2^e .* x
+        const float f = pow2i(reinterpret_cast<const int8_t*>(st + L.sexp)[c * 16 + e]);
+        xr[e] *= f;
+        yr[e] *= f;
+      }
     }
     for (int row = tid / CPR; row < D; row += RPP) {
       float cv[16];
@@ -777,7 +829,8 @@ __device__ __forceinline__ void step_head(const WinArgs& a, const WinLayout& L, 
   requantize_store<C>(tile, r, a.codes + (size_t)head * a.code_stride,
                       a.scales + (size_t)head * a.scale_stride,
                       a.comp_idx + (size_t)head * ((r + 3) & ~3), a.comp_u + (size_t)head * r * D,
-                      ys, reinterpret_cast<int32_t*>(misc + 4));
+                      ys, reinterpret_cast<int32_t*>(misc + 4),
+                      C::SMOOTH ? a.smooth_exp + (size_t)head * D : nullptr);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -935,7 +988,8 @@ __device__ __forceinline__ void window_state_body(const WinArgs& a, uint8_t* sm,
     requantize_store<C>(tile, r, a.codes + (size_t)head * a.code_stride,
                         a.scales + (size_t)head * a.scale_stride,
                         a.comp_idx + (size_t)head * ((r + 3) & ~3),
-                        a.comp_u + (size_t)head * r * D, colmax, sel);
+                        a.comp_u + (size_t)head * r * D, colmax, sel,
+                        C::SMOOTH ? a.smooth_exp + (size_t)head * D : nullptr);
     if (tid == 0) a.pos[head] = 0;
   } else {
     const int cg = tid % C::CG, rg = tid / C::CG;
@@ -980,7 +1034,8 @@ __device__ __forceinline__ void quantize_body(const WinArgs& a, int head) {
   requantize_store<C>(tile, a.r, a.codes + (size_t)head * a.code_stride,
                       a.scales + (size_t)head * a.scale_stride,
                       a.comp_idx + (size_t)head * ((a.r + 3) & ~3),
-                      a.comp_u + (size_t)head * a.r * D, colmax, sel);
+                      a.comp_u + (size_t)head * a.r * D, colmax, sel,
+                      C::SMOOTH ? a.smooth_exp + (size_t)head * D : nullptr);
   if (threadIdx.x == 0) a.pos[head] = 0;
 }
 

@@ -101,7 +101,12 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
         l = (P > 0 ? s_bL[(P - 1) * D + jj] : 0.f) + s_g[jj];
         e = fast_exp(l);
       }
-      const float xv = e * __bfloat162float(s_k[jj]), yv = e * __bfloat162float(s_q[jj]);
+      float xv = e * __bfloat162float(s_k[jj]), yv = e * __bfloat162float(s_q[jj]);
+      if constexpr (C::SMOOTH) {  // F = dequant Diag(2^e): the codes meet 2^e .* x
+        const float f = pow2i(reinterpret_cast<const int8_t*>(st + L.sexp)[jj]);
+        xv *= f;
+        yv *= f;
+      }
       mx = fmaxf(mx, fabsf(xv));
       my = fmaxf(my, fabsf(yv));
       if (mm == warp) {  // this lane's own column j
@@ -480,7 +485,12 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
         c10 = __uint_as_float(__byte_perm(h1, 0x4B000000u, 0x7650)) - 8388736.f;
         c11 = __uint_as_float(__byte_perm(h1, 0x4B000000u, 0x7651)) - 8388736.f;
       }
-      const float e0 = colexp[j], e1 = colexp[j + 1];
+      float e0 = colexp[j], e1 = colexp[j + 1];
+      if constexpr (C::SMOOTH) {  // the frozen codes' factor 2^e (the old exponents)
+        const int8_t* s_sexp = reinterpret_cast<const int8_t*>(st + L.sexp);
+        e0 *= pow2i(s_sexp[j]);
+        e1 *= pow2i(s_sexp[j + 1]);
+      }
       acc[nt][0] = t0 * c00 * e0;
       acc[nt][1] = t0 * c01 * e1;
       acc[nt][2] = t1 * c10 * e0;
@@ -547,7 +557,7 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
   }
 
   // ---- compensators: column max-abs, the top r (ties: lower index), taken out exactly -----
-  if (r > 0) {
+  if (r > 0 || C::SMOOTH) {
 #pragma unroll
     for (int nt = 0; nt < 16; ++nt) {
       float m0 = fmaxf(fabsf(acc[nt][0]), fabsf(acc[nt][2]));
@@ -609,6 +619,24 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
       if (here) {
         g_cu[c * D + v0] = x0;
         g_cu[c * D + v1] = x1;
+      }
+    }
+    // residual smoothing: column j's exponent from the residual's max-abs (a taken column has
+    // colmax -2: exponent 0), the residual times 2^-e_j before the row absmax
+    if constexpr (C::SMOOTH) {
+      for (int j = tid; j < D; j += C::NT) {
+        const int e = smooth_exponent(colmax[j]);
+        a.smooth_exp[(size_t)head * D + j] = (int8_t)e;
+        colexp[j] = pow2i(-e);  // colexp is dead once the tile is materialised
+      }
+      csync();
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt) {
+        const float f0 = colexp[8 * nt + 2 * q4], f1 = colexp[8 * nt + 2 * q4 + 1];
+        acc[nt][0] *= f0;
+        acc[nt][1] *= f1;
+        acc[nt][2] *= f0;
+        acc[nt][3] *= f1;
       }
     }
   }

@@ -78,7 +78,24 @@ typedef struct {
     int32_t fmt;       /* gdn_state_format */
     int32_t act_dtype; /* gdn_dtype of q, k, v, o and of the buffered keys */
     int32_t buf_dtype; /* gdn_dtype of the buffered write vectors u */
+    int32_t smooth;    /* gdn_smoothing: residual smoothing at every quantization (INT8 and
+                          INT4_G32 states; 0 elsewhere) */
 } gdn_config;
+
+/*
+ * Residual smoothing ("LeapQuant ..." Abstract: the residual left after the compensators is
+ * smoothed before quantization; the page gives no mechanism, this is the reading built here).
+ * At every quantization (gdn_state_quantize, each window end, gdn_window_flush), after the
+ * compensator columns are taken out, key column j of the residual R gets an exponent
+ *     e_j = floor(E_j / 2) clamped to [-63, 63],  E_j = floor(log2 max_i |R_ij|)  (e_j = 0 for a
+ *                                                    zero column),
+ * and the residual is quantized as R Diag(2^-e) (per-row or per-group scales as usual), so the
+ * frozen state is dequant(codes, scales) Diag(2^e): a column's factor is the power of two at or
+ * below the square root of its max-abs, which halves (in log scale) the spread of column ranges
+ * a row's scale must cover. Powers of two make the rescaling exact (fp32, away from the
+ * subnormal range); the exponents live in gdn_state.smooth_exp.
+ */
+typedef enum { GDN_SMOOTH_NONE = 0, GDN_SMOOTH_POW2_COLUMNS = 1 } gdn_smoothing;
 
 /*
  * The windowed low-bit state of a batch: caller-owned device buffers, per head (D = d_k = d_v,
@@ -99,6 +116,8 @@ typedef struct {
  *   status   int32 [1], optional       device word the kernels OR GDN_DEVICE_* bits into
  *   head_fmt int8  [B][H]              (GDN_FMT_MIXED only) GDN_FMT_INT8 or GDN_FMT_INT4_G32 for
  *                                       each head; read by every call, written by none
+ *   smooth_exp int8 [B][H][D]          (smooth != 0 only, 16-byte aligned) the smoothing exponent
+ *                                       e_j of each key column of the frozen codes
  * With GDN_FMT_MIXED ("Low-Bit GDN Recurrent-State Quantization ...", Abstract: bit widths
  * allocated per head under a model-wide budget) every head has the slot of the larger format:
  *   codes    uint8 [B][H][D][D]        an INT8 head fills its slot as above; an INT4_G32 head
@@ -113,9 +132,10 @@ typedef struct {
  * copy each and read eight consecutive rows at one column without bank conflicts.
  * gdn_state_materialize returns the logical state in plain row-major order.
  * The logical state of a head with P = pos pairs and L = buf_L[P-1] (0 when P == 0) is
- *   S = dequant(codes, scales) Diag(e^L) + sum_c comp_u[c] (e_{comp_idx[c]} e^{L})^T
+ *   S = dequant(codes, scales) Diag(2^e) Diag(e^L) + sum_c comp_u[c] (e_{comp_idx[c]} e^{L})^T
  *       + sum_{i<P} buf_u[i] (buf_k[i] * e^{L - buf_L[i]})^T.
- * Entries of buf_k / buf_u / buf_L at index >= pos are scratch and never read.
+ * (Diag(2^e) only with smoothing.) Entries of buf_k / buf_u / buf_L at index >= pos are scratch
+ * and never read.
  */
 typedef struct {
     void* codes;
@@ -128,6 +148,7 @@ typedef struct {
     int32_t* pos;
     int32_t* status;
     const int8_t* head_fmt;
+    int8_t* smooth_exp;
 } gdn_state;
 
 /* Byte sizes of each buffer of gdn_state for the whole batch (0 where unused), and the dynamic
@@ -136,6 +157,7 @@ typedef struct {
     size_t codes, scales, buf_k, buf_u, buf_L, comp_idx, comp_u, pos;
     size_t smem_step;
     size_t head_fmt;
+    size_t smooth_exp;
 } gdn_sizes;
 
 /* Checks cfg and fills *out. Host-only: touches no device. Errors: GDN_ERR_INVALID_ARG for a
@@ -148,7 +170,8 @@ gdn_status gdn_state_sizes(const gdn_config* cfg, gdn_sizes* out);
  * S with the largest max-abs (ties to the lower index) are copied to comp_u / comp_idx and
  * zeroed, then each row (int4: each 32-column group) gets s = absmax / qmax (qmax 127 or 7,
  * IEEE single division) and codes c = clamp(rint(x / s), -qmax, qmax); a zero row gets s = 0
- * and codes 0. pos is set to 0; the window buffer is left as it is.
+ * and codes 0 (with smoothing, the rows are those of the rescaled residual and smooth_exp is
+ * written). pos is set to 0; the window buffer is left as it is.
  *   S   device fp32 [B][H][D][D], read only.
  */
 gdn_status gdn_state_quantize(const gdn_config* cfg, const float* S, const gdn_state* state,

@@ -5,11 +5,13 @@
  * The method ("LinQuant: Functional Invariances for Low-Precision Linear Recurrences",
  * Abstract: a linear recurrence's prefill evaluated chunk by chunk as dense matrix products):
  * the L tokens of a prompt run through the gated delta rule of gdnq.h,
- *     S_t = S_{t-1} a_t (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,     o_t = S_t q_t,
- * for every (sequence, head), in chunks of 64 tokens whose intra-chunk part is a handful of
- * 64 x 64 and 64 x 128 products (the UT / WY form of the delta rule); only the state passes
- * from one chunk to the next. The final state can then be quantized for decode with
- * gdn_state_quantize.
+ *     S_t = S_{t-1} Diag(a_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,     o_t = S_t q_t,
+ * for every (sequence, head), with a scalar gate (GDN: a_t = e^{g_t} on every key channel) or a
+ * per-key-channel gate (KDA: a_t = e^{g_t}, one log-gate per key channel), in chunks whose
+ * intra-chunk part is a handful of dense products (the UT / WY form of the delta rule); only the
+ * state passes from one chunk to the next. Scalar gate: 64-token chunks. Per-channel gate:
+ * 16-token chunks, the pairwise decays e^{G_t - G_s} taken through the chunk's eighth token. The
+ * final state can then be quantized for decode with gdn_state_quantize.
  *
  * Conventions are those of gdnq.h (device pointers, caller-owned buffers, asynchronous work on
  * `stream`, argument checks before anything is enqueued, B * H == 0 a valid empty batch).
@@ -25,19 +27,28 @@ extern "C" {
 
 /*
  * L prompt tokens of every head, in place on S.
- *   cfg     B, H, d_k = d_v = 128, gate GDN_GATE_SCALAR, act_dtype GDN_DTYPE_BF16 (this build);
- *           W, r, fmt and buf_dtype are ignored.
+ *   cfg     B, H, d_k = d_v = 128, gate GDN_GATE_SCALAR or GDN_GATE_DIAG, act_dtype
+ *           GDN_DTYPE_BF16 (this build); W, r, fmt and buf_dtype are ignored.
  *   L       tokens per sequence, >= 0 (any length: a last partial chunk is padded inside the
  *           kernel with tokens that change nothing).
  *   q, k, v device bf16 [B][H][L][D] (head-major: each head's tokens contiguous), 16-byte
  *           aligned; k and q as the decode step takes them (the layer's normalisation applied).
- *   g       device fp32 [B][H][L], the log of the scalar gate; beta device fp32 [B][H][L].
+ *   g       device fp32, the log of the gate, finite: [B][H][L] for the scalar gate (4-byte
+ *           aligned); [B][H][L][D] for the per-channel gate (16-byte aligned), where every
+ *           channel's log-gate summed over any 8 consecutive tokens must stay above -80 (for
+ *           example g >= -10 everywhere) so that the chunk's decay factors e^{+-(G_t - G_r)} stay
+ *           finite in fp32; beyond that the results are undefined.
+ *   beta    device fp32 [B][H][L].
  *   o       device bf16 [B][H][L][D], written for every token.
  *   S       device fp32 [B][H][D][D], 16-byte aligned: the state before the prompt on entry, after
  *           it on return (row = value channel, column = key channel).
  * Arithmetic: products on tensor cores with fp32 accumulation; q, k, v enter exactly, every
  * fp32 operand (the state, the chunk's triangular inverse, the corrected values, the decayed
- * scores, the write vectors) as the sum of two bf16 parts; the triangular inverse in fp32.
+ * scores, keys and queries, the write vectors) as the sum of two bf16 parts; the triangular
+ * inverse in fp32.
+ * Errors: GDN_ERR_INVALID_ARG for a null or misaligned pointer (when B * H > 0 and L > 0), L < 0
+ * or a malformed cfg; GDN_ERR_UNSUPPORTED for d_k or d_v other than 128 or activations other
+ * than bf16 (nothing is enqueued on either); a failed launch as GDN_ERR_CUDA.
  */
 gdn_status gdn_prefill(const gdn_config* cfg, int32_t L, const void* q, const void* k,
                        const void* v, const float* g, const float* beta, void* o, float* S,

@@ -228,8 +228,9 @@ int orc_smooth_exponent(double colmax) {
 
 /* Window-end operation on a full state S (overwritten by the residual): take out r compensator
  * columns exactly, then (smooth) rescale the residual's columns by 2^{-e_j} into sexp, then
- * quantize the residual. fmt == NONE keeps the (rescaled) residual unquantized in S. Returns the
- * near-tie flag of the column choice. sexp may be NULL when smooth is 0. */
+ * quantize the residual. fmt == NONE keeps the (rescaled) residual unquantized in S. Returns 1
+ * on a near tie (of the column choice, or of a smoothing exponent). sexp may be NULL when smooth
+ * is 0. */
 static int window_end(int D, int fmt, int r, int prec32, int smooth, double* S, int8_t* codes,
                       double* scales, int* cidx, double* cu, int8_t* sexp) {
     int near = orc_select_columns(D, r, S, cidx);
@@ -243,6 +244,12 @@ static int window_end(int D, int fmt, int r, int prec32, int smooth, double* S, 
             double m = 0.0;
             for (int i = 0; i < D; ++i) m = fmax(m, fabs(S[(size_t)i * D + j]));
             sexp[j] = (int8_t)orc_smooth_exponent(m);
+            /* the exponent steps where the max-abs crosses a power of 4: within 1e-6 relative
+             * of one, another correct implementation may round it to the other side */
+            if (m > 0.0) {
+                double p4 = ldexp(1.0, 2 * (int)floor(log2(m) / 2.0 + 0.5));
+                if (fabs(m - p4) <= 1e-6 * p4) near = 1;
+            }
             for (int i = 0; i < D; ++i) S[(size_t)i * D + j] = ldexp(S[(size_t)i * D + j], -sexp[j]);
         }
     }

@@ -21,7 +21,8 @@ from workloads import Workload, decode_inputs, outlier_scales, step_inputs, torc
 
 
 def cfg_of(wl: Workload):
-    return gdn.make_config(wl.B, wl.H, wl.D, wl.W, wl.r, wl.gate, wl.fmt, wl.act, wl.buf)
+    return gdn.make_config(wl.B, wl.H, wl.D, wl.W, wl.r, wl.gate, wl.fmt, wl.act, wl.buf,
+                           smooth=wl.smooth)
 
 
 def gpu_warmup(wl: Workload, device="cuda") -> torch.Tensor:
@@ -40,8 +41,8 @@ def gpu_warmup(wl: Workload, device="cuda") -> torch.Tensor:
 
 def _heads_np(x: torch.Tensor, heads: np.ndarray) -> np.ndarray:
     """[T][B][H](...) device tensor -> [T][n](...) float64 numpy for the flat head indices."""
-    T = x.shape[0]
-    flat = x.reshape(T, -1, *x.shape[3:]) if x.dim() > 3 else x.reshape(T, -1)
+    T, nh = x.shape[0], x.shape[1] * x.shape[2]
+    flat = x.reshape(T, nh, *x.shape[3:])
     idx = torch.as_tensor(heads, device=x.device, dtype=torch.long)
     return flat.index_select(1, idx).double().cpu().numpy()
 
@@ -97,7 +98,8 @@ def gpu_run(wl: Workload, device="cuda", T: int | None = None, inputs=None, S0=N
 def oracle_run(wl: Workload, heads: np.ndarray, inputs: dict, S0: np.ndarray, flush_mask=None):
     q, k, v, g, beta = (_heads_np(inputs[n], heads) for n in ("q", "k", "v", "g", "beta"))
     return oracle.o2_run(q, k, v, g, beta, W=wl.W, r=wl.r, fmt=wl.fmt, S0=S0,
-                         round_storage=True, buf_round=wl.buf, flush_mask=flush_mask)
+                         round_storage=True, buf_round=wl.buf, flush_mask=flush_mask,
+                         smooth=wl.smooth)
 
 
 # ---------------------------------------------------------------------------------------------
@@ -212,6 +214,10 @@ def compare(wl: Workload, run: GpuRun, heads: np.ndarray, res) -> Parity:
         assert np.array_equal(cidx[ok], res.cidx[ok]), "compensator columns differ"
         crel = rel_l2(cu[ok], res.cu[ok]) if ok.any() else 0.0
     pos = run.state.pos[torch.as_tensor(heads, device=run.state.pos.device)].cpu().numpy()
+    if wl.smooth:  # smoothing exponents are integer decisions: equal away from near ties
+        sexp = run.state.smooth_exp[: wl.heads * wl.D].view(-1, wl.D)[
+            torch.as_tensor(heads, device=run.state.pos.device)].cpu().numpy()
+        assert np.array_equal(sexp[ok], res.sexp[ok]), "smoothing exponents differ"
     # a flipped code changes that row's scale only when the flip is the absmax entry; scales are
     # compared where every code of the row agrees
     rows_same = (diff.reshape(diff.shape[0], wl.D, -1).max(axis=-1) == 0) if diff.size else diff

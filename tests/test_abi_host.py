@@ -84,6 +84,7 @@ BAD_CONFIGS = [
     ("baseline fmt", dict(fmt="bf16"), _abi.GDN_ERR_INVALID_ARG),
     ("window too big", dict(W=5000), _abi.GDN_ERR_UNSUPPORTED),
     ("B<0", dict(B=-1), _abi.GDN_ERR_INVALID_ARG),
+    ("smoothing of a mixed state", dict(fmt="mixed", smooth=True), _abi.GDN_ERR_UNSUPPORTED),
 ]
 
 
@@ -102,7 +103,8 @@ def test_raw_field_errors(lib):
     assert lib.gdn_state_sizes(None, ctypes.byref(out)) == _abi.GDN_ERR_INVALID_ARG
     cfg = _cfg()
     assert lib.gdn_state_sizes(ctypes.byref(cfg), None) == _abi.GDN_ERR_INVALID_ARG
-    for field, val in (("gate", 7), ("fmt", 9), ("act_dtype", 3), ("buf_dtype", -1)):
+    for field, val in (("gate", 7), ("fmt", 9), ("act_dtype", 3), ("buf_dtype", -1),
+                       ("smooth", 2), ("smooth", -1)):
         c = _cfg()
         setattr(c, field, val)
         assert lib.gdn_state_sizes(ctypes.byref(c), ctypes.byref(out)) == _abi.GDN_ERR_INVALID_ARG
@@ -129,6 +131,20 @@ def test_state_pointer_checks(field, lib):
         rc = lib.gdn_decode_window_step(ctypes.byref(cfg), ctypes.byref(st), q, q, q, q, q, q, None)
         assert rc == _abi.GDN_ERR_INVALID_ARG
         assert field.encode() in lib.gdn_last_error()
+
+
+@pytest.mark.parametrize("fmt", ["int8", "int4_g32"])
+def test_smoothing_sizes_and_exponent_pointer(fmt, lib):
+    """A smoothed state has D exponent bytes per head; its pointer is required (16-byte
+    aligned) only when smoothing is on, and checked before anything is enqueued."""
+    cfg = _cfg(fmt=fmt, smooth=True)
+    assert gdn.gdn_state_sizes(cfg).smooth_exp == 6 * 128
+    assert gdn.gdn_state_sizes(_cfg(fmt=fmt)).smooth_exp == 0
+    q = ctypes.c_void_p(0x900000)
+    for st in (_fake_state(null="smooth_exp"), _fake_state(misalign="smooth_exp")):
+        rc = lib.gdn_decode_window_step(ctypes.byref(cfg), ctypes.byref(st), q, q, q, q, q, q, None)
+        assert rc == _abi.GDN_ERR_INVALID_ARG
+        assert b"smooth_exp" in lib.gdn_last_error()
 
 
 def test_compensator_pointers_needed_only_with_r(lib):

@@ -152,3 +152,17 @@ def test_prefill_then_window_decode(base):
     res = oracle.o2_run(q, k, v, g, beta, W=wl.W, fmt="int8", S0=S_ref, round_storage=True)
     o_rel = rel_l2(_heads_np(o, heads), round_act(res.o, "bf16"))
     assert o_rel <= O_TOL, o_rel
+
+
+@pytest.mark.parametrize("name", ["gdn-prefill", "kda-prefill"])
+def test_prefill_full_size_sampled_heads(name):
+    """The prompt workloads the benchmark times (8 x 32 heads, 4096-token prompts, one launch),
+    checked on sampled heads against the plain fp64 recurrence."""
+    wl = WORKLOADS[name]
+    inp = decode_inputs(wl, "cuda")
+    o, S = pf_run(wl, inp, torch.zeros((wl.B, wl.H, wl.D, wl.D), device="cuda"))
+    assert bool(torch.isfinite(S).all())
+    heads = sample_heads(wl, 4, seed=wl.seed)
+    o_rel, s_rel = compare(wl, inp, o, S, heads)
+    print(name, o_rel, s_rel)
+    assert o_rel <= O_TOL and s_rel <= S_TOL, (o_rel, s_rel)

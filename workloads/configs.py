@@ -20,6 +20,7 @@ class Workload:
     outliers: bool = True  # 2% of key and value channels scaled x20
     warmup: int = 512      # fp32 recurrence tokens that make the initial state (0: zero state)
     seed: int = 0
+    smooth: bool = False   # residual smoothing at every quantization
 
     @property
     def heads(self) -> int:
@@ -45,6 +46,9 @@ WORKLOADS = {
     # prompt prefill before decode: T = prompt length L, one chunkwise launch over all of it
     "gdn-prefill": Workload("gdn-prefill", B=8, H=32, D=128, T=4096, W=64, warmup=0,
                             seed=1006),
+    # the same prompt batch with the per-key-channel gate
+    "kda-prefill": Workload("kda-prefill", B=8, H=32, D=128, T=4096, W=64, gate="diag",
+                            warmup=0, seed=1007),
 }
 
 

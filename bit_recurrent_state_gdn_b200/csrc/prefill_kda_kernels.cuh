@@ -93,11 +93,10 @@ __device__ __forceinline__ void kda_load_chunk(uint8_t* st, const PfArgs& a, siz
 
 // Two adjacent fp32 values as hi / lo bf16 pairs at element idx of the tiles hi and lo.
 __device__ __forceinline__ void put_split2(uint8_t* hi, uint8_t* lo, int idx, float x, float y) {
-  __nv_bfloat162 h, l;
-  split_bf16(x, h.x, l.x);
-  split_bf16(y, h.y, l.y);
-  reinterpret_cast<__nv_bfloat162*>(hi)[idx >> 1] = h;
-  reinterpret_cast<__nv_bfloat162*>(lo)[idx >> 1] = l;
+  uint32_t h, l;
+  split2_bf16(x, y, h, l);
+  reinterpret_cast<uint32_t*>(hi)[idx >> 1] = h;
+  reinterpret_cast<uint32_t*>(lo)[idx >> 1] = l;
 }
 
 __global__ void __launch_bounds__(kPfThreads, kKdaCtas) prefill_kda_kernel(const PfArgs a) {
@@ -138,15 +137,17 @@ __global__ void __launch_bounds__(kPfThreads, kKdaCtas) prefill_kda_kernel(const
     __syncthreads();  // this chunk's inputs; every warp done with the previous chunk
 
     // ---- decayed operands: thread = (channels 2 jp, 2 jp + 1; tokens 4 tq..4 tq + 3) ----------
+    // (cumulative log-gates in base 2, G log2(e), so each factor is one hardware exp2)
     {
+      constexpr float kLog2e = 1.4426950408889634f;
       const int jp = tid & 63, tq = tid >> 6, j0 = 2 * jp;
       const float* G = reinterpret_cast<const float*>(st + L_::RG);
       float2 run = make_float2(0.f, 0.f), gr = run, gt[4];
 #pragma unroll
       for (int t = 0; t < kKc; ++t) {
         const float2 gg = *reinterpret_cast<const float2*>(G + t * kPfD + j0);
-        run.x += gg.x;
-        run.y += gg.y;
+        run.x = fmaf(gg.x, kLog2e, run.x);
+        run.y = fmaf(gg.y, kLog2e, run.y);
         if (t == kKref) gr = run;
         if ((t >> 2) == tq) gt[t & 3] = run;
       }
@@ -155,9 +156,9 @@ __global__ void __launch_bounds__(kPfThreads, kKdaCtas) prefill_kda_kernel(const
       for (int i = 0; i < 4; ++i) {
         const int t = 4 * tq + i, idx = t * kLd128 + j0;
         const float dx = gt[i].x - gr.x, dy = gt[i].y - gr.y;
-        const float tx = expf(dx), ty = expf(dy);        // e^{G_t - G_r}
-        const float hx = expf(-dx), hy = expf(-dy);      // e^{G_r - G_t}
-        const float cx = expf(gc.x - gt[i].x), cy = expf(gc.y - gt[i].y);  // e^{G_C - G_t}
+        const float tx = fast_exp2(dx), ty = fast_exp2(dy);    // e^{G_t - G_r}
+        const float hx = fast_exp2(-dx), hy = fast_exp2(-dy);  // e^{G_r - G_t}
+        const float cx = fast_exp2(gc.x - gt[i].x), cy = fast_exp2(gc.y - gt[i].y);  // e^{G_C - G_t}
         const float2 kk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(st + L_::RK + 2 * idx));
         const float2 qq = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(st + L_::RQ + 2 * idx));
         put_split2(sm + L_::KT, sm + L_::KT + L_::T128, idx, kk.x * tx, kk.y * ty);
@@ -166,8 +167,8 @@ __global__ void __launch_bounds__(kPfThreads, kKdaCtas) prefill_kda_kernel(const
         put_split2(sm + L_::KC, sm + L_::KC + L_::T128, idx, kk.x * cx, kk.y * cy);
       }
       if (tq == 0) {
-        *reinterpret_cast<float2*>(sm + L_::ER + 4 * j0) = make_float2(expf(gr.x), expf(gr.y));
-        *reinterpret_cast<float2*>(sm + L_::EC + 4 * j0) = make_float2(expf(gc.x), expf(gc.y));
+        *reinterpret_cast<float2*>(sm + L_::ER + 4 * j0) = make_float2(fast_exp2(gr.x), fast_exp2(gr.y));
+        *reinterpret_cast<float2*>(sm + L_::EC + 4 * j0) = make_float2(fast_exp2(gc.x), fast_exp2(gc.y));
       }
     }
     __syncthreads();
@@ -186,12 +187,9 @@ __global__ void __launch_bounds__(kPfThreads, kKdaCtas) prefill_kda_kernel(const
         for (int half = 0; half < 2; ++half) {
           const float2 e = *reinterpret_cast<const float2*>(ER + 16 * ks + 8 * half + 2 * q4);
 #pragma unroll
-          for (int nn = 0; nn < 2; ++nn) {
-            const float x0 = sacc[2 * ks + half][2 * nn] * e.x, x1 = sacc[2 * ks + half][2 * nn + 1] * e.y;
-            const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
-            bh[nn][half] = pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
-            bl[nn][half] = pack_bf16(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
-          }
+          for (int nn = 0; nn < 2; ++nn)
+            split2_bf16(sacc[2 * ks + half][2 * nn] * e.x, sacc[2 * ks + half][2 * nn + 1] * e.y,
+                        bh[nn][half], bl[nn][half]);
         }
         const uint32_t off = 2u * ((lane & 15) * kLd128 + 16 * ks + 8 * (lane >> 4));
         uint32_t ah[4], al[4];

@@ -79,6 +79,20 @@ __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bflo
   lo = __float2bfloat16_rn(x - __bfloat162float(hi));
 }
 
+// 2^x on the hardware path (relative error about 2^-22; a result below 2^-126 flushes to 0).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// The same for two values at once, as packed bf16 pairs (x0 in the low half): hi = RN(x),
+// lo = RN(x - hi), with one packed conversion each.
+__device__ __forceinline__ void split2_bf16(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16(x0, x1);
+  lo = pack_bf16(x0 - bf16_lo(hi), x1 - bf16_hi(hi));
+}
+
 // acc (16 x 8 NT) += A (16 x 16 KS) * B (16 KS x 8 NT) on mma.m16n8k16 bf16.
 //   A: rows m0.., columns k0.. of a bf16 tile at a_base (row stride lda elements); A_T: the tile
 //      is stored transposed ([k][m]).
@@ -129,14 +143,10 @@ __device__ __forceinline__ void store_split(const float (&acc)[NT][4], __nv_bflo
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       const int r = m0 + gid + 8 * hh, c = n0 + 8 * nt + 2 * q4;
-      __nv_bfloat16 h0, l0, h1, l1;
-      split_bf16(f(r, c, acc[nt][2 * hh]), h0, l0);
-      split_bf16(f(r, c + 1, acc[nt][2 * hh + 1]), h1, l1);
-      __nv_bfloat162 hv, lv;
-      hv.x = h0; hv.y = h1;
-      lv.x = l0; lv.y = l1;
-      *reinterpret_cast<__nv_bfloat162*>(hi + r * ld + c) = hv;
-      *reinterpret_cast<__nv_bfloat162*>(lo + r * ld + c) = lv;
+      uint32_t hv, lv;
+      split2_bf16(f(r, c, acc[nt][2 * hh]), f(r, c + 1, acc[nt][2 * hh + 1]), hv, lv);
+      *reinterpret_cast<uint32_t*>(hi + r * ld + c) = hv;
+      *reinterpret_cast<uint32_t*>(lo + r * ld + c) = lv;
     }
   }
 }
@@ -202,12 +212,9 @@ __device__ __forceinline__ void mma_state_slab(float (&acc)[8][4], uint32_t a_ba
 #pragma unroll
     for (int nn = 0; nn < 2; ++nn)
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const float x0 = sacc[2 * ks + half][2 * nn], x1 = sacc[2 * ks + half][2 * nn + 1];
-        const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
-        bh[nn][half] = pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
-        bl[nn][half] = pack_bf16(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
-      }
+      for (int half = 0; half < 2; ++half)
+        split2_bf16(sacc[2 * ks + half][2 * nn], sacc[2 * ks + half][2 * nn + 1], bh[nn][half],
+                    bl[nn][half]);
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) {
       uint32_t a[4];

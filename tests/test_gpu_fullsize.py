@@ -1,8 +1,9 @@
 """CUDA path vs the CPU oracle at the workloads' full sizes, in the launch configuration the
 benchmark times (every head of the batch, one launch per decode step through
 gdn_decode_window_steps), compared on sampled heads that the oracle recomputes from their own
-inputs: every head of the first and the last sequence plus random others. Also the largest
-window and compensator count the build accepts.
+inputs: every head of the first and the last sequence plus random others; the serving and KDA
+workloads also with residual smoothing. Also the largest window and compensator count the build
+accepts.
 
 Each run also reports the quality figure: the GPU output against the unquantized fp64
 recurrence from the same initial state (not a parity bar; the windowed low-bit state is an
@@ -30,12 +31,13 @@ def _quality(wl, run, heads, S0):
     return rel_l2(o_gpu, o_ref)
 
 
-@pytest.mark.parametrize("name", list(SAMPLE))
+@pytest.mark.parametrize("name", list(SAMPLE) + ["gdn-serving+smooth", "kda+smooth"])
 def test_full_size_sampled_heads(name):
-    wl = WORKLOADS[name]
+    base, _, extra = name.partition("+")
+    wl = WORKLOADS[base].with_(smooth=extra == "smooth")
     run = gpu_run(wl)
     assert int(run.state.status[0].item()) == 0
-    heads = sample_heads(wl, SAMPLE[name], seed=wl.seed)
+    heads = sample_heads(wl, SAMPLE[base], seed=wl.seed)
     S0 = oracle_initial_state(wl, heads)
     res = oracle_run(wl, heads, run.inputs, S0)
     p = compare(wl, run, heads, res)

@@ -890,6 +890,17 @@ __global__ void __launch_bounds__(kStepThreads, 2)
     }
     stage_issue<C>(a, L, st, bar, head, P, true);
   };
+  // every stage's write-vector rows start at zero (tensor-core path): a row past a head's pairs
+  // then holds zeros or an earlier head's finite write vector, and meets a zero coefficient in
+  // the buffer product; the zeros are ordered before the stage copies by the proxy fence
+  if (mma) {
+    const int n16 = cap * C::D * (int)sizeof(typename C::Buf) / 16;
+    for (int s = 0; s < nstages; ++s) {
+      uint4* bu = reinterpret_cast<uint4*>(sm + L.stage0 + s * L.stage_bytes + L.bu);
+      for (int e = tid; e < n16; e += C::NT) bu[e] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L.bars);
   if (tid == 0) {
     for (int s = 0; s < nstages; ++s) mbar_init(&bars[s], 1);

@@ -227,11 +227,12 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
     }
   } else {
     const int ty = tid - 128, wy = warp - 4;
-    // padding of the phase-3 product to a multiple of 16 pairs: zero rows of U and zero
-    // coefficients (the product must not see stale or non-finite shared memory)
-    for (int e2 = ty; e2 < (Pp - P) * D; e2 += 128) s_bu[P * D + e2] = __float2bfloat16_rn(0.f);
-    for (int e2 = ty; e2 < 6 * (Pp - P); e2 += 128)
-      Bc[(e2 / (Pp - P)) * bcs + P + e2 % (Pp - P)] = __float2bfloat16_rn(0.f);
+    // padding of the phase-3 product to a multiple of 16 pairs: zero coefficients for the rows
+    // past the P pairs, whose write-vector rows hold zeros or an earlier head's finite values
+    if (ty < 96) {
+      const int i = P + (ty & 15);
+      if (i < Pp) Bc[(ty >> 4) * bcs + i] = __float2bfloat16_rn(0.f);
+    }
     if (ty < r) {  // compensator pairs: key e_j entered at L = 0, so their coefficient is x[j]
       const int j = s_cidx[ty] & (D - 1);
       float e;

@@ -1,5 +1,6 @@
-// Chunkwise-parallel prefill with a per-key-channel gate (KDA, "Kimi Linear" gating in the
-// gated delta rule), the counterpart of prefill_kernels.cuh's scalar-gate kernel ("LinQuant:
+// Chunkwise-parallel prefill with a per-key-channel gate (Kimi Delta Attention, KDA, which
+// "LeapQuant: Efficient Linear Attention with Accurate Recurrent State Quantization", Abstract,
+// names beside GDN), the counterpart of prefill_kernels.cuh's scalar-gate kernel ("LinQuant:
 // Functional Invariances for Low-Precision Linear Recurrences", Abstract: prefill of a linear
 // recurrence cast as chunked dense matmuls).
 //

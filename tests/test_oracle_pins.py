@@ -45,3 +45,17 @@ def test_zero_steps_and_empty_batch(orc):
     o, S = oracle.plain_run(np.zeros((0, 2, 4)), np.zeros((0, 2, 4)), np.zeros((0, 2, 4)),
                             np.zeros((0, 2)), np.zeros((0, 2)))
     assert o.shape == (0, 2, 4) and not S.any()
+
+
+def test_smoothing_exponent_near_ties_are_reported(orc):
+    """A residual column max-abs within 1e-6 of a power of 4 sits where the smoothing exponent
+    steps; the oracle reports the head as a near tie (another correct implementation may put
+    the column on the other side), and does not for column maxima away from one."""
+    lib = orc.load()
+    rng = np.random.default_rng(29)
+    S = rng.uniform(-1, 1, size=(16, 16))
+    S *= (2.0 + rng.uniform(size=16))[None, :] / np.abs(S).max(axis=0)  # column maxima in [2, 3)
+    assert oracle.window_end(S, "int8", smooth=True, lib=lib).near_tie == 0
+    S[3, 5] = 4.0 * (1 - 3e-7)  # just below 4 = 2^2
+    assert oracle.window_end(S, "int8", smooth=True, lib=lib).near_tie == 1
+    assert oracle.window_end(S, "int8", smooth=False, lib=lib).near_tie == 0

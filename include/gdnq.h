@@ -183,11 +183,13 @@ gdn_status gdn_state_quantize(const gdn_config* cfg, const float* S, const gdn_s
  * state is quantized once, at the window's end). With P = pos, L = buf_L[P-1] (0 if P == 0):
  *   L_t = L + g_t;  x = e^{L_t} k_t;  y = e^{L_t} q_t   (scalar gate: e^{L_t} is a scalar)
  *   w = F x + sum_c comp_u[c] x[comp_idx[c]] + sum_{i<P} buf_u[i] <buf_k[i] e^{L_t - buf_L[i]}, k_t>
- *   r = the same with y and q_t                         (F = dequantised codes)
+ *   r = the same with y and q_t                         (F = dequantised codes, times
+ *                                                        Diag(2^smooth_exp) with smoothing)
  *   u_t = round_buf(beta_t (v_t - w));  o_t = round_act(r + u_t <k_t, q_t>)
  * then (k_t, u_t, L_t) is appended at index P. When P + 1 == W the window is flushed in the same
- * kernel: the logical state (with the new pair) is materialised in fp32, compensators and codes
- * are rebuilt exactly as in gdn_state_quantize, and pos becomes 0; otherwise pos becomes P + 1.
+ * kernel: the logical state (with the new pair) is materialised in fp32, compensators, codes (and
+ * with smoothing the exponents) are rebuilt exactly as in gdn_state_quantize, and pos becomes 0;
+ * otherwise pos becomes P + 1.
  * The step's output is taken before that requantisation.
  *   q, k, v  device act [B][H][D];  g device fp32 [B][H] (scalar) or [B][H][D] (diagonal), the
  *   log of the gate (<= 0 for a decaying gate);  beta device fp32 [B][H];  o device act [B][H][D].

@@ -80,7 +80,9 @@ def load(path: Optional[str] = None):
     lib.orc_o1_run.restype = _int
     lib.orc_o1_run.argtypes = [_int] * 8 + [_vp] * 8
     lib.orc_o2_run.restype = _int
-    lib.orc_o2_run.argtypes = [_int] * 10 + [_vp] * 19
+    lib.orc_o2_run.argtypes = [_int] * 10 + [_vp] * 21
+    lib.orc_round_other.restype = ctypes.c_double
+    lib.orc_round_other.argtypes = [_int, ctypes.c_double]
     lib.orc_smooth_exponent.restype = _int
     lib.orc_smooth_exponent.argtypes = [ctypes.c_double]
     lib.orc_window_end.restype = _int
@@ -113,6 +115,11 @@ def _f64(a):
 # ---------------------------------------------------------------------------------------------
 def round_bf16(x: float, lib=None) -> float:
     return (lib or load()).orc_round_bf16(float(x))
+
+
+def round_other(x: float, mode: str = "bf16", lib=None) -> float:
+    """The neighbour of x in the storage format on the other side from its rounding."""
+    return (lib or load()).orc_round_other(_ROUND[mode], float(x))
 
 
 def round_bf16_array(a: np.ndarray, lib=None) -> np.ndarray:
@@ -257,14 +264,17 @@ class O2Result:
     near_ties: int
     ties: np.ndarray       # [nh] near ties per head
     sexp: np.ndarray       # [nh][D] int8 smoothing exponents (zeros without smoothing)
+    u_raw: Optional[np.ndarray] = None  # [T][nh][D] write vectors before storage rounding
 
 
 def o2_run(q, k, v, g, beta, W: int, r: int = 0, fmt: str = "int8", S0=None,
            round_storage: bool = False, buf_round: str = "bf16", flush_mask=None,
-           smooth: bool = False, lib=None) -> O2Result:
+           smooth: bool = False, want_u_raw: bool = False, u_flip=None, lib=None) -> O2Result:
     """Buffered-window form. ``round_storage`` mirrors GPU storage (fp32 state / L / scales,
     ``buf_round`` write vectors, fp32 quantizer decisions); ``smooth`` adds the residual
-    smoothing at every quantization."""
+    smoothing at every quantization. ``want_u_raw`` returns every write vector before its
+    storage rounding; ``u_flip`` ([T][nh][D], nonzero entries) stores those write-vector entries
+    rounded to the other neighbour (an alternative result for entries on a rounding midpoint)."""
     lib = lib or load()
     q, k, v, beta = _f64(q), _f64(k), _f64(v), _f64(beta)
     T, nh, D = k.shape
@@ -280,11 +290,15 @@ def o2_run(q, k, v, g, beta, W: int, r: int = 0, fmt: str = "int8", S0=None,
         S=np.zeros((nh, D, D)), near_ties=0, ties=np.zeros(nh, np.int32),
         sexp=np.zeros((nh, D), np.int8))
     fm = None if flush_mask is None else np.ascontiguousarray(flush_mask, np.uint8).reshape(T, nh)
+    if want_u_raw:
+        res.u_raw = np.zeros((T, nh, D))
+    uf = None if u_flip is None else np.ascontiguousarray(u_flip, np.uint8).reshape(T, nh, D)
     res.near_ties = lib.orc_o2_run(
         D, T, W, r, f, nh, Dg, int(round_storage), _ROUND[buf_round], int(smooth), _p(S0),
         _p(q), _p(k), _p(v), _p(g), _p(beta), _p(fm), _p(res.o), _p(res.codes), _p(res.scales),
         _p(res.cidx) if r > 0 else None, _p(res.cu) if r > 0 else None, _p(res.pos),
-        _p(res.bk), _p(res.bu), _p(res.bL), _p(res.S), _p(res.ties), _p(res.sexp))
+        _p(res.bk), _p(res.bu), _p(res.bL), _p(res.S), _p(res.ties), _p(res.sexp),
+        _p(res.u_raw), _p(uf))
     return res
 
 

@@ -104,6 +104,27 @@ static double round_to(int mode, double x) {
     return x;
 }
 
+/* The storage value on the other side of x from round_to(mode, x): the two values of the
+ * format that bracket x are lo = floor(x / q) q and lo + q, q the quantum of x's binade
+ * (2^(e-8) for bfloat16, 2^(e-24) for single, never finer than the subnormal quantum); the
+ * nearest one is the rounding, the other one is returned. When x is itself representable there
+ * is no other side and x is returned. Used for the alternative result of a value that lies
+ * within rounding noise of a midpoint (another correct implementation may round it the other
+ * way). */
+double orc_round_other(int mode, double x) {
+    if (mode == ORC_ROUND_NONE || x == 0.0 || !isfinite(x)) return x;
+    int e;
+    frexp(x, &e);
+    const int bits = mode == ORC_ROUND_BF16 ? 8 : 24;
+    int qexp = e - bits;
+    const int qmin = mode == ORC_ROUND_BF16 ? -133 : -149;
+    if (qexp < qmin) qexp = qmin;
+    const double quantum = ldexp(1.0, qexp);
+    const double lo = floor(x / quantum) * quantum, hi = lo + quantum;
+    if (lo == x) return x;
+    return round_to(mode, x) == lo ? hi : lo;
+}
+
 /* ------------------------------------------------------------------------------------------
  * Quantizer. codes are one int8 per entry (int4 codes lie in [-7, 7]); scales are [D][groups].
  * prec32 = 1 takes every decision in single precision, as a GPU does: the caller passes
@@ -427,8 +448,11 @@ int orc_o1_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int smooth, 
  * cidx [nh][r]; cu [nh][r][D]; pos [nh]; bk, bu, bL [nh][W][D]; S_out [nh][D][D] (the logical
  * state at the end); ties_out [nh] (near ties met per head); sexp_out [nh][D] (the smoothing
  * exponents of the last quantization); flush_mask [T][nh] forces a flush
- * after step t of head h when nonzero. Returns the number of near ties met in compensator
- * choices.
+ * after step t of head h when nonzero; u_raw [T][nh][D] receives every write vector before its
+ * storage rounding; u_flip [T][nh][D], when nonzero at an entry, stores that write-vector entry
+ * rounded to the other neighbour of its storage format (orc_round_other: the alternative result
+ * of an entry that lies within rounding noise of a midpoint). Returns the number of near ties
+ * met in compensator choices.
  * ---------------------------------------------------------------------------------------- */
 typedef struct {
     int D, W, r, fmt, Dg, round_storage, buf_round, smooth;
@@ -483,7 +507,7 @@ static int o2_flush(const o2_cfg* c, o2_head* s, double* scratch_S, double* scra
 
 static void o2_step(const o2_cfg* c, o2_head* s, const double* qt, const double* kt, const double* vt,
                     const double* gt, double bt, double* ot, double* Lt, double* x, double* y,
-                    double* w, double* rr) {
+                    double* w, double* rr, double* u_raw, const uint8_t* u_flip) {
     int D = c->D;
     o2_current_L(c, s, Lt);
     for (int j = 0; j < D; ++j) {
@@ -525,7 +549,9 @@ static void o2_step(const o2_cfg* c, o2_head* s, const double* qt, const double*
     double* un = s->bu + (size_t)s->P * D;
     for (int i = 0; i < D; ++i) {
         double u = bt * (vt[i] - w[i]);
-        if (c->round_storage) u = round_to(c->buf_round, u);
+        if (u_raw) u_raw[i] = u;
+        if (c->round_storage)
+            u = (u_flip && u_flip[i]) ? orc_round_other(c->buf_round, u) : round_to(c->buf_round, u);
         un[i] = u;
         if (ot) ot[i] = rr[i] + u * kq;
     }
@@ -539,7 +565,7 @@ int orc_o2_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int round_st
                const double* g, const double* beta, const uint8_t* flush_mask, double* o,
                int8_t* codes_out, double* scales_out, int* cidx_out, double* cu_out, int* pos_out,
                double* bk_out, double* bu_out, double* bL_out, double* S_out, int* ties_out,
-               int8_t* sexp_out) {
+               int8_t* sexp_out, double* u_raw, const uint8_t* u_flip) {
     o2_cfg c = {D, W, r, fmt, Dg, round_storage, buf_round, smooth};
     int ng = orc_num_groups(fmt == ORC_FMT_NONE ? ORC_FMT_INT8 : fmt, D);
     int ties = 0;
@@ -566,7 +592,8 @@ int orc_o2_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int round_st
         for (int t = 0; t < T; ++t) {
             size_t th = (size_t)t * nh + h;
             o2_step(&c, &s, q + th * D, k + th * D, v + th * D, g + th * Dg, beta[th],
-                    o ? o + th * D : NULL, Lt, x, y, w, rr);
+                    o ? o + th * D : NULL, Lt, x, y, w, rr, u_raw ? u_raw + th * D : NULL,
+                    u_flip ? u_flip + th * D : NULL);
             int forced = flush_mask && flush_mask[th];
             if (s.P == W || forced) hties += o2_flush(&c, &s, Sx, Lt);
         }

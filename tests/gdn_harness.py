@@ -25,17 +25,21 @@ def cfg_of(wl: Workload):
                            smooth=wl.smooth)
 
 
-def gpu_warmup(wl: Workload, device="cuda") -> torch.Tensor:
-    """fp32 [B][H][D][D] initial states from the library's fp32-state baseline kernel."""
+def gpu_warmup(wl: Workload, device="cuda", draw=None) -> torch.Tensor:
+    """fp32 [B][H][D][D] initial states from the library's fp32-state baseline kernel. The
+    warm-up inputs are drawn on ``draw`` (default: ``device``) and copied to ``device``; the
+    oracle's initial state must be drawn on the same device (the generators differ)."""
+    draw = draw or device
     S = torch.zeros((wl.B, wl.H, wl.D, wl.D), dtype=torch.float32, device=device)
     if wl.warmup == 0:
         return S
     cfg = gdn.make_config(wl.B, wl.H, wl.D, gate=wl.gate, fmt="fp32", act=wl.act)
-    scales = outlier_scales(wl, device)
+    scales = outlier_scales(wl, draw)
     o = torch.empty((wl.B, wl.H, wl.D), dtype=torch_dtype(wl.act), device=device)
     for t in range(wl.warmup):
-        s = step_inputs(wl, "warmup", t, device, scales)
-        gdn.gdn_baseline_step(cfg, S, s.q, s.k, s.v, s.g, s.beta, o)
+        s = step_inputs(wl, "warmup", t, draw, scales)
+        q, k, v, g, beta = (x.to(device) for x in (s.q, s.k, s.v, s.g, s.beta))
+        gdn.gdn_baseline_step(cfg, S, q, k, v, g, beta, o)
     return S
 
 
@@ -95,11 +99,19 @@ def gpu_run(wl: Workload, device="cuda", T: int | None = None, inputs=None, S0=N
     return GpuRun(o, state, S0, inputs)
 
 
-def oracle_run(wl: Workload, heads: np.ndarray, inputs: dict, S0: np.ndarray, flush_mask=None):
-    q, k, v, g, beta = (_heads_np(inputs[n], heads) for n in ("q", "k", "v", "g", "beta"))
+def _o2(wl: Workload, q, k, v, g, beta, S0, flush_mask, **kw):
     return oracle.o2_run(q, k, v, g, beta, W=wl.W, r=wl.r, fmt=wl.fmt, S0=S0,
                          round_storage=True, buf_round=wl.buf, flush_mask=flush_mask,
-                         smooth=wl.smooth)
+                         smooth=wl.smooth, **kw)
+
+
+def oracle_run(wl: Workload, heads: np.ndarray, inputs: dict, S0: np.ndarray, flush_mask=None):
+    q, k, v, g, beta = (_heads_np(inputs[n], heads) for n in ("q", "k", "v", "g", "beta"))
+    res = _o2(wl, q, k, v, g, beta, S0, flush_mask)
+    # what a re-run of single heads needs (loose scale rows are explained by re-running)
+    fm = None if flush_mask is None else np.asarray(flush_mask).reshape(q.shape[0], -1)
+    res.rerun = (q, k, v, g, beta, np.asarray(S0), fm)
+    return res
 
 
 # ---------------------------------------------------------------------------------------------
@@ -157,14 +169,59 @@ def rel_l2(a, b) -> float:
 # ---------------------------------------------------------------------------------------------
 O_TOL = 2e-3
 FLIP_FRAC = 1e-3
+# Scales: the largest scale error measured over every parity case is about 1e-5 of the row's
+# largest scale (the fp32 materialisation sums up to W + r terms in another order than the
+# oracle), so a 1e-5 bar would sit at the measured edge; 1e-4 keeps a 10x margin. Compensator
+# columns are single fp32 entries of the materialised state: measured <= 1.5e-7 rel-L2, bar 1e-5.
 SCALE_TOL = 1e-4
-COMP_TOL = 1e-4
-# Both sides round each buffered write u to bf16 from their own w (fp64 in the oracle, fp32 on
-# the GPU); when w lies within rounding noise of a bf16 rounding boundary the two roundings land
-# one bf16 ulp (2^-8 relative) apart, and the rows that pair touches move by up to that much.
-# Like a 1-LSB code flip this is a valid alternative result: allowed on <= FLIP_FRAC of the
-# compared rows (at least one), never beyond one bf16 ulp.
+COMP_TOL = 1e-5
+# Both sides round each buffered write u to the buffer dtype from their own w (fp64 in the
+# oracle, fp32 on the GPU). A u whose unrounded value lies within the GPU's fp32 noise of a
+# rounding midpoint may land on either neighbour, and the later values of its state row follow
+# (a valid alternative result, like a 1-LSB code flip). A row whose scale misses SCALE_TOL is
+# accepted only when it is explained: some step's unrounded oracle u of that row lies within
+# U_MIDPOINT_NOISE quanta of a midpoint, and the oracle re-run with that one entry rounded to
+# its other neighbour reproduces the GPU's scale row within SCALE_TOL. Explained rows stay
+# within one bf16 ulp (SCALE_TOL_ROUNDING) and on at most FLIP_FRAC of the compared rows.
 SCALE_TOL_ROUNDING = 2.0 ** -8
+U_MIDPOINT_NOISE = 2.0 ** -8   # distance to a midpoint, in quanta of the buffer format
+EXPLAIN_CANDIDATES = 8         # the closest candidate entries tried per loose row
+
+
+def _midpoint_distance(u: np.ndarray, buf: str) -> np.ndarray:
+    """|u / q - (floor(u / q) + 1/2)|: distance of u to the midpoint between its two storage
+    neighbours, in quanta q of u's binade (bf16: 2^(e-8), fp32: 2^(e-24))."""
+    bits = 8 if buf == "bf16" else 24
+    _, e = np.frexp(u)
+    q = np.ldexp(1.0, e - bits)
+    f = u / q
+    d = np.abs(f - np.floor(f) - 0.5)
+    return np.where(u == 0, 1.0, d)
+
+
+def explain_loose_row(wl: Workload, res, a: int, v: int, gpu_row: np.ndarray) -> bool:
+    """Whether the GPU's scale row ``gpu_row`` of compared head ``a`` (index into the compared
+    heads), state row ``v``, is the oracle's alternative result of one write-vector entry of
+    that row rounded to its other neighbour (see U_MIDPOINT_NOISE)."""
+    q, k, vv, g, beta, S0, fm = res.rerun
+    one = slice(a, a + 1)
+    args = (q[:, one], k[:, one], vv[:, one], g[:, one], beta[:, one], S0[one],
+            None if fm is None else np.ascontiguousarray(fm[:, one]))
+    base = _o2(wl, *args, want_u_raw=True)
+    u = base.u_raw[:, 0, v]
+    d = _midpoint_distance(u, wl.buf)
+    cands = [t for t in np.argsort(d, kind="stable")[:EXPLAIN_CANDIDATES]
+             if d[t] <= U_MIDPOINT_NOISE]
+    T = q.shape[0]
+    for t in cands:
+        flip = np.zeros((T, 1, wl.D), np.uint8)
+        flip[t, 0, v] = 1
+        alt = _o2(wl, *args, u_flip=flip)
+        ref = alt.scales[0, v]
+        den = max(float(np.abs(ref).max()), 1e-30)
+        if float(np.abs(gpu_row - ref).max()) / den <= SCALE_TOL:
+            return True
+    return False
 
 
 @dataclass
@@ -175,6 +232,7 @@ class Parity:
     max_code_diff: int
     scale_rel: float
     scale_loose_rows: int
+    scale_unexplained: int
     scale_rows: int
     comp_rel: float
     tie_heads: int
@@ -187,6 +245,7 @@ class Parity:
         assert self.flip_frac <= FLIP_FRAC, self
         assert self.scale_rel <= SCALE_TOL_ROUNDING, self
         assert self.scale_loose_rows <= max(1, int(FLIP_FRAC * self.scale_rows)), self
+        assert self.scale_unexplained == 0, self
         assert self.comp_rel <= COMP_TOL, self
         assert self.tie_heads <= max(1, int(FLIP_FRAC * self.n_heads)), self
         assert self.pos_equal, self
@@ -222,6 +281,14 @@ def compare(wl: Workload, run: GpuRun, heads: np.ndarray, res) -> Parity:
     # compared where every code of the row agrees
     rows_same = (diff.reshape(diff.shape[0], wl.D, -1).max(axis=-1) == 0) if diff.size else diff
     srel_cmp = srel.reshape(srel.shape[0], wl.D, -1)
+    unexplained = 0
+    if np.any(rows_same):
+        loose = rows_same & (srel_cmp.max(axis=-1) > SCALE_TOL)
+        ok_idx = np.flatnonzero(ok)
+        sc_ok = sc[ok].reshape(-1, wl.D, ref.shape[-1])
+        for ai, v in zip(*np.nonzero(loose)):
+            if not explain_loose_row(wl, res, int(ok_idx[ai]), int(v), sc_ok[ai, v]):
+                unexplained += 1
     return Parity(
         o_rel=rel_l2(o_gpu, o_ref), o_rel_unrounded=rel_l2(o_gpu, res.o),
         flip_frac=float((diff > 0).mean()) if diff.size else 0.0,
@@ -229,6 +296,7 @@ def compare(wl: Workload, run: GpuRun, heads: np.ndarray, res) -> Parity:
         scale_rel=float(srel_cmp[rows_same].max()) if np.any(rows_same) else 0.0,
         scale_loose_rows=int((srel_cmp[rows_same].max(axis=-1) > SCALE_TOL).sum())
         if np.any(rows_same) else 0,
+        scale_unexplained=unexplained,
         scale_rows=int(np.sum(rows_same)),
         comp_rel=crel, tie_heads=int((~ok).sum()), n_heads=len(heads),
         pos_equal=bool(np.array_equal(pos, res.pos)))

@@ -1,4 +1,5 @@
-"""Reader for the hand-worked fixtures under tests/golden (format in tests/golden/README.md)."""
+"""Reader for the hand-worked fixtures under tests/golden: one `name = v1 v2 ...` line per array
+(values in row-major order), `#` starts a comment (the derivation and its citation)."""
 import os
 
 import numpy as np

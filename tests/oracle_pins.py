@@ -399,6 +399,78 @@ def pin_storage_roundings(lib):
     close(res.o, exact.o, 2e-2, "storage roundings stay small")
 
 
+def _bracket_bf16(x):
+    """(toward zero, away from zero) bf16 neighbours of fp32 values, from their bit patterns."""
+    b = np.asarray(x, np.float32).view(np.uint32)
+    t = (b & np.uint32(0xFFFF0000))
+    up = t + np.uint32(0x10000)
+    return t.view(np.float32).astype(np.float64), up.view(np.float32).astype(np.float64)
+
+
+def pin_round_other(lib):
+    """The alternative rounding of a value is the other storage neighbour: together with the
+    rounding it brackets the value (bf16 from fp32 bit patterns, single from numpy's nextafter);
+    representable values have no other side."""
+    rng = np.random.default_rng(17)
+    x = (rng.standard_normal(3000) * 10.0 ** rng.uniform(-20, 20, 3000)).astype(np.float32)
+    x = x[(x.view(np.uint32) & np.uint32(0xFFFF)) != 0]          # not bf16-representable
+    t, up = _bracket_bf16(x)
+    r = np.array([lib.orc_round_bf16(float(v)) for v in x])
+    o = np.array([lib.orc_round_other(oracle.ROUND_BF16, float(v)) for v in x])
+    assert np.array_equal(np.minimum(np.abs(r), np.abs(o)), np.abs(t))
+    assert np.array_equal(np.maximum(np.abs(r), np.abs(o)), np.abs(up))
+    assert np.all(np.sign(o) == np.sign(x))
+    assert lib.orc_round_other(oracle.ROUND_BF16, 1 + 2.0**-8 + 2.0**-12) == 1.0
+    assert lib.orc_round_other(oracle.ROUND_BF16, 1.5) == 1.5
+    y = rng.standard_normal(2000) * 10.0 ** rng.uniform(-20, 20, 2000)
+    y = y[y.astype(np.float32).astype(np.float64) != y]
+    lo = np.nextafter(y.astype(np.float32), np.float32(0)).astype(np.float64)
+    lo = np.where(np.abs(lo) > np.abs(y), np.nextafter(lo.astype(np.float32), np.float32(0)), lo)
+    lo = np.where(np.abs(y.astype(np.float32).astype(np.float64)) < np.abs(y),
+                  y.astype(np.float32).astype(np.float64), lo)
+    hi = np.nextafter(lo.astype(np.float32), np.sign(y).astype(np.float32) * np.inf).astype(
+        np.float64)
+    o32 = np.array([lib.orc_round_other(oracle.ROUND_F32, float(v)) for v in y])
+    r32 = y.astype(np.float32).astype(np.float64)
+    assert np.array_equal(np.minimum(np.abs(r32), np.abs(o32)), np.abs(lo))
+    assert np.array_equal(np.maximum(np.abs(r32), np.abs(o32)), np.abs(hi))
+
+
+def pin_write_vectors_before_rounding(lib):
+    """The exported write vectors are u_t = beta_t (v_t - S_{t-1} Diag(a_t) k_t) before their
+    storage rounding, with S_{t-1} the logical state materialised after the previous step; the
+    stored ones are their bf16 roundings, and a flipped entry is stored as its other neighbour
+    while every earlier step stays as it was."""
+    T, nh, D, W = 7, 3, 16, 16
+    for gate in ("scalar", "diag"):
+        q, k, v, g, beta = rand_inputs(61, T, nh, D, gate)
+        S0 = np.random.default_rng(2).standard_normal((nh, D, D)).astype(np.float32)
+        kw = dict(W=W, r=1, S0=S0, round_storage=True, buf_round="bf16", lib=lib)
+        res = oracle.o2_run(q, k, v, g, beta, want_u_raw=True, **kw)
+        prev = oracle.o2_run(q[:-1], k[:-1], v[:-1], g[:-1], beta[:-1], **kw)
+        # the cumulative log-gates are stored in fp32 (round_storage), so the last step's
+        # decay is e^{L_T - L_{T-1}} of the rounded sums
+        gg = g[..., None] * np.ones((T, nh, D)) if gate == "scalar" else g
+        Lc = np.zeros((T + 1, nh, D))
+        for t in range(T):
+            Lc[t + 1] = (Lc[t] + gg[t]).astype(np.float32)
+        a = np.exp(Lc[T] - Lc[T - 1])
+        w = np.einsum("hij,hj->hi", prev.S, a * k[-1])
+        u = beta[-1][:, None] * (v[-1] - w)
+        close(res.u_raw[-1], u, 1e-12, "write vector from the materialised state")
+        ur = res.u_raw.transpose(1, 0, 2)                         # [nh][T][D]
+        assert np.mean(ur == torch.from_numpy(ur).to(torch.bfloat16).double().numpy()) < 0.05
+        assert np.array_equal(res.bu[:, :T], torch.from_numpy(ur).to(torch.bfloat16).double()
+                              .numpy())
+        flip = np.zeros((T, nh, D), np.uint8)
+        flip[4, 1, 5] = 1
+        alt = oracle.o2_run(q, k, v, g, beta, want_u_raw=True, u_flip=flip, **kw)
+        assert np.array_equal(alt.u_raw[:5], res.u_raw[:5])
+        assert alt.bu[1, 4, 5] == lib.orc_round_other(oracle.ROUND_BF16, res.u_raw[4, 1, 5])
+        assert alt.bu[1, 4, 5] != res.bu[1, 4, 5]
+        assert np.array_equal(alt.bu[[0, 2]], res.bu[[0, 2]])
+
+
 # ---------------------------------------------------------------------------------------------
 # Residual smoothing (reading: per-column power-of-two factors m_j = 2^floor(E_j / 2))
 # ---------------------------------------------------------------------------------------------
@@ -643,6 +715,8 @@ PINS = [
     pin_literal_equals_buffered_quantized,
     pin_compensator_decomposition,
     pin_storage_roundings,
+    pin_round_other,
+    pin_write_vectors_before_rounding,
     pin_golden_smoothing,
     pin_smooth_exponent,
     pin_smoothing_properties,

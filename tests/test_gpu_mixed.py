@@ -1,13 +1,20 @@
-"""Mixed per-head bit widths in one launch (GDN_FMT_MIXED): every head must come out exactly as
-it does in a launch whose whole state has that head's format -- outputs, codes, scales,
-compensators and pos bit-identical through decode steps with window flushes, a forced ragged
-flush and materialisation. (Each uniform format is checked against the oracle elsewhere.)"""
+"""Mixed per-head bit widths in one launch (GDN_FMT_MIXED), two ways:
+  - against the oracle: the heads of each format, read out of the mixed state, against the
+    oracle's buffered-window form run in that head's format (outputs, codes, scales,
+    compensators, pos), with the acceptance bars of the uniform formats;
+  - against the uniform launches: every head must come out exactly as it does in a launch whose
+    whole state has that head's format -- outputs, codes, scales, compensators and pos
+    bit-identical through decode steps with window flushes, a forced ragged flush and
+    materialisation."""
+from types import SimpleNamespace
+
 import numpy as np
 import pytest
 import torch
 
 import bit_recurrent_state_gdn_b200 as gdn
-from gdn_harness import gpu_warmup
+from gdn_harness import (GpuRun, compare, gpu_warmup, oracle_initial_state, oracle_run,
+                         sample_heads)
 from workloads import WORKLOADS, decode_inputs
 
 pytestmark = pytest.mark.gpu
@@ -52,6 +59,41 @@ def _head_views(wl, st, fmt, n):
     code_slot = D * D // 2 if fmt == "int4_g32" else D * D
     scale_slot = D * (D // 32) if fmt in ("int4_g32", "mixed") else D
     return st.codes.view(n, code_slot), st.scales.view(n, scale_slot)
+
+
+def _format_view(wl, mst, mo, fmt, heads):
+    """The heads ``heads`` of a mixed state and its outputs, laid out as a uniform state of
+    ``fmt`` holding only those heads (the harness reads it like any other run)."""
+    n, D, T = wl.heads, wl.D, mo.shape[0]
+    idx = torch.as_tensor(heads, device="cuda")
+    cb = D * D // 2 if fmt == "int4_g32" else D * D
+    sb = D * (D // 32) if fmt == "int4_g32" else D
+    rp = (wl.r + 3) // 4 * 4
+    st = SimpleNamespace(
+        codes=mst.codes.view(n, D * D)[idx, :cb].contiguous().view(-1),
+        scales=mst.scales.view(n, D * (D // 32))[idx, :sb].contiguous().view(-1),
+        comp_idx=mst.comp_idx.view(n, max(rp, 1))[idx].contiguous().view(-1) if wl.r else
+        mst.comp_idx,
+        comp_u=mst.comp_u.view(n, -1)[idx].contiguous().view(-1) if wl.r else mst.comp_u,
+        pos=mst.pos[idx].contiguous())
+    o = mo.view(T, n, D)[:, idx].contiguous().view(T, 1, len(heads), D)
+    return GpuRun(o, st, None, None)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_mixed_launch_against_the_oracle(name):
+    wl = CASES[name]
+    fmts = np.array(_pattern(wl.heads, wl.seed))
+    inp = decode_inputs(wl, "cuda")
+    _, mst, mo, _ = _run(wl, "mixed", gpu_warmup(wl), inp, head_fmt=list(fmts))
+    pick = set(sample_heads(wl, 64, seed=7).tolist()) if wl.heads > 64 else None
+    for f in ("int8", "int4_g32"):
+        heads = np.array([h for h in np.flatnonzero(fmts == f) if pick is None or h in pick])
+        wf = wl.with_(fmt=f)
+        res = oracle_run(wf, heads, inp, oracle_initial_state(wf, heads))
+        p = compare(wf, _format_view(wl, mst, mo, f, heads), np.arange(len(heads)), res)
+        print(name, f, len(heads), p)
+        p.check()
 
 
 @pytest.mark.parametrize("name", list(CASES))

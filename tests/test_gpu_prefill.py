@@ -19,7 +19,12 @@ pytestmark = pytest.mark.gpu
 
 MID = WORKLOADS["gdn-mid"]
 KDA = WORKLOADS["kda"].with_(r=0)
-S_TOL = 2e-3  # final state, rel-L2 (the outputs' bar)
+# Final state: the prefill's fp32 state feeds gdn_state_quantize, so its bar is set by what the
+# kernels achieve (a few 1e-6 rel-L2), not by the outputs' bf16 bar: rel-L2 over the compared
+# heads, and entry by entry the largest error of a state row relative to that row's largest
+# entry (an error big enough to move an int8 code, 1/254 of the row's absmax, fails it).
+S_TOL = 5e-5
+S_ELEM_TOL = 5e-4
 
 CASES = {
     "one-chunk": MID.with_(name="pf-64", B=1, H=3, T=64, warmup=32),
@@ -65,7 +70,15 @@ def compare(wl, inp, o, S, heads):
     h = torch.as_tensor(heads, device="cuda")
     o_gpu = o.view(-1, L, wl.D)[h].permute(1, 0, 2).double().cpu().numpy()
     S_gpu = S.view(-1, wl.D, wl.D)[h].double().cpu().numpy()
-    return (rel_l2(o_gpu, round_act(o_ref, "bf16")) if L else 0.0), rel_l2(S_gpu, S_ref)
+    row_max = np.maximum(np.abs(S_ref).max(axis=-1, keepdims=True), 1e-30)
+    s_elem = float((np.abs(S_gpu - S_ref) / row_max).max()) if S_ref.size else 0.0
+    return ((rel_l2(o_gpu, round_act(o_ref, "bf16")) if L else 0.0), rel_l2(S_gpu, S_ref),
+            s_elem)
+
+
+def check(m):
+    o_rel, s_rel, s_elem = m
+    assert o_rel <= O_TOL and s_rel <= S_TOL and s_elem <= S_ELEM_TOL, m
 
 
 @pytest.mark.parametrize("name", list(CASES))
@@ -73,9 +86,9 @@ def test_prefill_parity(name):
     wl = CASES[name]
     inp = decode_inputs(wl, "cuda")
     o, S = pf_run(wl, inp, gpu_warmup(wl))
-    o_rel, s_rel = compare(wl, inp, o, S, np.arange(wl.heads))
-    print(name, o_rel, s_rel)
-    assert o_rel <= O_TOL and s_rel <= S_TOL, (o_rel, s_rel)
+    m = compare(wl, inp, o, S, np.arange(wl.heads))
+    print(name, m)
+    check(m)
 
 
 @pytest.mark.parametrize("name", ["ragged", "kda-ragged"])
@@ -84,8 +97,9 @@ def test_prefill_split_over_calls_carries_the_state(name):
     inp = decode_inputs(wl, "cuda")
     S0 = gpu_warmup(wl)
     o, S = pf_run(wl, inp, S0, cuts=[0, 5, 70, 131, 200])  # chunk boundaries inside the calls
-    o_rel, s_rel = compare(wl, inp, o, S, np.arange(wl.heads))
-    assert o_rel <= O_TOL and s_rel <= S_TOL, (o_rel, s_rel)
+    m = compare(wl, inp, o, S, np.arange(wl.heads))
+    print(name, m)
+    check(m)
 
 
 def test_kda_prefill_strong_decays():
@@ -96,10 +110,10 @@ def test_kda_prefill_strong_decays():
     inp["g"] = (3.0 * inp["g"]).clamp_min(-10.0)
     inp["g"][5:13, :, :, :7] = -10.0  # a run of 8 tokens at the floor on a few channels
     o, S = pf_run(wl, inp, gpu_warmup(wl))
-    o_rel, s_rel = compare(wl, inp, o, S, np.arange(wl.heads))
-    print("strong", o_rel, s_rel)
-    assert np.isfinite(o_rel) and np.isfinite(s_rel)
-    assert o_rel <= O_TOL and s_rel <= S_TOL, (o_rel, s_rel)
+    m = compare(wl, inp, o, S, np.arange(wl.heads))
+    print("strong", m)
+    assert np.all(np.isfinite(m))
+    check(m)
 
 
 @pytest.mark.parametrize("base", ["gdn", "kda"])
@@ -108,9 +122,9 @@ def test_prefill_batch_sampled_heads(base):
     inp = decode_inputs(wl, "cuda")
     o, S = pf_run(wl, inp, gpu_warmup(wl))
     heads = sample_heads(wl, 24, seed=3)
-    o_rel, s_rel = compare(wl, inp, o, S, heads)
-    print("batch", o_rel, s_rel)
-    assert o_rel <= O_TOL and s_rel <= S_TOL, (o_rel, s_rel)
+    m = compare(wl, inp, o, S, heads)
+    print("batch", m)
+    check(m)
 
 
 @pytest.mark.parametrize("name", ["one-chunk", "kda-one-chunk"])
@@ -163,6 +177,6 @@ def test_prefill_full_size_sampled_heads(name):
     o, S = pf_run(wl, inp, torch.zeros((wl.B, wl.H, wl.D, wl.D), device="cuda"))
     assert bool(torch.isfinite(S).all())
     heads = sample_heads(wl, 4, seed=wl.seed)
-    o_rel, s_rel = compare(wl, inp, o, S, heads)
-    print(name, o_rel, s_rel)
-    assert o_rel <= O_TOL and s_rel <= S_TOL, (o_rel, s_rel)
+    m = compare(wl, inp, o, S, heads)
+    print(name, m)
+    check(m)

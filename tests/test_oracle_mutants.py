@@ -124,6 +124,21 @@ MUTANTS = [
     ("e4m3: subnormal spacing too fine",
      "if (qexp < -9) qexp = -9;",
      "if (qexp < -10) qexp = -10;"),
+    ("alternative rounding: the rounding itself",
+     "return round_to(mode, x) == lo ? hi : lo;",
+     "return round_to(mode, x);"),
+    ("alternative rounding: one quantum too far",
+     "const double lo = floor(x / quantum) * quantum, hi = lo + quantum;",
+     "const double lo = floor(x / quantum) * quantum - quantum, hi = lo + 3 * quantum;"),
+    ("write vectors exported after their rounding",
+     "        if (u_raw) u_raw[i] = u;\n        if (c->round_storage)\n"
+     "            u = (u_flip && u_flip[i]) ? orc_round_other(c->buf_round, u) : round_to(c->buf_round, u);",
+     "        if (c->round_storage)\n"
+     "            u = (u_flip && u_flip[i]) ? orc_round_other(c->buf_round, u) : round_to(c->buf_round, u);\n"
+     "        if (u_raw) u_raw[i] = u;"),
+    ("flipped write vector rounded as usual",
+     "u = (u_flip && u_flip[i]) ? orc_round_other",
+     "u = (0) ? orc_round_other"),
     ("FP8 vector: scale for a largest value of 240",
      "double s = m / 448.0;",
      "double s = m / 240.0;"),

@@ -229,12 +229,17 @@ __device__ __forceinline__ void report(int32_t* status, int bit) {
 // the step's q, k, v (and diagonal g), copied into a stage with bulk async copies completing on
 // the stage's mbarrier. Issued by one thread. An out-of-range P arms the barrier with no copies.
 // ------------------------------------------------------------------------------------------
+// Zero rows for the stages' write-vector regions (read by bulk copies; never written).
+constexpr int kZeroRowBytes = 4096;
+static __device__ __align__(128) uint8_t g_zero_rows[kZeroRowBytes];
+
 template <class C>
 __device__ __forceinline__ void stage_issue(const WinArgs& a, const WinLayout& L, uint8_t* st,
                                             uint64_t* bar, int head, int P, bool with_io,
-                                            int part = -1) {
+                                            int part = -1, int zrows = 0) {
   // part -1: every copy; part 0: codes, scales, q, k; part 1: the rest (two issuers, each
-  // arriving once on a barrier that expects two arrivals)
+  // arriving once on a barrier that expects two arrivals). zrows > 0 (with part != 0) also
+  // copies zeros over the write-vector rows P .. P + zrows - 1 of the stage.
   using Act = typename C::Act;
   using Buf = typename C::Buf;
   constexpr int D = C::D;
@@ -254,6 +259,7 @@ __device__ __forceinline__ void stage_issue(const WinArgs& a, const WinLayout& L
     if (P > 0) bytes += (uint32_t)P * D * (sizeof(Act) + sizeof(Buf)) + lbytes;
     if (r > 0) bytes += 4u * rp + 4u * r * D;
     if (with_io) bytes += D * sizeof(Act) + (C::DIAG ? 4u * D : 0u);
+    bytes += (uint32_t)zrows * D * sizeof(Buf);
   }
   mbar_arrive_expect_tx(bar, bytes);
   if (p0) {
@@ -282,6 +288,9 @@ __device__ __forceinline__ void stage_issue(const WinArgs& a, const WinLayout& L
       bulk_g2s(st + L.v, static_cast<const Act*>(a.v) + (size_t)head * D, D * sizeof(Act), bar);
       if constexpr (C::DIAG) bulk_g2s(st + L.g, a.g + (size_t)head * D, 4u * D, bar);
     }
+    if (zrows > 0)
+      bulk_g2s(st + L.bu + (uint32_t)P * D * sizeof(Buf), g_zero_rows,
+               (uint32_t)zrows * D * sizeof(Buf), bar);
   }
 }
 
@@ -856,7 +865,10 @@ __global__ void __launch_bounds__(kStepThreads, 2)
   float* hg = reinterpret_cast<float*>(hpos + per_cta);
   float* hb = hg + per_cta;
   int* pmax = reinterpret_cast<int*>(sm + L0.bars + 64);  // after the stage barriers (<= 4)
+  // per stage: the furthest window position among the heads staged there so far (rows below it
+  // may hold another head's write vectors)
   if (tid == 0) *pmax = 0;
+  if (tid < kMaxStages) pmax[1 + tid] = 0;  // the stages' high-water marks (below)
   csync();
   int mp = 0;
   for (int i = tid; i < nh; i += C::NT) {
@@ -881,18 +893,21 @@ __global__ void __launch_bounds__(kStepThreads, 2)
                           (int)win_layout_mix<C, MIX>(a.W, a.r, 1, per_cta, cap, !mma).stage_bytes);
   const WinLayout L = win_layout_mix<C, MIX>(a.W, a.r, nstages, per_cta, cap, !mma);
   // a head's stage copies and step in its own format (both fit the mixed layout)
-  auto issue = [&](uint8_t* st, uint64_t* bar, int head, int P) {
+  auto issue = [&](uint8_t* st, uint64_t* bar, int head, int P, int zrows) {
     if constexpr (MIX) {
       if (head_is_int4(a, head)) {
-        stage_issue<Int4Of<C>>(a, L, st, bar, head, P, true);
+        stage_issue<Int4Of<C>>(a, L, st, bar, head, P, true, -1, zrows);
         return;
       }
     }
-    stage_issue<C>(a, L, st, bar, head, P, true);
+    stage_issue<C>(a, L, st, bar, head, P, true, -1, zrows);
   };
-  // every stage's write-vector rows start at zero (tensor-core path): a row past a head's pairs
-  // then holds zeros or an earlier head's finite write vector, and meets a zero coefficient in
-  // the buffer product; the zeros are ordered before the stage copies by the proxy fence
+  // Every stage's write-vector rows start at zero (tensor-core path). The buffer product reads a
+  // head's rows up to its position rounded up to 16, and the rows past its pairs meet zero
+  // coefficients, so they must hold finite values: zeros, or -- when an earlier head staged
+  // there had a further position (ragged windows) -- that head's write vectors, which
+  // `restage` zeroes first, so that one head's non-finite values never reach another head's
+  // results. The zeros are ordered before the stage copies by the proxy fence.
   if (mma) {
     const int n16 = cap * C::D * (int)sizeof(typename C::Buf) / 16;
     for (int s = 0; s < nstages; ++s) {
@@ -907,18 +922,28 @@ __global__ void __launch_bounds__(kStepThreads, 2)
     fence_barrier_init();
   }
   csync();
+  // Restage stage s with head index `hn` (one thread, once the stage is free). With ragged
+  // windows the stage may hold another head's write vectors in [P, P rounded up to 16): the
+  // copies then also bring zeros over them.
+  auto restage = [&](int s, int hn) {
+    int* hwm = reinterpret_cast<int*>(sm + 68) + s;  // after *pmax
+    const int P = hpos[hn];
+    int zrows = 0;
+    if (P >= 0 && P < a.W) {
+      const int m = *hwm;
+      zrows = max(0, min((P + 15) & ~15, m) - P);
+      *hwm = max(m, P + (P + 1 == a.W));  // a flush writes row P into the stage
+    }
+    issue(sm + L.stage0 + s * L.stage_bytes, &bars[s], h0 + hn, P, mma ? zrows : 0);
+  };
   if (tid == 0)
-    for (int s = 0; s < nstages && s < nh; ++s)
-      issue(sm + L.stage0 + s * L.stage_bytes, &bars[s], h0 + s, hpos[s]);
+    for (int s = 0; s < nstages && s < nh; ++s) restage(s, s);
   if (!stage_wait(a, &bars[0], 0u)) return;
   for (int n = 0; n < nh; ++n) {
-    // refill the stage head n - 1 left; the issuer is lane 0 of the last warp, which has the
-    // least work early in a head (the pair-coefficient tiles go to warps 4, 5, ... in order)
-    if (nstages > 1 && tid == kStepIssuer && n > 0 && n - 1 + nstages < nh) {
-      const int sp = (n - 1) % nstages;
-      issue(sm + L.stage0 + sp * L.stage_bytes, &bars[sp], h0 + n - 1 + nstages,
-            hpos[n - 1 + nstages]);
-    }
+    // refill the stage head n - 1 left; the issuer is the last warp, which has the least work
+    // early in a head (the pair-coefficient tiles go to warps 4, 5, ... in order)
+    if (nstages > 1 && tid == kStepIssuer && n > 0 && n - 1 + nstages < nh)
+      restage((n - 1) % nstages, n - 1 + nstages);
     uint8_t* st = sm + L.stage0 + (n % nstages) * L.stage_bytes;
     const int P = hpos[n];
     if (P >= 0 && P < a.W) {
@@ -937,7 +962,7 @@ __global__ void __launch_bounds__(kStepThreads, 2)
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
     if (nstages == 1) {  // a single stage is refilled only once this head is done with it
       csync();
-      if (tid == kStepIssuer && n + 1 < nh) issue(st, &bars[0], h0 + n + 1, hpos[n + 1]);
+      if (tid == kStepIssuer && n + 1 < nh) restage(0, n + 1);
     }
     // one barrier ends the head (stage and scratch free) and agrees on the next head's copies
     int timed_out = 0;

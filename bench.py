@@ -432,6 +432,16 @@ def main():
                       cpu=not args.no_cpu and world == 1 and rank == 0)
             for f in ("int4_g32", "int8")}
 
+    # ---- the other decode workloads, each on its own inputs, and int4 at the serving size ----
+    if not args.no_baselines and world == 1 and wl0.name == "gdn-serving":
+        cpu = not args.no_cpu and rank == 0
+        line["workloads"] = {
+            "int4-serving": decode_leg(wl.with_(name="int4-serving", fmt="int4_g32"), dev, peak,
+                                       cpu=False, inp=inp, S0=S0, o=o)}
+        for name in ("kda", "gdn-mid", "gdn-long-int4"):
+            line["workloads"][name] = decode_leg(WORKLOADS[name], dev, peak, cpu=cpu)
+            torch.cuda.empty_cache()
+
     # ---- chunkwise prefill of a prompt batch (its own workload) ----------------------------
     if not args.no_baselines and world == 1:
         line["prefill"] = prefill_leg(args, dev)
@@ -475,6 +485,87 @@ def main():
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+L2_BYTES = 126 * 2**20
+LEG_PROFILES = {"kda": ("window_step_kda.md", "traffic_bytes_per_launch")}
+
+
+def warm_states(wl, dev):
+    """fp32 initial states: the workload's warm-up tokens through the fp32-state baseline
+    kernel (zero states without warm-up)."""
+    import torch
+
+    import bit_recurrent_state_gdn_b200 as gdn
+
+    S0 = torch.zeros((wl.B, wl.H, wl.D, wl.D), dtype=torch.float32, device=dev)
+    cfg = gdn.make_config(wl.B, wl.H, wl.D, gate=wl.gate, fmt="fp32", act=wl.act)
+    scales = outlier_scales(wl, dev)
+    o = torch.empty((wl.B, wl.H, wl.D), dtype=torch_dtype(wl.act), device=dev)
+    for t in range(wl.warmup):
+        s = step_inputs(wl, "warmup", t, dev, scales)
+        gdn.gdn_baseline_step(cfg, S0, s.q, s.k, s.v, s.g, s.beta, o)
+    return S0
+
+
+def decode_leg(wl, dev, peak, cpu: bool, inp=None, S0=None, o=None, cpu_heads: int = 256):
+    """One decode workload on its own: its states quantized (untimed), then its T decode launches
+    timed with CUDA events; the roofline of the average launch from the workload's algorithmic
+    bytes; with cpu, the oracle on a bounded sample of its heads."""
+    import numpy as np
+    import torch
+
+    import bit_recurrent_state_gdn_b200 as gdn
+
+    if inp is None:
+        inp = decode_inputs(wl, dev)
+        S0 = warm_states(wl, dev)
+        o = torch.empty_like(inp["q"])
+    cfg = gdn.make_config(wl.B, wl.H, wl.D, wl.W, wl.r, wl.gate, wl.fmt, wl.act, wl.buf)
+    st = gdn.GdnState.allocate(cfg, dev)
+    gdn.gdn_state_quantize(cfg, S0, st)
+    n0 = min(4, wl.T)
+    gdn.gdn_decode_window_steps(cfg, st, inp["q"][:n0], inp["k"][:n0], inp["v"][:n0],
+                                inp["g"][:n0], inp["beta"][:n0], o[:n0])
+    gdn.gdn_state_quantize(cfg, S0, st)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    gdn.gdn_decode_window_steps(cfg, st, inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], o)
+    e1.record()
+    torch.cuda.synchronize()
+    if int(st.status[0].item()) != 0:
+        raise RuntimeError(f"{wl.name}: device status word set")
+    ms = e0.elapsed_time(e1)
+    per_launch = avg_step_bytes(wl) * wl.heads
+    avg_s = ms / 1e3 / wl.T
+    gbs = per_launch / avg_s / 1e9
+    resident = per_launch < L2_BYTES
+    traffic, src = None, None
+    if wl.name in LEG_PROFILES:
+        f, key = LEG_PROFILES[wl.name]
+        traffic, src = profiled_traffic(os.path.join(ROOT, "profiles", f), KERNEL_SOURCES, key)
+    out = {"value": wl.heads * wl.T / (ms / 1e3), "unit": UNIT, "ms_per_run": ms,
+           "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "D": wl.D, "T": wl.T,
+                      "W": wl.W, "r": wl.r, "gate": wl.gate, "state": wl.fmt, "act": wl.act},
+           "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                        "frac": gbs / peak, "traffic": traffic, "traffic_source": src,
+                        "algorithmic_bytes_per_launch": per_launch,
+                        "avg_launch_us": avg_s * 1e6,
+                        "kernel": "window_step_kernel (decode step + fused window flush)"}}
+    if resident:
+        out["roofline"]["note"] = (
+            "effective GB/s: one launch moves %.1f MB, under the 126 MB L2, so the state stays "
+            "L2-resident between launches and the launch is latency-bound" % (per_launch / 1e6))
+    if cpu:
+        n_seq = max(1, min(wl.B, cpu_heads // wl.H))
+        d, S0c = oracle_sample(wl, inp, n_seq, dev)
+        hs, dt, cores = time_oracle(wl, d["q"], d["k"], d["v"], d["g"], d["beta"], S0c)
+        out["cpu_baseline"] = {"value": hs, "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": f"{n_seq * wl.H} heads (sequences 0..{n_seq - 1}) x "
+                                         f"{wl.T} steps of the same inputs, {dt:.1f} s"}
+    del st
+    return out
 
 
 def mixed_leg(wl, S0, inp, o, peak):
@@ -687,10 +778,17 @@ def e2e(args, wl, cfg, inp, S0, state, world, dev):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
     ms = max_over_ranks(ms, world, dev)
-    h2d = hS0.numel() * 4 + sum(t.numel() * t.element_size() for t in host.values())
+    state_up = hS0.numel() * 4
+    h2d = state_up + sum(t.numel() * t.element_size() for t in host.values())
     d2h = ho.numel() * ho.element_size()
     return {"value": whole_job_rate(wl.heads * wl.T * n, world, ms), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
+            "link_gbs": (h2d + d2h) * n / (ms / 1e3) / 1e9,
+            "state_upload_bytes_per_step": state_up,
+            "state_upload_share": state_up / (h2d + d2h),
+            "note": "each step uploads the fp32 initial states (to quantize them) and every "
+                    "decode token's q / k / v / g / beta, and reads back every output: the "
+                    "host link, not the kernels, bounds this figure",
             "api": "gdn_decode_window_steps_host (pinned host buffers, copies pipelined)"}
 
 

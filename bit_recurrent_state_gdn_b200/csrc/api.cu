@@ -499,21 +499,13 @@ gdn_status gdn_decode_window_steps_host_fixed(const gdn_config* cfg, const gdn_s
                 "gdn_decode_window_steps_host_fixed: one staging slot needs %zu bytes for %lld "
                 "heads, the fixed staging array holds %zu; use gdn_decode_window_steps_host",
                 sl.bytes, (long long)heads_of(cfg), (size_t)GDN_FIXED_STAGING_BYTES);
-  // the array's address on the current device, looked up once per device
-  constexpr int kMaxDevices = 64;
-  static void* fixed_addr[kMaxDevices] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "gdn_decode_window_steps_host_fixed: cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices)
-    return fail(GDN_ERR_UNSUPPORTED, "device %d beyond the %d this build tracks", dev, kMaxDevices);
-  void* base_v = __atomic_load_n(&fixed_addr[dev], __ATOMIC_ACQUIRE);
-  if (!base_v) {
-    e = cudaGetSymbolAddress(&base_v, g_fixed_staging);
-    if (e != cudaSuccess)
-      return cuda_fail(e, "gdn_decode_window_steps_host_fixed: cudaGetSymbolAddress");
-    __atomic_store_n(&fixed_addr[dev], base_v, __ATOMIC_RELEASE);
-  }
+  // The array's device address in the current device's context, looked up on every call (a
+  // host-side use of the symbol itself is not a device address). Not cached: after a
+  // cudaDeviceReset the context and the module are created anew and the array may move.
+  void* base_v = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&base_v, g_fixed_staging);
+  if (e != cudaSuccess)
+    return cuda_fail(e, "gdn_decode_window_steps_host_fixed: cudaGetSymbolAddress");
   uint8_t* base = static_cast<uint8_t*>(base_v);
   const size_t H = (size_t)heads_of(cfg), D = (size_t)cfg->d_k;
   const size_t act_step = H * D * act_size(cfg);

@@ -160,8 +160,11 @@ typedef struct {
     size_t smooth_exp;
 } gdn_sizes;
 
-/* Checks cfg and fills *out. Host-only: touches no device. Errors: GDN_ERR_INVALID_ARG for a
- * null argument or bad field, GDN_ERR_UNSUPPORTED for a configuration this build lacks. */
+/* Checks cfg and fills *out. Host-only: touches no device. The buffers are the parts of the
+ * windowed state that "LeapQuant ..." (Abstract) names: the low-bit state frozen for the window
+ * (codes, scales), the window's high-precision buffered updates (buf_k, buf_u, buf_L) and the
+ * compensator tokens (comp_idx, comp_u). Errors: GDN_ERR_INVALID_ARG for a null argument or bad
+ * field, GDN_ERR_UNSUPPORTED for a configuration this build lacks. */
 gdn_status gdn_state_sizes(const gdn_config* cfg, gdn_sizes* out);
 
 /*
@@ -245,6 +248,9 @@ gdn_status gdn_decode_window_steps_host(const gdn_config* cfg, const gdn_state* 
  *     `stream` has finished. Pinned host memory is needed for the copies to be asynchronous.
  *   - All calls on one device share the array: two calls whose work overlaps in time (on
  *     different streams, or from different host threads) race on it. Serialise them.
+ *   - Every call looks up the array's address in the current device's context
+ *     (cudaGetSymbolAddress; GDN_ERR_CUDA if that fails), so a call after cudaDeviceReset uses
+ *     the array of the new context.
  * Arguments, layouts and errors otherwise as gdn_decode_window_steps_host.
  */
 #define GDN_FIXED_STAGING_BYTES ((size_t)16 << 20)
@@ -255,7 +261,9 @@ gdn_status gdn_decode_window_steps_host_fixed(const gdn_config* cfg, const gdn_s
                                               gdn_stream_t stream);
 
 /*
- * Forced window flush: for every head whose sequence is selected (seq_mask == NULL selects all;
+ * Forced window flush ("LeapQuant ..." Abstract: the state is quantized once, at its window's
+ * end; this runs that window-end operation early): for every head whose sequence is selected
+ * (seq_mask == NULL selects all;
  * otherwise device int32 [B], nonzero = selected) and whose pos > 0, materialise the logical
  * state, rebuild compensators and codes as gdn_state_quantize does, and set pos = 0. Heads with
  * pos == 0 are left untouched (their logical state is already the frozen one). Used to hand a
@@ -266,13 +274,17 @@ gdn_status gdn_window_flush(const gdn_config* cfg, const gdn_state* state,
 
 /*
  * Writes the logical state of every head (formula above) as fp32 [B][H][D][D] to S, without
- * changing the state.
+ * changing the state: the materialisation that "LeapQuant ..." (Abstract) performs at a
+ * window's end, before the requantisation, i.e. the frozen low-bit state carried through the
+ * window plus the buffered updates and the compensator tokens.
  */
 gdn_status gdn_state_materialize(const gdn_config* cfg, const gdn_state* state, float* S,
                                  gdn_stream_t stream);
 
 /*
- * Baseline: one plain decode step over a high-precision state (cfg->fmt GDN_FMT_FP32 or
+ * Baseline ("LeapQuant ..." Abstract: its kernel speedups are measured against decode over an
+ * FP32 recurrent state; the bf16 state is the usual half-precision alternative): one plain
+ * decode step over a high-precision state (cfg->fmt GDN_FMT_FP32 or
  * GDN_FMT_BF16; W, r and buf_dtype are ignored). The state S [B][H][D][D] is read once and
  * written once, in place:
  *   w = S (a_t * k_t);  u = beta_t (v_t - w);  S <- S Diag(a_t) + u k_t^T (rounded to nearest

@@ -699,8 +699,10 @@ def prefill_leg(args, dev, name: str = "gdn-prefill", reps: int = 5):
     tf = flops / (t / 1e3) / 1e12
     peak, src = peak_bf16()
     cpu = None if args.no_cpu else prefill_cpu_baseline(wl, inp, dev)
-    kernel = ("prefill_kda_kernel (one CTA per head, two per SM, 16-token chunks)"
-              if wl.gate == "diag" else "prefill_kernel (one CTA per head, 64-token chunks)")
+    kernel = ("prefill_kda_kernel (one CTA per head, two per SM, 16-token chunks, mma.sync)"
+              if wl.gate == "diag" else
+              "prefill_tc_kernel (one CTA per head, 64-token chunks, tcgen05.mma with the state "
+              "in TMEM, TMA-staged tiles)")
     return {"value": wl.heads * L / (t / 1e3), "unit": "head-tokens/s", "ms_per_launch": t,
             "cpu_baseline": cpu,
             "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "L": L, "D": wl.D,
@@ -709,7 +711,8 @@ def prefill_leg(args, dev, name: str = "gdn-prefill", reps: int = 5):
                          "frac": tf / peak, "peak_source": src,
                          "flops_per_launch": flops,
                          "note": "UT-form products at single precision; the kernel issues "
-                                 "up to three times that on mma.sync (hi/lo bf16 splits)"},
+                                 "up to three times that on the tensor cores (hi/lo bf16 "
+                                 "splits)"},
             "kernel": kernel}
 
 

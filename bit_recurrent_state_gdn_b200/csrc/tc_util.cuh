@@ -131,6 +131,69 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       : "memory");
 }
 
+// ---- TMEM <-> registers in the mma.sync accumulator layout (16 lanes x 8 columns per step) ----
+// Shape 16x256b: lane l of the warp holds TMEM lanes base + l / 4 and base + l / 4 + 8, columns
+// 2 (l % 4) and 2 (l % 4) + 1 of each 8-column step: acc[n][0..3] = (row l/4, col 8n + 2(l%4)),
+// (row l/4, +1), (row l/4 + 8, col), (row l/4 + 8, +1), the C fragment of an m16n8 product.
+__device__ __forceinline__ void tmem_st_frag8(uint32_t taddr, const float (&acc)[8][4]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+      "%29, %30, %31, %32};\n" ::"r"(taddr),
+      "f"(acc[0][0]), "f"(acc[0][1]), "f"(acc[0][2]), "f"(acc[0][3]), "f"(acc[1][0]),
+      "f"(acc[1][1]), "f"(acc[1][2]), "f"(acc[1][3]), "f"(acc[2][0]), "f"(acc[2][1]),
+      "f"(acc[2][2]), "f"(acc[2][3]), "f"(acc[3][0]), "f"(acc[3][1]), "f"(acc[3][2]),
+      "f"(acc[3][3]), "f"(acc[4][0]), "f"(acc[4][1]), "f"(acc[4][2]), "f"(acc[4][3]),
+      "f"(acc[5][0]), "f"(acc[5][1]), "f"(acc[5][2]), "f"(acc[5][3]), "f"(acc[6][0]),
+      "f"(acc[6][1]), "f"(acc[6][2]), "f"(acc[6][3]), "f"(acc[7][0]), "f"(acc[7][1]),
+      "f"(acc[7][2]), "f"(acc[7][3])
+      : "memory");
+}
+// Load (waits for completion).
+__device__ __forceinline__ void tmem_ld_frag8(uint32_t taddr, float (&acc)[8][4]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+      "%29, %30, %31}, [%32];\ntcgen05.wait::ld.sync.aligned;\n"
+      : "=f"(acc[0][0]), "=f"(acc[0][1]), "=f"(acc[0][2]), "=f"(acc[0][3]), "=f"(acc[1][0]),
+        "=f"(acc[1][1]), "=f"(acc[1][2]), "=f"(acc[1][3]), "=f"(acc[2][0]), "=f"(acc[2][1]),
+        "=f"(acc[2][2]), "=f"(acc[2][3]), "=f"(acc[3][0]), "=f"(acc[3][1]), "=f"(acc[3][2]),
+        "=f"(acc[3][3]), "=f"(acc[4][0]), "=f"(acc[4][1]), "=f"(acc[4][2]), "=f"(acc[4][3]),
+        "=f"(acc[5][0]), "=f"(acc[5][1]), "=f"(acc[5][2]), "=f"(acc[5][3]), "=f"(acc[6][0]),
+        "=f"(acc[6][1]), "=f"(acc[6][2]), "=f"(acc[6][3]), "=f"(acc[7][0]), "=f"(acc[7][1]),
+        "=f"(acc[7][2]), "=f"(acc[7][3])
+      : "r"(taddr)
+      : "memory");
+}
+// One 8-column step of packed 32-bit values (4 per thread) in the same layout.
+__device__ __forceinline__ void tmem_st_frag1(uint32_t taddr, uint32_t r0, uint32_t r1,
+                                              uint32_t r2, uint32_t r3) {
+  asm volatile("tcgen05.st.sync.aligned.16x256b.x1.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(taddr),
+               "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+               : "memory");
+}
+
+// D [TMEM] (+)= A [TMEM, 16-bit values packed two per column, K-consecutive] x B [smem
+// descriptor], kind::f16, one K = 16 step. Issued by one thread.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Operand without swizzle: 8 x 16-byte core matrices; lbo / sbo the byte strides between core
+// matrices along K and along M / N (MN-major) -- see the canonical layouts above.
+__device__ __forceinline__ uint64_t interleave_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version of sm_100; layout type 0: no swizzle
+  return d;
+}
+
 // ---- tensor-map (TMA) tile loads -------------------------------------------------------------
 // Box at coordinates (x, y, z) of a 3-D tensor map into shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,

@@ -29,10 +29,21 @@
 
 #include "device_util.cuh"
 #include "gdnq.h"
+#include "tc_util.cuh"
 
 namespace gdnq {
 
 constexpr int kThreads = 256;
+
+// Tensor memory of a persistent step CTA whose window flush runs its rank update on tcgen05
+// (scalar gate): the CTA's TMEM columns (128 for the materialised state, 3 x 32 for the split
+// write-vector operand), the mbarrier the products commit to, and that barrier's next phase.
+struct TcCtx {
+  uint32_t tmem;
+  uint64_t* bar;
+  uint32_t phase;
+};
+constexpr uint32_t kFlushTmemCols = 256;
 
 template <int D_, bool DIAG_, bool INT4_, typename Act_, typename Buf_, bool SMOOTH_ = false>
 struct WinCfg {
@@ -613,13 +624,13 @@ namespace gdnq {
 template <class C>
 __device__ __forceinline__ void step_head(const WinArgs& a, const WinLayout& L, uint8_t* sm,
                                           uint8_t* st, int head, int P, float g_scalar,
-                                          float beta) {
+                                          float beta, TcCtx& tc) {
   using Act = typename C::Act;
   using Buf = typename C::Buf;
   constexpr int D = C::D, CPR = C::CPR, RPP = C::RPP;
   if constexpr (C::MMA) {
     if (!C::DIAG || a.W <= kMmaDiagMaxW) {
-      step_head_mma<C>(a, L, sm, st, head, P, g_scalar, beta);
+      step_head_mma<C>(a, L, sm, st, head, P, g_scalar, beta, tc);
       return;
     }
   }
@@ -858,6 +869,14 @@ __global__ void __launch_bounds__(kStepThreads, 2)
   const int h0 = blockIdx.x * per_cta;
   const int nh = min(per_cta, heads - h0);
   if (nh <= 0) return;
+  // the scalar-gate tensor-core path flushes windows on tcgen05: TMEM for the whole launch
+  constexpr bool kTc = C::MMA && !C::DIAG;
+  if constexpr (kTc) {
+    if (tid < 32) {
+      tmem_alloc(reinterpret_cast<uint32_t*>(sm + 104), kFlushTmemCols);
+      tmem_relinquish();
+    }
+  }
   const bool mma = step_uses_mma<C>(a.W);
   const int Wr = (a.W + 15) & ~15;
   const WinLayout L0 = win_layout_mix<C, MIX>(a.W, a.r, 0, per_cta, Wr, !mma);  // the scratch part
@@ -917,11 +936,20 @@ __global__ void __launch_bounds__(kStepThreads, 2)
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L.bars);
+  // after the stage barriers: the row high-water marks (64..83), the flush products' barrier
+  // (96) and the TMEM address (104)
+  TcCtx tc{0u, reinterpret_cast<uint64_t*>(sm + 96), 0u};
   if (tid == 0) {
     for (int s = 0; s < nstages; ++s) mbar_init(&bars[s], 1);
+    if constexpr (kTc) mbar_init(tc.bar, 1);
     fence_barrier_init();
   }
+  tc_fence_before();
   csync();
+  if constexpr (kTc) {
+    tc_fence_after();
+    tc.tmem = *reinterpret_cast<const uint32_t*>(sm + 104);
+  }
   // Restage stage s with head index `hn` (one thread, once the stage is free). With ragged
   // windows the stage may hold another head's write vectors in [P, P rounded up to 16): the
   // copies then also bring zeros over them.
@@ -938,8 +966,8 @@ __global__ void __launch_bounds__(kStepThreads, 2)
   };
   if (tid == 0)
     for (int s = 0; s < nstages && s < nh; ++s) restage(s, s);
-  if (!stage_wait(a, &bars[0], 0u)) return;
-  for (int n = 0; n < nh; ++n) {
+  const bool first_ok = stage_wait(a, &bars[0], 0u);
+  for (int n = 0; first_ok && n < nh; ++n) {
     // refill the stage head n - 1 left; the issuer is the last warp, which has the least work
     // early in a head (the pair-coefficient tiles go to warps 4, 5, ... in order)
     if (nstages > 1 && tid == kStepIssuer && n > 0 && n - 1 + nstages < nh)
@@ -950,11 +978,11 @@ __global__ void __launch_bounds__(kStepThreads, 2)
       bool done = false;
       if constexpr (MIX) {
         if (head_is_int4(a, h0 + n)) {
-          step_head<Int4Of<C>>(a, L, sm, st, h0 + n, P, C::DIAG ? 0.f : hg[n], hb[n]);
+          step_head<Int4Of<C>>(a, L, sm, st, h0 + n, P, C::DIAG ? 0.f : hg[n], hb[n], tc);
           done = true;
         }
       }
-      if (!done) step_head<C>(a, L, sm, st, h0 + n, P, C::DIAG ? 0.f : hg[n], hb[n]);
+      if (!done) step_head<C>(a, L, sm, st, h0 + n, P, C::DIAG ? 0.f : hg[n], hb[n], tc);
     } else if (tid == 0) {
       report(a.status, GDN_DEVICE_BAD_POS);
     }
@@ -971,7 +999,15 @@ __global__ void __launch_bounds__(kStepThreads, 2)
                       ? 0 : 1;
     if (csync_or(timed_out)) {
       if (tid == 0) report(a.status, GDN_DEVICE_WAIT_TIMEOUT);
-      return;
+      break;
+    }
+  }
+  if constexpr (kTc) {  // every path ends here: the TMEM goes back
+    tc_fence_before();
+    csync();
+    if (tid < 32) {
+      tc_fence_after();
+      tmem_dealloc(tc.tmem, kFlushTmemCols);
     }
   }
 }

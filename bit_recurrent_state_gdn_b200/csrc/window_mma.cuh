@@ -29,7 +29,7 @@ namespace gdnq {
 
 template <class C>
 __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uint8_t* st, int head,
-                          int P, float Ls);
+                          int P, float Ls, TcCtx& tc);
 
 // Pair i's coefficients (a, b) as the three-way bf16 split rows of the phase-3 right-hand side.
 __device__ __forceinline__ void put_coef(__nv_bfloat16* Bc, int bcs, int i, float av, float bv) {
@@ -47,7 +47,7 @@ __device__ __forceinline__ void put_coef(__nv_bfloat16* Bc, int bcs, int i, floa
 template <class C>
 __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm,
                                               uint8_t* st, int head, int P, float g_scalar,
-                                              float beta) {
+                                              float beta, TcCtx& tc) {
   using bf = __nv_bfloat16;
   constexpr int D = 128;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, gid = lane >> 2, q4 = lane & 3;
@@ -373,7 +373,7 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
   if (tid == 0) a.pos[head] = flush ? 0 : P + 1;
   if (!flush) return;
   csync();
-  flush_mma<C>(a, L, sm, st, head, P, Ls);
+  flush_mma<C>(a, L, sm, st, head, P, Ls, tc);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -392,7 +392,7 @@ __device__ __forceinline__ uint32_t one_hot_opaque(int k) {
 
 template <class C>
 __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uint8_t* st, int head,
-                          int P, float Ls) {
+                          int P, float Ls, TcCtx& tc) {
   using bf = __nv_bfloat16;
   constexpr int D = 128, QMAX = C::QMAX;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, gid = lane >> 2, q4 = lane & 3;
@@ -459,8 +459,12 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
   csync();
 
   // ---- the materialised state, all 16 n-tiles of this warp's 16 rows, computed once -------
-  // acc[nt][0..3] = S_W at (v0, j), (v0, j+1), (v1, j), (v1, j+1), j = 8 nt + 2 q4
-  const int v0 = 16 * warp + gid, v1 = v0 + 8;
+  // acc[nt][0..3] = S_W at (v0, j), (v0, j+1), (v1, j), (v1, j+1), j = 8 nt + 2 q4. Warp w takes
+  // rows rbase .. rbase + 15, inside the TMEM lanes it may access (32 (w % 4) ..).
+  const int rbase = 32 * (warp & 3) + 16 * (warp >> 2);
+  const int v0 = rbase + gid, v1 = v0 + 8;
+  // scalar gate, at most 64 pairs: the rank update runs on tcgen05 with the accumulators in TMEM
+  const bool use_tc = !C::DIAG && Kp <= 64;
   float acc[16][4];
   {
     const float s0 = C::INT4 ? 0.f : s_scales[v0], s1 = C::INT4 ? 0.f : s_scales[v1];
@@ -515,13 +519,81 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
         acc[nt][3] += (h && odd) ? u1 : 0.f;
       }
     }
+    if (use_tc) {
+      if constexpr (!C::DIAG) {
+        // rank-Kp update on tcgen05: D (TMEM lanes = rows v, columns j) starts as the frozen part
+        // above; A = (U Diag(fac))^T split into hi / mid / lo bf16, in TMEM (lane v, two pairs a
+        // column); B = the keys, exact, permuted in place in the stage into 8 x 8 core matrices
+        const uint32_t tl = tc.tmem + ((uint32_t)rbase << 16);
+        tmem_st_frag8(tl, *reinterpret_cast<const float(*)[8][4]>(&acc[0]));
+        tmem_st_frag8(tl + 64, *reinterpret_cast<const float(*)[8][4]>(&acc[8]));
+        for (int n = 0; n < Kp / 16; ++n) {
+          const int k0 = 16 * n + 4 * q4;
+          uint32_t pk[3][4];
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int v = hh ? v1 : v0;
+            float h[4], m[4], l[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              split3(__bfloat162float(s_bu[swz_el<bf, D>(k0 + e, v)]) * fac[k0 + e], h[e], m[e], l[e]);
+            pk[0][2 * hh] = pack_bf16(h[0], h[1]);
+            pk[0][2 * hh + 1] = pack_bf16(h[2], h[3]);
+            pk[1][2 * hh] = pack_bf16(m[0], m[1]);
+            pk[1][2 * hh + 1] = pack_bf16(m[2], m[3]);
+            pk[2][2 * hh] = pack_bf16(l[0], l[1]);
+            pk[2][2 * hh + 1] = pack_bf16(l[2], l[3]);
+          }
+#pragma unroll
+          for (int p = 0; p < 3; ++p)
+            tmem_st_frag1(tl + 128 + 32 * p + 8 * n, pk[p][0], pk[p][1], pk[p][2], pk[p][3]);
+        }
+        // key rows [0, Kp): 16-byte chunk (i, c) to core matrix (c, i / 8), row i % 8
+        uint8_t* kbytes = reinterpret_cast<uint8_t*>(s_bk);
+        uint4 tmp[4];
+        int dst[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int e = tid + C::NT * t, i = e >> 4, c = e & 15;
+          dst[t] = -1;
+          if (i < Kp) {
+            tmp[t] = *reinterpret_cast<const uint4*>(kbytes + swz<256>(i, 16 * c));
+            dst[t] = (c * (Kp >> 3) + (i >> 3)) * 128 + (i & 7) * 16;
+          }
+        }
+        csync();
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          if (dst[t] >= 0) *reinterpret_cast<uint4*>(kbytes + dst[t]) = tmp[t];
+        fence_async_smem();
+        tc_wait_st();
+        tc_fence_before();
+        csync();
+        if (tid == 0) {
+          tc_fence_after();
+          constexpr uint32_t kIdesc = idesc_bf16(128, 128, false, true);
+          const uint32_t kb = smem_u32(kbytes);
+          for (int kk = 0; kk < Kp / 16; ++kk)
+#pragma unroll
+            for (int p = 0; p < 3; ++p)
+              umma_bf16_ts(tc.tmem, tc.tmem + 128 + 32 * p + 8 * kk,
+                           interleave_desc(kb + 256u * kk, 128u, 16u * (uint32_t)Kp), kIdesc, 1u);
+          umma_commit(tc.bar);
+        }
+        if (!mbar_wait_bounded(tc.bar, tc.phase)) report(a.status, GDN_DEVICE_WAIT_TIMEOUT);
+        tc.phase ^= 1u;
+        tc_fence_after();
+        tmem_ld_frag8(tl, *reinterpret_cast<float(*)[8][4]>(&acc[0]));
+        tmem_ld_frag8(tl + 64, *reinterpret_cast<float(*)[8][4]>(&acc[8]));
+      }
+    } else {
     // rank-Kp update U^T (v rows, pair k) times Kt (pair k, column j); the split left-hand
     // side of a k-step serves all 16 n-tiles
     const uint32_t ub = smem_u32(s_bu), kb = smem_u32(s_bk);
     const uint32_t mb = smem_u32(pl_mid), lb = smem_u32(pl_lo);
     for (int s = 0; s < Kp / 16; ++s) {
       uint32_t A[4];
-      ldsm_x4_t(ub + swz<256>(16 * s + r8 + 8 * (mi >> 1), 2 * (16 * warp + 8 * (mi & 1))), A);
+      ldsm_x4_t(ub + swz<256>(16 * s + r8 + 8 * (mi >> 1), 2 * (rbase + 8 * (mi & 1))), A);
       uint32_t Ah[4], Am[4], Al[4];
       if constexpr (!C::DIAG) {
         const int i0 = 16 * s + 2 * q4;
@@ -554,6 +626,7 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
           mma_bf16(acc[2 * n2 + 1], A, B[2], B[3]);
         }
       }
+    }
     }
   }
 
@@ -681,8 +754,8 @@ __device__ void flush_mma(const WinArgs& a, const WinLayout& L, uint8_t* sm, uin
   // ---- this warp's 16 code rows to HBM, 16 bytes per lane per store -----------------------
   {
     constexpr int RB = C::ROW_BYTES, CH = 16 * RB / 16;  // 16-byte chunks of the warp's rows
-    uint8_t* g_codes = a.codes + (size_t)head * a.code_stride + 16 * warp * RB;
-    const uint8_t* src = s_codes + 16 * warp * RB;
+    uint8_t* g_codes = a.codes + (size_t)head * a.code_stride + rbase * RB;
+    const uint8_t* src = s_codes + rbase * RB;
 #pragma unroll
     for (int ch = lane; ch < CH; ch += 32)
       *reinterpret_cast<uint4*>(g_codes + 16 * ch) = *reinterpret_cast<const uint4*>(src + 16 * ch);

@@ -34,6 +34,7 @@ import numpy as np
 from . import build as _build
 
 FMT_NONE, FMT_INT8, FMT_INT4 = 0, 1, 2
+COMP_RULES = {"columns": 0, "power": 1}
 ROUND_NONE, ROUND_F32, ROUND_BF16 = 0, 1, 2
 _FMT = {"none": FMT_NONE, "int8": FMT_INT8, "int4_g32": FMT_INT4, "int4": FMT_INT4}
 _ROUND = {"none": ROUND_NONE, "f32": ROUND_F32, "bf16": ROUND_BF16}
@@ -78,15 +79,15 @@ def load(path: Optional[str] = None):
     lib.orc_plain_run.restype = None
     lib.orc_plain_run.argtypes = [_int] * 5 + [_vp] * 8
     lib.orc_o1_run.restype = _int
-    lib.orc_o1_run.argtypes = [_int] * 8 + [_vp] * 8
+    lib.orc_o1_run.argtypes = [_int] * 9 + [_vp] * 8
     lib.orc_o2_run.restype = _int
-    lib.orc_o2_run.argtypes = [_int] * 10 + [_vp] * 21
+    lib.orc_o2_run.argtypes = [_int] * 11 + [_vp] * 22
     lib.orc_round_other.restype = ctypes.c_double
     lib.orc_round_other.argtypes = [_int, ctypes.c_double]
     lib.orc_smooth_exponent.restype = _int
     lib.orc_smooth_exponent.argtypes = [ctypes.c_double]
     lib.orc_window_end.restype = _int
-    lib.orc_window_end.argtypes = [_int] * 5 + [_vp] * 6
+    lib.orc_window_end.argtypes = [_int] * 6 + [_vp] * 7
     lib.orc_round_e4m3.restype = ctypes.c_double
     lib.orc_round_e4m3.argtypes = [ctypes.c_double]
     lib.orc_fp8_vector.restype = ctypes.c_double
@@ -188,27 +189,29 @@ class WindowEnd:
     residual: np.ndarray   # [D][D] the rescaled residual that was quantized
     codes: np.ndarray      # [D][D] int8
     scales: np.ndarray     # [D][groups]
-    cidx: np.ndarray       # [r]
-    cu: np.ndarray         # [r][D] compensator columns (value side)
+    cidx: np.ndarray       # [r] column rule's columns (-1 for the power rule)
+    cu: np.ndarray         # [r][D] compensator token values
+    ck: np.ndarray         # [r][D] compensator token keys (e_j for the column rule)
     sexp: np.ndarray       # [D] int8 smoothing exponents
     near_tie: int
 
 
 def window_end(S: np.ndarray, fmt: str = "int8", r: int = 0, smooth: bool = False,
-               prec32: bool = False, lib=None) -> WindowEnd:
-    """The window-end operation on one [D][D] state: compensators out, residual smoothing,
-    quantization. The state it leaves is dequant(codes, scales) Diag(2^sexp) plus the
-    compensator columns."""
+               prec32: bool = False, comp_rule: str = "columns", lib=None) -> WindowEnd:
+    """The window-end operation on one [D][D] state: compensator tokens out (``comp_rule``
+    "columns" or "power"), residual smoothing, quantization. The state it leaves is
+    dequant(codes, scales) Diag(2^sexp) plus sum_c cu_c ck_c^T."""
     lib = lib or load()
     R = _f64(S).copy()
     D = R.shape[0]
     f = _FMT[fmt]
     ng = lib.orc_num_groups(FMT_INT8 if f == FMT_NONE else f, D)
     out = WindowEnd(R, np.zeros((D, D), np.int8), np.zeros((D, ng)), np.zeros(max(r, 1), np.int32),
-                    np.zeros((max(r, 1), D)), np.zeros(D, np.int8), 0)
-    out.near_tie = lib.orc_window_end(D, f, r, int(prec32), int(smooth), _p(R), _p(out.codes),
-                                      _p(out.scales), _p(out.cidx), _p(out.cu), _p(out.sexp))
-    out.cidx, out.cu = out.cidx[:r], out.cu[:r]
+                    np.zeros((max(r, 1), D)), np.zeros((max(r, 1), D)), np.zeros(D, np.int8), 0)
+    out.near_tie = lib.orc_window_end(D, f, r, int(prec32), int(smooth), COMP_RULES[comp_rule],
+                                      _p(R), _p(out.codes), _p(out.scales), _p(out.cidx),
+                                      _p(out.cu), _p(out.ck), _p(out.sexp))
+    out.cidx, out.cu, out.ck = out.cidx[:r], out.cu[:r], out.ck[:r]
     return out
 
 
@@ -234,7 +237,7 @@ def plain_run(q, k, v, g, beta, S0=None, state_round: str = "none", want_o: bool
 
 
 def o1_run(q, k, v, g, beta, W: int, r: int = 0, fmt: str = "int8", S0=None,
-           smooth: bool = False, lib=None):
+           smooth: bool = False, comp_rule: str = "columns", lib=None):
     """Literal matrix-form recurrence with window-end requantisation (fp64 decisions; ``smooth``
     adds the residual smoothing). Returns (o, S_T, near_ties)."""
     lib = lib or load()
@@ -244,7 +247,8 @@ def o1_run(q, k, v, g, beta, W: int, r: int = 0, fmt: str = "int8", S0=None,
     S0 = _f64(S0)
     o = np.zeros((T, nh, D))
     S = np.zeros((nh, D, D))
-    ties = lib.orc_o1_run(D, T, W, r, _FMT[fmt], nh, Dg, int(smooth), _p(S0), _p(q), _p(k),
+    ties = lib.orc_o1_run(D, T, W, r, _FMT[fmt], nh, Dg, int(smooth), COMP_RULES[comp_rule],
+                          _p(S0), _p(q), _p(k),
                           _p(v), _p(g), _p(beta), _p(o), _p(S))
     return o, S, ties
 
@@ -256,6 +260,7 @@ class O2Result:
     scales: np.ndarray     # [nh][D][groups]
     cidx: np.ndarray       # [nh][r]
     cu: np.ndarray         # [nh][r][D]
+    ck: np.ndarray         # [nh][r][D] compensator keys
     pos: np.ndarray        # [nh]
     bk: np.ndarray         # [nh][W][D]
     bu: np.ndarray         # [nh][W][D]
@@ -269,7 +274,8 @@ class O2Result:
 
 def o2_run(q, k, v, g, beta, W: int, r: int = 0, fmt: str = "int8", S0=None,
            round_storage: bool = False, buf_round: str = "bf16", flush_mask=None,
-           smooth: bool = False, want_u_raw: bool = False, u_flip=None, lib=None) -> O2Result:
+           smooth: bool = False, want_u_raw: bool = False, u_flip=None,
+           comp_rule: str = "columns", lib=None) -> O2Result:
     """Buffered-window form. ``round_storage`` mirrors GPU storage (fp32 state / L / scales,
     ``buf_round`` write vectors, fp32 quantizer decisions); ``smooth`` adds the residual
     smoothing at every quantization. ``want_u_raw`` returns every write vector before its
@@ -285,7 +291,8 @@ def o2_run(q, k, v, g, beta, W: int, r: int = 0, fmt: str = "int8", S0=None,
     res = O2Result(
         o=np.zeros((T, nh, D)), codes=np.zeros((nh, D, D), np.int8),
         scales=np.zeros((nh, D, ng)), cidx=np.zeros((nh, max(r, 0)), np.int32),
-        cu=np.zeros((nh, max(r, 0), D)), pos=np.zeros(nh, np.int32),
+        cu=np.zeros((nh, max(r, 0), D)), ck=np.zeros((nh, max(r, 0), D)),
+        pos=np.zeros(nh, np.int32),
         bk=np.zeros((nh, W, D)), bu=np.zeros((nh, W, D)), bL=np.zeros((nh, W, D)),
         S=np.zeros((nh, D, D)), near_ties=0, ties=np.zeros(nh, np.int32),
         sexp=np.zeros((nh, D), np.int8))
@@ -294,9 +301,11 @@ def o2_run(q, k, v, g, beta, W: int, r: int = 0, fmt: str = "int8", S0=None,
         res.u_raw = np.zeros((T, nh, D))
     uf = None if u_flip is None else np.ascontiguousarray(u_flip, np.uint8).reshape(T, nh, D)
     res.near_ties = lib.orc_o2_run(
-        D, T, W, r, f, nh, Dg, int(round_storage), _ROUND[buf_round], int(smooth), _p(S0),
+        D, T, W, r, f, nh, Dg, int(round_storage), _ROUND[buf_round], int(smooth),
+        COMP_RULES[comp_rule], _p(S0),
         _p(q), _p(k), _p(v), _p(g), _p(beta), _p(fm), _p(res.o), _p(res.codes), _p(res.scales),
-        _p(res.cidx) if r > 0 else None, _p(res.cu) if r > 0 else None, _p(res.pos),
+        _p(res.cidx) if r > 0 else None, _p(res.cu) if r > 0 else None,
+        _p(res.ck) if r > 0 else None, _p(res.pos),
         _p(res.bk), _p(res.bu), _p(res.bL), _p(res.S), _p(res.ties), _p(res.sexp),
         _p(res.u_raw), _p(uf))
     return res

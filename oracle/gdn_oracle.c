@@ -252,14 +252,108 @@ int orc_smooth_exponent(double colmax) {
  * quantize the residual. fmt == NONE keeps the (rescaled) residual unquantized in S. Returns 1
  * on a near tie (of the column choice, or of a smoothing exponent). sexp may be NULL when smooth
  * is 0. */
-static int window_end(int D, int fmt, int r, int prec32, int smooth, double* S, int8_t* codes,
-                      double* scales, int* cidx, double* cu, int8_t* sexp) {
-    int near = orc_select_columns(D, r, S, cidx);
-    for (int c = 0; c < r; ++c)
-        for (int i = 0; i < D; ++i) {
-            cu[(size_t)c * D + i] = S[(size_t)i * D + cidx[c]];
-            S[(size_t)i * D + cidx[c]] = 0.0;
+/* ------------------------------------------------------------------------------------------
+ * Compensator rule "power" (the pages name compensator tokens that keep the state's largest
+ * outliers and share the update path of real tokens, and give no rule; this is the reading of
+ * the tokens as the state's dominant rank-one parts): the r keys are an orthonormal basis X of
+ * the state's dominant r-dimensional key (right singular) subspace, found by subspace
+ * iteration, and the values are S x_c, so the tokens carry S X X^T and the residual is
+ * S (I - X X^T).
+ *   start:   x_c = e_{j_c}, j_1.. j_r the key columns of largest L2 norm (ties: lower index);
+ *   iterate: ORC_POWER_ITERS times X <- orth(S^T (S X)), where orth is modified Gram-Schmidt
+ *            over the columns in order (x_c minus its projections on x_1 .. x_{c-1}, then
+ *            divided by its length; a column of length 0 stays 0);
+ *   tokens:  key x_c, value u_c = S x_c.
+ * prec32 stores keys and values in single precision, as a GPU does.
+ * ---------------------------------------------------------------------------------------- */
+#define ORC_POWER_ITERS 6
+
+static void power_keys(int D, int r, const double* S, double* X) {
+    double* nrm = (double*)calloc((size_t)D, sizeof(double));
+    char* taken = (char*)calloc((size_t)D, 1);
+    double* Y = (double*)malloc(sizeof(double) * (size_t)D * (r > 0 ? r : 1));
+    for (int j = 0; j < D; ++j)
+        for (int i = 0; i < D; ++i) nrm[j] += S[(size_t)i * D + j] * S[(size_t)i * D + j];
+    for (int c = 0; c < r; ++c) {
+        int best = -1;
+        for (int j = 0; j < D; ++j)
+            if (!taken[j] && (best < 0 || nrm[j] > nrm[best])) best = j;
+        if (best >= 0) taken[best] = 1;  /* (r <= D: always a column left) */
+        for (int j = 0; j < D; ++j) X[(size_t)c * D + j] = j == best ? 1.0 : 0.0;
+    }
+    for (int it = 0; it < ORC_POWER_ITERS; ++it) {
+        for (int c = 0; c < r; ++c)           /* Y = S X */
+            for (int i = 0; i < D; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < D; ++j) acc += S[(size_t)i * D + j] * X[(size_t)c * D + j];
+                Y[(size_t)c * D + i] = acc;
+            }
+        for (int c = 0; c < r; ++c)           /* X = S^T Y */
+            for (int j = 0; j < D; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < D; ++i) acc += S[(size_t)i * D + j] * Y[(size_t)c * D + i];
+                X[(size_t)c * D + j] = acc;
+            }
+        for (int c = 0; c < r; ++c) {         /* modified Gram-Schmidt */
+            double* xc = X + (size_t)c * D;
+            for (int p = 0; p < c; ++p) {
+                const double* xp = X + (size_t)p * D;
+                double dot = 0.0;
+                for (int j = 0; j < D; ++j) dot += xc[j] * xp[j];
+                for (int j = 0; j < D; ++j) xc[j] -= dot * xp[j];
+            }
+            double n2 = 0.0;
+            for (int j = 0; j < D; ++j) n2 += xc[j] * xc[j];
+            const double n = sqrt(n2);
+            for (int j = 0; j < D; ++j) xc[j] = n > 0.0 ? xc[j] / n : 0.0;
         }
+    }
+    free(nrm);
+    free(taken);
+    free(Y);
+}
+
+/* Window-end operation on a full state S (overwritten by the residual). The r compensator
+ * tokens (keys ck [r][D], values cu [r][D]) are taken out exactly: rule 0 (columns) picks the r
+ * key columns of largest max-abs (orc_select_columns), keys e_j, values the columns, zeroed in
+ * S; rule 1 (power) as power_keys above, S <- S - sum_c cu_c ck_c^T. Then (smooth) the
+ * residual's columns are rescaled by 2^{-e_j} into sexp and the residual is quantized.
+ * fmt == NONE keeps the (rescaled) residual unquantized in S. Returns 1 on a near tie (of the
+ * column choice, or of a smoothing exponent). sexp may be NULL when smooth is 0; cidx is the
+ * column choice of rule 0 (the power rule leaves it as its start columns are not kept). */
+static int window_end(int D, int fmt, int r, int prec32, int smooth, int rule, double* S,
+                      int8_t* codes, double* scales, int* cidx, double* cu, double* ck,
+                      int8_t* sexp) {
+    int near = 0;
+    if (rule == 1) {
+        power_keys(D, r, S, ck);
+        for (int c = 0; c < r; ++c) {
+            double* kc = ck + (size_t)c * D;
+            if (prec32)
+                for (int j = 0; j < D; ++j) kc[j] = orc_round_f32(kc[j]);
+            for (int i = 0; i < D; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < D; ++j) acc += S[(size_t)i * D + j] * kc[j];
+                cu[(size_t)c * D + i] = prec32 ? orc_round_f32(acc) : acc;
+            }
+            cidx[c] = -1;
+        }
+        for (int c = 0; c < r; ++c)
+            for (int i = 0; i < D; ++i)
+                for (int j = 0; j < D; ++j)
+                    S[(size_t)i * D + j] -= cu[(size_t)c * D + i] * ck[(size_t)c * D + j];
+        if (prec32)
+            for (size_t e = 0; e < (size_t)D * D; ++e) S[e] = orc_round_f32(S[e]);
+    } else {
+        near = orc_select_columns(D, r, S, cidx);
+        for (int c = 0; c < r; ++c) {
+            for (int i = 0; i < D; ++i) {
+                cu[(size_t)c * D + i] = S[(size_t)i * D + cidx[c]];
+                S[(size_t)i * D + cidx[c]] = 0.0;
+            }
+            for (int j = 0; j < D; ++j) ck[(size_t)c * D + j] = j == cidx[c] ? 1.0 : 0.0;
+        }
+    }
     if (smooth) {
         for (int j = 0; j < D; ++j) {
             double m = 0.0;
@@ -285,9 +379,10 @@ static void unsmooth(int D, const int8_t* sexp, double* S) {
 }
 
 /* The window-end operation on its own (pins): S is overwritten by the (rescaled) residual. */
-int orc_window_end(int D, int fmt, int r, int prec32, int smooth, double* S, int8_t* codes,
-                   double* scales, int* cidx, double* cu, int8_t* sexp) {
-    return window_end(D, fmt, r, prec32, smooth, S, codes, scales, cidx, cu, sexp);
+int orc_window_end(int D, int fmt, int r, int prec32, int smooth, int rule, double* S,
+                   int8_t* codes, double* scales, int* cidx, double* cu, double* ck,
+                   int8_t* sexp) {
+    return window_end(D, fmt, r, prec32, smooth, rule, S, codes, scales, cidx, cu, ck, sexp);
 }
 
 static double gate_log(const double* g, int Dg, int j) { return Dg == 1 ? g[0] : g[j]; }
@@ -351,28 +446,33 @@ void orc_plain_run(int D, int T, int nh, int Dg, int state_round, const double* 
  * W-th step, S <- dequant(quant(S - C)) + C, where C holds the r compensator columns of S
  * (fmt NONE: S is left as it is). All decisions in fp64. Returns the number of near ties.
  * ---------------------------------------------------------------------------------------- */
-static int dense_window_end(int D, int fmt, int r, int smooth, double* S) {
+static int dense_window_end(int D, int fmt, int r, int smooth, int rule, double* S) {
     if (fmt == ORC_FMT_NONE && r == 0 && !smooth) return 0;
     int ng = orc_num_groups(fmt == ORC_FMT_NONE ? ORC_FMT_INT8 : fmt, D);
     int8_t* codes = (int8_t*)malloc((size_t)D * D);
     double* scales = (double*)malloc(sizeof(double) * (size_t)D * ng);
     int* cidx = (int*)malloc(sizeof(int) * (size_t)(r > 0 ? r : 1));
     double* cu = (double*)malloc(sizeof(double) * (size_t)(r > 0 ? r : 1) * D);
+    double* ck = (double*)malloc(sizeof(double) * (size_t)(r > 0 ? r : 1) * D);
     int8_t* sexp = (int8_t*)calloc((size_t)D, 1);
-    int near = window_end(D, fmt, r, 0, smooth, S, codes, scales, cidx, cu, sexp);
+    int near = window_end(D, fmt, r, 0, smooth, rule, S, codes, scales, cidx, cu, ck, sexp);
     if (fmt != ORC_FMT_NONE) orc_dequantize(D, fmt, codes, scales, S);
     if (smooth) unsmooth(D, sexp, S);
     free(sexp);
-    for (int c = 0; c < r; ++c)
-        for (int i = 0; i < D; ++i) S[(size_t)i * D + cidx[c]] += cu[(size_t)c * D + i];
+    for (int c = 0; c < r; ++c)            /* the tokens back: S += cu_c ck_c^T */
+        for (int i = 0; i < D; ++i)
+            for (int j = 0; j < D; ++j)
+                S[(size_t)i * D + j] += cu[(size_t)c * D + i] * ck[(size_t)c * D + j];
     free(codes);
     free(scales);
     free(cidx);
     free(cu);
+    free(ck);
     return near;
 }
 
-int orc_o1_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int smooth, const double* S0,
+int orc_o1_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int smooth, int rule,
+               const double* S0,
                const double* q, const double* k, const double* v, const double* g,
                const double* beta, double* o, double* S_out) {
     int ties = 0;
@@ -384,7 +484,7 @@ int orc_o1_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int smooth, 
         double* N = (double*)malloc(sizeof(double) * DD);
         if (S0) memcpy(S, S0 + (size_t)h * DD, sizeof(double) * DD);
         else memset(S, 0, sizeof(double) * DD);
-        ties += dense_window_end(D, fmt, r, smooth, S);
+        ties += dense_window_end(D, fmt, r, smooth, rule, S);
         for (int t = 0; t < T; ++t) {
             const double* kt = k + ((size_t)t * nh + h) * D;
             const double* qt = q + ((size_t)t * nh + h) * D;
@@ -410,7 +510,7 @@ int orc_o1_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int smooth, 
                     ot[i] = acc;
                 }
             }
-            if ((t + 1) % W == 0) ties += dense_window_end(D, fmt, r, smooth, S);
+            if ((t + 1) % W == 0) ties += dense_window_end(D, fmt, r, smooth, rule, S);
         }
         if (S_out) memcpy(S_out + (size_t)h * DD, S, sizeof(double) * DD);
         free(S);
@@ -423,15 +523,16 @@ int orc_o1_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int smooth, 
 /* ------------------------------------------------------------------------------------------
  * O2: the buffered form. Per head the state is
  *   F          the frozen state: dequant(codes, scales) (fmt NONE: an unquantized matrix);
- *   (cidx, cu) r compensator pairs, key e_{cidx[c]}, value cu[c], entered at cumulative gate 0;
+ *   (ck, cu)   r compensator tokens, key ck[c], value cu[c], entered at cumulative gate 0 (the
+ *              column rule's keys are e_{cidx[c]}; the power rule's are dense unit vectors);
  *   (bk, bu, bL)[0..P) buffered write pairs: key, write vector, cumulative log-gate vector;
  *   P          pairs in the window so far.
  * The logical state after the window's P steps, with L = bL[P-1] (0 if P == 0), is
- *   S = F Diag(e^L) + sum_c cu_c (e_{cidx_c} * e^{L})^T + sum_i bu_i (bk_i * e^{L - bL_i})^T.
+ *   S = F Diag(e^L) + sum_c cu_c (ck_c * e^{L})^T + sum_i bu_i (bk_i * e^{L - bL_i})^T.
  * A step at position P:
  *   L_t = L + g_t;  x = e^{L_t} * k_t;  y = e^{L_t} * q_t
- *   w  = F x + sum_c cu_c x[cidx_c] + sum_i bu_i <bk_i * e^{L_t - bL_i}, k_t>   (= S Diag(a_t) k_t)
- *   r  = F y + sum_c cu_c y[cidx_c] + sum_i bu_i <bk_i * e^{L_t - bL_i}, q_t>   (= S Diag(a_t) q_t)
+ *   w  = F x + sum_c cu_c <ck_c, x> + sum_i bu_i <bk_i * e^{L_t - bL_i}, k_t>   (= S Diag(a_t) k_t)
+ *   r  = F y + sum_c cu_c <ck_c, y> + sum_i bu_i <bk_i * e^{L_t - bL_i}, q_t>   (= S Diag(a_t) q_t)
  *   u_t = beta_t (v_t - w);  o_t = r + u_t <k_t, q_t>;  append (k_t, u_t, L_t)
  * which is the recurrence through S Diag(a)(I - beta k k^T) + beta v k^T
  *   = S Diag(a) + beta (v - S Diag(a) k) k^T.
@@ -444,8 +545,9 @@ int orc_o1_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int smooth, 
  * materialised state are fp32, L is fp32, u_t is rounded to buf_round (bf16 / fp32), and the
  * quantizer decides in fp32. round_storage = 0 keeps everything in fp64.
  *
+ * rule selects the compensator rule of window_end (0 columns, 1 power).
  * Outputs (any may be NULL): o [T][nh][D]; codes [nh][D][D]; scales [nh][D][groups];
- * cidx [nh][r]; cu [nh][r][D]; pos [nh]; bk, bu, bL [nh][W][D]; S_out [nh][D][D] (the logical
+ * cidx [nh][r] (column rule); cu, ck [nh][r][D]; pos [nh]; bk, bu, bL [nh][W][D]; S_out [nh][D][D] (the logical
  * state at the end); ties_out [nh] (near ties met per head); sexp_out [nh][D] (the smoothing
  * exponents of the last quantization); flush_mask [T][nh] forces a flush
  * after step t of head h when nonzero; u_raw [T][nh][D] receives every write vector before its
@@ -455,11 +557,11 @@ int orc_o1_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int smooth, 
  * met in compensator choices.
  * ---------------------------------------------------------------------------------------- */
 typedef struct {
-    int D, W, r, fmt, Dg, round_storage, buf_round, smooth;
+    int D, W, r, fmt, Dg, round_storage, buf_round, smooth, rule;
 } o2_cfg;
 
 typedef struct {
-    double *F, *scales, *cu, *bk, *bu, *bL;
+    double *F, *scales, *cu, *ck, *bk, *bu, *bL;
     int8_t *codes, *sexp;
     int* cidx;
     int P;
@@ -474,10 +576,10 @@ static void o2_materialize(const o2_cfg* c, const o2_head* s, const double* L, d
     int D = c->D;
     for (int i = 0; i < D; ++i)
         for (int j = 0; j < D; ++j) S[(size_t)i * D + j] = s->F[(size_t)i * D + j] * exp(L[j]);
-    for (int cc = 0; cc < c->r; ++cc) {
-        int j = s->cidx[cc];
-        for (int i = 0; i < D; ++i) S[(size_t)i * D + j] += s->cu[(size_t)cc * D + i] * exp(L[j]);
-    }
+    for (int cc = 0; cc < c->r; ++cc)  /* token cu_c ck_c^T entered at gate 0 */
+        for (int i = 0; i < D; ++i)
+            for (int j = 0; j < D; ++j)
+                S[(size_t)i * D + j] += s->cu[(size_t)cc * D + i] * s->ck[(size_t)cc * D + j] * exp(L[j]);
     for (int p = 0; p < s->P; ++p)
         for (int i = 0; i < D; ++i)
             for (int j = 0; j < D; ++j)
@@ -490,8 +592,8 @@ static int o2_set_frozen(const o2_cfg* c, o2_head* s, double* S) {
     int D = c->D;
     if (c->round_storage)
         for (size_t e = 0; e < (size_t)D * D; ++e) S[e] = orc_round_f32(S[e]);
-    int near = window_end(D, c->fmt, c->r, c->round_storage, c->smooth, S, s->codes, s->scales,
-                          s->cidx, s->cu, s->sexp);
+    int near = window_end(D, c->fmt, c->r, c->round_storage, c->smooth, c->rule, S, s->codes,
+                          s->scales, s->cidx, s->cu, s->ck, s->sexp);
     if (c->fmt != ORC_FMT_NONE) orc_dequantize(D, c->fmt, s->codes, s->scales, s->F);
     else memcpy(s->F, S, sizeof(double) * (size_t)D * D);
     if (c->smooth) unsmooth(D, s->sexp, s->F);
@@ -525,11 +627,15 @@ static void o2_step(const o2_cfg* c, o2_head* s, const double* qt, const double*
         w[i] = a;
         rr[i] = b;
     }
-    for (int cc = 0; cc < c->r; ++cc) {
-        int j = s->cidx[cc];
+    for (int cc = 0; cc < c->r; ++cc) {  /* tokens: coefficients <ck_c, x>, <ck_c, y> */
+        double ax = 0.0, ay = 0.0;
+        for (int j = 0; j < D; ++j) {
+            ax += s->ck[(size_t)cc * D + j] * x[j];
+            ay += s->ck[(size_t)cc * D + j] * y[j];
+        }
         for (int i = 0; i < D; ++i) {
-            w[i] += s->cu[(size_t)cc * D + i] * x[j];
-            rr[i] += s->cu[(size_t)cc * D + i] * y[j];
+            w[i] += s->cu[(size_t)cc * D + i] * ax;
+            rr[i] += s->cu[(size_t)cc * D + i] * ay;
         }
     }
     for (int p = 0; p < s->P; ++p) {
@@ -561,12 +667,13 @@ static void o2_step(const o2_cfg* c, o2_head* s, const double* qt, const double*
 }
 
 int orc_o2_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int round_storage,
-               int buf_round, int smooth, const double* S0, const double* q, const double* k, const double* v,
-               const double* g, const double* beta, const uint8_t* flush_mask, double* o,
-               int8_t* codes_out, double* scales_out, int* cidx_out, double* cu_out, int* pos_out,
+               int buf_round, int smooth, int rule, const double* S0, const double* q, const double* k,
+               const double* v, const double* g, const double* beta, const uint8_t* flush_mask,
+               double* o, int8_t* codes_out, double* scales_out, int* cidx_out, double* cu_out,
+               double* ck_out, int* pos_out,
                double* bk_out, double* bu_out, double* bL_out, double* S_out, int* ties_out,
                int8_t* sexp_out, double* u_raw, const uint8_t* u_flip) {
-    o2_cfg c = {D, W, r, fmt, Dg, round_storage, buf_round, smooth};
+    o2_cfg c = {D, W, r, fmt, Dg, round_storage, buf_round, smooth, rule};
     int ng = orc_num_groups(fmt == ORC_FMT_NONE ? ORC_FMT_INT8 : fmt, D);
     int ties = 0;
 #pragma omp parallel for schedule(dynamic) reduction(+ : ties)
@@ -579,6 +686,7 @@ int orc_o2_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int round_st
         s.sexp = (int8_t*)calloc((size_t)D, 1);
         s.cidx = (int*)calloc((size_t)(r > 0 ? r : 1), sizeof(int));
         s.cu = (double*)calloc((size_t)(r > 0 ? r : 1) * D, sizeof(double));
+        s.ck = (double*)calloc((size_t)(r > 0 ? r : 1) * D, sizeof(double));
         s.bk = (double*)calloc((size_t)W * D, sizeof(double));
         s.bu = (double*)calloc((size_t)W * D, sizeof(double));
         s.bL = (double*)calloc((size_t)W * D, sizeof(double));
@@ -603,6 +711,7 @@ int orc_o2_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int round_st
         if (scales_out) memcpy(scales_out + (size_t)h * D * ng, s.scales, sizeof(double) * (size_t)D * ng);
         if (cidx_out && r > 0) memcpy(cidx_out + (size_t)h * r, s.cidx, sizeof(int) * (size_t)r);
         if (cu_out && r > 0) memcpy(cu_out + (size_t)h * r * D, s.cu, sizeof(double) * (size_t)r * D);
+        if (ck_out && r > 0) memcpy(ck_out + (size_t)h * r * D, s.ck, sizeof(double) * (size_t)r * D);
         if (pos_out) pos_out[h] = s.P;
         if (sexp_out) memcpy(sexp_out + (size_t)h * D, s.sexp, (size_t)D);
         if (bk_out) memcpy(bk_out + (size_t)h * W * D, s.bk, sizeof(double) * (size_t)W * D);
@@ -612,7 +721,7 @@ int orc_o2_run(int D, int T, int W, int r, int fmt, int nh, int Dg, int round_st
             o2_current_L(&c, &s, Lt);
             o2_materialize(&c, &s, Lt, S_out + h * DD);
         }
-        free(s.F); free(s.scales); free(s.codes); free(s.sexp); free(s.cidx); free(s.cu);
+        free(s.F); free(s.scales); free(s.codes); free(s.sexp); free(s.cidx); free(s.cu); free(s.ck);
         free(s.bk); free(s.bu); free(s.bL); free(Sx); free(vec);
     }
     return ties;

@@ -472,6 +472,96 @@ def pin_write_vectors_before_rounding(lib):
 
 
 # ---------------------------------------------------------------------------------------------
+# Power compensators (reading: tokens spanning the dominant key subspace, subspace iteration)
+# ---------------------------------------------------------------------------------------------
+def _tokens(we):
+    return we.cu.T @ we.ck  # sum_c cu_c ck_c^T
+
+
+def pin_power_exact_low_rank(lib):
+    """A state of rank r is carried entirely by r power tokens: residual 0, tokens = S."""
+    rng = np.random.default_rng(71)
+    for D, r in ((16, 2), (32, 4)):
+        A, B = rng.standard_normal((D, r)), rng.standard_normal((D, r))
+        S = A @ B.T
+        we = oracle.window_end(S, "none", r=r, comp_rule="power", lib=lib)
+        close(_tokens(we), S, 1e-10, "rank-r state rebuilt by its tokens")
+        assert np.abs(we.residual).max() <= 1e-10 * np.abs(S).max()
+
+
+def pin_power_planted_outlier(lib):
+    """A dominant rank-one outlier planted on noise is the first token: its key is the
+    outlier's key direction (up to sign), its value S times that key."""
+    rng = np.random.default_rng(72)
+    D = 32
+    u, v = rng.standard_normal(D), rng.standard_normal(D)
+    u, v = u / np.linalg.norm(u), v / np.linalg.norm(v)
+    S = 0.02 * rng.standard_normal((D, D)) + 30.0 * np.outer(u, v)
+    we = oracle.window_end(S, "none", r=1, comp_rule="power", lib=lib)
+    v1 = np.linalg.svd(S)[2][0]  # LAPACK's top right singular vector
+    assert abs(float(we.ck[0] @ v1)) >= 1 - 1e-12, we.ck[0] @ v1
+    assert abs(float(we.ck[0] @ v)) >= 1 - 1e-4, we.ck[0] @ v
+    close(we.cu[0], S @ we.ck[0], 1e-12, "token value = S key")
+
+
+def pin_power_energy_matches_svd(lib):
+    """With a clear spectral gap the tokens carry the top-r singular energy that LAPACK's SVD
+    gives; the keys are orthonormal, the residual is orthogonal to them, and residual + tokens
+    is the state exactly."""
+    rng = np.random.default_rng(73)
+    D, r = 32, 4
+    U, _ = np.linalg.qr(rng.standard_normal((D, D)))
+    V, _ = np.linalg.qr(rng.standard_normal((D, D)))
+    sig = np.concatenate([[100.0, 50.0, 25.0, 12.0], np.linspace(1.0, 0.1, D - 4)])
+    S = (U * sig) @ V.T
+    we = oracle.window_end(S, "none", r=r, comp_rule="power", lib=lib)
+    sv = np.linalg.svd(S, compute_uv=False)
+    e_tok = float(np.sum(_tokens(we) ** 2))
+    assert abs(e_tok - float(np.sum(sv[:r] ** 2))) <= 1e-9 * e_tok, (e_tok, sv[:r])
+    assert np.allclose(we.ck @ we.ck.T, np.eye(r), atol=1e-12)
+    assert np.abs(we.residual @ we.ck.T).max() <= 1e-10 * np.abs(S).max()
+    close(we.residual + _tokens(we), S, 1e-13, "residual + tokens")
+    # a random state (no gap): still orthonormal keys and an exact decomposition
+    S2 = rng.standard_normal((D, D))
+    we2 = oracle.window_end(S2, "none", r=r, comp_rule="power", lib=lib)
+    assert np.allclose(we2.ck @ we2.ck.T, np.eye(r), atol=1e-12)
+    close(we2.residual + _tokens(we2), S2, 1e-13, "residual + tokens, no gap")
+
+
+def pin_power_start_and_ties(lib):
+    """On a diagonal state the dominant key subspace is spanned by the coordinate vectors of
+    the largest entries, which is where the iteration starts (largest column norms) and stays:
+    the keys are exactly those e_j, ties going to the lower column."""
+    D = 8
+    d = np.array([0.5, -3.0, 1.0, 2.0, 0.25, -2.0, 0.1, 0.7])
+    we = oracle.window_end(np.diag(d), "none", r=2, comp_rule="power", lib=lib)
+    assert np.array_equal(we.ck, np.eye(D)[[1, 3]]), we.ck
+    assert np.array_equal(we.cu, np.diag(d)[:, [1, 3]].T)
+    tie = np.diag([1.0, 2.0, 2.0, 0.5])
+    we = oracle.window_end(tie, "none", r=1, comp_rule="power", lib=lib)
+    assert np.array_equal(we.ck, np.eye(4)[[1]]), we.ck
+
+
+def pin_power_windows_agree(lib):
+    """With power tokens: the literal form (O1) equals the buffered form (O2) with
+    quantization on, and without quantization the buffered form is the plain recurrence."""
+    T, nh, D = 12, 3, 16
+    for gate in ("scalar", "diag"):
+        q, k, v, g, beta = rand_inputs(81, T, nh, D, gate, outlier=True)
+        S0 = np.random.default_rng(3).standard_normal((nh, D, D))
+        for W, r in ((3, 2), (5, 1)):
+            o1, S1, _ = oracle.o1_run(q, k, v, g, beta, W=W, r=r, fmt="int8", S0=S0,
+                                      comp_rule="power", lib=lib)
+            o2 = oracle.o2_run(q, k, v, g, beta, W=W, r=r, fmt="int8", S0=S0,
+                               comp_rule="power", lib=lib)
+            close(o2.o, o1, 1e-10, f"O1 = O2 with power tokens ({gate}, W={W})")
+        plain, _ = oracle.plain_run(q, k, v, g, beta, S0=S0, lib=lib)
+        ex = oracle.o2_run(q, k, v, g, beta, W=4, r=2, fmt="none", S0=S0, comp_rule="power",
+                           lib=lib)
+        close(ex.o, plain, 1e-10, f"unquantized windows with power tokens = plain ({gate})")
+
+
+# ---------------------------------------------------------------------------------------------
 # Residual smoothing (reading: per-column power-of-two factors m_j = 2^floor(E_j / 2))
 # ---------------------------------------------------------------------------------------------
 def pin_golden_smoothing(lib):
@@ -717,6 +807,11 @@ PINS = [
     pin_storage_roundings,
     pin_round_other,
     pin_write_vectors_before_rounding,
+    pin_power_exact_low_rank,
+    pin_power_planted_outlier,
+    pin_power_energy_matches_svd,
+    pin_power_start_and_ties,
+    pin_power_windows_agree,
     pin_golden_smoothing,
     pin_smooth_exponent,
     pin_smoothing_properties,

@@ -29,8 +29,8 @@ MUTANTS = [
      "exp(gate_log(gt, Dg, j)) * ((j == l",
      "exp(gate_log(gt, Dg, l)) * ((j == l"),
     ("O1: window end one step early",
-     "if ((t + 1) % W == 0) ties += dense_window_end(D, fmt, r, smooth, S);",
-     "if (t % W == 0) ties += dense_window_end(D, fmt, r, smooth, S);"),
+     "if ((t + 1) % W == 0) ties += dense_window_end(D, fmt, r, smooth, rule, S);",
+     "if (t % W == 0) ties += dense_window_end(D, fmt, r, smooth, rule, S);"),
     ("O2: beta dropped from the write vector",
      "double u = bt * (vt[i] - w[i]);",
      "double u = (vt[i] - w[i]);"),
@@ -44,8 +44,8 @@ MUTANTS = [
      "if (ot) ot[i] = rr[i] + u * kq;",
      "if (ot) ot[i] = rr[i];"),
     ("O2: compensators dropped from the step",
-     "w[i] += s->cu[(size_t)cc * D + i] * x[j];",
-     "w[i] += 0.0 * x[j];"),
+     "w[i] += s->cu[(size_t)cc * D + i] * ax;",
+     "w[i] += 0.0 * ax;"),
     ("O2: key used for the query projection",
      "y[j] = exp(Lt[j]) * qt[j];",
      "y[j] = exp(Lt[j]) * kt[j];"),
@@ -53,8 +53,8 @@ MUTANTS = [
      "Lt[j] = Lt[j] + gate_log(gt, c->Dg, j);",
      "Lt[j] = gate_log(gt, c->Dg, j);"),
     ("O2: compensator not decayed at materialisation",
-     "S[(size_t)i * D + j] += s->cu[(size_t)cc * D + i] * exp(L[j]);",
-     "S[(size_t)i * D + j] += s->cu[(size_t)cc * D + i];"),
+     "S[(size_t)i * D + j] += s->cu[(size_t)cc * D + i] * s->ck[(size_t)cc * D + j] * exp(L[j]);",
+     "S[(size_t)i * D + j] += s->cu[(size_t)cc * D + i] * s->ck[(size_t)cc * D + j];"),
     ("O2: frozen state not decayed at materialisation",
      "S[(size_t)i * D + j] = s->F[(size_t)i * D + j] * exp(L[j]);",
      "S[(size_t)i * D + j] = s->F[(size_t)i * D + j];"),
@@ -124,6 +124,27 @@ MUTANTS = [
     ("e4m3: subnormal spacing too fine",
      "if (qexp < -9) qexp = -9;",
      "if (qexp < -10) qexp = -10;"),
+    ("power tokens: keys not normalised",
+     "xc[j] = n > 0.0 ? xc[j] / n : 0.0;",
+     "xc[j] = xc[j];"),
+    ("power tokens: S instead of S^T in the iteration",
+     "acc += S[(size_t)i * D + j] * Y[(size_t)c * D + i];",
+     "acc += S[(size_t)j * D + i] * Y[(size_t)c * D + i];"),
+    ("power tokens: Gram-Schmidt projection added",
+     "xc[j] -= dot * xp[j];",
+     "xc[j] += dot * xp[j];"),
+    ("power tokens: values from S^T",
+     "acc += S[(size_t)i * D + j] * kc[j];",
+     "acc += S[(size_t)j * D + i] * kc[j];"),
+    ("power tokens: residual keeps the tokens",
+     "S[(size_t)i * D + j] -= cu[(size_t)c * D + i] * ck[(size_t)c * D + j];",
+     "S[(size_t)i * D + j] -= 0.0 * cu[(size_t)c * D + i] * ck[(size_t)c * D + j];"),
+    ("power tokens: start from the smallest columns",
+     "if (!taken[j] && (best < 0 || nrm[j] > nrm[best])) best = j;",
+     "if (!taken[j] && (best < 0 || nrm[j] < nrm[best])) best = j;"),
+    ("O2: token coefficient from the ungated key",
+     "ax += s->ck[(size_t)cc * D + j] * x[j];",
+     "ax += s->ck[(size_t)cc * D + j] * kt[j];"),
     ("alternative rounding: the rounding itself",
      "return round_to(mode, x) == lo ? hi : lo;",
      "return round_to(mode, x);"),

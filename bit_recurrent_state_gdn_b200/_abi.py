@@ -24,11 +24,11 @@ _sz = ctypes.c_size_t
 class gdn_config(ctypes.Structure):
     _fields_ = [(n, _i32) for n in
                 ("B", "H", "d_k", "d_v", "W", "r", "gate", "fmt", "act_dtype", "buf_dtype",
-                 "smooth")]
+                 "smooth", "comp_rule")]
 
 
 STATE_FIELDS = ("codes", "scales", "buf_k", "buf_u", "buf_L", "comp_idx", "comp_u", "pos",
-                "status", "head_fmt", "smooth_exp")
+                "status", "head_fmt", "smooth_exp", "comp_k")
 
 
 class gdn_state(ctypes.Structure):
@@ -36,7 +36,7 @@ class gdn_state(ctypes.Structure):
 
 
 SIZE_FIELDS = ("codes", "scales", "buf_k", "buf_u", "buf_L", "comp_idx", "comp_u", "pos",
-               "smem_step", "head_fmt", "smooth_exp")
+               "smem_step", "head_fmt", "smooth_exp", "comp_k")
 
 
 class gdn_sizes(ctypes.Structure):

@@ -30,12 +30,17 @@ class GdnError(RuntimeError):
         super().__init__(f"{where}: {name}: {detail}")
 
 
+_COMP = {"columns": 0, "power": 1}
+
+
 def make_config(B: int, H: int, D: int, W: int = 1, r: int = 0, gate: str = "scalar",
                 fmt: str = "int8", act: str = "bf16", buf: str = "bf16",
-                smooth: bool = False) -> _abi.gdn_config:
-    """smooth: residual smoothing (per-key-column power-of-two factors) at every quantization."""
+                smooth: bool = False, comp_rule: str = "columns") -> _abi.gdn_config:
+    """smooth: residual smoothing (per-key-column power-of-two factors) at every quantization.
+    comp_rule: "columns" or "power" compensator tokens."""
     return _abi.gdn_config(B, H, D, D, W, r, _GATE[gate], _FMT[fmt], _DT[act], _DT[buf],
-                           _abi.GDN_SMOOTH_POW2_COLUMNS if smooth else _abi.GDN_SMOOTH_NONE)
+                           _abi.GDN_SMOOTH_POW2_COLUMNS if smooth else _abi.GDN_SMOOTH_NONE,
+                           _COMP[comp_rule])
 
 
 def _check(status: int, where: str):
@@ -87,6 +92,7 @@ class GdnState:
     status: torch.Tensor
     head_fmt: torch.Tensor  # int8 [B*H]: each head's format (mixed-format states only)
     smooth_exp: torch.Tensor  # int8 [B*H*D]: smoothing exponents (smoothed states only)
+    comp_k: torch.Tensor  # fp32 [B*H*r*D]: compensator token keys (power rule only)
 
     @staticmethod
     def allocate(cfg: _abi.gdn_config, device="cuda", head_fmt=None) -> "GdnState":
@@ -106,7 +112,8 @@ class GdnState:
             comp_u=buf(sz.comp_u, torch.float32), pos=buf(sz.pos, torch.int32),
             status=torch.zeros(4, dtype=torch.int32, device=dev),
             head_fmt=_head_fmt(cfg, head_fmt, sz.head_fmt, dev),
-            smooth_exp=torch.zeros(max(sz.smooth_exp, 16), dtype=torch.int8, device=dev))
+            smooth_exp=torch.zeros(max(sz.smooth_exp, 16), dtype=torch.int8, device=dev),
+            comp_k=torch.zeros(max(sz.comp_k // 4, 4), dtype=torch.float32, device=dev))
 
     def c_struct(self) -> _abi.gdn_state:
         return _abi.gdn_state(*[getattr(self, n).data_ptr() for n in _abi.STATE_FIELDS])

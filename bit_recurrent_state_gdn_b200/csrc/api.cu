@@ -87,6 +87,14 @@ gdn_status check_config(const gdn_config* c, Use use) {
   if ((c->fmt == GDN_FMT_INT4_G32 || c->fmt == GDN_FMT_MIXED) && c->d_k != 128)
     return fail(GDN_ERR_UNSUPPORTED, "int4 and mixed states are built for d_k = 128");
   if (c->W > (1 << 20)) return fail(GDN_ERR_UNSUPPORTED, "W=%d is too large", c->W);
+  if (c->comp_rule != GDN_COMP_COLUMNS && c->comp_rule != GDN_COMP_POWER)
+    return fail(GDN_ERR_INVALID_ARG, "comp_rule=%d is not a gdn_comp_rule", c->comp_rule);
+  if (c->comp_rule == GDN_COMP_POWER &&
+      (c->d_k != 128 || c->act_dtype != GDN_DTYPE_BF16 || c->buf_dtype != GDN_DTYPE_BF16 ||
+       c->fmt == GDN_FMT_MIXED || c->smooth != GDN_SMOOTH_NONE || c->W > 64))
+    return fail(GDN_ERR_UNSUPPORTED,
+                "power compensator tokens are built for d = 128, bf16 activations and buffers, "
+                "INT8 / INT4_G32 states without smoothing and W <= 64");
   const size_t smem = gdnq::window_smem_bytes(*c);
   if (smem > (size_t)gdnq::kMaxSmemPerCta)
     return fail(GDN_ERR_UNSUPPORTED, "W=%d, r=%d need %zu bytes of shared memory per CTA (max %d)",
@@ -95,8 +103,10 @@ gdn_status check_config(const gdn_config* c, Use use) {
 }
 
 struct PerHead {
-  size_t codes, scales, buf_k, buf_u, buf_L, comp_idx, comp_u;
+  size_t codes, scales, buf_k, buf_u, buf_L, comp_idx, comp_u, comp_k;
 };
+
+bool power_rule(const gdn_config* c) { return c->comp_rule == GDN_COMP_POWER && c->r > 0; }
 
 PerHead per_head_bytes(const gdn_config* c) {
   const size_t D = (size_t)c->d_k;
@@ -109,6 +119,7 @@ PerHead per_head_bytes(const gdn_config* c) {
   p.buf_L = 4 * (c->gate == GDN_GATE_DIAG ? (size_t)c->W * D : (size_t)round4(c->W));
   p.comp_idx = 4 * (size_t)round4(c->r);
   p.comp_u = 4 * (size_t)c->r * D;
+  p.comp_k = power_rule(c) ? 4 * (size_t)c->r * D : 0;
   return p;
 }
 
@@ -125,6 +136,7 @@ gdn_status check_state(const gdn_config* c, const gdn_state* s) {
     if ((st = need_ptr(s->comp_idx, "state.comp_idx")) != GDN_OK) return st;
     if ((st = need_ptr(s->comp_u, "state.comp_u")) != GDN_OK) return st;
   }
+  if (power_rule(c) && (st = need_ptr(s->comp_k, "state.comp_k")) != GDN_OK) return st;
   if (s->status && (reinterpret_cast<uintptr_t>(s->status) & 3u) != 0)
     return fail(GDN_ERR_INVALID_ARG, "state.status is not 4-byte aligned");
   if (c->fmt == GDN_FMT_MIXED && !s->head_fmt)
@@ -169,6 +181,7 @@ gdnq::WinArgs make_args(const gdn_config* c, const gdn_state* s) {
   a.scale_stride = (uint32_t)(ph.scales / 4);
   a.head_fmt = c->fmt == GDN_FMT_MIXED ? s->head_fmt : nullptr;
   a.smooth_exp = c->smooth != GDN_SMOOTH_NONE ? s->smooth_exp : nullptr;
+  a.comp_k = power_rule(c) ? s->comp_k : nullptr;
   a.H = c->H;
   a.W = c->W;
   a.r = c->r;
@@ -224,7 +237,7 @@ size_t window_smem_bytes(const gdn_config& c) {
   const int nscales = int4 || mixed ? D * (D / 32) : D;
   return win_layout(D, code_bytes, nscales, (int)act_size(&c), (int)buf_size(&c),
                     c.gate == GDN_GATE_DIAG, c.W, c.r, 1, kMaxHeadsPerCta, -1, true,
-                    c.smooth != GDN_SMOOTH_NONE)
+                    c.smooth != GDN_SMOOTH_NONE, c.comp_rule == GDN_COMP_POWER)
       .total;
 }
 
@@ -348,6 +361,7 @@ gdn_status gdn_state_sizes(const gdn_config* cfg, gdn_sizes* out) {
   out->smem_step = gdnq::window_smem_bytes(*cfg);
   out->head_fmt = cfg->fmt == GDN_FMT_MIXED ? n : 0;
   out->smooth_exp = cfg->smooth != GDN_SMOOTH_NONE ? n * (size_t)cfg->d_k : 0;
+  out->comp_k = n * p.comp_k;
   return GDN_OK;
 }
 

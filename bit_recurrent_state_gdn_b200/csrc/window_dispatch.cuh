@@ -48,7 +48,7 @@ struct StepPlan {
 };
 
 template <class C, bool MIX>
-StepPlan plan_step(int W, int r, int heads) {
+StepPlan plan_step(int W, int r, int heads, bool power = false) {
   constexpr int kSmemPerSm = 228 * 1024, kReserved = 1024;
   const int sms = num_sms();
   const bool red = !step_uses_mma<C>(W);
@@ -56,18 +56,58 @@ StepPlan plan_step(int W, int r, int heads) {
   StepPlan p;
   const size_t half = (size_t)kSmemPerSm / 2 - kReserved;
   int bps = 2;
-  if ((size_t)win_layout_mix<C, MIX>(W, r, 2, per(2 * sms), -1, red).total > half) bps = 1;
+  if ((size_t)win_layout_mix<C, MIX>(W, r, 2, per(2 * sms), -1, red, power).total > half) bps = 1;
   p.per_cta = per(bps * sms);
   p.grid = (heads + p.per_cta - 1) / p.per_cta;
   p.smem = bps == 2 ? half
                     : std::min((size_t)kMaxSmemPerCta,
                                (size_t)win_layout_mix<C, MIX>(W, r, kMaxStages, p.per_cta, -1,
-                                                              red).total);
+                                                              red, power).total);
   return p;
+}
+
+// Power compensator tokens: the step leaves full windows to power_end_kernel, launched right
+// after it on the same stream; forced flushes and the initial quantization run there too.
+template <class C>
+cudaError_t launch_power(WinOp op, const WinArgs& a, int heads, cudaStream_t st) {
+  const size_t pend = power_end_smem<C>(a.W, a.r), pq = power_scratch_bytes<C>();
+  cudaError_t e = cudaSuccess;
+  switch (op) {
+    case WinOp::Step: {
+      const StepPlan p = plan_step<C, false>(a.W, a.r, heads, true);
+      e = ensure_smem<window_step_kernel<C, false>>(p.smem);
+      if (e == cudaSuccess)
+        window_step_kernel<C, false><<<p.grid, kStepThreads, p.smem, st>>>(a, heads, p.per_cta,
+                                                                           (int)p.smem);
+      if (e == cudaSuccess) e = cudaGetLastError();
+      if (e == cudaSuccess) e = ensure_smem<power_end_kernel<C, 2>>(pend);
+      if (e == cudaSuccess) power_end_kernel<C, 2><<<heads, kThreads, pend, st>>>(a);
+      break;
+    }
+    case WinOp::Flush:
+      e = ensure_smem<power_end_kernel<C, 0>>(pend);
+      if (e == cudaSuccess) power_end_kernel<C, 0><<<heads, kThreads, pend, st>>>(a);
+      break;
+    case WinOp::Quantize:
+      e = ensure_smem<power_end_kernel<C, 3>>(pq);
+      if (e == cudaSuccess) power_end_kernel<C, 3><<<heads, kThreads, pq, st>>>(a);
+      break;
+    case WinOp::Materialize: {
+      const size_t sm1 = win_layout<C>(a.W, a.r, 1, 0, -1, true, true).total;
+      e = ensure_smem<window_state_kernel<C, 1, false>>(sm1);
+      if (e == cudaSuccess) window_state_kernel<C, 1, false><<<heads, kThreads, sm1, st>>>(a);
+      break;
+    }
+  }
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
 }
 
 template <class C, bool MIX = false>
 cudaError_t launch_window_cfg(WinOp op, const WinArgs& a, int heads, cudaStream_t st) {
+  if constexpr (!MIX && !C::SMOOTH && C::MMA) {
+    if (a.comp_k) return launch_power<C>(op, a, heads, st);
+  }
   size_t smem1 = win_layout<C>(a.W, a.r, 1, 0).total;
   if constexpr (MIX) smem1 = std::max(smem1, (size_t)win_layout<Int4Of<C>>(a.W, a.r, 1, 0).total);
   cudaError_t e = cudaSuccess;

@@ -90,7 +90,7 @@ __host__ __device__ constexpr uint32_t align128(uint32_t x) { return (x + 127u) 
 // coefficients, reduction space) and, for the persistent step kernel, the pos / gate / beta of
 // its whole head range.
 struct WinLayout {
-  uint32_t codes, scales, bk, bu, bL, cidx, cu, q, k, v, g, sexp, stage_bytes;  // within a stage
+  uint32_t codes, scales, bk, bu, bL, cidx, cu, ck, q, k, v, g, sexp, stage_bytes;  // within a stage
   uint32_t bars, stage0, vec, coef, red, tc, harr, total;                 // within the CTA
 };
 
@@ -105,11 +105,13 @@ __host__ __device__ constexpr uint32_t tc_scratch_bytes(int Wr) {
 // tensor-core scratch, the pos / gate / beta of the CTA's heads), then `nstages` stages whose
 // buffered-pair regions hold `cap` rows (a multiple of 16, at most W rounded up to 16; -1 means
 // that maximum). The kernels only ever read or write pair rows below the stage's cap. With
-// `smooth` a stage also holds the head's D smoothing exponents.
+// `smooth` a stage also holds the head's D smoothing exponents; with `power` the r compensator
+// token keys.
 __host__ __device__ inline WinLayout win_layout(int D, int code_bytes, int nscales, int act_size,
                                                 int buf_size, bool diag, int W, int r,
                                                 int nstages, int per_cta, int cap = -1,
-                                                bool red = true, bool smooth = false) {
+                                                bool red = true, bool smooth = false,
+                                                bool power = false) {
   // buffer rows rounded up to 16: the mma k-steps read (zero-filled) rows past the window
   const int Wp = (W + 3) & ~3, rp = (r + 3) & ~3, Wr = (W + 15) & ~15;
   if (cap < 0) cap = Wr;
@@ -128,7 +130,8 @@ __host__ __device__ inline WinLayout win_layout(int D, int code_bytes, int nscal
   L.bL = align128(L.bu + (uint32_t)cap * D * buf_size);
   L.cidx = align128(L.bL + 4u * (diag ? (uint32_t)cap * D : (uint32_t)Wp));
   L.cu = align128(L.cidx + 4u * rp);
-  L.q = align128(L.cu + 4u * r * D);
+  L.ck = align128(L.cu + 4u * r * D);
+  L.q = align128(L.ck + (power ? 4u * r * D : 0u));
   L.k = align128(L.q + (uint32_t)D * act_size);
   L.v = align128(L.k + (uint32_t)D * act_size);
   L.g = align128(L.v + (uint32_t)D * act_size);
@@ -140,10 +143,11 @@ __host__ __device__ inline WinLayout win_layout(int D, int code_bytes, int nscal
 
 template <class C>
 __host__ __device__ inline WinLayout win_layout(int W, int r, int nstages, int per_cta,
-                                                int cap = -1, bool red = true) {
+                                                int cap = -1, bool red = true,
+                                                bool power = false) {
   return win_layout(C::D, C::CODE_BYTES, C::NSCALES, (int)sizeof(typename C::Act),
                     (int)sizeof(typename C::Buf), C::DIAG, W, r, nstages, per_cta, cap, red,
-                    C::SMOOTH);
+                    C::SMOOTH, power);
 }
 
 // The int4 (group 32) configuration that shares C's head size, gate and dtypes, and the shared-
@@ -154,9 +158,10 @@ using Int4Of = WinCfg<C::D, C::DIAG, true, typename C::Act, typename C::Buf>;
 
 template <class C, bool MIX>
 __host__ __device__ inline WinLayout win_layout_mix(int W, int r, int nstages, int per_cta,
-                                                    int cap = -1, bool red = true) {
+                                                    int cap = -1, bool red = true,
+                                                    bool power = false) {
   if constexpr (!MIX) {
-    return win_layout<C>(W, r, nstages, per_cta, cap, red);
+    return win_layout<C>(W, r, nstages, per_cta, cap, red, power);
   } else {
     return win_layout(C::D, C::CODE_BYTES, Int4Of<C>::NSCALES, (int)sizeof(typename C::Act),
                       (int)sizeof(typename C::Buf), C::DIAG, W, r, nstages, per_cta, cap, red);
@@ -198,6 +203,7 @@ struct WinArgs {
   uint32_t scale_stride;   // scales (floats) per head
   int H, W, r;
   int8_t* smooth_exp;      // residual smoothing: [heads][D] column exponents, else null
+  float* comp_k;           // power compensator tokens: [heads][r][D] keys, else null
 };
 
 // 2^e for an integer e in [-126, 127], from the exponent bits (exact).
@@ -247,7 +253,7 @@ static __device__ __align__(128) uint8_t g_zero_rows[kZeroRowBytes];
 template <class C>
 __device__ __forceinline__ void stage_issue(const WinArgs& a, const WinLayout& L, uint8_t* st,
                                             uint64_t* bar, int head, int P, bool with_io,
-                                            int part = -1, int zrows = 0) {
+                                            int part = -1, int zrows = 0, bool full = false) {
   // part -1: every copy; part 0: codes, scales, q, k; part 1: the rest (two issuers, each
   // arriving once on a barrier that expects two arrivals). zrows > 0 (with part != 0) also
   // copies zeros over the write-vector rows P .. P + zrows - 1 of the stage.
@@ -255,7 +261,7 @@ __device__ __forceinline__ void stage_issue(const WinArgs& a, const WinLayout& L
   using Buf = typename C::Buf;
   constexpr int D = C::D;
   const int W = a.W, r = a.r, Wp = (W + 3) & ~3, rp = (r + 3) & ~3;
-  if (P < 0 || P >= W) {
+  if (P < 0 || P > W || (P == W && !full)) {  // full: a window end of all W pairs
     mbar_arrive_expect_tx(bar, 0);
     return;
   }
@@ -269,6 +275,7 @@ __device__ __forceinline__ void stage_issue(const WinArgs& a, const WinLayout& L
   if (p1) {
     if (P > 0) bytes += (uint32_t)P * D * (sizeof(Act) + sizeof(Buf)) + lbytes;
     if (r > 0) bytes += 4u * rp + 4u * r * D;
+    if (r > 0 && a.comp_k) bytes += 4u * r * D;
     if (with_io) bytes += D * sizeof(Act) + (C::DIAG ? 4u * D : 0u);
     bytes += (uint32_t)zrows * D * sizeof(Buf);
   }
@@ -294,6 +301,7 @@ __device__ __forceinline__ void stage_issue(const WinArgs& a, const WinLayout& L
     if (r > 0) {
       bulk_g2s(st + L.cidx, a.comp_idx + (size_t)head * rp, 4u * rp, bar);
       bulk_g2s(st + L.cu, a.comp_u + (size_t)head * r * D, 4u * r * D, bar);
+      if (a.comp_k) bulk_g2s(st + L.ck, a.comp_k + (size_t)head * r * D, 4u * r * D, bar);
     }
     if (with_io) {
       bulk_g2s(st + L.v, static_cast<const Act*>(a.v) + (size_t)head * D, D * sizeof(Act), bar);
@@ -336,6 +344,7 @@ struct WindowTile {
   const float* fac;
   const int32_t* cidx;
   const float* cu;
+  const float* ck;     // power tokens: keys [r][D] (null: column tokens, keys e_{cidx})
   const float* colexp;
   const int8_t* sexp;  // smoothing exponents of the frozen codes (SMOOTH only)
   int npairs, r;
@@ -373,6 +382,16 @@ struct WindowTile {
       for (int b = 0; b < TC; ++b) acc[a][b] = s * cv[b] * cf[b];
     }
     for (int c = 0; c < r; ++c) {
+      if (ck) {  // token cu_c (ck_c * e^{L_end})^T
+#pragma unroll
+        for (int b = 0; b < TC; ++b) {
+          const float kd = ck[c * D + c0 + b] * ce[b];
+#pragma unroll
+          for (int a = 0; a < TR; ++a)
+            acc[a][b] = fmaf(cu[c * D + ps * C::RPASS + rg * TR + a], kd, acc[a][b]);
+        }
+        continue;
+      }
       const int j = cidx[c];
       if (j / TC == cg) {
 #pragma unroll
@@ -596,7 +615,7 @@ __device__ __forceinline__ void prepare_window_end(uint8_t* st, const WinLayout&
 template <class C>
 __device__ __forceinline__ WindowTile<C> window_tile(const uint8_t* st, const WinLayout& L,
                                                      int npairs, int r, const float* colexp,
-                                                     const float* fac) {
+                                                     const float* fac, bool power = false) {
   WindowTile<C> t;
   t.codes = st + L.codes;
   t.scales = reinterpret_cast<const float*>(st + L.scales);
@@ -606,6 +625,7 @@ __device__ __forceinline__ WindowTile<C> window_tile(const uint8_t* st, const Wi
   t.fac = fac;
   t.cidx = reinterpret_cast<const int32_t*>(st + L.cidx);
   t.cu = reinterpret_cast<const float*>(st + L.cu);
+  t.ck = power ? reinterpret_cast<const float*>(st + L.ck) : nullptr;
   t.colexp = colexp;
   t.sexp = reinterpret_cast<const int8_t*>(st + L.sexp);
   t.npairs = npairs;
@@ -879,7 +899,8 @@ __global__ void __launch_bounds__(kStepThreads, 2)
   }
   const bool mma = step_uses_mma<C>(a.W);
   const int Wr = (a.W + 15) & ~15;
-  const WinLayout L0 = win_layout_mix<C, MIX>(a.W, a.r, 0, per_cta, Wr, !mma);  // the scratch part
+  const bool power = a.comp_k != nullptr;  // power tokens: their keys ride in each stage
+  const WinLayout L0 = win_layout_mix<C, MIX>(a.W, a.r, 0, per_cta, Wr, !mma, power);  // scratch
   int32_t* hpos = reinterpret_cast<int32_t*>(sm + L0.harr);
   float* hg = reinterpret_cast<float*>(hpos + per_cta);
   float* hb = hg + per_cta;
@@ -909,8 +930,9 @@ __global__ void __launch_bounds__(kStepThreads, 2)
   const int cap = mma ? min(Wr, (*pmax + 16) & ~15) : Wr;
   const int nstages =
       min(kMaxStages, (smem - (int)L0.stage0) /
-                          (int)win_layout_mix<C, MIX>(a.W, a.r, 1, per_cta, cap, !mma).stage_bytes);
-  const WinLayout L = win_layout_mix<C, MIX>(a.W, a.r, nstages, per_cta, cap, !mma);
+                          (int)win_layout_mix<C, MIX>(a.W, a.r, 1, per_cta, cap, !mma, power)
+                              .stage_bytes);
+  const WinLayout L = win_layout_mix<C, MIX>(a.W, a.r, nstages, per_cta, cap, !mma, power);
   // a head's stage copies and step in its own format (both fit the mixed layout)
   auto issue = [&](uint8_t* st, uint64_t* bar, int head, int P, int zrows) {
     if constexpr (MIX) {
@@ -1019,7 +1041,8 @@ __global__ void __launch_bounds__(kStepThreads, 2)
 template <class C, int MODE>
 __device__ __forceinline__ void window_state_body(const WinArgs& a, uint8_t* sm, int head) {
   constexpr int D = C::D;
-  const WinLayout L = win_layout<C>(a.W, a.r, 1, 0);
+  const bool power = a.comp_k != nullptr;
+  const WinLayout L = win_layout<C>(a.W, a.r, 1, 0, -1, true, power);
   const int tid = threadIdx.x;
   const int W = a.W, r = a.r;
   const int P = a.pos[head];
@@ -1055,7 +1078,7 @@ __device__ __forceinline__ void window_state_body(const WinArgs& a, uint8_t* sm,
   csync();
   prepare_window_end<C>(st, L, P, Lend, Ls, colexp, fac);
   csync();
-  const WindowTile<C> tile = window_tile<C>(st, L, P, r, colexp, fac);
+  const WindowTile<C> tile = window_tile<C>(st, L, P, r, colexp, fac, power);
   if constexpr (MODE == 0) {
     requantize_store<C>(tile, r, a.codes + (size_t)head * a.code_stride,
                         a.scales + (size_t)head * a.scale_stride,
@@ -1091,6 +1114,227 @@ __global__ void __launch_bounds__(kThreads) window_state_kernel(const WinArgs a)
     }
   }
   window_state_body<C, MODE>(a, sm, head);
+}
+
+// ------------------------------------------------------------------------------------------
+// Power compensator tokens: the window end (MODE 0: forced flush of the selected heads with
+// pos > 0; MODE 2: heads a decode step left full, pos == W) and the initial quantization
+// (MODE 3, from S_in). One CTA per head: the state materialised in shared memory as fp32
+// [D][D + 1], the tokens found by subspace iteration on it (as the header states: start from
+// the r key columns of largest L2 norm, ties to the lower index; six times X <- orth(S^T S X),
+// modified Gram-Schmidt in column order; keys x_c, values S x_c), the residual S (I - X X^T)
+// quantized like any other state.
+// ------------------------------------------------------------------------------------------
+constexpr int kPowerIters = 6;
+
+// Reads a [D][ld] fp32 tile of shared memory in the requantiser's tile mapping.
+template <class C>
+struct SmemTile {
+  const float* S;
+  int ld;
+  __device__ __forceinline__ void operator()(int ps, float (&acc)[C::TR][C::TC]) const {
+    const int tid = threadIdx.x, cg = tid % C::CG, rg = tid / C::CG;
+#pragma unroll
+    for (int a = 0; a < C::TR; ++a) {
+      const int row = ps * C::RPASS + rg * C::TR + a;
+#pragma unroll
+      for (int b = 0; b < C::TC; ++b) acc[a][b] = S[row * ld + cg * C::TC + b];
+    }
+  }
+};
+
+// Shared memory of power_end_kernel: the state tile, keys X and products Y ([r][D] each), 512
+// floats of scratch, then (window ends) a one-stage window layout.
+template <class C>
+__host__ __device__ constexpr uint32_t power_scratch_bytes() {
+  return align128(4u * (C::D * (C::D + 1) + 2 * GDN_MAX_COMPENSATORS * C::D + 512));
+}
+template <class C>
+__host__ __device__ inline uint32_t power_end_smem(int W, int r) {
+  return power_scratch_bytes<C>() + win_layout<C>(W, r, 1, 0, -1, true, true).total;
+}
+
+// Warp sum of a value.
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+// The tokens of the state Sm ([D][ld] in shared memory): writes keys and values to HBM and
+// leaves the residual in Sm. Called by all threads; r >= 1.
+template <class C>
+__device__ void power_tokens(float* Sm, int ld, int r, float* X, float* Y, float* scr,
+                             float* g_ck, float* g_cu) {
+  constexpr int D = C::D;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int* sel = reinterpret_cast<int*>(scr + D);
+  if (tid < D) {  // squared column norms
+    float s2 = 0.f;
+    for (int i = 0; i < D; ++i) s2 = fmaf(Sm[i * ld + tid], Sm[i * ld + tid], s2);
+    scr[tid] = s2;
+  }
+  csync();
+  if (warp == 0) {  // start columns: largest norm first, ties to the lower index
+    for (int c = 0; c < r; ++c) {
+      float bv = -2.f;
+      int bj = D;
+      for (int j = lane; j < D; j += 32)
+        if (scr[j] > bv) { bv = scr[j]; bj = j; }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
+        if (ov > bv || (ov == bv && oj < bj)) { bv = ov; bj = oj; }
+      }
+      if (lane == 0) {
+        sel[c] = bj;
+        scr[bj] = -1.f;  // taken (norms are >= 0)
+      }
+      __syncwarp();
+    }
+  }
+  csync();
+  for (int e = tid; e < r * D; e += C::NT) X[e] = (e % D) == sel[e / D] ? 1.f : 0.f;
+  csync();
+  auto times_S = [&]() {  // Y = S X: thread (row tid % D) for tokens tid / D, + 2, ...
+    const int i = tid % D;
+    for (int c = tid / D; c < r; c += C::NT / D) {
+      float acc = 0.f;
+      for (int j = 0; j < D; ++j) acc = fmaf(Sm[i * ld + j], X[c * D + j], acc);
+      Y[c * D + i] = acc;
+    }
+  };
+  for (int it = 0; it < kPowerIters; ++it) {
+    times_S();
+    csync();
+    {  // X = S^T Y: thread (column tid % D)
+      const int j = tid % D;
+      for (int c = tid / D; c < r; c += C::NT / D) {
+        float acc = 0.f;
+        for (int i = 0; i < D; ++i) acc = fmaf(Sm[i * ld + j], Y[c * D + i], acc);
+        X[c * D + j] = acc;
+      }
+    }
+    csync();
+    if (warp == 0) {  // modified Gram-Schmidt over the columns in order
+      for (int c = 0; c < r; ++c) {
+        float xc[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) xc[m] = X[c * D + lane + 32 * m];
+        for (int p = 0; p < c; ++p) {
+          float d = 0.f;
+#pragma unroll
+          for (int m = 0; m < 4; ++m) d = fmaf(xc[m], X[p * D + lane + 32 * m], d);
+          d = warp_sum(d);
+#pragma unroll
+          for (int m = 0; m < 4; ++m) xc[m] = fmaf(-d, X[p * D + lane + 32 * m], xc[m]);
+        }
+        float n2 = 0.f;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) n2 = fmaf(xc[m], xc[m], n2);
+        const float n = __fsqrt_rn(warp_sum(n2));
+#pragma unroll
+        for (int m = 0; m < 4; ++m) X[c * D + lane + 32 * m] = n > 0.f ? __fdiv_rn(xc[m], n) : 0.f;
+        __syncwarp();
+      }
+    }
+    csync();
+  }
+  times_S();  // the values S x_c
+  csync();
+  for (int e = tid; e < r * D; e += C::NT) {
+    g_ck[e] = X[e];
+    g_cu[e] = Y[e];
+  }
+  for (int e = tid; e < D * D; e += C::NT) {  // residual S - sum_c u_c x_c^T
+    const int i = e / D, j = e % D;
+    float acc = Sm[i * ld + j];
+    for (int c = 0; c < r; ++c) acc = fmaf(-Y[c * D + i], X[c * D + j], acc);
+    Sm[i * ld + j] = acc;
+  }
+  csync();
+}
+
+template <class C, int MODE>
+__global__ void __launch_bounds__(kThreads) power_end_kernel(const WinArgs a) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  constexpr int D = C::D, LD = D + 1;
+  const int head = blockIdx.x, tid = threadIdx.x;
+  const int W = a.W, r = a.r;
+  float* Sm = reinterpret_cast<float*>(sm);
+  float* X = Sm + D * LD;
+  float* Y = X + GDN_MAX_COMPENSATORS * D;
+  float* scr = Y + GDN_MAX_COMPENSATORS * D;
+  float* g_ck = a.comp_k + (size_t)head * r * D;
+  float* g_cu = a.comp_u + (size_t)head * r * D;
+  if constexpr (MODE == 3) {
+    const float* src = a.S_in + (size_t)head * D * D;
+    for (int e = tid; e < D * D / 4; e += C::NT) {
+      const float4 f = reinterpret_cast<const float4*>(src)[e];
+      const int i = (4 * e) / D, j = (4 * e) % D;
+      Sm[i * LD + j] = f.x;
+      Sm[i * LD + j + 1] = f.y;
+      Sm[i * LD + j + 2] = f.z;
+      Sm[i * LD + j + 3] = f.w;
+    }
+    csync();
+  } else {
+    const int P = a.pos[head];
+    if (MODE == 2) {
+      if (P != W) return;  // this head's window is not full
+    } else {
+      if (P < 0 || P >= W) {
+        if (tid == 0) report(a.status, GDN_DEVICE_BAD_POS);
+        return;
+      }
+      if (P == 0) return;
+      if (a.seq_mask && a.seq_mask[head / a.H] == 0) return;
+    }
+    uint8_t* wsm = sm + power_scratch_bytes<C>();
+    const WinLayout L = win_layout<C>(W, r, 1, 0, -1, true, true);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(wsm + L.bars);
+    uint8_t* st = wsm + L.stage0;
+    if (tid == 0) {
+      mbar_init(bar, 1);
+      fence_barrier_init();
+      stage_issue<C>(a, L, st, bar, head, P, false, -1, 0, true);
+    }
+    csync();
+    if (!stage_wait(a, bar, 0)) return;
+    float* vec = reinterpret_cast<float*>(wsm + L.vec);
+    float *Lend = vec, *colexp = vec + D;
+    float* fac = reinterpret_cast<float*>(wsm + L.coef);
+    const float* s_bL = reinterpret_cast<const float*>(st + L.bL);
+    float Ls = 0.f;
+    if constexpr (C::DIAG) {
+      for (int j = tid; j < D; j += C::NT) Lend[j] = P > 0 ? s_bL[(P - 1) * D + j] : 0.f;
+    } else {
+      Ls = P > 0 ? s_bL[P - 1] : 0.f;
+    }
+    csync();
+    prepare_window_end<C>(st, L, P, Lend, Ls, colexp, fac);
+    csync();
+    const WindowTile<C> tile = window_tile<C>(st, L, P, r, colexp, fac, true);
+    const int cg = tid % C::CG, rg = tid / C::CG;
+    float acc[C::TR][C::TC];
+    for (int ps = 0; ps < C::NPASS; ++ps) {
+      tile(ps, acc);
+#pragma unroll
+      for (int aa = 0; aa < C::TR; ++aa)
+#pragma unroll
+        for (int b = 0; b < C::TC; ++b)
+          Sm[(ps * C::RPASS + rg * C::TR + aa) * LD + cg * C::TC + b] = acc[aa][b];
+    }
+    csync();  // (the stage's old tokens are read out before the new ones go to HBM)
+  }
+  if (r > 0) power_tokens<C>(Sm, LD, r, X, Y, scr, g_ck, g_cu);
+  SmemTile<C> tile{Sm, LD};
+  requantize_store<C>(tile, 0, a.codes + (size_t)head * a.code_stride,
+                      a.scales + (size_t)head * a.scale_stride, nullptr, nullptr, scr,
+                      reinterpret_cast<int32_t*>(scr + 256), nullptr);
+  if (tid < r) a.comp_idx[(size_t)head * ((r + 3) & ~3) + tid] = -1;  // (no key columns)
+  if (tid == 0) a.pos[head] = 0;
 }
 
 // ------------------------------------------------------------------------------------------

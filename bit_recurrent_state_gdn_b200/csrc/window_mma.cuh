@@ -53,7 +53,8 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, gid = lane >> 2, q4 = lane & 3;
   const int mi = lane >> 3, r8 = lane & 7;
   const int W = a.W, r = a.r, Wp = (W + 3) & ~3, Wr = (W + 15) & ~15, bcs = Wr + 8;
-  const bool flush = (P + 1 == W);
+  // (with power tokens a full window is left to the window-end kernel: pos becomes W)
+  const bool flush = (P + 1 == W) && a.comp_k == nullptr;
   const int Pp = (P + 15) & ~15;
 
   float* vec = reinterpret_cast<float*>(sm + L.vec);
@@ -233,7 +234,31 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
       const int i = P + (ty & 15);
       if (i < Pp) Bc[(ty >> 4) * bcs + i] = __float2bfloat16_rn(0.f);
     }
-    if (ty < r) {  // compensator pairs: key e_j entered at L = 0, so their coefficient is x[j]
+    if (a.comp_k) {
+      // power tokens, entered at L = 0: coefficients <ck_c, x>, <ck_c, y>, one warp a token
+      const float* s_ck = reinterpret_cast<const float*>(st + L.ck);
+      for (int c = wy; c < r; c += 4) {
+        float ax = 0.f, ay = 0.f;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int jj = lane + 32 * m;
+          float kd = s_ck[c * D + jj];
+          if constexpr (C::DIAG) kd *= fast_exp((P > 0 ? s_bL[(P - 1) * D + jj] : 0.f) + s_g[jj]);
+          ax = fmaf(kd, __bfloat162float(s_k[jj]), ax);
+          ay = fmaf(kd, __bfloat162float(s_q[jj]), ay);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          ax += __shfl_xor_sync(0xffffffffu, ax, off);
+          ay += __shfl_xor_sync(0xffffffffu, ay, off);
+        }
+        if (lane == 0) {
+          const float e = C::DIAG ? 1.f : fast_exp(Ls);
+          ca[W + c] = e * ax;
+          cb[W + c] = e * ay;
+        }
+      }
+    } else if (ty < r) {  // compensator pairs: key e_j entered at L = 0, coefficient x[j]
       const int j = s_cidx[ty] & (D - 1);
       float e;
       if constexpr (C::DIAG) e = fast_exp((P > 0 ? s_bL[(P - 1) * D + j] : 0.f) + s_g[j]);

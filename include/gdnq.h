@@ -69,6 +69,25 @@ typedef enum { GDN_DTYPE_F32 = 0, GDN_DTYPE_BF16 = 1 } gdn_dtype;
 /* Largest compensator count per head. */
 #define GDN_MAX_COMPENSATORS 16
 
+/*
+ * How the r compensator tokens are chosen at every quantization ("LeapQuant ..." Abstract: the
+ * state's largest outliers are kept as a few high-precision compensator tokens that share the
+ * update path of real tokens; the page gives no rule -- both rules are readings):
+ *   GDN_COMP_COLUMNS  the r key columns of largest max-abs (ties: lower index); token c has key
+ *                     e_{comp_idx[c]} and value that column.
+ *   GDN_COMP_POWER    the state's dominant r-dimensional key subspace, by subspace iteration:
+ *                     start from the r key columns of largest L2 norm (ties: lower index), six
+ *                     times X <- orth(S^T S X) (modified Gram-Schmidt over the columns in order;
+ *                     a column of length 0 stays 0); token c has key x_c (comp_k[c], unit
+ *                     length) and value S x_c, and the residual S (I - X X^T) is quantized.
+ *                     Built for d = 128, bf16 activations and buffers, INT8 / INT4_G32 states
+ *                     without smoothing, W <= 64 (GDN_ERR_UNSUPPORTED elsewhere). A decode step
+ *                     whose window fills leaves it full (pos = W inside the call) and a second
+ *                     kernel of the same call runs the window end, so pos is back to 0 when the
+ *                     call's work is done.
+ */
+typedef enum { GDN_COMP_COLUMNS = 0, GDN_COMP_POWER = 1 } gdn_comp_rule;
+
 typedef struct {
     int32_t B, H;      /* sequences, heads per sequence (>= 0) */
     int32_t d_k, d_v;  /* head sizes; this build: d_k == d_v in {16, 128} */
@@ -80,6 +99,7 @@ typedef struct {
     int32_t buf_dtype; /* gdn_dtype of the buffered write vectors u */
     int32_t smooth;    /* gdn_smoothing: residual smoothing at every quantization (INT8 and
                           INT4_G32 states; 0 elsewhere) */
+    int32_t comp_rule; /* gdn_comp_rule of the compensator tokens (0: columns) */
 } gdn_config;
 
 /*
@@ -110,8 +130,10 @@ typedef enum { GDN_SMOOTH_NONE = 0, GDN_SMOOTH_POW2_COLUMNS = 1 } gdn_smoothing;
  *   buf_u    buf   [B][H][W][D]        buffered write vectors u_i = beta_i (v_i - w_i)
  *   buf_L    fp32  [B][H][Wp]          (scalar gate) cumulative log-gate of each pair
  *            fp32  [B][H][W][D]        (diagonal gate) the same per key channel
- *   comp_idx int32 [B][H][rp]          key column of each compensator pair (r > 0 only)
- *   comp_u   fp32  [B][H][r][D]        value column of each compensator pair (r > 0 only)
+ *   comp_idx int32 [B][H][rp]          key column of each compensator pair (r > 0, columns rule)
+ *   comp_u   fp32  [B][H][r][D]        value of each compensator token (r > 0 only)
+ *   comp_k   fp32  [B][H][r][D]        key of each compensator token (r > 0, power rule only;
+ *                                       16-byte aligned)
  *   pos      int32 [B][H]              pairs already in the window, 0 <= pos < W
  *   status   int32 [1], optional       device word the kernels OR GDN_DEVICE_* bits into
  *   head_fmt int8  [B][H]              (GDN_FMT_MIXED only) GDN_FMT_INT8 or GDN_FMT_INT4_G32 for
@@ -132,8 +154,9 @@ typedef enum { GDN_SMOOTH_NONE = 0, GDN_SMOOTH_POW2_COLUMNS = 1 } gdn_smoothing;
  * copy each and read eight consecutive rows at one column without bank conflicts.
  * gdn_state_materialize returns the logical state in plain row-major order.
  * The logical state of a head with P = pos pairs and L = buf_L[P-1] (0 when P == 0) is
- *   S = dequant(codes, scales) Diag(2^e) Diag(e^L) + sum_c comp_u[c] (e_{comp_idx[c]} e^{L})^T
- *       + sum_{i<P} buf_u[i] (buf_k[i] * e^{L - buf_L[i]})^T.
+ *   S = dequant(codes, scales) Diag(2^e) Diag(e^L) + sum_c comp_u[c] (ck_c * e^{L})^T
+ *       + sum_{i<P} buf_u[i] (buf_k[i] * e^{L - buf_L[i]})^T,
+ * ck_c = e_{comp_idx[c]} (columns rule) or comp_k[c] (power rule).
  * (Diag(2^e) only with smoothing.) Entries of buf_k / buf_u / buf_L at index >= pos are scratch
  * and never read.
  */
@@ -149,6 +172,7 @@ typedef struct {
     int32_t* status;
     const int8_t* head_fmt;
     int8_t* smooth_exp;
+    float* comp_k;
 } gdn_state;
 
 /* Byte sizes of each buffer of gdn_state for the whole batch (0 where unused), and the dynamic
@@ -158,6 +182,7 @@ typedef struct {
     size_t smem_step;
     size_t head_fmt;
     size_t smooth_exp;
+    size_t comp_k;
 } gdn_sizes;
 
 /* Checks cfg and fills *out. Host-only: touches no device. The buffers are the parts of the

@@ -22,7 +22,7 @@ from workloads import Workload, decode_inputs, outlier_scales, step_inputs, torc
 
 def cfg_of(wl: Workload):
     return gdn.make_config(wl.B, wl.H, wl.D, wl.W, wl.r, wl.gate, wl.fmt, wl.act, wl.buf,
-                           smooth=wl.smooth)
+                           smooth=wl.smooth, comp_rule=wl.comp_rule)
 
 
 def gpu_warmup(wl: Workload, device="cuda", draw=None) -> torch.Tensor:
@@ -102,7 +102,7 @@ def gpu_run(wl: Workload, device="cuda", T: int | None = None, inputs=None, S0=N
 def _o2(wl: Workload, q, k, v, g, beta, S0, flush_mask, **kw):
     return oracle.o2_run(q, k, v, g, beta, W=wl.W, r=wl.r, fmt=wl.fmt, S0=S0,
                          round_storage=True, buf_round=wl.buf, flush_mask=flush_mask,
-                         smooth=wl.smooth, **kw)
+                         smooth=wl.smooth, comp_rule=wl.comp_rule, **kw)
 
 
 def oracle_run(wl: Workload, heads: np.ndarray, inputs: dict, S0: np.ndarray, flush_mask=None):

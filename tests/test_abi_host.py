@@ -85,6 +85,14 @@ BAD_CONFIGS = [
     ("window too big", dict(W=5000), _abi.GDN_ERR_UNSUPPORTED),
     ("B<0", dict(B=-1), _abi.GDN_ERR_INVALID_ARG),
     ("smoothing of a mixed state", dict(fmt="mixed", smooth=True), _abi.GDN_ERR_UNSUPPORTED),
+    ("power tokens with smoothing", dict(r=4, comp_rule="power", smooth=True),
+     _abi.GDN_ERR_UNSUPPORTED),
+    ("power tokens, W = 65", dict(r=4, comp_rule="power", W=65), _abi.GDN_ERR_UNSUPPORTED),
+    ("power tokens, D = 16", dict(D=16, r=2, comp_rule="power"), _abi.GDN_ERR_UNSUPPORTED),
+    ("power tokens, fp32 buffers", dict(r=2, comp_rule="power", buf="f32"),
+     _abi.GDN_ERR_UNSUPPORTED),
+    ("power tokens, mixed widths", dict(r=2, comp_rule="power", fmt="mixed"),
+     _abi.GDN_ERR_UNSUPPORTED),
 ]
 
 
@@ -104,7 +112,7 @@ def test_raw_field_errors(lib):
     cfg = _cfg()
     assert lib.gdn_state_sizes(ctypes.byref(cfg), None) == _abi.GDN_ERR_INVALID_ARG
     for field, val in (("gate", 7), ("fmt", 9), ("act_dtype", 3), ("buf_dtype", -1),
-                       ("smooth", 2), ("smooth", -1)):
+                       ("smooth", 2), ("smooth", -1), ("comp_rule", 2), ("comp_rule", -1)):
         c = _cfg()
         setattr(c, field, val)
         assert lib.gdn_state_sizes(ctypes.byref(c), ctypes.byref(out)) == _abi.GDN_ERR_INVALID_ARG
@@ -145,6 +153,21 @@ def test_smoothing_sizes_and_exponent_pointer(fmt, lib):
         rc = lib.gdn_decode_window_step(ctypes.byref(cfg), ctypes.byref(st), q, q, q, q, q, q, None)
         assert rc == _abi.GDN_ERR_INVALID_ARG
         assert b"smooth_exp" in lib.gdn_last_error()
+
+
+def test_power_token_keys_sized_and_required(lib):
+    """Power tokens keep r keys of D floats per head next to the values; the key pointer is
+    required (16-byte aligned) only for the power rule with r > 0."""
+    cfg = _cfg(r=4, comp_rule="power")
+    sz = gdn.gdn_state_sizes(cfg)
+    assert sz.comp_k == 6 * 4 * 128 * 4 and sz.comp_u == sz.comp_k
+    assert gdn.gdn_state_sizes(_cfg(r=4)).comp_k == 0
+    assert gdn.gdn_state_sizes(_cfg(r=0, comp_rule="power")).comp_k == 0
+    q = ctypes.c_void_p(0x900000)
+    for st in (_fake_state(null="comp_k"), _fake_state(misalign="comp_k")):
+        rc = lib.gdn_decode_window_step(ctypes.byref(cfg), ctypes.byref(st), q, q, q, q, q, q, None)
+        assert rc == _abi.GDN_ERR_INVALID_ARG
+        assert b"comp_k" in lib.gdn_last_error()
 
 
 def test_compensator_pointers_needed_only_with_r(lib):

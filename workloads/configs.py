@@ -21,6 +21,7 @@ class Workload:
     warmup: int = 512      # fp32 recurrence tokens that make the initial state (0: zero state)
     seed: int = 0
     smooth: bool = False   # residual smoothing at every quantization
+    comp_rule: str = "columns"  # compensator tokens: "columns" or "power"
 
     @property
     def heads(self) -> int:

@@ -77,7 +77,7 @@ def step_bytes(wl, P: int) -> int:
     codes = D * D // 2 if wl.fmt == "int4_g32" else D * D
     scales = 4 * D * (D // 32 if wl.fmt == "int4_g32" else 1)
     scales += D if wl.smooth else 0  # residual smoothing: one exponent byte per key column
-    comps = r * (4 + 4 * D)
+    comps = r * (4 + 4 * D) + (r * 4 * D if wl.comp_rule == "power" else 0)
     pair = D * act + D * buf + lbytes
     io_ = 4 * D * act + (4 * D if wl.gate == "diag" else 4) + 4 + 8  # q k v o, g, beta, pos r/w
     read = codes + scales + comps + P * pair
@@ -439,7 +439,17 @@ def main():
             "int4-serving": decode_leg(wl.with_(name="int4-serving", fmt="int4_g32"), dev, peak,
                                        cpu=False, inp=inp, S0=S0, o=o)}
         for name in ("kda", "gdn-mid", "gdn-long-int4"):
-            line["workloads"][name] = decode_leg(WORKLOADS[name], dev, peak, cpu=cpu)
+            line["workloads"][name] = decode_leg(WORKLOADS[name], dev, peak, cpu=cpu,
+                                                 quality=cpu and name == "kda")
+            torch.cuda.empty_cache()
+        # compensator tokens on the KDA workload: power tokens against column tokens, int8 and
+        # int4 (quality figures from each leg's own outputs)
+        kda = WORKLOADS["kda"]
+        for name, wk in (("kda-power", kda.with_(name="kda-power", comp_rule="power")),
+                         ("kda-int4", kda.with_(name="kda-int4", fmt="int4_g32")),
+                         ("kda-int4-power", kda.with_(name="kda-int4-power", fmt="int4_g32",
+                                                      comp_rule="power"))):
+            line["workloads"][name] = decode_leg(wk, dev, peak, cpu=False, quality=cpu)
             torch.cuda.empty_cache()
 
     # ---- chunkwise prefill of a prompt batch (its own workload) ----------------------------
@@ -508,10 +518,12 @@ def warm_states(wl, dev):
     return S0
 
 
-def decode_leg(wl, dev, peak, cpu: bool, inp=None, S0=None, o=None, cpu_heads: int = 256):
+def decode_leg(wl, dev, peak, cpu: bool, inp=None, S0=None, o=None, cpu_heads: int = 256,
+               quality: bool = False):
     """One decode workload on its own: its states quantized (untimed), then its T decode launches
     timed with CUDA events; the roofline of the average launch from the workload's algorithmic
-    bytes; with cpu, the oracle on a bounded sample of its heads."""
+    bytes; with cpu, the oracle on a bounded sample of its heads; with quality, the outputs'
+    error against the unquantized fp64 recurrence on its first sequences."""
     import numpy as np
     import torch
 
@@ -521,7 +533,8 @@ def decode_leg(wl, dev, peak, cpu: bool, inp=None, S0=None, o=None, cpu_heads: i
         inp = decode_inputs(wl, dev)
         S0 = warm_states(wl, dev)
         o = torch.empty_like(inp["q"])
-    cfg = gdn.make_config(wl.B, wl.H, wl.D, wl.W, wl.r, wl.gate, wl.fmt, wl.act, wl.buf)
+    cfg = gdn.make_config(wl.B, wl.H, wl.D, wl.W, wl.r, wl.gate, wl.fmt, wl.act, wl.buf,
+                          comp_rule=wl.comp_rule)
     st = gdn.GdnState.allocate(cfg, dev)
     gdn.gdn_state_quantize(cfg, S0, st)
     n0 = min(4, wl.T)
@@ -547,7 +560,8 @@ def decode_leg(wl, dev, peak, cpu: bool, inp=None, S0=None, o=None, cpu_heads: i
         traffic, src = profiled_traffic(os.path.join(ROOT, "profiles", f), KERNEL_SOURCES, key)
     out = {"value": wl.heads * wl.T / (ms / 1e3), "unit": UNIT, "ms_per_run": ms,
            "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "D": wl.D, "T": wl.T,
-                      "W": wl.W, "r": wl.r, "gate": wl.gate, "state": wl.fmt, "act": wl.act},
+                      "W": wl.W, "r": wl.r, "gate": wl.gate, "state": wl.fmt, "act": wl.act,
+                      "compensators": wl.comp_rule},
            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                         "frac": gbs / peak, "traffic": traffic, "traffic_source": src,
                         "algorithmic_bytes_per_launch": per_launch,
@@ -564,6 +578,8 @@ def decode_leg(wl, dev, peak, cpu: bool, inp=None, S0=None, o=None, cpu_heads: i
         out["cpu_baseline"] = {"value": hs, "unit": UNIT, "cores": cores, "kind": "oracle",
                                "sample": f"{n_seq * wl.H} heads (sequences 0..{n_seq - 1}) x "
                                          f"{wl.T} steps of the same inputs, {dt:.1f} s"}
+    if quality:
+        out["quality"] = quality_figure(wl, inp, o, dev, n_seq=4)
     del st
     return out
 
@@ -678,15 +694,17 @@ def prefill_leg(args, dev, name: str = "gdn-prefill", reps: int = 5):
     cfg = gdn.make_config(wl.B, wl.H, wl.D, gate=wl.gate, act="bf16")
     o = torch.empty_like(hm["q"])
     S = torch.zeros((wl.B, wl.H, wl.D, wl.D), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(gdn.gdn_prefill_workspace_bytes(cfg, L), 16), dtype=torch.uint8,
+                     device=dev)
     for _ in range(2):
-        gdn.gdn_prefill(cfg, hm["q"], hm["k"], hm["v"], hm["g"], hm["beta"], o, S)
+        gdn.gdn_prefill(cfg, hm["q"], hm["k"], hm["v"], hm["g"], hm["beta"], o, S, ws)
     torch.cuda.synchronize()
     ms = []
     for _ in range(reps):
         S.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        gdn.gdn_prefill(cfg, hm["q"], hm["k"], hm["v"], hm["g"], hm["beta"], o, S)
+        gdn.gdn_prefill(cfg, hm["q"], hm["k"], hm["v"], hm["g"], hm["beta"], o, S, ws)
         e1.record()
         torch.cuda.synchronize()
         ms.append(e0.elapsed_time(e1))
@@ -701,8 +719,9 @@ def prefill_leg(args, dev, name: str = "gdn-prefill", reps: int = 5):
     cpu = None if args.no_cpu else prefill_cpu_baseline(wl, inp, dev)
     kernel = ("prefill_kda_kernel (one CTA per head, two per SM, 16-token chunks, mma.sync)"
               if wl.gate == "diag" else
-              "prefill_tc_kernel (one CTA per head, 64-token chunks, tcgen05.mma with the state "
-              "in TMEM, TMA-staged tiles)")
+              "prefill_chunk_kernel (every 64-token chunk in parallel: scores, inverse, T and P "
+              "on tcgen05) + prefill_tc_kernel (one CTA per head: the state in TMEM, "
+              "tcgen05.mma, TMA-staged tiles)")
     return {"value": wl.heads * L / (t / 1e3), "unit": "head-tokens/s", "ms_per_launch": t,
             "cpu_baseline": cpu,
             "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "L": L, "D": wl.D,
@@ -846,9 +865,10 @@ def quality_figure(wl, inp, o, dev, n_seq: int = 8):
     got = o.reshape(wl.T, wl.heads, wl.D)[:, :n].double().cpu().numpy()
     err = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
     return {"o_rel_l2_vs_fp64_recurrence": err, "heads": n, "steps": wl.T,
-            "note": "%s windowed state (W = %d%s) against the fp64 recurrence with no "
-                    "quantization; GPU outputs in bf16"
-                    % (wl.fmt, wl.W, ", residual smoothing" if wl.smooth else "")}
+            "note": "%s windowed state (W = %d, r = %d %s tokens%s) against the fp64 recurrence "
+                    "with no quantization; GPU outputs in bf16"
+                    % (wl.fmt, wl.W, wl.r, wl.comp_rule,
+                       ", residual smoothing" if wl.smooth else "")}
 
 
 def pw_cpu_baseline(wl, Wp, inp, dev, n_seq: int = 4):

@@ -28,4 +28,4 @@ from .pw import (  # noqa: F401
     gdn_pw_state_sizes,
     make_pw_config,
 )
-from .prefill import gdn_prefill  # noqa: F401,E402
+from .prefill import gdn_prefill, gdn_prefill_workspace_bytes  # noqa: F401,E402

@@ -85,7 +85,8 @@ SIGNATURES = {
     "gdn_pw_decode_step": (_i32, [_PWC, _PWS] + [_vp] * 7),
     "gdn_pw_decode_steps": (_i32, [_PWC, _PWS, _i32] + [_vp] * 7),
     "gdn_pw_materialize": (_i32, [_PWC, _PWS, _vp, _vp]),
-    "gdn_prefill": (_i32, [ctypes.POINTER(gdn_config), _i32] + [_vp] * 8),
+    "gdn_prefill": (_i32, [ctypes.POINTER(gdn_config), _i32] + [_vp] * 8 + [_sz, _vp]),
+    "gdn_prefill_workspace_bytes": (_sz, [ctypes.POINTER(gdn_config), _i32]),
     "gdn_status_string": (ctypes.c_char_p, [_i32]),
     "gdn_last_error": (ctypes.c_char_p, []),
 }

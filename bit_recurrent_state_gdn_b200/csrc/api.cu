@@ -688,10 +688,8 @@ gdn_status gdn_pw_materialize(const gdn_pw_config* cfg, const gdn_pw_state* stat
   return GDN_OK;
 }
 
-gdn_status gdn_prefill(const gdn_config* cfg, int32_t L, const void* q, const void* k,
-                       const void* v, const float* g, const float* beta, void* o, float* S,
-                       gdn_stream_t stream) {
-  g_last_error[0] = 0;
+namespace {
+gdn_status check_prefill_config(const gdn_config* cfg) {
   if (!cfg) return fail(GDN_ERR_INVALID_ARG, "cfg is null");
   if (cfg->B < 0 || cfg->H < 0)
     return fail(GDN_ERR_INVALID_ARG, "B=%d, H=%d must be >= 0", cfg->B, cfg->H);
@@ -706,6 +704,22 @@ gdn_status gdn_prefill(const gdn_config* cfg, int32_t L, const void* q, const vo
     return fail(GDN_ERR_UNSUPPORTED, "prefill is built for d_k = d_v = 128");
   if (cfg->act_dtype != GDN_DTYPE_BF16)
     return fail(GDN_ERR_UNSUPPORTED, "prefill is built for bf16 activations");
+  return GDN_OK;
+}
+}  // namespace
+
+size_t gdn_prefill_workspace_bytes(const gdn_config* cfg, int32_t L) {
+  g_last_error[0] = 0;
+  if (check_prefill_config(cfg) != GDN_OK || L < 0) return 0;
+  return gdnq::prefill_workspace_bytes(cfg->gate == GDN_GATE_DIAG, heads_of(cfg), L);
+}
+
+gdn_status gdn_prefill(const gdn_config* cfg, int32_t L, const void* q, const void* k,
+                       const void* v, const float* g, const float* beta, void* o, float* S,
+                       void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
+  g_last_error[0] = 0;
+  gdn_status st0 = check_prefill_config(cfg);
+  if (st0 != GDN_OK) return st0;
   if (L < 0) return fail(GDN_ERR_INVALID_ARG, "L=%d must be >= 0", L);
   if (heads_of(cfg) == 0) return GDN_OK;
   if ((size_t)heads_of(cfg) * (size_t)L * 128 > (size_t)INT64_MAX / 4)
@@ -719,6 +733,13 @@ gdn_status gdn_prefill(const gdn_config* cfg, int32_t L, const void* q, const vo
     if ((st = need_ptr(g, "g", cfg->gate == GDN_GATE_DIAG ? 16 : 4)) != GDN_OK) return st;
     if ((st = need_ptr(beta, "beta", 4)) != GDN_OK) return st;
     if ((st = need_ptr(o, "o", 4)) != GDN_OK) return st;
+    const size_t need = gdnq::prefill_workspace_bytes(cfg->gate == GDN_GATE_DIAG, heads_of(cfg), L);
+    if (need > 0) {
+      if ((st = need_ptr(workspace, "workspace")) != GDN_OK) return st;
+      if (workspace_bytes < need)
+        return fail(GDN_ERR_INVALID_ARG, "workspace holds %zu bytes, the prompt needs %zu",
+                    workspace_bytes, need);
+    }
   }
   gdnq::PfArgs a;
   a.q = static_cast<const __nv_bfloat16*>(q);
@@ -728,6 +749,7 @@ gdn_status gdn_prefill(const gdn_config* cfg, int32_t L, const void* q, const vo
   a.beta = beta;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.S = S;
+  a.ws = static_cast<uint8_t*>(workspace);
   a.L = L;
   const cudaError_t e = gdnq::launch_prefill(a, (int)heads_of(cfg), cfg->gate == GDN_GATE_DIAG,
                                              (cudaStream_t)stream);

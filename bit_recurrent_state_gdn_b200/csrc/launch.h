@@ -46,6 +46,7 @@ cudaError_t launch_pw(PwOp op, const gdn_pw_config& cfg, const PwArgs& a, int he
 // Chunkwise prefill: one CTA per head; diag selects the per-key-channel gate (g [heads][L][128]).
 cudaError_t launch_prefill(const PfArgs& a, int heads, bool diag, cudaStream_t stream);
 size_t prefill_smem_bytes(bool diag);
+size_t prefill_workspace_bytes(bool diag, int64_t heads, int L);
 cudaError_t launch_baseline(const gdn_config& cfg, const BaseArgs& a, int heads,
                             cudaStream_t stream);
 

@@ -53,12 +53,25 @@ cudaError_t launch_prefill(const PfArgs& a, int heads, bool diag, cudaStream_t s
   cudaError_t e = token_map(&maps.q, a.q, a.L, heads);
   if (e == cudaSuccess) e = token_map(&maps.k, a.k, a.L, heads);
   if (e == cudaSuccess) e = token_map(&maps.v, a.v, a.L, heads);
+  if (e == cudaSuccess) e = ensure_smem<prefill_chunk_kernel>(ChunkLayout::ALLOC);
   if (e == cudaSuccess) e = ensure_smem<prefill_tc_kernel>(TcLayout::ALLOC);
+  if (e != cudaSuccess) return e;
+  // the state-independent part of every chunk (persistent CTAs), then each head's chunks in
+  // order
+  const int total = heads * ((a.L + kPfC - 1) / kPfC);
+  const int grid = std::min(total, kChunkCtasPerSm * num_sms());
+  prefill_chunk_kernel<<<grid, kPfThreads, ChunkLayout::ALLOC, st>>>(a, maps, total);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   prefill_tc_kernel<<<heads, kPfThreads, TcLayout::ALLOC, st>>>(a, maps);
   return cudaGetLastError();
 }
 
 size_t prefill_smem_bytes(bool diag) { return diag ? KdaLayout::TOTAL : TcLayout::ALLOC; }
+
+size_t prefill_workspace_bytes(bool diag, int64_t heads, int L) {
+  if (diag || heads <= 0 || L <= 0) return 0;
+  return (size_t)heads * (size_t)((L + kPfC - 1) / kPfC) * kPfRecBytes;
+}
 
 }  // namespace gdnq

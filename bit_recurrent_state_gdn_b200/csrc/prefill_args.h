@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cstdint>
 
 namespace gdnq {
 
@@ -13,6 +14,7 @@ struct PfArgs {
   const float* beta;
   __nv_bfloat16* o;        // [heads][L][128]
   float* S;                // [heads][128][128], in place
+  uint8_t* ws;             // scalar gate: [heads][ceil(L / 64)] chunk records (workspace)
   int L;
 };
 

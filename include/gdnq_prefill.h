@@ -42,7 +42,15 @@ extern "C" {
  *   o       device bf16 [B][H][L][D], written for every token.
  *   S       device fp32 [B][H][D][D], 16-byte aligned: the state before the prompt on entry, after
  *           it on return (row = value channel, column = key channel).
- * Arithmetic: products on tensor cores with fp32 accumulation; q, k, v enter exactly, every
+ *   workspace, workspace_bytes  device scratch the caller provides, 16-byte aligned, at least
+ *           gdn_prefill_workspace_bytes(cfg, L) bytes (none for the per-channel gate, where the
+ *           pointer may be NULL). The scalar gate keeps there, for every 64-token chunk, what
+ *           does not depend on the state (the chunk's T = (I + A)^{-1} Diag(beta) and decayed
+ *           scores P as split operand tiles, and its gates: 33,792 bytes), computed by a first
+ *           kernel over all chunks at once; the second kernel carries the state through the
+ *           chunks. Contents on entry are ignored; on return they are scratch.
+ * Arithmetic: products on tensor cores (tcgen05 for the scalar gate, the state in tensor memory)
+ * with fp32 accumulation; q, k, v enter exactly, every
  * fp32 operand (the state, the chunk's triangular inverse, the corrected values, the decayed
  * scores, keys and queries, the write vectors) as the sum of two bf16 parts; the triangular
  * inverse in fp32.
@@ -52,7 +60,11 @@ extern "C" {
  */
 gdn_status gdn_prefill(const gdn_config* cfg, int32_t L, const void* q, const void* k,
                        const void* v, const float* g, const float* beta, void* o, float* S,
-                       gdn_stream_t stream);
+                       void* workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+/* Bytes of workspace gdn_prefill needs for cfg and a prompt of L tokens (0 for the per-channel
+ * gate, for an empty batch or prompt, or for a cfg gdn_prefill rejects). Host-only. */
+size_t gdn_prefill_workspace_bytes(const gdn_config* cfg, int32_t L);
 
 #ifdef __cplusplus
 }

@@ -309,7 +309,7 @@ PF_BAD = [
 @pytest.mark.parametrize("name,kw,L,status", PF_BAD, ids=[b[0] for b in PF_BAD])
 def test_prefill_rejects_bad_arguments(name, kw, L, status, lib):
     cfg = _cfg(**kw)
-    assert lib.gdn_prefill(ctypes.byref(cfg), L, *([None] * 8)) == status
+    assert lib.gdn_prefill(ctypes.byref(cfg), L, *([None] * 8), 0, None) == status
     assert lib.gdn_last_error() != b""
 
 
@@ -319,9 +319,29 @@ def test_prefill_diag_gate_wants_16_byte_aligned_gates(lib):
     p = ctypes.c_void_p(1 << 20)
     args = [p, p, p, ctypes.c_void_p((1 << 20) + 8), p, p, p]
     cfg = _cfg(gate="diag")
-    assert lib.gdn_prefill(ctypes.byref(cfg), 8, *args, None) == _abi.GDN_ERR_INVALID_ARG
+    assert lib.gdn_prefill(ctypes.byref(cfg), 8, *args, None, 0, None) == _abi.GDN_ERR_INVALID_ARG
     assert b"g is not 16-byte aligned" in lib.gdn_last_error()
 
 
+def test_prefill_workspace_size_and_checks(lib):
+    """The scalar gate needs one 33,792-byte record per 64-token chunk of every head; the
+    per-channel gate none. A missing, misaligned or short workspace is refused before anything
+    is enqueued."""
+    cfg = _cfg(B=2, H=3)
+    assert lib.gdn_prefill_workspace_bytes(ctypes.byref(cfg), 200) == 6 * 4 * 33792
+    assert lib.gdn_prefill_workspace_bytes(ctypes.byref(cfg), 0) == 0
+    assert lib.gdn_prefill_workspace_bytes(ctypes.byref(_cfg(gate="diag")), 200) == 0
+    assert lib.gdn_prefill_workspace_bytes(ctypes.byref(_cfg(D=16)), 200) == 0
+    p = ctypes.c_void_p(1 << 20)
+    args = [p] * 7
+    need = 6 * 4 * 33792
+    for ws, size, msg in ((None, need, b"workspace is null"),
+                          (ctypes.c_void_p((1 << 20) + 8), need, b"workspace is not"),
+                          (p, need - 16, b"workspace holds")):
+        rc = lib.gdn_prefill(ctypes.byref(cfg), 200, *args, ws, size, None)
+        assert rc == _abi.GDN_ERR_INVALID_ARG
+        assert msg in lib.gdn_last_error(), lib.gdn_last_error()
+
+
 def test_prefill_empty_batch_is_a_noop(lib):
-    assert lib.gdn_prefill(ctypes.byref(_cfg(B=0)), 100, *([None] * 8)) == _abi.GDN_OK
+    assert lib.gdn_prefill(ctypes.byref(_cfg(B=0)), 100, *([None] * 8), 0, None) == _abi.GDN_OK

@@ -121,12 +121,15 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// e^x through the hardware base-2 exponential (flushes results below 2^-126 to zero).
-__device__ __forceinline__ float fast_exp(float x) {
+// 2^x on the hardware path (flushes results below 2^-126 to zero).
+__device__ __forceinline__ float exp2_hw(float x) {
   float y;
-  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x * 1.4426950408889634f));
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
   return y;
 }
+
+// e^x through the hardware base-2 exponential (flushes results below 2^-126 to zero).
+__device__ __forceinline__ float fast_exp(float x) { return exp2_hw(x * 1.4426950408889634f); }
 
 // rint of the correctly rounded quotient x / s (|x / s| <= 128), given inv = the correctly
 // rounded 1 / s. q = x * inv differs from x / s by at most 2 rounding errors of size

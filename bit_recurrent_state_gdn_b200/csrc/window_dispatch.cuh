@@ -39,9 +39,11 @@ inline int num_sms() {
   return n;
 }
 
-// Shape of a persistent step launch: two CTAs per SM when two stages of the largest window
-// position fit into half of an SM's shared memory, else one CTA per SM. Each CTA gets all the
-// shared memory that allows and sizes its stages itself (up to kMaxStages).
+// Shape of a persistent step launch: two CTAs per SM when one stage of the largest window
+// position fits into half of an SM's shared memory, else one CTA per SM. Each CTA gets all the
+// shared memory that allows and sizes its stages itself (up to kMaxStages). Two CTAs with one
+// stage each late in a window (the per-channel gate's stages hold fp32 gates per pair) beat one
+// CTA with two stages: the other CTA's head runs while a CTA waits for its copies.
 struct StepPlan {
   int grid, per_cta;
   size_t smem;
@@ -56,7 +58,7 @@ StepPlan plan_step(int W, int r, int heads, bool power = false) {
   StepPlan p;
   const size_t half = (size_t)kSmemPerSm / 2 - kReserved;
   int bps = 2;
-  if ((size_t)win_layout_mix<C, MIX>(W, r, 2, per(2 * sms), -1, red, power).total > half) bps = 1;
+  if ((size_t)win_layout_mix<C, MIX>(W, r, 1, per(2 * sms), -1, red, power).total > half) bps = 1;
   p.per_cta = per(bps * sms);
   p.grid = (heads + p.per_cta - 1) / p.per_cta;
   p.smem = bps == 2 ? half

@@ -1143,11 +1143,12 @@ struct SmemTile {
   }
 };
 
-// Shared memory of power_end_kernel: the state tile, keys X and products Y ([r][D] each), 512
-// floats of scratch, then (window ends) a one-stage window layout.
+// Shared memory of power_end_kernel: the state tile, keys X, products Y and the second half's
+// partial products ([D][16] each, token-minor), 512 floats of scratch, then (window ends) a
+// one-stage window layout.
 template <class C>
 __host__ __device__ constexpr uint32_t power_scratch_bytes() {
-  return align128(4u * (C::D * (C::D + 1) + 2 * GDN_MAX_COMPENSATORS * C::D + 512));
+  return align128(4u * (C::D * (C::D + 1) + 3 * GDN_MAX_COMPENSATORS * C::D + 512));
 }
 template <class C>
 __host__ __device__ inline uint32_t power_end_smem(int W, int r) {
@@ -1161,13 +1162,62 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
+// out = S in (TRANS: S^T in) for the token vectors in, both [D][xs] token-minor (xs a multiple
+// of 4, r <= xs). Thread t takes index n = t % D of the product and one half of the summation
+// index (t / D), four tokens at a time (one 16-byte load of the vectors per summation index,
+// a broadcast); the second half's partial sums meet the first's through `part`.
+template <class C, bool TRANS>
+__device__ __forceinline__ void power_matvec(const float* Sm, int ld, int r, int xs,
+                                             const float* in, float* out, float* part) {
+  constexpr int D = C::D;
+  static_assert(C::NT == 2 * D, "two threads per row or column");
+  const int tid = threadIdx.x, n = tid % D, h = tid / D;
+  const int m0 = h * (D / 2);
+  float acc[GDN_MAX_COMPENSATORS];
+#pragma unroll
+  for (int c = 0; c < GDN_MAX_COMPENSATORS; ++c) acc[c] = 0.f;
+#pragma unroll
+  for (int c0 = 0; c0 < GDN_MAX_COMPENSATORS; c0 += 4) {
+    if (c0 < r) {
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 8
+      for (int m = m0; m < m0 + D / 2; ++m) {
+        const float sv = TRANS ? Sm[m * ld + n] : Sm[n * ld + m];
+        const float4 v = *reinterpret_cast<const float4*>(in + m * xs + c0);
+        a0 = fmaf(sv, v.x, a0);
+        a1 = fmaf(sv, v.y, a1);
+        a2 = fmaf(sv, v.z, a2);
+        a3 = fmaf(sv, v.w, a3);
+      }
+      acc[c0] = a0;
+      acc[c0 + 1] = a1;
+      acc[c0 + 2] = a2;
+      acc[c0 + 3] = a3;
+      if (h == 1) *reinterpret_cast<float4*>(part + n * xs + c0) = make_float4(a0, a1, a2, a3);
+    }
+  }
+  csync();
+  if (h == 0) {
+#pragma unroll
+    for (int c0 = 0; c0 < GDN_MAX_COMPENSATORS; c0 += 4) {
+      if (c0 < r) {
+        const float4 q = *reinterpret_cast<const float4*>(part + n * xs + c0);
+        *reinterpret_cast<float4*>(out + n * xs + c0) =
+            make_float4(acc[c0] + q.x, acc[c0 + 1] + q.y, acc[c0 + 2] + q.z, acc[c0 + 3] + q.w);
+      }
+    }
+  }
+  csync();
+}
+
 // The tokens of the state Sm ([D][ld] in shared memory): writes keys and values to HBM and
-// leaves the residual in Sm. Called by all threads; r >= 1.
+// leaves the residual in Sm. Called by all threads; r >= 1. X, Y and part are [D][xs].
 template <class C>
-__device__ void power_tokens(float* Sm, int ld, int r, float* X, float* Y, float* scr,
-                             float* g_ck, float* g_cu) {
+__device__ void power_tokens(float* Sm, int ld, int r, float* X, float* Y, float* part,
+                             float* scr, float* g_ck, float* g_cu) {
   constexpr int D = C::D;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int xs = (r + 3) & ~3;
   int* sel = reinterpret_cast<int*>(scr + D);
   if (tid < D) {  // squared column norms
     float s2 = 0.f;
@@ -1195,62 +1245,49 @@ __device__ void power_tokens(float* Sm, int ld, int r, float* X, float* Y, float
     }
   }
   csync();
-  for (int e = tid; e < r * D; e += C::NT) X[e] = (e % D) == sel[e / D] ? 1.f : 0.f;
+  for (int e = tid; e < D * xs; e += C::NT) {
+    const int j = e / xs, c = e % xs;
+    X[e] = (c < r && j == sel[c]) ? 1.f : 0.f;  // (padding tokens stay 0)
+  }
   csync();
-  auto times_S = [&]() {  // Y = S X: thread (row tid % D) for tokens tid / D, + 2, ...
-    const int i = tid % D;
-    for (int c = tid / D; c < r; c += C::NT / D) {
-      float acc = 0.f;
-      for (int j = 0; j < D; ++j) acc = fmaf(Sm[i * ld + j], X[c * D + j], acc);
-      Y[c * D + i] = acc;
-    }
-  };
   for (int it = 0; it < kPowerIters; ++it) {
-    times_S();
-    csync();
-    {  // X = S^T Y: thread (column tid % D)
-      const int j = tid % D;
-      for (int c = tid / D; c < r; c += C::NT / D) {
-        float acc = 0.f;
-        for (int i = 0; i < D; ++i) acc = fmaf(Sm[i * ld + j], Y[c * D + i], acc);
-        X[c * D + j] = acc;
-      }
-    }
-    csync();
+    power_matvec<C, false>(Sm, ld, r, xs, X, Y, part);  // Y = S X
+    power_matvec<C, true>(Sm, ld, r, xs, Y, X, part);   // X = S^T Y
     if (warp == 0) {  // modified Gram-Schmidt over the columns in order
       for (int c = 0; c < r; ++c) {
         float xc[4];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) xc[m] = X[c * D + lane + 32 * m];
+        for (int m = 0; m < 4; ++m) xc[m] = X[(lane + 32 * m) * xs + c];
         for (int p = 0; p < c; ++p) {
           float d = 0.f;
 #pragma unroll
-          for (int m = 0; m < 4; ++m) d = fmaf(xc[m], X[p * D + lane + 32 * m], d);
+          for (int m = 0; m < 4; ++m) d = fmaf(xc[m], X[(lane + 32 * m) * xs + p], d);
           d = warp_sum(d);
 #pragma unroll
-          for (int m = 0; m < 4; ++m) xc[m] = fmaf(-d, X[p * D + lane + 32 * m], xc[m]);
+          for (int m = 0; m < 4; ++m) xc[m] = fmaf(-d, X[(lane + 32 * m) * xs + p], xc[m]);
         }
         float n2 = 0.f;
 #pragma unroll
         for (int m = 0; m < 4; ++m) n2 = fmaf(xc[m], xc[m], n2);
-        const float n = __fsqrt_rn(warp_sum(n2));
+        const float nrm = __fsqrt_rn(warp_sum(n2));
 #pragma unroll
-        for (int m = 0; m < 4; ++m) X[c * D + lane + 32 * m] = n > 0.f ? __fdiv_rn(xc[m], n) : 0.f;
+        for (int m = 0; m < 4; ++m)
+          X[(lane + 32 * m) * xs + c] = nrm > 0.f ? __fdiv_rn(xc[m], nrm) : 0.f;
         __syncwarp();
       }
     }
     csync();
   }
-  times_S();  // the values S x_c
-  csync();
+  power_matvec<C, false>(Sm, ld, r, xs, X, Y, part);  // the values S x_c
   for (int e = tid; e < r * D; e += C::NT) {
-    g_ck[e] = X[e];
-    g_cu[e] = Y[e];
+    const int c = e / D, j = e % D;
+    g_ck[e] = X[j * xs + c];
+    g_cu[e] = Y[j * xs + c];
   }
   for (int e = tid; e < D * D; e += C::NT) {  // residual S - sum_c u_c x_c^T
     const int i = e / D, j = e % D;
     float acc = Sm[i * ld + j];
-    for (int c = 0; c < r; ++c) acc = fmaf(-Y[c * D + i], X[c * D + j], acc);
+    for (int c = 0; c < r; ++c) acc = fmaf(-Y[i * xs + c], X[j * xs + c], acc);
     Sm[i * ld + j] = acc;
   }
   csync();
@@ -1265,18 +1302,23 @@ __global__ void __launch_bounds__(kThreads) power_end_kernel(const WinArgs a) {
   float* Sm = reinterpret_cast<float*>(sm);
   float* X = Sm + D * LD;
   float* Y = X + GDN_MAX_COMPENSATORS * D;
-  float* scr = Y + GDN_MAX_COMPENSATORS * D;
+  float* part = Y + GDN_MAX_COMPENSATORS * D;
+  float* scr = part + GDN_MAX_COMPENSATORS * D;
   float* g_ck = a.comp_k + (size_t)head * r * D;
   float* g_cu = a.comp_u + (size_t)head * r * D;
   if constexpr (MODE == 3) {
-    const float* src = a.S_in + (size_t)head * D * D;
-    for (int e = tid; e < D * D / 4; e += C::NT) {
-      const float4 f = reinterpret_cast<const float4*>(src)[e];
-      const int i = (4 * e) / D, j = (4 * e) % D;
-      Sm[i * LD + j] = f.x;
-      Sm[i * LD + j + 1] = f.y;
-      Sm[i * LD + j + 2] = f.z;
-      Sm[i * LD + j + 3] = f.w;
+    const float4* src = reinterpret_cast<const float4*>(a.S_in + (size_t)head * D * D);
+    constexpr int kPer = D * D / 4 / C::NT;  // 16-byte loads per thread, all issued first
+    float4 f[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) f[u] = src[tid + u * C::NT];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int e = tid + u * C::NT, i = (4 * e) / D, j = (4 * e) % D;
+      Sm[i * LD + j] = f[u].x;
+      Sm[i * LD + j + 1] = f[u].y;
+      Sm[i * LD + j + 2] = f[u].z;
+      Sm[i * LD + j + 3] = f[u].w;
     }
     csync();
   } else {
@@ -1328,7 +1370,7 @@ __global__ void __launch_bounds__(kThreads) power_end_kernel(const WinArgs a) {
     }
     csync();  // (the stage's old tokens are read out before the new ones go to HBM)
   }
-  if (r > 0) power_tokens<C>(Sm, LD, r, X, Y, scr, g_ck, g_cu);
+  if (r > 0) power_tokens<C>(Sm, LD, r, X, Y, part, scr, g_ck, g_cu);
   SmemTile<C> tile{Sm, LD};
   requantize_store<C>(tile, 0, a.codes + (size_t)head * a.code_stride,
                       a.scales + (size_t)head * a.scale_stride, nullptr, nullptr, scr,

@@ -305,20 +305,23 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
       }
     } else {
       // per-element decay e^{L_t[j] - L_i[j]}: FMA, 8 threads per pair; thread c takes columns
-      // 8c..8c+7 and 64+8c..64+8c+7 (distinct banks across the 8 threads of a pair)
+      // 8c..8c+7 and 64+8c..64+8c+7 (distinct banks across the 8 threads of a pair), as
+      // adjacent column pairs in packed fp32 arithmetic
       const int c = ty & 7;
-      float kr[16], qr[16], lr[16];
+      F2 kr[8], qr[8], lr[8];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int j = (e < 8 ? 8 * c : 64 + 8 * c) + (e & 7);
-        kr[e] = __bfloat162float(s_k[j]);
-        qr[e] = __bfloat162float(s_q[j]);
-        lr[e] = (P > 0 ? s_bL[(P - 1) * D + j] : 0.f) + s_g[j];
+      for (int e2 = 0; e2 < 8; ++e2) {
+        const int j = (e2 < 4 ? 8 * c : 64 + 8 * c) + 2 * (e2 & 3);
+        kr[e2] = f2(__bfloat162float(s_k[j]), __bfloat162float(s_k[j + 1]));
+        qr[e2] = f2(__bfloat162float(s_q[j]), __bfloat162float(s_q[j + 1]));
+        lr[e2] = f2((P > 0 ? s_bL[(P - 1) * D + j] : 0.f) + s_g[j],
+                    (P > 0 ? s_bL[(P - 1) * D + j + 1] : 0.f) + s_g[j + 1]);
       }
+      const F2 neg1 = f2(-1.f, -1.f), log2e = f2(1.4426950408889634f, 1.4426950408889634f);
       const int npass = (P + 15) >> 4;
       for (int ps = 0; ps < npass; ++ps) {
         const int i = ps * 16 + (ty >> 3);
-        float pa = 0.f, pb = 0.f;
+        F2 pa2 = f2(0.f, 0.f), pb2 = f2(0.f, 0.f);
         if (i < P) {
           float kk[16], ll[16];
           load_sw<bf, D, 8>(s_bk, i, 8 * c, kk);
@@ -326,11 +329,23 @@ __device__ __forceinline__ void step_head_mma(const WinArgs& a, const WinLayout&
           Num<float>::load<8>(s_bL + i * D + 8 * c, ll);
           Num<float>::load<8>(s_bL + i * D + 64 + 8 * c, ll + 8);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float k2 = kk[e] * fast_exp(lr[e] - ll[e]);
-            pa = fmaf(k2, kr[e], pa);
-            pb = fmaf(k2, qr[e], pb);
+          for (int e2 = 0; e2 < 8; ++e2) {
+            // (l_t - l_i) log2(e), then 2^x: the arithmetic of fast_exp, two columns at once
+            const F2 d = f2_mul(f2_fma(f2(ll[2 * e2], ll[2 * e2 + 1]), neg1, lr[e2]), log2e);
+            float d0, d1;
+            f2_get(d, d0, d1);
+            const F2 k2 = f2_mul(f2(kk[2 * e2], kk[2 * e2 + 1]), f2(exp2_hw(d0), exp2_hw(d1)));
+            pa2 = f2_fma(k2, kr[e2], pa2);
+            pb2 = f2_fma(k2, qr[e2], pb2);
           }
+        }
+        float pa, pb;
+        {
+          float a0, a1, b0, b1;
+          f2_get(pa2, a0, a1);
+          f2_get(pb2, b0, b1);
+          pa = a0 + a1;
+          pb = b0 + b1;
         }
 #pragma unroll
         for (int off = 4; off > 0; off >>= 1) {

@@ -18,6 +18,11 @@ Parity unpinned: the compensator column-selection rule (top-r columns by max-abs
 name compensator tokens but give no selection rule and no numbers; the tests pin only that the
 taken-out columns plus the residual reproduce the state exactly.
 
+Parity unpinned: the "power" compensator rule (keys from six steps of subspace iteration started
+at the largest-norm key columns, values S x_c). The pages give no rule; the tests pin it to the
+mathematics (exact low-rank states, a planted dominant direction against LAPACK's singular
+vectors, the truncated SVD's energy), not to the pages.
+
 Conventions: a state S is [D][D] with row i = value channel, column j = key channel. Per-step
 arrays are time-major, ``[T][nh][D]``; the gate ``g = log a`` is ``[T][nh]`` (scalar, GDN) or
 ``[T][nh][D]`` (per key channel, KDA).

@@ -265,6 +265,10 @@ int orc_smooth_exponent(double colmax) {
  *            divided by its length; a column of length 0 stays 0);
  *   tokens:  key x_c, value u_c = S x_c.
  * prec32 stores keys and values in single precision, as a GPU does.
+ * PARITY UNPINNED against the pages (no rule, no numbers): the start, the iteration count and
+ * the orthogonalisation are this reading's choices. Pinned to the mathematics: an exactly
+ * rank-r state is taken out whole, a planted dominant direction is found, the tokens' energy
+ * matches the truncated SVD's, and the start and its ties follow the stated rule.
  * ---------------------------------------------------------------------------------------- */
 #define ORC_POWER_ITERS 6
 

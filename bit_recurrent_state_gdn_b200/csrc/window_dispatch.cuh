@@ -72,7 +72,8 @@ StepPlan plan_step(int W, int r, int heads, bool power = false) {
 // after it on the same stream; forced flushes and the initial quantization run there too.
 template <class C>
 cudaError_t launch_power(WinOp op, const WinArgs& a, int heads, cudaStream_t st) {
-  const size_t pend = power_end_smem<C>(a.W, a.r), pq = power_scratch_bytes<C>();
+  const size_t pend = power_end_smem<C>(a.W, a.r, true), pq = power_end_smem<C>(a.W, a.r, false);
+  const int pgrid = std::min(heads, 2 * num_sms());
   cudaError_t e = cudaSuccess;
   switch (op) {
     case WinOp::Step: {
@@ -83,16 +84,16 @@ cudaError_t launch_power(WinOp op, const WinArgs& a, int heads, cudaStream_t st)
                                                                            (int)p.smem);
       if (e == cudaSuccess) e = cudaGetLastError();
       if (e == cudaSuccess) e = ensure_smem<power_end_kernel<C, 2>>(pend);
-      if (e == cudaSuccess) power_end_kernel<C, 2><<<heads, kThreads, pend, st>>>(a);
+      if (e == cudaSuccess) power_end_kernel<C, 2><<<pgrid, kThreads, pend, st>>>(a, heads);
       break;
     }
     case WinOp::Flush:
       e = ensure_smem<power_end_kernel<C, 0>>(pend);
-      if (e == cudaSuccess) power_end_kernel<C, 0><<<heads, kThreads, pend, st>>>(a);
+      if (e == cudaSuccess) power_end_kernel<C, 0><<<pgrid, kThreads, pend, st>>>(a, heads);
       break;
     case WinOp::Quantize:
       e = ensure_smem<power_end_kernel<C, 3>>(pq);
-      if (e == cudaSuccess) power_end_kernel<C, 3><<<heads, kThreads, pq, st>>>(a);
+      if (e == cudaSuccess) power_end_kernel<C, 3><<<pgrid, kThreads, pq, st>>>(a, heads);
       break;
     case WinOp::Materialize: {
       const size_t sm1 = win_layout<C>(a.W, a.r, 1, 0, -1, true, true).total;

@@ -1143,16 +1143,21 @@ struct SmemTile {
   }
 };
 
-// Shared memory of power_end_kernel: the state tile, keys X, products Y and the second half's
-// partial products ([D][16] each, token-minor), 512 floats of scratch, then (window ends) a
-// one-stage window layout.
+// Shared memory of power_end_kernel: a region holding (window ends) a one-stage window layout
+// and, once the state is materialised, the fp32 state tile [D][D + 1] from byte 128 on (the
+// stage barrier keeps the first 128 bytes); then keys X, products Y and the second half's
+// partial products ([D][xs] each, token-minor, xs = r rounded up to 4) and 512 floats of
+// scratch. About 105 KB for W = 64, r = 4: two CTAs per SM.
 template <class C>
-__host__ __device__ constexpr uint32_t power_scratch_bytes() {
-  return align128(4u * (C::D * (C::D + 1) + 3 * GDN_MAX_COMPENSATORS * C::D + 512));
+__host__ __device__ inline uint32_t power_region_bytes(int W, int r, bool window) {
+  const uint32_t tile = align128(128u + 4u * C::D * (C::D + 1));
+  const uint32_t win = window ? win_layout<C>(W, r, 1, 0, -1, true, true).total : 0u;
+  return tile > win ? tile : win;
 }
 template <class C>
-__host__ __device__ inline uint32_t power_end_smem(int W, int r) {
-  return power_scratch_bytes<C>() + win_layout<C>(W, r, 1, 0, -1, true, true).total;
+__host__ __device__ inline uint32_t power_end_smem(int W, int r, bool window) {
+  const uint32_t xs = (uint32_t)(r + 3) & ~3u;
+  return power_region_bytes<C>(W, r, window) + align128(4u * (3u * C::D * xs + 512u));
 }
 
 // Warp sum of a value.
@@ -1293,17 +1298,19 @@ __device__ void power_tokens(float* Sm, int ld, int r, float* X, float* Y, float
   csync();
 }
 
+// One head of power_end_kernel; false when a stage wait ran out (reported; the CTA stops).
+// `phase` is the stage barrier's parity, flipped by every completed wait.
 template <class C, int MODE>
-__global__ void __launch_bounds__(kThreads) power_end_kernel(const WinArgs a) {
-  extern __shared__ __align__(128) uint8_t sm[];
+__device__ __forceinline__ bool power_end_head(const WinArgs& a, uint8_t* sm, uint64_t* bar,
+                                               int head, uint32_t& phase) {
   constexpr int D = C::D, LD = D + 1;
-  const int head = blockIdx.x, tid = threadIdx.x;
-  const int W = a.W, r = a.r;
-  float* Sm = reinterpret_cast<float*>(sm);
-  float* X = Sm + D * LD;
-  float* Y = X + GDN_MAX_COMPENSATORS * D;
-  float* part = Y + GDN_MAX_COMPENSATORS * D;
-  float* scr = part + GDN_MAX_COMPENSATORS * D;
+  const int tid = threadIdx.x;
+  const int W = a.W, r = a.r, xs = (r + 3) & ~3;
+  float* Sm = reinterpret_cast<float*>(sm + 128);
+  float* X = reinterpret_cast<float*>(sm + power_region_bytes<C>(W, r, MODE != 3));
+  float* Y = X + D * xs;
+  float* part = Y + D * xs;
+  float* scr = part + D * xs;
   float* g_ck = a.comp_k + (size_t)head * r * D;
   float* g_cu = a.comp_u + (size_t)head * r * D;
   if constexpr (MODE == 3) {
@@ -1324,29 +1331,23 @@ __global__ void __launch_bounds__(kThreads) power_end_kernel(const WinArgs a) {
   } else {
     const int P = a.pos[head];
     if (MODE == 2) {
-      if (P != W) return;  // this head's window is not full
+      if (P != W) return true;  // this head's window is not full
     } else {
       if (P < 0 || P >= W) {
         if (tid == 0) report(a.status, GDN_DEVICE_BAD_POS);
-        return;
+        return true;
       }
-      if (P == 0) return;
-      if (a.seq_mask && a.seq_mask[head / a.H] == 0) return;
+      if (P == 0) return true;
+      if (a.seq_mask && a.seq_mask[head / a.H] == 0) return true;
     }
-    uint8_t* wsm = sm + power_scratch_bytes<C>();
     const WinLayout L = win_layout<C>(W, r, 1, 0, -1, true, true);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(wsm + L.bars);
-    uint8_t* st = wsm + L.stage0;
-    if (tid == 0) {
-      mbar_init(bar, 1);
-      fence_barrier_init();
-      stage_issue<C>(a, L, st, bar, head, P, false, -1, 0, true);
-    }
-    csync();
-    if (!stage_wait(a, bar, 0)) return;
-    float* vec = reinterpret_cast<float*>(wsm + L.vec);
+    uint8_t* st = sm + L.stage0;
+    if (tid == 0) stage_issue<C>(a, L, st, bar, head, P, false, -1, 0, true);
+    if (!stage_wait(a, bar, phase)) return false;
+    phase ^= 1u;
+    float* vec = reinterpret_cast<float*>(sm + L.vec);
     float *Lend = vec, *colexp = vec + D;
-    float* fac = reinterpret_cast<float*>(wsm + L.coef);
+    float* fac = reinterpret_cast<float*>(sm + L.coef);
     const float* s_bL = reinterpret_cast<const float*>(st + L.bL);
     float Ls = 0.f;
     if constexpr (C::DIAG) {
@@ -1359,16 +1360,18 @@ __global__ void __launch_bounds__(kThreads) power_end_kernel(const WinArgs a) {
     csync();
     const WindowTile<C> tile = window_tile<C>(st, L, P, r, colexp, fac, true);
     const int cg = tid % C::CG, rg = tid / C::CG;
-    float acc[C::TR][C::TC];
-    for (int ps = 0; ps < C::NPASS; ++ps) {
-      tile(ps, acc);
+    float acc[C::NPASS][C::TR][C::TC];  // the whole state first: the tile overwrites the stage
+#pragma unroll
+    for (int ps = 0; ps < C::NPASS; ++ps) tile(ps, acc[ps]);
+    csync();  // (the stage's old tokens are read out before the new ones go to HBM)
+#pragma unroll
+    for (int ps = 0; ps < C::NPASS; ++ps)
 #pragma unroll
       for (int aa = 0; aa < C::TR; ++aa)
 #pragma unroll
         for (int b = 0; b < C::TC; ++b)
-          Sm[(ps * C::RPASS + rg * C::TR + aa) * LD + cg * C::TC + b] = acc[aa][b];
-    }
-    csync();  // (the stage's old tokens are read out before the new ones go to HBM)
+          Sm[(ps * C::RPASS + rg * C::TR + aa) * LD + cg * C::TC + b] = acc[ps][aa][b];
+    csync();
   }
   if (r > 0) power_tokens<C>(Sm, LD, r, X, Y, part, scr, g_ck, g_cu);
   SmemTile<C> tile{Sm, LD};
@@ -1377,6 +1380,28 @@ __global__ void __launch_bounds__(kThreads) power_end_kernel(const WinArgs a) {
                       reinterpret_cast<int32_t*>(scr + 256), nullptr);
   if (tid < r) a.comp_idx[(size_t)head * ((r + 3) & ~3) + tid] = -1;  // (no key columns)
   if (tid == 0) a.pos[head] = 0;
+  // the tile's generic writes are ordered before the next head's stage copies over them
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+  csync();
+  return true;
+}
+
+// Persistent: CTA b takes heads b, b + grid, ... (two CTAs per SM); a launch after a decode step
+// (MODE 2) passes over the heads whose windows are not full at the cost of one load each.
+template <class C, int MODE>
+__global__ void __launch_bounds__(kThreads, 2) power_end_kernel(const WinArgs a, const int heads) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm);  // the window layout's stage barrier
+  if constexpr (MODE != 3) {
+    if (threadIdx.x == 0) {
+      mbar_init(bar, 1);
+      fence_barrier_init();
+    }
+    csync();
+  }
+  uint32_t phase = 0u;
+  for (int head = blockIdx.x; head < heads; head += gridDim.x)
+    if (!power_end_head<C, MODE>(a, sm, bar, head, phase)) return;
 }
 
 // ------------------------------------------------------------------------------------------

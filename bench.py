@@ -35,7 +35,8 @@ KERNEL_SOURCES = ["bit_recurrent_state_gdn_b200/csrc/window_kernels.cuh",
                   "bit_recurrent_state_gdn_b200/csrc/window_mma.cuh",
                   "bit_recurrent_state_gdn_b200/csrc/window_dispatch.cuh",
                   "bit_recurrent_state_gdn_b200/csrc/device_util.cuh",
-                  "bit_recurrent_state_gdn_b200/csrc/mma_util.cuh"]
+                  "bit_recurrent_state_gdn_b200/csrc/mma_util.cuh",
+                  "bit_recurrent_state_gdn_b200/csrc/tc_util.cuh"]
 PW_PROFILE = os.path.join(ROOT, "profiles", "pw_step_gdn-serving.md")
 PW_KERNEL_SOURCES = ["bit_recurrent_state_gdn_b200/csrc/pw_kernels.cuh",
                      "bit_recurrent_state_gdn_b200/csrc/pw.cu",

@@ -328,7 +328,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     tc_fence_after();
   };
   constexpr uint32_t ID64 = idesc_bf16(128, 64, false, false);
+  constexpr uint32_t ID128 = idesc_bf16(128, 128, false, false);
   constexpr uint32_t ID128_BMN = idesc_bf16(128, 128, false, true);
+  static_assert(kTcColSQ == kTcColSK + 64, "S Q^T follows S K^T");
 
   for (int c = 0; c < nch; ++c) {
     const int c0 = kPfC * c, n = min(kPfC, L - c0), buf = c & 1;
@@ -369,14 +371,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     if (tid == 0) {
       tc_fence_after();
       if (!mbar_wait_bounded(&bar_kq[buf], (uint32_t)(c >> 1) & 1u)) *fail = 1;
+      // one N = 128 product: the tile's rows 0-63 are K, 64-127 Q, so [S K^T | S Q^T] lands in
+      // the adjacent column blocks kTcColSK, kTcColSQ
 #pragma unroll
       for (int p = 0; p < 2; ++p)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u;
-          const uint64_t sd = kmajor_desc(sb + TcLayout::SP + 32768u * p + off);
-          umma_bf16(tm + kTcColSK, sd, kmajor_desc(kq + off), ID64, (p | kk) != 0);
-          umma_bf16(tm + kTcColSQ, sd, kmajor_desc(kq + 8192u + off), ID64, (p | kk) != 0);
+          umma_bf16(tm + kTcColSK, kmajor_desc(sb + TcLayout::SP + 32768u * p + off),
+                    kmajor_desc(kq + off), ID128, (p | kk) != 0);
         }
       umma_commit(bar_mma);
       if (c + 1 < nch) load_kq(sm + (buf ? TcLayout::KQ0 : TcLayout::KQ1), maps, c + 1, head, &bar_kq[buf ^ 1]);

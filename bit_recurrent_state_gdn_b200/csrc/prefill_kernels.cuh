@@ -118,9 +118,11 @@ __device__ __forceinline__ void store_split(const float (&acc)[NT][4], __nv_bflo
 }
 
 // R = (I + A)^{-1} for the strictly lower triangular 64 x 64 A (fp32, stride kLdF), blocked in
-// 16 x 16: diagonal blocks by forward substitution (one lane per column), then
-// R_ij = -R_ii sum_{j <= k < i} A_ik R_kj level by level (i - j = 1, 2, 3), each level spread
-// over all threads. xs: 3 x 256 floats of scratch.
+// 16 x 16: diagonal blocks by column-oriented substitution (one lane per column: after row k of
+// the column is final, every later row takes its -A_tk R_k term, so the 15 updates of a step are
+// independent), then R_ij = -R_ii sum_{j <= k < i} A_ik R_kj level by level (i - j = 1, 2, 3),
+// each level spread over all threads, its sums split over four partial accumulators.
+// xs: 3 x 256 floats of scratch.
 __device__ __forceinline__ void unit_lower_inverse(const float* A, float* R, float* xs) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // diagonal blocks: warps 0-1, lanes 0-15 / 16-31 take blocks 2 warp and 2 warp + 1
@@ -128,12 +130,11 @@ __device__ __forceinline__ void unit_lower_inverse(const float* A, float* R, flo
     const int b = 2 * warp + (lane >> 4), c = lane & 15, o = 16 * b;
     float rc[16];
 #pragma unroll
-    for (int t = 0; t < 16; ++t) {
-      float sum = 0.f;
+    for (int t = 0; t < 16; ++t) rc[t] = t == c ? 1.f : 0.f;
 #pragma unroll
-      for (int s = 0; s < t; ++s) sum = fmaf(A[(o + t) * kLdF + o + s], rc[s], sum);
-      rc[t] = t < c ? 0.f : (t == c ? 1.f : -sum);
-    }
+    for (int k = 0; k < 15; ++k)
+#pragma unroll
+      for (int t = k + 1; t < 16; ++t) rc[t] = fmaf(-A[(o + t) * kLdF + o + k], rc[k], rc[t]);
 #pragma unroll
     for (int t = 0; t < 16; ++t) R[(o + t) * kLdF + o + c] = rc[t];
   }
@@ -144,21 +145,32 @@ __device__ __forceinline__ void unit_lower_inverse(const float* A, float* R, flo
     const int nb = 4 - lvl;
     for (int e = tid; e < 256 * nb; e += kPfThreads) {
       const int j = e >> 8, i = j + lvl, r = (e >> 4) & 15, c = e & 15;
-      float sum = 0.f;
+      float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
       for (int kb = j; kb < i; ++kb) {
+        const float* ar = A + (16 * i + r) * kLdF + 16 * kb;
+        const float* rcol = R + (16 * kb) * kLdF + 16 * j + c;
 #pragma unroll
-        for (int s = 0; s < 16; ++s)
-          sum = fmaf(A[(16 * i + r) * kLdF + 16 * kb + s], R[(16 * kb + s) * kLdF + 16 * j + c], sum);
+        for (int s = 0; s < 16; s += 4) {
+          p0 = fmaf(ar[s], rcol[s * kLdF], p0);
+          p1 = fmaf(ar[s + 1], rcol[(s + 1) * kLdF], p1);
+          p2 = fmaf(ar[s + 2], rcol[(s + 2) * kLdF], p2);
+          p3 = fmaf(ar[s + 3], rcol[(s + 3) * kLdF], p3);
+        }
       }
-      xs[e] = sum;
+      xs[e] = (p0 + p1) + (p2 + p3);
     }
     __syncthreads();
     for (int e = tid; e < 256 * nb; e += kPfThreads) {
       const int j = e >> 8, i = j + lvl, r = (e >> 4) & 15, c = e & 15;
-      float sum = 0.f;
+      const float* rr = R + (16 * i + r) * kLdF + 16 * i;
+      const float* xc = xs + (j << 8) + c;
+      float p0 = 0.f, p1 = 0.f;
 #pragma unroll
-      for (int s = 0; s < 16; ++s) sum = fmaf(R[(16 * i + r) * kLdF + 16 * i + s], xs[(j << 8) + s * 16 + c], sum);
-      R[(16 * i + r) * kLdF + 16 * j + c] = -sum;
+      for (int s = 0; s < 16; s += 2) {
+        p0 = fmaf(rr[s], xc[s * 16], p0);
+        p1 = fmaf(rr[s + 1], xc[(s + 1) * 16], p1);
+      }
+      R[(16 * i + r) * kLdF + 16 * j + c] = -(p0 + p1);
     }
     __syncthreads();
   }

@@ -44,9 +44,9 @@ cudaError_t token_map(CUtensorMap* m, const void* base, int L, int heads) {
 cudaError_t launch_prefill(const PfArgs& a, int heads, bool diag, cudaStream_t st) {
   if (heads <= 0 || a.L <= 0) return cudaSuccess;
   if (diag) {
-    cudaError_t e = ensure_smem<prefill_kda_kernel>(KdaLayout::ALLOC);
+    cudaError_t e = ensure_smem<prefill_kda_kernel>(KdaLayout::TOTAL);
     if (e != cudaSuccess) return e;
-    prefill_kda_kernel<<<heads, kPfThreads, KdaLayout::ALLOC, st>>>(a);
+    prefill_kda_kernel<<<heads, kPfThreads, KdaLayout::TOTAL, st>>>(a);
     return cudaGetLastError();
   }
   PfTcMaps maps;
@@ -67,7 +67,7 @@ cudaError_t launch_prefill(const PfArgs& a, int heads, bool diag, cudaStream_t s
   return cudaGetLastError();
 }
 
-size_t prefill_smem_bytes(bool diag) { return diag ? KdaLayout::ALLOC : TcLayout::ALLOC; }
+size_t prefill_smem_bytes(bool diag) { return diag ? KdaLayout::TOTAL : TcLayout::ALLOC; }
 
 size_t prefill_workspace_bytes(bool diag, int64_t heads, int L) {
   if (diag || heads <= 0 || L <= 0) return 0;

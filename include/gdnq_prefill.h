@@ -49,8 +49,9 @@ extern "C" {
  *           scores P as split operand tiles, and its gates: 33,792 bytes), computed by a first
  *           kernel over all chunks at once; the second kernel carries the state through the
  *           chunks. Contents on entry are ignored; on return they are scratch.
- * Arithmetic: products on tensor cores (tcgen05 for the scalar gate, the state in tensor memory)
- * with fp32 accumulation; q, k, v enter exactly, every
+ * Arithmetic: products on tensor cores (tcgen05 for the scalar gate, the state in tensor memory;
+ * mma.sync for the per-channel gate's 16-token chunks, the state in registers) with fp32
+ * accumulation; q, k, v enter exactly, every
  * fp32 operand (the state, the chunk's triangular inverse, the corrected values, the decayed
  * scores, keys and queries, the write vectors) as the sum of two bf16 parts; the triangular
  * inverse in fp32.

@@ -131,6 +131,18 @@ __global__ void __launch_bounds__(kPfThreads, kChunkCtasPerSm)
     const int c0 = kPfC * c, n = min(kPfC, L - c0);
     const size_t row0 = (size_t)head * L + c0;
     uint8_t* rec = a.ws + (size_t)idx * kPfRecBytes;  // records are in (head, chunk) order
+    bool ok = true;
+    if (tid == 0) {  // [K; Q] K^T, then the next chunk's K and Q into the same tile
+      tc_fence_after();
+      ok = mbar_wait_bounded(bar, phase);
+      const uint32_t kq = sb + ChunkLayout::KQ;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u;
+        umma_bf16(tm, kmajor_desc(kq + off), kmajor_desc(kq + off), ID64, kk > 0);
+      }
+      umma_commit(bar_mma);
+    }
     if (warp == 0) {  // cumulative log-gate over the chunk, two tokens per lane
       const int t0 = 2 * lane;
       const float g0 = t0 < n ? a.g[row0 + t0] : 0.f;
@@ -153,18 +165,6 @@ __global__ void __launch_bounds__(kPfThreads, kChunkCtasPerSm)
       bet[t0] = t0 < n ? a.beta[row0 + t0] : 0.f;
       bet[t0 + 1] = t0 + 1 < n ? a.beta[row0 + t0 + 1] : 0.f;
     }
-    bool ok = true;
-    if (tid == 0) {  // [K; Q] K^T, then the next chunk's K and Q into the same tile
-      tc_fence_after();
-      ok = mbar_wait_bounded(bar, phase);
-      const uint32_t kq = sb + ChunkLayout::KQ;
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u;
-        umma_bf16(tm, kmajor_desc(kq + off), kmajor_desc(kq + off), ID64, kk > 0);
-      }
-      umma_commit(bar_mma);
-    }
     if (!mbar_wait_bounded(bar_mma, phase)) ok = false;
     tc_fence_after();
     if (tid == 0 && idx + (int)gridDim.x < total) {
@@ -172,24 +172,18 @@ __global__ void __launch_bounds__(kPfThreads, kChunkCtasPerSm)
       load_kq(sm + ChunkLayout::KQ, maps, nx % nch, nx / nch, bar);
     }
     __syncthreads();  // the gates
-    if (warp < 2) {  // A rows t
-      const int t = 32 * warp + lane;
-#pragma unroll
-      for (int p = 0; p < 2; ++p) {
-        float x[32];
-        tmem_ld32(tl + 32 * p, x);
+    {  // row t of A (TMEM lanes 0-63: warps 0, 1, 4, 5) or P (lanes 64-127: warps 2, 3, 6, 7),
+       // columns 32 p .. 32 p + 31 (p = warp / 4)
+      const int t = 32 * (warp & 1) + lane, p = warp >> 2;
+      float x[32];
+      tmem_ld32(tl + 32 * p, x);
+      if ((warp & 2) == 0) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int s = 32 * p + i;
           Af[t * kLdF + s] = s < t ? bet[t] * __expf(Gs[t] - Gs[s]) * x[i] : 0.f;
         }
-      }
-    } else if (warp < 4) {  // P rows t, to the record
-      const int t = 32 * (warp - 2) + lane;
-#pragma unroll
-      for (int p = 0; p < 2; ++p) {
-        float x[32];
-        tmem_ld32(tl + 32 * p, x);
+      } else {  // P, to the record
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int s = 32 * p + i;
@@ -201,7 +195,8 @@ __global__ void __launch_bounds__(kPfThreads, kChunkCtasPerSm)
           store_split8_global(rec + off, rec + off + 8192u, x + 8 * q);
         }
       }
-    } else if (warp == 4) {  // the gates, to the record
+    }
+    if (warp == 4) {  // the gates, to the record
       float* rg = reinterpret_cast<float*>(rec + kPfRecPlanes);
       for (int e = lane; e < 4 * kPfC; e += 32) rg[e] = Gs[e];
     }

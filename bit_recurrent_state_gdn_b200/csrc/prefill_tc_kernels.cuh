@@ -327,6 +327,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   constexpr uint32_t ID128_BMN = idesc_bf16(128, 128, false, true);
   static_assert(kTcColSQ == kTcColSK + 64, "S Q^T follows S K^T");
 
+  int c_stop = nch;  // the chunk a failed run stopped at (its copies are in flight)
   for (int c = 0; c < nch; ++c) {
     const int c0 = kPfC * c, n = min(kPfC, L - c0), buf = c & 1;
     const size_t row0 = (size_t)head * L + c0;
@@ -336,7 +337,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const float* eGC = eG + kPfC;
     tc_fence_before();
     __syncthreads();  // every thread is done with the previous chunk
-    if (*fail) break;
+    if (*fail) {
+      c_stop = c;
+      break;
+    }
     if (tid == 0 && c + 1 < nch) issue_gates(c + 1);
     if (!mbar_wait_bounded(&bar_g[buf], (uint32_t)(c >> 1) & 1u)) *fail = 1;
 
@@ -494,7 +498,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                                  __int_as_float(0x7fc00000), __int_as_float(0x7fc00000))
                    : make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
   }
-  if (bad && tid == 0) mbar_wait_bounded(bar_mma, mma_phase);  // products still in flight
+  if (bad && tid == 0) {  // products and the stopped chunk's copies still in flight
+    mbar_wait_bounded(bar_mma, mma_phase);
+    if (c_stop < nch) {
+      const int b = c_stop & 1;
+      (void)mbar_wait_bounded(&bar_g[b], (uint32_t)(c_stop >> 1) & 1u);
+      (void)mbar_wait_bounded(&bar_kq[b], (uint32_t)(c_stop >> 1) & 1u);
+      (void)mbar_wait_bounded(bar_v, (uint32_t)c_stop & 1u);
+      (void)mbar_wait_bounded(bar_tp, (uint32_t)c_stop & 1u);
+    }
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {

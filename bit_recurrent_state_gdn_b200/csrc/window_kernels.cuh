@@ -1258,7 +1258,12 @@ __device__ void power_tokens(float* Sm, int ld, int r, float* X, float* Y, float
   for (int it = 0; it < kPowerIters; ++it) {
     power_matvec<C, false>(Sm, ld, r, xs, X, Y, part);  // Y = S X
     power_matvec<C, true>(Sm, ld, r, xs, Y, X, part);   // X = S^T Y
-    if (warp == 0) {  // modified Gram-Schmidt over the columns in order
+    // modified Gram-Schmidt over the columns in order, run twice: S^T S X has columns that all
+    // lean towards the dominant direction, and one pass in single precision leaves them
+    // orthogonal only to about eps (sigma_1 / sigma_c)^2; the second pass restores
+    // orthonormality (in exact arithmetic it changes nothing)
+    if (warp == 0) {
+      for (int pass = 0; pass < 2; ++pass)
       for (int c = 0; c < r; ++c) {
         float xc[4];
 #pragma unroll

@@ -46,12 +46,9 @@ def gpu_tokens(wl, st, n):
     return ck, cu
 
 
-@pytest.mark.parametrize("fmt", ["int8", "int4_g32"])
-@pytest.mark.parametrize("gate", ["scalar", "diag"])
-def test_power_quantize(fmt, gate):
-    wl = KDA.with_(name="pw-q", B=2, H=8, fmt=fmt, gate=gate)
-    n, D, r = wl.heads, wl.D, wl.r
-    S0 = synthetic_states(n, D, seed=31)
+def _check_power_quantize(wl, seed=31):
+    n, D, r, fmt = wl.heads, wl.D, wl.r, wl.fmt
+    S0 = synthetic_states(n, D, seed=seed)
     cfg = cfg_of(wl)
     st = gdn.GdnState.allocate(cfg)
     gdn.gdn_state_quantize(cfg, S0.view(wl.B, wl.H, D, D).cuda(), st)
@@ -77,18 +74,45 @@ def test_power_quantize(fmt, gate):
         srow = np.abs(scales[h] - qs).max(axis=-1) / np.maximum(np.abs(qs).max(axis=-1), 1e-30)
         worst_s = max(worst_s, float(srow[same].max()) if same.any() else 0.0)
         rows += 1
-    print(fmt, gate, "token rel-L2", worst_c, "flips", flips / (n * D * D), "scale", worst_s)
+    print(wl.fmt, wl.gate, "r", r, "token rel-L2", worst_c, "flips", flips / (n * D * D),
+          "scale", worst_s)
     assert worst_c <= 1e-4
     assert flips <= FLIP_FRAC * n * D * D
     assert worst_s <= SCALE_TOL
+
+
+@pytest.mark.parametrize("fmt", ["int8", "int4_g32"])
+@pytest.mark.parametrize("gate", ["scalar", "diag"])
+def test_power_quantize(fmt, gate):
+    _check_power_quantize(KDA.with_(name="pw-q", B=2, H=8, fmt=fmt, gate=gate))
+
+
+@pytest.mark.parametrize("r", [1, 5, 16])
+def test_power_quantize_token_counts(r):
+    """One token, a count that is not a multiple of four (padded token slots) and the largest
+    count the library takes."""
+    _check_power_quantize(KDA.with_(name="pw-q", B=2, H=4, r=r), seed=37 + r)
 
 
 @pytest.mark.parametrize("base,fmt", [("kda", "int8"), ("kda", "int4_g32"), ("mid", "int8")])
 def test_power_decode_against_the_oracle(base, fmt):
     """Decode over three window ends (and a forced flush of every other sequence) with power
     tokens: outputs and the final logical state against the oracle's buffered form."""
-    wl = (KDA if base == "kda" else MID).with_(name="pw-dec", B=2, H=4, T=150, fmt=fmt,
-                                               warmup=48)
+    _check_power_decode((KDA if base == "kda" else MID).with_(name="pw-dec", B=2, H=4, T=150,
+                                                              fmt=fmt, warmup=48), flush_at=100)
+
+
+@pytest.mark.parametrize("base,W,r,T,flush_at", [("mid", 1, 2, 24, 9), ("mid", 8, 5, 44, 13),
+                                                 ("kda", 64, 16, 140, 100)])
+def test_power_decode_window_lengths(base, W, r, T, flush_at):
+    """A window end after every step (W = 1), short windows with a padded token count, and the
+    largest token count over full windows, each with a forced flush of every other sequence."""
+    _check_power_decode((KDA if base == "kda" else MID).with_(name="pw-dec", B=2, H=4, T=T, W=W,
+                                                              r=r, warmup=48),
+                        flush_at=flush_at)
+
+
+def _check_power_decode(wl, flush_at):
     n = wl.heads
     inputs = decode_inputs(wl, "cuda")
     cfg = cfg_of(wl)
@@ -100,7 +124,7 @@ def test_power_decode_against_the_oracle(base, fmt):
     for t in range(wl.T):
         gdn.gdn_decode_window_step(cfg, st, *(inputs[x][t] for x in ("q", "k", "v", "g", "beta")),
                                    o[t])
-        if t == 100:
+        if t == flush_at:
             gdn.gdn_window_flush(cfg, st, mask)
             flush_mask[t, : wl.H] = 1
     S = torch.empty((wl.B, wl.H, wl.D, wl.D), device="cuda")
@@ -112,7 +136,7 @@ def test_power_decode_against_the_oracle(base, fmt):
     o_rel = rel_l2(_heads_np(o, heads), round_act(res.o, wl.act))
     s_rel = rel_l2(S.view(n, wl.D, wl.D).double().cpu().numpy(), res.S)
     pos = st.pos.cpu().numpy()
-    print(base, fmt, "o_rel", o_rel, "S_rel", s_rel)
+    print(wl.gate, wl.fmt, "W", wl.W, "r", wl.r, "o_rel", o_rel, "S_rel", s_rel)
     assert o_rel <= O_TOL and s_rel <= O_TOL
     assert np.array_equal(pos, res.pos)
     ck, _ = gpu_tokens(wl, st, n)

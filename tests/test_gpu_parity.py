@@ -37,6 +37,10 @@ SMALL = {
     "kda-int8-w160": KDA.with_(name="kda-w160", B=1, H=2, T=170, W=160, r=2, warmup=32),
     "gdn-int8-w16": MID.with_(name="gdn-w16", B=2, H=3, T=50, W=16, warmup=32),
     "gdn-int8-w20": MID.with_(name="gdn-w20", B=2, H=3, T=50, W=20, r=1, warmup=32),
+    # tensor-core flush with three 16-pair blocks (window 40 / 48: 48 padded pairs)
+    "gdn-int8-w40-r3": MID.with_(name="gdn-w40", B=2, H=3, T=90, W=40, r=3, warmup=32),
+    "gdn-int4-w48": MID.with_(name="gdn-w48-int4", B=2, H=3, T=100, W=48, fmt="int4_g32",
+                              warmup=32),
 }
 
 

@@ -77,7 +77,8 @@ typedef enum { GDN_DTYPE_F32 = 0, GDN_DTYPE_BF16 = 1 } gdn_dtype;
  *                     e_{comp_idx[c]} and value that column.
  *   GDN_COMP_POWER    the state's dominant r-dimensional key subspace, by subspace iteration:
  *                     start from the r key columns of largest L2 norm (ties: lower index), six
- *                     times X <- orth(S^T S X) (modified Gram-Schmidt over the columns in order;
+ *                     times X <- orth(S^T S X) (modified Gram-Schmidt over the columns in order,
+ *                     run twice in single precision, which is the same in exact arithmetic;
  *                     a column of length 0 stays 0); token c has key x_c (comp_k[c], unit
  *                     length) and value S x_c, and the residual S (I - X X^T) is quantized.
  *                     Built for d = 128, bf16 activations and buffers, INT8 / INT4_G32 states

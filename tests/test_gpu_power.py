@@ -102,13 +102,15 @@ def test_power_decode_against_the_oracle(base, fmt):
                                                               fmt=fmt, warmup=48), flush_at=100)
 
 
-@pytest.mark.parametrize("base,W,r,T,flush_at", [("mid", 1, 2, 24, 9), ("mid", 8, 5, 44, 13),
-                                                 ("kda", 64, 16, 140, 100)])
-def test_power_decode_window_lengths(base, W, r, T, flush_at):
+@pytest.mark.parametrize("base,fmt,W,r,T,flush_at", [
+    ("mid", "int8", 1, 2, 24, 9), ("mid", "int8", 8, 5, 44, 13), ("kda", "int8", 64, 16, 140, 100),
+    ("mid", "int8", 64, 16, 140, 90), ("kda", "int4_g32", 32, 16, 80, 50)])
+def test_power_decode_window_lengths(base, fmt, W, r, T, flush_at):
     """A window end after every step (W = 1), short windows with a padded token count, and the
-    largest token count over full windows, each with a forced flush of every other sequence."""
+    largest token count over full windows (both gates, int8 and int4-g32), each with a forced
+    flush of every other sequence."""
     _check_power_decode((KDA if base == "kda" else MID).with_(name="pw-dec", B=2, H=4, T=T, W=W,
-                                                              r=r, warmup=48),
+                                                              r=r, fmt=fmt, warmup=48),
                         flush_at=flush_at)
 
 
